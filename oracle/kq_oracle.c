@@ -1,0 +1,198 @@
+/*
+ * kq_oracle — plain, slow, obviously correct CPU reference for the K-quant
+ * dequant-GEMV.  TEST INFRASTRUCTURE ONLY: tests, the smoke check and the
+ * benchmark's CPU-baseline leg use it; the product (libkq) never links,
+ * loads or calls it, and it shares no code, header or table with libkq.
+ *
+ * What it computes (the method's definition, written out):
+ *   y_r = sum_i w_{r,i} * x_i       (double precision, natural index order)
+ *   s_r = sum_i |w_{r,i} * x_i|     (for the per-output tolerance)
+ * where w is obtained by dequantising every super-block of row r to double
+ * by its block formula.  Sources:
+ *  - "Out-of-core LLM inference engine written from scratch in Rust",
+ *    Approach: quantised weights are dequantised inside the fused matmul
+ *    kernels; Results: Llama-3.3-70B Q4_K_M.
+ *  - "Kortex: Streaming 70B Models on Consumer GPUs", Key components item 3:
+ *    weights are dequantised only in GPU registers (so the product equals the
+ *    plain matvec over dequantised weights, up to rounding).
+ *  - "RunNburn - Run a 295B MoE ...": native K-quant kernels Q2_K..Q6_K.
+ *  The pages name the formats (GGUF K-quants, "Q4_K_M") but print no bit
+ *  layout; the layout below is the public GGUF one, restated:
+ *   Q4_K (144 B, 256 weights = 8 sub-blocks of 32):
+ *     w = d*sc_j*q - dmin*m_j for weight in sub-block j.
+ *   Q6_K (210 B, 256 weights = 16 groups of 16):
+ *     w = d*s_g*(q - 32) for weight in group g, s_g a signed byte.
+ *
+ * Every step is a literal loop; no blocking, fusion or reordering.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { KQO_Q4_K = 1, KQO_Q6_K = 2 };
+
+/* IEEE binary16 -> double (exact), including subnormals, inf and NaN. */
+double kqo_f16(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 31;
+    int mant = h & 1023;
+    double v;
+    if (e == 0) v = ldexp((double)mant, -24);                 /* subnormal / zero */
+    else if (e == 31) v = mant ? NAN : INFINITY;
+    else v = ldexp((double)(1024 + mant), e - 25);            /* (1 + mant/1024) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+static uint16_t rd16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+
+/* Q4_K super-block -> logical fields.
+ * Header: d (fp16), dmin (fp16), 12 bytes of packed 6-bit scales and mins.
+ * For j < 4 the scale and min are the low 6 bits of bytes j and j+4.
+ * For j >= 4 the low 4 bits come from byte j+4 (scale: low nibble, min:
+ * high nibble) and the top 2 bits from bits 6..7 of byte j-4 (scale) and
+ * byte j (min).
+ * Quants: 4 chunks of 32 bytes; byte l of chunk c holds weight 64c+l in its
+ * low nibble and weight 64c+32+l in its high nibble. */
+void kqo_q4k_unpack(const uint8_t* blk, uint8_t q[256], uint8_t sc[8], uint8_t m[8],
+                    double* d, double* dmin) {
+    const uint8_t* s = blk + 4;
+    const uint8_t* qs = blk + 16;
+    *d = kqo_f16(rd16(blk));
+    *dmin = kqo_f16(rd16(blk + 2));
+    for (int j = 0; j < 8; ++j) {
+        if (j < 4) {
+            sc[j] = s[j] & 63;
+            m[j] = s[j + 4] & 63;
+        } else {
+            sc[j] = (uint8_t)((s[j + 4] & 15) | ((s[j - 4] >> 6) << 4));
+            m[j] = (uint8_t)((s[j + 4] >> 4) | ((s[j] >> 6) << 4));
+        }
+    }
+    for (int i = 0; i < 256; ++i) {
+        int c = i / 64;           /* 32-byte chunk */
+        int within = i % 64;      /* 0..31 low nibbles, 32..63 high nibbles */
+        uint8_t byte = qs[32 * c + (within % 32)];
+        q[i] = within < 32 ? (byte & 15) : (byte >> 4);
+    }
+}
+
+/* Q6_K super-block -> logical fields.
+ * Layout: ql[128] (low 4 bits), qh[64] (top 2 bits), 16 signed scales, d.
+ * Weight i = 128h + 32t + l (h<2, t<4, l<32): low bits from
+ * ql[64h + l + 32*(t%2)] (low nibble for t<2, high nibble for t>=2), top
+ * bits from bits 2t..2t+1 of qh[32h + l]; its scale is scales[i/16]. */
+void kqo_q6k_unpack(const uint8_t* blk, uint8_t q[256], int8_t s[16], double* d) {
+    const uint8_t* ql = blk;
+    const uint8_t* qh = blk + 128;
+    for (int i = 0; i < 256; ++i) {
+        int h = i / 128, t = (i % 128) / 32, l = i % 32;
+        uint8_t lb = ql[64 * h + l + 32 * (t % 2)];
+        int lo = t < 2 ? (lb & 15) : (lb >> 4);
+        int hi = (qh[32 * h + l] >> (2 * t)) & 3;
+        q[i] = (uint8_t)(lo | (hi << 4));
+    }
+    for (int g = 0; g < 16; ++g) s[g] = (int8_t)blk[192 + g];
+    *d = kqo_f16(rd16(blk + 208));
+}
+
+static int64_t block_bytes(int fmt) { return fmt == KQO_Q4_K ? 144 : fmt == KQO_Q6_K ? 210 : -1; }
+
+/* Dequantise one row of K weights (K/256 consecutive super-blocks). */
+int kqo_dequant_row(int fmt, const uint8_t* row, int64_t K, double* w) {
+    int64_t bb = block_bytes(fmt);
+    if (bb < 0 || K % 256 != 0) return -1;
+    for (int64_t b = 0; b < K / 256; ++b) {
+        const uint8_t* blk = row + b * bb;
+        uint8_t q[256];
+        double* wb = w + 256 * b;
+        if (fmt == KQO_Q4_K) {
+            uint8_t sc[8], m[8];
+            double d, dmin;
+            kqo_q4k_unpack(blk, q, sc, m, &d, &dmin);
+            for (int i = 0; i < 256; ++i) {
+                int j = i / 32;
+                wb[i] = d * sc[j] * q[i] - dmin * m[j];
+            }
+        } else {
+            int8_t s[16];
+            double d;
+            kqo_q6k_unpack(blk, q, s, &d);
+            for (int i = 0; i < 256; ++i) {
+                int g = i / 16;
+                wb[i] = d * s[g] * ((int)q[i] - 32);
+            }
+        }
+    }
+    return 0;
+}
+
+/* y and s for the listed rows of W (row r starts at W + r*row_bytes). */
+int kqo_gemv_rows(int fmt, const uint8_t* W, int64_t K, const int64_t* rows, int64_t nrows,
+                  const float* x, double* y, double* sabs, int nthreads) {
+    int64_t bb = block_bytes(fmt);
+    if (bb < 0 || K % 256 != 0) return -1;
+    int64_t row_bytes = K / 256 * bb;
+    int bad = 0;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel num_threads(nthreads)
+    {
+        double* w = (double*)malloc(sizeof(double) * (size_t)K);
+        if (!w) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(static)
+        for (int64_t t = 0; t < nrows; ++t) {
+            if (!w) continue;
+            kqo_dequant_row(fmt, W + rows[t] * row_bytes, K, w);
+            double acc = 0.0, acc_abs = 0.0;
+            for (int64_t i = 0; i < K; ++i) {
+                double p = w[i] * (double)x[i];
+                acc += p;
+                acc_abs += fabs(p);
+            }
+            y[t] = acc;
+            if (sabs) sabs[t] = acc_abs;
+        }
+        free(w);
+    }
+    return bad ? -2 : 0;
+}
+
+/* Full matvec: all N rows. */
+int kqo_gemv(int fmt, const uint8_t* W, int64_t N, int64_t K, const float* x, double* y,
+             double* sabs, int nthreads) {
+    int64_t* rows = (int64_t*)malloc(sizeof(int64_t) * (size_t)(N > 0 ? N : 1));
+    if (!rows) return -2;
+    for (int64_t r = 0; r < N; ++r) rows[r] = r;
+    int rc = kqo_gemv_rows(fmt, W, K, rows, N, x, y, sabs, nthreads);
+    free(rows);
+    return rc;
+}
+
+/* Logical fields of `nblocks` consecutive super-blocks, in the layout the
+ * bit-exact unpack check compares:
+ *   q[256*b + i]      quant of weight i (Q4_K 0..15, Q6_K 0..63, before -32)
+ *   sc[16*b + j]      Q4_K: sc_0..7 then m_0..7; Q6_K: the 16 signed scales
+ *                     as two's-complement bytes
+ *   d[2*b], d[2*b+1]  Q4_K: d, dmin; Q6_K: d, 0 (fp16 widened exactly) */
+int kqo_unpack(int fmt, const uint8_t* W, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d) {
+    int64_t bb = block_bytes(fmt);
+    if (bb < 0) return -1;
+    for (int64_t b = 0; b < nblocks; ++b) {
+        const uint8_t* blk = W + b * bb;
+        if (fmt == KQO_Q4_K) {
+            double dd, dm;
+            kqo_q4k_unpack(blk, q + 256 * b, sc + 16 * b, sc + 16 * b + 8, &dd, &dm);
+            d[2 * b] = (float)dd;
+            d[2 * b + 1] = (float)dm;
+        } else {
+            double dd;
+            kqo_q6k_unpack(blk, q + 256 * b, (int8_t*)(sc + 16 * b), &dd);
+            d[2 * b] = (float)dd;
+            d[2 * b + 1] = 0.0f;
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,302 @@
+"""Pins for the CPU oracle: checks against values fixed by something other
+than the oracle itself — hand-worked blocks, library routines, closed forms,
+invariants and exhaustive round trips.
+
+Formats: GGUF K-quants Q4_K (w = d*sc_j*q - dmin*m_j per 32-weight
+sub-block) and Q6_K (w = d*s_g*(q-32) per 16-weight group), the formats the
+pages name ("Out-of-core LLM inference engine written from scratch in Rust",
+Results: Q4_K_M; "RunNburn - Run a 295B MoE ...": K-quants Q2_K..Q6_K).
+"""
+import os
+
+import numpy as np
+import pytest
+
+import kqgen
+import oracle
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def _read_golden(path):
+    rec = {"w": []}
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        key, *vals = line.split()
+        if key == "w":
+            rec["w"].append((int(vals[0]), int(vals[1]), float(vals[2])))
+        else:
+            rec[key] = vals
+    return rec
+
+
+# ------------------------------------------------------------------ fp16
+def test_f16_decode_matches_numpy_all_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.f16(int(b)) for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_generator_f16_encode_matches_numpy():
+    rng = np.random.default_rng(7)
+    vals = np.concatenate([
+        rng.standard_normal(20000) * 1e-3,
+        rng.standard_normal(5000) * 1e-6,           # subnormal range
+        rng.standard_normal(5000) * 1e4,
+        np.array([0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e6, 2.0**-24, 2.0**-25, 3 * 2.0**-26,
+                  2.0**-14, 2.0**-14 - 2.0**-25, 1.0 + 2.0**-11, 1.0 + 3 * 2.0**-11]),
+    ])
+    for v in vals:
+        want = int(np.array(v, np.float64).astype(np.float16).view(np.uint16))
+        assert kqgen.f16_bits(float(v)) == want, v
+
+
+# ----------------------------------------------------- hand-worked blocks
+def test_q4k_hand_worked_block(golden_dir):
+    g = _read_golden(os.path.join(golden_dir, "q4k_block_worked.txt"))
+    blk = np.array([int(h, 16) for h in g["header"]] + list(range(128)), np.uint8)
+    assert blk.size == 144
+    q, sc, d = oracle.unpack("q4_k", blk, 1)
+    assert sc[:8].tolist() == [int(v) for v in g["sc"]]
+    assert sc[8:].tolist() == [int(v) for v in g["m"]]
+    assert d.tolist() == [1.0, 0.5]
+    w = oracle.dequant("q4_k", blk, 1, 256)[0]
+    for i, qi, wi in g["w"]:
+        assert q[i] == qi, i
+        assert w[i] == wi, i
+    y, _ = oracle.gemv("q4_k", blk, 1, 256, np.ones(256, np.float32))
+    assert y[0] == float(g["y_ones"][0])
+
+
+def test_q6k_hand_worked_block(golden_dir):
+    g = _read_golden(os.path.join(golden_dir, "q6k_block_worked.txt"))
+    s = np.array([int(v) for v in g["s"]], np.int8)
+    blk = np.concatenate([np.arange(128, dtype=np.uint8),
+                          np.full(64, int(g["qh_fill"][0], 16), np.uint8),
+                          s.view(np.uint8),
+                          np.array([int(h, 16) for h in g["d"]], np.uint8)])
+    assert blk.size == 210
+    q, sc, d = oracle.unpack("q6_k", blk, 1)
+    assert sc.view(np.int8).tolist() == s.tolist()
+    assert d[0] == 1.0
+    w = oracle.dequant("q6_k", blk, 1, 256)[0]
+    for i, qi, wi in g["w"]:
+        assert q[i] == qi, i
+        assert w[i] == wi, i
+
+
+# ----------------------------------------------- exhaustive round trips
+def test_q4k_scale_min_roundtrip_exhaustive():
+    # every 6-bit value in every scale and min slot, others varied
+    for v in range(64):
+        nb = 8
+        q = np.zeros((nb, 256), np.uint8)
+        sc = np.zeros((nb, 8), np.uint8)
+        m = np.zeros((nb, 8), np.uint8)
+        for j in range(8):
+            sc[j, j] = v
+            m[j, j] = 63 - v
+            sc[j, (j + 3) % 8] = (v * 7 + j) % 64
+            m[j, (j + 5) % 8] = (v * 11 + j) % 64
+        d = np.full(nb, 0x3C00, np.uint16)
+        dm = np.full(nb, 0x3800, np.uint16)
+        W = kqgen.q4k_pack(q, sc, m, d, dm)
+        _, sc2, d2 = oracle.unpack("q4_k", W, nb)
+        sc2 = sc2.reshape(nb, 16)
+        assert np.array_equal(sc2[:, :8], sc) and np.array_equal(sc2[:, 8:], m)
+        assert np.all(d2.reshape(nb, 2) == [1.0, 0.5])
+
+
+def test_q4k_quant_roundtrip_all_positions():
+    nb = 16
+    q = (np.arange(nb * 256).reshape(nb, 256) * 7 + np.arange(nb)[:, None]) % 16
+    q = q.astype(np.uint8)
+    z8 = np.zeros((nb, 8), np.uint8)
+    W = kqgen.q4k_pack(q, z8, z8, np.zeros(nb, np.uint16), np.zeros(nb, np.uint16))
+    q2, _, _ = oracle.unpack("q4_k", W, nb)
+    assert np.array_equal(q2.reshape(nb, 256), q)
+
+
+def test_q6k_roundtrip_exhaustive():
+    nb = 64
+    q = ((np.arange(256)[None, :] + 17 * np.arange(nb)[:, None]) % 64).astype(np.uint8)
+    s = ((np.arange(16)[None, :] * 16 + np.arange(nb)[:, None]) % 256 - 128).astype(np.int8)
+    d = (np.arange(nb) * 977 % 0x7C00).astype(np.uint16)
+    W = kqgen.q6k_pack(q, s, d)
+    q2, s2, d2 = oracle.unpack("q6_k", W, nb)
+    assert np.array_equal(q2.reshape(nb, 256), q)
+    assert np.array_equal(s2.view(np.int8).reshape(nb, 16), s)
+    want_d = d.view(np.float16).astype(np.float32)
+    assert np.array_equal(d2.reshape(nb, 2)[:, 0], want_d)
+    # every q value in every position across the 64 blocks
+    assert all(len(set(q[:, i].tolist())) == 64 for i in range(256))
+    assert len(set(s.ravel().tolist())) == 256
+
+
+# ---------------------------- special cases that reduce to library routines
+@pytest.mark.parametrize("N,K", [(5, 256), (7, 768), (3, 2048)])
+def test_q4k_unit_scales_is_integer_matvec(N, K):
+    """d=1, sc=1, dmin=0, m=0: W is the integer quant matrix; y = Q @ x."""
+    nb = N * K // 256
+    lg = kqgen.q4k_draw(101 + K, nb)
+    ones = np.ones((nb, 8), np.uint8)
+    W = kqgen.q4k_pack(lg["q"], ones, np.zeros((nb, 8), np.uint8),
+                       np.full(nb, 0x3C00, np.uint16), np.zeros(nb, np.uint16))
+    x = kqgen.normal_f32(5, K)
+    Q = lg["q"].reshape(N, K).astype(np.float64)
+    y, _ = oracle.gemv("q4_k", W, N, K, x)
+    assert np.allclose(y, Q @ x.astype(np.float64), rtol=1e-13, atol=1e-12)
+
+
+def test_q4k_zero_quants_closed_form():
+    """q = 0 everywhere: y_r = -sum_b dmin_b * sum_j m_bj * (sum of x over sub-block j)."""
+    N, K = 6, 1024
+    nb = N * K // 256
+    lg = kqgen.q4k_draw(77, nb)
+    W = kqgen.q4k_pack(np.zeros_like(lg["q"]), lg["sc"], lg["m"], lg["d"], lg["dmin"])
+    x = kqgen.normal_f32(8, K)
+    X = x.astype(np.float64).reshape(K // 32, 32).sum(axis=1).reshape(K // 256, 8)
+    dmin = lg["dmin"].view(np.float16).astype(np.float64).reshape(N, K // 256)
+    m = lg["m"].astype(np.float64).reshape(N, K // 256, 8)
+    want = -np.einsum("rb,rbj,bj->r", dmin, m, X)
+    y, _ = oracle.gemv("q4_k", W, N, K, x)
+    assert np.allclose(y, want, rtol=1e-12, atol=1e-15)
+
+
+def test_q4k_zero_scales_gives_exact_zero():
+    N, K = 4, 512
+    nb = N * K // 256
+    lg = kqgen.q4k_draw(78, nb)
+    z = np.zeros((nb, 8), np.uint8)
+    W = kqgen.q4k_pack(lg["q"], z, z, lg["d"], lg["dmin"])
+    y, s = oracle.gemv("q4_k", W, N, K, kqgen.normal_f32(9, K))
+    assert np.all(y == 0.0) and np.all(s == 0.0)
+
+
+def test_q4k_one_hot_reads_subblock_scale():
+    """d=1, dmin=0, q=1, sc_j = j+1: x = e_i gives y = (i%256)//32 + 1."""
+    K = 512
+    sc = np.tile(np.arange(1, 9, dtype=np.uint8), (2, 1))
+    W = kqgen.q4k_pack(np.ones((2, 256), np.uint8), sc, np.zeros((2, 8), np.uint8),
+                       np.full(2, 0x3C00, np.uint16), np.zeros(2, np.uint16))
+    for i in range(K):
+        x = np.zeros(K, np.float32)
+        x[i] = 1.0
+        y, _ = oracle.gemv("q4_k", W, 1, K, x)
+        assert y[0] == (i % 256) // 32 + 1
+
+
+@pytest.mark.parametrize("N,K", [(4, 256), (3, 2048)])
+def test_q6k_unit_scale_is_centered_integer_matvec(N, K):
+    """d=1, s=1: W = Q - 32; y = (Q - 32) @ x."""
+    nb = N * K // 256
+    lg = kqgen.q6k_draw(202 + K, nb)
+    W = kqgen.q6k_pack(lg["q"], np.ones((nb, 16), np.int8), np.full(nb, 0x3C00, np.uint16))
+    x = kqgen.normal_f32(6, K)
+    Q = lg["q"].reshape(N, K).astype(np.float64) - 32
+    y, _ = oracle.gemv("q6_k", W, N, K, x)
+    assert np.allclose(y, Q @ x.astype(np.float64), rtol=1e-13, atol=1e-12)
+
+
+def test_q6k_mid_quants_give_exact_zero_and_zero_quants_closed_form():
+    N, K = 3, 768
+    nb = N * K // 256
+    lg = kqgen.q6k_draw(303, nb)
+    x = kqgen.normal_f32(10, K)
+    W32 = kqgen.q6k_pack(np.full_like(lg["q"], 32), lg["s"], lg["d"])
+    y, _ = oracle.gemv("q6_k", W32, N, K, x)
+    assert np.all(y == 0.0)
+    W0 = kqgen.q6k_pack(np.zeros_like(lg["q"]), lg["s"], lg["d"])
+    y0, _ = oracle.gemv("q6_k", W0, N, K, x)
+    X = x.astype(np.float64).reshape(K // 16, 16).sum(axis=1).reshape(K // 256, 16)
+    d = lg["d"].view(np.float16).astype(np.float64).reshape(N, K // 256)
+    s = lg["s"].astype(np.float64).reshape(N, K // 256, 16)
+    want = -32.0 * np.einsum("rb,rbg,bg->r", d, s, X)
+    assert np.allclose(y0, want, rtol=1e-12, atol=1e-15)
+
+
+# -------------------------------------------------------------- invariants
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+def test_linearity_in_x(fmt):
+    N, K = 8, 1024
+    W = kqgen.matrix(fmt, 11, N, K)
+    rng = np.random.default_rng(3)
+    x1 = rng.integers(-50, 50, K).astype(np.float32)
+    x2 = rng.integers(-50, 50, K).astype(np.float32)
+    xc = (2.0 * x1 - 3.0 * x2).astype(np.float32)   # exact in fp32
+    y1, s1 = oracle.gemv(fmt, W, N, K, x1)
+    y2, s2 = oracle.gemv(fmt, W, N, K, x2)
+    yc, _ = oracle.gemv(fmt, W, N, K, xc)
+    assert np.all(np.abs(yc - (2 * y1 - 3 * y2)) <= 1e-12 * (2 * s1 + 3 * s2))
+
+
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+def test_one_hot_extracts_column_and_ones_give_row_sums(fmt):
+    N, K = 4, 512
+    W = kqgen.matrix(fmt, 12, N, K)
+    Wd = oracle.dequant(fmt, W, N, K)
+    for i in (0, 1, 31, 32, 255, 256, 300, 511):
+        x = np.zeros(K, np.float32)
+        x[i] = 1.0
+        y, _ = oracle.gemv(fmt, W, N, K, x)
+        assert np.array_equal(y, Wd[:, i])
+    y, s = oracle.gemv(fmt, W, N, K, np.ones(K, np.float32))
+    assert np.allclose(y, Wd.sum(axis=1), rtol=1e-13, atol=1e-15)
+    assert np.allclose(s, np.abs(Wd).sum(axis=1), rtol=1e-13)
+
+
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+def test_brute_force_tiny_from_logical_values(fmt):
+    """Dense W built from the generator's logical values (never its bytes)
+    matches the oracle's byte path."""
+    N, K = 8, 512
+    nb = N * K // 256
+    if fmt == "q4_k":
+        lg = kqgen.q4k_draw(31, nb)
+        W = kqgen.q4k_pack(**lg)
+        d = lg["d"].view(np.float16).astype(np.float64)[:, None]
+        dm = lg["dmin"].view(np.float16).astype(np.float64)[:, None]
+        sc = np.repeat(lg["sc"].astype(np.float64), 32, axis=1)
+        m = np.repeat(lg["m"].astype(np.float64), 32, axis=1)
+        dense = (d * sc * lg["q"] - dm * m).reshape(N, K)
+    else:
+        lg = kqgen.q6k_draw(32, nb)
+        W = kqgen.q6k_pack(**lg)
+        d = lg["d"].view(np.float16).astype(np.float64)[:, None]
+        s = np.repeat(lg["s"].astype(np.float64), 16, axis=1)
+        dense = (d * s * (lg["q"].astype(np.float64) - 32)).reshape(N, K)
+    x = kqgen.normal_f32(33, K)
+    y, _ = oracle.gemv(fmt, W, N, K, x)
+    ref = dense @ x.astype(np.float64)
+    assert np.all(np.abs(y - ref) <= 1e-12 * np.abs(dense) @ np.abs(x.astype(np.float64)))
+
+
+def test_multi_moe_forms_are_loops_of_gemv():
+    K, N, E = 512, 6, 5
+    W = kqgen.matrix("q4_k", 40, E * N, K)
+    X = np.stack([kqgen.normal_f32(41 + c, K) for c in range(3)])
+    ym, _ = oracle.gemv_multi("q4_k", W[: N * 2 * 144], N, K, X)
+    for c in range(3):
+        assert np.array_equal(ym[c], oracle.gemv("q4_k", W, N, K, X[c])[0])
+    ids = np.array([4, 0, 2], np.int32)
+    ye, _ = oracle.moe_gemv("q4_k", W, E, N, K, ids, X)
+    stride = N * 2 * 144
+    for i, e in enumerate(ids):
+        assert np.array_equal(ye[i], oracle.gemv("q4_k", W[e * stride:], N, K, X[i])[0])
+    with pytest.raises(ValueError):
+        oracle.moe_gemv("q4_k", W, E, N, K, np.array([5]), X[:1])
+
+
+def test_rows_subset_matches_full():
+    N, K = 40, 1024
+    W = kqgen.matrix("q6_k", 50, N, K)
+    x = kqgen.normal_f32(51, K)
+    y, s = oracle.gemv("q6_k", W, N, K, x, nthreads=3)
+    rows = np.array([39, 0, 17, 17, 5])
+    yr, sr = oracle.gemv_rows("q6_k", W, K, rows, x)
+    assert np.array_equal(yr, y[rows]) and np.array_equal(sr, s[rows])
