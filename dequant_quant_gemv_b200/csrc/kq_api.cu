@@ -1,0 +1,386 @@
+// kq_api.cu — the libkq C ABI: argument validation, schedule planning and
+// launch of the fused K-quant GEMV kernels (see include/kq.h).
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/kq.h"
+#include "kq_device.cuh"
+#include "kq_internal.h"
+
+namespace kq {
+
+static thread_local char g_last_error[512] = "";
+
+static int fail(int status, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+static int cuda_fail(cudaError_t err, const char* what) {
+    return fail(KQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+}
+
+// Per-device properties, read once.
+struct DevInfo {
+    int sm_count = 0;
+    int smem_optin = 0;
+    int smem_per_sm = 0;
+};
+static std::mutex g_dev_mu;
+static DevInfo g_dev[64];
+
+static cudaError_t dev_info(DevInfo& out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (g_dev[dev].sm_count == 0) {
+        int sms = 0, smem = 0;
+        err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (err != cudaSuccess) return err;
+        err = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (err != cudaSuccess) return err;
+        int smem_sm = 0;
+        err = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        if (err != cudaSuccess) return err;
+        g_dev[dev].sm_count = sms;
+        g_dev[dev].smem_optin = smem;
+        g_dev[dev].smem_per_sm = smem_sm;
+    }
+    out = g_dev[dev];
+    return cudaSuccess;
+}
+
+cudaError_t ensure_smem_attr(const void* func, size_t bytes) {
+    // cudaFuncSetAttribute is cheap but not free; remember the largest value
+    // set per (device, kernel).
+    struct Entry {
+        int dev;
+        const void* func;
+        size_t bytes;
+    };
+    static std::mutex mu;
+    static Entry cache[256];
+    static int n = 0;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (int i = 0; i < n; ++i)
+            if (cache[i].dev == dev && cache[i].func == func && cache[i].bytes >= bytes) return cudaSuccess;
+    }
+    err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < n; ++i)
+        if (cache[i].dev == dev && cache[i].func == func) {
+            if (cache[i].bytes < bytes) cache[i].bytes = bytes;
+            return cudaSuccess;
+        }
+    if (n < 256) cache[n++] = Entry{dev, func, bytes};
+    return cudaSuccess;
+}
+
+static int next_pow2(int v) {
+    int p = 1;
+    while (p < v) p <<= 1;
+    return p;
+}
+
+static size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
+
+int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
+    DevInfo di;
+    cudaError_t err = dev_info(di);
+    if (err != cudaSuccess) return cuda_fail(err, "device query");
+    const int nb = a.nb;
+    if (fmt == KQ_FMT_Q4_K) {
+        const int ur = 2 * nb;  // half-block units per row pair
+        const int lr = ur <= 32 ? next_pow2(ur) : static_cast<int>(round_up(ur, 32));
+        if (lr > kConsumers) return fail(KQ_ERR_UNSUPPORTED, "Q4_K with K=%lld > 32768", (long long)a.K);
+        a.lanes_per_rp = lr;
+        a.ps = kConsumers / lr;
+        a.parts = lr > 32 ? lr / 32 : 1;
+    } else {
+        if (nb % 8 != 0)
+            return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld",
+                        (long long)a.K);
+        const int urw = 2 * (nb / 8);  // units per row pair in each of the 8 warps
+        if (urw > 32) return fail(KQ_ERR_UNSUPPORTED, "Q6_K with K=%lld > 32768", (long long)a.K);
+        const int lrw = next_pow2(urw);
+        a.lanes_per_rp = lrw;
+        a.ps = 32 / lrw;
+        a.parts = kConsumerWarps;
+    }
+    const size_t stage = round_up(static_cast<size_t>(a.ps) * 2 * a.row_bytes + 32, 128);
+    const size_t wp_bytes = round_up(sizeof(float) * 2 * a.ps * a.parts * 2 * ncol, 128);
+    const size_t xs_bytes = round_up(sizeof(float) * ncol * 2 * nb * kRegion, 128);
+    const size_t head = 256;
+    const size_t fixed = head + wp_bytes + xs_bytes;
+    size_t limit = static_cast<size_t>(di.smem_optin);
+    if (fixed + 2 * stage > limit)
+        return fail(KQ_ERR_UNSUPPORTED, "K=%lld with %d columns needs %zu bytes of shared memory (limit %zu)",
+                    (long long)a.K, ncol, fixed + 2 * stage, limit);
+    // Two resident CTAs per SM hide more latency (measured +17% on the
+    // 28672 x 4096 Q4_K matrix); used for the single-column Q4_K kernel
+    // whenever two copies of its shared memory fit in one SM.
+    int ctas = 1;
+    const size_t share = static_cast<size_t>(di.smem_per_sm) / 2 - 1024;
+    if (fmt == KQ_FMT_Q4_K && ncol == 1 && fixed + 2 * stage <= share) {
+        ctas = 2;
+        limit = share;
+    }
+    size_t ns = (limit - fixed) / stage;
+    if (ns > 6) ns = 6;
+    // no more stages than the busiest CTA will ever use
+    const int64_t rps = (a.N + 1) / 2;
+    const int64_t P = static_cast<int64_t>(a.n_seg) * rps;
+    const int64_t slots = static_cast<int64_t>(di.sm_count) * ctas;
+    const int64_t grid = P < slots ? P : slots;
+    const int64_t per_cta = (P + grid - 1) / grid;
+    const int64_t need = (per_cta + a.ps - 1) / a.ps + (a.n_seg > 1 ? 1 : 0);
+    if (static_cast<int64_t>(ns) > need) ns = need < 2 ? 2 : static_cast<size_t>(need);
+    a.nstage = static_cast<int>(ns);
+    a.stage_bytes = static_cast<int>(stage);
+    a.wp_offset = static_cast<int>(head);
+    a.xs_offset = static_cast<int>(head + wp_bytes);
+    a.sbuf_offset = static_cast<int>(fixed);
+    p.grid = static_cast<int>(grid);
+    p.ctas = ctas;
+    p.smem_bytes = fixed + ns * stage;
+    p.pdl = true;
+    return KQ_OK;
+}
+
+static bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+static int check_matrix(const void* W, int fmt, int64_t N, int64_t K) {
+    if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q6_K) return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
+    if (N < 0 || K < 0) return fail(KQ_ERR_INVALID_ARG, "negative size N=%lld K=%lld", (long long)N, (long long)K);
+    if (K % 256 != 0) return fail(KQ_ERR_INVALID_ARG, "K=%lld is not a multiple of 256", (long long)K);
+    if (N > 0 && K > 0) {
+        if (!W) return fail(KQ_ERR_INVALID_ARG, "W is NULL");
+        if (!aligned(W, 16)) return fail(KQ_ERR_INVALID_ARG, "W is not 16-byte aligned");
+    }
+    if (N > (int64_t(1) << 31)) return fail(KQ_ERR_UNSUPPORTED, "N=%lld too large", (long long)N);
+    return KQ_OK;
+}
+
+// Kernels exist for 1, 2, 4 and 8 columns; other counts run padded (the
+// extra columns repeat the last real one and are not written back), which
+// leaves every real column's arithmetic unchanged.
+static int padded_cols(int k) { return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : 8; }
+
+static cudaError_t dispatch(const GemvArgs& a, const LaunchPlan& p, int fmt, int ncol, cudaStream_t s) {
+    if (fmt == KQ_FMT_Q4_K) {
+        switch (ncol) {
+            case 1: return p.ctas == 2 ? launch_one<1, 1, 2>(a, p, s) : launch_one<1, 1, 1>(a, p, s);
+            case 2: return launch_one<1, 2, 1>(a, p, s);
+            case 4: return launch_one<1, 4, 1>(a, p, s);
+            default: return launch_one<1, 8, 1>(a, p, s);
+        }
+    }
+    switch (ncol) {
+        case 1: return launch_one<2, 1, 1>(a, p, s);
+        case 2: return launch_one<2, 2, 1>(a, p, s);
+        case 4: return launch_one<2, 4, 1>(a, p, s);
+        default: return launch_one<2, 8, 1>(a, p, s);
+    }
+}
+
+static int run(GemvArgs& a, int fmt, int k, cudaStream_t stream) {
+    const int ncol = padded_cols(k);
+    a.ncol_real = k;
+    cudaError_t err = fault_word(&a.fault);
+    if (err != cudaSuccess) return cuda_fail(err, "fault word");
+    LaunchPlan p;
+    int st = plan_gemv(fmt, ncol, a, p);
+    if (st != KQ_OK) return st;
+    err = dispatch(a, p, fmt, ncol, stream);
+    if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    return KQ_OK;
+}
+
+// Largest padded column count whose staged activations fit in shared
+// memory next to a two-stage weight ring (0 if not even one column fits).
+static int max_fitting_cols(const GemvArgs& proto, int fmt) {
+    for (int c = 8; c >= 1; c >>= 1) {
+        GemvArgs t = proto;
+        LaunchPlan p;
+        if (plan_gemv(fmt, c, t, p) == KQ_OK) return c;
+    }
+    return 0;
+}
+
+// k columns in groups that fit; each group is one launch (the weights are
+// read once per group).  Every column's arithmetic is the same whatever the
+// grouping, so results do not depend on it.
+static int run_grouped(GemvArgs& a, int fmt, int k, cudaStream_t stream) {
+    const int g = max_fitting_cols(a, fmt);
+    if (g == 0) {
+        LaunchPlan p;
+        return plan_gemv(fmt, 1, a, p);  // fails again, recording the reason
+    }
+    g_last_error[0] = 0;
+    for (int c0 = 0; c0 < k; c0 += g) {
+        GemvArgs t = a;
+        t.x = a.x + static_cast<int64_t>(c0) * a.ldx;
+        t.y = a.y + static_cast<int64_t>(c0) * a.ldy;
+        const int kk = k - c0 < g ? k - c0 : g;
+        int st = run(t, fmt, kk, stream);
+        if (st != KQ_OK) return st;
+    }
+    return KQ_OK;
+}
+
+// Outputs of an empty dot product (K == 0) are zero.
+static int zero_outputs(float* y, int64_t ldy, int64_t rows, int cols, cudaStream_t stream) {
+    for (int j = 0; j < cols; ++j) {
+        cudaError_t err = cudaMemsetAsync(y + j * ldy, 0, sizeof(float) * rows, stream);
+        if (err != cudaSuccess) return cuda_fail(err, "cudaMemsetAsync");
+    }
+    return KQ_OK;
+}
+
+}  // namespace kq
+
+using namespace kq;
+
+extern "C" {
+
+int kq_version(void) { return 100; }
+
+const char* kq_status_str(int status) {
+    switch (status) {
+        case KQ_OK: return "ok";
+        case KQ_ERR_INVALID_ARG: return "invalid argument";
+        case KQ_ERR_UNSUPPORTED: return "unsupported";
+        case KQ_ERR_NOT_PINNED: return "host memory not pinned";
+        case KQ_ERR_OOM: return "out of memory";
+        case KQ_ERR_CUDA: return "CUDA error";
+        case KQ_ERR_TIMEOUT: return "timeout";
+        case KQ_ERR_DEVICE_CHECK: return "device-side check failed";
+        case KQ_ERR_INJECTED: return "injected failure";
+        default: return "unknown status";
+    }
+}
+
+const char* kq_last_error(void) { return g_last_error; }
+
+size_t kq_block_bytes(int fmt) {
+    return fmt == KQ_FMT_Q4_K ? kQ4Bytes : fmt == KQ_FMT_Q6_K ? kQ6Bytes : 0;
+}
+
+size_t kq_row_bytes(int fmt, int64_t K) {
+    if (K < 0 || K % 256 != 0) return 0;
+    return static_cast<size_t>(K / 256) * kq_block_bytes(fmt);
+}
+
+int kq_device_fault(int* out) {
+    g_last_error[0] = 0;
+    if (!out) return fail(KQ_ERR_INVALID_ARG, "out is NULL");
+    cudaError_t err = read_and_clear_fault(out);
+    if (err != cudaSuccess) return cuda_fail(err, "read fault word");
+    return KQ_OK;
+}
+
+int kq_gemv_multi(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx, int k, float* y,
+                  int64_t ldy, kq_stream_t stream) {
+    g_last_error[0] = 0;
+    int st = check_matrix(W, fmt, N, K);
+    if (st != KQ_OK) return st;
+    if (k < 1 || k > 8) return fail(KQ_ERR_INVALID_ARG, "k=%d outside 1..8", k);
+    if (N == 0) return KQ_OK;
+    if (!y || !aligned(y, 4)) return fail(KQ_ERR_INVALID_ARG, "y is NULL or misaligned");
+    if (k > 1 && ldy < N) return fail(KQ_ERR_INVALID_ARG, "ldy=%lld < N", (long long)ldy);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (K == 0) return zero_outputs(y, ldy, N, k, s);
+    if (!x || !aligned(x, 4)) return fail(KQ_ERR_INVALID_ARG, "x is NULL or misaligned");
+    if (k > 1 && ldx < K) return fail(KQ_ERR_INVALID_ARG, "ldx=%lld < K", (long long)ldx);
+    GemvArgs a = {};
+    a.W = static_cast<const uint8_t*>(W);
+    a.N = N;
+    a.K = K;
+    a.row_bytes = static_cast<int64_t>(kq_row_bytes(fmt, K));
+    a.nb = static_cast<int>(K / 256);
+    a.n_seg = 1;
+    a.ids = nullptr;
+    a.E = 1;
+    a.seg_stride = 0;
+    a.x = x;
+    a.ldx = ldx;
+    a.x_seg_stride = 0;
+    a.y = y;
+    a.ldy = ldy;
+    a.y_seg_stride = 0;
+    a.status = nullptr;
+    return run_grouped(a, fmt, k, s);
+}
+
+int kq_gemv(const void* W, int fmt, int64_t N, int64_t K, const float* x, float* y, kq_stream_t stream) {
+    return kq_gemv_multi(W, fmt, N, K, x, K, 1, y, N, stream);
+}
+
+int kq_moe_gemv(const void* W_experts, int fmt, int E, int64_t N, int64_t K, size_t expert_stride_bytes,
+                const int32_t* ids, int n_ids, const float* x, int64_t x_stride, float* y, int32_t* status,
+                kq_stream_t stream) {
+    g_last_error[0] = 0;
+    int st = check_matrix(W_experts, fmt, N, K);
+    if (st != KQ_OK) return st;
+    if (E < 1) return fail(KQ_ERR_INVALID_ARG, "E=%d < 1", E);
+    if (n_ids < 0) return fail(KQ_ERR_INVALID_ARG, "n_ids=%d < 0", n_ids);
+    if (n_ids == 0 || N == 0) return KQ_OK;
+    if (!ids || !aligned(ids, 4)) return fail(KQ_ERR_INVALID_ARG, "ids is NULL or misaligned");
+    if (!y || !aligned(y, 4)) return fail(KQ_ERR_INVALID_ARG, "y is NULL or misaligned");
+    if (status && !aligned(status, 4)) return fail(KQ_ERR_INVALID_ARG, "status misaligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (K == 0) return zero_outputs(y, N, N, n_ids, s);
+    const size_t rb = kq_row_bytes(fmt, K);
+    if (expert_stride_bytes < static_cast<size_t>(N) * rb || expert_stride_bytes % 16 != 0)
+        return fail(KQ_ERR_INVALID_ARG, "expert stride %zu must be >= N*row_bytes and a multiple of 16",
+                    expert_stride_bytes);
+    if (!x || !aligned(x, 4)) return fail(KQ_ERR_INVALID_ARG, "x is NULL or misaligned");
+    if (x_stride != 0 && x_stride < K) return fail(KQ_ERR_INVALID_ARG, "x_stride=%lld < K", (long long)x_stride);
+    GemvArgs a = {};
+    a.W = static_cast<const uint8_t*>(W_experts);
+    a.N = N;
+    a.K = K;
+    a.row_bytes = static_cast<int64_t>(rb);
+    a.nb = static_cast<int>(K / 256);
+    a.n_seg = n_ids;
+    a.ids = ids;
+    a.E = E;
+    a.seg_stride = static_cast<int64_t>(expert_stride_bytes);
+    a.x = x;
+    a.ldx = K;
+    a.x_seg_stride = x_stride;
+    a.y = y;
+    a.ldy = 0;
+    a.y_seg_stride = N;
+    a.status = status;
+    return run(a, fmt, 1, s);
+}
+
+int kq_unpack(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d, kq_stream_t stream) {
+    g_last_error[0] = 0;
+    if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q6_K) return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
+    if (n_blocks < 0) return fail(KQ_ERR_INVALID_ARG, "n_blocks < 0");
+    if (n_blocks == 0) return KQ_OK;
+    if (!W || !q || !sc || !d) return fail(KQ_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(W, 16) || !aligned(d, 4)) return fail(KQ_ERR_INVALID_ARG, "misaligned pointer");
+    cudaError_t err = launch_unpack(static_cast<const uint8_t*>(W), fmt, n_blocks, q, sc, d,
+                                    reinterpret_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return cuda_fail(err, "unpack launch");
+    return KQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,164 @@
+// kq_device.cuh — sm_100a device helpers for libkq: mbarrier / bulk-copy
+// (TMA) PTX wrappers, bounded waits, and the K-quant unpack primitives the
+// GEMV kernels and the debug unpack kernel share.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+
+namespace kq {
+
+constexpr int kQ4Bytes = 144;      // Q4_K super-block
+constexpr int kQ6Bytes = 210;      // Q6_K super-block
+constexpr int kConsumerWarps = 8;  // warps that dequantise and multiply
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers + 32;  // + one producer (TMA) warp
+constexpr int kRegion = 132;       // floats per activation region: 128 x + 4 sums
+constexpr int kMaxStages = 8;
+constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded-wait limit (2 s)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Make initialised barriers visible to the async (TMA) proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete, giving up after kWaitNs or
+// when another thread of the CTA has raised `abort_flag`.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 15u) == 0) {  // the timer and the flag are checked now and then
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitNs) return false;
+        }
+    }
+}
+
+// 1-D bulk copy global -> shared (the TMA engine, no tensor map, no
+// multicast), completing `bytes` of transaction count on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier that also returns the OR of `pred` over its threads, so a
+// decision taken after it is the same in every participating thread.
+__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+// Programmatic dependent launch: wait for the preceding grid's memory, and
+// allow the next grid to start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ float4 lds128f(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+__device__ __forceinline__ uint32_t u4w(const uint4& v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// ----------------------------------------------------------------- Q4_K
+
+// The four 6-bit scales and four 6-bit mins of half H (sub-blocks
+// 4H..4H+3) of a Q4_K super-block, one per byte.  w1, w2, w3 are the 12
+// scale bytes (little-endian words).  For j < 4 the scale/min are the low 6
+// bits of bytes j / j+4; for j >= 4 the low 4 bits come from byte j+4 (scale
+// in its low nibble, min in its high nibble) and the top 2 bits from bits
+// 6-7 of byte j-4 (scale) / byte j (min).
+__device__ __forceinline__ void q4k_half_scales(uint32_t w1, uint32_t w2, uint32_t w3, int H, uint32_t& sc4,
+                                                uint32_t& m4) {
+    const uint32_t sc_lo = w1 & 0x3F3F3F3Fu;
+    const uint32_t m_lo = w2 & 0x3F3F3F3Fu;
+    const uint32_t sc_hi = (w3 & 0x0F0F0F0Fu) | ((w1 >> 2) & 0x30303030u);
+    const uint32_t m_hi = ((w3 >> 4) & 0x0F0F0F0Fu) | ((w2 >> 2) & 0x30303030u);
+    sc4 = H ? sc_hi : sc_lo;
+    m4 = H ? m_hi : m_lo;
+}
+
+// ----------------------------------------------------------------- Q6_K
+
+// The 6-bit quants of 4 consecutive positions l..l+3 of a Q6_K half, for
+// the four 32-weight quarters t = 0..3, one per byte.  A = ql[l..l+3],
+// B = ql[32+l..], Hh = qh[l..] of that half.  Quarter t takes its low 4 bits
+// from A (t = 0, 2) or B (t = 1, 3), low nibble for t < 2, high nibble
+// otherwise, and its top 2 bits from bits 2t..2t+1 of Hh.
+__device__ __forceinline__ void q6k_build(uint32_t A, uint32_t B, uint32_t Hh, uint32_t& q0, uint32_t& q1,
+                                          uint32_t& q2, uint32_t& q3) {
+    q0 = (A & 0x0F0F0F0Fu) | ((Hh << 4) & 0x30303030u);
+    q1 = (B & 0x0F0F0F0Fu) | ((Hh << 2) & 0x30303030u);
+    q2 = ((A >> 4) & 0x0F0F0F0Fu) | (Hh & 0x30303030u);
+    q3 = ((B >> 4) & 0x0F0F0F0Fu) | ((Hh >> 2) & 0x30303030u);
+}
+
+// ------------------------------------------------------ float conversion
+
+// Float with value 1 + b/128 from a byte b|0x80 placed in bits 16..23
+// (exponent byte 0x3F supplied by the constant); `sel_k` picks byte k.
+__device__ __forceinline__ float magic_unit(uint32_t packed, int k) {
+    return __uint_as_float(__byte_perm(packed, 0x3F000000u, 0x7054u | (static_cast<uint32_t>(k) << 8)));
+}
+
+// Float with value 2^23 + b for byte k of `packed`.
+__device__ __forceinline__ float magic_2p23(uint32_t packed, int k) {
+    return __uint_as_float(__byte_perm(packed, 0x4B000000u, 0x7650u | static_cast<uint32_t>(k)));
+}
+
+}  // namespace kq

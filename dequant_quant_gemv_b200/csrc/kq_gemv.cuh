@@ -1,0 +1,572 @@
+// kq_gemv.cuh — fused dequant-GEMV kernels for GGUF Q4_K / Q6_K on sm_100a.
+//
+// The product computed is y = W x with W dequantised only in registers
+// ("Out-of-core LLM inference engine written from scratch in Rust",
+// Approach: dequantisation inside fused matmul kernels; "Kortex: Streaming
+// 70B Models on Consumer GPUs", Key components 3).  Decode is bound by
+// weight bytes (same page, the paragraph before the first table), so the
+// kernel is organised around streaming the weights once from HBM:
+//
+//  * One persistent CTA per SM owns a contiguous range of row pairs.  Rows
+//    are contiguous in memory, so a stage (a few row pairs, ~37-54 KB) is ONE
+//    1-D TMA bulk copy into a ring of shared-memory buffers, tracked by
+//    mbarriers (full: transaction bytes landed; empty: consumers done).
+//  * Warp 0 is the producer.  Warps 1..8 dequantise from shared memory in
+//    registers.  A consumer lane owns one unit = (row pair, super-block,
+//    half) = 2 x 128 weights, so the activation values it loads serve two
+//    rows.  The lane->unit order makes every 16-byte shared load of a
+//    quarter-warp hit distinct banks.
+//  * Activations are staged once per CTA in a permuted, padded layout that
+//    matches the lane's consumption order (pairs for the packed fp32 FMA).
+//  * Reduction: butterfly over the lanes of a row pair, then a fixed-order
+//    sum over warps.  Every output has one fixed summation order, so results
+//    are bitwise reproducible and independent of the column count, the grid
+//    and the stage boundaries.
+//
+// Quant -> float.  Q4_K: a nibble n becomes 1 + n/128 (low nibble) or
+// 1 + n/16 (high nibble) by one byte permute into an exponent-0x7F float;
+// the unit offset is removed after the dot product by subtracting the
+// sub-block's activation sum, which the staging pass accumulates with the
+// very same fused-multiply-add sequence (so all-zero quants cancel exactly).
+// Q6_K: q becomes 2^23 + q by a byte permute, then q - 32 exactly by one
+// packed add.  Products and sums are fp32 (packed f32x2 FMA on sm_100a).
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kq_device.cuh"
+#include "kq_internal.h"
+
+namespace kq {
+
+// Packed fp32 (f32x2) fused multiply-add / add, round to nearest: one
+// instruction for two independent lanes on sm_100a.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// ------------------------------------------------------------ the units
+
+// Q4_K unit: rows r0 (and r0+1) of a row pair, super-block b, half H
+// (sub-blocks 4H..4H+3, i.e. 32-byte quant chunks c = 2H and 2H+1).
+// xr: the unit's activation region for column 0; column j at xr + j*xcs.
+template <int NCOL>
+__device__ __forceinline__ void q4k_unit(const uint8_t* row0, int row_bytes, int b, int H, const float* xr,
+                                         int xcs, float (&out)[2][NCOL]) {
+    const uint8_t* blk[2] = {row0 + b * kQ4Bytes, row0 + row_bytes + b * kQ4Bytes};
+    float2 A2[2][2], NB2[2][2];  // [row][c'] (128 d sc, 16 d sc'), (-dmin m, -dmin m')
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint4 hd = lds128(blk[r]);
+        uint32_t sc4, m4;
+        q4k_half_scales(hd.y, hd.z, hd.w, H, sc4, m4);
+        const float2 dd = make_float2(__half2float(__ushort_as_half(static_cast<unsigned short>(hd.x & 0xFFFFu))),
+                                      __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x >> 16))));
+        const float2 dscale = make_float2(dd.x * 128.0f, dd.x * 16.0f);
+        const float2 nmin = make_float2(-dd.y, -dd.y);
+        const float2 m23 = make_float2(-8388608.0f, -8388608.0f);
+#pragma unroll
+        for (int cp = 0; cp < 2; ++cp) {
+            float2 scf = make_float2(magic_2p23(sc4, 2 * cp), magic_2p23(sc4, 2 * cp + 1));
+            float2 mf = make_float2(magic_2p23(m4, 2 * cp), magic_2p23(m4, 2 * cp + 1));
+            scf = __fadd2_rn(scf, m23);
+            mf = __fadd2_rn(mf, m23);
+            A2[r][cp] = __fmul2_rn(dscale, scf);
+            NB2[r][cp] = __fmul2_rn(nmin, mf);
+        }
+    }
+    float2 y2[2][NCOL];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int j = 0; j < NCOL; ++j) y2[r][j] = make_float2(0.f, 0.f);
+
+#pragma unroll
+    for (int cp = 0; cp < 2; ++cp) {
+        float2 acc[2][NCOL];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int j = 0; j < NCOL; ++j) acc[r][j] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int qoff = 16 + 64 * H + 32 * cp + 16 * h;
+            const uint4 q0 = lds128(blk[0] + qoff);
+            const uint4 q1 = lds128(blk[1] + qoff);
+            const float* xp = xr + (cp * 2 + h) * 32;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const uint32_t w0 = u4w(q0, t), w1 = u4w(q1, t);
+                const uint32_t lo0 = (w0 & 0x0F0F0F0Fu) | 0x80808080u;
+                const uint32_t hi0 = ((w0 >> 1) & 0x78787878u) | 0x80808080u;
+                const uint32_t lo1 = (w1 & 0x0F0F0F0Fu) | 0x80808080u;
+                const uint32_t hi1 = ((w1 >> 1) & 0x78787878u) | 0x80808080u;
+                float4 xa[NCOL], xb[NCOL];
+#pragma unroll
+                for (int j = 0; j < NCOL; ++j) {
+                    xa[j] = lds128f(xp + j * xcs + 8 * t);
+                    xb[j] = lds128f(xp + j * xcs + 8 * t + 4);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 f0 = make_float2(magic_unit(lo0, k), magic_unit(hi0, k));
+                    const float2 f1 = make_float2(magic_unit(lo1, k), magic_unit(hi1, k));
+#pragma unroll
+                    for (int j = 0; j < NCOL; ++j) {
+                        const float2 xv = k == 0   ? make_float2(xa[j].x, xa[j].y)
+                                          : k == 1 ? make_float2(xa[j].z, xa[j].w)
+                                          : k == 2 ? make_float2(xb[j].x, xb[j].y)
+                                                   : make_float2(xb[j].z, xb[j].w);
+                        acc[0][j] = fma2(f0, xv, acc[0][j]);
+                        acc[1][j] = fma2(f1, xv, acc[1][j]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < NCOL; ++j) {
+            const float2 X2 = *reinterpret_cast<const float2*>(xr + j * xcs + 128 + 2 * cp);
+            const float2 nX2 = make_float2(-X2.x, -X2.y);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const float2 D = __fadd2_rn(acc[r][j], nX2);
+                y2[r][j] = __ffma2_rn(A2[r][cp], D, y2[r][j]);
+                y2[r][j] = __ffma2_rn(NB2[r][cp], X2, y2[r][j]);
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int j = 0; j < NCOL; ++j) out[r][j] = y2[r][j].x + y2[r][j].y;
+}
+
+// Activation sums of one Q4_K region, accumulated exactly as q4k_unit
+// accumulates a chunk whose quants are all zero (factor 1.0).
+__device__ __forceinline__ float2 q4k_region_sum(const float* xr, int cp) {
+    float2 acc = make_float2(0.f, 0.f);
+    const float2 one = make_float2(1.0f, 1.0f);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float* xp = xr + (cp * 2 + h) * 32;
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 xv = *reinterpret_cast<const float2*>(xp + 8 * t + 2 * k);
+                acc = __ffma2_rn(one, xv, acc);
+            }
+    }
+    return acc;
+}
+
+// Q6_K unit: row pair, super-block b, half H (groups 8H..8H+7).  Blocks
+// are 210 bytes, so within a 16-byte aligned row a block starts at an even
+// but not necessarily 4-byte aligned offset: ODD marks blocks that start 2
+// bytes past a 4-byte boundary (b odd).  The warp's blocks all share that
+// class, so the branch is uniform and only two code paths exist.  Loads are
+// 4-byte words; for ODD blocks each stream word is rebuilt from two loaded
+// words with one byte permute.
+template <int NCOL, bool ODD>
+__device__ __forceinline__ void q6k_unit(const uint8_t* row0, int row_bytes, int b, int H, const float* xr,
+                                         int xcs, float (&out)[2][NCOL]) {
+    uint32_t QL[2][16], QH[2][8];
+    float2 sA[2][2], sB[2][2];
+    float dsc[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint8_t* blk = row0 + r * row_bytes + b * kQ6Bytes;
+        const uint32_t* bw = reinterpret_cast<const uint32_t*>(blk - (ODD ? 2 : 0));
+        auto sw = [&](int i) -> uint32_t {
+            if constexpr (ODD) return __byte_perm(bw[i], bw[i + 1], 0x5432);
+            else return bw[i];
+        };
+#pragma unroll
+        for (int i = 0; i < 16; ++i) QL[r][i] = sw(16 * H + i);   // ql[64H .. 64H+63]
+#pragma unroll
+        for (int i = 0; i < 8; ++i) QH[r][i] = sw(32 + 8 * H + i);  // qh[32H .. 32H+31]
+        // 8 signed scales of this half (bytes 192+8H..) as floats: flip the
+        // sign bit to get s+128 as an unsigned byte, 2^23 + (s+128) by byte
+        // permute, then subtract 2^23 + 128.
+        const uint32_t s0 = sw(48 + 2 * H) ^ 0x80808080u;
+        const uint32_t s1 = sw(49 + 2 * H) ^ 0x80808080u;
+        const uint32_t dword = ODD ? (bw[52] >> 16) : bw[52];  // d = bytes 208..209
+        const float2 off = make_float2(-8388736.0f, -8388736.0f);
+        // groups: sh = 0 -> (8H+0, 8H+4) / (8H+2, 8H+6); sh = 1 -> +1
+        sA[r][0] = __fadd2_rn(make_float2(magic_2p23(s0, 0), magic_2p23(s1, 0)), off);
+        sA[r][1] = __fadd2_rn(make_float2(magic_2p23(s0, 1), magic_2p23(s1, 1)), off);
+        sB[r][0] = __fadd2_rn(make_float2(magic_2p23(s0, 2), magic_2p23(s1, 2)), off);
+        sB[r][1] = __fadd2_rn(make_float2(magic_2p23(s0, 3), magic_2p23(s1, 3)), off);
+        dsc[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(dword & 0xFFFFu)));
+    }
+    float2 accA[2][2][NCOL], accB[2][2][NCOL];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int sh = 0; sh < 2; ++sh)
+#pragma unroll
+            for (int j = 0; j < NCOL; ++j) accA[r][sh][j] = accB[r][sh][j] = make_float2(0.f, 0.f);
+    const float2 c32 = make_float2(-8388640.0f, -8388640.0f);  // -(2^23 + 32)
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        const int sh = s >> 2;
+        uint32_t qv[2][4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) q6k_build(QL[r][s], QL[r][8 + s], QH[r][s], qv[r][0], qv[r][1], qv[r][2], qv[r][3]);
+        const float* xp = xr + 16 * s;
+        float4 xa0[NCOL], xa1[NCOL], xb0[NCOL], xb1[NCOL];
+#pragma unroll
+        for (int j = 0; j < NCOL; ++j) {
+            xa0[j] = lds128f(xp + j * xcs);
+            xa1[j] = lds128f(xp + j * xcs + 4);
+            xb0[j] = lds128f(xp + j * xcs + 8);
+            xb1[j] = lds128f(xp + j * xcs + 12);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const float2 fA = fadd2(make_float2(magic_2p23(qv[r][0], k), magic_2p23(qv[r][2], k)), c32);
+                const float2 fB = fadd2(make_float2(magic_2p23(qv[r][1], k), magic_2p23(qv[r][3], k)), c32);
+#pragma unroll
+                for (int j = 0; j < NCOL; ++j) {
+                    const float2 xA = k == 0   ? make_float2(xa0[j].x, xa0[j].y)
+                                      : k == 1 ? make_float2(xa0[j].z, xa0[j].w)
+                                      : k == 2 ? make_float2(xa1[j].x, xa1[j].y)
+                                               : make_float2(xa1[j].z, xa1[j].w);
+                    const float2 xB = k == 0   ? make_float2(xb0[j].x, xb0[j].y)
+                                      : k == 1 ? make_float2(xb0[j].z, xb0[j].w)
+                                      : k == 2 ? make_float2(xb1[j].x, xb1[j].y)
+                                               : make_float2(xb1[j].z, xb1[j].w);
+                    accA[r][sh][j] = fma2(fA, xA, accA[r][sh][j]);
+                    accB[r][sh][j] = fma2(fB, xB, accB[r][sh][j]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int j = 0; j < NCOL; ++j) {
+            float2 y2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int sh = 0; sh < 2; ++sh) {
+                y2 = __ffma2_rn(sA[r][sh], accA[r][sh][j], y2);
+                y2 = __ffma2_rn(sB[r][sh], accB[r][sh][j], y2);
+            }
+            out[r][j] = dsc[r] * (y2.x + y2.y);
+        }
+}
+
+// ------------------------------------------------------- stage sequence
+
+struct Stage {
+    int64_t seg;    // segment (matrix or routed id) index
+    int64_t row0;   // first row within the segment
+    int nrp;        // row pairs in the stage
+    int nrows;      // real rows (nrp*2, or one less at an odd tail)
+};
+
+// The CTA's stages: consecutive groups of at most `ps` row pairs of its
+// range [rp, rp_end), never crossing a segment boundary.
+// (One division at construction; next() only adds and compares.)  Also
+// tracks the ring slot and mbarrier phase of the stage it returns.
+struct StageIter {
+    int64_t left;        // row pairs still to hand out
+    int64_t seg, off;    // segment and row-pair offset within it
+    int64_t rps, N;
+    int ps, ns;
+    int slot = -1;       // ring slot of the last stage returned
+    uint32_t phase = 0;  // its mbarrier phase parity
+    int count = 0;       // stages returned so far
+    __device__ StageIter(int64_t rp_begin, int64_t rp_end, int64_t rps_, int64_t N_, int ps_, int ns_)
+        : left(rp_end - rp_begin), seg(rp_begin / rps_), off(rp_begin - (rp_begin / rps_) * rps_), rps(rps_),
+          N(N_), ps(ps_), ns(ns_) {}
+    __device__ bool next(Stage& st) {
+        if (left <= 0) return false;
+        if (off == rps) {
+            ++seg;
+            off = 0;
+        }
+        int64_t n = left < ps ? left : ps;
+        if (n > rps - off) n = rps - off;
+        st.seg = seg;
+        st.row0 = 2 * off;
+        st.nrp = static_cast<int>(n);
+        const int64_t rows = N - st.row0;
+        st.nrows = static_cast<int>(rows < 2 * n ? rows : 2 * n);
+        off += n;
+        left -= n;
+        if (++slot == ns) {
+            slot = 0;
+            phase ^= 1u;
+        }
+        ++count;
+        return true;
+    }
+};
+
+__device__ __forceinline__ void raise_fault(const GemvArgs& a, volatile int* abort_flag, int code) {
+    *abort_flag = 1;
+    if (a.status) atomicExch(a.status, code);
+    if (a.fault) atomicExch(a.fault, code);
+}
+
+// ------------------------------------------------------ activation stage
+
+// Stage the activations of segment `seg` (all NCOL columns) into the
+// padded, permuted layout the units read, then (Q4_K) the region sums.
+template <int FMT, int NCOL>
+__device__ void stage_x(const GemvArgs& a, int64_t seg, float* xs, int ct) {
+    const float* xg = a.x + seg * a.x_seg_stride;
+    const int nb = a.nb;
+    const int nreg = 2 * nb;
+    const int xcs = nreg * kRegion;
+    // fill: one item = 4 consecutive activations (a coalesced 16-byte load
+    // when the column is 16-byte aligned), scattered into the region layout;
+    // the 4 values land 2 floats apart (pair members alternate).
+    const int k4 = static_cast<int>(a.K >> 2);
+    const int items = NCOL * k4;
+    for (int it = ct; it < items; it += kConsumers) {
+        const int j = it / k4;
+        const int i = 4 * (it - j * k4);
+        const float* xc = xg + (j < a.ncol_real ? j : a.ncol_real - 1) * a.ldx;
+        float4 v;
+        if ((reinterpret_cast<uintptr_t>(xc) & 15u) == 0) v = *reinterpret_cast<const float4*>(xc + i);
+        else v = make_float4(xc[i], xc[i + 1], xc[i + 2], xc[i + 3]);
+        const int b = i >> 8, within = i & 255;
+        int off;
+        if constexpr (FMT == 1) {
+            // weight 64c + 32*hi + 16h + 4t + k of block b -> region 2b + c/2,
+            // pair (c%2, h, t, k), member hi
+            const int c = within >> 6, w64 = within & 63, hi = w64 >> 5, l = w64 & 31;
+            const int h = l >> 4, t = (l >> 2) & 3;
+            off = (2 * b + (c >> 1)) * kRegion + ((c & 1) * 2 + h) * 32 + 8 * t + hi;
+        } else {
+            // weight 128H + 32t + 4s + k of block b = 8i + kappa -> region
+            // (kappa*nb8 + i)*2 + H; pair A = (t0, t2), pair B = (t1, t3)
+            const int H = within >> 7, w128 = within & 127, t = w128 >> 5, sidx = (w128 & 31) >> 2;
+            const int kappa = b & 7, ib = b >> 3;
+            off = ((kappa * (nb >> 3) + ib) * 2 + H) * kRegion + 16 * sidx + ((t & 1) ? 8 : 0) + (t >> 1);
+        }
+        float* dst = xs + j * xcs + off;
+        dst[0] = v.x;
+        dst[2] = v.y;
+        dst[4] = v.z;
+        dst[6] = v.w;
+    }
+    named_bar_sync(1, kConsumers);
+    if constexpr (FMT == 1) {
+        const int sums = NCOL * nreg * 2;
+        for (int it = ct; it < sums; it += kConsumers) {
+            const int j = it / (nreg * 2);
+            const int rem = it - j * nreg * 2;
+            const int reg = rem >> 1, cp = rem & 1;
+            float* xr = xs + j * xcs + reg * kRegion;
+            const float2 X = q4k_region_sum(xr, cp);
+            *reinterpret_cast<float2*>(xr + 128 + 2 * cp) = X;
+        }
+        named_bar_sync(1, kConsumers);
+    }
+}
+
+// Dispatch a Q6_K unit to the code path of its alignment class.
+template <int NCOL>
+__device__ __forceinline__ void q6k_unit_dispatch(int kappa, const uint8_t* row0, int row_bytes, int b, int H,
+                                                  const float* xr, int xcs, float (&out)[2][NCOL]) {
+    if (kappa & 1) q6k_unit<NCOL, true>(row0, row_bytes, b, H, xr, xcs, out);
+    else q6k_unit<NCOL, false>(row0, row_bytes, b, H, xr, xcs, out);
+}
+
+// ------------------------------------------------------------ the kernel
+
+template <int FMT, int NCOL, int CTAS>
+__global__ void __launch_bounds__(kThreads, CTAS) gemv_kernel(const __grid_constant__ GemvArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 2 * kMaxStages * 8);
+    float* wp = reinterpret_cast<float*>(smem + a.wp_offset);
+    float* xs = reinterpret_cast<float*>(smem + a.xs_offset);
+    uint8_t* sbuf = smem + a.sbuf_offset;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int ns = a.nstage;
+
+    if (tid == 0) {
+        for (int s = 0; s < ns; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    const int64_t rps = (a.N + 1) / 2;
+    const int64_t P = static_cast<int64_t>(a.n_seg) * rps;
+    const int64_t rp_begin = P * blockIdx.x / gridDim.x;
+    const int64_t rp_end = P * (blockIdx.x + 1) / gridDim.x;
+
+    if (warp == 0) {
+        // ------------------------------------------------ producer (TMA)
+        if (lane != 0) return;
+        if (a.ids) pdl_wait();  // routed ids may come from the previous grid
+        StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
+        Stage st;
+        bool ok = true;
+        while (it.next(st)) {
+            const int slot = it.slot;
+            // a reused slot: wait until the consumers released its last stage
+            if (it.count > ns && !mbar_wait_bounded(&empty[slot], it.phase ^ 1u, abort_flag)) {
+                raise_fault(a, abort_flag, 6);
+                ok = false;
+                break;
+            }
+            int64_t e = st.seg;
+            if (a.ids) e = a.ids[st.seg];
+            if (e >= 0 && e < a.E) {
+                const uint8_t* src = a.W + e * a.seg_stride + st.row0 * a.row_bytes;
+                const uint32_t bytes = static_cast<uint32_t>(st.nrows * a.row_bytes);
+                mbar_arrive_expect_tx(&full[slot], bytes);
+                bulk_g2s(sbuf + static_cast<size_t>(slot) * a.stage_bytes, src, bytes, &full[slot]);
+            } else {
+                mbar_arrive(&full[slot]);
+            }
+        }
+        // Let every copy this CTA issued land before the CTA can exit.
+        int issued = ok ? it.count : it.count - 1;
+        int sl = ok ? it.slot : (it.slot == 0 ? ns - 1 : it.slot - 1);
+        uint32_t ph = ok ? it.phase : (it.slot == 0 ? it.phase ^ 1u : it.phase);
+        for (int i = 0; i < issued && i < ns; ++i) {
+            if (!mbar_wait_bounded(&full[sl], ph, abort_flag)) break;
+            if (--sl < 0) {
+                sl = ns - 1;
+                ph ^= 1u;
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    const int ct = tid - 32;        // consumer thread 0..255
+    const int cw = warp - 1;        // consumer warp 0..7
+    const int nb = a.nb;
+    const int xcs = 2 * nb * kRegion;
+    pdl_wait();                      // activations may come from the previous grid
+    pdl_launch_dependents();
+
+    // this lane's unit within a stage
+    int u_rp, u_b, u_H, group, part;
+    bool u_active;
+    int kappa = 0;
+    if (FMT == 1) {
+        const int LR = a.lanes_per_rp;
+        u_rp = ct / LR;
+        const int u = ct - u_rp * LR;
+        u_active = u < 2 * nb;
+        u_b = u >> 1;
+        u_H = u & 1;
+        group = LR < 32 ? LR : 32;
+        part = LR > 32 ? (u >> 5) : 0;
+    } else {
+        const int LRw = a.lanes_per_rp;  // lanes per row pair inside one warp
+        kappa = cw;
+        u_rp = lane / LRw;
+        const int u = lane - u_rp * LRw;
+        const int nb8 = nb >> 3;
+        u_active = u < 2 * nb8;
+        const int i = u >> 1;
+        u_H = u & 1;
+        u_b = 8 * i + kappa;
+        group = LRw;
+        part = kappa;
+    }
+    const int parts = a.parts;
+    int region;
+    if (FMT == 1) region = 2 * u_b + u_H;
+    else region = ((kappa * (nb >> 3) + (u_b >> 3)) << 1) + u_H;
+    const float* xr = xs + region * kRegion;
+
+    StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
+    Stage st;
+    int64_t staged_seg = -1;
+    while (it.next(st)) {
+        if (staged_seg < 0 || (a.x_seg_stride != 0 && st.seg != staged_seg)) {
+            stage_x<FMT, NCOL>(a, st.seg, xs, ct);
+            staged_seg = st.seg;
+        }
+        const int slot = it.slot;
+        if (!mbar_wait_bounded(&full[slot], it.phase, abort_flag)) raise_fault(a, abort_flag, 6);
+        float out[2][NCOL];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int j = 0; j < NCOL; ++j) out[r][j] = 0.f;
+        const bool work = u_active && u_rp < st.nrp && !*abort_flag;
+        if (work) {
+            const uint8_t* row0 = sbuf + static_cast<size_t>(slot) * a.stage_bytes +
+                                  static_cast<size_t>(2 * u_rp) * a.row_bytes;
+            if constexpr (FMT == 1) q4k_unit<NCOL>(row0, static_cast<int>(a.row_bytes), u_b, u_H, xr, xcs, out);
+            else q6k_unit_dispatch<NCOL>(kappa, row0, static_cast<int>(a.row_bytes), u_b, u_H, xr, xcs, out);
+        }
+        // butterfly over the lanes of this row pair (fixed order)
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            if (off < group) {
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+#pragma unroll
+                    for (int j = 0; j < NCOL; ++j) out[r][j] += __shfl_xor_sync(0xffffffffu, out[r][j], off);
+            }
+        }
+        float* wb = wp + (it.count & 1) * (a.ps * parts * 2 * NCOL);
+        if ((lane & (group - 1)) == 0 && u_rp < a.ps) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int j = 0; j < NCOL; ++j) wb[((u_rp * parts + part) * 2 + r) * NCOL + j] = out[r][j];
+        }
+        const bool stop = named_bar_or(1, kConsumers, *abort_flag != 0);
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (stop) break;
+        // fixed-order sum over parts, then store
+        int64_t e = st.seg;
+        if (a.ids) e = a.ids[st.seg];
+        const bool valid = e >= 0 && e < a.E;
+        if (!valid && ct == 0 && a.status) atomicExch(a.status, 7);
+        for (int t = ct; t < st.nrows * NCOL; t += kConsumers) {
+            const int row = t / NCOL, j = t - row * NCOL;
+            const int rp = row >> 1, r = row & 1;
+            float v = 0.f;
+            if (valid) {
+                for (int p = 0; p < parts; ++p) v += wb[((rp * parts + p) * 2 + r) * NCOL + j];
+            }
+            if (j < a.ncol_real) a.y[st.seg * a.y_seg_stride + j * a.ldy + st.row0 + row] = v;
+        }
+    }
+}
+
+
+// ----------------------------------------------------------- launchers
+
+template <int FMT, int NCOL, int CTAS>
+cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream) {
+    auto kern = gemv_kernel<FMT, NCOL, CTAS>;
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), p.smem_bytes);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = p.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = p.pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+}  // namespace kq

@@ -1,0 +1,59 @@
+// kq_internal.h — host/device shared definitions of libkq (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace kq {
+
+// Kernel arguments of one fused GEMV launch.  A launch covers n_seg
+// "segments" of N rows each: one matrix (n_seg = 1), or the routed experts
+// of a MoE layer (segment i = expert ids[i]).
+struct GemvArgs {
+    const uint8_t* W;        // matrix, or expert 0 of the expert stack
+    int64_t N, K;
+    int64_t row_bytes;
+    int nb;                  // super-blocks per row (K / 256)
+    int n_seg;
+    const int32_t* ids;      // routed expert ids (device) or nullptr
+    int E;                   // valid segment ids are [0, E)
+    int64_t seg_stride;      // bytes between experts
+    const float* x;
+    int64_t ldx;             // floats between activation columns
+    int64_t x_seg_stride;    // floats between segments' activations (0 = shared)
+    float* y;
+    int64_t ldy;             // floats between output columns
+    int64_t y_seg_stride;    // floats between segments' outputs
+    int32_t* status;         // optional device status word
+    int* fault;              // device fault word (timeouts)
+    int ncol_real;           // columns written (the kernel may pad to 2/4/8)
+    // schedule (from plan_gemv)
+    int ps;                  // row pairs per stage
+    int lanes_per_rp;        // Q4_K: lanes per row pair; Q6_K: per row pair and warp
+    int parts;               // partial sums per row pair
+    int nstage;
+    int stage_bytes;
+    int wp_offset, xs_offset, sbuf_offset;
+};
+
+struct LaunchPlan {
+    int grid;
+    int ctas;        // CTAs resident per SM the schedule was sized for (1 or 2)
+    size_t smem_bytes;
+    bool pdl;
+};
+
+// Fills the schedule fields of `a` and the launch plan; returns a kq_status.
+int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p);
+
+template <int FMT, int NCOL, int CTAS>
+cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
+cudaError_t fault_word(int** out);
+cudaError_t launch_unpack(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d,
+                          cudaStream_t stream);
+cudaError_t ensure_smem_attr(const void* func, size_t bytes);
+cudaError_t read_and_clear_fault(int* out);
+
+}  // namespace kq

@@ -1,0 +1,96 @@
+// kq_misc.cu — the debug unpack kernel and the device fault word.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kq_device.cuh"
+#include "kq_internal.h"
+
+namespace kq {
+
+// Set by a kernel whose bounded wait ran out (launches without a caller
+// status pointer); read and cleared by kq_device_fault().
+__device__ int g_kq_fault = 0;
+
+// ------------------------------------------------------- debug unpack
+
+// One thread per super-block: the integer fields, decoded with the same
+// helpers the GEMV kernels use.
+__global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d) {
+    const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (b >= nblocks) return;
+    if (fmt == 1) {
+        const uint8_t* blk = W + b * kQ4Bytes;
+        const uint4 hd = *reinterpret_cast<const uint4*>(blk);
+        for (int H = 0; H < 2; ++H) {
+            uint32_t sc4, m4;
+            q4k_half_scales(hd.y, hd.z, hd.w, H, sc4, m4);
+            for (int k = 0; k < 4; ++k) {
+                sc[16 * b + 4 * H + k] = static_cast<uint8_t>(sc4 >> (8 * k));
+                sc[16 * b + 8 + 4 * H + k] = static_cast<uint8_t>(m4 >> (8 * k));
+            }
+        }
+        d[2 * b] = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x & 0xFFFFu)));
+        d[2 * b + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x >> 16)));
+        for (int w = 0; w < 32; ++w) {
+            const uint32_t v = *reinterpret_cast<const uint32_t*>(blk + 16 + 4 * w);
+            const int c = w >> 3, l0 = (w & 7) * 4;
+            for (int k = 0; k < 4; ++k) {
+                q[256 * b + 64 * c + l0 + k] = static_cast<uint8_t>((v >> (8 * k)) & 15u);
+                q[256 * b + 64 * c + 32 + l0 + k] = static_cast<uint8_t>((v >> (8 * k + 4)) & 15u);
+            }
+        }
+    } else {
+        const uint8_t* blk = W + b * kQ6Bytes;  // 2-byte aligned only
+        auto word = [&](int off) -> uint32_t {
+            return static_cast<uint32_t>(blk[off]) | (static_cast<uint32_t>(blk[off + 1]) << 8) |
+                   (static_cast<uint32_t>(blk[off + 2]) << 16) | (static_cast<uint32_t>(blk[off + 3]) << 24);
+        };
+        for (int H = 0; H < 2; ++H)
+            for (int s = 0; s < 8; ++s) {
+                uint32_t qv[4];
+                q6k_build(word(64 * H + 4 * s), word(64 * H + 32 + 4 * s), word(128 + 32 * H + 4 * s), qv[0], qv[1],
+                          qv[2], qv[3]);
+                for (int t = 0; t < 4; ++t)
+                    for (int k = 0; k < 4; ++k)
+                        q[256 * b + 128 * H + 32 * t + 4 * s + k] = static_cast<uint8_t>(qv[t] >> (8 * k));
+            }
+        for (int g = 0; g < 16; ++g) sc[16 * b + g] = blk[192 + g];
+        const unsigned short dh = static_cast<unsigned short>(blk[208] | (blk[209] << 8));
+        d[2 * b] = __half2float(__ushort_as_half(dh));
+        d[2 * b + 1] = 0.0f;
+    }
+}
+
+cudaError_t launch_unpack(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d,
+                          cudaStream_t stream) {
+    const int threads = 128;
+    const int64_t grid = (nblocks + threads - 1) / threads;
+    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+    unpack_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(W, fmt, nblocks, q, sc, d);
+    return cudaGetLastError();
+}
+
+// The fault word's device address, looked up once per device.
+cudaError_t fault_word(int** out) {
+    static int* cache[64] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= 0 && dev < 64 && cache[dev]) {
+        *out = cache[dev];
+        return cudaSuccess;
+    }
+    err = cudaGetSymbolAddress(reinterpret_cast<void**>(out), g_kq_fault);
+    if (err == cudaSuccess && dev >= 0 && dev < 64) cache[dev] = *out;
+    return err;
+}
+
+cudaError_t read_and_clear_fault(int* out) {
+    int zero = 0;
+    cudaError_t err = cudaMemcpyFromSymbol(out, g_kq_fault, sizeof(int));
+    if (err != cudaSuccess) return err;
+    return cudaMemcpyToSymbol(g_kq_fault, &zero, sizeof(int));
+}
+
+}  // namespace kq

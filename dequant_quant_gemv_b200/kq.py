@@ -1,0 +1,145 @@
+"""Python binding of libkq (argument marshalling only).
+
+Every computation runs in the CUDA kernels of ``libkq.so``; this module only
+passes device pointers, sizes and the current torch stream through the C
+ABI declared in ``include/kq.h``.  There is no CPU fallback: if the library
+is missing or fails to load, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkq.so")
+
+Q4_K = 1
+Q6_K = 2
+FORMATS = {"q4_k": Q4_K, "q6_k": Q6_K}
+BLOCK_BYTES = {Q4_K: 144, Q6_K: 210}
+
+OK = 0
+STATUS = {0: "KQ_OK", 1: "KQ_ERR_INVALID_ARG", 2: "KQ_ERR_UNSUPPORTED", 3: "KQ_ERR_NOT_PINNED",
+          4: "KQ_ERR_OOM", 5: "KQ_ERR_CUDA", 6: "KQ_ERR_TIMEOUT", 7: "KQ_ERR_DEVICE_CHECK",
+          8: "KQ_ERR_INJECTED"}
+
+_lib = None
+
+
+class KQError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({detail})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libkq.so (built in-tree by ``dequant_quant_gemv_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libkq.so not built at {LIB_PATH}; run python -m dequant_quant_gemv_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, i32, vp, sz = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+        L.kq_version.restype = i32
+        L.kq_status_str.restype = ctypes.c_char_p
+        L.kq_status_str.argtypes = [i32]
+        L.kq_last_error.restype = ctypes.c_char_p
+        L.kq_device_fault.restype = i32
+        L.kq_device_fault.argtypes = [ctypes.POINTER(ctypes.c_int)]
+        L.kq_block_bytes.restype = sz
+        L.kq_block_bytes.argtypes = [i32]
+        L.kq_row_bytes.restype = sz
+        L.kq_row_bytes.argtypes = [i32, i64]
+        L.kq_gemv.restype = i32
+        L.kq_gemv.argtypes = [vp, i32, i64, i64, vp, vp, vp]
+        L.kq_gemv_multi.restype = i32
+        L.kq_gemv_multi.argtypes = [vp, i32, i64, i64, vp, i64, i32, vp, i64, vp]
+        L.kq_moe_gemv.restype = i32
+        L.kq_moe_gemv.argtypes = [vp, i32, i32, i64, i64, sz, vp, i32, vp, i64, vp, vp, vp]
+        L.kq_unpack.restype = i32
+        L.kq_unpack.argtypes = [vp, i32, i64, vp, vp, vp, vp]
+        _lib = L
+    return _lib
+
+
+def _fmt(fmt) -> int:
+    return FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def _check(status: int, what: str) -> None:
+    if status != OK:
+        raise KQError(status, what, lib().kq_last_error().decode())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def row_bytes(fmt, K: int) -> int:
+    return int(lib().kq_row_bytes(_fmt(fmt), K))
+
+
+def gemv(W: torch.Tensor, fmt, N: int, K: int, x: torch.Tensor, y: torch.Tensor | None = None,
+         stream=None) -> torch.Tensor:
+    """y = W x.  W: uint8 device tensor of N*row_bytes; x: K float32."""
+    if y is None:
+        y = torch.empty(N, dtype=torch.float32, device=x.device)
+    _check(lib().kq_gemv(_dev(W, "W"), _fmt(fmt), N, K, _dev(x, "x", torch.float32),
+                         _dev(y, "y", torch.float32), _stream(stream)), "kq_gemv")
+    return y
+
+
+def gemv_multi(W: torch.Tensor, fmt, N: int, K: int, X: torch.Tensor, Y: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """Y[c] = W X[c] for the k rows of X (shape (k, K), rows may be strided)."""
+    k = X.shape[0]
+    if Y is None:
+        Y = torch.empty((k, N), dtype=torch.float32, device=X.device)
+    _check(lib().kq_gemv_multi(_dev(W, "W"), _fmt(fmt), N, K, _dev(X, "X", torch.float32), X.stride(0), k,
+                               _dev(Y, "Y", torch.float32), Y.stride(0), _stream(stream)), "kq_gemv_multi")
+    return Y
+
+
+def moe_gemv(W_experts: torch.Tensor, fmt, E: int, N: int, K: int, ids: torch.Tensor, x: torch.Tensor,
+             y: torch.Tensor | None = None, status: torch.Tensor | None = None, expert_stride: int | None = None,
+             stream=None) -> torch.Tensor:
+    """y[i] = W_{ids[i]} x_i; x is (K,) shared or (n_ids, K) per id."""
+    n = ids.numel()
+    if expert_stride is None:
+        expert_stride = N * row_bytes(fmt, K)
+    if y is None:
+        y = torch.empty((n, N), dtype=torch.float32, device=x.device)
+    x_stride = 0 if x.dim() == 1 else x.stride(0)
+    _check(lib().kq_moe_gemv(_dev(W_experts, "W_experts"), _fmt(fmt), E, N, K, expert_stride,
+                             _dev(ids, "ids", torch.int32), n, _dev(x, "x", torch.float32), x_stride,
+                             _dev(y, "y", torch.float32), None if status is None else _dev(status, "status"),
+                             _stream(stream)), "kq_moe_gemv")
+    return y
+
+
+def unpack(W: torch.Tensor, fmt, n_blocks: int, stream=None):
+    """(q, sc, d) integer fields as decoded on the GPU (see kq.h)."""
+    q = torch.empty(n_blocks * 256, dtype=torch.uint8, device=W.device)
+    sc = torch.empty(n_blocks * 16, dtype=torch.uint8, device=W.device)
+    d = torch.empty(n_blocks * 2, dtype=torch.float32, device=W.device)
+    _check(lib().kq_unpack(_dev(W, "W"), _fmt(fmt), n_blocks, q.data_ptr(), sc.data_ptr(), d.data_ptr(),
+                           _stream(stream)), "kq_unpack")
+    return q, sc, d
+
+
+def device_fault() -> int:
+    out = ctypes.c_int(0)
+    _check(lib().kq_device_fault(ctypes.byref(out)), "kq_device_fault")
+    return out.value

@@ -1,0 +1,162 @@
+/*
+ * kq.h — libkq: decode-time matrix-vector products over GGUF K-quant
+ * weights (Q4_K, Q6_K) on NVIDIA B200 (sm_100a), with the weights
+ * dequantised only in registers inside the fused kernels.
+ *
+ * What the method is (by page):
+ *  - "Out-of-core LLM inference engine written from scratch in Rust",
+ *    Approach: quantised weights are dequantised inside fused matmul kernels;
+ *    speculative decoding verifies several positions with one pass; layer
+ *    weights move through a ring of VRAM slots while the GPU computes nearby
+ *    layers.  Results: Llama-3.3-70B Q4_K_M; a fully resident 30B MoE.
+ *  - "Kortex: Streaming 70B Models on Consumer GPUs", Key components 2-3:
+ *    the streaming pipeline overlaps transfers with compute; weights are
+ *    dequantised only in GPU registers.  Token generation is memory-bandwidth
+ *    bound (the paragraph before the first table).
+ *  - "RunNburn - Run a 295B MoE from a 98GB GGUF ...": only the experts the
+ *    router selects for a token are touched; native K-quant kernels.
+ *
+ * Weight layout.  A matrix has N output rows and K inputs (K % 256 == 0).
+ * Row r is K/256 consecutive super-blocks; rows follow each other with no
+ * gap, so row r starts at W + r * kq_row_bytes(fmt, K).
+ *   Q4_K super-block, 144 bytes, 256 weights in 8 sub-blocks of 32:
+ *     fp16 d | fp16 dmin | 12 bytes of 6-bit scales sc_j and mins m_j |
+ *     128 bytes of 4-bit quants q.   w = d*sc_j*q - dmin*m_j.
+ *   Q6_K super-block, 210 bytes, 256 weights in 16 groups of 16:
+ *     128 bytes low 4 bits | 64 bytes high 2 bits | 16 int8 scales s_g |
+ *     fp16 d.   w = d*s_g*(q - 32), q in 0..63.
+ *   (The GGUF K-quant bit layout; the pages name the formats but print no
+ *   layout.)
+ *
+ * Conventions for every entry point:
+ *  - All pointers named W, x, y, ids, status are DEVICE pointers owned by the
+ *    caller; libkq never frees or retains them past the call (the chain object
+ *    below is the exception and says so).
+ *  - W must be 16-byte aligned, and so must every row: always true for Q4_K;
+ *    for Q6_K it requires K % 2048 == 0.  x and y must be 4-byte aligned.
+ *  - Calls are asynchronous on `stream` (0 = the legacy default stream).  The
+ *    return value reports argument validation and launch errors only
+ *    (KQ_ERR_CUDA carries cudaGetLastError()); kq_last_error() gives text.
+ *  - Arithmetic: quants are unpacked exactly; products and sums are fp32.
+ *    Every output satisfies |y - y_exact| <= 1e-3 * sum_i |w_i x_i| + 1e-6.
+ *    Results are deterministic: the same inputs give bitwise-equal outputs,
+ *    and column c of kq_gemv_multi equals kq_gemv on column c.
+ *  - No C++ exception crosses this interface.  Functions without shared state
+ *    are thread-safe; a kq_chain must not be used by two threads at once.
+ */
+#ifndef KQ_H_
+#define KQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KQ_API __attribute__((visibility("default")))
+#else
+#define KQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA runtime's cudaStream_t, without pulling in the CUDA headers. */
+typedef struct CUstream_st* kq_stream_t;
+
+typedef enum {
+    KQ_FMT_Q4_K = 1,
+    KQ_FMT_Q6_K = 2
+} kq_fmt;
+
+typedef enum {
+    KQ_OK = 0,
+    KQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad format, misalignment */
+    KQ_ERR_UNSUPPORTED = 2,   /* valid but not handled (e.g. Q6_K with K % 2048 != 0) */
+    KQ_ERR_NOT_PINNED = 3,    /* host memory that must be page-locked is not */
+    KQ_ERR_OOM = 4,           /* a device or pinned allocation failed */
+    KQ_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+    KQ_ERR_TIMEOUT = 6,       /* a bounded wait ran out */
+    KQ_ERR_DEVICE_CHECK = 7,  /* a device-side check failed (see kq_moe_gemv) */
+    KQ_ERR_INJECTED = 8       /* a failure requested through KQ_FAULT (tests) */
+} kq_status;
+
+/* Library version as 10000*major + 100*minor + patch. */
+KQ_API int kq_version(void);
+
+/* Static text for a status code. */
+KQ_API const char* kq_status_str(int status);
+
+/* Text describing the last failure on the calling thread ("" if none). */
+KQ_API const char* kq_last_error(void);
+
+/* Reads and clears the current device's fault word (0 if no fault): a
+ * kernel whose bounded wait ran out sets it to KQ_ERR_TIMEOUT instead of
+ * hanging.  Synchronous.  *out is a HOST int. */
+KQ_API int kq_device_fault(int* out);
+
+/* Bytes per super-block (144 or 210) or 0 for an unknown format. */
+KQ_API size_t kq_block_bytes(int fmt);
+
+/* Bytes per weight row: (K/256) * kq_block_bytes(fmt); 0 if K % 256 != 0. */
+KQ_API size_t kq_row_bytes(int fmt, int64_t K);
+
+/*
+ * kq_gemv — y = W x for one quantised matrix.
+ *   W: N x K matrix in `fmt` (device).  x: K floats (device).  y: N floats
+ *   (device, written).  N >= 1, K >= 256, K % 256 == 0.
+ * The fused dequant-matmul of "Out-of-core LLM inference engine written from
+ * scratch in Rust" (Approach) and "Kortex: Streaming 70B Models on Consumer
+ * GPUs" (Key components 3): each weight is read from HBM once and
+ * dequantised in registers.
+ */
+KQ_API int kq_gemv(const void* W, int fmt, int64_t N, int64_t K, const float* x, float* y,
+            kq_stream_t stream);
+
+/*
+ * kq_gemv_multi — Y = W X for k activation columns sharing one weight read.
+ *   X column c is x + c*ldx (K floats each, ldx >= K); Y column c is
+ *   y + c*ldy (N floats each, ldy >= N); 1 <= k <= 8.
+ * The verify pass of speculative decoding ("Out-of-core LLM inference engine
+ * ...", Approach: several positions verified with one pass of the large
+ * model).  Column c equals kq_gemv(W, x + c*ldx) bitwise.
+ */
+KQ_API int kq_gemv_multi(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx,
+                  int k, float* y, int64_t ldy, kq_stream_t stream);
+
+/*
+ * kq_moe_gemv — routed-expert GEMV.
+ *   W_experts: E matrices, each N x K in `fmt`, matrix e at
+ *   W_experts + e*expert_stride_bytes (stride >= N*row_bytes, 16-byte
+ *   multiple).  ids: n_ids int32 expert ids (DEVICE memory, read by the
+ *   kernel).  x: if x_stride == 0 one K-vector shared by all ids, else id i
+ *   uses x + i*x_stride (x_stride >= K).  y: n_ids x N floats, row-major
+ *   (y + i*N is the output for the i-th id).
+ *   An id outside [0, E) is not dereferenced: its N outputs are set to 0 and,
+ *   if status is not NULL, *status (device int32) is set to
+ *   KQ_ERR_DEVICE_CHECK.  The kernel never traps.
+ * Only the selected experts' weights are read ("RunNburn ...": the selected
+ * experts for each token; "Out-of-core LLM inference engine ...", Results:
+ * a fully resident 30B MoE).  Output i equals kq_gemv on expert ids[i].
+ */
+KQ_API int kq_moe_gemv(const void* W_experts, int fmt, int E, int64_t N, int64_t K,
+                size_t expert_stride_bytes, const int32_t* ids, int n_ids, const float* x,
+                int64_t x_stride, float* y, int32_t* status, kq_stream_t stream);
+
+/*
+ * kq_unpack — debug: the integer fields of n_blocks consecutive super-blocks
+ * as the GEMV kernels decode them (for bit-exact comparison).
+ *   q:  n_blocks*256 bytes, quant of weight i of block b at q[256b+i]
+ *       (Q4_K 0..15; Q6_K 0..63, before the -32 offset)
+ *   sc: n_blocks*16 bytes; Q4_K: sc_0..7 then m_0..7; Q6_K: the 16 int8
+ *       scales as two's-complement bytes
+ *   d:  n_blocks*2 floats; Q4_K: d, dmin; Q6_K: d, 0 (fp16 widened exactly)
+ * All device pointers; W must be 16-byte aligned.
+ */
+KQ_API int kq_unpack(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d,
+              kq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KQ_H_ */

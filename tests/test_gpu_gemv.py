@@ -1,0 +1,216 @@
+"""GPU parity of the fused K-quant GEMV (kq_gemv, kq_gemv_multi, kq_unpack)
+against the CPU oracle, on identical seeded inputs.
+
+Acceptance: integer fields bit-exact; every output within
+|y - y_ref| <= 1e-3 * sum_i |w_i x_i| + 1e-6 (the bound stated for the
+method's decode GEMV); cross-API equalities bitwise.
+"""
+import numpy as np
+import pytest
+import torch
+
+import kqgen
+import oracle
+from kqtest import ABS, assert_close, dev, matrix, oracle_gemv, x_vec
+
+pytestmark = pytest.mark.gpu
+
+kq = pytest.importorskip("dequant_quant_gemv_b200.kq")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    kq.lib()
+
+
+# ------------------------------------------------------------ bit-exact
+@pytest.mark.parametrize("fmt,N,K", [("q4_k", 4096, 4096), ("q6_k", 64, 14336), ("q6_k", 3, 2048)])
+def test_unpack_bit_exact(fmt, N, K):
+    W = matrix(fmt, 1000 + N, N, K)
+    nb = N * K // 256
+    q, sc, d = kq.unpack(dev(W), fmt, nb)
+    torch.cuda.synchronize()
+    q0, sc0, d0 = oracle.unpack(fmt, W, nb)
+    assert np.array_equal(q.cpu().numpy(), q0)
+    assert np.array_equal(sc.cpu().numpy(), sc0)
+    assert np.array_equal(d.cpu().numpy().view(np.uint32), d0.view(np.uint32))
+
+
+# -------------------------------------------------- parity, many shapes
+SHAPES = [
+    ("q4_k", 1, 256), ("q4_k", 3, 256), ("q4_k", 7, 768), ("q4_k", 33, 2048), ("q4_k", 64, 4096),
+    ("q4_k", 257, 4096), ("q4_k", 301, 8192), ("q4_k", 5, 1280), ("q4_k", 9, 32768), ("q4_k", 2, 5120),
+    ("q6_k", 1, 2048), ("q6_k", 5, 2048), ("q6_k", 64, 14336), ("q6_k", 37, 28672), ("q6_k", 300, 4096),
+    ("q6_k", 11, 16384),
+]
+
+
+@pytest.mark.parametrize("fmt,N,K", SHAPES)
+def test_gemv_parity(fmt, N, K):
+    W = matrix(fmt, 7 * N + K, N, K)
+    x = x_vec(N + 3 * K, K)
+    y = kq.gemv(dev(W), fmt, N, K, dev(x))
+    y_ref, s_ref = oracle_gemv(fmt, W, N, K, x)
+    assert_close(y, y_ref, s_ref, f"{fmt} {N}x{K}")
+
+
+def test_gemv_single_q4k_4096_full():
+    """The 4096 x 4096 Q4_K GEMV, every output against the oracle."""
+    N = K = 4096
+    W = matrix("q4_k", 0xC0FFEE, N, K)
+    x = x_vec(0xC0FFEE + 1, K)
+    y = kq.gemv(dev(W), "q4_k", N, K, dev(x))
+    y_ref, s_ref = oracle_gemv("q4_k", W, N, K, x)
+    worst = assert_close(y, y_ref, s_ref, "cfg 4096x4096")
+    assert worst < 0.05   # typical error is far inside the bound
+
+
+def test_deterministic():
+    N, K = 1000, 4096
+    Wd = dev(matrix("q4_k", 5, N, K))
+    xd = dev(x_vec(6, K))
+    a = kq.gemv(Wd, "q4_k", N, K, xd)
+    b = kq.gemv(Wd, "q4_k", N, K, xd)
+    assert torch.equal(a, b)
+
+
+# --------------------------------------------------- degenerate cases
+def test_q4k_zero_quants_and_zero_mins_give_exact_zero():
+    N, K = 70, 4096
+    nb = N * K // 256
+    lg = kqgen.q4k_draw(21, nb)
+    W = kqgen.q4k_pack(np.zeros_like(lg["q"]), lg["sc"], np.zeros_like(lg["m"]), lg["d"], lg["dmin"])
+    y = kq.gemv(dev(W), "q4_k", N, K, dev(x_vec(22, K)))
+    assert torch.all(y == 0)
+
+
+def test_q4k_zero_quants_closed_form():
+    N, K = 70, 4096
+    nb = N * K // 256
+    lg = kqgen.q4k_draw(23, nb)
+    W = kqgen.q4k_pack(np.zeros_like(lg["q"]), lg["sc"], lg["m"], lg["d"], lg["dmin"])
+    x = x_vec(24, K)
+    y = kq.gemv(dev(W), "q4_k", N, K, dev(x))
+    X = x.astype(np.float64).reshape(K // 32, 32).sum(axis=1).reshape(K // 256, 8)
+    dmin = lg["dmin"].view(np.float16).astype(np.float64).reshape(N, K // 256)
+    m = lg["m"].astype(np.float64).reshape(N, K // 256, 8)
+    want = -np.einsum("rb,rbj,bj->r", dmin, m, X)
+    s = np.einsum("rb,rbj,bj->r", dmin, m, np.abs(x.astype(np.float64)).reshape(K // 32, 32).sum(1).reshape(K // 256, 8))
+    assert_close(y, want, s, "zero quants")
+
+
+def test_q6k_mid_quants_give_exact_zero():
+    N, K = 40, 14336
+    nb = N * K // 256
+    lg = kqgen.q6k_draw(25, nb)
+    W = kqgen.q6k_pack(np.full_like(lg["q"], 32), lg["s"], lg["d"])
+    y = kq.gemv(dev(W), "q6_k", N, K, dev(x_vec(26, K)))
+    assert torch.all(y == 0)
+
+
+def test_unit_scales_integer_matvec():
+    N, K = 50, 4096
+    nb = N * K // 256
+    lg = kqgen.q4k_draw(27, nb)
+    W = kqgen.q4k_pack(lg["q"], np.ones((nb, 8), np.uint8), np.zeros((nb, 8), np.uint8),
+                       np.full(nb, 0x3C00, np.uint16), np.zeros(nb, np.uint16))
+    x = x_vec(28, K)
+    Q = lg["q"].reshape(N, K).astype(np.float64)
+    y = kq.gemv(dev(W), "q4_k", N, K, dev(x))
+    assert_close(y, Q @ x.astype(np.float64), np.abs(Q) @ np.abs(x.astype(np.float64)), "unit scales")
+
+
+@pytest.mark.parametrize("fmt,K", [("q4_k", 4096), ("q6_k", 14336)])
+def test_one_hot_extracts_column(fmt, K):
+    N = 16
+    W = matrix(fmt, 29, N, K)
+    Wd = oracle.dequant(fmt, W, N, K)
+    Wt = dev(W)
+    for i in (0, 1, 31, 32, 33, 255, 256, K - 1):
+        x = np.zeros(K, np.float32)
+        x[i] = 1.0
+        y = kq.gemv(Wt, fmt, N, K, dev(x)).cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(y - Wd[:, i]) <= 1e-6 * np.abs(Wd[:, i]) + ABS), i
+
+
+def test_linearity():
+    N, K = 128, 4096
+    Wt = dev(matrix("q4_k", 30, N, K))
+    rng = np.random.default_rng(0)
+    x1 = rng.integers(-8, 8, K).astype(np.float32)
+    x2 = rng.integers(-8, 8, K).astype(np.float32)
+    y1 = kq.gemv(Wt, "q4_k", N, K, dev(x1)).double()
+    y2 = kq.gemv(Wt, "q4_k", N, K, dev(x2)).double()
+    yc = kq.gemv(Wt, "q4_k", N, K, dev(2 * x1 - 3 * x2)).double()
+    _, s1 = oracle_gemv("q4_k", matrix("q4_k", 30, N, K), N, K, x1)
+    _, s2 = oracle_gemv("q4_k", matrix("q4_k", 30, N, K), N, K, x2)
+    bound = torch.from_numpy(2 * (2 * 1e-3 * s1 + 3 * 1e-3 * s2) + 1e-5).cuda()
+    assert torch.all((yc - (2 * y1 - 3 * y2)).abs() <= bound)
+
+
+# ---------------------------------------------------------- multi column
+@pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q4_k", 17, 768)])
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 5, 8])
+def test_multi_matches_single_bitwise_and_oracle(fmt, N, K, k):
+    W = matrix(fmt, 31 + k, N, K)
+    Wt = dev(W)
+    X = np.stack([x_vec(100 + c, K) for c in range(k)])
+    Xt = dev(X)
+    Y = kq.gemv_multi(Wt, fmt, N, K, Xt)
+    for c in range(k):
+        yc = kq.gemv(Wt, fmt, N, K, Xt[c].contiguous())
+        assert torch.equal(Y[c], yc), c
+    y_ref, s_ref = oracle.gemv_multi(fmt, W, N, K, X, nthreads=0)
+    for c in range(k):
+        assert_close(Y[c], y_ref[c], s_ref[c], f"col {c}")
+
+
+def test_multi_strided_columns():
+    N, K, k = 100, 4096, 4
+    W = matrix("q4_k", 40, N, K)
+    big = np.zeros((k, K + 64), np.float32)
+    for c in range(k):
+        big[c, :K] = x_vec(200 + c, K)
+    Xt = dev(big)[:, :K]
+    Yb = torch.full((k, N + 8), 7.0, device="cuda")
+    Y = kq.gemv_multi(dev(W), "q4_k", N, K, Xt, Yb[:, :N])
+    assert torch.all(Yb[:, N:] == 7.0)   # padding untouched
+    y_ref, s_ref = oracle.gemv_multi("q4_k", W, N, K, big[:, :K], nthreads=0)
+    for c in range(k):
+        assert_close(Y[c], y_ref[c], s_ref[c])
+
+
+# ----------------------------------------------------------------- edges
+def test_empty_and_degenerate_sizes():
+    x = torch.zeros(256, device="cuda")
+    y = torch.full((4,), 5.0, device="cuda")
+    W = torch.zeros(144 * 4, dtype=torch.uint8, device="cuda")
+    kq.gemv(W, "q4_k", 0, 256, x, y)               # N = 0: no-op
+    assert torch.all(y == 5.0)
+    kq.gemv(W, "q4_k", 4, 0, x, y)                 # K = 0: empty sums
+    assert torch.all(y == 0.0)
+
+
+def test_invalid_arguments_are_rejected():
+    W = torch.zeros(144 * 4, dtype=torch.uint8, device="cuda")
+    x = torch.zeros(256, device="cuda")
+    y = torch.zeros(4, device="cuda")
+    with pytest.raises(kq.KQError) as e:
+        kq.gemv(W, 9, 4, 256, x, y)
+    assert e.value.status == 1
+    with pytest.raises(kq.KQError) as e:
+        kq.gemv(W, "q4_k", 4, 300, x, y)
+    assert e.value.status == 1
+    with pytest.raises(kq.KQError) as e:
+        kq.gemv(W[1:], "q4_k", 1, 256, x, y)    # misaligned W
+    assert e.value.status == 1
+    Wq6 = torch.zeros(210 * 9, dtype=torch.uint8, device="cuda")
+    x9 = torch.zeros(2304, device="cuda")
+    with pytest.raises(kq.KQError) as e:
+        kq.gemv(Wq6, "q6_k", 1, 2304, x9, y)    # rows not 16-byte aligned
+    assert e.value.status == 2
+    with pytest.raises(kq.KQError):
+        kq.gemv_multi(W, "q4_k", 4, 256, torch.zeros((9, 256), device="cuda"))
+    assert kq.device_fault() == 0
