@@ -1,19 +1,26 @@
 #!/usr/bin/env python3
 """Benchmark of the fused K-quant dequant-GEMV path (libkq) on B200.
 
-Default workload: the Llama-3.1-8B-shaped decode chain at batch 1 -- per
-layer Wq|Wk|Wv (6144 x 4096), Wo (4096 x 4096), Wgate|Wup (28672 x 4096) in
-Q4_K and Wdown (4096 x 14336) in Q6_K, 32 layers, 4.41 GB of weights, which
-is larger than L2, so every step streams the weights from HBM.  One step is
-one pass of the whole chain (128 fused GEMV launches, replayed as one CUDA
-graph).  Metric: weight GB/s (algorithmic weight bytes / time) and
-layer-chain tokens/s.
+Default workload (the metric's configuration): the Llama-3.1-8B-shaped
+decode chain at batch 1 -- per layer Wq|Wk|Wv (6144 x 4096), Wo
+(4096 x 4096), Wgate|Wup (28672 x 4096) in Q4_K and Wdown (4096 x 14336) in
+Q6_K, 32 layers, 4.41 GB of weights (larger than L2, so every step streams
+the weights from HBM).  One step is one pass of the chain: 128 fused GEMV
+launches replayed as one CUDA graph.  Metric: weight GB/s (algorithmic weight
+bytes / time) and layer-chain tokens/s.
+
+Other workloads (--workload): gemv_q4k_4096 (one 4096 x 4096 Q4_K GEMV),
+verify8b_k{1,2,4,8} (the 8B chain with k activation columns),
+moe30b (Qwen3-30B-A3B-shaped routed experts, top-8 of 128, 48 layers),
+llama70b_resident / llama70b_stream (80-layer 70B-shaped chain in HBM, or
+streamed from pinned host memory through 4 device slots), gateup_q4k and
+down_q6k (single kernels, for profiling).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle on a bounded sample
 
-Multi-GPU: the chain does not shard in this benchmark; N ranks run N
-independent replicas (weak scaling) with no collective on the data path.
+Multi-GPU: the decode chain is one token's matvecs; ranks run independent
+replicas (weak scaling) with no collective on the data path.
 """
 from __future__ import annotations
 
@@ -33,36 +40,55 @@ sys.path.insert(0, ROOT)
 METRIC = "K-quant dequant-GEMV weight GB/s (% of B200 HBM peak); layer-chain tok/s"
 QK = 256
 BLOCK = {"q4_k": 144, "q6_k": 210}
+SEED = 0xC0FFEE + 1
 
 
 def row_bytes(fmt, K):
     return K // QK * BLOCK[fmt]
 
 
-# ----------------------------------------------------------------- workloads
-def chain_layers(hidden, heads, kv_heads, head_dim, ffn, n_layers):
-    """Per layer: (name, fmt, N, K, x-slot).  q|k|v share the attention input,
-    gate|up share the FFN input; each is one fused launch over the stacked rows."""
+def dense_layer(hidden, heads, kv_heads, head_dim, ffn):
+    """(name, fmt, N, K, x-slot): q|k|v share the attention input, gate|up
+    share the FFN input; each is one launch over the stacked rows."""
     qkv = (heads + 2 * kv_heads) * head_dim
-    mats = [("qkv", "q4_k", qkv, hidden, 0), ("o", "q4_k", hidden, heads * head_dim, 1),
+    return [("qkv", "q4_k", qkv, hidden, 0), ("o", "q4_k", hidden, heads * head_dim, 1),
             ("gate_up", "q4_k", 2 * ffn, hidden, 2), ("down", "q6_k", hidden, ffn, 3)]
-    return [mats for _ in range(n_layers)]
+
+
+L8B = dict(hidden=4096, heads=32, kv_heads=8, head_dim=128, ffn=14336)
+L70B = dict(hidden=8192, heads=64, kv_heads=8, head_dim=128, ffn=28672)
+MOE30B = dict(hidden=2048, experts=128, top=8, ffn=768, layers=48)
+
+
+def chain_spec(kind):
+    if kind == "llama8b":
+        return [dense_layer(**L8B) for _ in range(32)]
+    if kind == "llama70b":
+        return [dense_layer(**L70B) for _ in range(80)]
+    if kind == "gemv_q4k_4096":
+        return [[("w", "q4_k", 4096, 4096, 0)] for _ in range(64)]
+    if kind == "gateup_q4k":
+        return [[("gate_up", "q4_k", 28672, 4096, 0)] for _ in range(8)]
+    if kind == "down_q6k":
+        return [[("down", "q6_k", 4096, 14336, 0)] for _ in range(8)]
+    raise KeyError(kind)
 
 
 WORKLOADS = {
-    "llama8b_chain": dict(desc="Llama-3.1-8B-shaped decode chain, 32 layers, Q4_K + Q6_K down, batch 1",
-                          layers=lambda: chain_layers(4096, 32, 8, 128, 14336, 32)),
-    "gemv_q4k_4096": dict(desc="single Q4_K GEMV 4096 x 4096, batch 1 (64 distinct copies rotated)",
-                          layers=lambda: [[("w", "q4_k", 4096, 4096, 0)] for _ in range(64)]),
-    "gateup_q4k": dict(desc="Q4_K GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
-                       layers=lambda: [[("gate_up", "q4_k", 28672, 4096, 0)] for _ in range(8)]),
-    "down_q6k": dict(desc="Q6_K GEMV 4096 x 14336 (8B down), 8 distinct copies rotated",
-                     layers=lambda: [[("down", "q6_k", 4096, 14336, 0)] for _ in range(8)]),
+    "llama8b_chain": "Llama-3.1-8B-shaped decode chain, 32 layers, Q4_K + Q6_K down, batch 1",
+    "gemv_q4k_4096": "single Q4_K GEMV 4096 x 4096, batch 1 (64 distinct copies rotated)",
+    "gateup_q4k": "Q4_K GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
+    "down_q6k": "Q6_K GEMV 4096 x 14336 (8B down), 8 distinct copies rotated",
+    "verify8b_k1": "8B-shaped chain, speculative-verify GEMV with k=1 activation column",
+    "verify8b_k2": "8B-shaped chain, speculative-verify GEMV with k=2 activation columns",
+    "verify8b_k4": "8B-shaped chain, speculative-verify GEMV with k=4 activation columns",
+    "verify8b_k8": "8B-shaped chain, speculative-verify GEMV with k=8 activation columns",
+    "moe30b": "Qwen3-30B-A3B-shaped MoE GEMVs: 48 layers x 128 experts (gate|up 1536x2048, down 2048x768, "
+              "Q4_K), top-8 routed ids per token, batch 1",
+    "llama70b_resident": "Llama-3.3-70B-shaped decode chain, 80 layers, Q4_K + Q6_K down, resident in HBM",
+    "llama70b_stream": "Llama-3.3-70B-shaped decode chain, 80 layers, weights in pinned host memory streamed "
+                       "through 4 device layer slots",
 }
-
-
-def weight_bytes(layers):
-    return sum(N * row_bytes(fmt, K) for mats in layers for (_, fmt, N, K, _) in mats)
 
 
 # ------------------------------------------------------------------- clocks
@@ -81,10 +107,11 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            time.sleep(0.2)
         except (FileNotFoundError, OSError):
             self.proc = None
         return self
@@ -102,7 +129,7 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons, pw = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -111,42 +138,241 @@ class ClockSampler:
             try:
                 sm.append(float(parts[0]))
                 mx = float(parts[1])
+                pw.append(float(parts[2]))
             except ValueError:
                 continue
             for nm, v in zip(names, parts[3:7]):
                 if v.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "power_w_max": max(pw) if pw else None, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-# ------------------------------------------------------------ device setup
-def build_device_chain(layers, seed, torch, kqgen, pinned_host=False):
-    """Generate every weight matrix (host, parallel) and place it on the
-    device; activation vectors per layer slot; output buffers."""
-    dev_w, xs, ys = [], [], []
-    for li, mats in enumerate(layers):
-        wl, xl, yl = [], {}, []
-        for mi, (name, fmt, N, K, slot) in enumerate(mats):
-            host = np.empty(N * row_bytes(fmt, K), dtype=np.uint8)
-            kqgen.matrix(fmt, kqgen.tensor_seed(seed, li, mi), N, K, out=host)
-            t = torch.from_numpy(host)
-            wl.append(t.pin_memory() if pinned_host else t.cuda())
-            if slot not in xl:
-                xh = torch.from_numpy(kqgen.normal_f32(kqgen.tensor_seed(seed ^ 0x5A5A, li, slot), K))
-                xl[slot] = xh.cuda()
-            yl.append(torch.empty(N, dtype=torch.float32, device="cuda"))
+# --------------------------------------------------------------- workloads
+class Resident:
+    """A chain of fused GEMV launches over weights resident in HBM.
+
+    Activations of all matrices live in one device buffer (and one pinned
+    host buffer for the end-to-end leg), outputs likewise."""
+
+    graphable = True
+
+    def __init__(self, torch, kq, kqgen, spec, seed, k=1):
+        self.torch, self.kq, self.spec, self.k = torch, kq, spec, k
+        self.launches = [(li, mi) for li, mats in enumerate(spec) for mi in range(len(mats))]
+        self.weight_bytes = sum(N * row_bytes(f, K) for mats in spec for (_, f, N, K, _) in mats)
+        # activations: one slot per (layer, x-slot), k columns each
+        xoff, yoff, self.xslot, self.yslot = 0, 0, {}, {}
+        for li, mats in enumerate(spec):
+            for mi, (_, f, N, K, slot) in enumerate(mats):
+                if (li, slot) not in self.xslot:
+                    self.xslot[(li, slot)] = (xoff, K)
+                    xoff += k * K
+                self.yslot[(li, mi)] = (yoff, N)
+                yoff += k * N
+        self.X = torch.empty(xoff, dtype=torch.float32, device="cuda")
+        self.Y = torch.empty(yoff, dtype=torch.float32, device="cuda")
+        xh = np.empty(xoff, np.float32)
+        for (li, slot), (off, K) in self.xslot.items():
+            kqgen.normal_f32(kqgen.tensor_seed(seed ^ 0x5A5A, li, slot), k * K, out=xh[off:off + k * K])
+        self.X.copy_(torch.from_numpy(xh))
+        self.W = []
+        for li, mats in enumerate(spec):
+            row = []
+            for mi, (_, f, N, K, _) in enumerate(mats):
+                host = np.empty(N * row_bytes(f, K), np.uint8)
+                kqgen.matrix(f, kqgen.tensor_seed(seed, li, mi), N, K, out=host)
+                row.append(torch.from_numpy(host).cuda())
+            self.W.append(row)
         torch.cuda.synchronize()
-        dev_w.append(wl)
-        xs.append(xl)
-        ys.append(yl)
-    return dev_w, xs, ys
+
+    def x_of(self, li, mi):
+        off, K = self.xslot[(li, self.spec[li][mi][4])]
+        return self.X[off:off + self.k * K].view(self.k, K)
+
+    def y_of(self, li, mi):
+        off, N = self.yslot[(li, mi)]
+        return self.Y[off:off + self.k * N].view(self.k, N)
+
+    def launch(self, li, mi, stream):
+        _, f, N, K, _ = self.spec[li][mi]
+        if self.k == 1:
+            self.kq.gemv(self.W[li][mi], f, N, K, self.x_of(li, mi)[0], self.y_of(li, mi)[0], stream=stream)
+        else:
+            self.kq.gemv_multi(self.W[li][mi], f, N, K, self.x_of(li, mi), self.y_of(li, mi), stream=stream)
+
+    def step(self, stream):
+        for li, mi in self.launches:
+            self.launch(li, mi, stream)
+
+    def kinds(self):
+        out = {}
+        for li, mi in self.launches:
+            name, f, N, K, _ = self.spec[li][mi]
+            out.setdefault(name, dict(fmt=f, N=N, K=K, bytes=N * row_bytes(f, K), launches=[]))
+            out[name]["launches"].append((li, mi))
+        return out
+
+    def io(self):
+        return [self.X], [self.Y]
 
 
-def run_chain(kq, layers, dev_w, xs, ys, stream):
-    for li, mats in enumerate(layers):
-        for mi, (name, fmt, N, K, slot) in enumerate(mats):
-            kq.gemv(dev_w[li][mi], fmt, N, K, xs[li][slot], ys[li][mi], stream=stream)
+class MoE:
+    """Routed-expert GEMVs: per layer one launch for the routed experts'
+    gate|up rows (shared x) and one for their down rows (one x per id)."""
+
+    graphable = True
+
+    def __init__(self, torch, kq, kqgen, seed, tokens=4):
+        c = MOE30B
+        self.torch, self.kq = torch, kq
+        H, E, top, F, Lyr = c["hidden"], c["experts"], c["top"], c["ffn"], c["layers"]
+        self.E, self.top, self.H, self.F, self.L = E, top, H, F, Lyr
+        self.gu_stride = 2 * F * row_bytes("q4_k", H)
+        self.dn_stride = H * row_bytes("q4_k", F)
+        self.weight_bytes = Lyr * top * (self.gu_stride + self.dn_stride)
+        self.Wgu, self.Wdn = [], []
+        for l in range(Lyr):
+            h = np.empty(E * self.gu_stride, np.uint8)
+            kqgen.matrix("q4_k", kqgen.tensor_seed(seed, l, 0), E * 2 * F, H, out=h)
+            self.Wgu.append(torch.from_numpy(h).cuda())
+            h = np.empty(E * self.dn_stride, np.uint8)
+            kqgen.matrix("q4_k", kqgen.tensor_seed(seed, l, 1), E * H, F, out=h)
+            self.Wdn.append(torch.from_numpy(h).cuda())
+        # routed ids for `tokens` tokens; the step copies the next token's ids
+        # into the buffer the kernels read (as a router would write them)
+        ids = np.stack([np.stack([kqgen.topk_ids(kqgen.tensor_seed(seed ^ 0x1D5, t, l), E, top)
+                                  for l in range(Lyr)]) for t in range(tokens)])
+        self.ids_all = torch.from_numpy(ids).cuda()               # (tokens, L, top)
+        self.ids = torch.empty((Lyr, top), dtype=torch.int32, device="cuda")
+        self.t = 0
+        self.X = torch.from_numpy(kqgen.normal_f32(seed ^ 0x77, Lyr * H + Lyr * top * F)).cuda()
+        self.Y = torch.empty(Lyr * top * 2 * F + Lyr * top * H, dtype=torch.float32, device="cuda")
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.launches = [(l, j) for l in range(Lyr) for j in range(2)]
+        torch.cuda.synchronize()
+
+    def xg(self, l):
+        return self.X[l * self.H:(l + 1) * self.H]
+
+    def xd(self, l):
+        o = self.L * self.H + l * self.top * self.F
+        return self.X[o:o + self.top * self.F].view(self.top, self.F)
+
+    def yg(self, l):
+        o = l * self.top * 2 * self.F
+        return self.Y[o:o + self.top * 2 * self.F].view(self.top, 2 * self.F)
+
+    def yd(self, l):
+        o = self.L * self.top * 2 * self.F + l * self.top * self.H
+        return self.Y[o:o + self.top * self.H].view(self.top, self.H)
+
+    def launch(self, l, j, stream):
+        kq = self.kq
+        if j == 0:
+            kq.moe_gemv(self.Wgu[l], "q4_k", self.E, 2 * self.F, self.H, self.ids[l], self.xg(l), self.yg(l),
+                        status=self.status, expert_stride=self.gu_stride, stream=stream)
+        else:
+            kq.moe_gemv(self.Wdn[l], "q4_k", self.E, self.H, self.F, self.ids[l], self.xd(l), self.yd(l),
+                        status=self.status, expert_stride=self.dn_stride, stream=stream)
+
+    def step(self, stream):
+        for l, j in self.launches:
+            self.launch(l, j, stream)
+
+    def advance(self):
+        self.ids.copy_(self.ids_all[self.t % self.ids_all.shape[0]], non_blocking=True)
+        self.t += 1
+
+    def kinds(self):
+        return {"moe_gate_up": dict(fmt="q4_k", N=2 * self.F, K=self.H, bytes=self.top * self.gu_stride,
+                                    launches=[(l, 0) for l in range(self.L)]),
+                "moe_down": dict(fmt="q4_k", N=self.H, K=self.F, bytes=self.top * self.dn_stride,
+                                 launches=[(l, 1) for l in range(self.L)])}
+
+    def io(self):
+        return [self.X], [self.Y]
+
+
+class Streamed:
+    """The chain with its weights in pinned host memory (kq_chain)."""
+
+    graphable = False
+
+    def __init__(self, torch, kq, kqgen, spec, seed, n_slots=4):
+        self.torch, self.kq, self.spec = torch, kq, spec
+        self.weight_bytes = sum(N * row_bytes(f, K) for mats in spec for (_, f, N, K, _) in mats)
+        # one host buffer for every weight, page-locked in place (the torch
+        # pinned allocator would round each tensor up to a power of two)
+        self.host = np.empty(self.weight_bytes, np.uint8)
+        mats, xs, ys, off = [], [], [], 0
+        for li, layer in enumerate(spec):
+            row = []
+            for mi, (_, f, N, K, _) in enumerate(layer):
+                nb = N * row_bytes(f, K)
+                view = self.host[off:off + nb]
+                kqgen.matrix(f, kqgen.tensor_seed(seed, li, mi), N, K, out=view)
+                row.append((torch.from_numpy(view), f, N, K))
+                off += nb
+            mats.append(row)
+        rc = torch.cuda.cudart().cudaHostRegister(self.host.ctypes.data, self.host.nbytes, 0)
+        if int(rc) != 0:
+            raise RuntimeError(f"cudaHostRegister failed ({rc})")
+        self.X = torch.from_numpy(kqgen.normal_f32(seed ^ 0x5A5A, sum(m[3] for r in mats for m in r))).cuda()
+        self.Y = torch.empty(sum(m[2] for r in mats for m in r), dtype=torch.float32, device="cuda")
+        xo = yo = 0
+        for r in mats:
+            for (_, f, N, K) in r:
+                xs.append(self.X[xo:xo + K])
+                ys.append(self.Y[yo:yo + N])
+                xo += K
+                yo += N
+        self.xs, self.ys = xs, ys
+        self.chain = kq.Chain(mats, n_slots=n_slots)
+        self.launches = [None] * sum(len(r) for r in mats)
+
+    def step(self, stream):
+        self.chain.run(self.xs, self.ys, stream=stream)
+
+    def kinds(self):
+        return {}
+
+    def io(self):
+        return [self.X], [self.Y]
+
+
+def make_workload(name, torch, kq, kqgen, seed):
+    if name == "llama8b_chain":
+        return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed)
+    if name in ("gemv_q4k_4096", "gateup_q4k", "down_q6k"):
+        return Resident(torch, kq, kqgen, chain_spec(name), seed)
+    if name.startswith("verify8b_k"):
+        return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed, k=int(name[len("verify8b_k"):]))
+    if name == "moe30b":
+        return MoE(torch, kq, kqgen, seed)
+    if name == "llama70b_resident":
+        return Resident(torch, kq, kqgen, chain_spec("llama70b"), seed)
+    if name == "llama70b_stream":
+        return Streamed(torch, kq, kqgen, chain_spec("llama70b"), seed)
+    raise KeyError(name)
+
+
+def h2d_peak_gbs(torch, nbytes=512 << 20, reps=5):
+    """Pinned host -> device copy bandwidth (the streamed chain's roofline)."""
+    h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    d.copy_(h, non_blocking=True)
+    torch.cuda.synchronize()
+    best = 0.0
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        d.copy_(h, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        best = max(best, nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del h, d
+    return best
 
 
 # --------------------------------------------------------------- the bench
@@ -158,35 +384,43 @@ def bench_kq(args, rank, world):
 
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
     kq.lib()
-    wl = WORKLOADS[args.workload]
-    layers = wl["layers"]()
-    wbytes = weight_bytes(layers)
-    n_launch = sum(len(m) for m in layers)
-    dev_w, xs, ys = build_device_chain(layers, 0xC0FFEE + 1 + rank, torch, kqgen)
-
-    stream = torch.cuda.Stream()
-    # every launch, graph replay and event of the bench goes to this stream
-    torch.cuda.set_stream(stream)
-    with torch.cuda.stream(stream):
-        run_chain(kq, layers, dev_w, xs, ys, stream)  # sets kernel attributes before capture
-    stream.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        run_chain(kq, layers, dev_w, xs, ys, stream)
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
-
     dist = world > 1
     if dist:
         import torch.distributed as tdist
+    wl = make_workload(args.workload, torch, kq, kqgen, SEED + rank)
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)   # every launch, replay and event goes here
+    advance = getattr(wl, "advance", None)
+
+    def one_step():
+        if advance:
+            advance()
+        wl.step(stream)
+
+    one_step()                       # sets kernel attributes before any capture
+    torch.cuda.synchronize()
+    if wl.graphable:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            wl.step(stream)
+
+        def run_step():
+            if advance:
+                advance()
+            graph.replay()
+    else:
+        run_step = one_step
+    for _ in range(args.warmup):
+        run_step()
+    torch.cuda.synchronize()
+    if dist:
         tdist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
         torch.cuda.synchronize()
         e0.record(stream)
         for _ in range(args.steps):
-            graph.replay()
+            run_step()
         e1.record(stream)
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
@@ -195,73 +429,66 @@ def bench_kq(args, rank, world):
         tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
         ms = float(t.item())
     ms_step = ms / args.steps
-    gbs = wbytes * args.steps * world / (ms * 1e-3) / 1e9
-    tok_s = args.steps * world / (ms * 1e-3)
+    k = getattr(wl, "k", 1)
+    gbs = wl.weight_bytes * args.steps * world / (ms * 1e-3) / 1e9
+    tok_s = k * args.steps * world / (ms * 1e-3)
 
-    # dominant kernel: per-launch device time of each matrix kind, measured
-    # with events on its own stream over all layers (weights never L2-hot)
+    # per-kernel device time of each matrix kind: a graph of all its
+    # launches (different layers' weights, so never L2-hot), events around it
     per_kind = {}
-    kinds = sorted({m[0] for mats in layers for m in mats})
-    for kind in kinds:
-        idx = [(li, mi) for li, mats in enumerate(layers) for mi, m in enumerate(mats) if m[0] == kind]
-        reps = max(1, 64 // len(idx))
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for _ in range(reps):
-                for li, mi in idx:
-                    name, fmt, N, K, slot = layers[li][mi]
-                    kq.gemv(dev_w[li][mi], fmt, N, K, xs[li][slot], ys[li][mi], stream=stream)
-        g.replay()
-        torch.cuda.synchronize()
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
+    if wl.graphable:
+        for name, kd in wl.kinds().items():
+            reps = max(1, 64 // len(kd["launches"]))
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(reps):
+                    for (a, b) in kd["launches"]:
+                        wl.launch(a, b, stream)
+            g.replay()
+            torch.cuda.synchronize()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s0.record(stream)
             g.replay()
             s1.record(stream)
-        torch.cuda.synchronize()
-        del g
-        n = reps * len(idx)
-        t_us = s0.elapsed_time(s1) * 1e3 / n
-        name, fmt, N, K, _ = layers[idx[0][0]][idx[0][1]]
-        b = N * row_bytes(fmt, K)
-        per_kind[kind] = dict(fmt=fmt, N=N, K=K, bytes=b, us=t_us, gbs=b / (t_us * 1e-6) / 1e9,
-                              share=t_us * len(idx) / (ms_step * 1e3))
-    dom = max(per_kind, key=lambda k: per_kind[k]["share"])
+            torch.cuda.synchronize()
+            n = reps * len(kd["launches"])
+            t_us = s0.elapsed_time(s1) * 1e3 / n
+            per_kind[name] = dict(fmt=kd["fmt"], N=kd["N"], K=kd["K"], bytes=kd["bytes"], us=round(t_us, 3),
+                                  gbs=round(kd["bytes"] / (t_us * 1e-6) / 1e9, 1),
+                                  share=round(t_us * len(kd["launches"]) / (ms_step * 1e3), 4))
+            del g
 
-    # end to end through the public API with host buffers: activations in
-    # from pinned memory, outputs back, every step
-    x_host = [{s: t.cpu().pin_memory() for s, t in xl.items()} for xl in xs]
-    y_host = [[torch.empty(t.numel(), dtype=torch.float32, pin_memory=True) for t in yl] for yl in ys]
-    h2d = sum(t.numel() * 4 for xl in x_host for t in xl.values())
-    d2h = sum(t.numel() * 4 for yl in y_host for t in yl)
+    # end to end through the public API with host buffers: the step's
+    # activations in from pinned memory and its outputs back, every step
+    xin, yout = wl.io()
+    xh = [t.cpu().pin_memory() for t in xin]
+    yh = [torch.empty(t.numel(), dtype=t.dtype, pin_memory=True) for t in yout]
+    h2d = sum(t.numel() * t.element_size() for t in xh)
+    d2h = sum(t.numel() * t.element_size() for t in yh)
 
     def e2e_step():
-        for li, xl in enumerate(x_host):
-            for s, t in xl.items():
-                xs[li][s].copy_(t, non_blocking=True)
-        graph.replay()
-        for li, yl in enumerate(y_host):
-            for mi, t in enumerate(yl):
-                t.copy_(ys[li][mi], non_blocking=True)
+        for d, h in zip(xin, xh):
+            d.copy_(h, non_blocking=True)
+        run_step()
+        for h, d in zip(yh, yout):
+            h.copy_(d, non_blocking=True)
 
-    with torch.cuda.stream(stream):
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
-        torch.cuda.synchronize()
-        if dist:
-            tdist.barrier()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        f1.record(stream)
-        torch.cuda.synchronize()
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        tdist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
     ems = f0.elapsed_time(f1)
     if dist:
         t = torch.tensor([ems], device="cuda")
         tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
         ems = float(t.item())
-    e2e_gbs = wbytes * args.steps * world / (ems * 1e-3) / 1e9
 
     peaks = {}
     try:
@@ -271,44 +498,62 @@ def bench_kq(args, rank, world):
     hbm = peaks.get("hbm_gbs")
     peak_src = "measured" if hbm else "fallback"
     hbm = hbm or 6650.0
-    dk = per_kind[dom]
     result = {
         "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32 (q4_k/q6_k weights)", "data": "synthetic",
-        "tok_per_s": round(tok_s, 2), "frac_of_hbm_peak": round(gbs / world / hbm, 4),
-        "config": {"workload": args.workload, "desc": wl["desc"], "weight_bytes_per_step": wbytes,
-                   "launches_per_step": n_launch, "batch": 1, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (no flush)" if wbytes > 2 * 126e6 else "rotating copies"},
-        "roofline": {"bound": "hbm", "kernel": f"gemv_kernel<{dk['fmt']}> {dom} {dk['N']}x{dk['K']}",
-                     "achieved": round(dk["gbs"], 1), "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
-                     "frac": round(dk["gbs"] / hbm, 4), "traffic": None},
-        "kernels": {k: {kk: (round(vv, 4) if isinstance(vv, float) else vv) for kk, vv in v.items()}
-                    for k, v in per_kind.items()},
-        "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "tok_per_s": round(args.steps * world / (ems * 1e-3), 2),
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, kqgen)",
+        "tok_per_s": round(tok_s, 3), "frac_of_hbm_peak": round(gbs / world / hbm, 4),
+        "config": {"workload": args.workload, "desc": WORKLOADS[args.workload],
+                   "weight_bytes_per_step": wl.weight_bytes, "launches_per_step": len(wl.launches),
+                   "columns": k, "batch": 1, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (no flush)" if wl.weight_bytes > 2 * 126e6 else "rotating copies"},
+        "e2e": {"value": round(wl.weight_bytes * args.steps * world / (ems * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "tok_per_s": round(k * args.steps * world / (ems * 1e-3), 3),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
-        "gpu_launches": n_launch * args.steps,
+        "gpu_launches": len(wl.launches) * args.steps,
     }
+    if per_kind:
+        dom = max(per_kind, key=lambda n: per_kind[n]["share"])
+        dk = per_kind[dom]
+        result["roofline"] = {"bound": "hbm", "kernel": f"gemv_kernel {dk['fmt']} {dom} {dk['N']}x{dk['K']}",
+                              "achieved": dk["gbs"], "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
+                              "frac": round(dk["gbs"] / hbm, 4), "traffic": None}
+        result["kernels"] = per_kind
+    if isinstance(wl, Streamed):
+        pk = h2d_peak_gbs(torch)
+        result["roofline"] = {"bound": "pcie_h2d", "kernel": "H2D copies of the layer ring",
+                              "achieved": round(gbs / world, 2), "peak": round(pk, 2),
+                              "peak_source": "measured here (512 MiB pinned copy)", "unit": "GB/s",
+                              "frac": round(gbs / world / pk, 4), "traffic": None}
+        result["gpu_launches"] = 4 * len(wl.spec) * args.steps
     return result
 
 
 def cpu_baseline(args, budget_s=15.0):
-    """The oracle as it stands, on a bounded sample of the same workload:
-    a prefix of the chain's rows (every matrix kind), timed on all cores."""
+    """The oracle as it stands, on a bounded sample of the workload: the
+    first rows of each matrix kind, timed on all host cores."""
     import kqgen
     import oracle
 
-    layers = WORKLOADS[args.workload]["layers"]()
+    if args.workload == "moe30b":
+        spec = [[("moe_gate_up", "q4_k", 2 * MOE30B["ffn"], MOE30B["hidden"], 0),
+                 ("moe_down", "q4_k", MOE30B["hidden"], MOE30B["ffn"], 1)]] * MOE30B["layers"]
+        per_token = MOE30B["layers"] * MOE30B["top"] * (2 * MOE30B["ffn"] * row_bytes("q4_k", MOE30B["hidden"])
+                                                        + MOE30B["hidden"] * row_bytes("q4_k", MOE30B["ffn"]))
+    else:
+        base = {"llama8b_chain": "llama8b", "llama70b_resident": "llama70b", "llama70b_stream": "llama70b"}
+        name = base.get(args.workload, "llama8b" if args.workload.startswith("verify") else args.workload)
+        spec = chain_spec(name)
+        per_token = sum(N * row_bytes(f, K) for mats in spec for (_, f, N, K, _) in mats)
     cores = len(os.sched_getaffinity(0))
-    done_bytes, t_total, rows_done = 0, 0.0, 0
+    done_bytes, t_total, rows_done, li = 0, 0.0, 0, 0
     t_start = time.time()
-    li = 0
-    while time.time() - t_start < budget_s and li < len(layers):
-        for mi, (name, fmt, N, K, slot) in enumerate(layers[li]):
+    while time.time() - t_start < budget_s and li < len(spec):
+        for mi, (name, fmt, N, K, slot) in enumerate(spec[li]):
             nrows = min(N, 512)
-            W = kqgen.matrix(fmt, kqgen.tensor_seed(0xC0FFEE + 1, li, mi), nrows, K)
-            x = kqgen.normal_f32(kqgen.tensor_seed((0xC0FFEE + 1) ^ 0x5A5A, li, slot), K)
+            W = kqgen.matrix(fmt, kqgen.tensor_seed(SEED, li, mi), nrows, K)
+            x = kqgen.normal_f32(kqgen.tensor_seed(SEED ^ 0x5A5A, li, slot), K)
             t0 = time.perf_counter()
             oracle.gemv(fmt, W, nrows, K, x, nthreads=cores)
             t_total += time.perf_counter() - t0
@@ -316,33 +561,34 @@ def cpu_baseline(args, budget_s=15.0):
             rows_done += nrows
         li += 1
     gbs = done_bytes / t_total / 1e9
-    wb = weight_bytes(layers)
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "tok_per_s": round(gbs * 1e9 / wb, 6),
-            "sample": f"first {min(512, 4096)} rows of each matrix of {li} layer(s) ({rows_done} rows, "
-                      f"{done_bytes / 1e6:.1f} MB), fp64 oracle, OpenMP over rows"}
+            "tok_per_s": round(gbs * 1e9 / per_token, 6),
+            "sample": f"first <=512 rows of each matrix of {li} layer(s) ({rows_done} rows, "
+                      f"{done_bytes / 1e6:.1f} MB of weights), fp64 oracle, OpenMP over rows"}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="llama8b_chain", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="kq", choices=["kq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = {"llama70b_stream": 3, "llama70b_resident": 50}.get(args.workload, 300)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
 
     if args.impl == "reference":
         if rank != 0:
             return
-        cb = cpu_baseline(args, budget_s=max(5.0, 2.0 * args.steps))
+        cb = cpu_baseline(args, budget_s=min(60.0, max(5.0, 1.0 * args.steps)))
         line = {"metric": METRIC, "value": cb["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f64", "data": "synthetic", "impl": "reference",
-                "config": {"workload": args.workload, "desc": WORKLOADS[args.workload]["desc"]},
+                "dtype": "f64", "data": "synthetic (seeded, kqgen)", "impl": "reference",
+                "config": {"workload": args.workload, "desc": WORKLOADS[args.workload]},
                 "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)

@@ -143,3 +143,83 @@ def device_fault() -> int:
     out = ctypes.c_int(0)
     _check(lib().kq_device_fault(ctypes.byref(out)), "kq_device_fault")
     return out.value
+
+
+# --------------------------------------------------------------- chain
+class MatrixDesc(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("fmt", ctypes.c_int), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+def _chain_sigs(L):
+    if getattr(L, "_chain_ready", False):
+        return
+    vp = ctypes.c_void_p
+    L.kq_chain_create.restype = ctypes.c_int
+    L.kq_chain_create.argtypes = [ctypes.POINTER(MatrixDesc), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                  ctypes.POINTER(vp)]
+    L.kq_chain_slot_bytes.restype = ctypes.c_size_t
+    L.kq_chain_slot_bytes.argtypes = [vp]
+    L.kq_chain_run.restype = ctypes.c_int
+    L.kq_chain_run.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp]
+    L.kq_chain_wait.restype = ctypes.c_int
+    L.kq_chain_wait.argtypes = [vp, ctypes.c_int64]
+    L.kq_chain_last_error.restype = ctypes.c_char_p
+    L.kq_chain_destroy.restype = None
+    L.kq_chain_destroy.argtypes = [vp]
+    L._chain_ready = True
+
+
+class Chain:
+    """Layer chain whose weights stay in pinned host memory and stream
+    through ``n_slots`` device slots (kq_chain_* in kq.h).
+
+    mats: list over layers of lists of (W_host_pinned_uint8_tensor, fmt, N, K).
+    """
+
+    def __init__(self, mats, n_slots: int = 4):
+        L = lib()
+        _chain_sigs(L)
+        self._L = L
+        self.n_layers = len(mats)
+        self.per_layer = len(mats[0])
+        flat = [m for layer in mats for m in layer]
+        self._keep = [m[0] for m in flat]  # keep the host tensors alive
+        arr = (MatrixDesc * len(flat))()
+        for i, (W, fmt, N, K) in enumerate(flat):
+            if W.is_cuda:
+                raise ValueError("chain weights must be host memory")
+            arr[i] = MatrixDesc(W.data_ptr(), _fmt(fmt), N, K)
+        h = ctypes.c_void_p()
+        st = L.kq_chain_create(arr, self.n_layers, self.per_layer, n_slots, ctypes.byref(h))
+        if st != OK:
+            raise KQError(st, "kq_chain_create", L.kq_chain_last_error().decode())
+        self._h = h
+
+    @property
+    def slot_bytes(self) -> int:
+        return int(self._L.kq_chain_slot_bytes(self._h))
+
+    def run(self, xs, ys, stream=None) -> None:
+        n = self.n_layers * self.per_layer
+        assert len(xs) == n and len(ys) == n
+        xa = (ctypes.c_void_p * n)(*[_dev(x, "x", torch.float32) for x in xs])
+        ya = (ctypes.c_void_p * n)(*[_dev(y, "y", torch.float32) for y in ys])
+        st = self._L.kq_chain_run(self._h, xa, ya, _stream(stream))
+        if st != OK:
+            raise KQError(st, "kq_chain_run", self._L.kq_chain_last_error().decode())
+
+    def wait(self, timeout_ms: int = -1) -> None:
+        st = self._L.kq_chain_wait(self._h, timeout_ms)
+        if st != OK:
+            raise KQError(st, "kq_chain_wait", self._L.kq_chain_last_error().decode())
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._L.kq_chain_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

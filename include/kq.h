@@ -155,6 +155,64 @@ KQ_API int kq_moe_gemv(const void* W_experts, int fmt, int E, int64_t N, int64_t
 KQ_API int kq_unpack(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d,
               kq_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Streamed layer chain ("Out-of-core LLM inference engine written from
+ * scratch in Rust", Approach: layer weights move through a ring of VRAM
+ * slots while the GPU computes nearby layers; "Kortex: Streaming 70B Models
+ * on Consumer GPUs", Key components 2: the pipeline overlaps transfers with
+ * compute).
+ *
+ * A chain holds n_layers layers of mats_per_layer matrices whose weights
+ * stay in PAGE-LOCKED HOST memory.  kq_chain_run copies layer l into device
+ * slot l % n_slots on the chain's own copy stream and runs that layer's
+ * GEMVs (the kq_gemv kernels) on the caller's stream as soon as its copy has
+ * landed; the copy of layer l + n_slots waits until layer l's GEMVs are done
+ * with the slot.  Outputs equal a resident kq_gemv run bitwise.
+ * ---------------------------------------------------------------------- */
+
+/* One weight matrix: W is HOST page-locked memory (cudaHostAlloc or
+ * cudaHostRegister), N x K in format fmt. */
+typedef struct kq_matrix_desc {
+    const void* W;
+    int fmt;
+    int64_t N;
+    int64_t K;
+} kq_matrix_desc;
+
+typedef struct kq_chain kq_chain;
+
+/* Creates a chain.  mats: n_layers * mats_per_layer descriptors, layer
+ * major; every layer must have the same formats and shapes (matrix m of
+ * each layer alike).  The chain copies the descriptor array (not the
+ * weights: they must stay valid and pinned for the chain's lifetime) and
+ * allocates n_slots device slots of kq_chain_slot_bytes() bytes each, one
+ * copy stream and its events on the current device.
+ * Errors: KQ_ERR_INVALID_ARG, KQ_ERR_NOT_PINNED (a W that is not
+ * page-locked), KQ_ERR_OOM, KQ_ERR_CUDA.  On error *out is NULL. */
+KQ_API int kq_chain_create(const kq_matrix_desc* mats, int n_layers, int mats_per_layer, int n_slots,
+                           kq_chain** out);
+
+/* Device bytes of one slot (one layer's matrices, 256-byte aligned each). */
+KQ_API size_t kq_chain_slot_bytes(const kq_chain* c);
+
+/* Enqueues one pass over every layer.  x, y: HOST arrays of n_layers *
+ * mats_per_layer DEVICE pointers (activation K floats, output N floats per
+ * matrix).  Asynchronous: returns once everything is queued; the copy
+ * stream starts after the work already queued on `compute`.  The
+ * environment variable KQ_FAULT=copy@L makes the run stop before copying
+ * layer L and return KQ_ERR_INJECTED (what was queued still completes). */
+KQ_API int kq_chain_run(kq_chain* c, const float* const* x, float* const* y, kq_stream_t compute);
+
+/* Waits (host-side polling, no device spin) until the last run finished;
+ * KQ_ERR_TIMEOUT if it takes longer than timeout_ms (negative: no limit). */
+KQ_API int kq_chain_wait(kq_chain* c, int64_t timeout_ms);
+
+/* Text describing the last chain failure on the calling thread. */
+KQ_API const char* kq_chain_last_error(void);
+
+/* Waits for the chain's copies, then frees its slots, stream and events. */
+KQ_API void kq_chain_destroy(kq_chain* c);
+
 #ifdef __cplusplus
 }
 #endif
