@@ -122,30 +122,25 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
         a.parts = kConsumerWarps;
     }
     const size_t stage = round_up(static_cast<size_t>(a.ps) * 2 * a.row_bytes + 32, 128);
-    const size_t wp_bytes = round_up(sizeof(float) * 2 * a.ps * a.parts * 2 * ncol, 128);
-    const size_t xs_bytes = round_up(sizeof(float) * ncol * 2 * nb * kRegion, 128);
+    // Two consumer groups (16 compute warps) for the single-column kernels:
+    // measured to hide shared-memory latency better than one group; the
+    // multi-column kernels need more registers per thread and keep one.
+    const int ng = ncol == 1 ? 2 : 1;
+    const bool shared_x = a.x_seg_stride == 0;
+    const size_t wp_bytes = round_up(sizeof(float) * ng * 2 * a.ps * a.parts * 2 * ncol, 128);
+    const size_t xs_bytes = round_up(sizeof(float) * (shared_x ? 1 : ng) * ncol * 2 * nb * kRegion, 128);
     const size_t head = 256;
     const size_t fixed = head + wp_bytes + xs_bytes;
-    size_t limit = static_cast<size_t>(di.smem_optin);
+    const size_t limit = static_cast<size_t>(di.smem_optin);
     if (fixed + 2 * stage > limit)
         return fail(KQ_ERR_UNSUPPORTED, "K=%lld with %d columns needs %zu bytes of shared memory (limit %zu)",
                     (long long)a.K, ncol, fixed + 2 * stage, limit);
-    // Two resident CTAs per SM hide more latency (measured +17% on the
-    // 28672 x 4096 Q4_K matrix); used for the single-column Q4_K kernel
-    // whenever two copies of its shared memory fit in one SM.
-    int ctas = 1;
-    const size_t share = static_cast<size_t>(di.smem_per_sm) / 2 - 1024;
-    if (fmt == KQ_FMT_Q4_K && ncol == 1 && fixed + 2 * stage <= share) {
-        ctas = 2;
-        limit = share;
-    }
     size_t ns = (limit - fixed) / stage;
-    if (ns > 6) ns = 6;
+    if (ns > kMaxStages) ns = kMaxStages;
     // no more stages than the busiest CTA will ever use
     const int64_t rps = (a.N + 1) / 2;
     const int64_t P = static_cast<int64_t>(a.n_seg) * rps;
-    const int64_t slots = static_cast<int64_t>(di.sm_count) * ctas;
-    const int64_t grid = P < slots ? P : slots;
+    const int64_t grid = P < di.sm_count ? P : di.sm_count;
     const int64_t per_cta = (P + grid - 1) / grid;
     const int64_t need = (per_cta + a.ps - 1) / a.ps + (a.n_seg > 1 ? 1 : 0);
     if (static_cast<int64_t>(ns) > need) ns = need < 2 ? 2 : static_cast<size_t>(need);
@@ -155,7 +150,7 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     a.xs_offset = static_cast<int>(head + wp_bytes);
     a.sbuf_offset = static_cast<int>(fixed);
     p.grid = static_cast<int>(grid);
-    p.ctas = ctas;
+    p.ng = ng;
     p.smem_bytes = fixed + ns * stage;
     p.pdl = true;
     return KQ_OK;
@@ -183,14 +178,14 @@ static int padded_cols(int k) { return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : 8;
 static cudaError_t dispatch(const GemvArgs& a, const LaunchPlan& p, int fmt, int ncol, cudaStream_t s) {
     if (fmt == KQ_FMT_Q4_K) {
         switch (ncol) {
-            case 1: return p.ctas == 2 ? launch_one<1, 1, 2>(a, p, s) : launch_one<1, 1, 1>(a, p, s);
+            case 1: return launch_one<1, 1, 2>(a, p, s);
             case 2: return launch_one<1, 2, 1>(a, p, s);
             case 4: return launch_one<1, 4, 1>(a, p, s);
             default: return launch_one<1, 8, 1>(a, p, s);
         }
     }
     switch (ncol) {
-        case 1: return launch_one<2, 1, 1>(a, p, s);
+        case 1: return launch_one<2, 1, 2>(a, p, s);
         case 2: return launch_one<2, 2, 1>(a, p, s);
         case 4: return launch_one<2, 4, 1>(a, p, s);
         default: return launch_one<2, 8, 1>(a, p, s);

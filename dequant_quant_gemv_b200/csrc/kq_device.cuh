@@ -12,7 +12,6 @@ constexpr int kQ4Bytes = 144;      // Q4_K super-block
 constexpr int kQ6Bytes = 210;      // Q6_K super-block
 constexpr int kConsumerWarps = 8;  // warps that dequantise and multiply
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;  // + one producer (TMA) warp
 constexpr int kRegion = 132;       // floats per activation region: 128 x + 4 sums
 constexpr int kMaxStages = 8;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded-wait limit (2 s)

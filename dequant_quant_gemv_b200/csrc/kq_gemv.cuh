@@ -329,7 +329,7 @@ __device__ __forceinline__ void raise_fault(const GemvArgs& a, volatile int* abo
 // Stage the activations of segment `seg` (all NCOL columns) into the
 // padded, permuted layout the units read, then (Q4_K) the region sums.
 template <int FMT, int NCOL>
-__device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct) {
+__device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar) {
     const float* xg = a.x + seg * a.x_seg_stride;
     const int nb = a.nb;
     const int nreg = 2 * nb;
@@ -339,7 +339,7 @@ __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct) {
     // the 4 values land 2 floats apart (pair members alternate).
     const int k4 = static_cast<int>(a.K >> 2);
     const int items = NCOL * k4;
-    for (int it = ct; it < items; it += kConsumers) {
+    for (int it = ct; it < items; it += nthr) {
         const int j = it / k4;
         const int i = 4 * (it - j * k4);
         const float* xc = xg + (j < a.ncol_real ? j : a.ncol_real - 1) * a.ldx;
@@ -367,17 +367,17 @@ __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct) {
         st_s32f(dst + 16, v.z);
         st_s32f(dst + 24, v.w);
     }
-    named_bar_sync(1, kConsumers);
+    named_bar_sync(bar, nthr);
     if constexpr (FMT == 1) {
         const int sums = NCOL * nreg * 2;
-        for (int it = ct; it < sums; it += kConsumers) {
+        for (int it = ct; it < sums; it += nthr) {
             const int j = it / (nreg * 2);
             const int rem = it - j * nreg * 2;
             const int reg = rem >> 1, cp = rem & 1;
             const uint32_t xr = xs + 4 * (j * xcs + reg * kRegion);
             st_s64f(xr + 4 * (128 + 2 * cp), q4k_region_sum(xr, cp));
         }
-        named_bar_sync(1, kConsumers);
+        named_bar_sync(bar, nthr);
     }
 }
 
@@ -391,8 +391,12 @@ __device__ __forceinline__ void q6k_unit_dispatch(int kappa, uint32_t row0, int 
 
 // ------------------------------------------------------------ the kernel
 
-template <int FMT, int NCOL, int CTAS>
-__global__ void __launch_bounds__(kThreads, CTAS) gemv_kernel(const __grid_constant__ GemvArgs a) {
+// NG consumer groups of 8 warps each: group g consumes the stages whose
+// index is g mod NG, so two groups work on consecutive stages of one ring
+// while the producer keeps filling it (more warps per SM to hide shared-memory
+// latency, one activation copy, a deeper ring than two CTAs could hold).
+template <int FMT, int NCOL, int NG>
+__global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __grid_constant__ GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
@@ -461,10 +465,14 @@ __global__ void __launch_bounds__(kThreads, CTAS) gemv_kernel(const __grid_const
     }
 
     // ---------------------------------------------------------- consumers
-    const int ct = tid - 32;        // consumer thread 0..255
-    const int cw = warp - 1;        // consumer warp 0..7
+    const int ct_all = tid - 32;             // 0 .. NG*256-1
+    const int g = NG == 2 ? (ct_all >> 8) : 0;
+    const int ct = ct_all & (kConsumers - 1);  // thread within the group
+    const int cw = ct >> 5;                   // warp within the group
+    const int gbar = 1 + g;                   // the group's named barrier
     const int nb = a.nb;
     const int xcs = 2 * nb * kRegion;
+    const bool shared_x = a.x_seg_stride == 0;
     pdl_wait();                      // activations may come from the previous grid
     pdl_launch_dependents();
 
@@ -498,15 +506,24 @@ __global__ void __launch_bounds__(kThreads, CTAS) gemv_kernel(const __grid_const
     int region;
     if (FMT == 1) region = 2 * u_b + u_H;
     else region = ((kappa * (nb >> 3) + (u_b >> 3)) << 1) + u_H;
-    const uint32_t xs_s = smem_u32(xs), sbuf_s = smem_u32(sbuf), wp_s = smem_u32(wp);
+    const int wp_group = 2 * a.ps * parts * 2 * NCOL;     // floats of one group's double buffer
+    const uint32_t xs_s = smem_u32(xs) + (shared_x ? 0 : 4 * g * NCOL * xcs);
+    const uint32_t sbuf_s = smem_u32(sbuf), wp_s = smem_u32(wp) + 4 * g * wp_group;
     const uint32_t xr = xs_s + 4 * (region * kRegion);
 
     StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
     Stage st;
     int64_t staged_seg = -1;
+    if (shared_x) {
+        // one activation copy for all groups, staged by all consumer threads
+        stage_x<FMT, NCOL>(a, 0, xs_s, ct_all, NG * kConsumers, NG == 2 ? 3 : 1);
+        staged_seg = 0;
+    }
+    int own = 0;  // stages this group has consumed
     while (it.next(st)) {
-        if (staged_seg < 0 || (a.x_seg_stride != 0 && st.seg != staged_seg)) {
-            stage_x<FMT, NCOL>(a, st.seg, xs_s, ct);
+        if (NG == 2 && ((it.count - 1) & 1) != g) continue;
+        if (!shared_x && st.seg != staged_seg) {
+            stage_x<FMT, NCOL>(a, st.seg, xs_s, ct, kConsumers, gbar);
             staged_seg = st.seg;
         }
         const int slot = it.slot;
@@ -532,14 +549,16 @@ __global__ void __launch_bounds__(kThreads, CTAS) gemv_kernel(const __grid_const
                     for (int j = 0; j < NCOL; ++j) out[r][j] += __shfl_xor_sync(0xffffffffu, out[r][j], off);
             }
         }
-        const uint32_t wb = wp_s + 4 * ((it.count & 1) * (a.ps * parts * 2 * NCOL));
+        // the group's own stages alternate between two partial-sum buffers
+        const uint32_t wb = wp_s + 4 * ((own & 1) * (a.ps * parts * 2 * NCOL));
+        ++own;
         if ((lane & (group - 1)) == 0 && u_rp < a.ps) {
 #pragma unroll
             for (int r = 0; r < 2; ++r)
 #pragma unroll
                 for (int j = 0; j < NCOL; ++j) st_s32f(wb + 4 * (((u_rp * parts + part) * 2 + r) * NCOL + j), out[r][j]);
         }
-        const bool stop = named_bar_or(1, kConsumers, *abort_flag != 0);
+        const bool stop = named_bar_or(gbar, kConsumers, *abort_flag != 0);
         if (lane == 0) mbar_arrive(&empty[slot]);
         if (stop) break;
         // fixed-order sum over parts, then store
@@ -562,14 +581,14 @@ __global__ void __launch_bounds__(kThreads, CTAS) gemv_kernel(const __grid_const
 
 // ----------------------------------------------------------- launchers
 
-template <int FMT, int NCOL, int CTAS>
+template <int FMT, int NCOL, int NG>
 cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream) {
-    auto kern = gemv_kernel<FMT, NCOL, CTAS>;
+    auto kern = gemv_kernel<FMT, NCOL, NG>;
     cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), p.smem_bytes);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(32 + NG * kConsumers);
     cfg.dynamicSmemBytes = p.smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];

@@ -2,6 +2,6 @@
 #include "kq_gemv.cuh"
 
 namespace kq {
-template cudaError_t launch_one<2, 1, 1>(const GemvArgs&, const LaunchPlan&, cudaStream_t);
+template cudaError_t launch_one<2, 1, 2>(const GemvArgs&, const LaunchPlan&, cudaStream_t);
 template cudaError_t launch_one<2, 2, 1>(const GemvArgs&, const LaunchPlan&, cudaStream_t);
 }  // namespace kq

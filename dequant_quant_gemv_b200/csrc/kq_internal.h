@@ -40,7 +40,7 @@ struct GemvArgs {
 
 struct LaunchPlan {
     int grid;
-    int ctas;        // CTAs resident per SM the schedule was sized for (1 or 2)
+    int ng;          // consumer groups of 8 warps (1 or 2)
     size_t smem_bytes;
     bool pdl;
 };
@@ -48,7 +48,7 @@ struct LaunchPlan {
 // Fills the schedule fields of `a` and the launch plan; returns a kq_status.
 int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p);
 
-template <int FMT, int NCOL, int CTAS>
+template <int FMT, int NCOL, int NG>
 cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
 cudaError_t fault_word(int** out);
 cudaError_t launch_unpack(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d,
