@@ -102,7 +102,7 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     DevInfo di;
     cudaError_t err = dev_info(di);
     if (err != cudaSuccess) return cuda_fail(err, "device query");
-    const int nb = a.nb;
+    const int nb = a.nbs;  // blocks per K range (all of K unless split)
     if (fmt == KQ_FMT_Q4_K) {
         const int ur = 2 * nb;  // half-block units per row pair
         const int lr = ur <= 32 ? next_pow2(ur) : static_cast<int>(round_up(ur, 32));
@@ -121,7 +121,9 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
         a.ps = 32 / lrw;
         a.parts = kConsumerWarps;
     }
-    const size_t stage = round_up(static_cast<size_t>(a.ps) * 2 * a.row_bytes + 32, 128);
+    const size_t srow = a.ksplit > 1 ? static_cast<size_t>(a.nbs) * kq_block_bytes(fmt)
+                                     : static_cast<size_t>(a.row_bytes);
+    const size_t stage = round_up(static_cast<size_t>(a.ps) * 2 * srow + 32, 128);
     // Two consumer groups (16 compute warps) for the single-column kernels:
     // measured to hide shared-memory latency better than one group; the
     // multi-column kernels need more registers per thread and keep one.
@@ -140,8 +142,9 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     // no more stages than the busiest CTA will ever use
     const int64_t rps = (a.N + 1) / 2;
     const int64_t P = static_cast<int64_t>(a.n_seg) * rps;
-    const int64_t grid = P < di.sm_count ? P : di.sm_count;
-    const int64_t per_cta = (P + grid - 1) / grid;
+    const int64_t ranges = di.sm_count / a.ksplit;        // row-pair ranges per K range
+    const int64_t grid = (P < ranges ? P : ranges) * a.ksplit;
+    const int64_t per_cta = (P + grid / a.ksplit - 1) / (grid / a.ksplit);
     const int64_t need = (per_cta + a.ps - 1) / a.ps + (a.n_seg > 1 ? 1 : 0);
     if (static_cast<int64_t>(ns) > need) ns = need < 2 ? 2 : static_cast<size_t>(need);
     a.nstage = static_cast<int>(ns);
@@ -202,7 +205,31 @@ static int run(GemvArgs& a, int fmt, int k, cudaStream_t stream) {
     if (st != KQ_OK) return st;
     err = dispatch(a, p, fmt, ncol, stream);
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    if (a.ksplit > 1) {
+        err = launch_splitk_combine(a.partial, a.ksplit, k, a.N, a.y, a.ldy, stream);
+        if (err != cudaSuccess) return cuda_fail(err, "split-K combine launch");
+    }
     return KQ_OK;
+}
+
+// Split over K across CTAs for matrices with fewer row pairs than SMs:
+// S ranges of nbs super-blocks each (a multiple of 8 for Q6_K, keeping every
+// range 16-byte aligned).  A pure function of (fmt, N, K, SM count), so
+// single- and multi-column calls split alike.
+static void choose_split(int fmt, int64_t N, int nb, int sm_count, int* S, int* nbs) {
+    *S = 1;
+    *nbs = nb;
+    const int64_t P = (N + 1) / 2;
+    if (P * 2 > sm_count) return;                       // enough row pairs already
+    const int unit = fmt == KQ_FMT_Q6_K ? 8 : 1;
+    const int max_s = nb / unit;
+    int want = static_cast<int>((sm_count + P - 1) / P);
+    if (want > max_s) want = max_s;
+    if (want <= 1) return;
+    int per = (nb / unit + want - 1) / want * unit;      // blocks per range
+    *nbs = per;
+    *S = (nb + per - 1) / per;
+    if (*S <= 1) *nbs = nb;
 }
 
 // Largest padded column count whose staged activations fit in shared
@@ -229,7 +256,7 @@ static int run_grouped(GemvArgs& a, int fmt, int k, cudaStream_t stream) {
     for (int c0 = 0; c0 < k; c0 += g) {
         GemvArgs t = a;
         t.x = a.x + static_cast<int64_t>(c0) * a.ldx;
-        t.y = a.y + static_cast<int64_t>(c0) * a.ldy;
+        t.y = a.y + static_cast<int64_t>(c0) * a.ldy;  // partial sums restart at the workspace base
         const int kk = k - c0 < g ? k - c0 : g;
         int st = run(t, fmt, kk, stream);
         if (st != KQ_OK) return st;
@@ -318,6 +345,9 @@ int kq_gemv_multi(const void* W, int fmt, int64_t N, int64_t K, const float* x, 
     a.ldy = ldy;
     a.y_seg_stride = 0;
     a.status = nullptr;
+    a.ksplit = 1;
+    a.nbs = a.nb;
+    a.partial = nullptr;
     return run_grouped(a, fmt, k, s);
 }
 
@@ -362,7 +392,59 @@ int kq_moe_gemv(const void* W_experts, int fmt, int E, int64_t N, int64_t K, siz
     a.ldy = 0;
     a.y_seg_stride = N;
     a.status = status;
+    a.ksplit = 1;
+    a.nbs = a.nb;
+    a.partial = nullptr;
     return run(a, fmt, 1, s);
+}
+
+static int split_for(int fmt, int64_t N, int64_t K, int* S, int* nbs) {
+    DevInfo di;
+    cudaError_t err = dev_info(di);
+    if (err != cudaSuccess) return cuda_fail(err, "device query");
+    choose_split(fmt, N, static_cast<int>(K / 256), di.sm_count, S, nbs);
+    return KQ_OK;
+}
+
+size_t kq_splitk_workspace_bytes(int fmt, int64_t N, int64_t K, int k) {
+    if ((fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q6_K) || N < 1 || K < 256 || K % 256 != 0 || k < 1 || k > 8) return 0;
+    int S = 1, nbs = 0;
+    if (split_for(fmt, N, K, &S, &nbs) != KQ_OK || S <= 1) return 0;
+    return sizeof(float) * static_cast<size_t>(S) * k * static_cast<size_t>(N);
+}
+
+int kq_gemv_splitk(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx, int k, float* y,
+                   int64_t ldy, void* workspace, size_t workspace_bytes, kq_stream_t stream) {
+    g_last_error[0] = 0;
+    int st = check_matrix(W, fmt, N, K);
+    if (st != KQ_OK) return st;
+    if (k < 1 || k > 8) return fail(KQ_ERR_INVALID_ARG, "k=%d outside 1..8", k);
+    if (N == 0 || K == 0) return kq_gemv_multi(W, fmt, N, K, x, ldx, k, y, ldy, stream);
+    int S = 1, nbs = 0;
+    st = split_for(fmt, N, K, &S, &nbs);
+    if (st != KQ_OK) return st;
+    if (S <= 1) return kq_gemv_multi(W, fmt, N, K, x, ldx, k, y, ldy, stream);
+    const size_t need = sizeof(float) * static_cast<size_t>(S) * k * static_cast<size_t>(N);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 4))
+        return fail(KQ_ERR_INVALID_ARG, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes);
+    if (!y || !aligned(y, 4) || !x || !aligned(x, 4)) return fail(KQ_ERR_INVALID_ARG, "x or y NULL or misaligned");
+    if (k > 1 && (ldx < K || ldy < N)) return fail(KQ_ERR_INVALID_ARG, "ldx < K or ldy < N");
+    GemvArgs a = {};
+    a.W = static_cast<const uint8_t*>(W);
+    a.N = N;
+    a.K = K;
+    a.row_bytes = static_cast<int64_t>(kq_row_bytes(fmt, K));
+    a.nb = static_cast<int>(K / 256);
+    a.n_seg = 1;
+    a.E = 1;
+    a.x = x;
+    a.ldx = k > 1 ? ldx : K;
+    a.y = y;
+    a.ldy = k > 1 ? ldy : N;
+    a.ksplit = S;
+    a.nbs = nbs;
+    a.partial = static_cast<float*>(workspace);
+    return run_grouped(a, fmt, k, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int kq_unpack(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d, kq_stream_t stream) {

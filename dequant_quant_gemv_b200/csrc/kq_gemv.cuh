@@ -329,15 +329,17 @@ __device__ __forceinline__ void raise_fault(const GemvArgs& a, volatile int* abo
 // Stage the activations of segment `seg` (all NCOL columns) into the
 // padded, permuted layout the units read, then (Q4_K) the region sums.
 template <int FMT, int NCOL>
-__device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar) {
-    const float* xg = a.x + seg * a.x_seg_stride;
-    const int nb = a.nb;
+__device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar, int kb0,
+                        int nbl) {
+    // the K range [256*kb0, 256*(kb0+nbl)) in regions laid out for a.nbs blocks
+    const float* xg = a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256;
+    const int nb = a.nbs;
     const int nreg = 2 * nb;
     const int xcs = nreg * kRegion;
     // fill: one item = 4 consecutive activations (a coalesced 16-byte load
     // when the column is 16-byte aligned), scattered into the region layout;
     // the 4 values land 2 floats apart (pair members alternate).
-    const int k4 = static_cast<int>(a.K >> 2);
+    const int k4 = nbl * 64;
     const int items = NCOL * k4;
     for (int it = ct; it < items; it += nthr) {
         const int j = it / k4;
@@ -369,10 +371,10 @@ __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int
     }
     named_bar_sync(bar, nthr);
     if constexpr (FMT == 1) {
-        const int sums = NCOL * nreg * 2;
+        const int sums = NCOL * 2 * nbl * 2;
         for (int it = ct; it < sums; it += nthr) {
-            const int j = it / (nreg * 2);
-            const int rem = it - j * nreg * 2;
+            const int j = it / (2 * nbl * 2);
+            const int rem = it - j * 2 * nbl * 2;
             const int reg = rem >> 1, cp = rem & 1;
             const uint32_t xr = xs + 4 * (j * xcs + reg * kRegion);
             st_s64f(xr + 4 * (128 + 2 * cp), q4k_region_sum(xr, cp));
@@ -421,8 +423,15 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
 
     const int64_t rps = (a.N + 1) / 2;
     const int64_t P = static_cast<int64_t>(a.n_seg) * rps;
-    const int64_t rp_begin = P * blockIdx.x / gridDim.x;
-    const int64_t rp_end = P * (blockIdx.x + 1) / gridDim.x;
+    // split-K: CTA c covers K range c % ksplit of row-pair range c / ksplit
+    const int ks = static_cast<int>(blockIdx.x) % a.ksplit;
+    const int64_t rc = blockIdx.x / a.ksplit, G = gridDim.x / a.ksplit;
+    const int64_t rp_begin = P * rc / G;
+    const int64_t rp_end = P * (rc + 1) / G;
+    constexpr int BS = FMT == 1 ? kQ4Bytes : kQ6Bytes;
+    const int kb0 = ks * a.nbs;
+    const int nbl = a.nb - kb0 < a.nbs ? a.nb - kb0 : a.nbs;       // blocks in this range
+    const int srow = a.ksplit > 1 ? a.nbs * BS : static_cast<int>(a.row_bytes);  // staged row stride
 
     if (warp == 0) {
         // ------------------------------------------------ producer (TMA)
@@ -443,9 +452,18 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             if (a.ids) e = a.ids[st.seg];
             if (e >= 0 && e < a.E) {
                 const uint8_t* src = a.W + e * a.seg_stride + st.row0 * a.row_bytes;
-                const uint32_t bytes = static_cast<uint32_t>(st.nrows * a.row_bytes);
-                mbar_arrive_expect_tx(&full[slot], bytes);
-                bulk_g2s(sbuf + static_cast<size_t>(slot) * a.stage_bytes, src, bytes, &full[slot]);
+                uint8_t* dst = sbuf + static_cast<size_t>(slot) * a.stage_bytes;
+                if (a.ksplit == 1) {  // whole rows: one contiguous copy
+                    const uint32_t bytes = static_cast<uint32_t>(st.nrows * a.row_bytes);
+                    mbar_arrive_expect_tx(&full[slot], bytes);
+                    bulk_g2s(dst, src, bytes, &full[slot]);
+                } else {              // this K range of each row
+                    const uint32_t rbytes = static_cast<uint32_t>(nbl * BS);
+                    mbar_arrive_expect_tx(&full[slot], rbytes * st.nrows);
+                    for (int i = 0; i < st.nrows; ++i)
+                        bulk_g2s(dst + i * srow, src + i * a.row_bytes + static_cast<int64_t>(kb0) * BS, rbytes,
+                                 &full[slot]);
+                }
             } else {
                 mbar_arrive(&full[slot]);
             }
@@ -470,7 +488,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     const int ct = ct_all & (kConsumers - 1);  // thread within the group
     const int cw = ct >> 5;                   // warp within the group
     const int gbar = 1 + g;                   // the group's named barrier
-    const int nb = a.nb;
+    const int nb = a.nbs;                     // lane layout: blocks of a full K range
     const int xcs = 2 * nb * kRegion;
     const bool shared_x = a.x_seg_stride == 0;
     pdl_wait();                      // activations may come from the previous grid
@@ -484,7 +502,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
         const int LR = a.lanes_per_rp;
         u_rp = ct / LR;
         const int u = ct - u_rp * LR;
-        u_active = u < 2 * nb;
+        u_active = u < 2 * nbl;
         u_b = u >> 1;
         u_H = u & 1;
         group = LR < 32 ? LR : 32;
@@ -495,7 +513,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
         u_rp = lane / LRw;
         const int u = lane - u_rp * LRw;
         const int nb8 = nb >> 3;
-        u_active = u < 2 * nb8;
+        u_active = u < 2 * (nbl >> 3);
         const int i = u >> 1;
         u_H = u & 1;
         u_b = 8 * i + kappa;
@@ -516,14 +534,14 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     int64_t staged_seg = -1;
     if (shared_x) {
         // one activation copy for all groups, staged by all consumer threads
-        stage_x<FMT, NCOL>(a, 0, xs_s, ct_all, NG * kConsumers, NG == 2 ? 3 : 1);
+        stage_x<FMT, NCOL>(a, 0, xs_s, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, kb0, nbl);
         staged_seg = 0;
     }
     int own = 0;  // stages this group has consumed
     while (it.next(st)) {
         if (NG == 2 && ((it.count - 1) & 1) != g) continue;
         if (!shared_x && st.seg != staged_seg) {
-            stage_x<FMT, NCOL>(a, st.seg, xs_s, ct, kConsumers, gbar);
+            stage_x<FMT, NCOL>(a, st.seg, xs_s, ct, kConsumers, gbar, kb0, nbl);
             staged_seg = st.seg;
         }
         const int slot = it.slot;
@@ -535,9 +553,9 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             for (int j = 0; j < NCOL; ++j) out[r][j] = 0.f;
         const bool work = u_active && u_rp < st.nrp && !*abort_flag;
         if (work) {
-            const uint32_t row0 = sbuf_s + slot * a.stage_bytes + 2 * u_rp * static_cast<int>(a.row_bytes);
-            if constexpr (FMT == 1) q4k_unit<NCOL>(row0, static_cast<int>(a.row_bytes), u_b, u_H, xr, xcs, out);
-            else q6k_unit_dispatch<NCOL>(kappa, row0, static_cast<int>(a.row_bytes), u_b, u_H, xr, xcs, out);
+            const uint32_t row0 = sbuf_s + slot * a.stage_bytes + 2 * u_rp * srow;
+            if constexpr (FMT == 1) q4k_unit<NCOL>(row0, srow, u_b, u_H, xr, xcs, out);
+            else q6k_unit_dispatch<NCOL>(kappa, row0, srow, u_b, u_H, xr, xcs, out);
         }
         // butterfly over the lanes of this row pair (fixed order)
 #pragma unroll
@@ -573,7 +591,10 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             if (valid) {
                 for (int p = 0; p < parts; ++p) v += ld_s32f(wb + 4 * (((rp * parts + p) * 2 + r) * NCOL + j));
             }
-            if (j < a.ncol_real) a.y[st.seg * a.y_seg_stride + j * a.ldy + st.row0 + row] = v;
+            if (j < a.ncol_real) {
+                if (a.ksplit == 1) a.y[st.seg * a.y_seg_stride + j * a.ldy + st.row0 + row] = v;
+                else a.partial[(static_cast<int64_t>(ks) * a.ncol_real + j) * a.N + st.row0 + row] = v;
+            }
         }
     }
 }

@@ -29,6 +29,10 @@ struct GemvArgs {
     int32_t* status;         // optional device status word
     int* fault;              // device fault word (timeouts)
     int ncol_real;           // columns written (the kernel may pad to 2/4/8)
+    // split-K across CTAs (ksplit == 1: every CTA covers all of K)
+    int ksplit;              // number of K ranges
+    int nbs;                 // super-blocks per K range (the last may be shorter)
+    float* partial;          // ksplit x ncol_real x N partial sums (ksplit > 1)
     // schedule (from plan_gemv)
     int ps;                  // row pairs per stage
     int lanes_per_rp;        // Q4_K: lanes per row pair; Q6_K: per row pair and warp
@@ -51,6 +55,8 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p);
 template <int FMT, int NCOL, int NG>
 cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
 cudaError_t fault_word(int** out);
+cudaError_t launch_splitk_combine(const float* partial, int S, int ncol, int64_t N, float* y, int64_t ldy,
+                                  cudaStream_t stream);
 cudaError_t launch_unpack(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d,
                           cudaStream_t stream);
 cudaError_t ensure_smem_attr(const void* func, size_t bytes);

@@ -71,6 +71,27 @@ cudaError_t launch_unpack(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q
     return cudaGetLastError();
 }
 
+// Split-K combine: y[j][r] = sum over K ranges s = 0..S-1 (in that order)
+// of partial[s][j][r].  Launched after gemv_kernel on the same stream.
+__global__ void splitk_combine_kernel(const float* __restrict__ partial, int S, int ncol, int64_t N, float* y,
+                                      int64_t ldy) {
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t >= ncol * N) return;
+    const int64_t j = t / N, r = t - j * N;
+    float v = 0.f;
+    for (int s = 0; s < S; ++s) v += partial[(static_cast<int64_t>(s) * ncol + j) * N + r];
+    y[j * ldy + r] = v;
+}
+
+cudaError_t launch_splitk_combine(const float* partial, int S, int ncol, int64_t N, float* y, int64_t ldy,
+                                  cudaStream_t stream) {
+    const int64_t n = static_cast<int64_t>(ncol) * N;
+    const int threads = 256;
+    const int64_t grid = (n + threads - 1) / threads;
+    splitk_combine_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(partial, S, ncol, N, y, ldy);
+    return cudaGetLastError();
+}
+
 // The fault word's device address, looked up once per device.
 cudaError_t fault_word(int** out) {
     static int* cache[64] = {};

@@ -112,6 +112,41 @@ def gemv_multi(W: torch.Tensor, fmt, N: int, K: int, X: torch.Tensor, Y: torch.T
     return Y
 
 
+def _splitk_sigs(L):
+    if not getattr(L, "_splitk_ready", False):
+        L.kq_splitk_workspace_bytes.restype = ctypes.c_size_t
+        L.kq_splitk_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
+        L.kq_gemv_splitk.restype = ctypes.c_int
+        L.kq_gemv_splitk.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                     ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                     ctypes.c_size_t, ctypes.c_void_p]
+        L._splitk_ready = True
+    return L
+
+
+def splitk_workspace_bytes(fmt, N: int, K: int, k: int = 1) -> int:
+    return int(_splitk_sigs(lib()).kq_splitk_workspace_bytes(_fmt(fmt), N, K, k))
+
+
+def gemv_splitk(W: torch.Tensor, fmt, N: int, K: int, X: torch.Tensor, Y: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """kq_gemv_splitk: X is (K,) or (k, K); the workspace is allocated here
+    (torch) when not given."""
+    L = _splitk_sigs(lib())
+    X2 = X.view(1, -1) if X.dim() == 1 else X
+    k = X2.shape[0]
+    if Y is None:
+        Y = torch.empty((k, N), dtype=torch.float32, device=X.device)
+    Y2 = Y.view(1, -1) if Y.dim() == 1 else Y
+    need = splitk_workspace_bytes(fmt, N, K, k)
+    if workspace is None:
+        workspace = torch.empty(max(1, (need + 3) // 4), dtype=torch.float32, device=X.device)
+    _check(L.kq_gemv_splitk(_dev(W, "W"), _fmt(fmt), N, K, _dev(X2, "X", torch.float32), X2.stride(0), k,
+                            _dev(Y2, "Y", torch.float32), Y2.stride(0), _dev(workspace, "workspace"),
+                            workspace.numel() * workspace.element_size(), _stream(stream)), "kq_gemv_splitk")
+    return Y
+
+
 def moe_gemv(W_experts: torch.Tensor, fmt, E: int, N: int, K: int, ids: torch.Tensor, x: torch.Tensor,
              y: torch.Tensor | None = None, status: torch.Tensor | None = None, expert_stride: int | None = None,
              stream=None) -> torch.Tensor:

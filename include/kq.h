@@ -124,6 +124,24 @@ KQ_API int kq_gemv_multi(const void* W, int fmt, int64_t N, int64_t K, const flo
                   int k, float* y, int64_t ldy, kq_stream_t stream);
 
 /*
+ * kq_gemv_splitk — kq_gemv_multi for tall-skinny matrices: when the matrix
+ * has fewer row pairs than the GPU has SMs, K is also split across CTAs.
+ * Each CTA writes the partial sums of its K range to `workspace`, and a
+ * second kernel adds the ranges in a fixed order (deterministic, but not
+ * bitwise equal to kq_gemv, whose summation order differs).  For matrices
+ * that need no split it is exactly kq_gemv_multi and ignores the workspace.
+ *   workspace: DEVICE scratch of at least kq_splitk_workspace_bytes(fmt, N,
+ *   K, k) bytes, owned by the caller; calls that share a workspace must not
+ *   overlap on the GPU.  Other arguments as kq_gemv_multi.
+ * Split-K for tall-skinny shapes; the pages' decode matvecs ("Kortex:
+ * Streaming 70B Models on Consumer GPUs", the paragraph before the first
+ * table) include narrow projections such as the grouped k/v heads.
+ */
+KQ_API size_t kq_splitk_workspace_bytes(int fmt, int64_t N, int64_t K, int k);
+KQ_API int kq_gemv_splitk(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx, int k,
+                          float* y, int64_t ldy, void* workspace, size_t workspace_bytes, kq_stream_t stream);
+
+/*
  * kq_moe_gemv — routed-expert GEMV.
  *   W_experts: E matrices, each N x K in `fmt`, matrix e at
  *   W_experts + e*expert_stride_bytes (stride >= N*row_bytes, 16-byte
