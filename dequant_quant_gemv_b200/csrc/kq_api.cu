@@ -23,6 +23,8 @@ static int fail(int status, const char* fmt, ...) {
     return status;
 }
 
+int set_last_error(int status, const char* msg) { return fail(status, "%s", msg); }
+
 static int cuda_fail(cudaError_t err, const char* what) {
     return fail(KQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
 }

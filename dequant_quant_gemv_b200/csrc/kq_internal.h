@@ -61,5 +61,7 @@ cudaError_t launch_unpack(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q
                           cudaStream_t stream);
 cudaError_t ensure_smem_attr(const void* func, size_t bytes);
 cudaError_t read_and_clear_fault(int* out);
+// Records `msg` as the calling thread's kq_last_error() text; returns status.
+int set_last_error(int status, const char* msg);
 
 }  // namespace kq

@@ -147,6 +147,27 @@ def gemv_splitk(W: torch.Tensor, fmt, N: int, K: int, X: torch.Tensor, Y: torch.
     return Y
 
 
+def gemv_splitk_noalloc(W: torch.Tensor, fmt, N: int, K: int, X: torch.Tensor, Y: torch.Tensor,
+                        stream=None) -> torch.Tensor:
+    """kq_gemv_splitk_noalloc: split-K GEMV with its partial sums in the
+    library's built-in scratch, for callers that cannot allocate device
+    memory.  X is (K,) or (k, K); Y must be given (this call allocates
+    nothing)."""
+    L = lib()
+    if not getattr(L, "_noalloc_ready", False):
+        L.kq_gemv_splitk_noalloc.restype = ctypes.c_int
+        L.kq_gemv_splitk_noalloc.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                             ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p,
+                                             ctypes.c_int64, ctypes.c_void_p]
+        L._noalloc_ready = True
+    X2 = X.view(1, -1) if X.dim() == 1 else X
+    Y2 = Y.view(1, -1) if Y.dim() == 1 else Y
+    _check(L.kq_gemv_splitk_noalloc(_dev(W, "W"), _fmt(fmt), N, K, _dev(X2, "X", torch.float32), X2.stride(0),
+                                    X2.shape[0], _dev(Y2, "Y", torch.float32), Y2.stride(0), _stream(stream)),
+           "kq_gemv_splitk_noalloc")
+    return Y
+
+
 def moe_gemv(W_experts: torch.Tensor, fmt, E: int, N: int, K: int, ids: torch.Tensor, x: torch.Tensor,
              y: torch.Tensor | None = None, status: torch.Tensor | None = None, expert_stride: int | None = None,
              stream=None) -> torch.Tensor:

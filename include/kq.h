@@ -142,6 +142,32 @@ KQ_API int kq_gemv_splitk(const void* W, int fmt, int64_t N, int64_t K, const fl
                           float* y, int64_t ldy, void* workspace, size_t workspace_bytes, kq_stream_t stream);
 
 /*
+ * kq_gemv_splitk_noalloc — kq_gemv_splitk for callers that cannot allocate
+ * device memory: a real-time or callback thread that must not enter the
+ * allocator (its locks, its implicit synchronisation), an engine whose device
+ * memory is all owned by its own arena, or a plugin given only its inputs and
+ * outputs.  Such callers cannot supply the split-K workspace, so this call
+ * keeps the partial sums in a 64 KiB array built into the library (every GPU
+ * that loads libkq holds it until the process exits).  It calls no cudaMalloc,
+ * cudaFree or allocating routine.
+ *   Arguments, layout and results are those of kq_gemv_splitk (the same
+ *   kernels and summation order, so the outputs are identical).
+ *   Errors: KQ_ERR_UNSUPPORTED when the split would need more partial sums
+ *   than the 64 KiB hold (16384 floats = ranges * k * N); the text is in
+ *   kq_last_error().  Other errors as kq_gemv_splitk.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   All calls share the one array: calls that overlap on the GPU (other
+ *   streams, other threads) race on it and must be ordered by the caller.
+ *   Nothing in it needs clearing between calls: each call writes every
+ *   partial sum it later reads.
+ * The pages have no counterpart to this entry point.
+ */
+KQ_API int kq_gemv_splitk_noalloc(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx,
+                                  int k, float* y, int64_t ldy, kq_stream_t stream);
+
+/*
  * kq_moe_gemv — routed-expert GEMV.
  *   W_experts: E matrices, each N x K in `fmt`, matrix e at
  *   W_experts + e*expert_stride_bytes (stride >= N*row_bytes, 16-byte
