@@ -375,6 +375,33 @@ def h2d_peak_gbs(torch, nbytes=512 << 20, reps=5):
     return best
 
 
+# ------------------------------------------------------ replicas over ranks
+def rank_seed(rank):
+    """Each rank decodes its own replica: same shapes, its own weights and
+    activations."""
+    return SEED + rank
+
+
+def max_over_ranks(value, device):
+    """The largest `value` over all ranks (the slowest replica's time); the
+    process group's own backend does the reduction (NCCL on GPUs, gloo on
+    CPU)."""
+    import torch
+    import torch.distributed as tdist
+
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank_step, steps, world, ms_max):
+    """Whole-job rate: the units every rank processed over the slowest
+    rank's time (weak scaling, each rank a full replica)."""
+    return units_per_rank_step * steps * world / (ms_max * 1e-3)
+
+
 # --------------------------------------------------------------- the bench
 def bench_kq(args, rank, world):
     import torch
@@ -387,7 +414,7 @@ def bench_kq(args, rank, world):
     dist = world > 1
     if dist:
         import torch.distributed as tdist
-    wl = make_workload(args.workload, torch, kq, kqgen, SEED + rank)
+    wl = make_workload(args.workload, torch, kq, kqgen, rank_seed(rank))
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)   # every launch, replay and event goes here
     advance = getattr(wl, "advance", None)
@@ -423,15 +450,11 @@ def bench_kq(args, rank, world):
             run_step()
         e1.record(stream)
         torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), "cuda")
     ms_step = ms / args.steps
     k = getattr(wl, "k", 1)
-    gbs = wl.weight_bytes * args.steps * world / (ms * 1e-3) / 1e9
-    tok_s = k * args.steps * world / (ms * 1e-3)
+    gbs = job_rate(wl.weight_bytes, args.steps, world, ms) / 1e9
+    tok_s = job_rate(k, args.steps, world, ms)
 
     # per-kernel device time of each matrix kind: a graph of all its
     # launches (different layers' weights, so never L2-hot), events around it
@@ -484,11 +507,7 @@ def bench_kq(args, rank, world):
         e2e_step()
     f1.record(stream)
     torch.cuda.synchronize()
-    ems = f0.elapsed_time(f1)
-    if dist:
-        t = torch.tensor([ems], device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ems = float(t.item())
+    ems = max_over_ranks(f0.elapsed_time(f1), "cuda")
 
     peaks = {}
     try:
@@ -507,8 +526,8 @@ def bench_kq(args, rank, world):
                    "weight_bytes_per_step": wl.weight_bytes, "launches_per_step": len(wl.launches),
                    "columns": k, "batch": 1, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (no flush)" if wl.weight_bytes > 2 * 126e6 else "rotating copies"},
-        "e2e": {"value": round(wl.weight_bytes * args.steps * world / (ems * 1e-3) / 1e9, 2), "unit": "GB/s",
-                "tok_per_s": round(k * args.steps * world / (ems * 1e-3), 3),
+        "e2e": {"value": round(job_rate(wl.weight_bytes, args.steps, world, ems) / 1e9, 2), "unit": "GB/s",
+                "tok_per_s": round(job_rate(k, args.steps, world, ems), 3),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
         "gpu_launches": len(wl.launches) * args.steps,
