@@ -161,6 +161,53 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     return KQ_OK;
 }
 
+// Schedule of the tensor-core kernel (2..8 columns): 16-row stages, rows
+// `sp` bytes apart in smem (sp >= the staged row, sp = 64 mod 128), B
+// fragments of the CTA's K range for NT n-tiles, two partial-sum buffers.
+int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
+    DevInfo di;
+    cudaError_t err = dev_info(di);
+    if (err != cudaSuccess) return cuda_fail(err, "device query");
+    if (fmt != KQ_FMT_Q4_K) return fail(KQ_ERR_UNSUPPORTED, "tensor-core kernel: Q4_K only");
+    const size_t srow = static_cast<size_t>(a.nbs) * kq_block_bytes(fmt);
+    const size_t sp = srow <= 64 ? 64 : round_up(srow - 64, 128) + 64;
+    const size_t stage = round_up(16 * sp, 128);
+    const int nc = 4 * nt;
+    const size_t head = 256;
+    const size_t wp_bytes = sizeof(float) * 2 * kConsumerWarps * 16 * nc;
+    const size_t bs_bytes = round_up(sizeof(float) * 2 * nc * a.nbs, 128);
+    const size_t xb_bytes = static_cast<size_t>(a.nbs) * 17 * 32 * nt * 8;
+    const size_t fixed = head + wp_bytes + bs_bytes + xb_bytes;
+    const size_t limit = static_cast<size_t>(di.smem_optin);
+    if (fixed + 2 * stage > limit)
+        return fail(KQ_ERR_UNSUPPORTED, "K=%lld with %d columns needs %zu bytes of shared memory (limit %zu)",
+                    (long long)a.K, nc, fixed + 2 * stage, limit);
+    size_t ns = (limit - fixed) / stage;
+    if (ns > kMaxStages) ns = kMaxStages;
+    const int64_t rps = (a.N + 1) / 2;
+    const int64_t tiles = (rps + 7) / 8;                  // 16-row stages of the matrix
+    const int64_t ranges = di.sm_count / a.ksplit;
+    const int64_t grid = (tiles < ranges ? tiles : ranges) * a.ksplit;
+    const int64_t per_cta = (rps + grid / a.ksplit - 1) / (grid / a.ksplit);
+    const int64_t need = (per_cta + 7) / 8 + 1;
+    if (static_cast<int64_t>(ns) > need) ns = need < 2 ? 2 : static_cast<size_t>(need);
+    a.ps = 8;
+    a.parts = 1;
+    a.lanes_per_rp = 0;
+    a.sp = static_cast<int>(sp);
+    a.nstage = static_cast<int>(ns);
+    a.stage_bytes = static_cast<int>(stage);
+    a.wp_offset = static_cast<int>(head);
+    a.xscale_offset = static_cast<int>(head + wp_bytes);
+    a.xs_offset = static_cast<int>(head + wp_bytes + bs_bytes);
+    a.sbuf_offset = static_cast<int>(fixed);
+    p.grid = static_cast<int>(grid);
+    p.ng = 1;
+    p.smem_bytes = fixed + ns * stage;
+    p.pdl = true;
+    return KQ_OK;
+}
+
 static bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
 static int check_matrix(const void* W, int fmt, int64_t N, int64_t K) {
@@ -197,15 +244,25 @@ static cudaError_t dispatch(const GemvArgs& a, const LaunchPlan& p, int fmt, int
     }
 }
 
-static int run(GemvArgs& a, int fmt, int k, cudaStream_t stream) {
-    const int ncol = padded_cols(k);
+// Calls with 2 or more columns (speculative verify) run on the tensor-core
+// kernel, every column group of the call included, so a column's arithmetic
+// never depends on how the call was grouped.
+static bool use_mma(int fmt, int k) { return k >= 2 && fmt == KQ_FMT_Q4_K; }
+
+static int plan_for(int fmt, int k, bool mma, GemvArgs& a, LaunchPlan& p) {
+    if (mma) return plan_mma(fmt, k <= 4 ? 1 : 2, a, p);
+    return plan_gemv(fmt, padded_cols(k), a, p);
+}
+
+static int run(GemvArgs& a, int fmt, int k, bool mma, cudaStream_t stream) {
     a.ncol_real = k;
     cudaError_t err = fault_word(&a.fault);
     if (err != cudaSuccess) return cuda_fail(err, "fault word");
     LaunchPlan p;
-    int st = plan_gemv(fmt, ncol, a, p);
+    int st = plan_for(fmt, k, mma, a, p);
     if (st != KQ_OK) return st;
-    err = dispatch(a, p, fmt, ncol, stream);
+    if (mma) err = k <= 4 ? launch_mma<1, 1>(a, p, stream) : launch_mma<1, 2>(a, p, stream);
+    else err = dispatch(a, p, fmt, padded_cols(k), stream);
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
     if (a.ksplit > 1) {
         err = launch_splitk_combine(a.partial, a.ksplit, k, a.N, a.y, a.ldy, stream);
@@ -236,11 +293,11 @@ static void choose_split(int fmt, int64_t N, int nb, int sm_count, int* S, int* 
 
 // Largest padded column count whose staged activations fit in shared
 // memory next to a two-stage weight ring (0 if not even one column fits).
-static int max_fitting_cols(const GemvArgs& proto, int fmt) {
-    for (int c = 8; c >= 1; c >>= 1) {
+static int max_fitting_cols(const GemvArgs& proto, int fmt, bool mma) {
+    for (int c = 8; c >= (mma ? 4 : 1); c >>= 1) {
         GemvArgs t = proto;
         LaunchPlan p;
-        if (plan_gemv(fmt, c, t, p) == KQ_OK) return c;
+        if (plan_for(fmt, c, mma, t, p) == KQ_OK) return c;
     }
     return 0;
 }
@@ -249,10 +306,17 @@ static int max_fitting_cols(const GemvArgs& proto, int fmt) {
 // read once per group).  Every column's arithmetic is the same whatever the
 // grouping, so results do not depend on it.
 static int run_grouped(GemvArgs& a, int fmt, int k, cudaStream_t stream) {
-    const int g = max_fitting_cols(a, fmt);
+    // the tensor-core kernel when its activation fragments fit (for the
+    // whole call), else the CUDA-core kernel
+    bool mma = use_mma(fmt, k);
+    int g = mma ? max_fitting_cols(a, fmt, true) : 0;
+    if (g == 0) {
+        mma = false;
+        g = max_fitting_cols(a, fmt, false);
+    }
     if (g == 0) {
         LaunchPlan p;
-        return plan_gemv(fmt, 1, a, p);  // fails again, recording the reason
+        return plan_for(fmt, 1, false, a, p);  // fails again, recording the reason
     }
     g_last_error[0] = 0;
     for (int c0 = 0; c0 < k; c0 += g) {
@@ -260,7 +324,7 @@ static int run_grouped(GemvArgs& a, int fmt, int k, cudaStream_t stream) {
         t.x = a.x + static_cast<int64_t>(c0) * a.ldx;
         t.y = a.y + static_cast<int64_t>(c0) * a.ldy;  // partial sums restart at the workspace base
         const int kk = k - c0 < g ? k - c0 : g;
-        int st = run(t, fmt, kk, stream);
+        int st = run(t, fmt, kk, mma, stream);
         if (st != KQ_OK) return st;
     }
     return KQ_OK;
@@ -397,7 +461,7 @@ int kq_moe_gemv(const void* W_experts, int fmt, int E, int64_t N, int64_t K, siz
     a.ksplit = 1;
     a.nbs = a.nb;
     a.partial = nullptr;
-    return run(a, fmt, 1, s);
+    return run(a, fmt, 1, false, s);
 }
 
 static int split_for(int fmt, int64_t N, int64_t K, int* S, int* nbs) {

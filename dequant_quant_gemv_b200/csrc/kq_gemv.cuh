@@ -324,6 +324,62 @@ __device__ __forceinline__ void raise_fault(const GemvArgs& a, volatile int* abo
     if (a.fault) atomicExch(a.fault, code);
 }
 
+// ------------------------------------------------------------ producer
+
+// The producer thread: walks the CTA's stages and brings each one's rows
+// into its ring slot with 1-D bulk copies (no multicast), waiting for the
+// consumers to release a slot before reusing it.  `contiguous`: whole rows
+// stored back to back (one copy per stage); otherwise each row's K range
+// [kb0, kb0 + nbl) blocks is copied to its own smem row `srow` bytes apart.
+template <int BS>
+__device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empty, volatile int* abort_flag,
+                               uint8_t* sbuf, int64_t rp_begin, int64_t rp_end, int64_t rps, int ns, int kb0,
+                               int nbl, int srow, bool contiguous) {
+    if (a.ids) pdl_wait();  // routed ids may come from the previous grid
+    StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
+    Stage st;
+    bool ok = true;
+    while (it.next(st)) {
+        const int slot = it.slot;
+        // a reused slot: wait until the consumers released its last stage
+        if (it.count > ns && !mbar_wait_bounded(&empty[slot], it.phase ^ 1u, abort_flag)) {
+            raise_fault(a, abort_flag, 6);
+            ok = false;
+            break;
+        }
+        int64_t e = st.seg;
+        if (a.ids) e = a.ids[st.seg];
+        if (e >= 0 && e < a.E) {
+            const uint8_t* src = a.W + e * a.seg_stride + st.row0 * a.row_bytes;
+            uint8_t* dst = sbuf + static_cast<size_t>(slot) * a.stage_bytes;
+            if (contiguous) {
+                const uint32_t bytes = static_cast<uint32_t>(st.nrows * a.row_bytes);
+                mbar_arrive_expect_tx(&full[slot], bytes);
+                bulk_g2s(dst, src, bytes, &full[slot]);
+            } else {
+                const uint32_t rbytes = static_cast<uint32_t>(nbl * BS);
+                mbar_arrive_expect_tx(&full[slot], rbytes * st.nrows);
+                for (int i = 0; i < st.nrows; ++i)
+                    bulk_g2s(dst + i * srow, src + i * a.row_bytes + static_cast<int64_t>(kb0) * BS, rbytes,
+                             &full[slot]);
+            }
+        } else {
+            mbar_arrive(&full[slot]);
+        }
+    }
+    // Let every copy this CTA issued land before the CTA can exit.
+    int issued = ok ? it.count : it.count - 1;
+    int sl = ok ? it.slot : (it.slot == 0 ? ns - 1 : it.slot - 1);
+    uint32_t ph = ok ? it.phase : (it.slot == 0 ? it.phase ^ 1u : it.phase);
+    for (int i = 0; i < issued && i < ns; ++i) {
+        if (!mbar_wait_bounded(&full[sl], ph, abort_flag)) break;
+        if (--sl < 0) {
+            sl = ns - 1;
+            ph ^= 1u;
+        }
+    }
+}
+
 // ------------------------------------------------------ activation stage
 
 // Stage the activations of segment `seg` (all NCOL columns) into the
@@ -434,51 +490,9 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     const int srow = a.ksplit > 1 ? a.nbs * BS : static_cast<int>(a.row_bytes);  // staged row stride
 
     if (warp == 0) {
-        // ------------------------------------------------ producer (TMA)
-        if (lane != 0) return;
-        if (a.ids) pdl_wait();  // routed ids may come from the previous grid
-        StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
-        Stage st;
-        bool ok = true;
-        while (it.next(st)) {
-            const int slot = it.slot;
-            // a reused slot: wait until the consumers released its last stage
-            if (it.count > ns && !mbar_wait_bounded(&empty[slot], it.phase ^ 1u, abort_flag)) {
-                raise_fault(a, abort_flag, 6);
-                ok = false;
-                break;
-            }
-            int64_t e = st.seg;
-            if (a.ids) e = a.ids[st.seg];
-            if (e >= 0 && e < a.E) {
-                const uint8_t* src = a.W + e * a.seg_stride + st.row0 * a.row_bytes;
-                uint8_t* dst = sbuf + static_cast<size_t>(slot) * a.stage_bytes;
-                if (a.ksplit == 1) {  // whole rows: one contiguous copy
-                    const uint32_t bytes = static_cast<uint32_t>(st.nrows * a.row_bytes);
-                    mbar_arrive_expect_tx(&full[slot], bytes);
-                    bulk_g2s(dst, src, bytes, &full[slot]);
-                } else {              // this K range of each row
-                    const uint32_t rbytes = static_cast<uint32_t>(nbl * BS);
-                    mbar_arrive_expect_tx(&full[slot], rbytes * st.nrows);
-                    for (int i = 0; i < st.nrows; ++i)
-                        bulk_g2s(dst + i * srow, src + i * a.row_bytes + static_cast<int64_t>(kb0) * BS, rbytes,
-                                 &full[slot]);
-                }
-            } else {
-                mbar_arrive(&full[slot]);
-            }
-        }
-        // Let every copy this CTA issued land before the CTA can exit.
-        int issued = ok ? it.count : it.count - 1;
-        int sl = ok ? it.slot : (it.slot == 0 ? ns - 1 : it.slot - 1);
-        uint32_t ph = ok ? it.phase : (it.slot == 0 ? it.phase ^ 1u : it.phase);
-        for (int i = 0; i < issued && i < ns; ++i) {
-            if (!mbar_wait_bounded(&full[sl], ph, abort_flag)) break;
-            if (--sl < 0) {
-                sl = ns - 1;
-                ph ^= 1u;
-            }
-        }
+        if (lane == 0)
+            produce_stages<BS>(a, full, empty, abort_flag, sbuf, rp_begin, rp_end, rps, ns, kb0, nbl, srow,
+                               a.ksplit == 1);
         return;
     }
 

@@ -40,6 +40,9 @@ struct GemvArgs {
     int nstage;
     int stage_bytes;
     int wp_offset, xs_offset, sbuf_offset;
+    // tensor-core (multi-column) kernel only
+    int sp;                  // smem bytes between staged rows (padded)
+    int xscale_offset;       // power-of-two scales per super-block and column
 };
 
 struct LaunchPlan {
@@ -54,6 +57,10 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p);
 
 template <int FMT, int NCOL, int NG>
 cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
+// Tensor-core kernel for 2..8 columns: NT n-tiles of 8 (4 columns each).
+int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p);
+template <int FMT, int NT>
+cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
 cudaError_t fault_word(int** out);
 cudaError_t launch_splitk_combine(const float* partial, int S, int ncol, int64_t N, float* y, int64_t ldy,
                                   cudaStream_t stream);

@@ -1,0 +1,416 @@
+// kq_mma.cuh — the fused K-quant GEMV for 2..8 activation columns on the
+// tensor cores: the speculative-verify shape, where k token columns share
+// one read of every weight block (Kortex and runNburn pages: the
+// multi-token verify matvec).
+//
+// With k columns the per-weight work of the CUDA-core kernel grows with k
+// (one FMA per weight per column); here the multiply-adds go to mma.sync
+// m16n8k16 (f16 inputs, f32 accumulation) and the per-weight cost is the
+// dequantisation alone, whatever k is.
+//
+// Exactness.  The A operand (weights) is the integer product sc*q of a
+// sub-block scale and a quant, which fp16 represents exactly for Q4_K
+// (|sc*q| <= 63*15 < 2048): one fp16 FMA per two weights turns a nibble
+// placed in the mantissa of 1024 (0x6400 | n) into sc*n with no rounding.
+// The B operand (activations) is each fp32 value split into two fp16 terms
+// hi + lo (22 bits), after a power-of-two scale per column and super-block
+// that keeps the largest |x| of the block in [2^14, 2^15), so neither term
+// overflows and small values keep their absolute precision.  d and the min
+// term are applied per super-block in fp32: y = sum_b 2^-e_b d_b S_b - sum_b
+// 2^(5-e_b) dmin_b M_b, where S_b = sum sc*q*x (16 K-steps) and M_b =
+// sum_j m_j X_j (one more K-step whose A holds the 8 mins and B the
+// sub-block sums of x, scaled by 2^(e_b-5) to stay in fp16 range).
+//
+// Schedule.  The persistent CTA and its TMA ring are those of gemv_kernel;
+// a stage is 16 rows (one m16 tile), copied row by row into smem rows
+// `a.sp` bytes apart (a.sp = 64 mod 128 keeps the fragment loads free of
+// bank conflicts).  The 8 consumer warps split the stage's super-blocks
+// (warp w takes blocks w, w+8, ...) and add their partial sums in a fixed
+// order, so results are deterministic and each column's value does not
+// depend on the other columns.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "kq_gemv.cuh"
+
+namespace kq {
+
+constexpr int kMmaRowPairs = 8;  // 16 rows per stage
+constexpr int kMmaSteps = 17;    // K-steps per super-block: 16 of quants + 1 of mins
+
+// D += A * B for one m16n8k16 tile (row-major A, column-major B).
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t hfma2u(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t hadd2u(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
+    return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+}
+__device__ __forceinline__ void st_s64u(uint32_t a, uint32_t x, uint32_t y) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void st_s32u(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_s16u(uint32_t a, uint16_t v) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(v) : "memory");
+}
+__device__ __forceinline__ uint2 ld_s64u(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+
+constexpr uint32_t kH2_1024 = 0x64006400u;    // (1024, 1024)
+constexpr uint32_t kH2_m1024 = 0xE400E400u;   // (-1024, -1024)
+constexpr uint32_t kH2_1_16 = 0x2C002C00u;    // (1/16, 1/16)
+constexpr uint32_t kH2_m64 = 0xD400D400u;     // (-64, -64)
+
+// Two 6-bit values (bytes p and p+1 of `packed`) as the fp16 pair
+// (v_p, v_p+1), exactly: 1024 + v by byte permute, then minus 1024.
+__device__ __forceinline__ uint32_t byte_pair_h2(uint32_t packed, uint32_t sel) {
+    return hadd2u(__byte_perm(packed, 0x64646464u, sel), kH2_m1024);
+}
+
+// ------------------------------------------------------ activation stage
+
+// Power-of-two scale exponent that brings a largest |x| (amax) into
+// [2^14, 2^15): 14 - floor(log2(amax)), clamped so 2^+-sh stays a normal
+// float.  Zero columns get 0.
+__device__ __forceinline__ int col_shift(uint32_t amax_bits) {
+    if (amax_bits == 0) return 0;
+    int sh = 14 - (static_cast<int>(amax_bits >> 23) - 127);
+    return sh > 120 ? 120 : sh < -120 ? -120 : sh;
+}
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
+
+// B-fragment store of one column's 4 consecutive activations of super-block
+// `bl` (relative), K position `w` (multiple of 4) within it.  Weight w of a
+// Q4_K block is quant byte beta = 32*(w/64) + w%32, low nibble for
+// (w/32) even, high nibble otherwise; byte beta sits in 16-byte chunk
+// beta/16, word (beta/4)%4.  A thread whose lane has q = chunk%4 feeds
+// that word to K-step pair j = 4*(chunk/4) + word, step 2j (low nibbles) or
+// 2j+1 (high); its K positions 2q, 2q+1 hold bytes 0 and 2 of the word and
+// 2q+8, 2q+9 bytes 1 and 3.  The column occupies B columns 2c' (hi term)
+// and 2c'+1 (lo term) of n-tile col/4, c' = col%4, i.e. lanes with
+// g = 2c' and 2c'+1.
+template <int NT>
+__device__ __forceinline__ void q4k_store_b(uint32_t xb, int bl, int w, int col, float4 v) {
+    const int hi = (w >> 5) & 1;
+    const int beta = 32 * (w >> 6) + (w & 31);
+    const int ch = beta >> 4, u = (beta >> 2) & 3;
+    const int q = ch & 3, j = ((ch >> 2) << 2) | u, s = 2 * j + hi;
+    const int nt = col >> 2, gh = 2 * (col & 3);
+    const __half h0 = __float2half_rn(v.x), h1 = __float2half_rn(v.y), h2 = __float2half_rn(v.z),
+                 h3 = __float2half_rn(v.w);
+    const __half l0 = __float2half_rn(v.x - __half2float(h0)), l1 = __float2half_rn(v.y - __half2float(h1)),
+                 l2 = __float2half_rn(v.z - __half2float(h2)), l3 = __float2half_rn(v.w - __half2float(h3));
+    const uint32_t step = xb + 8u * static_cast<uint32_t>(((bl * kMmaSteps + s) * 32) * NT + nt);
+    st_s64u(step + 8u * NT * (4 * gh + q), pack_h2(h0, h2), pack_h2(h1, h3));
+    st_s64u(step + 8u * NT * (4 * (gh + 1) + q), pack_h2(l0, l2), pack_h2(l1, l3));
+}
+
+// Stage the activations of the K range [256*kb0, 256*(kb0+nbl)) as
+// B fragments (see q4k_store_b) plus, per block, the min step: lane (g, q)
+// holds (X_2q, X_2q+1) of its column's hi or lo term and zeros for K
+// positions 8..15, X_j being the sub-block sum of 32 activations.  Each
+// (column, block) is scaled by its own power of two 2^sh (largest |x| of
+// the block into [2^14, 2^15)) and its sums by 2^(sh-5); `bscale` gets
+// (2^-sh, 2^(5-sh)) per block and column.  Columns >= ncol_real are zero.
+// One warp per (column, block) item, two float4 per lane, several items'
+// loads in flight.
+template <int NT>
+__device__ void stage_xb_q4k(const GemvArgs& a, uint32_t xb, float* bscale, int cw, int lane, int bar, int kb0,
+                             int nbl) {
+    constexpr int NC = 4 * NT;
+    constexpr int U = 4;  // items per warp in flight
+    const float* xg = a.x + static_cast<int64_t>(kb0) * 256;
+    const int kr = a.ncol_real;
+    const int items = NC * nbl;
+    for (int base = cw; base < items; base += kConsumerWarps * U) {
+        float4 v[U][2];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int it = base + kConsumerWarps * u;
+            const int col = it / nbl, bl = it - col * nbl;
+            v[u][0] = v[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (it < items && col < kr) {
+                const float* xc = xg + col * a.ldx + 256 * bl + 4 * lane;
+                if ((reinterpret_cast<uintptr_t>(xc) & 15u) == 0) {
+                    v[u][0] = *reinterpret_cast<const float4*>(xc);
+                    v[u][1] = *reinterpret_cast<const float4*>(xc + 128);
+                } else {
+                    v[u][0] = make_float4(xc[0], xc[1], xc[2], xc[3]);
+                    v[u][1] = make_float4(xc[128], xc[129], xc[130], xc[131]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int it = base + kConsumerWarps * u;
+            if (it >= items) break;  // warp-uniform
+            const int col = it / nbl, bl = it - col * nbl;
+            float m = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(v[u][h].x), fabsf(v[u][h].y)), fmaxf(fabsf(v[u][h].z), fabsf(v[u][h].w))));
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            const int sh = col_shift(__float_as_uint(m));
+            const float sc = pow2f(sh), scm = pow2f(sh - 5);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float4 t = make_float4(v[u][h].x * sc, v[u][h].y * sc, v[u][h].z * sc, v[u][h].w * sc);
+                q4k_store_b<NT>(xb, bl, 128 * h + 4 * lane, col, t);
+                // sub-block 4h + lane/8: the 8 lanes of this group, fixed order
+                float X = (v[u][h].x + v[u][h].y) + (v[u][h].z + v[u][h].w);
+                X += __shfl_xor_sync(0xffffffffu, X, 1);
+                X += __shfl_xor_sync(0xffffffffu, X, 2);
+                X += __shfl_xor_sync(0xffffffffu, X, 4);
+                if ((lane & 7) == 0) {
+                    const int j = 4 * h + (lane >> 3);
+                    X *= scm;
+                    const __half xh = __float2half_rn(X);
+                    const __half xl = __float2half_rn(X - __half2float(xh));
+                    const int nt = col >> 2, gh = 2 * (col & 3), q = j >> 1;
+                    const uint32_t step = xb + 8u * static_cast<uint32_t>(((bl * kMmaSteps + 16) * 32) * NT + nt);
+                    const uint32_t eh = step + 8u * NT * (4 * gh + q), el = step + 8u * NT * (4 * (gh + 1) + q);
+                    st_s16u(eh + 2 * (j & 1), __half_as_ushort(xh));
+                    st_s16u(el + 2 * (j & 1), __half_as_ushort(xl));
+                    if ((j & 1) == 0) {
+                        st_s32u(eh + 4, 0u);
+                        st_s32u(el + 4, 0u);
+                    }
+                }
+            }
+            if (lane == 0) {
+                bscale[2 * (bl * NC + col)] = pow2f(-sh);
+                bscale[2 * (bl * NC + col) + 1] = pow2f(5 - sh);
+            }
+        }
+    }
+    named_bar_sync(bar, kConsumers);
+}
+
+// ------------------------------------------------------ one super-block
+
+// Rows g and g+8 of the stage (smem rows rg, rg8), super-block b, this
+// lane's K positions (q = lane%4); B fragments of the block at `xbl` (this
+// lane's entry of step 0).  Adds d*S and dmin*M into ys / ym for the lane's
+// columns 4*nt + q.
+template <int NT>
+__device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t bsc,
+                                              uint32_t sel, uint32_t msel, int q, float (&ys)[2][NT],
+                                              float (&ym)[2][NT]) {
+    const uint32_t o = static_cast<uint32_t>(b) * kQ4Bytes;
+    const uint4 hg = ld_s128(rg + o), hg8 = ld_s128(rg8 + o);
+    uint4 w[2][2];  // [row][chunk q / q+4]
+    w[0][0] = ld_s128(rg + o + 16 + 16 * q);
+    w[0][1] = ld_s128(rg + o + 80 + 16 * q);
+    w[1][0] = ld_s128(rg8 + o + 16 + 16 * q);
+    w[1][1] = ld_s128(rg8 + o + 80 + 16 * q);
+    // per row and chunk: (scale of the low-nibble sub-block, of the high)
+    uint32_t mlo[2][2], alo[2][2], mhi[2][2], ahi[2][2], mins[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint4 h = r ? hg8 : hg;
+        uint32_t sc0, m0, sc1, m1;
+        q4k_half_scales(h.y, h.z, h.w, 0, sc0, m0);
+        q4k_half_scales(h.y, h.z, h.w, 1, sc1, m1);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint32_t S = byte_pair_h2(c ? sc1 : sc0, sel);
+            const uint32_t slo = __byte_perm(S, 0u, 0x1010u), shi = __byte_perm(S, 0u, 0x3232u);
+            mlo[r][c] = slo;
+            alo[r][c] = hmul2u(slo, kH2_m1024);
+            mhi[r][c] = hmul2u(shi, kH2_1_16);
+            ahi[r][c] = hmul2u(shi, kH2_m64);
+        }
+        mins[r] = byte_pair_h2(q < 2 ? m0 : m1, msel);
+    }
+    float acc[NT][4], accm[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = accm[n][i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int c = j >> 2;
+        uint32_t L02[2], L13[2], H02[2], H13[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint32_t x = u4w(w[r][c], j & 3);
+            const uint32_t xs = x >> 8;
+            L02[r] = hfma2u((x & 0x000F000Fu) | kH2_1024, mlo[r][c], alo[r][c]);
+            L13[r] = hfma2u((xs & 0x000F000Fu) | kH2_1024, mlo[r][c], alo[r][c]);
+            H02[r] = hfma2u((x & 0x00F000F0u) | kH2_1024, mhi[r][c], ahi[r][c]);
+            H13[r] = hfma2u((xs & 0x00F000F0u) | kH2_1024, mhi[r][c], ahi[r][c]);
+        }
+        const uint32_t s_lo = xbl + 8u * NT * 32 * (2 * j), s_hi = s_lo + 8u * NT * 32;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const uint2 bl = ld_s64u(s_lo + 8 * n), bh = ld_s64u(s_hi + 8 * n);
+            mma16816(acc[n], L02[0], L02[1], L13[0], L13[1], bl.x, bl.y);
+            mma16816(acc[n], H02[0], H02[1], H13[0], H13[1], bh.x, bh.y);
+        }
+    }
+    {
+        const uint32_t s_m = xbl + 8u * NT * 32 * 16;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const uint2 bm = ld_s64u(s_m + 8 * n);
+            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bm.x, bm.y);
+        }
+    }
+    const float d0 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg.x & 0xFFFFu)));
+    const float m0 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg.x >> 16)));
+    const float d1 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg8.x & 0xFFFFu)));
+    const float m1 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg8.x >> 16)));
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const float2 f = ld_s64f(bsc + 8u * (4 * n + q));  // (2^-sh, 2^(5-sh)) of column 4n+q
+        ys[0][n] = fmaf(d0 * f.x, acc[n][0] + acc[n][1], ys[0][n]);
+        ys[1][n] = fmaf(d1 * f.x, acc[n][2] + acc[n][3], ys[1][n]);
+        ym[0][n] = fmaf(m0 * f.y, accm[n][0] + accm[n][1], ym[0][n]);
+        ym[1][n] = fmaf(m1 * f.y, accm[n][2] + accm[n][3], ym[1][n]);
+    }
+}
+
+// ------------------------------------------------------------ the kernel
+
+template <int FMT, int NT>
+__global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_constant__ GemvArgs a) {
+    constexpr int NC = 4 * NT;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 2 * kMaxStages * 8);
+    float* bscale = reinterpret_cast<float*>(smem + a.xscale_offset);  // [block][column] (2^-sh, 2^(5-sh))
+    uint8_t* sbuf = smem + a.sbuf_offset;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int ns = a.nstage;
+    if (tid == 0) {
+        for (int s = 0; s < ns; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    const int64_t rps = (a.N + 1) / 2;
+    const int ks = static_cast<int>(blockIdx.x) % a.ksplit;
+    const int64_t rc = blockIdx.x / a.ksplit, G = gridDim.x / a.ksplit;
+    const int64_t rp_begin = rps * rc / G;
+    const int64_t rp_end = rps * (rc + 1) / G;
+    constexpr int BS = FMT == 1 ? kQ4Bytes : kQ6Bytes;
+    const int kb0 = ks * a.nbs;
+    const int nbl = a.nb - kb0 < a.nbs ? a.nb - kb0 : a.nbs;
+
+    if (warp == 0) {
+        if (lane == 0)
+            produce_stages<BS>(a, full, empty, abort_flag, sbuf, rp_begin, rp_end, rps, ns, kb0, nbl, a.sp, false);
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    const int ct = tid - 32;
+    const int cw = ct >> 5;
+    const int g = lane >> 2, q = lane & 3;
+    const uint32_t xb_s = smem_u32(smem + a.xs_offset);
+    const uint32_t wp_s = smem_u32(smem + a.wp_offset);
+    const uint32_t sbuf_s = smem_u32(sbuf);
+    pdl_wait();
+    pdl_launch_dependents();
+    stage_xb_q4k<NT>(a, xb_s, bscale, cw, lane, 1, kb0, nbl);
+
+    // byte selectors: scales of chunk q (half 0) / q+4 (half 1) sit at bytes
+    // 2*(q/2), 2*(q/2)+1 of either half; mins 2q, 2q+1 at bytes 2*(q%2), +1
+    const uint32_t p0 = 2u * static_cast<uint32_t>(q >> 1), pm = 2u * static_cast<uint32_t>(q & 1);
+    const uint32_t sel = 0x4040u | p0 | ((p0 + 1) << 8);
+    const uint32_t msel = 0x4040u | pm | ((pm + 1) << 8);
+    const uint32_t xlane = xb_s + 8u * NT * lane;
+    const uint32_t bsc_s = smem_u32(bscale);
+
+    StageIter it(rp_begin, rp_end, rps, a.N, kMmaRowPairs, ns);
+    Stage st;
+    int own = 0;
+    while (it.next(st)) {
+        const int slot = it.slot;
+        if (!mbar_wait_bounded(&full[slot], it.phase, abort_flag)) raise_fault(a, abort_flag, 6);
+        float ys[2][NT], ym[2][NT];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int n = 0; n < NT; ++n) ys[r][n] = ym[r][n] = 0.f;
+        if (!*abort_flag) {
+            const uint32_t rg = sbuf_s + slot * a.stage_bytes + g * a.sp;
+            const uint32_t rg8 = rg + 8 * a.sp;
+            for (int b = cw; b < nbl; b += kConsumerWarps)
+                q4k_mma_block<NT>(rg, rg8, b, xlane + 8u * NT * 32 * kMmaSteps * b, bsc_s + 8u * NC * b, sel,
+                                  msel, q, ys, ym);
+        }
+        const uint32_t wb = wp_s + 4u * ((own & 1) * (kConsumerWarps * 16 * NC));
+        ++own;
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+                st_s32f(wb + 4u * ((cw * 16 + g + 8 * r) * NC + 4 * n + q), ys[r][n] - ym[r][n]);
+        const bool stop = named_bar_or(1, kConsumers, *abort_flag != 0);
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (stop) break;
+        for (int t = ct; t < st.nrows * NC; t += kConsumers) {
+            const int row = t / NC, j = t - row * NC;
+            if (j >= a.ncol_real) continue;
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) v += ld_s32f(wb + 4u * ((w * 16 + row) * NC + j));
+            if (a.ksplit == 1) a.y[j * a.ldy + st.row0 + row] = v;
+            else a.partial[(static_cast<int64_t>(ks) * a.ncol_real + j) * a.N + st.row0 + row] = v;
+        }
+    }
+}
+
+template <int FMT, int NT>
+cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream) {
+    auto kern = mma_kernel<FMT, NT>;
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), p.smem_bytes);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(32 + kConsumers);
+    cfg.dynamicSmemBytes = p.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = p.pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+}  // namespace kq

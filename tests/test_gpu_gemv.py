@@ -151,20 +151,53 @@ def test_linearity():
 
 
 # ---------------------------------------------------------- multi column
-@pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q4_k", 17, 768)])
-@pytest.mark.parametrize("k", [1, 2, 3, 4, 5, 8])
-def test_multi_matches_single_bitwise_and_oracle(fmt, N, K, k):
-    W = matrix(fmt, 31 + k, N, K)
+@pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q4_k", 17, 768),
+                                     ("q4_k", 4096, 4096), ("q4_k", 33, 14336)])
+@pytest.mark.parametrize("k", [2, 3, 4, 5, 8])
+def test_multi_columns_independent_and_match_oracle(fmt, N, K, k):
+    """Each column of a k-column call equals the same column of an 8-column
+    call bitwise (a column's value never depends on the other columns or
+    on k) and is within the bound of the oracle."""
+    W = matrix(fmt, 31, N, K)
     Wt = dev(W)
-    X = np.stack([x_vec(100 + c, K) for c in range(k)])
+    X = np.stack([x_vec(100 + c, K) for c in range(8)])
     Xt = dev(X)
-    Y = kq.gemv_multi(Wt, fmt, N, K, Xt)
-    for c in range(k):
-        yc = kq.gemv(Wt, fmt, N, K, Xt[c].contiguous())
-        assert torch.equal(Y[c], yc), c
-    y_ref, s_ref = oracle.gemv_multi(fmt, W, N, K, X, nthreads=0)
+    Y8 = kq.gemv_multi(Wt, fmt, N, K, Xt)
+    Y = kq.gemv_multi(Wt, fmt, N, K, Xt[:k].contiguous())
+    assert torch.equal(Y, Y8[:k])
+    y_ref, s_ref = oracle.gemv_multi(fmt, W, N, K, X[:k], nthreads=0)
     for c in range(k):
         assert_close(Y[c], y_ref[c], s_ref[c], f"col {c}")
+
+
+@pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336)])
+def test_single_column_of_multi_call_matches_oracle(fmt, N, K):
+    """k = 1 through gemv_multi is the single-column kernel, bitwise."""
+    W = matrix(fmt, 32, N, K)
+    Wt = dev(W)
+    x = x_vec(150, K)
+    xt = dev(x)
+    Y = kq.gemv_multi(Wt, fmt, N, K, xt[None, :].contiguous())
+    assert torch.equal(Y[0], kq.gemv(Wt, fmt, N, K, xt))
+    y_ref, s_ref = oracle_gemv(fmt, W, N, K, x)
+    assert_close(Y[0], y_ref, s_ref)
+
+
+@pytest.mark.parametrize("scale", [1e-30, 1e-6, 1.0, 3e3, 1e20])
+def test_multi_column_scale_range(scale):
+    """Activations far from 1 in either direction (the kernel rescales each
+    column by a power of two before splitting it into fp16 terms); one
+    column of zeros."""
+    fmt, N, K, k = "q4_k", 48, 4096, 3
+    W = matrix(fmt, 33, N, K)
+    X = np.stack([x_vec(160 + c, K) for c in range(k)]) * np.float32(scale)
+    X[1] = 0.0
+    X = X.astype(np.float32)
+    Y = kq.gemv_multi(dev(W), fmt, N, K, dev(X))
+    y_ref, s_ref = oracle.gemv_multi(fmt, W, N, K, X, nthreads=0)
+    for c in range(k):
+        assert_close(Y[c], y_ref[c], s_ref[c], f"col {c} scale {scale}")
+    assert torch.all(Y[1] == 0)
 
 
 def test_multi_strided_columns():

@@ -1,7 +1,7 @@
 """GPU parity of kq_gemv_splitk: tall-skinny matrices (fewer row pairs than
 SMs) split K across CTAs, write partial sums to a caller workspace and add
 them in a fixed order.  Checked against the oracle; deterministic; column c
-of a multi-column call equals the single-column call bitwise."""
+of a k-column call equals column c of an 8-column call bitwise."""
 import numpy as np
 import pytest
 import torch
@@ -39,15 +39,15 @@ def test_splitk_parity(fmt, N, K):
 
 
 @pytest.mark.parametrize("k", [2, 3, 8])
-def test_splitk_multi_columns_match_single(k):
+def test_splitk_multi_columns_independent(k):
     fmt, N, K = "q4_k", 40, 8192
     W = matrix(fmt, 950, N, K)
-    X = np.stack([x_vec(960 + c, K) for c in range(k)])
+    X = np.stack([x_vec(960 + c, K) for c in range(8)])
     Wt, Xt = dev(W), dev(X)
-    Y = kq.gemv_splitk(Wt, fmt, N, K, Xt)
-    for c in range(k):
-        assert torch.equal(Y[c], kq.gemv_splitk(Wt, fmt, N, K, Xt[c].contiguous())[0]), c
-    y_ref, s_ref = oracle.gemv_multi(fmt, W, N, K, X, nthreads=0)
+    Y8 = kq.gemv_splitk(Wt, fmt, N, K, Xt)
+    Y = kq.gemv_splitk(Wt, fmt, N, K, Xt[:k].contiguous())
+    assert torch.equal(Y, Y8[:k])
+    y_ref, s_ref = oracle.gemv_multi(fmt, W, N, K, X[:k], nthreads=0)
     for c in range(k):
         assert_close(Y[c], y_ref[c], s_ref[c])
 
