@@ -168,15 +168,20 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     DevInfo di;
     cudaError_t err = dev_info(di);
     if (err != cudaSuccess) return cuda_fail(err, "device query");
-    if (fmt != KQ_FMT_Q4_K) return fail(KQ_ERR_UNSUPPORTED, "tensor-core kernel: Q4_K only");
-    const size_t srow = static_cast<size_t>(a.nbs) * kq_block_bytes(fmt);
-    const size_t sp = srow <= 64 ? 64 : round_up(srow - 64, 128) + 64;
+    if (fmt == KQ_FMT_Q6_K && a.nbs % 8 != 0)
+        return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
+    // the staged row plus 4 bytes (Q6_K word loads may read 2 bytes past a
+    // block), rounded up to the residue mod 128 that spreads the 8 rows of
+    // a warp over distinct banks
+    const size_t srow = static_cast<size_t>(a.nbs) * kq_block_bytes(fmt) + 4;
+    const size_t res = fmt == KQ_FMT_Q4_K ? 64 : 16;
+    const size_t sp = srow <= res ? res : round_up(srow - res, 128) + res;
     const size_t stage = round_up(16 * sp, 128);
     const int nc = 4 * nt;
     const size_t head = 256;
     const size_t wp_bytes = sizeof(float) * 2 * kConsumerWarps * 16 * nc;
     const size_t bs_bytes = round_up(sizeof(float) * 2 * nc * a.nbs, 128);
-    const size_t xb_bytes = static_cast<size_t>(a.nbs) * 17 * 32 * nt * 8;
+    const size_t xb_bytes = static_cast<size_t>(a.nbs) * (fmt == KQ_FMT_Q4_K ? 17 : 16) * 32 * nt * 8;
     const size_t fixed = head + wp_bytes + bs_bytes + xb_bytes;
     const size_t limit = static_cast<size_t>(di.smem_optin);
     if (fixed + 2 * stage > limit)
@@ -247,7 +252,7 @@ static cudaError_t dispatch(const GemvArgs& a, const LaunchPlan& p, int fmt, int
 // Calls with 2 or more columns (speculative verify) run on the tensor-core
 // kernel, every column group of the call included, so a column's arithmetic
 // never depends on how the call was grouped.
-static bool use_mma(int fmt, int k) { return k >= 2 && fmt == KQ_FMT_Q4_K; }
+static bool use_mma(int, int k) { return k >= 2; }
 
 static int plan_for(int fmt, int k, bool mma, GemvArgs& a, LaunchPlan& p) {
     if (mma) return plan_mma(fmt, k <= 4 ? 1 : 2, a, p);
@@ -261,7 +266,8 @@ static int run(GemvArgs& a, int fmt, int k, bool mma, cudaStream_t stream) {
     LaunchPlan p;
     int st = plan_for(fmt, k, mma, a, p);
     if (st != KQ_OK) return st;
-    if (mma) err = k <= 4 ? launch_mma<1, 1>(a, p, stream) : launch_mma<1, 2>(a, p, stream);
+    if (mma && fmt == KQ_FMT_Q4_K) err = k <= 4 ? launch_mma<1, 1>(a, p, stream) : launch_mma<1, 2>(a, p, stream);
+    else if (mma) err = k <= 4 ? launch_mma<2, 1>(a, p, stream) : launch_mma<2, 2>(a, p, stream);
     else err = dispatch(a, p, fmt, padded_cols(k), stream);
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
     if (a.ksplit > 1) {

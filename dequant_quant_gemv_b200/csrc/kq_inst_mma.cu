@@ -5,4 +5,6 @@
 namespace kq {
 template cudaError_t launch_mma<1, 1>(const GemvArgs&, const LaunchPlan&, cudaStream_t);
 template cudaError_t launch_mma<1, 2>(const GemvArgs&, const LaunchPlan&, cudaStream_t);
+template cudaError_t launch_mma<2, 1>(const GemvArgs&, const LaunchPlan&, cudaStream_t);
+template cudaError_t launch_mma<2, 2>(const GemvArgs&, const LaunchPlan&, cudaStream_t);
 }  // namespace kq

@@ -23,8 +23,9 @@
 //
 // Schedule.  The persistent CTA and its TMA ring are those of gemv_kernel;
 // a stage is 16 rows (one m16 tile), copied row by row into smem rows
-// `a.sp` bytes apart (a.sp = 64 mod 128 keeps the fragment loads free of
-// bank conflicts).  The 8 consumer warps split the stage's super-blocks
+// `a.sp` bytes apart (a.sp = 64 mod 128 for the 16-byte loads of Q4_K and
+// 16 mod 128 for the 4-byte loads of Q6_K keep them free of bank
+// conflicts).  The 8 consumer warps split the stage's super-blocks
 // (warp w takes blocks w, w+8, ...) and add their partial sums in a fixed
 // order, so results are deterministic and each column's value does not
 // depend on the other columns.
@@ -37,7 +38,9 @@
 namespace kq {
 
 constexpr int kMmaRowPairs = 8;  // 16 rows per stage
-constexpr int kMmaSteps = 17;    // K-steps per super-block: 16 of quants + 1 of mins
+// K-steps per super-block: 16 of quants, plus one of mins for Q4_K
+template <int FMT>
+__host__ __device__ constexpr int mma_steps() { return FMT == 1 ? 17 : 16; }
 
 // D += A * B for one m16n8k16 tile (row-major A, column-major B).
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -63,6 +66,8 @@ __device__ __forceinline__ uint32_t hadd2u(uint32_t a, uint32_t b) {
     asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
+__device__ __forceinline__ __half2 u2h2(uint32_t v) { return *reinterpret_cast<const __half2*>(&v); }
+__device__ __forceinline__ uint32_t h22u(__half2 v) { return *reinterpret_cast<const uint32_t*>(&v); }
 __device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
     return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
 }
@@ -104,34 +109,53 @@ __device__ __forceinline__ int col_shift(uint32_t amax_bits) {
 }
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
 
-// B-fragment store of one column's 4 consecutive activations of super-block
-// `bl` (relative), K position `w` (multiple of 4) within it.  Weight w of a
-// Q4_K block is quant byte beta = 32*(w/64) + w%32, low nibble for
-// (w/32) even, high nibble otherwise; byte beta sits in 16-byte chunk
-// beta/16, word (beta/4)%4.  A thread whose lane has q = chunk%4 feeds
-// that word to K-step pair j = 4*(chunk/4) + word, step 2j (low nibbles) or
-// 2j+1 (high); its K positions 2q, 2q+1 hold bytes 0 and 2 of the word and
-// 2q+8, 2q+9 bytes 1 and 3.  The column occupies B columns 2c' (hi term)
-// and 2c'+1 (lo term) of n-tile col/4, c' = col%4, i.e. lanes with
-// g = 2c' and 2c'+1.
-template <int NT>
-__device__ __forceinline__ void q4k_store_b(uint32_t xb, int bl, int w, int col, float4 v) {
-    const int hi = (w >> 5) & 1;
-    const int beta = 32 * (w >> 6) + (w & 31);
-    const int ch = beta >> 4, u = (beta >> 2) & 3;
-    const int q = ch & 3, j = ((ch >> 2) << 2) | u, s = 2 * j + hi;
+// B-fragment entry of K-step s for this column's hi and lo terms: the
+// column occupies B columns 2c' (hi) and 2c'+1 (lo) of n-tile col/4,
+// c' = col%4, i.e. lanes g = 2c' and 2c'+1 (lane = 4g + q).  reg0 holds
+// the K positions 2q, 2q+1 and reg1 2q+8, 2q+9: activations 0, 2 and 1, 3
+// of the group of four that feeds the quant word at those positions.
+template <int FMT, int NT>
+__device__ __forceinline__ void store_b_entry(uint32_t xb, int bl, int s, int q, int col, float4 v) {
     const int nt = col >> 2, gh = 2 * (col & 3);
     const __half h0 = __float2half_rn(v.x), h1 = __float2half_rn(v.y), h2 = __float2half_rn(v.z),
                  h3 = __float2half_rn(v.w);
     const __half l0 = __float2half_rn(v.x - __half2float(h0)), l1 = __float2half_rn(v.y - __half2float(h1)),
                  l2 = __float2half_rn(v.z - __half2float(h2)), l3 = __float2half_rn(v.w - __half2float(h3));
-    const uint32_t step = xb + 8u * static_cast<uint32_t>(((bl * kMmaSteps + s) * 32) * NT + nt);
+    const uint32_t step = xb + 8u * static_cast<uint32_t>(((bl * mma_steps<FMT>() + s) * 32) * NT + nt);
     st_s64u(step + 8u * NT * (4 * gh + q), pack_h2(h0, h2), pack_h2(h1, h3));
     st_s64u(step + 8u * NT * (4 * (gh + 1) + q), pack_h2(l0, l2), pack_h2(l1, l3));
 }
 
+// Where 4 consecutive activations w..w+3 (w a multiple of 4) of a block go:
+// the K-step s and lane q whose quant word holds weights w..w+3.
+//
+// Q4_K: weight w is quant byte beta = 32*(w/64) + w%32, low nibble for
+// (w/32) even, high otherwise; byte beta is word (beta/4)%4 of 16-byte
+// chunk beta/16.  Lane q reads chunks q and q+4; word u of chunk q+4c feeds
+// K-step pair j = 4c + u: step 2j (low nibbles) or 2j+1 (high).
+//
+// Q6_K: weight w = 128n + 32t + l takes its low bits from ql[64n + l +
+// 32(t%2)] (nibble t/2) and its top bits from bits 2t of qh[32n + l].  Lane
+// q reads the 4-byte groups lg = q and q+4 of each half n, l = 4lg..4lg+3;
+// group (n, lg) is combination c = 2n + lg/4, and the quants of quarter t
+// feed K-step s = 4c + t.
+template <int FMT>
+__device__ __forceinline__ void b_slot(int w, int& s, int& q) {
+    if constexpr (FMT == 1) {
+        const int hi = (w >> 5) & 1;
+        const int beta = 32 * (w >> 6) + (w & 31);
+        const int ch = beta >> 4, u = (beta >> 2) & 3;
+        q = ch & 3;
+        s = 2 * (((ch >> 2) << 2) | u) + hi;
+    } else {
+        const int n = w >> 7, t = (w >> 5) & 3, lg = (w & 31) >> 2;
+        q = lg & 3;
+        s = 4 * (2 * n + (lg >> 2)) + t;
+    }
+}
+
 // Stage the activations of the K range [256*kb0, 256*(kb0+nbl)) as
-// B fragments (see q4k_store_b) plus, per block, the min step: lane (g, q)
+// B fragments (see b_slot) plus, for Q4_K, per block the min step: lane (g, q)
 // holds (X_2q, X_2q+1) of its column's hi or lo term and zeros for K
 // positions 8..15, X_j being the sub-block sum of 32 activations.  Each
 // (column, block) is scaled by its own power of two 2^sh (largest |x| of
@@ -139,9 +163,9 @@ __device__ __forceinline__ void q4k_store_b(uint32_t xb, int bl, int w, int col,
 // (2^-sh, 2^(5-sh)) per block and column.  Columns >= ncol_real are zero.
 // One warp per (column, block) item, two float4 per lane, several items'
 // loads in flight.
-template <int NT>
-__device__ void stage_xb_q4k(const GemvArgs& a, uint32_t xb, float* bscale, int cw, int lane, int bar, int kb0,
-                             int nbl) {
+template <int FMT, int NT>
+__device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, int lane, int bar, int kb0,
+                         int nbl) {
     constexpr int NC = 4 * NT;
     constexpr int U = 4;  // items per warp in flight
     const float* xg = a.x + static_cast<int64_t>(kb0) * 256;
@@ -181,7 +205,10 @@ __device__ void stage_xb_q4k(const GemvArgs& a, uint32_t xb, float* bscale, int 
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const float4 t = make_float4(v[u][h].x * sc, v[u][h].y * sc, v[u][h].z * sc, v[u][h].w * sc);
-                q4k_store_b<NT>(xb, bl, 128 * h + 4 * lane, col, t);
+                int st, sq;
+                b_slot<FMT>(128 * h + 4 * lane, st, sq);
+                store_b_entry<FMT, NT>(xb, bl, st, sq, col, t);
+                if constexpr (FMT != 1) continue;
                 // sub-block 4h + lane/8: the 8 lanes of this group, fixed order
                 float X = (v[u][h].x + v[u][h].y) + (v[u][h].z + v[u][h].w);
                 X += __shfl_xor_sync(0xffffffffu, X, 1);
@@ -193,7 +220,8 @@ __device__ void stage_xb_q4k(const GemvArgs& a, uint32_t xb, float* bscale, int 
                     const __half xh = __float2half_rn(X);
                     const __half xl = __float2half_rn(X - __half2float(xh));
                     const int nt = col >> 2, gh = 2 * (col & 3), q = j >> 1;
-                    const uint32_t step = xb + 8u * static_cast<uint32_t>(((bl * kMmaSteps + 16) * 32) * NT + nt);
+                    const uint32_t step =
+                        xb + 8u * static_cast<uint32_t>(((bl * mma_steps<FMT>() + 16) * 32) * NT + nt);
                     const uint32_t eh = step + 8u * NT * (4 * gh + q), el = step + 8u * NT * (4 * (gh + 1) + q);
                     st_s16u(eh + 2 * (j & 1), __half_as_ushort(xh));
                     st_s16u(el + 2 * (j & 1), __half_as_ushort(xl));
@@ -239,12 +267,12 @@ __device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, 
         q4k_half_scales(h.y, h.z, h.w, 1, sc1, m1);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            const uint32_t S = byte_pair_h2(c ? sc1 : sc0, sel);
-            const uint32_t slo = __byte_perm(S, 0u, 0x1010u), shi = __byte_perm(S, 0u, 0x3232u);
-            mlo[r][c] = slo;
-            alo[r][c] = hmul2u(slo, kH2_m1024);
-            mhi[r][c] = hmul2u(shi, kH2_1_16);
-            ahi[r][c] = hmul2u(shi, kH2_m64);
+            const __half2 S = u2h2(byte_pair_h2(c ? sc1 : sc0, sel));
+            const __half2 slo = __low2half2(S), shi = __high2half2(S);
+            mlo[r][c] = h22u(slo);
+            alo[r][c] = h22u(__hmul2(slo, u2h2(kH2_m1024)));
+            mhi[r][c] = h22u(__hmul2(shi, u2h2(kH2_1_16)));
+            ahi[r][c] = h22u(__hmul2(shi, u2h2(kH2_m64)));
         }
         mins[r] = byte_pair_h2(q < 2 ? m0 : m1, msel);
     }
@@ -266,7 +294,7 @@ __device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, 
             H02[r] = hfma2u((x & 0x00F000F0u) | kH2_1024, mhi[r][c], ahi[r][c]);
             H13[r] = hfma2u((xs & 0x00F000F0u) | kH2_1024, mhi[r][c], ahi[r][c]);
         }
-        const uint32_t s_lo = xbl + 8u * NT * 32 * (2 * j), s_hi = s_lo + 8u * NT * 32;
+        const uint32_t s_lo = xbl + 8u * NT * 32 * (2 * j), s_hi = s_lo + 8u * NT * 32;  // steps 2j, 2j+1
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
             const uint2 bl = ld_s64u(s_lo + 8 * n), bh = ld_s64u(s_hi + 8 * n);
@@ -293,6 +321,86 @@ __device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, 
         ys[1][n] = fmaf(d1 * f.x, acc[n][2] + acc[n][3], ys[1][n]);
         ym[0][n] = fmaf(m0 * f.y, accm[n][0] + accm[n][1], ym[0][n]);
         ym[1][n] = fmaf(m1 * f.y, accm[n][2] + accm[n][3], ym[1][n]);
+    }
+}
+
+// Q6_K: rows g and g+8, super-block b (starting 2 bytes past a 4-byte
+// boundary when ODD, i.e. b odd), this lane's quant groups (see b_slot).
+// A = sc*(q-32): q in the mantissa of 1024 by byte permute, minus 1056,
+// times the group's int8 scale (exact while |sc| <= 64; otherwise rounded
+// to fp16, within 2^-11 of that weight).  Adds 2^-sh * d * S into ys.
+template <int NT, bool ODD>
+__device__ __forceinline__ void q6k_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t bsc, int q,
+                                              float (&ys)[2][NT]) {
+    uint32_t A[2][4], B[2][4], H[2][4];
+    __half2 S[2][4][2];  // [row][combination][t/2]: scales of quarters (t even, t odd)
+    float dsc[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint32_t bw = (r ? rg8 : rg) + static_cast<uint32_t>(b) * kQ6Bytes - (ODD ? 2u : 0u);
+        auto ldw = [&](int i) -> uint32_t {
+            if constexpr (ODD) return __byte_perm(ld_s32(bw + 4 * i), ld_s32(bw + 4 * i + 4), 0x5432);
+            else return ld_s32(bw + 4 * i);
+        };
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int n = c >> 1, lg = q + 4 * (c & 1);
+            A[r][c] = ldw(16 * n + lg);
+            B[r][c] = ldw(16 * n + 8 + lg);
+            H[r][c] = ldw(32 + 8 * n + lg);
+        }
+        // int8 scale s as fp16: byte s^0x80 = s+128 in the mantissa of 1024,
+        // minus 1152.  Combination c uses scales 8n + c%2 + 2t (t = 0..3):
+        // bytes c%2 and c%2+2 of scale words 2n and 2n+1.
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+            const uint32_t w0 = ldw(48 + 2 * n) ^ 0x80808080u, w1 = ldw(49 + 2 * n) ^ 0x80808080u;
+#pragma unroll
+            for (int h4 = 0; h4 < 2; ++h4) {
+                const uint32_t sel = 0x4040u | static_cast<uint32_t>(h4) | (static_cast<uint32_t>(h4 + 2) << 8);
+                S[r][2 * n + h4][0] = __hadd2(u2h2(__byte_perm(w0, 0x64646464u, sel)), u2h2(0xE480E480u));
+                S[r][2 * n + h4][1] = __hadd2(u2h2(__byte_perm(w1, 0x64646464u, sel)), u2h2(0xE480E480u));
+            }
+        }
+        const uint32_t dword = ODD ? (ld_s32(bw + 208) >> 16) : ld_s32(bw + 208);
+        dsc[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(dword & 0xFFFFu)));
+    }
+    const __half2 m1056 = u2h2(0xE420E420u);  // (-1056, -1056)
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            uint32_t lo[2], hi[2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t src = (t & 1) ? B[r][c] : A[r][c];
+                const uint32_t low4 = (t & 2) ? ((src >> 4) & 0x0F0F0F0Fu) : (src & 0x0F0F0F0Fu);
+                const uint32_t top2 = (t == 0 ? (H[r][c] << 4) : t == 1 ? (H[r][c] << 2) : t == 2 ? H[r][c]
+                                                                                                : (H[r][c] >> 2)) &
+                                      0x30303030u;
+                const uint32_t qw = low4 | top2;
+                const __half2 sc = (t & 1) ? __high2half2(S[r][c][t >> 1]) : __low2half2(S[r][c][t >> 1]);
+                lo[r] = h22u(__hmul2(__hadd2(u2h2(__byte_perm(qw, 0x64646464u, 0x4240u)), m1056), sc));
+                hi[r] = h22u(__hmul2(__hadd2(u2h2(__byte_perm(qw, 0x64646464u, 0x4341u)), m1056), sc));
+            }
+            const uint32_t sp = xbl + 8u * NT * 32 * (4 * c + t);
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const uint2 bv = ld_s64u(sp + 8 * n);
+                mma16816(acc[n], lo[0], lo[1], hi[0], hi[1], bv.x, bv.y);
+            }
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const float f = ld_s32f(bsc + 8u * (4 * n + q));  // 2^-sh of column 4n+q
+        ys[0][n] = fmaf(dsc[0] * f, acc[n][0] + acc[n][1], ys[0][n]);
+        ys[1][n] = fmaf(dsc[1] * f, acc[n][2] + acc[n][3], ys[1][n]);
     }
 }
 
@@ -345,7 +453,7 @@ __global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_co
     const uint32_t sbuf_s = smem_u32(sbuf);
     pdl_wait();
     pdl_launch_dependents();
-    stage_xb_q4k<NT>(a, xb_s, bscale, cw, lane, 1, kb0, nbl);
+    stage_xb<FMT, NT>(a, xb_s, bscale, cw, lane, 1, kb0, nbl);
 
     // byte selectors: scales of chunk q (half 0) / q+4 (half 1) sit at bytes
     // 2*(q/2), 2*(q/2)+1 of either half; mins 2q, 2q+1 at bytes 2*(q%2), +1
@@ -369,9 +477,12 @@ __global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_co
         if (!*abort_flag) {
             const uint32_t rg = sbuf_s + slot * a.stage_bytes + g * a.sp;
             const uint32_t rg8 = rg + 8 * a.sp;
-            for (int b = cw; b < nbl; b += kConsumerWarps)
-                q4k_mma_block<NT>(rg, rg8, b, xlane + 8u * NT * 32 * kMmaSteps * b, bsc_s + 8u * NC * b, sel,
-                                  msel, q, ys, ym);
+            for (int b = cw; b < nbl; b += kConsumerWarps) {
+                const uint32_t xbl = xlane + 8u * NT * 32 * mma_steps<FMT>() * b, bsc = bsc_s + 8u * NC * b;
+                if constexpr (FMT == 1) q4k_mma_block<NT>(rg, rg8, b, xbl, bsc, sel, msel, q, ys, ym);
+                else if (b & 1) q6k_mma_block<NT, true>(rg, rg8, b, xbl, bsc, q, ys);
+                else q6k_mma_block<NT, false>(rg, rg8, b, xbl, bsc, q, ys);
+            }
         }
         const uint32_t wb = wp_s + 4u * ((own & 1) * (kConsumerWarps * 16 * NC));
         ++own;

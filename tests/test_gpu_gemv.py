@@ -152,7 +152,8 @@ def test_linearity():
 
 # ---------------------------------------------------------- multi column
 @pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q4_k", 17, 768),
-                                     ("q4_k", 4096, 4096), ("q4_k", 33, 14336)])
+                                     ("q4_k", 4096, 4096), ("q4_k", 33, 14336), ("q6_k", 64, 4096),
+                                     ("q6_k", 41, 2048), ("q6_k", 4096, 2048)])
 @pytest.mark.parametrize("k", [2, 3, 4, 5, 8])
 def test_multi_columns_independent_and_match_oracle(fmt, N, K, k):
     """Each column of a k-column call equals the same column of an 8-column
@@ -183,12 +184,13 @@ def test_single_column_of_multi_call_matches_oracle(fmt, N, K):
     assert_close(Y[0], y_ref, s_ref)
 
 
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
 @pytest.mark.parametrize("scale", [1e-30, 1e-6, 1.0, 3e3, 1e20])
-def test_multi_column_scale_range(scale):
+def test_multi_column_scale_range(fmt, scale):
     """Activations far from 1 in either direction (the kernel rescales each
-    column by a power of two before splitting it into fp16 terms); one
-    column of zeros."""
-    fmt, N, K, k = "q4_k", 48, 4096, 3
+    column and super-block by a power of two before splitting it into fp16
+    terms); one column of zeros."""
+    N, K, k = 48, 4096, 3
     W = matrix(fmt, 33, N, K)
     X = np.stack([x_vec(160 + c, K) for c in range(k)]) * np.float32(scale)
     X[1] = 0.0
