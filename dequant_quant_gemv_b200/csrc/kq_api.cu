@@ -155,60 +155,154 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     a.xs_offset = static_cast<int>(head + wp_bytes);
     a.sbuf_offset = static_cast<int>(fixed);
     p.grid = static_cast<int>(grid);
+    p.cluster = 1;
     p.ng = ng;
     p.smem_bytes = fixed + ns * stage;
     p.pdl = true;
     return KQ_OK;
 }
 
+// Shared-memory layout of the tensor-core kernel for K ranges of `nbs`
+// blocks split over `S` CTAs of a cluster (S = 1: no cluster).
+struct MmaLayout {
+    size_t sp, stage, wp, bs, red, xb, fixed;
+};
+static MmaLayout mma_layout(int fmt, int nt, int nbs, int S) {
+    MmaLayout L;
+    // the staged row (which may start up to 14 bytes into the smem row) plus
+    // 4 bytes (Q6_K word loads may read 2 bytes past a block), rounded up to
+    // the residue mod 128 that spreads the 8 rows of a warp over distinct
+    // banks
+    const size_t srow = static_cast<size_t>(nbs) * kq_block_bytes(fmt) + 16 + 4;
+    const size_t res = fmt == KQ_FMT_Q4_K ? 64 : 16;
+    L.sp = srow <= res ? res : round_up(srow - res, 128) + res;
+    L.stage = round_up(16 * L.sp, 128);
+    const size_t nc = 4 * static_cast<size_t>(nt);
+    L.wp = sizeof(float) * 2 * kConsumerWarps * 16 * nc;
+    L.bs = round_up(sizeof(float) * 2 * nc * nbs, 128);
+    L.red = S > 1 ? sizeof(float) * 2 * (S - 1) * 16 * nc : 0;
+    L.xb = static_cast<size_t>(nbs) * (fmt == KQ_FMT_Q4_K ? 17 : 16) * 32 * nt * 8;
+    L.fixed = 256 + L.wp + L.bs + L.red + L.xb;
+    return L;
+}
+
+static cudaError_t active_clusters(int fmt, int nt, int S, size_t smem, int* out) {
+    struct Entry {
+        int dev, fmt, nt, S;
+        size_t smem;
+        int n;
+    };
+    static std::mutex mu;
+    static Entry cache[64];
+    static int count = 0;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (int i = 0; i < count; ++i)
+            if (cache[i].dev == dev && cache[i].fmt == fmt && cache[i].nt == nt && cache[i].S == S &&
+                cache[i].smem == smem) {
+                *out = cache[i].n;
+                return cudaSuccess;
+            }
+    }
+    if (fmt == KQ_FMT_Q4_K) err = nt == 1 ? mma_active_clusters<1, 1>(S, smem, out) : mma_active_clusters<1, 2>(S, smem, out);
+    else err = nt == 1 ? mma_active_clusters<2, 1>(S, smem, out) : mma_active_clusters<2, 2>(S, smem, out);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lk(mu);
+    if (count < 64) cache[count++] = Entry{dev, fmt, nt, S, smem, *out};
+    return cudaSuccess;
+}
+
 // Schedule of the tensor-core kernel (2..8 columns): 16-row stages, rows
-// `sp` bytes apart in smem (sp >= the staged row, sp = 64 mod 128), B
-// fragments of the CTA's K range for NT n-tiles, two partial-sum buffers.
+// `sp` bytes apart in smem, B fragments of the CTA's K range for NT
+// n-tiles, two partial-sum buffers.  Unless the caller split K itself
+// (a.ksplit > 1, partial sums in its workspace), K is split into S equal
+// ranges over the CTAs of a cluster when the activations of 8 columns and
+// two stages do not fit otherwise: the smallest S (<= 8, dividing the
+// blocks) that fits and whose clusters still occupy 85% of the SMs, else
+// the fitting S that occupies the most.  The split depends on (format, K)
+// only, so every column count sums alike and a column's result does not
+// depend on how many columns share the call.
 int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     DevInfo di;
     cudaError_t err = dev_info(di);
     if (err != cudaSuccess) return cuda_fail(err, "device query");
-    if (fmt == KQ_FMT_Q6_K && a.nbs % 8 != 0)
+    if (fmt == KQ_FMT_Q6_K && a.nb % 8 != 0)
         return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
-    // the staged row plus 4 bytes (Q6_K word loads may read 2 bytes past a
-    // block), rounded up to the residue mod 128 that spreads the 8 rows of
-    // a warp over distinct banks
-    const size_t srow = static_cast<size_t>(a.nbs) * kq_block_bytes(fmt) + 4;
-    const size_t res = fmt == KQ_FMT_Q4_K ? 64 : 16;
-    const size_t sp = srow <= res ? res : round_up(srow - res, 128) + res;
-    const size_t stage = round_up(16 * sp, 128);
-    const int nc = 4 * nt;
-    const size_t head = 256;
-    const size_t wp_bytes = sizeof(float) * 2 * kConsumerWarps * 16 * nc;
-    const size_t bs_bytes = round_up(sizeof(float) * 2 * nc * a.nbs, 128);
-    const size_t xb_bytes = static_cast<size_t>(a.nbs) * (fmt == KQ_FMT_Q4_K ? 17 : 16) * 32 * nt * 8;
-    const size_t fixed = head + wp_bytes + bs_bytes + xb_bytes;
     const size_t limit = static_cast<size_t>(di.smem_optin);
-    if (fixed + 2 * stage > limit)
+    int S = a.ksplit, nbs = a.nbs;
+    bool cl = false;
+    if (S == 1) {
+        int best = 0, best_use = 0;
+        for (int s = 1; s <= 8 && s <= a.nb; ++s) {
+            if (a.nb % s != 0) continue;
+            const MmaLayout L8 = mma_layout(fmt, 2, a.nb / s, s);
+            if (L8.fixed + 2 * L8.stage > limit) continue;
+            int use = di.sm_count;
+            if (s > 1) {
+                const MmaLayout Ln = mma_layout(fmt, nt, a.nb / s, s);
+                size_t nsn = (limit - Ln.fixed) / Ln.stage;
+                if (nsn > kMaxStages) nsn = kMaxStages;
+                int fit = 0;
+                err = active_clusters(fmt, nt, s, Ln.fixed + nsn * Ln.stage, &fit);
+                if (err != cudaSuccess) return cuda_fail(err, "cluster occupancy query");
+                use = fit * s;
+            }
+            if (use > best_use) {
+                best = s;
+                best_use = use;
+            }
+            if (20 * use >= 17 * di.sm_count) {
+                best = s;
+                break;
+            }
+        }
+        if (best > 1) {
+            S = best;
+            nbs = a.nb / best;
+            cl = true;
+        }
+    }
+    const MmaLayout L = mma_layout(fmt, nt, nbs, S);
+    if (L.fixed + 2 * L.stage > limit)
         return fail(KQ_ERR_UNSUPPORTED, "K=%lld with %d columns needs %zu bytes of shared memory (limit %zu)",
-                    (long long)a.K, nc, fixed + 2 * stage, limit);
-    size_t ns = (limit - fixed) / stage;
+                    (long long)a.K, 4 * nt, L.fixed + 2 * L.stage, limit);
+    size_t ns = (limit - L.fixed) / L.stage;
     if (ns > kMaxStages) ns = kMaxStages;
     const int64_t rps = (a.N + 1) / 2;
-    const int64_t tiles = (rps + 7) / 8;                  // 16-row stages of the matrix
-    const int64_t ranges = di.sm_count / a.ksplit;
-    const int64_t grid = (tiles < ranges ? tiles : ranges) * a.ksplit;
-    const int64_t per_cta = (rps + grid / a.ksplit - 1) / (grid / a.ksplit);
+    const int64_t tiles = (rps + 7) / 8;  // 16-row stages of the matrix
+    int64_t ranges = di.sm_count / S;     // row ranges (clusters, or CTAs per K range)
+    if (cl) {
+        int fit = 0;
+        err = active_clusters(fmt, nt, S, L.fixed + ns * L.stage, &fit);
+        if (err != cudaSuccess) return cuda_fail(err, "cluster occupancy query");
+        if (fit < 1) return fail(KQ_ERR_UNSUPPORTED, "no cluster of %d CTAs fits", S);
+        ranges = fit;
+    }
+    const int64_t grid = (tiles < ranges ? tiles : ranges) * S;
+    const int64_t per_cta = (rps + grid / S - 1) / (grid / S);
     const int64_t need = (per_cta + 7) / 8 + 1;
     if (static_cast<int64_t>(ns) > need) ns = need < 2 ? 2 : static_cast<size_t>(need);
+    a.ksplit = S;
+    a.nbs = nbs;
+    a.cluster = cl ? 1 : 0;
     a.ps = 8;
     a.parts = 1;
     a.lanes_per_rp = 0;
-    a.sp = static_cast<int>(sp);
+    a.sp = static_cast<int>(L.sp);
     a.nstage = static_cast<int>(ns);
-    a.stage_bytes = static_cast<int>(stage);
-    a.wp_offset = static_cast<int>(head);
-    a.xscale_offset = static_cast<int>(head + wp_bytes);
-    a.xs_offset = static_cast<int>(head + wp_bytes + bs_bytes);
-    a.sbuf_offset = static_cast<int>(fixed);
+    a.stage_bytes = static_cast<int>(L.stage);
+    a.wp_offset = 256;
+    a.xscale_offset = static_cast<int>(256 + L.wp);
+    a.red_offset = static_cast<int>(256 + L.wp + L.bs);
+    a.xs_offset = static_cast<int>(256 + L.wp + L.bs + L.red);
+    a.sbuf_offset = static_cast<int>(L.fixed);
     p.grid = static_cast<int>(grid);
+    p.cluster = cl ? S : 1;
     p.ng = 1;
-    p.smem_bytes = fixed + ns * stage;
+    p.smem_bytes = L.fixed + ns * L.stage;
     p.pdl = true;
     return KQ_OK;
 }
@@ -270,7 +364,7 @@ static int run(GemvArgs& a, int fmt, int k, bool mma, cudaStream_t stream) {
     else if (mma) err = k <= 4 ? launch_mma<2, 1>(a, p, stream) : launch_mma<2, 2>(a, p, stream);
     else err = dispatch(a, p, fmt, padded_cols(k), stream);
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
-    if (a.ksplit > 1) {
+    if (a.ksplit > 1 && !a.cluster) {  // cluster splits add their partial sums in the kernel
         err = launch_splitk_combine(a.partial, a.ksplit, k, a.N, a.y, a.ldy, stream);
         if (err != cudaSuccess) return cuda_fail(err, "split-K combine launch");
     }

@@ -330,7 +330,10 @@ __device__ __forceinline__ void raise_fault(const GemvArgs& a, volatile int* abo
 // into its ring slot with 1-D bulk copies (no multicast), waiting for the
 // consumers to release a slot before reusing it.  `contiguous`: whole rows
 // stored back to back (one copy per stage); otherwise each row's K range
-// [kb0, kb0 + nbl) blocks is copied to its own smem row `srow` bytes apart.
+// [kb0, kb0 + nbl) blocks is copied to its own smem row `srow` bytes apart,
+// from the 16-byte boundary at or below the range start (bulk copies move
+// whole 16-byte units), so the range begins (kb0 * BS) % 16 bytes into the
+// smem row.  Rows are multiples of 16 bytes, so no copy leaves its row.
 template <int BS>
 __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empty, volatile int* abort_flag,
                                uint8_t* sbuf, int64_t rp_begin, int64_t rp_end, int64_t rps, int ns, int kb0,
@@ -357,11 +360,12 @@ __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empt
                 mbar_arrive_expect_tx(&full[slot], bytes);
                 bulk_g2s(dst, src, bytes, &full[slot]);
             } else {
-                const uint32_t rbytes = static_cast<uint32_t>(nbl * BS);
+                const int64_t off = static_cast<int64_t>(kb0) * BS;
+                const int64_t off16 = off & ~int64_t(15);
+                const uint32_t rbytes = static_cast<uint32_t>((off + nbl * BS - off16 + 15) & ~int64_t(15));
                 mbar_arrive_expect_tx(&full[slot], rbytes * st.nrows);
                 for (int i = 0; i < st.nrows; ++i)
-                    bulk_g2s(dst + i * srow, src + i * a.row_bytes + static_cast<int64_t>(kb0) * BS, rbytes,
-                             &full[slot]);
+                    bulk_g2s(dst + i * srow, src + i * a.row_bytes + off16, rbytes, &full[slot]);
             }
         } else {
             mbar_arrive(&full[slot]);

@@ -7,4 +7,8 @@ template cudaError_t launch_mma<1, 1>(const GemvArgs&, const LaunchPlan&, cudaSt
 template cudaError_t launch_mma<1, 2>(const GemvArgs&, const LaunchPlan&, cudaStream_t);
 template cudaError_t launch_mma<2, 1>(const GemvArgs&, const LaunchPlan&, cudaStream_t);
 template cudaError_t launch_mma<2, 2>(const GemvArgs&, const LaunchPlan&, cudaStream_t);
+template cudaError_t mma_active_clusters<1, 1>(int, size_t, int*);
+template cudaError_t mma_active_clusters<1, 2>(int, size_t, int*);
+template cudaError_t mma_active_clusters<2, 1>(int, size_t, int*);
+template cudaError_t mma_active_clusters<2, 2>(int, size_t, int*);
 }  // namespace kq

@@ -43,10 +43,13 @@ struct GemvArgs {
     // tensor-core (multi-column) kernel only
     int sp;                  // smem bytes between staged rows (padded)
     int xscale_offset;       // power-of-two scales per super-block and column
+    int cluster;             // 1: the ksplit K ranges are the CTAs of a cluster, reduced in shared memory
+    int red_offset;          // cluster reduction buffers (rank 0)
 };
 
 struct LaunchPlan {
     int grid;
+    int cluster;     // CTAs per cluster (1: no cluster launch)
     int ng;          // consumer groups of 8 warps (1 or 2)
     size_t smem_bytes;
     bool pdl;
@@ -61,6 +64,8 @@ cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stre
 int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p);
 template <int FMT, int NT>
 cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
+template <int FMT, int NT>
+cudaError_t mma_active_clusters(int cluster, size_t smem_bytes, int* out);
 cudaError_t fault_word(int** out);
 cudaError_t launch_splitk_combine(const float* partial, int S, int ncol, int64_t N, float* y, int64_t ldy,
                                   cudaStream_t stream);

@@ -325,7 +325,7 @@ __device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, 
 }
 
 // Q6_K: rows g and g+8, super-block b (starting 2 bytes past a 4-byte
-// boundary when ODD, i.e. b odd), this lane's quant groups (see b_slot).
+// boundary when ODD), this lane's quant groups (see b_slot).
 // A = sc*(q-32): q in the mantissa of 1024 by byte permute, minus 1056,
 // times the group's int8 scale (exact while |sc| <= 64; otherwise rounded
 // to fp16, within 2^-11 of that weight).  Adds 2^-sh * d * S into ys.
@@ -406,104 +406,153 @@ __device__ __forceinline__ void q6k_mma_block(uint32_t rg, uint32_t rg8, int b, 
 
 // ------------------------------------------------------------ the kernel
 
+// Split K inside a cluster (a.cluster): the ksplit CTAs of a cluster share
+// one row range, CTA r covering K range r (and staging only that range's
+// activations).  Each stage's partial sums of CTAs 1..S-1 go into rank 0's
+// shared memory (two buffers, by stage parity) with a remote arrive per
+// value on rank 0's `recv` barrier; rank 0 adds them in rank order, writes
+// y and releases the buffer to each sender through its `sent` barrier
+// (skipped for the last two stages, which no sender waits for).  A cluster
+// barrier at the start (barriers initialised) and at the end (no CTA leaves
+// while another may still address its shared memory) brackets it all.
 template <int FMT, int NT>
 __global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_constant__ GemvArgs a) {
     constexpr int NC = 4 * NT;
+    constexpr int NRED = 16 * NC;  // values of one stage's partial sums
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 2 * kMaxStages * 8);
+    uint64_t* recv = reinterpret_cast<uint64_t*>(smem + 2 * kMaxStages * 8 + 8);  // [2], rank 0
+    uint64_t* sent = recv + 2;                                                    // [2], ranks > 0
     float* bscale = reinterpret_cast<float*>(smem + a.xscale_offset);  // [block][column] (2^-sh, 2^(5-sh))
     uint8_t* sbuf = smem + a.sbuf_offset;
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int ns = a.nstage;
+    const int S = a.ksplit;
+    const bool cl = a.cluster != 0;
     if (tid == 0) {
         for (int s = 0; s < ns; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kConsumerWarps);
         }
+        if (cl)
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(&recv[i], static_cast<uint32_t>((S - 1) * NRED));
+                mbar_init(&sent[i], 1);
+            }
         *abort_flag = 0;
         fence_barrier_init();
     }
     __syncthreads();
+    if (cl) cluster_sync();
 
     const int64_t rps = (a.N + 1) / 2;
-    const int ks = static_cast<int>(blockIdx.x) % a.ksplit;
-    const int64_t rc = blockIdx.x / a.ksplit, G = gridDim.x / a.ksplit;
+    const int ks = static_cast<int>(blockIdx.x) % S;  // = the rank within the cluster
+    const int64_t rc = blockIdx.x / S, G = gridDim.x / S;
     const int64_t rp_begin = rps * rc / G;
     const int64_t rp_end = rps * (rc + 1) / G;
+    const int total = static_cast<int>((rp_end - rp_begin + kMmaRowPairs - 1) / kMmaRowPairs);
     constexpr int BS = FMT == 1 ? kQ4Bytes : kQ6Bytes;
     const int kb0 = ks * a.nbs;
     const int nbl = a.nb - kb0 < a.nbs ? a.nb - kb0 : a.nbs;
+    const uint32_t rem = static_cast<uint32_t>(kb0 * BS) & 15u;  // Q6_K ranges may start off a 16-byte boundary
 
     if (warp == 0) {
         if (lane == 0)
             produce_stages<BS>(a, full, empty, abort_flag, sbuf, rp_begin, rp_end, rps, ns, kb0, nbl, a.sp, false);
-        return;
-    }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ consumers
+        const int ct = tid - 32;
+        const int cw = ct >> 5;
+        const int g = lane >> 2, q = lane & 3;
+        const uint32_t xb_s = smem_u32(smem + a.xs_offset);
+        const uint32_t wp_s = smem_u32(smem + a.wp_offset);
+        const uint32_t red_s = smem_u32(smem + a.red_offset);
+        const uint32_t sbuf_s = smem_u32(sbuf);
+        pdl_wait();
+        pdl_launch_dependents();
+        stage_xb<FMT, NT>(a, xb_s, bscale, cw, lane, 1, kb0, nbl);
 
-    // ---------------------------------------------------------- consumers
-    const int ct = tid - 32;
-    const int cw = ct >> 5;
-    const int g = lane >> 2, q = lane & 3;
-    const uint32_t xb_s = smem_u32(smem + a.xs_offset);
-    const uint32_t wp_s = smem_u32(smem + a.wp_offset);
-    const uint32_t sbuf_s = smem_u32(sbuf);
-    pdl_wait();
-    pdl_launch_dependents();
-    stage_xb<FMT, NT>(a, xb_s, bscale, cw, lane, 1, kb0, nbl);
+        // byte selectors: scales of chunk q (half 0) / q+4 (half 1) sit at
+        // bytes 2*(q/2), 2*(q/2)+1 of either half; mins 2q, 2q+1 at bytes
+        // 2*(q%2), +1
+        const uint32_t p0 = 2u * static_cast<uint32_t>(q >> 1), pm = 2u * static_cast<uint32_t>(q & 1);
+        const uint32_t sel = 0x4040u | p0 | ((p0 + 1) << 8);
+        const uint32_t msel = 0x4040u | pm | ((pm + 1) << 8);
+        const uint32_t xlane = xb_s + 8u * NT * lane;
+        const uint32_t bsc_s = smem_u32(bscale);
 
-    // byte selectors: scales of chunk q (half 0) / q+4 (half 1) sit at bytes
-    // 2*(q/2), 2*(q/2)+1 of either half; mins 2q, 2q+1 at bytes 2*(q%2), +1
-    const uint32_t p0 = 2u * static_cast<uint32_t>(q >> 1), pm = 2u * static_cast<uint32_t>(q & 1);
-    const uint32_t sel = 0x4040u | p0 | ((p0 + 1) << 8);
-    const uint32_t msel = 0x4040u | pm | ((pm + 1) << 8);
-    const uint32_t xlane = xb_s + 8u * NT * lane;
-    const uint32_t bsc_s = smem_u32(bscale);
-
-    StageIter it(rp_begin, rp_end, rps, a.N, kMmaRowPairs, ns);
-    Stage st;
-    int own = 0;
-    while (it.next(st)) {
-        const int slot = it.slot;
-        if (!mbar_wait_bounded(&full[slot], it.phase, abort_flag)) raise_fault(a, abort_flag, 6);
-        float ys[2][NT], ym[2][NT];
+        StageIter it(rp_begin, rp_end, rps, a.N, kMmaRowPairs, ns);
+        Stage st;
+        while (it.next(st)) {
+            const int slot = it.slot;
+            const int si = it.count - 1;  // this stage's index in the CTA's sequence
+            if (!mbar_wait_bounded(&full[slot], it.phase, abort_flag)) raise_fault(a, abort_flag, 6);
+            float ys[2][NT], ym[2][NT];
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
+            for (int r = 0; r < 2; ++r)
 #pragma unroll
-            for (int n = 0; n < NT; ++n) ys[r][n] = ym[r][n] = 0.f;
-        if (!*abort_flag) {
-            const uint32_t rg = sbuf_s + slot * a.stage_bytes + g * a.sp;
-            const uint32_t rg8 = rg + 8 * a.sp;
-            for (int b = cw; b < nbl; b += kConsumerWarps) {
-                const uint32_t xbl = xlane + 8u * NT * 32 * mma_steps<FMT>() * b, bsc = bsc_s + 8u * NC * b;
-                if constexpr (FMT == 1) q4k_mma_block<NT>(rg, rg8, b, xbl, bsc, sel, msel, q, ys, ym);
-                else if (b & 1) q6k_mma_block<NT, true>(rg, rg8, b, xbl, bsc, q, ys);
-                else q6k_mma_block<NT, false>(rg, rg8, b, xbl, bsc, q, ys);
+                for (int n = 0; n < NT; ++n) ys[r][n] = ym[r][n] = 0.f;
+            if (!*abort_flag) {
+                // the K range starts `rem` bytes into each smem row (see produce_stages)
+                const uint32_t rg = sbuf_s + slot * a.stage_bytes + g * a.sp + rem;
+                const uint32_t rg8 = rg + 8 * a.sp;
+                for (int b = cw; b < nbl; b += kConsumerWarps) {
+                    const uint32_t xbl = xlane + 8u * NT * 32 * mma_steps<FMT>() * b, bsc = bsc_s + 8u * NC * b;
+                    if constexpr (FMT == 1) q4k_mma_block<NT>(rg, rg8, b, xbl, bsc, sel, msel, q, ys, ym);
+                    else if (((rem >> 1) + b) & 1) q6k_mma_block<NT, true>(rg, rg8, b, xbl, bsc, q, ys);
+                    else q6k_mma_block<NT, false>(rg, rg8, b, xbl, bsc, q, ys);
+                }
+            }
+            const int p = si & 1;
+            const uint32_t wb = wp_s + 4u * (p * (kConsumerWarps * 16 * NC));
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+                    st_s32f(wb + 4u * ((cw * 16 + g + 8 * r) * NC + 4 * n + q), ys[r][n] - ym[r][n]);
+            const bool stop = named_bar_or(1, kConsumers, *abort_flag != 0);
+            if (lane == 0) mbar_arrive(&empty[slot]);
+            if (stop) break;
+            if (!cl) {
+                for (int t = ct; t < st.nrows * NC; t += kConsumers) {
+                    const int row = t / NC, j = t - row * NC;
+                    if (j >= a.ncol_real) continue;
+                    float v = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) v += ld_s32f(wb + 4u * ((w * 16 + row) * NC + j));
+                    if (S == 1) a.y[j * a.ldy + st.row0 + row] = v;
+                    else a.partial[(static_cast<int64_t>(ks) * a.ncol_real + j) * a.N + st.row0 + row] = v;
+                }
+                continue;
+            }
+            // cluster reduction: thread ct < NRED owns (row, column) ct
+            if (ct < NRED) {
+                const int row = ct / NC, j = ct - row * NC;
+                float v = 0.f;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) v += ld_s32f(wb + 4u * ((w * 16 + row) * NC + j));
+                if (ks == 0) {
+                    if (!mbar_wait_cluster_bounded(&recv[p], (si >> 1) & 1, abort_flag)) raise_fault(a, abort_flag, 6);
+                    for (int r = 1; r < S; ++r) v += ld_s32f(red_s + 4u * ((p * (S - 1) + r - 1) * NRED + ct));
+                    if (row < st.nrows && j < a.ncol_real) a.y[j * a.ldy + st.row0 + row] = v;
+                    named_bar_sync(2, NRED);  // every value of buffer p read
+                    if (ct < S - 1 && si + 2 < total) mbar_arrive_remote(map_rank(smem_u32(&sent[p]), ct + 1));
+                } else {
+                    if (si >= 2 && !mbar_wait_cluster_bounded(&sent[p], ((si >> 1) - 1) & 1, abort_flag))
+                        raise_fault(a, abort_flag, 6);
+                    st_cluster_f32(map_rank(red_s + 4u * ((p * (S - 1) + ks - 1) * NRED + ct), 0), v);
+                    mbar_arrive_remote(map_rank(smem_u32(&recv[p]), 0));
+                }
             }
         }
-        const uint32_t wb = wp_s + 4u * ((own & 1) * (kConsumerWarps * 16 * NC));
-        ++own;
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-                st_s32f(wb + 4u * ((cw * 16 + g + 8 * r) * NC + 4 * n + q), ys[r][n] - ym[r][n]);
-        const bool stop = named_bar_or(1, kConsumers, *abort_flag != 0);
-        if (lane == 0) mbar_arrive(&empty[slot]);
-        if (stop) break;
-        for (int t = ct; t < st.nrows * NC; t += kConsumers) {
-            const int row = t / NC, j = t - row * NC;
-            if (j >= a.ncol_real) continue;
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) v += ld_s32f(wb + 4u * ((w * 16 + row) * NC + j));
-            if (a.ksplit == 1) a.y[j * a.ldy + st.row0 + row] = v;
-            else a.partial[(static_cast<int64_t>(ks) * a.ncol_real + j) * a.N + st.row0 + row] = v;
-        }
     }
+    __syncwarp();
+    if (cl) cluster_sync();
 }
 
 template <int FMT, int NT>
@@ -516,12 +565,37 @@ cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stre
     cfg.blockDim = dim3(32 + kConsumers);
     cfg.dynamicSmemBytes = p.smem_bytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = p.pdl ? 1 : 0;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = p.cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.cluster > 1 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// Clusters of `cluster` CTAs of this kernel with `smem_bytes` each that fit
+// on the device at once (0 if none).
+template <int FMT, int NT>
+cudaError_t mma_active_clusters(int cluster, size_t smem_bytes, int* out) {
+    auto kern = mma_kernel<FMT, NT>;
+    cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem_bytes);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cluster);
+    cfg.blockDim = dim3(32 + kConsumers);
+    cfg.dynamicSmemBytes = smem_bytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a);
+    return cudaOccupancyMaxActiveClusters(out, kern, &cfg);
 }
 
 }  // namespace kq

@@ -153,7 +153,7 @@ def test_linearity():
 # ---------------------------------------------------------- multi column
 @pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q4_k", 17, 768),
                                      ("q4_k", 4096, 4096), ("q4_k", 33, 14336), ("q6_k", 64, 4096),
-                                     ("q6_k", 41, 2048), ("q6_k", 4096, 2048)])
+                                     ("q6_k", 41, 2048), ("q6_k", 4096, 2048), ("q6_k", 3, 14336)])
 @pytest.mark.parametrize("k", [2, 3, 4, 5, 8])
 def test_multi_columns_independent_and_match_oracle(fmt, N, K, k):
     """Each column of a k-column call equals the same column of an 8-column
