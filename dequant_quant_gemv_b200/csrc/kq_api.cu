@@ -167,7 +167,7 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
 struct MmaLayout {
     size_t sp, stage, wp, bs, red, xb, fixed;
 };
-static MmaLayout mma_layout(int fmt, int nt, int nbs, int S) {
+static MmaLayout mma_layout(int fmt, int nt, int nbs, int S, int ng) {
     MmaLayout L;
     // the staged row (which may start up to 14 bytes into the smem row) plus
     // 4 bytes (Q6_K word loads may read 2 bytes past a block), rounded up to
@@ -178,7 +178,7 @@ static MmaLayout mma_layout(int fmt, int nt, int nbs, int S) {
     L.sp = srow <= res ? res : round_up(srow - res, 128) + res;
     L.stage = round_up(16 * L.sp, 128);
     const size_t nc = 4 * static_cast<size_t>(nt);
-    L.wp = sizeof(float) * 2 * kConsumerWarps * 16 * nc;
+    L.wp = sizeof(float) * ng * 2 * kConsumerWarps * 16 * nc;
     L.bs = round_up(sizeof(float) * 2 * nc * nbs, 128);
     L.red = S > 1 ? sizeof(float) * 2 * (S - 1) * 16 * nc : 0;
     L.xb = static_cast<size_t>(nbs) * (fmt == KQ_FMT_Q4_K ? 17 : 16) * 32 * nt * 8;
@@ -186,9 +186,9 @@ static MmaLayout mma_layout(int fmt, int nt, int nbs, int S) {
     return L;
 }
 
-static cudaError_t active_clusters(int fmt, int nt, int S, size_t smem, int* out) {
+static cudaError_t active_clusters(int fmt, int nt, int ng, int S, size_t smem, int* out) {
     struct Entry {
-        int dev, fmt, nt, S;
+        int dev, fmt, nt, ng, S;
         size_t smem;
         int n;
     };
@@ -201,17 +201,26 @@ static cudaError_t active_clusters(int fmt, int nt, int S, size_t smem, int* out
     {
         std::lock_guard<std::mutex> lk(mu);
         for (int i = 0; i < count; ++i)
-            if (cache[i].dev == dev && cache[i].fmt == fmt && cache[i].nt == nt && cache[i].S == S &&
-                cache[i].smem == smem) {
+            if (cache[i].dev == dev && cache[i].fmt == fmt && cache[i].nt == nt && cache[i].ng == ng &&
+                cache[i].S == S && cache[i].smem == smem) {
                 *out = cache[i].n;
                 return cudaSuccess;
             }
     }
-    if (fmt == KQ_FMT_Q4_K) err = nt == 1 ? mma_active_clusters<1, 1>(S, smem, out) : mma_active_clusters<1, 2>(S, smem, out);
-    else err = nt == 1 ? mma_active_clusters<2, 1>(S, smem, out) : mma_active_clusters<2, 2>(S, smem, out);
+    const int key = (fmt == KQ_FMT_Q4_K ? 0 : 4) + (nt - 1) * 2 + (ng - 1);
+    switch (key) {
+        case 0: err = mma_active_clusters<1, 1, 1>(S, smem, out); break;
+        case 1: err = mma_active_clusters<1, 1, 2>(S, smem, out); break;
+        case 2: err = mma_active_clusters<1, 2, 1>(S, smem, out); break;
+        case 3: err = mma_active_clusters<1, 2, 2>(S, smem, out); break;
+        case 4: err = mma_active_clusters<2, 1, 1>(S, smem, out); break;
+        case 5: err = mma_active_clusters<2, 1, 2>(S, smem, out); break;
+        case 6: err = mma_active_clusters<2, 2, 1>(S, smem, out); break;
+        default: err = mma_active_clusters<2, 2, 2>(S, smem, out); break;
+    }
     if (err != cudaSuccess) return err;
     std::lock_guard<std::mutex> lk(mu);
-    if (count < 64) cache[count++] = Entry{dev, fmt, nt, S, smem, *out};
+    if (count < 64) cache[count++] = Entry{dev, fmt, nt, ng, S, smem, *out};
     return cudaSuccess;
 }
 
@@ -238,15 +247,15 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
         int best = 0, best_use = 0;
         for (int s = 1; s <= 8 && s <= a.nb; ++s) {
             if (a.nb % s != 0) continue;
-            const MmaLayout L8 = mma_layout(fmt, 2, a.nb / s, s);
+            const MmaLayout L8 = mma_layout(fmt, 2, a.nb / s, s, 1);
             if (L8.fixed + 2 * L8.stage > limit) continue;
             int use = di.sm_count;
             if (s > 1) {
-                const MmaLayout Ln = mma_layout(fmt, nt, a.nb / s, s);
+                const MmaLayout Ln = mma_layout(fmt, nt, a.nb / s, s, 1);
                 size_t nsn = (limit - Ln.fixed) / Ln.stage;
                 if (nsn > kMaxStages) nsn = kMaxStages;
                 int fit = 0;
-                err = active_clusters(fmt, nt, s, Ln.fixed + nsn * Ln.stage, &fit);
+                err = active_clusters(fmt, nt, 1, s, Ln.fixed + nsn * Ln.stage, &fit);
                 if (err != cudaSuccess) return cuda_fail(err, "cluster occupancy query");
                 use = fit * s;
             }
@@ -265,7 +274,13 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
             cl = true;
         }
     }
-    const MmaLayout L = mma_layout(fmt, nt, nbs, S);
+    // two consumer groups when they leave room for three stages
+    int ng = 2;
+    MmaLayout L = mma_layout(fmt, nt, nbs, S, 2);
+    if (L.fixed + 3 * L.stage > limit) {
+        ng = 1;
+        L = mma_layout(fmt, nt, nbs, S, 1);
+    }
     if (L.fixed + 2 * L.stage > limit)
         return fail(KQ_ERR_UNSUPPORTED, "K=%lld with %d columns needs %zu bytes of shared memory (limit %zu)",
                     (long long)a.K, 4 * nt, L.fixed + 2 * L.stage, limit);
@@ -276,7 +291,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     int64_t ranges = di.sm_count / S;     // row ranges (clusters, or CTAs per K range)
     if (cl) {
         int fit = 0;
-        err = active_clusters(fmt, nt, S, L.fixed + ns * L.stage, &fit);
+        err = active_clusters(fmt, nt, ng, S, L.fixed + ns * L.stage, &fit);
         if (err != cudaSuccess) return cuda_fail(err, "cluster occupancy query");
         if (fit < 1) return fail(KQ_ERR_UNSUPPORTED, "no cluster of %d CTAs fits", S);
         ranges = fit;
@@ -301,7 +316,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     a.sbuf_offset = static_cast<int>(L.fixed);
     p.grid = static_cast<int>(grid);
     p.cluster = cl ? S : 1;
-    p.ng = 1;
+    p.ng = ng;
     p.smem_bytes = L.fixed + ns * L.stage;
     p.pdl = true;
     return KQ_OK;
@@ -343,6 +358,20 @@ static cudaError_t dispatch(const GemvArgs& a, const LaunchPlan& p, int fmt, int
     }
 }
 
+static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt, int nt, cudaStream_t s) {
+    const int key = (fmt == KQ_FMT_Q4_K ? 0 : 4) + (nt - 1) * 2 + (p.ng - 1);
+    switch (key) {
+        case 0: return launch_mma<1, 1, 1>(a, p, s);
+        case 1: return launch_mma<1, 1, 2>(a, p, s);
+        case 2: return launch_mma<1, 2, 1>(a, p, s);
+        case 3: return launch_mma<1, 2, 2>(a, p, s);
+        case 4: return launch_mma<2, 1, 1>(a, p, s);
+        case 5: return launch_mma<2, 1, 2>(a, p, s);
+        case 6: return launch_mma<2, 2, 1>(a, p, s);
+        default: return launch_mma<2, 2, 2>(a, p, s);
+    }
+}
+
 // Calls with 2 or more columns (speculative verify) run on the tensor-core
 // kernel, every column group of the call included, so a column's arithmetic
 // never depends on how the call was grouped.
@@ -360,8 +389,7 @@ static int run(GemvArgs& a, int fmt, int k, bool mma, cudaStream_t stream) {
     LaunchPlan p;
     int st = plan_for(fmt, k, mma, a, p);
     if (st != KQ_OK) return st;
-    if (mma && fmt == KQ_FMT_Q4_K) err = k <= 4 ? launch_mma<1, 1>(a, p, stream) : launch_mma<1, 2>(a, p, stream);
-    else if (mma) err = k <= 4 ? launch_mma<2, 1>(a, p, stream) : launch_mma<2, 2>(a, p, stream);
+    if (mma) err = dispatch_mma(a, p, fmt, k <= 4 ? 1 : 2, stream);
     else err = dispatch(a, p, fmt, padded_cols(k), stream);
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
     if (a.ksplit > 1 && !a.cluster) {  // cluster splits add their partial sums in the kernel

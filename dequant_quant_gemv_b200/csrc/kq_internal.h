@@ -62,9 +62,9 @@ template <int FMT, int NCOL, int NG>
 cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
 // Tensor-core kernel for 2..8 columns: NT n-tiles of 8 (4 columns each).
 int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p);
-template <int FMT, int NT>
+template <int FMT, int NT, int NG>
 cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
-template <int FMT, int NT>
+template <int FMT, int NT, int NG>
 cudaError_t mma_active_clusters(int cluster, size_t smem_bytes, int* out);
 cudaError_t fault_word(int** out);
 cudaError_t launch_splitk_combine(const float* partial, int S, int ncol, int64_t N, float* y, int64_t ldy,

@@ -164,18 +164,18 @@ __device__ __forceinline__ void b_slot(int w, int& s, int& q) {
 // One warp per (column, block) item, two float4 per lane, several items'
 // loads in flight.
 template <int FMT, int NT>
-__device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, int lane, int bar, int kb0,
-                         int nbl) {
+__device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, int nwarps, int lane, int bar,
+                         int kb0, int nbl) {
     constexpr int NC = 4 * NT;
     constexpr int U = 4;  // items per warp in flight
     const float* xg = a.x + static_cast<int64_t>(kb0) * 256;
     const int kr = a.ncol_real;
     const int items = NC * nbl;
-    for (int base = cw; base < items; base += kConsumerWarps * U) {
+    for (int base = cw; base < items; base += nwarps * U) {
         float4 v[U][2];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int it = base + kConsumerWarps * u;
+            const int it = base + nwarps * u;
             const int col = it / nbl, bl = it - col * nbl;
             v[u][0] = v[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (it < items && col < kr) {
@@ -191,7 +191,7 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int it = base + kConsumerWarps * u;
+            const int it = base + nwarps * u;
             if (it >= items) break;  // warp-uniform
             const int col = it / nbl, bl = it - col * nbl;
             float m = 0.f;
@@ -237,7 +237,55 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
             }
         }
     }
-    named_bar_sync(bar, kConsumers);
+    named_bar_sync(bar, 32 * nwarps);
+}
+
+// One Q4_K K-step in a single PTX block, so that the A quad and B pair are
+// born in the registers the mma reads (separate statements left the
+// compiler copying operands into place around every mma).  xg / xg8: quant
+// words of rows g and g+8; xsg / xsg8: the same shifted right by 8 (bytes 1
+// and 3 in the low halves); MASK picks the nibble (0x000F000F low,
+// 0x00F000F0 high); (m, a): the fp16 FMA that turns 1024 + n (or 1024 + 16n)
+// into sc*n; baddr: this lane's B entry (NT pairs of registers).
+template <int NT, uint32_t MASK>
+__device__ __forceinline__ void q4k_step(float (&d)[NT][4], uint32_t xg, uint32_t xg8, uint32_t xsg, uint32_t xsg8,
+                                         uint32_t mg, uint32_t ag, uint32_t mg8, uint32_t ag8, uint32_t baddr) {
+    if constexpr (NT == 1) {
+        asm volatile(
+            "{\n\t.reg .b32 t0, t1, t2, t3, a0, a1, a2, a3, b0, b1;\n\t"
+            "lop3.b32 t0, %4, %13, 0x64006400, 0xEA;\n\t"
+            "lop3.b32 t1, %5, %13, 0x64006400, 0xEA;\n\t"
+            "lop3.b32 t2, %6, %13, 0x64006400, 0xEA;\n\t"
+            "lop3.b32 t3, %7, %13, 0x64006400, 0xEA;\n\t"
+            "fma.rn.f16x2 a0, t0, %8, %9;\n\t"
+            "fma.rn.f16x2 a1, t1, %10, %11;\n\t"
+            "fma.rn.f16x2 a2, t2, %8, %9;\n\t"
+            "fma.rn.f16x2 a3, t3, %10, %11;\n\t"
+            "ld.shared.v2.b32 {b0, b1}, [%12];\n\t"
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {a0, a1, a2, a3}, {b0, b1}, "
+            "{%0, %1, %2, %3};\n\t}"
+            : "+f"(d[0][0]), "+f"(d[0][1]), "+f"(d[0][2]), "+f"(d[0][3])
+            : "r"(xg), "r"(xg8), "r"(xsg), "r"(xsg8), "r"(mg), "r"(ag), "r"(mg8), "r"(ag8), "r"(baddr), "n"(MASK));
+    } else {
+        asm volatile(
+            "{\n\t.reg .b32 t0, t1, t2, t3, a0, a1, a2, a3, b0, b1, b2, b3;\n\t"
+            "lop3.b32 t0, %8, %17, 0x64006400, 0xEA;\n\t"
+            "lop3.b32 t1, %9, %17, 0x64006400, 0xEA;\n\t"
+            "lop3.b32 t2, %10, %17, 0x64006400, 0xEA;\n\t"
+            "lop3.b32 t3, %11, %17, 0x64006400, 0xEA;\n\t"
+            "fma.rn.f16x2 a0, t0, %12, %13;\n\t"
+            "fma.rn.f16x2 a1, t1, %14, %15;\n\t"
+            "fma.rn.f16x2 a2, t2, %12, %13;\n\t"
+            "fma.rn.f16x2 a3, t3, %14, %15;\n\t"
+            "ld.shared.v4.b32 {b0, b1, b2, b3}, [%16];\n\t"
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {a0, a1, a2, a3}, {b0, b1}, "
+            "{%0, %1, %2, %3};\n\t"
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%4, %5, %6, %7}, {a0, a1, a2, a3}, {b2, b3}, "
+            "{%4, %5, %6, %7};\n\t}"
+            : "+f"(d[0][0]), "+f"(d[0][1]), "+f"(d[0][2]), "+f"(d[0][3]), "+f"(d[1][0]), "+f"(d[1][1]),
+              "+f"(d[1][2]), "+f"(d[1][3])
+            : "r"(xg), "r"(xg8), "r"(xsg), "r"(xsg8), "r"(mg), "r"(ag), "r"(mg8), "r"(ag8), "r"(baddr), "n"(MASK));
+    }
 }
 
 // ------------------------------------------------------ one super-block
@@ -284,23 +332,10 @@ __device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, 
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int c = j >> 2;
-        uint32_t L02[2], L13[2], H02[2], H13[2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const uint32_t x = u4w(w[r][c], j & 3);
-            const uint32_t xs = x >> 8;
-            L02[r] = hfma2u((x & 0x000F000Fu) | kH2_1024, mlo[r][c], alo[r][c]);
-            L13[r] = hfma2u((xs & 0x000F000Fu) | kH2_1024, mlo[r][c], alo[r][c]);
-            H02[r] = hfma2u((x & 0x00F000F0u) | kH2_1024, mhi[r][c], ahi[r][c]);
-            H13[r] = hfma2u((xs & 0x00F000F0u) | kH2_1024, mhi[r][c], ahi[r][c]);
-        }
+        const uint32_t x0 = u4w(w[0][c], j & 3), x1 = u4w(w[1][c], j & 3);
         const uint32_t s_lo = xbl + 8u * NT * 32 * (2 * j), s_hi = s_lo + 8u * NT * 32;  // steps 2j, 2j+1
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const uint2 bl = ld_s64u(s_lo + 8 * n), bh = ld_s64u(s_hi + 8 * n);
-            mma16816(acc[n], L02[0], L02[1], L13[0], L13[1], bl.x, bl.y);
-            mma16816(acc[n], H02[0], H02[1], H13[0], H13[1], bh.x, bh.y);
-        }
+        q4k_step<NT, 0x000F000Fu>(acc, x0, x1, x0 >> 8, x1 >> 8, mlo[0][c], alo[0][c], mlo[1][c], alo[1][c], s_lo);
+        q4k_step<NT, 0x00F000F0u>(acc, x0, x1, x0 >> 8, x1 >> 8, mhi[0][c], ahi[0][c], mhi[1][c], ahi[1][c], s_hi);
     }
     {
         const uint32_t s_m = xbl + 8u * NT * 32 * 16;
@@ -415,8 +450,8 @@ __device__ __forceinline__ void q6k_mma_block(uint32_t rg, uint32_t rg8, int b, 
 // (skipped for the last two stages, which no sender waits for).  A cluster
 // barrier at the start (barriers initialised) and at the end (no CTA leaves
 // while another may still address its shared memory) brackets it all.
-template <int FMT, int NT>
-__global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_constant__ GemvArgs a) {
+template <int FMT, int NT, int NG>
+__global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __grid_constant__ GemvArgs a) {
     constexpr int NC = 4 * NT;
     constexpr int NRED = 16 * NC;  // values of one stage's partial sums
     extern __shared__ __align__(128) uint8_t smem[];
@@ -466,7 +501,11 @@ __global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_co
         __syncwarp();
     } else {
         // ------------------------------------------------------ consumers
-        const int ct = tid - 32;
+        // NG groups of 8 warps take alternate stages (group g: stages with
+        // index = g mod NG), hiding each other's latencies
+        const int ct_all = tid - 32;
+        const int g_id = NG == 2 ? (ct_all >> 8) : 0;
+        const int ct = ct_all & (kConsumers - 1);
         const int cw = ct >> 5;
         const int g = lane >> 2, q = lane & 3;
         const uint32_t xb_s = smem_u32(smem + a.xs_offset);
@@ -475,7 +514,7 @@ __global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_co
         const uint32_t sbuf_s = smem_u32(sbuf);
         pdl_wait();
         pdl_launch_dependents();
-        stage_xb<FMT, NT>(a, xb_s, bscale, cw, lane, 1, kb0, nbl);
+        stage_xb<FMT, NT>(a, xb_s, bscale, ct_all >> 5, NG * kConsumerWarps, lane, 3, kb0, nbl);
 
         // byte selectors: scales of chunk q (half 0) / q+4 (half 1) sit at
         // bytes 2*(q/2), 2*(q/2)+1 of either half; mins 2q, 2q+1 at bytes
@@ -491,6 +530,7 @@ __global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_co
         while (it.next(st)) {
             const int slot = it.slot;
             const int si = it.count - 1;  // this stage's index in the CTA's sequence
+            if (NG == 2 && (si & 1) != g_id) continue;
             if (!mbar_wait_bounded(&full[slot], it.phase, abort_flag)) raise_fault(a, abort_flag, 6);
             float ys[2][NT], ym[2][NT];
 #pragma unroll
@@ -508,14 +548,15 @@ __global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_co
                     else q6k_mma_block<NT, false>(rg, rg8, b, xbl, bsc, q, ys);
                 }
             }
-            const int p = si & 1;
-            const uint32_t wb = wp_s + 4u * (p * (kConsumerWarps * 16 * NC));
+            const int p = si & 1;  // reduction buffer (with two groups: the group's own)
+            const uint32_t wb =
+                wp_s + 4u * ((2 * g_id + ((si / NG) & 1)) * (kConsumerWarps * 16 * NC));
 #pragma unroll
             for (int r = 0; r < 2; ++r)
 #pragma unroll
                 for (int n = 0; n < NT; ++n)
                     st_s32f(wb + 4u * ((cw * 16 + g + 8 * r) * NC + 4 * n + q), ys[r][n] - ym[r][n]);
-            const bool stop = named_bar_or(1, kConsumers, *abort_flag != 0);
+            const bool stop = named_bar_or(1 + g_id, kConsumers, *abort_flag != 0);
             if (lane == 0) mbar_arrive(&empty[slot]);
             if (stop) break;
             if (!cl) {
@@ -540,7 +581,7 @@ __global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_co
                     if (!mbar_wait_cluster_bounded(&recv[p], (si >> 1) & 1, abort_flag)) raise_fault(a, abort_flag, 6);
                     for (int r = 1; r < S; ++r) v += ld_s32f(red_s + 4u * ((p * (S - 1) + r - 1) * NRED + ct));
                     if (row < st.nrows && j < a.ncol_real) a.y[j * a.ldy + st.row0 + row] = v;
-                    named_bar_sync(2, NRED);  // every value of buffer p read
+                    named_bar_sync(4 + g_id, NRED);  // every value of buffer p read
                     if (ct < S - 1 && si + 2 < total) mbar_arrive_remote(map_rank(smem_u32(&sent[p]), ct + 1));
                 } else {
                     if (si >= 2 && !mbar_wait_cluster_bounded(&sent[p], ((si >> 1) - 1) & 1, abort_flag))
@@ -555,14 +596,14 @@ __global__ void __launch_bounds__(32 + kConsumers, 1) mma_kernel(const __grid_co
     if (cl) cluster_sync();
 }
 
-template <int FMT, int NT>
+template <int FMT, int NT, int NG>
 cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream) {
-    auto kern = mma_kernel<FMT, NT>;
+    auto kern = mma_kernel<FMT, NT, NG>;
     cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), p.smem_bytes);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
-    cfg.blockDim = dim3(32 + kConsumers);
+    cfg.blockDim = dim3(32 + NG * kConsumers);
     cfg.dynamicSmemBytes = p.smem_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -579,14 +620,14 @@ cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stre
 
 // Clusters of `cluster` CTAs of this kernel with `smem_bytes` each that fit
 // on the device at once (0 if none).
-template <int FMT, int NT>
+template <int FMT, int NT, int NG>
 cudaError_t mma_active_clusters(int cluster, size_t smem_bytes, int* out) {
-    auto kern = mma_kernel<FMT, NT>;
+    auto kern = mma_kernel<FMT, NT, NG>;
     cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem_bytes);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cluster);
-    cfg.blockDim = dim3(32 + kConsumers);
+    cfg.blockDim = dim3(32 + NG * kConsumers);
     cfg.dynamicSmemBytes = smem_bytes;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
