@@ -25,6 +25,7 @@ replicas (weak scaling) with no collective on the data path.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import subprocess
@@ -375,6 +376,38 @@ def h2d_peak_gbs(torch, nbytes=512 << 20, reps=5):
     return best
 
 
+# -------------------------------------------------- measured DRAM traffic
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant
+# kernel, from one ncu capture (the summaries and commands are kept with
+# the profiles), keyed by (format, N, K, columns).  Valid only for the kernel sources they
+# were taken on: any change to csrc/ changes the hash and the bench reports
+# traffic as null until the counters are taken again.
+TRAFFIC_SOURCES = "0f6dfc3cfd7fff53"
+TRAFFIC = {
+    ("q4_k", 28672, 4096, 1): 66_125_056 + 270_336,  # gemv_kernel, 8B gate|up
+    ("q6_k", 4096, 14336, 1): 48_288_000,             # gemv_kernel, 8B down
+    ("q4_k", 28672, 4096, 8): 66_244_352 + 294_912,  # mma_kernel, 8B gate|up, 8 columns
+    ("q6_k", 4096, 14336, 8): 48_682_240 + 28_928,   # mma_kernel, 8B down, 8 columns, clusters of 4
+}
+
+
+def kernel_sources_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "dequant_quant_gemv_b200", "csrc")
+    for n in sorted(os.listdir(d)):
+        if n.endswith((".cu", ".cuh", ".h")):
+            h.update(n.encode())
+            with open(os.path.join(d, n), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(fmt, N, K, k):
+    if kernel_sources_hash() != TRAFFIC_SOURCES:
+        return None
+    return TRAFFIC.get((fmt, N, K, k))
+
+
 # ------------------------------------------------------ replicas over ranks
 def rank_seed(rank):
     """Each rank decodes its own replica: same shapes, its own weights and
@@ -535,9 +568,12 @@ def bench_kq(args, rank, world):
     if per_kind:
         dom = max(per_kind, key=lambda n: per_kind[n]["share"])
         dk = per_kind[dom]
-        result["roofline"] = {"bound": "hbm", "kernel": f"gemv_kernel {dk['fmt']} {dom} {dk['N']}x{dk['K']}",
+        kname = "mma_kernel (tensor cores)" if k >= 2 else "gemv_kernel"
+        result["roofline"] = {"bound": "hbm", "kernel": f"{kname} {dk['fmt']} {dom} {dk['N']}x{dk['K']}",
                               "achieved": dk["gbs"], "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
-                              "frac": round(dk["gbs"] / hbm, 4), "traffic": None}
+                              "frac": round(dk["gbs"] / hbm, 4),
+                              "traffic": measured_traffic(dk["fmt"], dk["N"], dk["K"], k),
+                              "algorithmic_bytes": dk["bytes"]}
         result["kernels"] = per_kind
     if isinstance(wl, Streamed):
         pk = h2d_peak_gbs(torch)
