@@ -132,7 +132,11 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     const int ng = ncol == 1 ? 2 : 1;
     const bool shared_x = a.x_seg_stride == 0;
     const size_t wp_bytes = round_up(sizeof(float) * ng * 2 * a.ps * a.parts * 2 * ncol, 128);
-    const size_t xs_bytes = round_up(sizeof(float) * (shared_x ? 1 : ng) * ncol * 2 * nb * kRegion, 128);
+    // one column of Q4_K: integer activation regions (2 x 336 bytes per
+    // super-block); otherwise fp32 regions
+    const size_t xcopy = ncol == 1 && fmt == KQ_FMT_Q4_K ? static_cast<size_t>(672) * nb
+                                                          : sizeof(float) * ncol * 2 * nb * kRegion;
+    const size_t xs_bytes = round_up((shared_x ? 1 : ng) * xcopy, 128);
     const size_t head = 256;
     const size_t fixed = head + wp_bytes + xs_bytes;
     const size_t limit = static_cast<size_t>(di.smem_optin);

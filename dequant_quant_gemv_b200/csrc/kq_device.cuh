@@ -195,6 +195,21 @@ __device__ __forceinline__ uint32_t u4w(const uint4& v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
+// -------------------------------------------------------- integer dots
+
+// Four byte products summed into an int32 (DP4A): unsigned quants with
+// signed (us) or unsigned (uu) activation bytes.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
 // ----------------------------------------------------------------- Q4_K
 
 // The four 6-bit scales and four 6-bit mins of half H (sub-blocks
