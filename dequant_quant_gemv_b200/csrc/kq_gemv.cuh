@@ -443,45 +443,40 @@ __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int
     }
 }
 
-// ----------------------------------------- single column: integer dot path
+// ----------------------------------- single column, Q4_K: integer dot path
 //
-// One column runs its inner products on DP4A (four byte products per
+// One Q4_K column runs its inner products on DP4A (four byte products per
 // instruction, exact int32 sums).  The activations of each group of 32
 // consecutive weights are scaled by a power of two 2^sh that puts the
 // group's largest |x| in [2^13, 2^14), rounded to integers xi (|xi| <= 2^14)
 // and stored as a signed high byte xi >> 8 and an unsigned low byte xi & 255
 // (xi = 256*hi + lo).  Per group the staging also keeps Xg = sum of the
-// fp32 activations (fixed order), P = 2^-sh and the integer sums of xi over
-// each half of 16.  A sub-block's sum of q*xi is then exact (|.| < 2^23, so
-// exact in fp32 too), and y = sum over sub-blocks of d*sc*P*S - dmin*m*Xg
-// (Q4_K) or d*s*P*(S - 32*XI16) (Q6_K) in fp32.  The only approximation
+// fp32 activations (fixed order) and P = 2^-sh.  A sub-block's sum S of
+// q*xi is then exact (|S| < 2^23, so exact in fp32 too), and y = sum over
+// sub-blocks of d*sc*P*S - dmin*m*Xg in fp32.  The only approximation
 // beyond fp32 rounding is xi: |x - P*xi| <= P/2 <= 2^-14 * (largest |x| of
 // the group), so |y - y_exact| <= 2^-14 * sum over groups of
 // (max_g |x|) * sum_{i in g} |w_i|.  All-zero quants with zero mins give
-// y = 0 exactly and Q6_K quants all 32 give y = 0 exactly (S - 32*XI16 = 0).
+// y = 0 exactly.  (A Q6_K variant measured slower than its fp32 units: its
+// 6-bit codes cost more to assemble than the DP4A saves.)
 
 constexpr int kXGroupBytes = 64;  // 32 high bytes, then 32 low bytes
-constexpr int kXInfoBytes = 16;   // Xg, P, XI16 of the first and second half
+constexpr int kXInfoBytes = 16;   // Xg, P (and 8 bytes of padding)
 // A region holds the 4 groups of one half super-block (its bytes, then its
 // 4 info records) plus 16 bytes of padding: 336 bytes = 21 16-byte units,
-// an odd count, so the regions of 8 consecutive lanes fall on distinct
-// banks.  Region of (block b, half H) = 2*slot(b) + H, with slot(b) = b for
-// Q4_K and (b mod 8)*(nb/8) + b/8 for Q6_K (whose warps take blocks
-// b = w mod 8): in both, the lanes of a warp read consecutive regions.
+// an odd count, so the regions of 8 consecutive lanes (consecutive halves
+// of consecutive blocks) fall on distinct banks.
 constexpr int kXRegionBytes = 4 * (kXGroupBytes + kXInfoBytes) + 16;
 
-template <int FMT>
-__device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H, int nb) {
-    const int slot = FMT == 1 ? b : (b & 7) * (nb >> 3) + (b >> 3);
-    return xs + kXRegionBytes * (2 * slot + H);
+__device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H) {
+    return xs + kXRegionBytes * (2 * b + H);
 }
 
 // Stage the K range [256*kb0, 256*(kb0+nbl)) of segment `seg` as above,
-// into the regions at `xs` (nb: blocks of the lane layout).  One warp per
-// group of 32 activations (lane = position), U groups' loads in flight.
-template <int FMT>
-__device__ void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, int nb, int warp, int nwarps, int lane,
-                            int bar, int nthr, int kb0, int nbl) {
+// into the regions at `xs`.  One warp per group of 32 activations (lane =
+// position), U groups' loads in flight.
+__device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, int warp, int nwarps, int lane,
+                                   int bar, int nthr, int kb0, int nbl) {
     constexpr int U = 4;
     const float* xg = a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256;
     const int groups = 8 * nbl;
@@ -508,18 +503,13 @@ __device__ void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, int nb,
                 sh = sh > 100 ? 100 : sh < -100 ? -100 : sh;
             }
             const int xi = __float2int_rn(v[u] * __int_as_float((sh + 127) << 23));
-            const uint32_t xr = x_region<FMT>(xs, G >> 3, (G >> 2) & 1, nb), k = G & 3;
+            const uint32_t xr = x_region(xs, G >> 3, (G >> 2) & 1), k = G & 3;
             asm volatile("st.shared.u8 [%0], %1;" ::"r"(xr + kXGroupBytes * k + lane), "r"(xi >> 8) : "memory");
             asm volatile("st.shared.u8 [%0], %1;" ::"r"(xr + kXGroupBytes * k + 32 + lane), "r"(xi & 255)
                          : "memory");
-            int xs = xi;
-#pragma unroll
-            for (int off = 8; off >= 1; off >>= 1) xs += __shfl_xor_sync(0xffffffffu, xs, off);
-            const int xs_hi = __shfl_sync(0xffffffffu, xs, 16);
             if (lane == 0) {
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xr + 4 * kXGroupBytes + kXInfoBytes * k),
-                             "r"(__float_as_uint(X)), "r"(static_cast<uint32_t>((127 - sh) << 23)), "r"(xs),
-                             "r"(xs_hi)
+                asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(xr + 4 * kXGroupBytes + kXInfoBytes * k),
+                             "r"(__float_as_uint(X)), "r"(static_cast<uint32_t>((127 - sh) << 23))
                              : "memory");
             }
         }
@@ -580,73 +570,6 @@ __device__ __forceinline__ void q4k_unit_int(uint32_t row0, int row_bytes, int b
             y[r] = fmaf(dd[r] * byte_f(sc4[r], 2 * cc + 1) * iH.y, sH, y[r]);
             y[r] = fmaf(-dm[r] * byte_f(m4[r], 2 * cc + 1), iH.x, y[r]);
         }
-    }
-    out[0][0] = y[0];
-    out[1][0] = y[1];
-}
-
-// Q6_K unit, one column: row pair, super-block b, half H (16-weight groups
-// 8H..8H+7), alignment class as in q6k_unit.  Quarter t of the half is x
-// group 8b + 4H + t; its byte group lg = 0..7 covers positions 4lg..4lg+3,
-// 16-weight group 2t + lg/4.
-template <bool ODD>
-__device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
-                                             float (&out)[2][1]) {
-    uint32_t QL[2][16], QH[2][8], S8[2][2];
-    float dsc[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const uint32_t bw = row0 + r * row_bytes + b * kQ6Bytes - (ODD ? 2 : 0);  // 4-byte aligned
-        auto sw = [&](int i) -> uint32_t {
-            if constexpr (ODD) return __byte_perm(ld_s32(bw + 4 * i), ld_s32(bw + 4 * i + 4), 0x5432);
-            else return ld_s32(bw + 4 * i);
-        };
-#pragma unroll
-        for (int i = 0; i < 16; ++i) QL[r][i] = sw(16 * H + i);   // ql[64H .. 64H+63]
-#pragma unroll
-        for (int i = 0; i < 8; ++i) QH[r][i] = sw(32 + 8 * H + i);  // qh[32H .. 32H+31]
-        S8[r][0] = sw(48 + 2 * H);                                  // int8 scales of groups 8H..8H+3
-        S8[r][1] = sw(49 + 2 * H);                                  // and 8H+4..8H+7
-        const uint32_t dword = ODD ? (ld_s32(bw + 208) >> 16) : ld_s32(bw + 208);
-        dsc[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(dword & 0xFFFFu)));
-    }
-    float y[2] = {0.f, 0.f};
-    // quarters in the order 0, 2, 1, 3: after 0 and 2 the first 8 ql words
-    // are dead (fewer live registers)
-#pragma unroll
-    for (int tt = 0; tt < 4; ++tt) {
-        const int t = (tt >> 1) | ((tt & 1) << 1);
-        const uint32_t gx = xr + kXGroupBytes * t;
-        const uint4 xh0 = ld_s128(gx), xh1 = ld_s128(gx + 16), xl0 = ld_s128(gx + 32), xl1 = ld_s128(gx + 48);
-        const float4 inf = ld_s128f(xr + 4 * kXGroupBytes + kXInfoBytes * t);
-        int hs[2][2] = {{0, 0}, {0, 0}};
-        uint32_t ls[2][2] = {{0u, 0u}, {0u, 0u}};
-#pragma unroll
-        for (int lg = 0; lg < 8; ++lg) {
-            const uint32_t xh = lg < 4 ? u4w(xh0, lg) : u4w(xh1, lg - 4);
-            const uint32_t xl = lg < 4 ? u4w(xl0, lg) : u4w(xl1, lg - 4);
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const uint32_t src = (t & 1) ? QL[r][8 + lg] : QL[r][lg];
-                const uint32_t low4 = (t & 2) ? ((src >> 4) & 0x0F0F0F0Fu) : (src & 0x0F0F0F0Fu);
-                const uint32_t hh = QH[r][lg];
-                const uint32_t top2 =
-                    (t == 0 ? (hh << 4) : t == 1 ? (hh << 2) : t == 2 ? hh : (hh >> 2)) & 0x30303030u;
-                const uint32_t qw = low4 | top2;
-                hs[r][lg >> 2] = dp4a_us(qw, xh, hs[r][lg >> 2]);
-                ls[r][lg >> 2] = dp4a_uu(qw, xl, ls[r][lg >> 2]);
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int g16 = 2 * t + hh;  // 16-weight group within the half
-                const int s = static_cast<int>(static_cast<int8_t>((S8[r][g16 >> 2] >> (8 * (g16 & 3))) & 0xFFu));
-                const int xsum = __float_as_int(hh ? inf.w : inf.z);
-                const int S = hs[r][hh] * 256 + static_cast<int>(ls[r][hh]) - 32 * xsum;
-                y[r] = fmaf(dsc[r] * static_cast<float>(s) * inf.y, static_cast<float>(S), y[r]);
-            }
     }
     out[0][0] = y[0];
     out[1][0] = y[1];
@@ -759,7 +682,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     constexpr bool INT = NCOL == 1 && FMT == 1;
     const uint32_t xcopy = INT ? kXRegionBytes * 2 * nb : 4 * NCOL * xcs;
     const uint32_t xs_s = smem_u32(xs) + (shared_x ? 0 : g * xcopy);
-    const uint32_t xri = x_region<FMT>(xs_s, u_b, u_H, nb);  // this lane's integer region
+    const uint32_t xri = x_region(xs_s, u_b, u_H);  // this lane's integer region (Q4_K)
     const uint32_t sbuf_s = smem_u32(sbuf), wp_s = smem_u32(wp) + 4 * g * wp_group;
     const uint32_t xr = xs_s + 4 * (region * kRegion);
 
@@ -769,8 +692,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     if (shared_x) {
         // one activation copy for all groups, staged by all consumer threads
         if constexpr (INT)
-            stage_x_int<FMT>(a, 0, xs_s, nb, ct_all >> 5, NG * kConsumerWarps, lane, NG == 2 ? 3 : 1,
-                             NG * kConsumers, kb0, nbl);
+            stage_x_int(a, 0, xs_s, ct_all >> 5, NG * kConsumerWarps, lane, NG == 2 ? 3 : 1, NG * kConsumers,
+                        kb0, nbl);
         else stage_x<FMT, NCOL>(a, 0, xs_s, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, kb0, nbl);
         staged_seg = 0;
     }
@@ -779,7 +702,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
         if (NG == 2 && ((it.count - 1) & 1) != g) continue;
         if (!shared_x && st.seg != staged_seg) {
             if constexpr (INT)
-                stage_x_int<FMT>(a, st.seg, xs_s, nb, cw, kConsumerWarps, lane, gbar, kConsumers, kb0, nbl);
+                stage_x_int(a, st.seg, xs_s, cw, kConsumerWarps, lane, gbar, kConsumers, kb0, nbl);
             else stage_x<FMT, NCOL>(a, st.seg, xs_s, ct, kConsumers, gbar, kb0, nbl);
             staged_seg = st.seg;
         }
