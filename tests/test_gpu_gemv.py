@@ -249,3 +249,36 @@ def test_invalid_arguments_are_rejected():
     with pytest.raises(kq.KQError):
         kq.gemv_multi(W, "q4_k", 4, 256, torch.zeros((9, 256), device="cuda"))
     assert kq.device_fault() == 0
+
+
+# ------------------------------------------- single-column integer path
+def test_q4k_single_column_within_activation_rounding_bound():
+    """Single-column Q4_K rounds each activation to a 14-bit integer on a
+    power-of-two grid per group of 32, so |x - x'| <= 2^-14 * (largest |x|
+    of the group).  The error must stay within that bound (plus fp32
+    rounding slack), computed from the oracle's dequantised weights."""
+    fmt, N, K = "q4_k", 256, 4096
+    W = matrix(fmt, 77, N, K)
+    x = x_vec(78, K)
+    y = kq.gemv(dev(W), fmt, N, K, dev(x)).cpu().numpy().astype(np.float64)
+    Wd = oracle.dequant(fmt, W, N, K).reshape(N, K)
+    xd = x.astype(np.float64)
+    err = np.abs(y - Wd @ xd)
+    gmax = np.abs(xd).reshape(-1, 32).max(axis=1)
+    bound = 2.0 ** -14 * (np.abs(Wd).reshape(N, -1, 32).sum(axis=2) * gmax[None, :]).sum(axis=1)
+    slack = 1e-5 * (np.abs(Wd) @ np.abs(xd)) + 1e-6
+    assert np.all(err <= bound + slack), float(np.max(err / (bound + slack)))
+
+
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+@pytest.mark.parametrize("scale", [1e-30, 1e-6, 3e3, 1e20])
+def test_single_column_scale_range(fmt, scale):
+    """Single column with activations far from 1: the integer path scales
+    each group of 32 by its own power of two."""
+    N, K = 96, 4096
+    W = matrix(fmt, 79, N, K)
+    x = (x_vec(80, K) * np.float32(scale)).astype(np.float32)
+    x[:64] = 0.0                                   # two all-zero groups
+    y = kq.gemv(dev(W), fmt, N, K, dev(x))
+    y_ref, s_ref = oracle_gemv(fmt, W, N, K, x)
+    assert_close(y, y_ref, s_ref, f"scale {scale}")
