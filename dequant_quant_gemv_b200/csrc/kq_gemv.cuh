@@ -284,27 +284,31 @@ struct Stage {
 // (One division at construction; next() only adds and compares.)  Also
 // tracks the ring slot and mbarrier phase of the stage it returns.
 struct StageIter {
-    int64_t left;        // row pairs still to hand out
-    int64_t seg, off;    // segment and row-pair offset within it
-    int64_t rps, N;
+    // 32-bit counters: a CTA's range, the row pairs of a segment (N <= 2^31
+    // rows) and the segment count (an int at the ABI) all fit
+    int left;            // row pairs still to hand out
+    int seg, off;        // segment and row-pair offset within it
+    int rps;
+    int64_t N;
     int ps, ns;
     int slot = -1;       // ring slot of the last stage returned
     uint32_t phase = 0;  // its mbarrier phase parity
     int count = 0;       // stages returned so far
     __device__ StageIter(int64_t rp_begin, int64_t rp_end, int64_t rps_, int64_t N_, int ps_, int ns_)
-        : left(rp_end - rp_begin), seg(rp_begin / rps_), off(rp_begin - (rp_begin / rps_) * rps_), rps(rps_),
-          N(N_), ps(ps_), ns(ns_) {}
+        : left(static_cast<int>(rp_end - rp_begin)), seg(static_cast<int>(rp_begin / rps_)),
+          off(static_cast<int>(rp_begin - (rp_begin / rps_) * rps_)), rps(static_cast<int>(rps_)), N(N_), ps(ps_),
+          ns(ns_) {}
     __device__ bool next(Stage& st) {
         if (left <= 0) return false;
         if (off == rps) {
             ++seg;
             off = 0;
         }
-        int64_t n = left < ps ? left : ps;
+        int n = left < ps ? left : ps;
         if (n > rps - off) n = rps - off;
         st.seg = seg;
-        st.row0 = 2 * off;
-        st.nrp = static_cast<int>(n);
+        st.row0 = 2 * static_cast<int64_t>(off);
+        st.nrp = n;
         const int64_t rows = N - st.row0;
         st.nrows = static_cast<int>(rows < 2 * n ? rows : 2 * n);
         off += n;
