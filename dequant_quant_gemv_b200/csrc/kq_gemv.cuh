@@ -675,6 +675,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
         part = kappa;
     }
     const int parts = a.parts;
+    // single column with whole row pairs per warp: no cross-warp reduction
+    const bool direct = NCOL == 1 && parts == 1;
     int region;
     if (FMT == 1) region = 2 * u_b + u_H;
     else region = ((kappa * (nb >> 3) + (u_b >> 3)) << 1) + u_H;
@@ -705,6 +707,9 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     while (it.next(st)) {
         if (NG == 2 && ((it.count - 1) & 1) != g) continue;
         if (!shared_x && st.seg != staged_seg) {
+            // (with warps running free between stages, all of the group must
+            // be done with the previous segment's activations first)
+            if (direct && staged_seg >= 0) named_bar_sync(gbar, kConsumers);
             if constexpr (INT)
                 stage_x_int(a, st.seg, xs_s, cw, kConsumerWarps, lane, gbar, kConsumers, kb0, nbl);
             else stage_x<FMT, NCOL>(a, st.seg, xs_s, ct, kConsumers, gbar, kb0, nbl);
@@ -737,6 +742,30 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
 #pragma unroll
                     for (int j = 0; j < NCOL; ++j) out[r][j] += __shfl_xor_sync(0xffffffffu, out[r][j], off);
             }
+        }
+        if (direct) {
+            // one warp holds all units of each of its row pairs: its lead
+            // lanes write y, and warps need not wait for each other between
+            // stages (the shuffles above have ended the warp's reads)
+            // (after a fault the warps keep walking the stages -- every wait
+            // then returns at once and no unit runs -- so that all of them
+            // reach the same barriers)
+            if (lane == 0) mbar_arrive(&empty[slot]);
+            if ((lane & (group - 1)) == 0 && u_rp < st.nrp) {
+                int64_t e = st.seg;
+                if (a.ids) e = a.ids[st.seg];
+                const bool valid = e >= 0 && e < a.E;
+                if (!valid && a.status) atomicExch(a.status, 7);
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int row = 2 * u_rp + r;
+                    if (row >= st.nrows) continue;
+                    const float v = valid ? out[r][0] : 0.f;
+                    if (a.ksplit == 1) a.y[st.seg * a.y_seg_stride + st.row0 + row] = v;
+                    else a.partial[static_cast<int64_t>(ks) * a.N + st.row0 + row] = v;
+                }
+            }
+            continue;
         }
         // the group's own stages alternate between two partial-sum buffers
         const uint32_t wb = wp_s + 4 * ((own & 1) * (a.ps * parts * 2 * NCOL));
