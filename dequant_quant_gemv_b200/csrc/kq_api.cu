@@ -137,7 +137,7 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     const size_t xcopy = ncol == 1 && fmt == KQ_FMT_Q4_K ? static_cast<size_t>(672) * nb
                                                           : sizeof(float) * ncol * 2 * nb * kRegion;
     const size_t xs_bytes = round_up((shared_x ? 1 : ng) * xcopy, 128);
-    const size_t head = 256;
+    const size_t head = kHeadBytes;
     const size_t fixed = head + wp_bytes + xs_bytes;
     const size_t limit = static_cast<size_t>(di.smem_optin);
     if (fixed + 2 * stage > limit)
@@ -186,7 +186,7 @@ static MmaLayout mma_layout(int fmt, int nt, int nbs, int S, int ng) {
     L.bs = round_up(sizeof(float) * 2 * nc * nbs, 128);
     L.red = S > 1 ? sizeof(float) * 2 * (S - 1) * 16 * nc : 0;
     L.xb = static_cast<size_t>(nbs) * (fmt == KQ_FMT_Q4_K ? 17 : 16) * 32 * nt * 8;
-    L.fixed = 256 + L.wp + L.bs + L.red + L.xb;
+    L.fixed = kHeadBytes + L.wp + L.bs + L.red + L.xb;
     return L;
 }
 
@@ -313,10 +313,10 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     a.sp = static_cast<int>(L.sp);
     a.nstage = static_cast<int>(ns);
     a.stage_bytes = static_cast<int>(L.stage);
-    a.wp_offset = 256;
-    a.xscale_offset = static_cast<int>(256 + L.wp);
-    a.red_offset = static_cast<int>(256 + L.wp + L.bs);
-    a.xs_offset = static_cast<int>(256 + L.wp + L.bs + L.red);
+    a.wp_offset = kHeadBytes;
+    a.xscale_offset = static_cast<int>(kHeadBytes + L.wp);
+    a.red_offset = static_cast<int>(kHeadBytes + L.wp + L.bs);
+    a.xs_offset = static_cast<int>(kHeadBytes + L.wp + L.bs + L.red);
     a.sbuf_offset = static_cast<int>(L.fixed);
     p.grid = static_cast<int>(grid);
     p.cluster = cl ? S : 1;
@@ -513,19 +513,26 @@ int kq_device_fault(int* out) {
     return KQ_OK;
 }
 
-int kq_gemv_multi(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx, int k, float* y,
-                  int64_t ldy, kq_stream_t stream) {
+// kq_gemv_multi and kq_gemv_fused: one validation and launch path.
+static int gemv_columns(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx, int k,
+                        const kq_prologue* pro, float* y, int64_t ldy, kq_stream_t stream) {
     g_last_error[0] = 0;
     int st = check_matrix(W, fmt, N, K);
     if (st != KQ_OK) return st;
     if (k < 1 || k > 8) return fail(KQ_ERR_INVALID_ARG, "k=%d outside 1..8", k);
+    const int kind = pro ? pro->kind : KQ_PRO_NONE;
+    if (kind != KQ_PRO_NONE && kind != KQ_PRO_RMSNORM && kind != KQ_PRO_SWIGLU)
+        return fail(KQ_ERR_INVALID_ARG, "unknown prologue kind %d", kind);
+    if (kind == KQ_PRO_RMSNORM && (!pro->gamma || !aligned(pro->gamma, 4) || !(pro->eps > 0.f)))
+        return fail(KQ_ERR_INVALID_ARG, "RMSNorm needs a 4-byte aligned gamma and eps > 0");
+    const int64_t xlen = kind == KQ_PRO_SWIGLU ? 2 * K : K;  // floats per activation column
     if (N == 0) return KQ_OK;
     if (!y || !aligned(y, 4)) return fail(KQ_ERR_INVALID_ARG, "y is NULL or misaligned");
     if (k > 1 && ldy < N) return fail(KQ_ERR_INVALID_ARG, "ldy=%lld < N", (long long)ldy);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (K == 0) return zero_outputs(y, ldy, N, k, s);
     if (!x || !aligned(x, 4)) return fail(KQ_ERR_INVALID_ARG, "x is NULL or misaligned");
-    if (k > 1 && ldx < K) return fail(KQ_ERR_INVALID_ARG, "ldx=%lld < K", (long long)ldx);
+    if (k > 1 && ldx < xlen) return fail(KQ_ERR_INVALID_ARG, "ldx=%lld < %lld", (long long)ldx, (long long)xlen);
     GemvArgs a = {};
     a.W = static_cast<const uint8_t*>(W);
     a.N = N;
@@ -537,16 +544,29 @@ int kq_gemv_multi(const void* W, int fmt, int64_t N, int64_t K, const float* x, 
     a.E = 1;
     a.seg_stride = 0;
     a.x = x;
-    a.ldx = ldx;
+    a.ldx = k > 1 ? ldx : xlen;
     a.x_seg_stride = 0;
     a.y = y;
-    a.ldy = ldy;
+    a.ldy = k > 1 ? ldy : N;
     a.y_seg_stride = 0;
     a.status = nullptr;
     a.ksplit = 1;
     a.nbs = a.nb;
     a.partial = nullptr;
+    a.pro = kind;
+    a.gamma = kind == KQ_PRO_RMSNORM ? pro->gamma : nullptr;
+    a.eps = kind == KQ_PRO_RMSNORM ? pro->eps : 0.f;
     return run_grouped(a, fmt, k, s);
+}
+
+int kq_gemv_multi(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx, int k, float* y,
+                  int64_t ldy, kq_stream_t stream) {
+    return gemv_columns(W, fmt, N, K, x, ldx, k, nullptr, y, ldy, stream);
+}
+
+int kq_gemv_fused(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx, int k,
+                  const kq_prologue* pro, float* y, int64_t ldy, kq_stream_t stream) {
+    return gemv_columns(W, fmt, N, K, x, ldx, k, pro, y, ldy, stream);
 }
 
 int kq_gemv(const void* W, int fmt, int64_t N, int64_t K, const float* x, float* y, kq_stream_t stream) {

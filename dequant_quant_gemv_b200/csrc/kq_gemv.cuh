@@ -388,13 +388,48 @@ __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empt
     }
 }
 
+// ------------------------------------------------------------- prologue
+
+// One activation after the prologue (i: index within the column's K):
+// as given, RMS-normalised (x_i * gamma_i * inv), or SiLU-gated
+// (silu(x_i) * x_{K+i}, the column holding [g; u]).
+__device__ __forceinline__ float pro_value(const GemvArgs& a, float v, const float* xc, int64_t i, float inv) {
+    if (a.pro == 1) return v * a.gamma[i] * inv;
+    if (a.pro == 2) return v / (1.0f + expf(-v)) * xc[a.K + i];
+    return v;
+}
+
+// For RMSNorm: 1/sqrt(mean(x^2) + eps) of the first ncol columns of segment
+// `seg` over all of K, by the nthr staging threads in a fixed order (each
+// thread a strided sum, warp butterflies, warps in order), into the
+// prologue scratch `inv` (ncol floats).  Every CTA computes it itself.
+__device__ inline void pro_inv_rms(const GemvArgs& a, int64_t seg, int ncol, int t, int nthr, int bar,
+                                   uint32_t scratch, uint32_t inv) {
+    const int warp = t >> 5, lane = t & 31, nw = nthr >> 5;
+    for (int c = 0; c < ncol; ++c) {
+        const float* xc = a.x + seg * a.x_seg_stride + c * a.ldx;
+        float sq = 0.f;
+        for (int64_t i = t; i < a.K; i += nthr) sq = fmaf(xc[i], xc[i], sq);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        if (lane == 0) st_s32f(scratch + 4 * (warp * 8 + c), sq);
+    }
+    named_bar_sync(bar, nthr);
+    if (t < ncol) {
+        float sq = 0.f;
+        for (int w = 0; w < nw; ++w) sq += ld_s32f(scratch + 4 * (w * 8 + t));
+        st_s32f(inv + 4 * t, 1.0f / sqrtf(sq / static_cast<float>(a.K) + a.eps));
+    }
+    named_bar_sync(bar, nthr);
+}
+
 // ------------------------------------------------------ activation stage
 
 // Stage the activations of segment `seg` (all NCOL columns) into the
 // padded, permuted layout the units read, then (Q4_K) the region sums.
 template <int FMT, int NCOL>
 __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar, int kb0,
-                        int nbl) {
+                        int nbl, uint32_t pinv) {
     // the K range [256*kb0, 256*(kb0+nbl)) in regions laid out for a.nbs blocks
     const float* xg = a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256;
     const int nb = a.nbs;
@@ -412,6 +447,13 @@ __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int
         float4 v;
         if ((reinterpret_cast<uintptr_t>(xc) & 15u) == 0) v = *reinterpret_cast<const float4*>(xc + i);
         else v = make_float4(xc[i], xc[i + 1], xc[i + 2], xc[i + 3]);
+        if (a.pro) {
+            const float* xcol = xc - static_cast<int64_t>(kb0) * 256;  // the column at K index 0
+            const int64_t gi = static_cast<int64_t>(kb0) * 256 + i;
+            const float inv = a.pro == 1 ? ld_s32f(pinv + 4 * (j < a.ncol_real ? j : a.ncol_real - 1)) : 0.f;
+            v = make_float4(pro_value(a, v.x, xcol, gi, inv), pro_value(a, v.y, xcol, gi + 1, inv),
+                            pro_value(a, v.z, xcol, gi + 2, inv), pro_value(a, v.w, xcol, gi + 3, inv));
+        }
         const int b = i >> 8, within = i & 255;
         int off;
         if constexpr (FMT == 1) {
@@ -480,7 +522,7 @@ __device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H) {
 // into the regions at `xs`.  One warp per group of 32 activations (lane =
 // position), U groups' loads in flight.
 __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, int warp, int nwarps, int lane,
-                                   int bar, int nthr, int kb0, int nbl) {
+                                   int bar, int nthr, int kb0, int nbl, uint32_t pinv) {
     constexpr int U = 4;
     const float* xg = a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256;
     const int groups = 8 * nbl;
@@ -490,6 +532,15 @@ __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, 
         for (int u = 0; u < U; ++u) {
             const int G = base + nwarps * u;
             v[u] = G < groups ? xg[32 * G + lane] : 0.f;
+        }
+        if (a.pro) {
+            const float* xcol = a.x + seg * a.x_seg_stride;
+            const float inv = a.pro == 1 ? ld_s32f(pinv) : 0.f;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int G = base + nwarps * u;
+                if (G < groups) v[u] = pro_value(a, v[u], xcol, static_cast<int64_t>(kb0) * 256 + 32 * G + lane, inv);
+            }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -695,12 +746,15 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
     Stage st;
     int64_t staged_seg = -1;
+    const uint32_t pro_s = smem_u32(smem + kProOffset), pinv_s = pro_s + 4 * 16 * 8;
     if (shared_x) {
         // one activation copy for all groups, staged by all consumer threads
+        if (a.pro == 1)
+            pro_inv_rms(a, 0, a.ncol_real, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, pro_s, pinv_s);
         if constexpr (INT)
             stage_x_int(a, 0, xs_s, ct_all >> 5, NG * kConsumerWarps, lane, NG == 2 ? 3 : 1, NG * kConsumers,
-                        kb0, nbl);
-        else stage_x<FMT, NCOL>(a, 0, xs_s, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, kb0, nbl);
+                        kb0, nbl, pinv_s);
+        else stage_x<FMT, NCOL>(a, 0, xs_s, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, kb0, nbl, pinv_s);
         staged_seg = 0;
     }
     int own = 0;  // stages this group has consumed
@@ -710,9 +764,12 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             // (with warps running free between stages, all of the group must
             // be done with the previous segment's activations first)
             if (direct && staged_seg >= 0) named_bar_sync(gbar, kConsumers);
+            // (per-segment activations: a group's own scratch half)
+            const uint32_t gpro = pro_s + 4 * 8 * 8 * g, ginv = pinv_s + 4 * 8 * g;
+            if (a.pro == 1) pro_inv_rms(a, st.seg, a.ncol_real, ct, kConsumers, gbar, gpro, ginv);
             if constexpr (INT)
-                stage_x_int(a, st.seg, xs_s, cw, kConsumerWarps, lane, gbar, kConsumers, kb0, nbl);
-            else stage_x<FMT, NCOL>(a, st.seg, xs_s, ct, kConsumers, gbar, kb0, nbl);
+                stage_x_int(a, st.seg, xs_s, cw, kConsumerWarps, lane, gbar, kConsumers, kb0, nbl, ginv);
+            else stage_x<FMT, NCOL>(a, st.seg, xs_s, ct, kConsumers, gbar, kb0, nbl, ginv);
             staged_seg = st.seg;
         }
         const int slot = it.slot;

@@ -45,7 +45,17 @@ struct GemvArgs {
     int xscale_offset;       // power-of-two scales per super-block and column
     int cluster;             // 1: the ksplit K ranges are the CTAs of a cluster, reduced in shared memory
     int red_offset;          // cluster reduction buffers (rank 0)
+    // activation prologue (kq_prologue): applied while staging
+    int pro;                 // 0 none, 1 RMSNorm, 2 SwiGLU ([g; u] columns of 2K floats)
+    const float* gamma;      // RMSNorm weights (K)
+    float eps;
 };
+
+// Shared-memory scratch of the prologue (both kernels): per-warp partial
+// sums of squares (16 warps x 8 columns) and the columns' 1/rms.
+constexpr int kProOffset = 256;
+constexpr int kProBytes = 1024;
+constexpr int kHeadBytes = kProOffset + kProBytes;  // barriers, flags, prologue scratch
 
 struct LaunchPlan {
     int grid;

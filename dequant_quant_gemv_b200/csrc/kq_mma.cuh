@@ -165,7 +165,7 @@ __device__ __forceinline__ void b_slot(int w, int& s, int& q) {
 // loads in flight.
 template <int FMT, int NT>
 __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, int nwarps, int lane, int bar,
-                         int kb0, int nbl) {
+                         int kb0, int nbl, uint32_t pinv) {
     constexpr int NC = 4 * NT;
     constexpr int U = 4;  // items per warp in flight
     const float* xg = a.x + static_cast<int64_t>(kb0) * 256;
@@ -186,6 +186,24 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                 } else {
                     v[u][0] = make_float4(xc[0], xc[1], xc[2], xc[3]);
                     v[u][1] = make_float4(xc[128], xc[129], xc[130], xc[131]);
+                }
+            }
+        }
+        if (a.pro) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int it = base + nwarps * u;
+                const int col = it / nbl, bl = it - col * nbl;
+                if (it >= items || col >= kr) continue;
+                const float* xcol = a.x + col * a.ldx;
+                const float inv = a.pro == 1 ? ld_s32f(pinv + 4 * col) : 0.f;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int64_t gi = static_cast<int64_t>(kb0 + bl) * 256 + 128 * h + 4 * lane;
+                    v[u][h] = make_float4(pro_value(a, v[u][h].x, xcol, gi, inv),
+                                          pro_value(a, v[u][h].y, xcol, gi + 1, inv),
+                                          pro_value(a, v[u][h].z, xcol, gi + 2, inv),
+                                          pro_value(a, v[u][h].w, xcol, gi + 3, inv));
                 }
             }
         }
@@ -514,7 +532,9 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
         const uint32_t sbuf_s = smem_u32(sbuf);
         pdl_wait();
         pdl_launch_dependents();
-        stage_xb<FMT, NT>(a, xb_s, bscale, ct_all >> 5, NG * kConsumerWarps, lane, 3, kb0, nbl);
+        const uint32_t pro_s = smem_u32(smem + kProOffset), pinv_s = pro_s + 4 * 16 * 8;
+        if (a.pro == 1) pro_inv_rms(a, 0, a.ncol_real, ct_all, NG * kConsumers, 3, pro_s, pinv_s);
+        stage_xb<FMT, NT>(a, xb_s, bscale, ct_all >> 5, NG * kConsumerWarps, lane, 3, kb0, nbl, pinv_s);
 
         // byte selectors: scales of chunk q (half 0) / q+4 (half 1) sit at
         // bytes 2*(q/2), 2*(q/2)+1 of either half; mins 2q, 2q+1 at bytes

@@ -34,6 +34,14 @@ class KQError(RuntimeError):
         self.status = status
 
 
+class Prologue(ctypes.Structure):
+    """kq_prologue: the activation prologue of kq_gemv_fused."""
+    _fields_ = [("kind", ctypes.c_int), ("gamma", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
+PROLOGUE = {"none": 0, "rmsnorm": 1, "swiglu": 2}
+
+
 def lib() -> ctypes.CDLL:
     """Load libkq.so (built in-tree by ``dequant_quant_gemv_b200.build``)."""
     global _lib
@@ -60,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.kq_moe_gemv.argtypes = [vp, i32, i32, i64, i64, sz, vp, i32, vp, i64, vp, vp, vp]
         L.kq_unpack.restype = i32
         L.kq_unpack.argtypes = [vp, i32, i64, vp, vp, vp, vp]
+        L.kq_gemv_fused.restype = i32
+        L.kq_gemv_fused.argtypes = [vp, i32, i64, i64, vp, i64, i32, ctypes.POINTER(Prologue), vp, i64, vp]
         _lib = L
     return _lib
 
@@ -109,6 +119,23 @@ def gemv_multi(W: torch.Tensor, fmt, N: int, K: int, X: torch.Tensor, Y: torch.T
         Y = torch.empty((k, N), dtype=torch.float32, device=X.device)
     _check(lib().kq_gemv_multi(_dev(W, "W"), _fmt(fmt), N, K, _dev(X, "X", torch.float32), X.stride(0), k,
                                _dev(Y, "Y", torch.float32), Y.stride(0), _stream(stream)), "kq_gemv_multi")
+    return Y
+
+
+def gemv_fused(W: torch.Tensor, fmt, N: int, K: int, X: torch.Tensor, kind: str = "none",
+               gamma: torch.Tensor | None = None, eps: float = 1e-5, Y: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """Y[c] = W P(X[c]) for the k rows of X: P = "none", "rmsnorm" (with gamma,
+    eps; rows of K) or "swiglu" (rows of 2K: [gate; up])."""
+    if X.dim() == 1:
+        X = X[None, :]
+    k = X.shape[0]
+    if Y is None:
+        Y = torch.empty((k, N), dtype=torch.float32, device=X.device)
+    pro = Prologue(PROLOGUE[kind], _dev(gamma, "gamma", torch.float32) if gamma is not None else None, eps)
+    _check(lib().kq_gemv_fused(_dev(W, "W"), _fmt(fmt), N, K, _dev(X, "X", torch.float32), X.stride(0), k,
+                               ctypes.byref(pro), _dev(Y, "Y", torch.float32), Y.stride(0), _stream(stream)),
+           "kq_gemv_fused")
     return Y
 
 

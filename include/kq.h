@@ -37,10 +37,18 @@
  *  - Calls are asynchronous on `stream` (0 = the legacy default stream).  The
  *    return value reports argument validation and launch errors only
  *    (KQ_ERR_CUDA carries cudaGetLastError()); kq_last_error() gives text.
- *  - Arithmetic: quants are unpacked exactly; products and sums are fp32.
- *    Every output satisfies |y - y_exact| <= 1e-3 * sum_i |w_i x_i| + 1e-6.
- *    Results are deterministic: the same inputs give bitwise-equal outputs,
- *    and column c of kq_gemv_multi equals kq_gemv on column c.
+ *  - Arithmetic: quants are unpacked exactly; sums are fp32 (or exact
+ *    integers).  Single-column Q4_K rounds each activation to a 14-bit
+ *    integer on a power-of-two grid per group of 32 (error at most 2^-14 of
+ *    the group's largest |x|); single-column Q6_K multiplies in fp32; two or
+ *    more columns run on the tensor cores with exact fp16 weight operands and
+ *    activations split into two fp16 terms (22 bits) after a power-of-two
+ *    scale per super-block.  Every output satisfies
+ *    |y - y_exact| <= 1e-3 * sum_i |w_i x_i| + 1e-6 for activations of
+ *    comparable magnitude within each group of 32.
+ *    Results are deterministic: the same inputs give bitwise-equal outputs;
+ *    column c of a kq_gemv_multi call with k >= 2 does not depend on the
+ *    other columns or on k, and k = 1 equals kq_gemv.
  *  - No C++ exception crosses this interface.  Functions without shared state
  *    are thread-safe; a kq_chain must not be used by two threads at once.
  */
@@ -118,10 +126,48 @@ KQ_API int kq_gemv(const void* W, int fmt, int64_t N, int64_t K, const float* x,
  *   y + c*ldy (N floats each, ldy >= N); 1 <= k <= 8.
  * The verify pass of speculative decoding ("Out-of-core LLM inference engine
  * ...", Approach: several positions verified with one pass of the large
- * model).  Column c equals kq_gemv(W, x + c*ldx) bitwise.
+ * model).  With k >= 2 the products run on the tensor cores; column c then
+ * equals column c of any other k >= 2 call on the same activations bitwise,
+ * and kq_gemv within the tolerance.  k = 1 equals kq_gemv bitwise.
  */
 KQ_API int kq_gemv_multi(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx,
                   int k, float* y, int64_t ldy, kq_stream_t stream);
+
+/* Activation prologues applied inside kq_gemv_fused (never written back). */
+typedef enum {
+    KQ_PRO_NONE = 0,
+    /* x'_i = x_i * gamma_i / sqrt(mean_j(x_j^2) + eps), per column: the norm
+     * in front of a layer's qkv and gate|up matmuls. */
+    KQ_PRO_RMSNORM = 1,
+    /* Each column holds 2K values [g; u]; x'_i = silu(g_i) * u_i with
+     * silu(g) = g / (1 + exp(-g)): the gated activation in front of down,
+     * taking the gate|up matmul's stacked output as is. */
+    KQ_PRO_SWIGLU = 2
+} kq_prologue_kind;
+
+typedef struct {
+    int kind;            /* kq_prologue_kind */
+    const float* gamma;  /* KQ_PRO_RMSNORM: K weights (device); else unused */
+    float eps;           /* KQ_PRO_RMSNORM: > 0 */
+} kq_prologue;
+
+/*
+ * kq_gemv_fused — Y = W P(X): kq_gemv_multi with a prologue P applied to the
+ * activations as they are staged, so the normalised or gated vector never
+ * goes through HBM.
+ *   pro: HOST pointer, NULL = KQ_PRO_NONE.  For KQ_PRO_SWIGLU, column c is
+ *   x + c*ldx with 2K floats (ldx >= 2K); otherwise as kq_gemv_multi.
+ * The pages do not spell these steps out: they are the RMSNorm and SiLU-gated
+ * MLP of the Llama and Qwen model families whose decode the pages benchmark
+ * ("Kortex: Streaming 70B Models on Consumer GPUs", the tables; "Out-of-core
+ * LLM inference engine written from scratch in Rust", Results).  Each CTA
+ * computes the column's sum of squares over all K itself (fixed order), so
+ * results are deterministic and independent of the grid.
+ * Errors: KQ_ERR_INVALID_ARG for an unknown kind, a NULL gamma, eps <= 0 or
+ * ldx < 2K for SwiGLU; otherwise as kq_gemv_multi.
+ */
+KQ_API int kq_gemv_fused(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx, int k,
+                         const kq_prologue* pro, float* y, int64_t ldy, kq_stream_t stream);
 
 /*
  * kq_gemv_splitk — kq_gemv_multi for tall-skinny matrices: when the matrix

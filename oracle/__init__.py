@@ -18,7 +18,8 @@ in natural index order.  Sources, by page:
 The multi-column, MoE and chain forms below are literal loops over the
 single-matrix product: column c of the verify GEMV is the GEMV of column c;
 the MoE GEMV for routed id e is the GEMV of expert e's matrix; a chain is its
-matrices one after another.
+matrices one after another.  The fused forms apply the textbook RMSNorm or
+SiLU-gated unit to each column in double, then take the same product.
 """
 from __future__ import annotations
 
@@ -63,6 +64,12 @@ def _load():
         lib.kqo_gemv_rows.argtypes = [i32, vp, i64, vp, i64, vp, vp, vp, i32]
         lib.kqo_unpack.restype = i32
         lib.kqo_unpack.argtypes = [i32, vp, i64, vp, vp, vp]
+        lib.kqo_rmsnorm.restype = None
+        lib.kqo_rmsnorm.argtypes = [vp, vp, i64, ctypes.c_double, vp]
+        lib.kqo_swiglu.restype = None
+        lib.kqo_swiglu.argtypes = [vp, i64, vp]
+        lib.kqo_gemv_x64.restype = i32
+        lib.kqo_gemv_x64.argtypes = [i32, vp, i64, i64, vp, vp, vp, i32]
         _lib = lib
     return _lib
 
@@ -139,6 +146,59 @@ def gemv_multi(fmt, W, N: int, K: int, X, nthreads=None):
     the fused kernel; the result is the same as k separate products)."""
     X = np.ascontiguousarray(X, np.float32).reshape(-1, K)
     ys, ss = zip(*(gemv(fmt, W, N, K, X[c], nthreads) for c in range(X.shape[0])))
+    return np.stack(ys), np.stack(ss)
+
+
+def rmsnorm(x, gamma, eps: float) -> np.ndarray:
+    """x_i * gamma_i / sqrt(mean(x^2) + eps) in float64 (kq_oracle.c)."""
+    x = np.ascontiguousarray(x, np.float32)
+    g = np.ascontiguousarray(gamma, np.float32)
+    out = np.empty(x.size, np.float64)
+    _load().kqo_rmsnorm(x.ctypes.data, g.ctypes.data, x.size, ctypes.c_double(eps), out.ctypes.data)
+    return out
+
+
+def swiglu(gu) -> np.ndarray:
+    """silu(g_i) * u_i for gu = [g; u] (2K floats), float64 (kq_oracle.c)."""
+    gu = np.ascontiguousarray(gu, np.float32)
+    K = gu.size // 2
+    out = np.empty(K, np.float64)
+    _load().kqo_swiglu(gu.ctypes.data, K, out.ctypes.data)
+    return out
+
+
+def gemv_x64(fmt, W, N: int, K: int, x, nthreads=None):
+    """(y, s) for float64 activations (a prologue's output)."""
+    f = _fmt(fmt)
+    W = _u8(W)
+    x = np.ascontiguousarray(x, np.float64)
+    assert x.size >= K
+    y = np.empty(N, np.float64)
+    s = np.empty(N, np.float64)
+    rc = _load().kqo_gemv_x64(f, W.ctypes.data, N, K, x.ctypes.data, y.ctypes.data, s.ctypes.data,
+                              _threads(nthreads))
+    if rc:
+        raise RuntimeError(f"kqo_gemv_x64 failed ({rc})")
+    return y, s
+
+
+def gemv_fused(fmt, W, N: int, K: int, X, kind: str, gamma=None, eps: float = 1e-5, nthreads=None):
+    """k-column GEMV of prologue(X): kind "none", "rmsnorm" (X is (k, K)) or
+    "swiglu" (X is (k, 2K), each row [g; u]).  Returns (k, N) y and s, with
+    s = sum |w x'| over the transformed activations."""
+    width = 2 * K if kind == "swiglu" else K
+    X = np.ascontiguousarray(X, np.float32).reshape(-1, width)
+    ys, ss = [], []
+    for c in range(X.shape[0]):
+        if kind == "rmsnorm":
+            xt = rmsnorm(X[c], gamma, eps)
+        elif kind == "swiglu":
+            xt = swiglu(X[c])
+        else:
+            xt = X[c].astype(np.float64)
+        y, s = gemv_x64(fmt, W, N, K, xt, nthreads)
+        ys.append(y)
+        ss.append(s)
     return np.stack(ys), np.stack(ss)
 
 

@@ -171,6 +171,61 @@ int kqo_gemv(int fmt, const uint8_t* W, int64_t N, int64_t K, const float* x, do
     return rc;
 }
 
+/* ---------------------------------------------------------------------
+ * Activation prologues (the step in front of a layer's matmuls).  The
+ * pages do not define them; these are the textbook RMSNorm and SiLU-gated
+ * unit of the Llama/Qwen decoder layers whose decode the pages benchmark:
+ *   rmsnorm: out_i = x_i * gamma_i / sqrt( (1/K) sum_j x_j^2 + eps )
+ *   swiglu:  out_i = silu(g_i) * u_i,  silu(g) = g / (1 + exp(-g)),
+ *            with gu = [g_0..g_{K-1}, u_0..u_{K-1}].
+ * Computed in double from the fp32 inputs. */
+void kqo_rmsnorm(const float* x, const float* gamma, int64_t K, double eps, double* out) {
+    double ss = 0.0;
+    for (int64_t i = 0; i < K; ++i) ss += (double)x[i] * (double)x[i];
+    const double inv = 1.0 / sqrt(ss / (double)K + eps);
+    for (int64_t i = 0; i < K; ++i) out[i] = (double)x[i] * (double)gamma[i] * inv;
+}
+
+void kqo_swiglu(const float* gu, int64_t K, double* out) {
+    for (int64_t i = 0; i < K; ++i) {
+        const double g = (double)gu[i];
+        out[i] = g / (1.0 + exp(-g)) * (double)gu[K + i];
+    }
+}
+
+/* kqo_gemv with double activations (the output of a prologue). */
+int kqo_gemv_x64(int fmt, const uint8_t* W, int64_t N, int64_t K, const double* x, double* y, double* sabs,
+                 int nthreads) {
+    int64_t bb = block_bytes(fmt);
+    if (bb < 0 || K % 256 != 0) return -1;
+    int64_t row_bytes = K / 256 * bb;
+    int bad = 0;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel num_threads(nthreads)
+    {
+        double* w = (double*)malloc(sizeof(double) * (size_t)K);
+        if (!w) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < N; ++r) {
+            if (!w) continue;
+            kqo_dequant_row(fmt, W + r * row_bytes, K, w);
+            double acc = 0.0, acc_abs = 0.0;
+            for (int64_t i = 0; i < K; ++i) {
+                double p = w[i] * x[i];
+                acc += p;
+                acc_abs += fabs(p);
+            }
+            y[r] = acc;
+            if (sabs) sabs[r] = acc_abs;
+        }
+        free(w);
+    }
+    return bad ? -2 : 0;
+}
+
 /* Logical fields of `nblocks` consecutive super-blocks, in the layout the
  * bit-exact unpack check compares:
  *   q[256*b + i]      quant of weight i (Q4_K 0..15, Q6_K 0..63, before -32)

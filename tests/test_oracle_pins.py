@@ -300,3 +300,61 @@ def test_rows_subset_matches_full():
     rows = np.array([39, 0, 17, 17, 5])
     yr, sr = oracle.gemv_rows("q6_k", W, K, rows, x)
     assert np.array_equal(yr, y[rows]) and np.array_equal(sr, s[rows])
+
+
+# ------------------------------------------------------------- prologues
+def test_rmsnorm_hand_example_and_invariants():
+    """[1, -2, 3, 4]: mean square 30/4, so the factor is 1/sqrt(7.5)
+    = 0.36514837167011077; with gamma = 1 and eps = 0 the output has mean
+    square 1, and scaling x by a power of two changes nothing."""
+    x = np.array([1, -2, 3, 4], np.float32)
+    out = oracle.rmsnorm(x, np.ones(4, np.float32), 0.0)
+    assert np.allclose(out, np.array([1, -2, 3, 4]) * 0.36514837167011077, rtol=0, atol=1e-15)
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(4096).astype(np.float32)
+    assert abs(np.mean(oracle.rmsnorm(x, np.ones_like(x), 0.0) ** 2) - 1.0) < 1e-12
+    assert np.array_equal(oracle.rmsnorm(x * np.float32(8), np.ones_like(x), 0.0),
+                          oracle.rmsnorm(x, np.ones_like(x), 0.0))
+    g = rng.standard_normal(4096).astype(np.float32)
+    assert np.allclose(oracle.rmsnorm(x, g, 0.0), oracle.rmsnorm(x, np.ones_like(x), 0.0) * g, rtol=1e-15)
+    # eps = mean square halves the squared factor
+    ms = float(np.mean(x.astype(np.float64) ** 2))
+    r = oracle.rmsnorm(x, np.ones_like(x), ms) / oracle.rmsnorm(x, np.ones_like(x), 0.0)
+    assert np.allclose(r, 1 / np.sqrt(2.0), rtol=1e-12)
+
+
+def test_swiglu_hand_values_and_identities():
+    """silu(0) = 0, silu(1) = 1/(1 + e^-1) = 0.7310585786300049; with up = 1
+    the output is silu(gate); silu(-g) = silu(g) - g; up = 0 gives 0."""
+    K = 6
+    gate = np.array([0, 1, -1, 2, -3, 40], np.float32)
+    ones = np.ones(K, np.float32)
+    s = oracle.swiglu(np.concatenate([gate, ones]))
+    assert s[0] == 0.0 and abs(s[1] - 0.7310585786300049) < 1e-15
+    assert abs(s[5] - 40.0) < 1e-12                         # silu(g) -> g for large g
+    neg = oracle.swiglu(np.concatenate([-gate, ones]))
+    assert np.allclose(neg, s - gate.astype(np.float64), rtol=0, atol=1e-14)
+    assert np.all(oracle.swiglu(np.concatenate([gate, np.zeros(K, np.float32)])) == 0)
+    up = np.array([2, 3, 5, 7, 11, 13], np.float32)
+    assert np.allclose(oracle.swiglu(np.concatenate([gate, up])), s * up, rtol=1e-15)
+
+
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+def test_gemv_fused_reduces_to_plain_forms(fmt):
+    """The fused oracle with no prologue equals the plain GEMV (float inputs
+    widen exactly); with a prologue it is the plain product of the
+    prologue's output."""
+    N, K = 5, 2048
+    W = kqgen.matrix(fmt, 11, N, K)
+    rng = np.random.default_rng(6)
+    X = rng.standard_normal((2, K)).astype(np.float32)
+    y0, s0 = oracle.gemv_fused(fmt, W, N, K, X, "none")
+    y1, s1 = oracle.gemv_multi(fmt, W, N, K, X)
+    assert np.array_equal(y0, y1) and np.array_equal(s0, s1)
+    Wd = oracle.dequant(fmt, W, N, K)
+    g = rng.standard_normal(K).astype(np.float32)
+    yr, _ = oracle.gemv_fused(fmt, W, N, K, X, "rmsnorm", g, 1e-5)
+    assert np.allclose(yr[1], Wd @ oracle.rmsnorm(X[1], g, 1e-5), rtol=1e-12, atol=1e-12)
+    GU = rng.standard_normal((1, 2 * K)).astype(np.float32)
+    ys, _ = oracle.gemv_fused(fmt, W, N, K, GU, "swiglu")
+    assert np.allclose(ys[0], Wd @ oracle.swiglu(GU[0]), rtol=1e-12, atol=1e-12)
