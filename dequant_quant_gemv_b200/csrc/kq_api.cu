@@ -139,7 +139,8 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     const size_t xs_bytes = round_up((shared_x ? 1 : ng) * xcopy, 128);
     const size_t head = kHeadBytes;
     const size_t fixed = head + wp_bytes + xs_bytes;
-    const size_t limit = static_cast<size_t>(di.smem_optin);
+    const size_t extra = a.pro == KQ_PRO_RMSNORM ? kProBytes : 0;  // RMSNorm scratch after the ring
+    const size_t limit = static_cast<size_t>(di.smem_optin) - extra;
     if (fixed + 2 * stage > limit)
         return fail(KQ_ERR_UNSUPPORTED, "K=%lld with %d columns needs %zu bytes of shared memory (limit %zu)",
                     (long long)a.K, ncol, fixed + 2 * stage, limit);
@@ -161,7 +162,8 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     p.grid = static_cast<int>(grid);
     p.cluster = 1;
     p.ng = ng;
-    p.smem_bytes = fixed + ns * stage;
+    a.pro_offset = static_cast<int>(fixed + ns * stage);
+    p.smem_bytes = fixed + ns * stage + extra;
     p.pdl = true;
     return KQ_OK;
 }
@@ -190,10 +192,11 @@ static MmaLayout mma_layout(int fmt, int nt, int nbs, int S, int ng) {
     return L;
 }
 
-static cudaError_t active_clusters(int fmt, int nt, int ng, int S, size_t smem, int* out) {
+static cudaError_t active_clusters(int fmt, int nt, int ng, int S, size_t smem, bool pro, int* out) {
     struct Entry {
         int dev, fmt, nt, ng, S;
         size_t smem;
+        bool pro;
         int n;
     };
     static std::mutex mu;
@@ -206,25 +209,25 @@ static cudaError_t active_clusters(int fmt, int nt, int ng, int S, size_t smem, 
         std::lock_guard<std::mutex> lk(mu);
         for (int i = 0; i < count; ++i)
             if (cache[i].dev == dev && cache[i].fmt == fmt && cache[i].nt == nt && cache[i].ng == ng &&
-                cache[i].S == S && cache[i].smem == smem) {
+                cache[i].S == S && cache[i].smem == smem && cache[i].pro == pro) {
                 *out = cache[i].n;
                 return cudaSuccess;
             }
     }
     const int key = (fmt == KQ_FMT_Q4_K ? 0 : 4) + (nt - 1) * 2 + (ng - 1);
     switch (key) {
-        case 0: err = mma_active_clusters<1, 1, 1>(S, smem, out); break;
-        case 1: err = mma_active_clusters<1, 1, 2>(S, smem, out); break;
-        case 2: err = mma_active_clusters<1, 2, 1>(S, smem, out); break;
-        case 3: err = mma_active_clusters<1, 2, 2>(S, smem, out); break;
-        case 4: err = mma_active_clusters<2, 1, 1>(S, smem, out); break;
-        case 5: err = mma_active_clusters<2, 1, 2>(S, smem, out); break;
-        case 6: err = mma_active_clusters<2, 2, 1>(S, smem, out); break;
-        default: err = mma_active_clusters<2, 2, 2>(S, smem, out); break;
+        case 0: err = mma_active_clusters<1, 1, 1>(S, smem, pro, out); break;
+        case 1: err = mma_active_clusters<1, 1, 2>(S, smem, pro, out); break;
+        case 2: err = mma_active_clusters<1, 2, 1>(S, smem, pro, out); break;
+        case 3: err = mma_active_clusters<1, 2, 2>(S, smem, pro, out); break;
+        case 4: err = mma_active_clusters<2, 1, 1>(S, smem, pro, out); break;
+        case 5: err = mma_active_clusters<2, 1, 2>(S, smem, pro, out); break;
+        case 6: err = mma_active_clusters<2, 2, 1>(S, smem, pro, out); break;
+        default: err = mma_active_clusters<2, 2, 2>(S, smem, pro, out); break;
     }
     if (err != cudaSuccess) return err;
     std::lock_guard<std::mutex> lk(mu);
-    if (count < 64) cache[count++] = Entry{dev, fmt, nt, ng, S, smem, *out};
+    if (count < 64) cache[count++] = Entry{dev, fmt, nt, ng, S, smem, pro, *out};
     return cudaSuccess;
 }
 
@@ -244,7 +247,8 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     if (err != cudaSuccess) return cuda_fail(err, "device query");
     if (fmt == KQ_FMT_Q6_K && a.nb % 8 != 0)
         return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
-    const size_t limit = static_cast<size_t>(di.smem_optin);
+    const size_t extra = a.pro == KQ_PRO_RMSNORM ? kProBytes : 0;  // RMSNorm scratch after the ring
+    const size_t limit = static_cast<size_t>(di.smem_optin) - extra;
     int S = a.ksplit, nbs = a.nbs;
     bool cl = false;
     if (S == 1) {
@@ -259,7 +263,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
                 size_t nsn = (limit - Ln.fixed) / Ln.stage;
                 if (nsn > kMaxStages) nsn = kMaxStages;
                 int fit = 0;
-                err = active_clusters(fmt, nt, 1, s, Ln.fixed + nsn * Ln.stage, &fit);
+                err = active_clusters(fmt, nt, 1, s, Ln.fixed + nsn * Ln.stage + extra, a.pro != 0, &fit);
                 if (err != cudaSuccess) return cuda_fail(err, "cluster occupancy query");
                 use = fit * s;
             }
@@ -295,7 +299,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     int64_t ranges = di.sm_count / S;     // row ranges (clusters, or CTAs per K range)
     if (cl) {
         int fit = 0;
-        err = active_clusters(fmt, nt, ng, S, L.fixed + ns * L.stage, &fit);
+        err = active_clusters(fmt, nt, ng, S, L.fixed + ns * L.stage + extra, a.pro != 0, &fit);
         if (err != cudaSuccess) return cuda_fail(err, "cluster occupancy query");
         if (fit < 1) return fail(KQ_ERR_UNSUPPORTED, "no cluster of %d CTAs fits", S);
         ranges = fit;
@@ -321,7 +325,8 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     p.grid = static_cast<int>(grid);
     p.cluster = cl ? S : 1;
     p.ng = ng;
-    p.smem_bytes = L.fixed + ns * L.stage;
+    a.pro_offset = static_cast<int>(L.fixed + ns * L.stage);
+    p.smem_bytes = L.fixed + ns * L.stage + extra;
     p.pdl = true;
     return KQ_OK;
 }

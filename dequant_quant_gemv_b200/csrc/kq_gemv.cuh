@@ -427,7 +427,9 @@ __device__ inline void pro_inv_rms(const GemvArgs& a, int64_t seg, int ncol, int
 
 // Stage the activations of segment `seg` (all NCOL columns) into the
 // padded, permuted layout the units read, then (Q4_K) the region sums.
-template <int FMT, int NCOL>
+// PRO: apply the prologue a.pro (a separate instantiation, so the plain
+// loop keeps its loads in flight).
+template <int FMT, int NCOL, bool PRO>
 __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar, int kb0,
                         int nbl, uint32_t pinv) {
     // the K range [256*kb0, 256*(kb0+nbl)) in regions laid out for a.nbs blocks
@@ -447,7 +449,7 @@ __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int
         float4 v;
         if ((reinterpret_cast<uintptr_t>(xc) & 15u) == 0) v = *reinterpret_cast<const float4*>(xc + i);
         else v = make_float4(xc[i], xc[i + 1], xc[i + 2], xc[i + 3]);
-        if (a.pro) {
+        if constexpr (PRO) {
             const float* xcol = xc - static_cast<int64_t>(kb0) * 256;  // the column at K index 0
             const int64_t gi = static_cast<int64_t>(kb0) * 256 + i;
             const float inv = a.pro == 1 ? ld_s32f(pinv + 4 * (j < a.ncol_real ? j : a.ncol_real - 1)) : 0.f;
@@ -520,7 +522,8 @@ __device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H) {
 
 // Stage the K range [256*kb0, 256*(kb0+nbl)) of segment `seg` as above,
 // into the regions at `xs`.  One warp per group of 32 activations (lane =
-// position), U groups' loads in flight.
+// position), U groups' loads in flight.  PRO as for stage_x.
+template <bool PRO>
 __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, int warp, int nwarps, int lane,
                                    int bar, int nthr, int kb0, int nbl, uint32_t pinv) {
     constexpr int U = 4;
@@ -533,7 +536,7 @@ __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, 
             const int G = base + nwarps * u;
             v[u] = G < groups ? xg[32 * G + lane] : 0.f;
         }
-        if (a.pro) {
+        if constexpr (PRO) {
             const float* xcol = a.x + seg * a.x_seg_stride;
             const float inv = a.pro == 1 ? ld_s32f(pinv) : 0.f;
 #pragma unroll
@@ -638,13 +641,25 @@ __device__ __forceinline__ void q6k_unit_dispatch(int kappa, uint32_t row0, int 
     else q6k_unit<NCOL, false>(row0, row_bytes, b, H, xr, xcs, out);
 }
 
+// Stage a segment's activations for the kernel below: threads ct of nthr
+// (whole warps), integer regions (INT) or fp32 regions, with or without the
+// prologue (PRO).
+template <int FMT, int NCOL, bool INT, bool PRO>
+__device__ __forceinline__ void stage_all(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar,
+                                          int kb0, int nbl, uint32_t pinv) {
+    if constexpr (INT) stage_x_int<PRO>(a, seg, xs, ct >> 5, nthr >> 5, ct & 31, bar, nthr, kb0, nbl, pinv);
+    else stage_x<FMT, NCOL, PRO>(a, seg, xs, ct, nthr, bar, kb0, nbl, pinv);
+}
+
 // ------------------------------------------------------------ the kernel
 
 // NG consumer groups of 8 warps each: group g consumes the stages whose
 // index is g mod NG, so two groups work on consecutive stages of one ring
 // while the producer keeps filling it (more warps per SM to hide shared-memory
 // latency, one activation copy, a deeper ring than two CTAs could hold).
-template <int FMT, int NCOL, int NG>
+// PRO: the instantiation that applies the prologue a.pro while staging
+// (kept apart so that the plain kernel carries none of its code).
+template <int FMT, int NCOL, int NG, bool PRO>
 __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __grid_constant__ GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -746,15 +761,12 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
     Stage st;
     int64_t staged_seg = -1;
-    const uint32_t pro_s = smem_u32(smem + kProOffset), pinv_s = pro_s + 4 * 16 * 8;
+    const uint32_t pro_s = smem_u32(smem + a.pro_offset), pinv_s = pro_s + 4 * 16 * 8;
     if (shared_x) {
         // one activation copy for all groups, staged by all consumer threads
-        if (a.pro == 1)
+        if (PRO && a.pro == 1)
             pro_inv_rms(a, 0, a.ncol_real, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, pro_s, pinv_s);
-        if constexpr (INT)
-            stage_x_int(a, 0, xs_s, ct_all >> 5, NG * kConsumerWarps, lane, NG == 2 ? 3 : 1, NG * kConsumers,
-                        kb0, nbl, pinv_s);
-        else stage_x<FMT, NCOL>(a, 0, xs_s, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, kb0, nbl, pinv_s);
+        stage_all<FMT, NCOL, INT, PRO>(a, 0, xs_s, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, kb0, nbl, pinv_s);
         staged_seg = 0;
     }
     int own = 0;  // stages this group has consumed
@@ -766,10 +778,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             if (direct && staged_seg >= 0) named_bar_sync(gbar, kConsumers);
             // (per-segment activations: a group's own scratch half)
             const uint32_t gpro = pro_s + 4 * 8 * 8 * g, ginv = pinv_s + 4 * 8 * g;
-            if (a.pro == 1) pro_inv_rms(a, st.seg, a.ncol_real, ct, kConsumers, gbar, gpro, ginv);
-            if constexpr (INT)
-                stage_x_int(a, st.seg, xs_s, cw, kConsumerWarps, lane, gbar, kConsumers, kb0, nbl, ginv);
-            else stage_x<FMT, NCOL>(a, st.seg, xs_s, ct, kConsumers, gbar, kb0, nbl, ginv);
+            if (PRO && a.pro == 1) pro_inv_rms(a, st.seg, a.ncol_real, ct, kConsumers, gbar, gpro, ginv);
+            stage_all<FMT, NCOL, INT, PRO>(a, st.seg, xs_s, ct, kConsumers, gbar, kb0, nbl, ginv);
             staged_seg = st.seg;
         }
         const int slot = it.slot;
@@ -861,7 +871,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
 
 template <int FMT, int NCOL, int NG>
 cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream) {
-    auto kern = gemv_kernel<FMT, NCOL, NG>;
+    auto kern = a.pro ? gemv_kernel<FMT, NCOL, NG, true> : gemv_kernel<FMT, NCOL, NG, false>;
     cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), p.smem_bytes);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};

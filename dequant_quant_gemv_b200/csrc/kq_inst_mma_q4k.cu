@@ -5,7 +5,7 @@
 namespace kq {
 #define KQ_MMA_INST(F, T, G)                                                                    \
     template cudaError_t launch_mma<F, T, G>(const GemvArgs&, const LaunchPlan&, cudaStream_t); \
-    template cudaError_t mma_active_clusters<F, T, G>(int, size_t, int*);
+    template cudaError_t mma_active_clusters<F, T, G>(int, size_t, bool, int*);
 KQ_MMA_INST(1, 1, 1)
 KQ_MMA_INST(1, 1, 2)
 KQ_MMA_INST(1, 2, 1)

@@ -49,13 +49,14 @@ struct GemvArgs {
     int pro;                 // 0 none, 1 RMSNorm, 2 SwiGLU ([g; u] columns of 2K floats)
     const float* gamma;      // RMSNorm weights (K)
     float eps;
+    int pro_offset;          // RMSNorm scratch (kProBytes) after the stage ring
 };
 
-// Shared-memory scratch of the prologue (both kernels): per-warp partial
-// sums of squares (16 warps x 8 columns) and the columns' 1/rms.
-constexpr int kProOffset = 256;
+// Shared-memory scratch of RMSNorm (both kernels): per-warp partial sums of
+// squares (16 warps x 8 columns) and the columns' 1/rms.  Reserved only by
+// launches that normalise.
 constexpr int kProBytes = 1024;
-constexpr int kHeadBytes = kProOffset + kProBytes;  // barriers, flags, prologue scratch
+constexpr int kHeadBytes = 256;  // barriers and flags
 
 struct LaunchPlan {
     int grid;
@@ -75,7 +76,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p);
 template <int FMT, int NT, int NG>
 cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
 template <int FMT, int NT, int NG>
-cudaError_t mma_active_clusters(int cluster, size_t smem_bytes, int* out);
+cudaError_t mma_active_clusters(int cluster, size_t smem_bytes, bool pro, int* out);
 cudaError_t fault_word(int** out);
 cudaError_t launch_splitk_combine(const float* partial, int S, int ncol, int64_t N, float* y, int64_t ldy,
                                   cudaStream_t stream);

@@ -162,8 +162,9 @@ __device__ __forceinline__ void b_slot(int w, int& s, int& q) {
 // the block into [2^14, 2^15)) and its sums by 2^(sh-5); `bscale` gets
 // (2^-sh, 2^(5-sh)) per block and column.  Columns >= ncol_real are zero.
 // One warp per (column, block) item, two float4 per lane, several items'
-// loads in flight.
-template <int FMT, int NT>
+// loads in flight.  PRO: apply the prologue a.pro (a separate
+// instantiation, so the plain loop keeps its loads in flight).
+template <int FMT, int NT, bool PRO>
 __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, int nwarps, int lane, int bar,
                          int kb0, int nbl, uint32_t pinv) {
     constexpr int NC = 4 * NT;
@@ -189,7 +190,7 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                 }
             }
         }
-        if (a.pro) {
+        if constexpr (PRO) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int it = base + nwarps * u;
@@ -468,7 +469,7 @@ __device__ __forceinline__ void q6k_mma_block(uint32_t rg, uint32_t rg8, int b, 
 // (skipped for the last two stages, which no sender waits for).  A cluster
 // barrier at the start (barriers initialised) and at the end (no CTA leaves
 // while another may still address its shared memory) brackets it all.
-template <int FMT, int NT, int NG>
+template <int FMT, int NT, int NG, bool PRO>
 __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __grid_constant__ GemvArgs a) {
     constexpr int NC = 4 * NT;
     constexpr int NRED = 16 * NC;  // values of one stage's partial sums
@@ -532,9 +533,9 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
         const uint32_t sbuf_s = smem_u32(sbuf);
         pdl_wait();
         pdl_launch_dependents();
-        const uint32_t pro_s = smem_u32(smem + kProOffset), pinv_s = pro_s + 4 * 16 * 8;
-        if (a.pro == 1) pro_inv_rms(a, 0, a.ncol_real, ct_all, NG * kConsumers, 3, pro_s, pinv_s);
-        stage_xb<FMT, NT>(a, xb_s, bscale, ct_all >> 5, NG * kConsumerWarps, lane, 3, kb0, nbl, pinv_s);
+        const uint32_t pro_s = smem_u32(smem + a.pro_offset), pinv_s = pro_s + 4 * 16 * 8;
+        if (PRO && a.pro == 1) pro_inv_rms(a, 0, a.ncol_real, ct_all, NG * kConsumers, 3, pro_s, pinv_s);
+        stage_xb<FMT, NT, PRO>(a, xb_s, bscale, ct_all >> 5, NG * kConsumerWarps, lane, 3, kb0, nbl, pinv_s);
 
         // byte selectors: scales of chunk q (half 0) / q+4 (half 1) sit at
         // bytes 2*(q/2), 2*(q/2)+1 of either half; mins 2q, 2q+1 at bytes
@@ -618,7 +619,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
 
 template <int FMT, int NT, int NG>
 cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream) {
-    auto kern = mma_kernel<FMT, NT, NG>;
+    auto kern = a.pro ? mma_kernel<FMT, NT, NG, true> : mma_kernel<FMT, NT, NG, false>;
     cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), p.smem_bytes);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
@@ -638,11 +639,11 @@ cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stre
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-// Clusters of `cluster` CTAs of this kernel with `smem_bytes` each that fit
-// on the device at once (0 if none).
+// Clusters of `cluster` CTAs of this kernel (the prologue instantiation if
+// `pro`) with `smem_bytes` each that fit on the device at once (0 if none).
 template <int FMT, int NT, int NG>
-cudaError_t mma_active_clusters(int cluster, size_t smem_bytes, int* out) {
-    auto kern = mma_kernel<FMT, NT, NG>;
+cudaError_t mma_active_clusters(int cluster, size_t smem_bytes, bool pro, int* out) {
+    auto kern = pro ? mma_kernel<FMT, NT, NG, true> : mma_kernel<FMT, NT, NG, false>;
     cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem_bytes);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
