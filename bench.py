@@ -9,7 +9,9 @@ the weights from HBM).  One step is one pass of the chain: 128 fused GEMV
 launches replayed as one CUDA graph.  Metric: weight GB/s (algorithmic weight
 bytes / time) and layer-chain tokens/s.
 
-Other workloads (--workload): gemv_q4k_4096 (one 4096 x 4096 Q4_K GEMV),
+Other workloads (--workload): llama8b_layer_fused (the same chain with the
+layer's RMSNorm and SiLU-gated product fused into the GEMVs), gemv_q4k_4096
+(one 4096 x 4096 Q4_K GEMV),
 verify8b_k{1,2,4,8} (the 8B chain with k activation columns),
 moe30b (Qwen3-30B-A3B-shaped routed experts, top-8 of 128, 48 layers),
 llama70b_resident / llama70b_stream (80-layer 70B-shaped chain in HBM, or
@@ -77,6 +79,8 @@ def chain_spec(kind):
 
 WORKLOADS = {
     "llama8b_chain": "Llama-3.1-8B-shaped decode chain, 32 layers, Q4_K + Q6_K down, batch 1",
+    "llama8b_layer_fused": "the 8B-shaped chain with RMSNorm fused into qkv and gate|up and the SiLU-gated "
+                           "product of gate|up's output fused into down",
     "gemv_q4k_4096": "single Q4_K GEMV 4096 x 4096, batch 1 (64 distinct copies rotated)",
     "gateup_q4k": "Q4_K GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
     "down_q6k": "Q6_K GEMV 4096 x 14336 (8B down), 8 distinct copies rotated",
@@ -166,7 +170,7 @@ class Resident:
         xoff, yoff, self.xslot, self.yslot = 0, 0, {}, {}
         for li, mats in enumerate(spec):
             for mi, (_, f, N, K, slot) in enumerate(mats):
-                if (li, slot) not in self.xslot:
+                if slot is not None and (li, slot) not in self.xslot:
                     self.xslot[(li, slot)] = (xoff, K)
                     xoff += k * K
                 self.yslot[(li, mi)] = (yoff, N)
@@ -216,6 +220,38 @@ class Resident:
 
     def io(self):
         return [self.X], [self.Y]
+
+
+class FusedLayer(Resident):
+    """The 8B chain with the decode layer's glue inside the GEMVs: qkv and
+    gate|up normalise their input (RMSNorm, per-layer weights), and down
+    takes gate|up's output [g; u] directly through the SiLU-gated prologue,
+    so the layer needs no separate norm or activation kernel.  Attention and
+    the residual adds are not on this path: o and each layer's norm inputs
+    keep their own seeded activations."""
+
+    EPS = 1e-5
+
+    def __init__(self, torch, kq, kqgen, spec, seed):
+        fused = [[m if m[0] != "down" else m[:4] + (None,) for m in mats] for mats in spec]
+        super().__init__(torch, kq, kqgen, fused, seed)
+        self.gu = {li: mi for li, mats in enumerate(fused) for mi, m in enumerate(mats) if m[0] == "gate_up"}
+        n = len(fused)
+        K = fused[0][0][3]
+        g = 1.0 + 0.1 * kqgen.normal_f32(seed ^ 0x6A3, 2 * n * K).astype(np.float32)
+        self.gamma = torch.from_numpy(g).cuda().view(n, 2, K)
+        torch.cuda.synchronize()
+
+    def launch(self, li, mi, stream):
+        name, f, N, K, _ = self.spec[li][mi]
+        W, y = self.W[li][mi], self.y_of(li, mi)[0]
+        if name == "qkv" or name == "gate_up":
+            self.kq.gemv_fused(W, f, N, K, self.x_of(li, mi)[0], "rmsnorm",
+                               self.gamma[li, 0 if name == "qkv" else 1], self.EPS, Y=y, stream=stream)
+        elif name == "down":
+            self.kq.gemv_fused(W, f, N, K, self.y_of(li, self.gu[li])[0], "swiglu", Y=y, stream=stream)
+        else:
+            self.kq.gemv(W, f, N, K, self.x_of(li, mi)[0], y, stream=stream)
 
 
 class MoE:
@@ -345,6 +381,8 @@ class Streamed:
 def make_workload(name, torch, kq, kqgen, seed):
     if name == "llama8b_chain":
         return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed)
+    if name == "llama8b_layer_fused":
+        return FusedLayer(torch, kq, kqgen, chain_spec("llama8b"), seed)
     if name in ("gemv_q4k_4096", "gateup_q4k", "down_q6k"):
         return Resident(torch, kq, kqgen, chain_spec(name), seed)
     if name.startswith("verify8b_k"):
@@ -597,7 +635,8 @@ def cpu_baseline(args, budget_s=15.0):
         per_token = MOE30B["layers"] * MOE30B["top"] * (2 * MOE30B["ffn"] * row_bytes("q4_k", MOE30B["hidden"])
                                                         + MOE30B["hidden"] * row_bytes("q4_k", MOE30B["ffn"]))
     else:
-        base = {"llama8b_chain": "llama8b", "llama70b_resident": "llama70b", "llama70b_stream": "llama70b"}
+        base = {"llama8b_chain": "llama8b", "llama8b_layer_fused": "llama8b", "llama70b_resident": "llama70b",
+                "llama70b_stream": "llama70b"}
         name = base.get(args.workload, "llama8b" if args.workload.startswith("verify") else args.workload)
         spec = chain_spec(name)
         per_token = sum(N * row_bytes(f, K) for mats in spec for (_, f, N, K, _) in mats)
@@ -610,7 +649,17 @@ def cpu_baseline(args, budget_s=15.0):
             W = kqgen.matrix(fmt, kqgen.tensor_seed(SEED, li, mi), nrows, K)
             x = kqgen.normal_f32(kqgen.tensor_seed(SEED ^ 0x5A5A, li, slot), K)
             t0 = time.perf_counter()
-            oracle.gemv(fmt, W, nrows, K, x, nthreads=cores)
+            if args.workload == "llama8b_layer_fused" and name != "o":
+                # the fused forms: RMSNorm (unit weights) before qkv and
+                # gate|up, the SiLU-gated product of a [g; u] input before down
+                if name == "down":
+                    gu = kqgen.normal_f32(kqgen.tensor_seed(SEED ^ 0x5A5A, li, slot), 2 * K)
+                    oracle.gemv_fused(fmt, W, nrows, K, gu, "swiglu", nthreads=cores)
+                else:
+                    oracle.gemv_fused(fmt, W, nrows, K, x, "rmsnorm", np.ones(K, np.float32), 1e-5,
+                                      nthreads=cores)
+            else:
+                oracle.gemv(fmt, W, nrows, K, x, nthreads=cores)
             t_total += time.perf_counter() - t0
             done_bytes += nrows * row_bytes(fmt, K)
             rows_done += nrows

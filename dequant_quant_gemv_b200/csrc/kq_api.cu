@@ -247,7 +247,8 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     if (err != cudaSuccess) return cuda_fail(err, "device query");
     if (fmt == KQ_FMT_Q6_K && a.nb % 8 != 0)
         return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
-    const size_t extra = a.pro == KQ_PRO_RMSNORM ? kProBytes : 0;  // RMSNorm scratch after the ring
+    // RMSNorm scratch after the ring: 8 columns' sums per super-block, 8 norms
+    const size_t extra = a.pro == KQ_PRO_RMSNORM ? round_up(sizeof(float) * (8 * static_cast<size_t>(a.nb) + 8), 128) : 0;
     const size_t limit = static_cast<size_t>(di.smem_optin) - extra;
     int S = a.ksplit, nbs = a.nbs;
     bool cl = false;

@@ -330,6 +330,29 @@ __device__ __forceinline__ void raise_fault(const GemvArgs& a, volatile int* abo
 
 // ------------------------------------------------------------ producer
 
+// Ask L2 for the bytes the consumers will stage: every column's K range
+// [kb0, kb0 + nbl) blocks of a shared activation copy, and the prologue's
+// second operand (gamma, or the u half of [g; u]).  Issued by the producer
+// at the CTA's start, before the previous grid has finished: a hint only
+// (L2 is where the previous grid's writes land, so nothing stale can be
+// read); the staging then reads from L2 instead of HBM.  16-byte aligned
+// ranges only.
+__device__ __forceinline__ void prefetch_l2(const float* p, uint32_t bytes) {
+    if ((reinterpret_cast<uintptr_t>(p) & 15u) == 0)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ inline void prefetch_activations(const GemvArgs& a, int kb0, int nbl) {
+    if (a.x_seg_stride != 0) return;  // one copy per segment: staged as the segments come
+    const int64_t k0 = static_cast<int64_t>(kb0) * 256;
+    const uint32_t bytes = static_cast<uint32_t>(nbl) * 1024u;
+    for (int j = 0; j < a.ncol_real; ++j) {
+        prefetch_l2(a.x + j * a.ldx + k0, bytes);
+        if (a.pro == 2) prefetch_l2(a.x + j * a.ldx + a.K + k0, bytes);
+    }
+    if (a.pro == 1) prefetch_l2(a.gamma + k0, bytes);
+}
+
 // The producer thread: walks the CTA's stages and brings each one's rows
 // into its ring slot with 1-D bulk copies (no multicast), waiting for the
 // consumers to release a slot before reusing it.  `contiguous`: whole rows
@@ -389,49 +412,121 @@ __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empt
 }
 
 // ------------------------------------------------------------- prologue
+//
+// RMSNorm: W (x o gamma o inv) = inv * W (x o gamma), inv = 1/sqrt(sum(x^2)/K
+// + eps) per column.  The staging pass applies gamma and collects partial
+// sums of squares of the raw x as it loads them; after it, one warp per
+// column combines the partials into inv, and the outputs are scaled by it.
+// SiLU-gated product: the column holds [g; u] (2K floats) and the staging
+// replaces x_i by silu(g_i) * u_i.  Both fetch their second operand (gamma,
+// or u) in the same pass as x.
 
-// One activation after the prologue (i: index within the column's K):
-// as given, RMS-normalised (x_i * gamma_i * inv), or SiLU-gated
-// (silu(x_i) * x_{K+i}, the column holding [g; u]).
-__device__ __forceinline__ float pro_value(const GemvArgs& a, float v, const float* xc, int64_t i, float inv) {
-    if (a.pro == 1) return v * a.gamma[i] * inv;
-    if (a.pro == 2) return v / (1.0f + expf(-v)) * xc[a.K + i];
-    return v;
+// Prologue scratch of the single-column kernel: per consumer group, partial
+// sums of up to kProParts warps for each of 8 columns, then 8 inverse norms.
+constexpr int kProParts = 16;
+constexpr int kProRegion = 4 * (8 * kProParts + 8);
+static_assert(2 * kProRegion <= kProBytes, "prologue scratch");
+__device__ __forceinline__ uint32_t pro_inv_addr(uint32_t region) { return region + 4 * 8 * kProParts; }
+
+// silu(g) * u with the fast exponential and division (relative error of a
+// few 1e-7 for the activations' range; g -> -inf gives -0, g -> +inf g*u).
+__device__ __forceinline__ float silu_gate(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
+// A float4 at p, one 16-byte load when p is 16-byte aligned.
+__device__ __forceinline__ float4 ld_f4(const float* p) {
+    if ((reinterpret_cast<uintptr_t>(p) & 15u) == 0) return *reinterpret_cast<const float4*>(p);
+    return make_float4(p[0], p[1], p[2], p[3]);
 }
 
-// For RMSNorm: 1/sqrt(mean(x^2) + eps) of the first ncol columns of segment
-// `seg` over all of K, by the nthr staging threads in a fixed order (each
-// thread a strided sum, warp butterflies, warps in order), into the
-// prologue scratch `inv` (ncol floats).  Every CTA computes it itself.
-__device__ inline void pro_inv_rms(const GemvArgs& a, int64_t seg, int ncol, int t, int nthr, int bar,
-                                   uint32_t scratch, uint32_t inv) {
-    const int warp = t >> 5, lane = t & 31, nw = nthr >> 5;
-    for (int c = 0; c < ncol; ++c) {
-        const float* xc = a.x + seg * a.x_seg_stride + c * a.ldx;
-        float sq = 0.f;
-        for (int64_t i = t; i < a.K; i += nthr) sq = fmaf(xc[i], xc[i], sq);
+// inv[c] = 1/sqrt(sum_i part[c][i] / K + eps) for the columns c < ncol from
+// `count` partial sums per column, `stride` floats apart: warp c of the
+// staging warps, lane l summing i = l, l + 32, ... in order, then a fixed
+// butterfly; then the staging threads' barrier.  With `nbs` > 0 partial i
+// lives in the shared memory of cluster rank i / nbs (the same offset).
+__device__ inline void rms_finish(float K, float eps, uint32_t part, int stride, int count, uint32_t inv, int ncol,
+                                  int warp, int lane, int bar, int nthr, int nbs) {
+    if (warp < ncol) {
+        float s = 0.f;
+        for (int i = lane; i < count; i += 32) {
+            const uint32_t ad = part + 4 * (warp * stride + i);
+            s += nbs > 0 ? ld_cluster_f32(map_rank(ad, static_cast<uint32_t>(i / nbs))) : ld_s32f(ad);
+        }
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-        if (lane == 0) st_s32f(scratch + 4 * (warp * 8 + c), sq);
+        for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (lane == 0) st_s32f(inv + 4 * warp, 1.0f / sqrtf(s / K + eps));
     }
     named_bar_sync(bar, nthr);
-    if (t < ncol) {
-        float sq = 0.f;
-        for (int w = 0; w < nw; ++w) sq += ld_s32f(scratch + 4 * (w * 8 + t));
-        st_s32f(inv + 4 * t, 1.0f / sqrtf(sq / static_cast<float>(a.K) + a.eps));
-    }
-    named_bar_sync(bar, nthr);
+}
+
+// Sum of squares of one 256-activation block held two float4 per lane (lane
+// l: elements 4l..4l+3 and 128+4l..128+4l+3), in one fixed order: lane-local
+// then a butterfly.  Every warp gets the same value for the same block.
+__device__ __forceinline__ float block_sq(const float4& p, const float4& q) {
+    float s = p.x * p.x;
+    s = fmaf(p.y, p.y, s);
+    s = fmaf(p.z, p.z, s);
+    s = fmaf(p.w, p.w, s);
+    s = fmaf(q.x, q.x, s);
+    s = fmaf(q.y, q.y, s);
+    s = fmaf(q.z, q.z, s);
+    s = fmaf(q.w, q.w, s);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    return s;
 }
 
 // ------------------------------------------------------ activation stage
 
+// Where activation i (0..256*nb-1 of a K range) of a column sits in its
+// fp32 regions (a float offset; the 4 activations i..i+3 sit 2 floats apart,
+// pair members alternating).
+template <int FMT>
+__device__ __forceinline__ int x_offset(int i, int nb) {
+    const int b = i >> 8, within = i & 255;
+    if constexpr (FMT == 1) {
+        // weight 64c + 32*hi + 16h + 4t + k of block b -> region 2b + c/2,
+        // pair (c%2, h, t, k), member hi
+        const int c = within >> 6, w64 = within & 63, hi = w64 >> 5, l = w64 & 31;
+        const int h = l >> 4, t = (l >> 2) & 3;
+        return (2 * b + (c >> 1)) * kRegion + ((c & 1) * 2 + h) * 32 + 8 * t + hi;
+    } else {
+        // weight 128H + 32t + 4s + k of block b = 8i + kappa -> region
+        // (kappa*nb8 + i)*2 + H; pair A = (t0, t2), pair B = (t1, t3)
+        const int H = within >> 7, w128 = within & 127, t = w128 >> 5, sidx = (w128 & 31) >> 2;
+        const int kappa = b & 7, ib = b >> 3;
+        return ((kappa * (nb >> 3) + ib) * 2 + H) * kRegion + 16 * sidx + ((t & 1) ? 8 : 0) + (t >> 1);
+    }
+}
+
+template <int FMT>
+__device__ __forceinline__ void st_x4(uint32_t dst, const float4& v) {
+    st_s32f(dst, v.x);
+    st_s32f(dst + 8, v.y);
+    st_s32f(dst + 16, v.z);
+    st_s32f(dst + 24, v.w);
+}
+
+// Q4_K: the sub-block sums of each staged region (after the fill's barrier).
+template <int FMT, int NCOL>
+__device__ __forceinline__ void stage_x_sums(uint32_t xs, int ct, int nthr, int bar, int nbl, int xcs) {
+    if constexpr (FMT == 1) {
+        const int sums = NCOL * 2 * nbl * 2;
+        for (int it = ct; it < sums; it += nthr) {
+            const int j = it / (2 * nbl * 2);
+            const int rem = it - j * 2 * nbl * 2;
+            const int reg = rem >> 1, cp = rem & 1;
+            const uint32_t xr = xs + 4 * (j * xcs + reg * kRegion);
+            st_s64f(xr + 4 * (128 + 2 * cp), q4k_region_sum(xr, cp));
+        }
+        named_bar_sync(bar, nthr);
+    }
+}
+
 // Stage the activations of segment `seg` (all NCOL columns) into the
 // padded, permuted layout the units read, then (Q4_K) the region sums.
-// PRO: apply the prologue a.pro (a separate instantiation, so the plain
-// loop keeps its loads in flight).
-template <int FMT, int NCOL, bool PRO>
+template <int FMT, int NCOL>
 __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar, int kb0,
-                        int nbl, uint32_t pinv) {
+                        int nbl) {
     // the K range [256*kb0, 256*(kb0+nbl)) in regions laid out for a.nbs blocks
     const float* xg = a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256;
     const int nb = a.nbs;
@@ -449,46 +544,87 @@ __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int
         float4 v;
         if ((reinterpret_cast<uintptr_t>(xc) & 15u) == 0) v = *reinterpret_cast<const float4*>(xc + i);
         else v = make_float4(xc[i], xc[i + 1], xc[i + 2], xc[i + 3]);
-        if constexpr (PRO) {
-            const float* xcol = xc - static_cast<int64_t>(kb0) * 256;  // the column at K index 0
-            const int64_t gi = static_cast<int64_t>(kb0) * 256 + i;
-            const float inv = a.pro == 1 ? ld_s32f(pinv + 4 * (j < a.ncol_real ? j : a.ncol_real - 1)) : 0.f;
-            v = make_float4(pro_value(a, v.x, xcol, gi, inv), pro_value(a, v.y, xcol, gi + 1, inv),
-                            pro_value(a, v.z, xcol, gi + 2, inv), pro_value(a, v.w, xcol, gi + 3, inv));
-        }
-        const int b = i >> 8, within = i & 255;
-        int off;
-        if constexpr (FMT == 1) {
-            // weight 64c + 32*hi + 16h + 4t + k of block b -> region 2b + c/2,
-            // pair (c%2, h, t, k), member hi
-            const int c = within >> 6, w64 = within & 63, hi = w64 >> 5, l = w64 & 31;
-            const int h = l >> 4, t = (l >> 2) & 3;
-            off = (2 * b + (c >> 1)) * kRegion + ((c & 1) * 2 + h) * 32 + 8 * t + hi;
-        } else {
-            // weight 128H + 32t + 4s + k of block b = 8i + kappa -> region
-            // (kappa*nb8 + i)*2 + H; pair A = (t0, t2), pair B = (t1, t3)
-            const int H = within >> 7, w128 = within & 127, t = w128 >> 5, sidx = (w128 & 31) >> 2;
-            const int kappa = b & 7, ib = b >> 3;
-            off = ((kappa * (nb >> 3) + ib) * 2 + H) * kRegion + 16 * sidx + ((t & 1) ? 8 : 0) + (t >> 1);
-        }
-        const uint32_t dst = xs + 4 * (j * xcs + off);
-        st_s32f(dst, v.x);
-        st_s32f(dst + 8, v.y);
-        st_s32f(dst + 16, v.z);
-        st_s32f(dst + 24, v.w);
+        st_x4<FMT>(xs + 4 * (j * xcs + x_offset<FMT>(i, nb)), v);
     }
     named_bar_sync(bar, nthr);
-    if constexpr (FMT == 1) {
-        const int sums = NCOL * 2 * nbl * 2;
-        for (int it = ct; it < sums; it += nthr) {
-            const int j = it / (2 * nbl * 2);
-            const int rem = it - j * 2 * nbl * 2;
-            const int reg = rem >> 1, cp = rem & 1;
-            const uint32_t xr = xs + 4 * (j * xcs + reg * kRegion);
-            st_s64f(xr + 4 * (128 + 2 * cp), q4k_region_sum(xr, cp));
+    stage_x_sums<FMT, NCOL>(xs, ct, nthr, bar, nbl, xcs);
+}
+
+// What the prologue staging reads, by value (the staging below is kept out
+// of line, so that the kernel's main loop compiles as it does without it).
+struct ProStage {
+    const float* xg;   // column 0 of the segment at the K range start
+    const float* gg;   // RMSNorm: gamma at the K range start
+    int64_t K, ldx;
+    int ncol_real, pro, nbs;
+    float eps;
+};
+
+// stage_x with the prologue: the same layout, U items per thread with their
+// loads (x, and gamma or u) in flight together; RMSNorm's partial sums of
+// squares (raw x, per thread in item order, then a butterfly) go to
+// part[column][warp], the inverse norms to pro_inv_addr(part).
+template <int FMT, int NCOL>
+__device__ __noinline__ void stage_x_pro(const ProStage p, uint32_t xs, int ct, int nthr, int bar, int nbl,
+                                         uint32_t part) {
+    constexpr int U = 4;
+    const bool rms = p.pro == 1;
+    const int nb = p.nbs;
+    const int xcs = 2 * nb * kRegion;
+    const int k4 = nbl * 64;
+    const int items = NCOL * k4;
+    float sq[NCOL];
+#pragma unroll
+    for (int j = 0; j < NCOL; ++j) sq[j] = 0.f;
+    for (int it0 = ct; it0 < items; it0 += U * nthr) {
+        float4 v[U], w[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int it = it0 + u * nthr;
+            v[u] = w[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (it < items) {
+                const int j = it / k4;
+                const int i = 4 * (it - j * k4);
+                const float* xc = p.xg + (j < p.ncol_real ? j : p.ncol_real - 1) * p.ldx;
+                v[u] = ld_f4(xc + i);
+                w[u] = ld_f4(rms ? p.gg + i : xc + p.K + i);
+            }
         }
-        named_bar_sync(bar, nthr);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int it = it0 + u * nthr;
+            if (it >= items) break;
+            const int j = it / k4;
+            const int i = 4 * (it - j * k4);
+            float4 t = v[u];
+            if (rms) {
+                const float s = fmaf(t.w, t.w, fmaf(t.z, t.z, fmaf(t.y, t.y, t.x * t.x)));
+#pragma unroll
+                for (int c = 0; c < NCOL; ++c)
+                    if (c == j) sq[c] += s;
+                t = make_float4(t.x * w[u].x, t.y * w[u].y, t.z * w[u].z, t.w * w[u].w);
+            } else {
+                t = make_float4(silu_gate(t.x, w[u].x), silu_gate(t.y, w[u].y), silu_gate(t.z, w[u].z),
+                                silu_gate(t.w, w[u].w));
+            }
+            st_x4<FMT>(xs + 4 * (j * xcs + x_offset<FMT>(i, nb)), t);
+        }
     }
+    if (rms) {
+        const int warp = ct >> 5, lane = ct & 31;
+#pragma unroll
+        for (int c = 0; c < NCOL; ++c) {
+            float s = sq[c];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            if (lane == 0) st_s32f(part + 4 * (c * kProParts + warp), s);
+        }
+    }
+    named_bar_sync(bar, nthr);
+    stage_x_sums<FMT, NCOL>(xs, ct, nthr, bar, nbl, xcs);
+    if (rms)
+        rms_finish(static_cast<float>(p.K), p.eps, part, kProParts, nthr >> 5, pro_inv_addr(part), p.ncol_real,
+                   ct >> 5, ct & 31, bar, nthr, 0);
 }
 
 // ----------------------------------- single column, Q4_K: integer dot path
@@ -498,14 +634,17 @@ __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int
 // consecutive weights are scaled by a power of two 2^sh that puts the
 // group's largest |x| in [2^13, 2^14), rounded to integers xi (|xi| <= 2^14)
 // and stored as a signed high byte xi >> 8 and an unsigned low byte xi & 255
-// (xi = 256*hi + lo).  Per group the staging also keeps Xg = sum of the
-// fp32 activations (fixed order) and P = 2^-sh.  A sub-block's sum S of
-// q*xi is then exact (|S| < 2^23, so exact in fp32 too), and y = sum over
-// sub-blocks of d*sc*P*S - dmin*m*Xg in fp32.  The only approximation
-// beyond fp32 rounding is xi: |x - P*xi| <= P/2 <= 2^-14 * (largest |x| of
-// the group), so |y - y_exact| <= 2^-14 * sum over groups of
-// (max_g |x|) * sum_{i in g} |w_i|.  All-zero quants with zero mins give
-// y = 0 exactly.  (A Q6_K variant measured slower than its fp32 units: its
+// (xi = 256*hi + lo).  Per group the staging also keeps P = 2^-sh and
+// Xg = P * sum of the xi (an exact integer sum, |sum| <= 2^19).  A
+// sub-block's sum S of q*xi is then exact (|S| < 2^23, so exact in fp32
+// too), and y = sum over sub-blocks of d*sc*P*S - dmin*m*Xg in fp32: the
+// exact dot product of the dequantised weights with the rounded activations
+// P*xi, up to fp32 rounding of the per-sub-block terms.  |x - P*xi| <= P/2
+// <= 2^-14 * (largest |x| of the group), so |y - y_exact| <= 2^-14 * sum
+// over groups of (max_g |x|) * sum_{i in g} |w_i|.  All-zero quants with
+// zero mins give y = 0 exactly.  The group's largest |x| and the sum of
+// its xi are one warp reduction each (redux.sync on the bit patterns of
+// |x|, which order like the values, and on the xi).  (A Q6_K variant measured slower than its fp32 units: its
 // 6-bit codes cost more to assemble than the DP4A saves.)
 
 constexpr int kXGroupBytes = 64;  // 32 high bytes, then 32 low bytes
@@ -522,45 +661,50 @@ __device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H) {
 
 // Stage the K range [256*kb0, 256*(kb0+nbl)) of segment `seg` as above,
 // into the regions at `xs`.  One warp per group of 32 activations (lane =
-// position), U groups' loads in flight.  PRO as for stage_x.
+// position), U groups' loads in flight.  PRO: with the prologue a.pro, its
+// second operand (gamma, or u) loaded beside x; RMSNorm's partial sums of
+// squares (raw x, per lane in group order, then a butterfly) go to
+// part[0][warp] and the inverse norm to pro_inv_addr(part).
 template <bool PRO>
 __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, int warp, int nwarps, int lane,
-                                   int bar, int nthr, int kb0, int nbl, uint32_t pinv) {
-    constexpr int U = 4;
+                                   int bar, int nthr, int kb0, int nbl, uint32_t part) {
+    constexpr int U = 8;  // one round of loads for K = 4096 and 16 warps
     const float* xg = a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256;
     const int groups = 8 * nbl;
+    const bool rms = PRO && a.pro == 1;
+    const float* sg = PRO ? (rms ? a.gamma + static_cast<int64_t>(kb0) * 256 : xg + a.K) : nullptr;
+    float sq = 0.f;
     for (int base = warp; base < groups; base += nwarps * U) {
-        float v[U];
+        float v[U], w[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int G = base + nwarps * u;
             v[u] = G < groups ? xg[32 * G + lane] : 0.f;
+            if constexpr (PRO) w[u] = G < groups ? sg[32 * G + lane] : 0.f;
         }
         if constexpr (PRO) {
-            const float* xcol = a.x + seg * a.x_seg_stride;
-            const float inv = a.pro == 1 ? ld_s32f(pinv) : 0.f;
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int G = base + nwarps * u;
-                if (G < groups) v[u] = pro_value(a, v[u], xcol, static_cast<int64_t>(kb0) * 256 + 32 * G + lane, inv);
+                if (rms) {
+                    sq = fmaf(v[u], v[u], sq);
+                    v[u] *= w[u];
+                } else {
+                    v[u] = silu_gate(v[u], w[u]);
+                }
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int G = base + nwarps * u;
             if (G >= groups) break;  // warp-uniform
-            float m = fabsf(v[u]), X = v[u];
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) {
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-                X += __shfl_xor_sync(0xffffffffu, X, off);
-            }
+            const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(v[u]) & 0x7FFFFFFFu);
             int sh = 0;
-            if (m > 0.f) {
-                sh = 13 - (static_cast<int>(__float_as_uint(m) >> 23) - 127);
+            if (mb != 0u) {
+                sh = 13 - (static_cast<int>(mb >> 23) - 127);
                 sh = sh > 100 ? 100 : sh < -100 ? -100 : sh;
             }
             const int xi = __float2int_rn(v[u] * __int_as_float((sh + 127) << 23));
+            const float X = static_cast<float>(__reduce_add_sync(0xffffffffu, xi)) * __int_as_float((127 - sh) << 23);
             const uint32_t xr = x_region(xs, G >> 3, (G >> 2) & 1), k = G & 3;
             asm volatile("st.shared.u8 [%0], %1;" ::"r"(xr + kXGroupBytes * k + lane), "r"(xi >> 8) : "memory");
             asm volatile("st.shared.u8 [%0], %1;" ::"r"(xr + kXGroupBytes * k + 32 + lane), "r"(xi & 255)
@@ -572,7 +716,15 @@ __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, 
             }
         }
     }
+    if (rms) {
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        if (lane == 0) st_s32f(part + 4 * warp, sq);
+    }
     named_bar_sync(bar, nthr);
+    if (rms)
+        rms_finish(static_cast<float>(a.K), a.eps, part, kProParts, nwarps, pro_inv_addr(part), 1, warp, lane, bar,
+                   nthr, 0);
 }
 
 __device__ __forceinline__ float byte_f(uint32_t w, int k) { return static_cast<float>((w >> (8 * k)) & 0xFFu); }
@@ -646,9 +798,14 @@ __device__ __forceinline__ void q6k_unit_dispatch(int kappa, uint32_t row0, int 
 // prologue (PRO).
 template <int FMT, int NCOL, bool INT, bool PRO>
 __device__ __forceinline__ void stage_all(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar,
-                                          int kb0, int nbl, uint32_t pinv) {
-    if constexpr (INT) stage_x_int<PRO>(a, seg, xs, ct >> 5, nthr >> 5, ct & 31, bar, nthr, kb0, nbl, pinv);
-    else stage_x<FMT, NCOL, PRO>(a, seg, xs, ct, nthr, bar, kb0, nbl, pinv);
+                                          int kb0, int nbl, uint32_t part) {
+    if constexpr (INT) stage_x_int<PRO>(a, seg, xs, ct >> 5, nthr >> 5, ct & 31, bar, nthr, kb0, nbl, part);
+    else if constexpr (PRO)
+        stage_x_pro<FMT, NCOL>(ProStage{a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256,
+                                        a.pro == 1 ? a.gamma + static_cast<int64_t>(kb0) * 256 : nullptr, a.K, a.ldx,
+                                        a.ncol_real, a.pro, a.nbs, a.eps},
+                               xs, ct, nthr, bar, nbl, part);
+    else stage_x<FMT, NCOL>(a, seg, xs, ct, nthr, bar, kb0, nbl);
 }
 
 // ------------------------------------------------------------ the kernel
@@ -696,9 +853,11 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     const int srow = a.ksplit > 1 ? a.nbs * BS : static_cast<int>(a.row_bytes);  // staged row stride
 
     if (warp == 0) {
-        if (lane == 0)
+        if (lane == 0) {
+            prefetch_activations(a, kb0, nbl);
             produce_stages<BS>(a, full, empty, abort_flag, sbuf, rp_begin, rp_end, rps, ns, kb0, nbl, srow,
                                a.ksplit == 1);
+        }
         return;
     }
 
@@ -732,7 +891,6 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
         kappa = cw;
         u_rp = lane / LRw;
         const int u = lane - u_rp * LRw;
-        const int nb8 = nb >> 3;
         u_active = u < 2 * (nbl >> 3);
         const int i = u >> 1;
         u_H = u & 1;
@@ -761,12 +919,14 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
     Stage st;
     int64_t staged_seg = -1;
-    const uint32_t pro_s = smem_u32(smem + a.pro_offset), pinv_s = pro_s + 4 * 16 * 8;
+    // prologue scratch: one region for a shared copy, else the group's own
+    const uint32_t pro_r = smem_u32(smem + a.pro_offset) + (shared_x ? 0 : g * kProRegion);
+    const uint32_t pro_inv = pro_inv_addr(pro_r);  // RMSNorm: the columns' 1/rms
+    float rinv = 1.f;  // RMSNorm: the column's 1/rms, read once per staging (single column)
     if (shared_x) {
         // one activation copy for all groups, staged by all consumer threads
-        if (PRO && a.pro == 1)
-            pro_inv_rms(a, 0, a.ncol_real, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, pro_s, pinv_s);
-        stage_all<FMT, NCOL, INT, PRO>(a, 0, xs_s, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, kb0, nbl, pinv_s);
+        stage_all<FMT, NCOL, INT, PRO>(a, 0, xs_s, ct_all, NG * kConsumers, NG == 2 ? 3 : 1, kb0, nbl, pro_r);
+        if (PRO && a.pro == 1) rinv = ld_s32f(pro_inv);
         staged_seg = 0;
     }
     int own = 0;  // stages this group has consumed
@@ -776,10 +936,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             // (with warps running free between stages, all of the group must
             // be done with the previous segment's activations first)
             if (direct && staged_seg >= 0) named_bar_sync(gbar, kConsumers);
-            // (per-segment activations: a group's own scratch half)
-            const uint32_t gpro = pro_s + 4 * 8 * 8 * g, ginv = pinv_s + 4 * 8 * g;
-            if (PRO && a.pro == 1) pro_inv_rms(a, st.seg, a.ncol_real, ct, kConsumers, gbar, gpro, ginv);
-            stage_all<FMT, NCOL, INT, PRO>(a, st.seg, xs_s, ct, kConsumers, gbar, kb0, nbl, ginv);
+            stage_all<FMT, NCOL, INT, PRO>(a, st.seg, xs_s, ct, kConsumers, gbar, kb0, nbl, pro_r);
+            if (PRO && a.pro == 1) rinv = ld_s32f(pro_inv);
             staged_seg = st.seg;
         }
         const int slot = it.slot;
@@ -827,7 +985,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
                 for (int r = 0; r < 2; ++r) {
                     const int row = 2 * u_rp + r;
                     if (row >= st.nrows) continue;
-                    const float v = valid ? out[r][0] : 0.f;
+                    float v = valid ? out[r][0] : 0.f;
+                    if constexpr (PRO) v *= rinv;
                     if (a.ksplit == 1) a.y[st.seg * a.y_seg_stride + st.row0 + row] = v;
                     else a.partial[static_cast<int64_t>(ks) * a.N + st.row0 + row] = v;
                 }
@@ -857,6 +1016,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             float v = 0.f;
             if (valid) {
                 for (int p = 0; p < parts; ++p) v += ld_s32f(wb + 4 * (((rp * parts + p) * 2 + r) * NCOL + j));
+                if constexpr (PRO) v *= NCOL == 1 ? rinv : (a.pro == 1 ? ld_s32f(pro_inv + 4 * j) : 1.f);
             }
             if (j < a.ncol_real) {
                 if (a.ksplit == 1) a.y[st.seg * a.y_seg_stride + j * a.ldy + st.row0 + row] = v;

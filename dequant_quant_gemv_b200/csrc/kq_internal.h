@@ -52,10 +52,11 @@ struct GemvArgs {
     int pro_offset;          // RMSNorm scratch (kProBytes) after the stage ring
 };
 
-// Shared-memory scratch of RMSNorm (both kernels): per-warp partial sums of
-// squares (16 warps x 8 columns) and the columns' 1/rms.  Reserved only by
-// launches that normalise.
-constexpr int kProBytes = 1024;
+// Shared-memory scratch of RMSNorm in the single-column kernel: per consumer
+// group, partial sums of squares (16 warps x 8 columns) and the columns'
+// 1/rms.  Reserved only by launches that normalise.  (The tensor-core
+// kernel sizes its own: 8 columns x the row's super-blocks, and 8 floats.)
+constexpr int kProBytes = 2 * 4 * (8 * 16 + 8);
 constexpr int kHeadBytes = 256;  // barriers and flags
 
 struct LaunchPlan {

@@ -162,23 +162,28 @@ __device__ __forceinline__ void b_slot(int w, int& s, int& q) {
 // the block into [2^14, 2^15)) and its sums by 2^(sh-5); `bscale` gets
 // (2^-sh, 2^(5-sh)) per block and column.  Columns >= ncol_real are zero.
 // One warp per (column, block) item, two float4 per lane, several items'
-// loads in flight.  PRO: apply the prologue a.pro (a separate
-// instantiation, so the plain loop keeps its loads in flight).
+// loads in flight.  PRO: with the prologue a.pro, its second operand
+// (gamma, or u) loaded beside x; for RMSNorm each item's sum of squares of
+// the raw x (block_sq) goes to part[col][kb0 + bl] (a.nb per column), and
+// with `publish` (a cluster) each storing lane also releases it at cluster
+// scope.
 template <int FMT, int NT, bool PRO>
 __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, int nwarps, int lane, int bar,
-                         int kb0, int nbl, uint32_t pinv) {
+                         int kb0, int nbl, uint32_t part, bool publish) {
     constexpr int NC = 4 * NT;
     constexpr int U = 4;  // items per warp in flight
     const float* xg = a.x + static_cast<int64_t>(kb0) * 256;
     const int kr = a.ncol_real;
     const int items = NC * nbl;
+    const bool rms = PRO && a.pro == 1;
     for (int base = cw; base < items; base += nwarps * U) {
-        float4 v[U][2];
+        float4 v[U][2], w[U][2];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int it = base + nwarps * u;
             const int col = it / nbl, bl = it - col * nbl;
             v[u][0] = v[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if constexpr (PRO) w[u][0] = w[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (it < items && col < kr) {
                 const float* xc = xg + col * a.ldx + 256 * bl + 4 * lane;
                 if ((reinterpret_cast<uintptr_t>(xc) & 15u) == 0) {
@@ -188,6 +193,11 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                     v[u][0] = make_float4(xc[0], xc[1], xc[2], xc[3]);
                     v[u][1] = make_float4(xc[128], xc[129], xc[130], xc[131]);
                 }
+                if constexpr (PRO) {
+                    const float* sc = rms ? a.gamma + static_cast<int64_t>(kb0 + bl) * 256 + 4 * lane : xc + a.K;
+                    w[u][0] = ld_f4(sc);
+                    w[u][1] = ld_f4(sc + 128);
+                }
             }
         }
         if constexpr (PRO) {
@@ -195,16 +205,20 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
             for (int u = 0; u < U; ++u) {
                 const int it = base + nwarps * u;
                 const int col = it / nbl, bl = it - col * nbl;
-                if (it >= items || col >= kr) continue;
-                const float* xcol = a.x + col * a.ldx;
-                const float inv = a.pro == 1 ? ld_s32f(pinv + 4 * col) : 0.f;
+                if (it >= items || col >= kr) continue;  // warp-uniform
+                if (rms) {
+                    const float sq = block_sq(v[u][0], v[u][1]);
+                    if (lane == 0) {
+                        st_s32f(part + 4u * (col * a.nb + kb0 + bl), sq);
+                        if (publish) fence_acq_rel_cluster();
+                    }
+                }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int64_t gi = static_cast<int64_t>(kb0 + bl) * 256 + 128 * h + 4 * lane;
-                    v[u][h] = make_float4(pro_value(a, v[u][h].x, xcol, gi, inv),
-                                          pro_value(a, v[u][h].y, xcol, gi + 1, inv),
-                                          pro_value(a, v[u][h].z, xcol, gi + 2, inv),
-                                          pro_value(a, v[u][h].w, xcol, gi + 3, inv));
+                    const float4 t = v[u][h], m = w[u][h];
+                    v[u][h] = rms ? make_float4(t.x * m.x, t.y * m.y, t.z * m.z, t.w * m.w)
+                                  : make_float4(silu_gate(t.x, m.x), silu_gate(t.y, m.y), silu_gate(t.z, m.z),
+                                                silu_gate(t.w, m.w));
                 }
             }
         }
@@ -479,6 +493,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 2 * kMaxStages * 8);
     uint64_t* recv = reinterpret_cast<uint64_t*>(smem + 2 * kMaxStages * 8 + 8);  // [2], rank 0
     uint64_t* sent = recv + 2;                                                    // [2], ranks > 0
+    uint64_t* pready = sent + 2;  // RMSNorm in a cluster: the other ranks' partial sums are in place
     float* bscale = reinterpret_cast<float*>(smem + a.xscale_offset);  // [block][column] (2^-sh, 2^(5-sh))
     uint8_t* sbuf = smem + a.sbuf_offset;
 
@@ -497,6 +512,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
                 mbar_init(&recv[i], static_cast<uint32_t>((S - 1) * NRED));
                 mbar_init(&sent[i], 1);
             }
+        if (PRO && cl) mbar_init(pready, static_cast<uint32_t>(S - 1));
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -515,8 +531,10 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
     const uint32_t rem = static_cast<uint32_t>(kb0 * BS) & 15u;  // Q6_K ranges may start off a 16-byte boundary
 
     if (warp == 0) {
-        if (lane == 0)
+        if (lane == 0) {
+            prefetch_activations(a, kb0, nbl);
             produce_stages<BS>(a, full, empty, abort_flag, sbuf, rp_begin, rp_end, rps, ns, kb0, nbl, a.sp, false);
+        }
         __syncwarp();
     } else {
         // ------------------------------------------------------ consumers
@@ -533,9 +551,28 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
         const uint32_t sbuf_s = smem_u32(sbuf);
         pdl_wait();
         pdl_launch_dependents();
-        const uint32_t pro_s = smem_u32(smem + a.pro_offset), pinv_s = pro_s + 4 * 16 * 8;
-        if (PRO && a.pro == 1) pro_inv_rms(a, 0, a.ncol_real, ct_all, NG * kConsumers, 3, pro_s, pinv_s);
-        stage_xb<FMT, NT, PRO>(a, xb_s, bscale, ct_all >> 5, NG * kConsumerWarps, lane, 3, kb0, nbl, pinv_s);
+        // RMSNorm scratch: partial sums of squares [column][super-block], then
+        // the columns' 1/rms
+        const uint32_t pro_s = smem_u32(smem + a.pro_offset), pro_inv = pro_s + 4u * 8 * a.nb;
+        stage_xb<FMT, NT, PRO>(a, xb_s, bscale, ct_all >> 5, NG * kConsumerWarps, lane, 3, kb0, nbl, pro_s, cl);
+        if constexpr (PRO) {
+            if (a.pro == 1) {
+                // each CTA of a cluster has its own blocks' sums: tell the
+                // other ranks they are in place, wait for theirs, and read
+                // them from their shared memory
+                if (cl && ct_all == 0)
+                    for (int r = 0; r < S; ++r)
+                        if (r != ks) mbar_arrive_remote(map_rank(smem_u32(pready), static_cast<uint32_t>(r)));
+                if (cl && (ct_all >> 5) < a.ncol_real && !mbar_wait_cluster_bounded(pready, 0, abort_flag))
+                    raise_fault(a, abort_flag, 6);
+                rms_finish(static_cast<float>(a.K), a.eps, pro_s, a.nb, a.nb, pro_inv, a.ncol_real, ct_all >> 5, lane,
+                           3, NG * kConsumers, cl ? a.nbs : 0);
+            }
+        }
+        // RMSNorm: this thread's outputs are all of column ct % NC (NC
+        // divides the group's thread count), so its 1/rms is read once
+        float rinv = 1.f;
+        if (PRO && a.pro == 1) rinv = ld_s32f(pro_inv + 4u * (ct % NC));
 
         // byte selectors: scales of chunk q (half 0) / q+4 (half 1) sit at
         // bytes 2*(q/2), 2*(q/2)+1 of either half; mins 2q, 2q+1 at bytes
@@ -587,6 +624,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
                     float v = 0.f;
 #pragma unroll
                     for (int w = 0; w < kConsumerWarps; ++w) v += ld_s32f(wb + 4u * ((w * 16 + row) * NC + j));
+                    if constexpr (PRO) v *= rinv;
                     if (S == 1) a.y[j * a.ldy + st.row0 + row] = v;
                     else a.partial[(static_cast<int64_t>(ks) * a.ncol_real + j) * a.N + st.row0 + row] = v;
                 }
@@ -601,6 +639,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
                 if (ks == 0) {
                     if (!mbar_wait_cluster_bounded(&recv[p], (si >> 1) & 1, abort_flag)) raise_fault(a, abort_flag, 6);
                     for (int r = 1; r < S; ++r) v += ld_s32f(red_s + 4u * ((p * (S - 1) + r - 1) * NRED + ct));
+                    if constexpr (PRO) v *= rinv;
                     if (row < st.nrows && j < a.ncol_real) a.y[j * a.ldy + st.row0 + row] = v;
                     named_bar_sync(4 + g_id, NRED);  // every value of buffer p read
                     if (ct < S - 1 && si + 2 < total) mbar_arrive_remote(map_rank(smem_u32(&sent[p]), ct + 1));

@@ -87,3 +87,22 @@ def test_invalid_prologues_are_rejected():
     pro = kq.Prologue(2, None, 0.0)
     st = L.kq_gemv_fused(W.data_ptr(), 1, N, K, X.data_ptr(), K, 2, pro, Y.data_ptr(), N, None)
     assert st == 1
+
+
+@pytest.mark.parametrize("H,F", [(512, 2048), (4096, 14336)])
+def test_chained_ffn_each_stage_matches_oracle(H, F):
+    """The decode FFN as the fused path runs it: gate|up (2F x H, Q4_K) with
+    RMSNorm on x, then down (H x F, Q6_K) reading gate|up's device output
+    [g; u] through the SiLU-gated prologue.  Each stage is compared with the
+    oracle on that stage's own inputs (down on the device's [g; u])."""
+    Wgu = matrix("q4_k", 730, 2 * F, H)
+    Wdn = matrix("q6_k", 731, H, F)
+    x = x_vec(732, H)
+    g = x_vec(733, H) * np.float32(0.1) + np.float32(1.0)
+    GU = kq.gemv_fused(dev(Wgu), "q4_k", 2 * F, H, dev(x), "rmsnorm", dev(g), 1e-5)
+    Y = kq.gemv_fused(dev(Wdn), "q6_k", H, F, GU, "swiglu")
+    gu_host = GU.cpu().numpy()
+    gu_ref, gu_s = oracle.gemv_fused("q4_k", Wgu, 2 * F, H, x[None, :], "rmsnorm", g, 1e-5, nthreads=0)
+    assert_close(GU[0], gu_ref[0], gu_s[0], "gate|up")
+    y_ref, y_s = oracle.gemv_fused("q6_k", Wdn, H, F, gu_host, "swiglu", nthreads=0)
+    assert_close(Y[0], y_ref[0], y_s[0], "down")
