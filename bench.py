@@ -79,8 +79,11 @@ def chain_spec(kind):
 
 WORKLOADS = {
     "llama8b_chain": "Llama-3.1-8B-shaped decode chain, 32 layers, Q4_K + Q6_K down, batch 1",
+    "llama8b_chain_steps": "the same chain through kq_gemv_steps (16 matvecs per persistent launch, each "
+                           "waiting for the one before)",
     "llama8b_layer_fused": "the 8B-shaped chain with RMSNorm fused into qkv and gate|up and the SiLU-gated "
                            "product of gate|up's output fused into down",
+    "llama8b_layer_fused_steps": "the fused-glue chain through kq_gemv_steps",
     "gemv_q4k_4096": "single Q4_K GEMV 4096 x 4096, batch 1 (64 distinct copies rotated)",
     "gateup_q4k": "Q4_K GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
     "down_q6k": "Q6_K GEMV 4096 x 14336 (8B down), 8 distinct copies rotated",
@@ -91,6 +94,7 @@ WORKLOADS = {
     "moe30b": "Qwen3-30B-A3B-shaped MoE GEMVs: 48 layers x 128 experts (gate|up 1536x2048, down 2048x768, "
               "Q4_K), top-8 routed ids per token, batch 1",
     "llama70b_resident": "Llama-3.3-70B-shaped decode chain, 80 layers, Q4_K + Q6_K down, resident in HBM",
+    "llama70b_resident_steps": "the 70B-shaped resident chain through kq_gemv_steps",
     "llama70b_stream": "Llama-3.3-70B-shaped decode chain, 80 layers, weights in pinned host memory streamed "
                        "through 4 device layer slots",
 }
@@ -162,8 +166,9 @@ class Resident:
 
     graphable = True
 
-    def __init__(self, torch, kq, kqgen, spec, seed, k=1):
+    def __init__(self, torch, kq, kqgen, spec, seed, k=1, steps=False):
         self.torch, self.kq, self.spec, self.k = torch, kq, spec, k
+        self.use_steps = steps
         self.launches = [(li, mi) for li, mats in enumerate(spec) for mi in range(len(mats))]
         self.weight_bytes = sum(N * row_bytes(f, K) for mats in spec for (_, f, N, K, _) in mats)
         # activations: one slot per (layer, x-slot), k columns each
@@ -190,6 +195,29 @@ class Resident:
                 row.append(torch.from_numpy(host).cuda())
             self.W.append(row)
         torch.cuda.synchronize()
+        if steps:
+            self.build_steps()
+
+    # ---- the chain as one list of steps (kq_gemv_steps)
+    def step_args(self, li, mi):
+        """(x, prologue kind, gamma) of matrix mi of layer li."""
+        return self.x_of(li, mi)[0], "none", None
+
+    def build_steps(self):
+        """Every matrix of the chain as a step of kq_gemv_steps, each marked
+        `after`: as in decode, a step starts only when the step before it has
+        finished on the whole GPU (the launches-per-matrix order)."""
+        self.steps, self.kind_steps = [], {}
+        for li, mi in self.launches:
+            name, f, N, K, _ = self.spec[li][mi]
+            x, kind, gamma = self.step_args(li, mi)
+            st = self.kq.make_step(self.W[li][mi], f, N, K, x, self.y_of(li, mi)[0], kind, gamma, 1e-5, after=True)
+            self.steps.append(st)
+            self.kind_steps.setdefault(name, []).append(st)
+        self.launches_per_step = -(-len(self.steps) // 16)
+
+    def launch_kind(self, name, stream):
+        self.kq.gemv_steps(self.kind_steps[name], stream=stream)
 
     def x_of(self, li, mi):
         off, K = self.xslot[(li, self.spec[li][mi][4])]
@@ -207,6 +235,9 @@ class Resident:
             self.kq.gemv_multi(self.W[li][mi], f, N, K, self.x_of(li, mi), self.y_of(li, mi), stream=stream)
 
     def step(self, stream):
+        if self.use_steps:
+            self.kq.gemv_steps(self.steps, stream=stream)
+            return
         for li, mi in self.launches:
             self.launch(li, mi, stream)
 
@@ -232,7 +263,7 @@ class FusedLayer(Resident):
 
     EPS = 1e-5
 
-    def __init__(self, torch, kq, kqgen, spec, seed):
+    def __init__(self, torch, kq, kqgen, spec, seed, steps=False):
         fused = [[m if m[0] != "down" else m[:4] + (None,) for m in mats] for mats in spec]
         super().__init__(torch, kq, kqgen, fused, seed)
         self.gu = {li: mi for li, mats in enumerate(fused) for mi, m in enumerate(mats) if m[0] == "gate_up"}
@@ -241,6 +272,17 @@ class FusedLayer(Resident):
         g = 1.0 + 0.1 * kqgen.normal_f32(seed ^ 0x6A3, 2 * n * K).astype(np.float32)
         self.gamma = torch.from_numpy(g).cuda().view(n, 2, K)
         torch.cuda.synchronize()
+        self.use_steps = steps
+        if steps:
+            self.build_steps()
+
+    def step_args(self, li, mi):
+        name = self.spec[li][mi][0]
+        if name == "qkv" or name == "gate_up":
+            return self.x_of(li, mi)[0], "rmsnorm", self.gamma[li, 0 if name == "qkv" else 1]
+        if name == "down":
+            return self.y_of(li, self.gu[li])[0], "swiglu", None
+        return self.x_of(li, mi)[0], "none", None
 
     def launch(self, li, mi, stream):
         name, f, N, K, _ = self.spec[li][mi]
@@ -379,18 +421,19 @@ class Streamed:
 
 
 def make_workload(name, torch, kq, kqgen, seed):
-    if name == "llama8b_chain":
-        return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed)
-    if name == "llama8b_layer_fused":
-        return FusedLayer(torch, kq, kqgen, chain_spec("llama8b"), seed)
+    if name in ("llama8b_chain", "llama8b_chain_steps"):
+        return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed, steps=name.endswith("_steps"))
+    if name in ("llama8b_layer_fused", "llama8b_layer_fused_steps"):
+        return FusedLayer(torch, kq, kqgen, chain_spec("llama8b"), seed, steps=name.endswith("_steps"))
     if name in ("gemv_q4k_4096", "gateup_q4k", "down_q6k"):
         return Resident(torch, kq, kqgen, chain_spec(name), seed)
     if name.startswith("verify8b_k"):
-        return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed, k=int(name[len("verify8b_k"):]))
+        k = int(name[len("verify8b_k"):])
+        return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed, k=k)
     if name == "moe30b":
         return MoE(torch, kq, kqgen, seed)
-    if name == "llama70b_resident":
-        return Resident(torch, kq, kqgen, chain_spec("llama70b"), seed)
+    if name in ("llama70b_resident", "llama70b_resident_steps"):
+        return Resident(torch, kq, kqgen, chain_spec("llama70b"), seed, steps=name.endswith("_steps"))
     if name == "llama70b_stream":
         return Streamed(torch, kq, kqgen, chain_spec("llama70b"), seed)
     raise KeyError(name)
@@ -536,8 +579,11 @@ def bench_kq(args, rank, world):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 for _ in range(reps):
-                    for (a, b) in kd["launches"]:
-                        wl.launch(a, b, stream)
+                    if getattr(wl, "use_steps", False):
+                        wl.launch_kind(name, stream)
+                    else:
+                        for (a, b) in kd["launches"]:
+                            wl.launch(a, b, stream)
             g.replay()
             torch.cuda.synchronize()
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -594,19 +640,21 @@ def bench_kq(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, kqgen)",
         "tok_per_s": round(tok_s, 3), "frac_of_hbm_peak": round(gbs / world / hbm, 4),
         "config": {"workload": args.workload, "desc": WORKLOADS[args.workload],
-                   "weight_bytes_per_step": wl.weight_bytes, "launches_per_step": len(wl.launches),
+                   "weight_bytes_per_step": wl.weight_bytes,
+                   "launches_per_step": wl.launches_per_step if getattr(wl, "use_steps", False) else len(wl.launches),
                    "columns": k, "batch": 1, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (no flush)" if wl.weight_bytes > 2 * 126e6 else "rotating copies"},
         "e2e": {"value": round(job_rate(wl.weight_bytes, args.steps, world, ems) / 1e9, 2), "unit": "GB/s",
                 "tok_per_s": round(job_rate(k, args.steps, world, ems), 3),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
-        "gpu_launches": len(wl.launches) * args.steps,
+        "gpu_launches": (wl.launches_per_step if getattr(wl, "use_steps", False) else len(wl.launches)) * args.steps,
     }
     if per_kind:
         dom = max(per_kind, key=lambda n: per_kind[n]["share"])
         dk = per_kind[dom]
-        kname = "mma_kernel (tensor cores)" if k >= 2 else "gemv_kernel"
+        kname = ("mma_kernel (tensor cores)" if k >= 2 else
+                 "steps_kernel (multi-step launch)" if getattr(wl, "use_steps", False) else "gemv_kernel")
         result["roofline"] = {"bound": "hbm", "kernel": f"{kname} {dk['fmt']} {dom} {dk['N']}x{dk['K']}",
                               "achieved": dk["gbs"], "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
                               "frac": round(dk["gbs"] / hbm, 4),
@@ -635,8 +683,9 @@ def cpu_baseline(args, budget_s=15.0):
         per_token = MOE30B["layers"] * MOE30B["top"] * (2 * MOE30B["ffn"] * row_bytes("q4_k", MOE30B["hidden"])
                                                         + MOE30B["hidden"] * row_bytes("q4_k", MOE30B["ffn"]))
     else:
-        base = {"llama8b_chain": "llama8b", "llama8b_layer_fused": "llama8b", "llama70b_resident": "llama70b",
-                "llama70b_stream": "llama70b"}
+        base = {"llama8b_chain": "llama8b", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
+                "llama8b_layer_fused_steps": "llama8b", "llama70b_resident": "llama70b",
+                "llama70b_resident_steps": "llama70b", "llama70b_stream": "llama70b"}
         name = base.get(args.workload, "llama8b" if args.workload.startswith("verify") else args.workload)
         spec = chain_spec(name)
         per_token = sum(N * row_bytes(f, K) for mats in spec for (_, f, N, K, _) in mats)
@@ -649,7 +698,7 @@ def cpu_baseline(args, budget_s=15.0):
             W = kqgen.matrix(fmt, kqgen.tensor_seed(SEED, li, mi), nrows, K)
             x = kqgen.normal_f32(kqgen.tensor_seed(SEED ^ 0x5A5A, li, slot), K)
             t0 = time.perf_counter()
-            if args.workload == "llama8b_layer_fused" and name != "o":
+            if args.workload.startswith("llama8b_layer_fused") and name != "o":
                 # the fused forms: RMSNorm (unit weights) before qkv and
                 # gate|up, the SiLU-gated product of a [g; u] input before down
                 if name == "down":
@@ -681,7 +730,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.steps is None:
-        args.steps = {"llama70b_stream": 3, "llama70b_resident": 50}.get(args.workload, 300)
+        args.steps = {"llama70b_stream": 3, "llama70b_resident": 50, "llama70b_resident_steps": 50}.get(args.workload,
+                                                                                                       300)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
 

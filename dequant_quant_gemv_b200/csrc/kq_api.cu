@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/kq.h"
 #include "kq_device.cuh"
@@ -573,6 +574,166 @@ int kq_gemv_multi(const void* W, int fmt, int64_t N, int64_t K, const float* x, 
 int kq_gemv_fused(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx, int k,
                   const kq_prologue* pro, float* y, int64_t ldy, kq_stream_t stream) {
     return gemv_columns(W, fmt, N, K, x, ldx, k, pro, y, ldy, stream);
+}
+
+int kq_gemv_steps(const kq_step* steps, int n_steps, kq_stream_t stream) {
+    g_last_error[0] = 0;
+    if (n_steps < 0) return fail(KQ_ERR_INVALID_ARG, "n_steps=%d < 0", n_steps);
+    if (n_steps == 0) return KQ_OK;
+    if (!steps) return fail(KQ_ERR_INVALID_ARG, "steps is NULL");
+    DevInfo di;
+    cudaError_t err = dev_info(di);
+    if (err != cudaSuccess) return cuda_fail(err, "device query");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // validate and plan every step (the single-column kernel's schedule)
+    struct Planned {
+        StepArgs a;
+        size_t stage, wp, xs;
+        bool zero;  // K = 0: y is all zeros
+        bool skip;  // N = 0: nothing to do
+    };
+    std::vector<Planned> pl(static_cast<size_t>(n_steps));
+    for (int i = 0; i < n_steps; ++i) {
+        const kq_step& q = steps[i];
+        Planned& P = pl[static_cast<size_t>(i)];
+        P.zero = P.skip = false;
+        int st = check_matrix(q.W, q.fmt, q.N, q.K);
+        const int kind = q.pro.kind;
+        if (st == KQ_OK && kind != KQ_PRO_NONE && kind != KQ_PRO_RMSNORM && kind != KQ_PRO_SWIGLU)
+            st = fail(KQ_ERR_INVALID_ARG, "unknown prologue kind %d", kind);
+        if (st == KQ_OK && kind == KQ_PRO_RMSNORM && (!q.pro.gamma || !aligned(q.pro.gamma, 4) || !(q.pro.eps > 0.f)))
+            st = fail(KQ_ERR_INVALID_ARG, "RMSNorm needs a 4-byte aligned gamma and eps > 0");
+        if (st == KQ_OK && q.N > 0 && (!q.y || !aligned(q.y, 4))) st = fail(KQ_ERR_INVALID_ARG, "y is NULL or misaligned");
+        if (st == KQ_OK && q.N > 0 && q.K > 0 && (!q.x || !aligned(q.x, 4)))
+            st = fail(KQ_ERR_INVALID_ARG, "x is NULL or misaligned");
+        if (st == KQ_OK && q.N > 0 && q.K > 0) {
+            GemvArgs a = {};
+            a.W = static_cast<const uint8_t*>(q.W);
+            a.N = q.N;
+            a.K = q.K;
+            a.row_bytes = static_cast<int64_t>(kq_row_bytes(q.fmt, q.K));
+            a.nb = static_cast<int>(q.K / 256);
+            a.n_seg = 1;
+            a.E = 1;
+            a.ksplit = 1;
+            a.nbs = a.nb;
+            a.ncol_real = 1;
+            a.pro = kind;
+            LaunchPlan lp;
+            st = plan_gemv(q.fmt, 1, a, lp);
+            if (st == KQ_OK) {
+                StepArgs& sa = P.a;
+                sa = StepArgs{};
+                sa.W = a.W;
+                sa.x = q.x;
+                sa.y = q.y;
+                sa.gamma = kind == KQ_PRO_RMSNORM ? q.pro.gamma : nullptr;
+                sa.N = q.N;
+                sa.row_bytes = a.row_bytes;
+                sa.K = static_cast<int>(q.K);
+                sa.nb = a.nb;
+                sa.fmt = q.fmt;
+                sa.pro = kind;
+                sa.eps = kind == KQ_PRO_RMSNORM ? q.pro.eps : 0.f;
+                sa.after = q.after != 0;
+                sa.ps = a.ps;
+                sa.lanes_per_rp = a.lanes_per_rp;
+                sa.parts = a.parts;
+                P.stage = static_cast<size_t>(a.stage_bytes);
+                P.wp = static_cast<size_t>(a.xs_offset - a.wp_offset);
+                P.xs = static_cast<size_t>(a.sbuf_offset - a.xs_offset);
+            }
+        }
+        if (st != KQ_OK) {
+            char msg[512];
+            snprintf(msg, sizeof(msg), "%s", g_last_error);
+            return fail(st, "step %d: %s", i, msg);
+        }
+        P.skip = q.N == 0;
+        P.zero = !P.skip && q.K == 0;
+    }
+    // launches: runs of at most kMaxSteps steps, ended also by a K = 0 step
+    // (its zeros are written in stream order between launches)
+    struct Op {
+        bool zero;
+        float* y;
+        int64_t N;
+        StepsArgs args;
+        size_t smem;
+    };
+    std::vector<Op> ops;
+    std::vector<int> run;
+    auto close_run = [&]() -> int {
+        if (run.empty()) return KQ_OK;
+        Op op = {};
+        op.zero = false;
+        size_t slot = 0, wp = 0, xs = 0;
+        bool rms = false;
+        for (size_t j = 0; j < run.size(); ++j) {
+            const Planned& P = pl[static_cast<size_t>(run[j])];
+            op.args.st[j] = P.a;
+            slot = P.stage > slot ? P.stage : slot;
+            wp = P.wp > wp ? P.wp : wp;
+            xs = P.xs > xs ? P.xs : xs;
+            rms = rms || P.a.pro == KQ_PRO_RMSNORM;
+        }
+        op.args.n = static_cast<int>(run.size());
+        const size_t pro = rms ? kProBytes : 0;
+        const size_t fixed = round_up(kHeadBytes + wp + xs + pro, 128);
+        const size_t limit = static_cast<size_t>(di.smem_optin);
+        size_t ns = fixed + 2 * slot <= limit ? (limit - fixed) / slot : 0;
+        if (ns < 2)
+            return fail(KQ_ERR_UNSUPPORTED, "steps %d..%d need %zu bytes of shared memory together (limit %zu)",
+                        run.front(), run.back(), fixed + 2 * slot, limit);
+        if (ns > kMaxStages) ns = kMaxStages;
+        op.args.ns = static_cast<int>(ns);
+        op.args.slot_bytes = static_cast<int>(slot);
+        op.args.wp_offset = kHeadBytes;
+        op.args.xs_offset = static_cast<int>(kHeadBytes + wp);
+        op.args.pro_offset = static_cast<int>(kHeadBytes + wp + xs);
+        op.args.sbuf_offset = static_cast<int>(fixed);
+        op.smem = fixed + ns * slot;
+        ops.push_back(op);
+        run.clear();
+        return KQ_OK;
+    };
+    for (int i = 0; i < n_steps; ++i) {
+        const Planned& P = pl[static_cast<size_t>(i)];
+        if (P.skip) continue;
+        if (P.zero) {
+            int st = close_run();
+            if (st != KQ_OK) return st;
+            Op op = {};
+            op.zero = true;
+            op.y = steps[i].y;
+            op.N = steps[i].N;
+            ops.push_back(op);
+            continue;
+        }
+        run.push_back(i);
+        if (static_cast<int>(run.size()) == kMaxSteps) {
+            int st = close_run();
+            if (st != KQ_OK) return st;
+        }
+    }
+    int st = close_run();
+    if (st != KQ_OK) return st;
+    int* fault = nullptr;
+    err = fault_word(&fault);
+    if (err != cudaSuccess) return cuda_fail(err, "fault word");
+    for (Op& op : ops) {
+        if (op.zero) {
+            st = zero_outputs(op.y, op.N, op.N, 1, s);
+            if (st != KQ_OK) return st;
+            continue;
+        }
+        op.args.fault = fault;
+        err = steps_sync_pair(&op.args.sync);
+        if (err != cudaSuccess) return cuda_fail(err, "step counters");
+        err = launch_steps<2>(op.args, di.sm_count, op.smem, true, s);
+        if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
+    }
+    return KQ_OK;
 }
 
 int kq_gemv(const void* W, int fmt, int64_t N, int64_t K, const float* x, float* y, kq_stream_t stream) {

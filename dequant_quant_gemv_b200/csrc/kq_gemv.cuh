@@ -432,10 +432,15 @@ __device__ __forceinline__ uint32_t pro_inv_addr(uint32_t region) { return regio
 // few 1e-7 for the activations' range; g -> -inf gives -0, g -> +inf g*u).
 __device__ __forceinline__ float silu_gate(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
+// Activation loads of the staging passes go to L2 only (ld.global.cg): a CTA
+// of a multi-step launch may read a buffer that another CTA rewrote since
+// this one last read it, and a line left in its L1 would be stale.
+__device__ __forceinline__ float ld_x(const float* p) { return __ldcg(p); }
+
 // A float4 at p, one 16-byte load when p is 16-byte aligned.
 __device__ __forceinline__ float4 ld_f4(const float* p) {
-    if ((reinterpret_cast<uintptr_t>(p) & 15u) == 0) return *reinterpret_cast<const float4*>(p);
-    return make_float4(p[0], p[1], p[2], p[3]);
+    if ((reinterpret_cast<uintptr_t>(p) & 15u) == 0) return __ldcg(reinterpret_cast<const float4*>(p));
+    return make_float4(ld_x(p), ld_x(p + 1), ld_x(p + 2), ld_x(p + 3));
 }
 
 // inv[c] = 1/sqrt(sum_i part[c][i] / K + eps) for the columns c < ncol from
@@ -542,8 +547,8 @@ __device__ void stage_x(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int
         const int i = 4 * (it - j * k4);
         const float* xc = xg + (j < a.ncol_real ? j : a.ncol_real - 1) * a.ldx;
         float4 v;
-        if ((reinterpret_cast<uintptr_t>(xc) & 15u) == 0) v = *reinterpret_cast<const float4*>(xc + i);
-        else v = make_float4(xc[i], xc[i + 1], xc[i + 2], xc[i + 3]);
+        if ((reinterpret_cast<uintptr_t>(xc) & 15u) == 0) v = __ldcg(reinterpret_cast<const float4*>(xc + i));
+        else v = make_float4(ld_x(xc + i), ld_x(xc + i + 1), ld_x(xc + i + 2), ld_x(xc + i + 3));
         st_x4<FMT>(xs + 4 * (j * xcs + x_offset<FMT>(i, nb)), v);
     }
     named_bar_sync(bar, nthr);
@@ -679,8 +684,8 @@ __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, 
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int G = base + nwarps * u;
-            v[u] = G < groups ? xg[32 * G + lane] : 0.f;
-            if constexpr (PRO) w[u] = G < groups ? sg[32 * G + lane] : 0.f;
+            v[u] = G < groups ? ld_x(xg + 32 * G + lane) : 0.f;
+            if constexpr (PRO) w[u] = G < groups ? ld_x(sg + 32 * G + lane) : 0.f;
         }
         if constexpr (PRO) {
 #pragma unroll

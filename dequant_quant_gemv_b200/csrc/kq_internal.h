@@ -52,6 +52,43 @@ struct GemvArgs {
     int pro_offset;          // RMSNorm scratch (kProBytes) after the stage ring
 };
 
+// ---------------------------------------------------- multi-step launch
+
+constexpr int kMaxSteps = 16;  // steps per launch (the host splits longer lists)
+
+// One step of a multi-step launch as the kernel sees it (planned on the host).
+struct StepArgs {
+    const uint8_t* W;
+    const float* x;
+    float* y;
+    const float* gamma;  // RMSNorm weights (pro == 1)
+    int64_t N;
+    int64_t row_bytes;
+    int K, nb, fmt, pro;
+    float eps;
+    int after;           // wait for every CTA to finish the steps before this one
+    int ps;              // row pairs per stage
+    int lanes_per_rp;    // as in GemvArgs
+    int parts;
+};
+
+struct StepsArgs {
+    StepArgs st[kMaxSteps];
+    int n;
+    int ns;              // ring slots
+    int slot_bytes;      // bytes between ring slots (the largest stage)
+    int wp_offset, xs_offset, pro_offset, sbuf_offset;
+    int* sync;           // (step completions, CTAs finished) pair, zero between launches
+    int* fault;
+};
+
+// Launch of the multi-step kernel (NG consumer groups), one CTA per SM.
+template <int NG>
+cudaError_t launch_steps(const StepsArgs& a, int grid, size_t smem_bytes, bool pdl, cudaStream_t stream);
+// The next counter pair of this device's pool for a multi-step launch.
+cudaError_t steps_sync_pair(int** out);
+constexpr int kSyncPairs = 4096;
+
 // Shared-memory scratch of RMSNorm in the single-column kernel: per consumer
 // group, partial sums of squares (16 warps x 8 columns) and the columns'
 // 1/rms.  Reserved only by launches that normalise.  (The tensor-core

@@ -1,6 +1,7 @@
 // kq_misc.cu — the debug unpack kernel and the device fault word.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "kq_device.cuh"
@@ -90,6 +91,29 @@ cudaError_t launch_splitk_combine(const float* partial, int S, int ncol, int64_t
     const int64_t grid = (n + threads - 1) / threads;
     splitk_combine_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(partial, S, ncol, N, y, ldy);
     return cudaGetLastError();
+}
+
+// Counter pairs of multi-step launches: pair i = (step completions, CTAs
+// finished).  Every pair is zero between launches: the last CTA of a launch
+// to finish resets its pair.  Launches take pairs round-robin, so two
+// launches share a pair only kSyncPairs launches apart.
+__device__ int g_kq_steps_sync[2 * kSyncPairs] = {};
+
+cudaError_t steps_sync_pair(int** out) {
+    static int* base[64] = {};
+    static std::atomic<unsigned> next[64];
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!base[dev]) {
+        int* b = nullptr;
+        err = cudaGetSymbolAddress(reinterpret_cast<void**>(&b), g_kq_steps_sync);
+        if (err != cudaSuccess) return err;
+        base[dev] = b;
+    }
+    *out = base[dev] + 2 * (next[dev].fetch_add(1u, std::memory_order_relaxed) % kSyncPairs);
+    return cudaSuccess;
 }
 
 // The fault word's device address, looked up once per device.

@@ -42,6 +42,12 @@ class Prologue(ctypes.Structure):
 PROLOGUE = {"none": 0, "rmsnorm": 1, "swiglu": 2}
 
 
+class Step(ctypes.Structure):
+    """kq_step: one GEMV of kq_gemv_steps."""
+    _fields_ = [("W", ctypes.c_void_p), ("fmt", ctypes.c_int), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("x", ctypes.c_void_p), ("y", ctypes.c_void_p), ("pro", Prologue), ("after", ctypes.c_int)]
+
+
 def lib() -> ctypes.CDLL:
     """Load libkq.so (built in-tree by ``dequant_quant_gemv_b200.build``)."""
     global _lib
@@ -70,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.kq_unpack.argtypes = [vp, i32, i64, vp, vp, vp, vp]
         L.kq_gemv_fused.restype = i32
         L.kq_gemv_fused.argtypes = [vp, i32, i64, i64, vp, i64, i32, ctypes.POINTER(Prologue), vp, i64, vp]
+        L.kq_gemv_steps.restype = i32
+        L.kq_gemv_steps.argtypes = [ctypes.POINTER(Step), i32, vp]
         _lib = L
     return _lib
 
@@ -137,6 +145,21 @@ def gemv_fused(W: torch.Tensor, fmt, N: int, K: int, X: torch.Tensor, kind: str 
                                ctypes.byref(pro), _dev(Y, "Y", torch.float32), Y.stride(0), _stream(stream)),
            "kq_gemv_fused")
     return Y
+
+
+def make_step(W: torch.Tensor, fmt, N: int, K: int, x: torch.Tensor, y: torch.Tensor, kind: str = "none",
+              gamma: torch.Tensor | None = None, eps: float = 1e-5, after: bool = False) -> Step:
+    """A kq_step for gemv_steps: y = W P(x), one column (x of K floats, 2K for
+    "swiglu"); `after`: x is written by an earlier step of the same call."""
+    pro = Prologue(PROLOGUE[kind], _dev(gamma, "gamma", torch.float32) if gamma is not None else None, eps)
+    return Step(_dev(W, "W"), _fmt(fmt), N, K, _dev(x, "x", torch.float32), _dev(y, "y", torch.float32), pro,
+                1 if after else 0)
+
+
+def gemv_steps(steps, stream=None) -> None:
+    """kq_gemv_steps over a list of Step (see make_step), in order."""
+    arr = (Step * max(1, len(steps)))(*steps)
+    _check(lib().kq_gemv_steps(arr, len(steps), _stream(stream)), "kq_gemv_steps")
 
 
 def _splitk_sigs(L):

@@ -169,6 +169,42 @@ typedef struct {
 KQ_API int kq_gemv_fused(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx, int k,
                          const kq_prologue* pro, float* y, int64_t ldy, kq_stream_t stream);
 
+/* One GEMV of a kq_gemv_steps call (one activation column). */
+typedef struct kq_step {
+    const void* W;       /* device: N rows of K/256 blocks of `fmt`, as kq_gemv */
+    int fmt;             /* kq_fmt */
+    int64_t N, K;
+    const float* x;      /* device: K floats (2K for KQ_PRO_SWIGLU), 4-byte aligned */
+    float* y;            /* device: N floats */
+    kq_prologue pro;     /* prologue of this step (kind KQ_PRO_NONE: none) */
+    int after;           /* nonzero: x (or gamma) is written by an earlier step of this call */
+} kq_step;
+
+/*
+ * kq_gemv_steps — run n_steps single-column GEMVs (each y = W P(x) as
+ * kq_gemv_fused with k = 1) in order, in as few launches as possible: one
+ * persistent grid streams the weights of step after step without a gap
+ * while the steps are computed.  A step with `after` set starts only when
+ * every earlier step of the call has finished on the whole GPU (its x may
+ * be an earlier step's y); other steps may overlap the step before them,
+ * so a step without `after` must not read what an earlier step of the call
+ * writes.  This is the decode chain of the pages' engines -- a token's
+ * matvecs one after another, each reading the weights once ("Kortex:
+ * Streaming 70B Models on Consumer GPUs", the paragraph before the first
+ * table; "Out-of-core LLM inference engine written from scratch in Rust",
+ * Approach) -- without a kernel boundary between matvecs.
+ *   steps: HOST array of n_steps descriptors (read during the call only).
+ * Results equal, bit for bit, the same steps run one by one with
+ * kq_gemv_fused (k = 1).  Asynchronous on `stream`; the call returns once
+ * the launches are queued.
+ * Errors: KQ_ERR_INVALID_ARG (n_steps < 0, a NULL steps array, or any step's
+ * arguments as kq_gemv_fused would reject them), KQ_ERR_UNSUPPORTED (a
+ * step's shape the single-column kernel does not take, or steps whose
+ * activations and stages do not fit shared memory together), KQ_ERR_CUDA.
+ * Nothing is launched unless every step is valid.
+ */
+KQ_API int kq_gemv_steps(const kq_step* steps, int n_steps, kq_stream_t stream);
+
 /*
  * kq_gemv_splitk — kq_gemv_multi for tall-skinny matrices: when the matrix
  * has fewer row pairs than the GPU has SMs, K is also split across CTAs.
