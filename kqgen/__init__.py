@@ -4,7 +4,7 @@ arithmetic).
 
 The C source ``kqgen.c`` draws logical values with a counter-based
 SplitMix64 stream and encodes them into the GGUF K-quant super-block layout
-(Q4_K: 144 bytes, Q6_K: 210 bytes, 256 weights each).  This wrapper builds it
+(Q4_K: 144 bytes, Q5_K: 176 bytes, Q6_K: 210 bytes, 256 weights each).  This wrapper builds it
 with gcc on first use and returns numpy arrays.
 """
 from __future__ import annotations
@@ -21,6 +21,7 @@ _LIB_PATH = os.path.join(_HERE, "libkqgen.so")
 _lib = None
 
 Q4_K_BLOCK_BYTES = 144
+Q5_K_BLOCK_BYTES = 176
 Q6_K_BLOCK_BYTES = 210
 QK = 256  # weights per super-block
 
@@ -49,6 +50,9 @@ def _load():
         lib.kqg_q4k_draw.argtypes = [u64, i64, vp, vp, vp, vp, vp]
         lib.kqg_q4k_pack.argtypes = [i64, vp, vp, vp, vp, vp, vp]
         lib.kqg_q4k_fill.argtypes = [u64, i64, i64, vp, i32]
+        lib.kqg_q5k_draw.argtypes = [u64, i64, vp, vp, vp, vp, vp]
+        lib.kqg_q5k_pack.argtypes = [i64, vp, vp, vp, vp, vp, vp]
+        lib.kqg_q5k_fill.argtypes = [u64, i64, i64, vp, i32]
         lib.kqg_q6k_draw.argtypes = [u64, i64, vp, vp, vp]
         lib.kqg_q6k_pack.argtypes = [i64, vp, vp, vp, vp]
         lib.kqg_q6k_fill.argtypes = [u64, i64, i64, vp, i32]
@@ -84,7 +88,7 @@ def f16_bits(v: float) -> int:
 
 
 def block_bytes(fmt: str) -> int:
-    return {"q4_k": Q4_K_BLOCK_BYTES, "q6_k": Q6_K_BLOCK_BYTES}[fmt]
+    return {"q4_k": Q4_K_BLOCK_BYTES, "q5_k": Q5_K_BLOCK_BYTES, "q6_k": Q6_K_BLOCK_BYTES}[fmt]
 
 
 def row_bytes(fmt: str, K: int) -> int:
@@ -128,6 +132,42 @@ def q4k_fill(key: int, nblocks: int, out: np.ndarray | None = None, b0: int = 0,
     return out
 
 
+# ----------------------------------------------------------------- Q5_K
+def q5k_draw(key: int, nblocks: int) -> dict:
+    """Logical values of ``nblocks`` Q5_K super-blocks: q (nb,256) u8 in 0..31,
+    sc/m (nb,8) u8 in 0..63, d/dmin (nb,) fp16 bit patterns (uint16)."""
+    q = np.empty((nblocks, 256), np.uint8)
+    sc = np.empty((nblocks, 8), np.uint8)
+    m = np.empty((nblocks, 8), np.uint8)
+    d = np.empty(nblocks, np.uint16)
+    dmin = np.empty(nblocks, np.uint16)
+    _load().kqg_q5k_draw(key, nblocks, _ptr(q), _ptr(sc), _ptr(m), _ptr(d), _ptr(dmin))
+    return dict(q=q, sc=sc, m=m, d=d, dmin=dmin)
+
+
+def q5k_pack(q, sc, m, d, dmin) -> np.ndarray:
+    """Encode logical Q5_K values (see :func:`q5k_draw`) into bytes (nb*176,)."""
+    q = np.ascontiguousarray(q, np.uint8).reshape(-1, 256)
+    nb = q.shape[0]
+    sc = np.ascontiguousarray(sc, np.uint8).reshape(nb, 8)
+    m = np.ascontiguousarray(m, np.uint8).reshape(nb, 8)
+    d = np.ascontiguousarray(d, np.uint16).reshape(nb)
+    dmin = np.ascontiguousarray(dmin, np.uint16).reshape(nb)
+    out = np.empty(nb * Q5_K_BLOCK_BYTES, np.uint8)
+    _load().kqg_q5k_pack(nb, _ptr(q), _ptr(sc), _ptr(m), _ptr(d), _ptr(dmin), _ptr(out))
+    return out
+
+
+def q5k_fill(key: int, nblocks: int, out: np.ndarray | None = None, b0: int = 0,
+             nthreads: int | None = None) -> np.ndarray:
+    """Draw + encode Q5_K super-blocks [b0, b0+nblocks) of stream ``key``."""
+    if out is None:
+        out = np.empty(nblocks * Q5_K_BLOCK_BYTES, np.uint8)
+    assert out.nbytes >= nblocks * Q5_K_BLOCK_BYTES and out.dtype == np.uint8
+    _load().kqg_q5k_fill(key, b0, nblocks, _ptr(out), nthreads or default_threads())
+    return out
+
+
 # ----------------------------------------------------------------- Q6_K
 def q6k_draw(key: int, nblocks: int) -> dict:
     """Logical values of Q6_K super-blocks: q (nb,256) u8 in 0..63,
@@ -162,6 +202,8 @@ def fill(fmt: str, key: int, nblocks: int, out: np.ndarray | None = None,
          nthreads: int | None = None) -> np.ndarray:
     if fmt == "q4_k":
         return q4k_fill(key, nblocks, out, nthreads=nthreads)
+    if fmt == "q5_k":
+        return q5k_fill(key, nblocks, out, nthreads=nthreads)
     if fmt == "q6_k":
         return q6k_fill(key, nblocks, out, nthreads=nthreads)
     raise ValueError(fmt)

@@ -29,6 +29,13 @@
  *     m_j's top 2 bits in bits 6-7 of byte j.
  *     Quant bytes: chunk c (0..3) of 32 bytes; byte 32c+l carries weight
  *     64c+l in its low nibble and weight 64c+32+l in its high nibble.
+ *   Q5_K, 176 B: [0,2) d fp16 | [2,4) dmin fp16 | [4,16) 12 scale bytes
+ *                (packed as Q4_K) | [16,48) qh | [48,176) 128 quant bytes.
+ *     Weight 64c+l (l<32, c<4) has its low 4 bits in the low nibble of quant
+ *     byte 32c+l and its 5th bit in bit 2c of qh[l]; weight 64c+32+l has its
+ *     low 4 bits in the high nibble of the same byte and its 5th bit in bit
+ *     2c+1 of qh[l].  The fill draws quants uniform over 0..31, the rest as
+ *     Q4_K.
  *   Q6_K, 210 B: [0,128) ql | [128,192) qh | [192,208) int8 scales |
  *                [208,210) d fp16.
  *     Half h (0..1) covers weights 128h..128h+127.  For l<32 and t<4, weight
@@ -158,6 +165,74 @@ void kqg_q4k_fill(uint64_t key, int64_t b0, int64_t nblocks, uint8_t* out, int n
         uint16_t d, dmin;
         kqg_q4k_draw_block(key, (uint64_t)(b0 + b), q, sc, m, &d, &dmin);
         kqg_q4k_pack_block(q, sc, m, d, dmin, out + 144 * b);
+    }
+}
+
+/* ---------------------------------------------------------------- Q5_K */
+
+/* Logical values of super-block `b` of stream `key`: 5-bit quants, then the
+ * scales, mins and block scales drawn as for Q4_K. */
+static void kqg_q5k_draw_block(uint64_t key, uint64_t b, uint8_t q[256], uint8_t sc[8],
+                               uint8_t m[8], uint16_t* d, uint16_t* dmin) {
+    const uint64_t base = b * 32;
+    for (int i = 0; i < 256; ++i) {
+        uint64_t r = kqg_draw(key, base + (uint64_t)(i / 12));
+        q[i] = (uint8_t)((r >> (5 * (i % 12))) & 31);
+    }
+    uint64_t rs = kqg_draw(key, base + 22), rm = kqg_draw(key, base + 23);
+    for (int j = 0; j < 8; ++j) {
+        sc[j] = (uint8_t)((rs >> (6 * j)) & 63);
+        m[j] = (uint8_t)((rm >> (6 * j)) & 63);
+    }
+    double z0, z1;
+    kqg_box_muller(key, base + 24, &z0, &z1);
+    *d = kqg_f16_bits(fabs(z0) * 1e-3);
+    *dmin = kqg_f16_bits(fabs(z1) * 1e-3);
+}
+
+static void kqg_q5k_pack_block(const uint8_t q[256], const uint8_t sc[8], const uint8_t m[8],
+                               uint16_t d, uint16_t dmin, uint8_t* out) {
+    out[0] = (uint8_t)(d & 0xFF);
+    out[1] = (uint8_t)(d >> 8);
+    out[2] = (uint8_t)(dmin & 0xFF);
+    out[3] = (uint8_t)(dmin >> 8);
+    uint8_t* s = out + 4;
+    for (int j = 0; j < 4; ++j) {
+        s[j] = (uint8_t)((sc[j] & 63) | (((sc[j + 4] >> 4) & 3) << 6));
+        s[j + 4] = (uint8_t)((m[j] & 63) | (((m[j + 4] >> 4) & 3) << 6));
+        s[j + 8] = (uint8_t)((sc[j + 4] & 15) | ((m[j + 4] & 15) << 4));
+    }
+    uint8_t* qh = out + 16;
+    uint8_t* qs = out + 48;
+    memset(qh, 0, 32);
+    for (int c = 0; c < 4; ++c)
+        for (int l = 0; l < 32; ++l) {
+            const uint8_t lo = q[64 * c + l] & 31, hi = q[64 * c + 32 + l] & 31;
+            qs[32 * c + l] = (uint8_t)((lo & 15) | ((hi & 15) << 4));
+            qh[l] |= (uint8_t)(((lo >> 4) << (2 * c)) | ((hi >> 4) << (2 * c + 1)));
+        }
+}
+
+void kqg_q5k_draw(uint64_t key, int64_t nblocks, uint8_t* q, uint8_t* sc, uint8_t* m,
+                  uint16_t* d, uint16_t* dmin) {
+    for (int64_t b = 0; b < nblocks; ++b)
+        kqg_q5k_draw_block(key, (uint64_t)b, q + 256 * b, sc + 8 * b, m + 8 * b, d + b, dmin + b);
+}
+
+void kqg_q5k_pack(int64_t nblocks, const uint8_t* q, const uint8_t* sc, const uint8_t* m,
+                  const uint16_t* d, const uint16_t* dmin, uint8_t* out) {
+    for (int64_t b = 0; b < nblocks; ++b)
+        kqg_q5k_pack_block(q + 256 * b, sc + 8 * b, m + 8 * b, d[b], dmin[b], out + 176 * b);
+}
+
+void kqg_q5k_fill(uint64_t key, int64_t b0, int64_t nblocks, uint8_t* out, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int64_t b = 0; b < nblocks; ++b) {
+        uint8_t q[256], sc[8], m[8];
+        uint16_t d, dmin;
+        kqg_q5k_draw_block(key, (uint64_t)(b0 + b), q, sc, m, &d, &dmin);
+        kqg_q5k_pack_block(q, sc, m, d, dmin, out + 176 * b);
     }
 }
 

@@ -20,6 +20,8 @@
  *  layout; the layout below is the public GGUF one, restated:
  *   Q4_K (144 B, 256 weights = 8 sub-blocks of 32):
  *     w = d*sc_j*q - dmin*m_j for weight in sub-block j.
+ *   Q5_K (176 B, 256 weights = 8 sub-blocks of 32):
+ *     w = d*sc_j*q - dmin*m_j as Q4_K, with q a 5-bit quant (0..31).
  *   Q6_K (210 B, 256 weights = 16 groups of 16):
  *     w = d*s_g*(q - 32) for weight in group g, s_g a signed byte.
  *
@@ -30,7 +32,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { KQO_Q4_K = 1, KQO_Q6_K = 2 };
+enum { KQO_Q4_K = 1, KQO_Q6_K = 2, KQO_Q5_K = 3 };
 
 /* IEEE binary16 -> double (exact), including subnormals, inf and NaN. */
 double kqo_f16(uint16_t h) {
@@ -77,6 +79,40 @@ void kqo_q4k_unpack(const uint8_t* blk, uint8_t q[256], uint8_t sc[8], uint8_t m
     }
 }
 
+/* Q5_K super-block -> logical fields.
+ * Header as Q4_K (d, dmin, the same 12 packed scale/min bytes), then 32
+ * bytes qh, then 128 quant bytes qs.  Weight i lies in 32-byte chunk
+ * c = i/64 of qs at byte l = i%32: its low 4 bits are the low nibble of that
+ * byte when i%64 < 32 and the high nibble otherwise; its 5th bit is bit
+ * 2c (low-nibble weights) or 2c+1 (high-nibble weights) of qh[l]. */
+void kqo_q5k_unpack(const uint8_t* blk, uint8_t q[256], uint8_t sc[8], uint8_t m[8],
+                    double* d, double* dmin) {
+    const uint8_t* s = blk + 4;
+    const uint8_t* qh = blk + 16;
+    const uint8_t* qs = blk + 48;
+    *d = kqo_f16(rd16(blk));
+    *dmin = kqo_f16(rd16(blk + 2));
+    for (int j = 0; j < 8; ++j) {
+        if (j < 4) {
+            sc[j] = s[j] & 63;
+            m[j] = s[j + 4] & 63;
+        } else {
+            sc[j] = (uint8_t)((s[j + 4] & 15) | ((s[j - 4] >> 6) << 4));
+            m[j] = (uint8_t)((s[j + 4] >> 4) | ((s[j] >> 6) << 4));
+        }
+    }
+    for (int i = 0; i < 256; ++i) {
+        int c = i / 64;
+        int within = i % 64;
+        int l = within % 32;
+        int upper = within >= 32;
+        uint8_t byte = qs[32 * c + l];
+        int lo4 = upper ? (byte >> 4) : (byte & 15);
+        int bit5 = (qh[l] >> (2 * c + upper)) & 1;
+        q[i] = (uint8_t)(lo4 | (bit5 << 4));
+    }
+}
+
 /* Q6_K super-block -> logical fields.
  * Layout: ql[128] (low 4 bits), qh[64] (top 2 bits), 16 signed scales, d.
  * Weight i = 128h + 32t + l (h<2, t<4, l<32): low bits from
@@ -96,7 +132,9 @@ void kqo_q6k_unpack(const uint8_t* blk, uint8_t q[256], int8_t s[16], double* d)
     *d = kqo_f16(rd16(blk + 208));
 }
 
-static int64_t block_bytes(int fmt) { return fmt == KQO_Q4_K ? 144 : fmt == KQO_Q6_K ? 210 : -1; }
+static int64_t block_bytes(int fmt) {
+    return fmt == KQO_Q4_K ? 144 : fmt == KQO_Q6_K ? 210 : fmt == KQO_Q5_K ? 176 : -1;
+}
 
 /* Dequantise one row of K weights (K/256 consecutive super-blocks). */
 int kqo_dequant_row(int fmt, const uint8_t* row, int64_t K, double* w) {
@@ -106,10 +144,11 @@ int kqo_dequant_row(int fmt, const uint8_t* row, int64_t K, double* w) {
         const uint8_t* blk = row + b * bb;
         uint8_t q[256];
         double* wb = w + 256 * b;
-        if (fmt == KQO_Q4_K) {
+        if (fmt == KQO_Q4_K || fmt == KQO_Q5_K) {
             uint8_t sc[8], m[8];
             double d, dmin;
-            kqo_q4k_unpack(blk, q, sc, m, &d, &dmin);
+            if (fmt == KQO_Q4_K) kqo_q4k_unpack(blk, q, sc, m, &d, &dmin);
+            else kqo_q5k_unpack(blk, q, sc, m, &d, &dmin);
             for (int i = 0; i < 256; ++i) {
                 int j = i / 32;
                 wb[i] = d * sc[j] * q[i] - dmin * m[j];
@@ -228,18 +267,20 @@ int kqo_gemv_x64(int fmt, const uint8_t* W, int64_t N, int64_t K, const double* 
 
 /* Logical fields of `nblocks` consecutive super-blocks, in the layout the
  * bit-exact unpack check compares:
- *   q[256*b + i]      quant of weight i (Q4_K 0..15, Q6_K 0..63, before -32)
- *   sc[16*b + j]      Q4_K: sc_0..7 then m_0..7; Q6_K: the 16 signed scales
- *                     as two's-complement bytes
- *   d[2*b], d[2*b+1]  Q4_K: d, dmin; Q6_K: d, 0 (fp16 widened exactly) */
+ *   q[256*b + i]      quant of weight i (Q4_K 0..15, Q5_K 0..31, Q6_K 0..63,
+ *                     before -32)
+ *   sc[16*b + j]      Q4_K, Q5_K: sc_0..7 then m_0..7; Q6_K: the 16 signed
+ *                     scales as two's-complement bytes
+ *   d[2*b], d[2*b+1]  Q4_K, Q5_K: d, dmin; Q6_K: d, 0 (fp16 widened exactly) */
 int kqo_unpack(int fmt, const uint8_t* W, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d) {
     int64_t bb = block_bytes(fmt);
     if (bb < 0) return -1;
     for (int64_t b = 0; b < nblocks; ++b) {
         const uint8_t* blk = W + b * bb;
-        if (fmt == KQO_Q4_K) {
+        if (fmt == KQO_Q4_K || fmt == KQO_Q5_K) {
             double dd, dm;
-            kqo_q4k_unpack(blk, q + 256 * b, sc + 16 * b, sc + 16 * b + 8, &dd, &dm);
+            if (fmt == KQO_Q4_K) kqo_q4k_unpack(blk, q + 256 * b, sc + 16 * b, sc + 16 * b + 8, &dd, &dm);
+            else kqo_q5k_unpack(blk, q + 256 * b, sc + 16 * b, sc + 16 * b + 8, &dd, &dm);
             d[2 * b] = (float)dd;
             d[2 * b + 1] = (float)dm;
         } else {

@@ -2,9 +2,9 @@
 than the oracle itself — hand-worked blocks, library routines, closed forms,
 invariants and exhaustive round trips.
 
-Formats: GGUF K-quants Q4_K (w = d*sc_j*q - dmin*m_j per 32-weight
-sub-block) and Q6_K (w = d*s_g*(q-32) per 16-weight group), the formats the
-pages name ("Out-of-core LLM inference engine written from scratch in Rust",
+Formats: GGUF K-quants Q4_K and Q5_K (w = d*sc_j*q - dmin*m_j per 32-weight
+sub-block, q of 4 or 5 bits) and Q6_K (w = d*s_g*(q-32) per 16-weight group),
+the formats the pages name ("Out-of-core LLM inference engine written from scratch in Rust",
 Results: Q4_K_M; "RunNburn - Run a 295B MoE ...": K-quants Q2_K..Q6_K).
 """
 import os
@@ -90,7 +90,58 @@ def test_q6k_hand_worked_block(golden_dir):
         assert w[i] == wi, i
 
 
+def test_q5k_hand_worked_block(golden_dir):
+    g = _read_golden(os.path.join(golden_dir, "q5k_block_worked.txt"))
+    qh = np.arange(32, dtype=np.uint8)
+    qh[31] = 0xFF
+    blk = np.concatenate([np.array([int(h, 16) for h in g["header"]], np.uint8), qh,
+                          np.arange(128, dtype=np.uint8)])
+    assert blk.size == 176
+    q, sc, d = oracle.unpack("q5_k", blk, 1)
+    assert sc[:8].tolist() == [int(v) for v in g["sc"]]
+    assert sc[8:].tolist() == [int(v) for v in g["m"]]
+    assert d.tolist() == [1.0, 0.5]
+    w = oracle.dequant("q5_k", blk, 1, 256)[0]
+    for i, qi, wi in g["w"]:
+        assert q[i] == qi, i
+        assert w[i] == wi, i
+    y, _ = oracle.gemv("q5_k", blk, 1, 256, np.ones(256, np.float32))
+    assert y[0] == float(g["y_ones"][0])
+
+
 # ----------------------------------------------- exhaustive round trips
+def test_q5k_quant_and_scale_roundtrip_all_positions():
+    """Every 5-bit value in every quant position, and every 6-bit value in
+    every scale and min slot, survive generator packing and oracle unpacking."""
+    nb = 64
+    q = ((np.arange(nb * 256).reshape(nb, 256) * 11 + np.arange(nb)[:, None] * 5) % 32).astype(np.uint8)
+    b, j = np.meshgrid(np.arange(nb), np.arange(8), indexing="ij")
+    sc = ((b + 5 * j) % 64).astype(np.uint8)
+    m = ((63 - b + 3 * j) % 64).astype(np.uint8)
+    W = kqgen.q5k_pack(q, sc, m, np.full(nb, 0x3C00, np.uint16), np.full(nb, 0x3800, np.uint16))
+    q2, sc2, d2 = oracle.unpack("q5_k", W, nb)
+    assert np.array_equal(q2.reshape(nb, 256), q)
+    sc2 = sc2.reshape(nb, 16)
+    assert np.array_equal(sc2[:, :8], sc) and np.array_equal(sc2[:, 8:], m)
+    # each position takes all 32 values across the blocks
+    assert all(len(set(q[:, i].tolist())) == 32 for i in range(256))
+    assert all(len(set(sc[:, j].tolist())) == 64 and len(set(m[:, j].tolist())) == 64 for j in range(8))
+
+
+def test_q5k_fifth_bit_alone():
+    """Quants 16 everywhere (only the 5th bit set), d=1, sc=1, m=0: y = 16 sum x;
+    and quants 15 (no 5th bit) give 15 sum x."""
+    K = 512
+    nb = 2
+    ones = np.ones((nb, 8), np.uint8)
+    z = np.zeros((nb, 8), np.uint8)
+    x = kqgen.normal_f32(41, K)
+    for qv in (16, 15):
+        W = kqgen.q5k_pack(np.full((nb, 256), qv, np.uint8), ones, z, np.full(nb, 0x3C00, np.uint16),
+                           np.zeros(nb, np.uint16))
+        y, _ = oracle.gemv("q5_k", W, 1, K, x)
+        assert np.isclose(y[0], qv * x.astype(np.float64).sum(), rtol=1e-13, atol=1e-12)
+
 def test_q4k_scale_min_roundtrip_exhaustive():
     # every 6-bit value in every scale and min slot, others varied
     for v in range(64):
@@ -221,7 +272,7 @@ def test_q6k_mid_quants_give_exact_zero_and_zero_quants_closed_form():
 
 
 # -------------------------------------------------------------- invariants
-@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k"])
 def test_linearity_in_x(fmt):
     N, K = 8, 1024
     W = kqgen.matrix(fmt, 11, N, K)
@@ -235,7 +286,7 @@ def test_linearity_in_x(fmt):
     assert np.all(np.abs(yc - (2 * y1 - 3 * y2)) <= 1e-12 * (2 * s1 + 3 * s2))
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k"])
 def test_one_hot_extracts_column_and_ones_give_row_sums(fmt):
     N, K = 4, 512
     W = kqgen.matrix(fmt, 12, N, K)
@@ -250,15 +301,15 @@ def test_one_hot_extracts_column_and_ones_give_row_sums(fmt):
     assert np.allclose(s, np.abs(Wd).sum(axis=1), rtol=1e-13)
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k"])
 def test_brute_force_tiny_from_logical_values(fmt):
     """Dense W built from the generator's logical values (never its bytes)
     matches the oracle's byte path."""
     N, K = 8, 512
     nb = N * K // 256
-    if fmt == "q4_k":
-        lg = kqgen.q4k_draw(31, nb)
-        W = kqgen.q4k_pack(**lg)
+    if fmt in ("q4_k", "q5_k"):
+        lg = kqgen.q4k_draw(31, nb) if fmt == "q4_k" else kqgen.q5k_draw(34, nb)
+        W = kqgen.q4k_pack(**lg) if fmt == "q4_k" else kqgen.q5k_pack(**lg)
         d = lg["d"].view(np.float16).astype(np.float64)[:, None]
         dm = lg["dmin"].view(np.float16).astype(np.float64)[:, None]
         sc = np.repeat(lg["sc"].astype(np.float64), 32, axis=1)
