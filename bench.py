@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "K-quant dequant-GEMV weight GB/s (% of B200 HBM peak); layer-chain tok/s"
 QK = 256
-BLOCK = {"q4_k": 144, "q6_k": 210}
+BLOCK = {"q4_k": 144, "q5_k": 176, "q6_k": 210}
 SEED = 0xC0FFEE + 1
 
 
@@ -50,12 +50,14 @@ def row_bytes(fmt, K):
     return K // QK * BLOCK[fmt]
 
 
-def dense_layer(hidden, heads, kv_heads, head_dim, ffn):
+def dense_layer(hidden, heads, kv_heads, head_dim, ffn, fmt="q4_k"):
     """(name, fmt, N, K, x-slot): q|k|v share the attention input, gate|up
-    share the FFN input; each is one launch over the stacked rows."""
+    share the FFN input; each is one launch over the stacked rows.  `fmt`
+    is the format of all but down, which stays Q6_K (as in Q4_K_M and Q5_K_M
+    files)."""
     qkv = (heads + 2 * kv_heads) * head_dim
-    return [("qkv", "q4_k", qkv, hidden, 0), ("o", "q4_k", hidden, heads * head_dim, 1),
-            ("gate_up", "q4_k", 2 * ffn, hidden, 2), ("down", "q6_k", hidden, ffn, 3)]
+    return [("qkv", fmt, qkv, hidden, 0), ("o", fmt, hidden, heads * head_dim, 1),
+            ("gate_up", fmt, 2 * ffn, hidden, 2), ("down", "q6_k", hidden, ffn, 3)]
 
 
 L8B = dict(hidden=4096, heads=32, kv_heads=8, head_dim=128, ffn=14336)
@@ -66,12 +68,16 @@ MOE30B = dict(hidden=2048, experts=128, top=8, ffn=768, layers=48)
 def chain_spec(kind):
     if kind == "llama8b":
         return [dense_layer(**L8B) for _ in range(32)]
+    if kind == "llama8b_q5k":
+        return [dense_layer(**L8B, fmt="q5_k") for _ in range(32)]
     if kind == "llama70b":
         return [dense_layer(**L70B) for _ in range(80)]
     if kind == "gemv_q4k_4096":
         return [[("w", "q4_k", 4096, 4096, 0)] for _ in range(64)]
     if kind == "gateup_q4k":
         return [[("gate_up", "q4_k", 28672, 4096, 0)] for _ in range(8)]
+    if kind == "gateup_q5k":
+        return [[("gate_up", "q5_k", 28672, 4096, 0)] for _ in range(8)]
     if kind == "down_q6k":
         return [[("down", "q6_k", 4096, 14336, 0)] for _ in range(8)]
     raise KeyError(kind)
@@ -79,6 +85,10 @@ def chain_spec(kind):
 
 WORKLOADS = {
     "llama8b_chain": "Llama-3.1-8B-shaped decode chain, 32 layers, Q4_K + Q6_K down, batch 1",
+    "llama8b_q5k_chain": "Llama-3.1-8B-shaped decode chain with Q5_K qkv, o and gate|up and Q6_K down "
+                         "(a Q5_K_M file's formats), 32 layers, batch 1",
+    "verify8b_q5k_k8": "the Q5_K 8B-shaped chain, speculative-verify GEMV with k=8 activation columns",
+    "gateup_q5k": "Q5_K GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
     "llama8b_chain_steps": "the same chain through kq_gemv_steps (16 matvecs per persistent launch, each "
                            "waiting for the one before)",
     "llama8b_layer_fused": "the 8B-shaped chain with RMSNorm fused into qkv and gate|up and the SiLU-gated "
@@ -425,7 +435,11 @@ def make_workload(name, torch, kq, kqgen, seed):
         return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed, steps=name.endswith("_steps"))
     if name in ("llama8b_layer_fused", "llama8b_layer_fused_steps"):
         return FusedLayer(torch, kq, kqgen, chain_spec("llama8b"), seed, steps=name.endswith("_steps"))
-    if name in ("gemv_q4k_4096", "gateup_q4k", "down_q6k"):
+    if name == "llama8b_q5k_chain":
+        return Resident(torch, kq, kqgen, chain_spec("llama8b_q5k"), seed)
+    if name == "verify8b_q5k_k8":
+        return Resident(torch, kq, kqgen, chain_spec("llama8b_q5k"), seed, k=8)
+    if name in ("gemv_q4k_4096", "gateup_q4k", "gateup_q5k", "down_q6k"):
         return Resident(torch, kq, kqgen, chain_spec(name), seed)
     if name.startswith("verify8b_k"):
         k = int(name[len("verify8b_k"):])
@@ -683,7 +697,7 @@ def cpu_baseline(args, budget_s=15.0):
         per_token = MOE30B["layers"] * MOE30B["top"] * (2 * MOE30B["ffn"] * row_bytes("q4_k", MOE30B["hidden"])
                                                         + MOE30B["hidden"] * row_bytes("q4_k", MOE30B["ffn"]))
     else:
-        base = {"llama8b_chain": "llama8b", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
+        base = {"llama8b_chain": "llama8b", "llama8b_q5k_chain": "llama8b_q5k", "verify8b_q5k_k8": "llama8b_q5k", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
                 "llama8b_layer_fused_steps": "llama8b", "llama70b_resident": "llama70b",
                 "llama70b_resident_steps": "llama70b", "llama70b_stream": "llama70b"}
         name = base.get(args.workload, "llama8b" if args.workload.startswith("verify") else args.workload)

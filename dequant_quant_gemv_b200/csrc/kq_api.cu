@@ -106,7 +106,9 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     cudaError_t err = dev_info(di);
     if (err != cudaSuccess) return cuda_fail(err, "device query");
     const int nb = a.nbs;  // blocks per K range (all of K unless split)
-    if (fmt == KQ_FMT_Q4_K) {
+    if (fmt == KQ_FMT_Q5_K && ncol > 1)
+        return fail(KQ_ERR_UNSUPPORTED, "Q5_K with %d columns runs on the tensor-core kernel only", ncol);
+    if (fmt != KQ_FMT_Q6_K) {  // Q4_K, Q5_K
         const int ur = 2 * nb;  // half-block units per row pair
         const int lr = ur <= 32 ? next_pow2(ur) : static_cast<int>(round_up(ur, 32));
         if (lr > kConsumers) return fail(KQ_ERR_UNSUPPORTED, "Q4_K with K=%lld > 32768", (long long)a.K);
@@ -135,7 +137,7 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     const size_t wp_bytes = round_up(sizeof(float) * ng * 2 * a.ps * a.parts * 2 * ncol, 128);
     // one column of Q4_K: integer activation regions (2 x 336 bytes per
     // super-block); otherwise fp32 regions
-    const size_t xcopy = ncol == 1 && fmt == KQ_FMT_Q4_K ? static_cast<size_t>(672) * nb
+    const size_t xcopy = ncol == 1 && fmt != KQ_FMT_Q6_K ? static_cast<size_t>(672) * nb
                                                           : sizeof(float) * ncol * 2 * nb * kRegion;
     const size_t xs_bytes = round_up((shared_x ? 1 : ng) * xcopy, 128);
     const size_t head = kHeadBytes;
@@ -181,14 +183,14 @@ static MmaLayout mma_layout(int fmt, int nt, int nbs, int S, int ng) {
     // the residue mod 128 that spreads the 8 rows of a warp over distinct
     // banks
     const size_t srow = static_cast<size_t>(nbs) * kq_block_bytes(fmt) + 16 + 4;
-    const size_t res = fmt == KQ_FMT_Q4_K ? 64 : 16;
+    const size_t res = fmt == KQ_FMT_Q6_K ? 16 : 64;
     L.sp = srow <= res ? res : round_up(srow - res, 128) + res;
     L.stage = round_up(16 * L.sp, 128);
     const size_t nc = 4 * static_cast<size_t>(nt);
     L.wp = sizeof(float) * ng * 2 * kConsumerWarps * 16 * nc;
     L.bs = round_up(sizeof(float) * 2 * nc * nbs, 128);
     L.red = S > 1 ? sizeof(float) * 2 * (S - 1) * 16 * nc : 0;
-    L.xb = static_cast<size_t>(nbs) * (fmt == KQ_FMT_Q4_K ? 17 : 16) * 32 * nt * 8;
+    L.xb = static_cast<size_t>(nbs) * (fmt == KQ_FMT_Q6_K ? 16 : 17) * 32 * nt * 8;
     L.fixed = kHeadBytes + L.wp + L.bs + L.red + L.xb;
     return L;
 }
@@ -215,8 +217,12 @@ static cudaError_t active_clusters(int fmt, int nt, int ng, int S, size_t smem, 
                 return cudaSuccess;
             }
     }
-    const int key = (fmt == KQ_FMT_Q4_K ? 0 : 4) + (nt - 1) * 2 + (ng - 1);
+    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 4 : 8) + (nt - 1) * 2 + (ng - 1);
     switch (key) {
+        case 8: err = mma_active_clusters<3, 1, 1>(S, smem, pro, out); break;
+        case 9: err = mma_active_clusters<3, 1, 2>(S, smem, pro, out); break;
+        case 10: err = mma_active_clusters<3, 2, 1>(S, smem, pro, out); break;
+        case 11: err = mma_active_clusters<3, 2, 2>(S, smem, pro, out); break;
         case 0: err = mma_active_clusters<1, 1, 1>(S, smem, pro, out); break;
         case 1: err = mma_active_clusters<1, 1, 2>(S, smem, pro, out); break;
         case 2: err = mma_active_clusters<1, 2, 1>(S, smem, pro, out); break;
@@ -336,7 +342,8 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
 static bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
 static int check_matrix(const void* W, int fmt, int64_t N, int64_t K) {
-    if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q6_K) return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
+    if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q5_K && fmt != KQ_FMT_Q6_K)
+        return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
     if (N < 0 || K < 0) return fail(KQ_ERR_INVALID_ARG, "negative size N=%lld K=%lld", (long long)N, (long long)K);
     if (K % 256 != 0) return fail(KQ_ERR_INVALID_ARG, "K=%lld is not a multiple of 256", (long long)K);
     if (N > 0 && K > 0) {
@@ -353,6 +360,10 @@ static int check_matrix(const void* W, int fmt, int64_t N, int64_t K) {
 static int padded_cols(int k) { return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : 8; }
 
 static cudaError_t dispatch(const GemvArgs& a, const LaunchPlan& p, int fmt, int ncol, cudaStream_t s) {
+    if (fmt == KQ_FMT_Q5_K) {
+        if (ncol == 1) return launch_one<3, 1, 2>(a, p, s);
+        return cudaErrorNotSupported;  // (plan_gemv refuses it first)
+    }
     if (fmt == KQ_FMT_Q4_K) {
         switch (ncol) {
             case 1: return launch_one<1, 1, 2>(a, p, s);
@@ -370,8 +381,12 @@ static cudaError_t dispatch(const GemvArgs& a, const LaunchPlan& p, int fmt, int
 }
 
 static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt, int nt, cudaStream_t s) {
-    const int key = (fmt == KQ_FMT_Q4_K ? 0 : 4) + (nt - 1) * 2 + (p.ng - 1);
+    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 4 : 8) + (nt - 1) * 2 + (p.ng - 1);
     switch (key) {
+        case 8: return launch_mma<3, 1, 1>(a, p, s);
+        case 9: return launch_mma<3, 1, 2>(a, p, s);
+        case 10: return launch_mma<3, 2, 1>(a, p, s);
+        case 11: return launch_mma<3, 2, 2>(a, p, s);
         case 0: return launch_mma<1, 1, 1>(a, p, s);
         case 1: return launch_mma<1, 1, 2>(a, p, s);
         case 2: return launch_mma<1, 2, 1>(a, p, s);
@@ -504,7 +519,7 @@ const char* kq_status_str(int status) {
 const char* kq_last_error(void) { return g_last_error; }
 
 size_t kq_block_bytes(int fmt) {
-    return fmt == KQ_FMT_Q4_K ? kQ4Bytes : fmt == KQ_FMT_Q6_K ? kQ6Bytes : 0;
+    return fmt == KQ_FMT_Q4_K ? kQ4Bytes : fmt == KQ_FMT_Q6_K ? kQ6Bytes : fmt == KQ_FMT_Q5_K ? kQ5Bytes : 0;
 }
 
 size_t kq_row_bytes(int fmt, int64_t K) {
@@ -792,7 +807,9 @@ static int split_for(int fmt, int64_t N, int64_t K, int* S, int* nbs) {
 }
 
 size_t kq_splitk_workspace_bytes(int fmt, int64_t N, int64_t K, int k) {
-    if ((fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q6_K) || N < 1 || K < 256 || K % 256 != 0 || k < 1 || k > 8) return 0;
+    if ((fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q5_K && fmt != KQ_FMT_Q6_K) || N < 1 || K < 256 || K % 256 != 0 || k < 1 ||
+        k > 8)
+        return 0;
     int S = 1, nbs = 0;
     if (split_for(fmt, N, K, &S, &nbs) != KQ_OK || S <= 1) return 0;
     return sizeof(float) * static_cast<size_t>(S) * k * static_cast<size_t>(N);
@@ -834,7 +851,8 @@ int kq_gemv_splitk(const void* W, int fmt, int64_t N, int64_t K, const float* x,
 
 int kq_unpack(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d, kq_stream_t stream) {
     g_last_error[0] = 0;
-    if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q6_K) return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
+    if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q5_K && fmt != KQ_FMT_Q6_K)
+        return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
     if (n_blocks < 0) return fail(KQ_ERR_INVALID_ARG, "n_blocks < 0");
     if (n_blocks == 0) return KQ_OK;
     if (!W || !q || !sc || !d) return fail(KQ_ERR_INVALID_ARG, "NULL pointer");

@@ -632,17 +632,17 @@ __device__ __noinline__ void stage_x_pro(const ProStage p, uint32_t xs, int ct, 
                    ct >> 5, ct & 31, bar, nthr, 0);
 }
 
-// ----------------------------------- single column, Q4_K: integer dot path
+// ------------------------- single column, Q4_K and Q5_K: integer dot path
 //
-// One Q4_K column runs its inner products on DP4A (four byte products per
+// One Q4_K or Q5_K column runs its inner products on DP4A (four byte products per
 // instruction, exact int32 sums).  The activations of each group of 32
 // consecutive weights are scaled by a power of two 2^sh that puts the
 // group's largest |x| in [2^13, 2^14), rounded to integers xi (|xi| <= 2^14)
 // and stored as a signed high byte xi >> 8 and an unsigned low byte xi & 255
 // (xi = 256*hi + lo).  Per group the staging also keeps P = 2^-sh and
 // Xg = P * sum of the xi (an exact integer sum, |sum| <= 2^19).  A
-// sub-block's sum S of q*xi is then exact (|S| < 2^23, so exact in fp32
-// too), and y = sum over sub-blocks of d*sc*P*S - dmin*m*Xg in fp32: the
+// sub-block's sum S of q*xi is then exact (|S| <= 31 * 32 * 2^14 < 2^24 for
+// Q5_K's 5-bit codes, so exact in fp32 too), and y = sum over sub-blocks of d*sc*P*S - dmin*m*Xg in fp32: the
 // exact dot product of the dequantised weights with the rounded activations
 // P*xi, up to fp32 rounding of the per-sub-block terms.  |x - P*xi| <= P/2
 // <= 2^-14 * (largest |x| of the group), so |y - y_exact| <= 2^-14 * sum
@@ -790,6 +790,66 @@ __device__ __forceinline__ void q4k_unit_int(uint32_t row0, int row_bytes, int b
     out[1][0] = y[1];
 }
 
+// Q5_K unit, one column, on DP4A: as q4k_unit_int, with each code's 5th bit
+// merged in.  Bytes: header 0..15 (as Q4_K), qh 16..47, quants 48..175.
+// Weight 64c+l takes bit 2c of qh[l] (low nibble) and 64c+32+l bit 2c+1
+// (high nibble); the lane's 16-byte half h of a chunk covers l = 16h..16h+15,
+// so one 16-byte load of qh serves both of its chunks.
+__device__ __forceinline__ void q5k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
+                                             float (&out)[2][1]) {
+    const uint32_t blk[2] = {row0 + b * kQ5Bytes, row0 + row_bytes + b * kQ5Bytes};
+    float dd[2], dm[2];
+    uint32_t sc4[2], m4[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint4 hd = ld_s128(blk[r]);
+        q4k_half_scales(hd.y, hd.z, hd.w, H, sc4[r], m4[r]);
+        dd[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x & 0xFFFFu)));
+        dm[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x >> 16)));
+    }
+    float y[2] = {0.f, 0.f};
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * H + cc;
+        const uint32_t gL = xr + kXGroupBytes * (2 * cc), gH = gL + kXGroupBytes;  // groups 2cc, 2cc+1 of the half
+        int hL[2] = {0, 0}, hH[2] = {0, 0};
+        uint32_t lL[2] = {0u, 0u}, lH[2] = {0u, 0u};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 q0 = ld_s128(blk[0] + 48 + 32 * c + 16 * h), q1 = ld_s128(blk[1] + 48 + 32 * c + 16 * h);
+            const uint4 e0 = ld_s128(blk[0] + 16 + 16 * h), e1 = ld_s128(blk[1] + 16 + 16 * h);
+            const uint4 xhL = ld_s128(gL + 16 * h), xlL = ld_s128(gL + 32 + 16 * h);
+            const uint4 xhH = ld_s128(gH + 16 * h), xlH = ld_s128(gH + 32 + 16 * h);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const uint32_t w = u4w(r ? q1 : q0, t), e = u4w(r ? e1 : e0, t);
+                    const uint32_t lo = (w & 0x0F0F0F0Fu) | (((e >> (2 * c)) & 0x01010101u) << 4);
+                    const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) | (((e >> (2 * c + 1)) & 0x01010101u) << 4);
+                    hL[r] = dp4a_us(lo, u4w(xhL, t), hL[r]);
+                    lL[r] = dp4a_uu(lo, u4w(xlL, t), lL[r]);
+                    hH[r] = dp4a_us(hi, u4w(xhH, t), hH[r]);
+                    lH[r] = dp4a_uu(hi, u4w(xlH, t), lH[r]);
+                }
+            }
+        }
+        const float4 iL = ld_s128f(xr + 4 * kXGroupBytes + kXInfoBytes * (2 * cc));
+        const float4 iH = ld_s128f(xr + 4 * kXGroupBytes + kXInfoBytes * (2 * cc + 1));
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const float sL = static_cast<float>(hL[r] * 256 + static_cast<int>(lL[r]));
+            const float sH = static_cast<float>(hH[r] * 256 + static_cast<int>(lH[r]));
+            y[r] = fmaf(dd[r] * byte_f(sc4[r], 2 * cc) * iL.y, sL, y[r]);
+            y[r] = fmaf(-dm[r] * byte_f(m4[r], 2 * cc), iL.x, y[r]);
+            y[r] = fmaf(dd[r] * byte_f(sc4[r], 2 * cc + 1) * iH.y, sH, y[r]);
+            y[r] = fmaf(-dm[r] * byte_f(m4[r], 2 * cc + 1), iH.x, y[r]);
+        }
+    }
+    out[0][0] = y[0];
+    out[1][0] = y[1];
+}
+
 // Dispatch a Q6_K unit to the code path of its alignment class.
 template <int NCOL>
 __device__ __forceinline__ void q6k_unit_dispatch(int kappa, uint32_t row0, int row_bytes, int b, int H,
@@ -852,7 +912,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     const int64_t rc = blockIdx.x / a.ksplit, G = gridDim.x / a.ksplit;
     const int64_t rp_begin = P * rc / G;
     const int64_t rp_end = P * (rc + 1) / G;
-    constexpr int BS = FMT == 1 ? kQ4Bytes : kQ6Bytes;
+    constexpr int BS = block_bytes_of<FMT>();
+    static_assert(FMT != 3 || NCOL == 1, "Q5_K with several columns runs on the tensor cores");
     const int kb0 = ks * a.nbs;
     const int nbl = a.nb - kb0 < a.nbs ? a.nb - kb0 : a.nbs;       // blocks in this range
     const int srow = a.ksplit > 1 ? a.nbs * BS : static_cast<int>(a.row_bytes);  // staged row stride
@@ -882,7 +943,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     int u_rp, u_b, u_H, group, part;
     bool u_active;
     int kappa = 0;
-    if (FMT == 1) {
+    if (FMT != 2) {  // Q4_K and Q5_K: lanes take (row pair, block, half)
         const int LR = a.lanes_per_rp;
         u_rp = ct / LR;
         const int u = ct - u_rp * LR;
@@ -907,14 +968,15 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     // single column with whole row pairs per warp: no cross-warp reduction
     const bool direct = NCOL == 1 && parts == 1;
     int region;
-    if (FMT == 1) region = 2 * u_b + u_H;
+    if (FMT != 2) region = 2 * u_b + u_H;
     else region = ((kappa * (nb >> 3) + (u_b >> 3)) << 1) + u_H;
     const int wp_group = 2 * a.ps * parts * 2 * NCOL;     // floats of one group's double buffer
     // activation copy: fp32 regions (several columns) or the integer groups
     // of the single-column path (kXGroupBytes + kXInfoBytes per 32 weights)
-    // the integer path serves single-column Q4_K; Q6_K keeps the fp32 units
-    // (measured faster for it: 21.0 vs 26.6 us on the 8B down matrix)
-    constexpr bool INT = NCOL == 1 && FMT == 1;
+    // the integer path serves single-column Q4_K and Q5_K; Q6_K keeps the
+    // fp32 units (measured faster for it twice: 21.0 vs 26.6 and 20.0 vs
+    // 22.4 us on the 8B down matrix)
+    constexpr bool INT = NCOL == 1 && FMT != 2;
     const uint32_t xcopy = INT ? kXRegionBytes * 2 * nb : 4 * NCOL * xcs;
     const uint32_t xs_s = smem_u32(xs) + (shared_x ? 0 : g * xcopy);
     const uint32_t xri = x_region(xs_s, u_b, u_H);  // this lane's integer region (Q4_K)
@@ -955,8 +1017,10 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
         const bool work = u_active && u_rp < st.nrp && !*abort_flag;
         if (work) {
             const uint32_t row0 = sbuf_s + slot * a.stage_bytes + 2 * u_rp * srow;
-            if constexpr (INT) {
+            if constexpr (INT && FMT == 1) {
                 q4k_unit_int(row0, srow, u_b, u_H, xri, out);
+            } else if constexpr (INT) {
+                q5k_unit_int(row0, srow, u_b, u_H, xri, out);
             } else if constexpr (FMT == 1) {
                 q4k_unit<NCOL>(row0, srow, u_b, u_H, xr, xcs, out);
             } else {

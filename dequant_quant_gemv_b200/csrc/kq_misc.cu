@@ -20,8 +20,10 @@ __device__ int g_kq_fault = 0;
 __global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d) {
     const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (b >= nblocks) return;
-    if (fmt == 1) {
-        const uint8_t* blk = W + b * kQ4Bytes;
+    if (fmt == 1 || fmt == 3) {
+        // Q4_K, Q5_K: the same header; Q5_K quants sit after its 32 qh bytes
+        const uint8_t* blk = W + b * (fmt == 1 ? kQ4Bytes : kQ5Bytes);
+        const uint8_t* qs = blk + (fmt == 1 ? 16 : 48);
         const uint4 hd = *reinterpret_cast<const uint4*>(blk);
         for (int H = 0; H < 2; ++H) {
             uint32_t sc4, m4;
@@ -34,11 +36,16 @@ __global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_
         d[2 * b] = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x & 0xFFFFu)));
         d[2 * b + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x >> 16)));
         for (int w = 0; w < 32; ++w) {
-            const uint32_t v = *reinterpret_cast<const uint32_t*>(blk + 16 + 4 * w);
+            const uint32_t v = *reinterpret_cast<const uint32_t*>(qs + 4 * w);
             const int c = w >> 3, l0 = (w & 7) * 4;
+            // Q5_K: 5th bits of chunk c at bits 2c, 2c+1 of qh[l]
+            const uint32_t e = fmt == 3 ? *reinterpret_cast<const uint32_t*>(blk + 16 + l0) : 0u;
             for (int k = 0; k < 4; ++k) {
-                q[256 * b + 64 * c + l0 + k] = static_cast<uint8_t>((v >> (8 * k)) & 15u);
-                q[256 * b + 64 * c + 32 + l0 + k] = static_cast<uint8_t>((v >> (8 * k + 4)) & 15u);
+                const uint32_t eb = e >> (8 * k);
+                q[256 * b + 64 * c + l0 + k] =
+                    static_cast<uint8_t>(((v >> (8 * k)) & 15u) | (((eb >> (2 * c)) & 1u) << 4));
+                q[256 * b + 64 * c + 32 + l0 + k] =
+                    static_cast<uint8_t>(((v >> (8 * k + 4)) & 15u) | (((eb >> (2 * c + 1)) & 1u) << 4));
             }
         }
     } else {

@@ -40,7 +40,7 @@ namespace kq {
 constexpr int kMmaRowPairs = 8;  // 16 rows per stage
 // K-steps per super-block: 16 of quants, plus one of mins for Q4_K
 template <int FMT>
-__host__ __device__ constexpr int mma_steps() { return FMT == 1 ? 17 : 16; }
+__host__ __device__ constexpr int mma_steps() { return FMT == 2 ? 16 : 17; }
 
 // D += A * B for one m16n8k16 tile (row-major A, column-major B).
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -141,7 +141,7 @@ __device__ __forceinline__ void store_b_entry(uint32_t xb, int bl, int s, int q,
 // feed K-step s = 4c + t.
 template <int FMT>
 __device__ __forceinline__ void b_slot(int w, int& s, int& q) {
-    if constexpr (FMT == 1) {
+    if constexpr (FMT != 2) {  // Q4_K and Q5_K share the quant order
         const int hi = (w >> 5) & 1;
         const int beta = 32 * (w >> 6) + (w & 31);
         const int ch = beta >> 4, u = (beta >> 2) & 3;
@@ -241,7 +241,7 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                 int st, sq;
                 b_slot<FMT>(128 * h + 4 * lane, st, sq);
                 store_b_entry<FMT, NT>(xb, bl, st, sq, col, t);
-                if constexpr (FMT != 1) continue;
+                if constexpr (FMT == 2) continue;
                 // sub-block 4h + lane/8: the 8 lanes of this group, fixed order
                 float X = (v[u][h].x + v[u][h].y) + (v[u][h].z + v[u][h].w);
                 X += __shfl_xor_sync(0xffffffffu, X, 1);
@@ -369,6 +369,134 @@ __device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, 
         const uint32_t s_lo = xbl + 8u * NT * 32 * (2 * j), s_hi = s_lo + 8u * NT * 32;  // steps 2j, 2j+1
         q4k_step<NT, 0x000F000Fu>(acc, x0, x1, x0 >> 8, x1 >> 8, mlo[0][c], alo[0][c], mlo[1][c], alo[1][c], s_lo);
         q4k_step<NT, 0x00F000F0u>(acc, x0, x1, x0 >> 8, x1 >> 8, mhi[0][c], ahi[0][c], mhi[1][c], ahi[1][c], s_hi);
+    }
+    {
+        const uint32_t s_m = xbl + 8u * NT * 32 * 16;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const uint2 bm = ld_s64u(s_m + 8 * n);
+            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bm.x, bm.y);
+        }
+    }
+    const float d0 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg.x & 0xFFFFu)));
+    const float m0 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg.x >> 16)));
+    const float d1 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg8.x & 0xFFFFu)));
+    const float m1 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg8.x >> 16)));
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const float2 f = ld_s64f(bsc + 8u * (4 * n + q));  // (2^-sh, 2^(5-sh)) of column 4n+q
+        ys[0][n] = fmaf(d0 * f.x, acc[n][0] + acc[n][1], ys[0][n]);
+        ys[1][n] = fmaf(d1 * f.x, acc[n][2] + acc[n][3], ys[1][n]);
+        ym[0][n] = fmaf(m0 * f.y, accm[n][0] + accm[n][1], ym[0][n]);
+        ym[1][n] = fmaf(m1 * f.y, accm[n][2] + accm[n][3], ym[1][n]);
+    }
+}
+
+// Q5_K K-step: as q4k_step, with each code's 5th bit merged in.  hc0..hc3
+// replace the exponent constant of the four fp16 pairs: 0x6400 in each half
+// with the 5th bit at bit 4 (low nibble: 1024 + q) or bit 8 (high nibble:
+// 1024 + 16q) of the half; the scale operands are Q4_K's.
+template <int NT, uint32_t MASK>
+__device__ __forceinline__ void q5k_step(float (&d)[NT][4], uint32_t xg, uint32_t xg8, uint32_t xsg, uint32_t xsg8,
+                                         uint32_t mg, uint32_t ag, uint32_t mg8, uint32_t ag8, uint32_t baddr,
+                                         uint32_t hc0, uint32_t hc1, uint32_t hc2, uint32_t hc3) {
+    if constexpr (NT == 1) {
+        asm volatile(
+            "{\n\t.reg .b32 t0, t1, t2, t3, a0, a1, a2, a3, b0, b1;\n\t"
+            "lop3.b32 t0, %4, %13, %14, 0xEA;\n\t"
+            "lop3.b32 t1, %5, %13, %15, 0xEA;\n\t"
+            "lop3.b32 t2, %6, %13, %16, 0xEA;\n\t"
+            "lop3.b32 t3, %7, %13, %17, 0xEA;\n\t"
+            "fma.rn.f16x2 a0, t0, %8, %9;\n\t"
+            "fma.rn.f16x2 a1, t1, %10, %11;\n\t"
+            "fma.rn.f16x2 a2, t2, %8, %9;\n\t"
+            "fma.rn.f16x2 a3, t3, %10, %11;\n\t"
+            "ld.shared.v2.b32 {b0, b1}, [%12];\n\t"
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {a0, a1, a2, a3}, {b0, b1}, "
+            "{%0, %1, %2, %3};\n\t}"
+            : "+f"(d[0][0]), "+f"(d[0][1]), "+f"(d[0][2]), "+f"(d[0][3])
+            : "r"(xg), "r"(xg8), "r"(xsg), "r"(xsg8), "r"(mg), "r"(ag), "r"(mg8), "r"(ag8), "r"(baddr), "n"(MASK),
+              "r"(hc0), "r"(hc1), "r"(hc2), "r"(hc3));
+    } else {
+        asm volatile(
+            "{\n\t.reg .b32 t0, t1, t2, t3, a0, a1, a2, a3, b0, b1, b2, b3;\n\t"
+            "lop3.b32 t0, %8, %17, %18, 0xEA;\n\t"
+            "lop3.b32 t1, %9, %17, %19, 0xEA;\n\t"
+            "lop3.b32 t2, %10, %17, %20, 0xEA;\n\t"
+            "lop3.b32 t3, %11, %17, %21, 0xEA;\n\t"
+            "fma.rn.f16x2 a0, t0, %12, %13;\n\t"
+            "fma.rn.f16x2 a1, t1, %14, %15;\n\t"
+            "fma.rn.f16x2 a2, t2, %12, %13;\n\t"
+            "fma.rn.f16x2 a3, t3, %14, %15;\n\t"
+            "ld.shared.v4.b32 {b0, b1, b2, b3}, [%16];\n\t"
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {a0, a1, a2, a3}, {b0, b1}, "
+            "{%0, %1, %2, %3};\n\t"
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%4, %5, %6, %7}, {a0, a1, a2, a3}, {b2, b3}, "
+            "{%4, %5, %6, %7};\n\t}"
+            : "+f"(d[0][0]), "+f"(d[0][1]), "+f"(d[0][2]), "+f"(d[0][3]), "+f"(d[1][0]), "+f"(d[1][1]),
+              "+f"(d[1][2]), "+f"(d[1][3])
+            : "r"(xg), "r"(xg8), "r"(xsg), "r"(xsg8), "r"(mg), "r"(ag), "r"(mg8), "r"(ag8), "r"(baddr), "n"(MASK),
+              "r"(hc0), "r"(hc1), "r"(hc2), "r"(hc3));
+    }
+}
+
+// Q5_K super-block b of rows g and g+8: q4k_mma_block on the Q5_K byte
+// offsets (quants at 48, qh at 16), the lane's 5th bits from qh bytes
+// l = 16(q%2) .. 16(q%2)+15, which serve both of its chunks q/2 and q/2 + 2.
+template <int NT>
+__device__ __forceinline__ void q5k_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t bsc,
+                                              uint32_t sel, uint32_t msel, int q, float (&ys)[2][NT],
+                                              float (&ym)[2][NT]) {
+    const uint32_t o = static_cast<uint32_t>(b) * kQ5Bytes;
+    const uint4 hg = ld_s128(rg + o), hg8 = ld_s128(rg8 + o);
+    uint4 w[2][2];  // [row][chunk q / q+4 (16-byte segments)]
+    w[0][0] = ld_s128(rg + o + 48 + 16 * q);
+    w[0][1] = ld_s128(rg + o + 112 + 16 * q);
+    w[1][0] = ld_s128(rg8 + o + 48 + 16 * q);
+    w[1][1] = ld_s128(rg8 + o + 112 + 16 * q);
+    const uint4 e[2] = {ld_s128(rg + o + 16 + 16 * (q & 1)), ld_s128(rg8 + o + 16 + 16 * (q & 1))};
+    uint32_t mlo[2][2], alo[2][2], mhi[2][2], ahi[2][2], mins[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint4 h = r ? hg8 : hg;
+        uint32_t sc0, m0, sc1, m1;
+        q4k_half_scales(h.y, h.z, h.w, 0, sc0, m0);
+        q4k_half_scales(h.y, h.z, h.w, 1, sc1, m1);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const __half2 S = u2h2(byte_pair_h2(c ? sc1 : sc0, sel));
+            const __half2 slo = __low2half2(S), shi = __high2half2(S);
+            mlo[r][c] = h22u(slo);
+            alo[r][c] = h22u(__hmul2(slo, u2h2(kH2_m1024)));
+            mhi[r][c] = h22u(__hmul2(shi, u2h2(kH2_1_16)));
+            ahi[r][c] = h22u(__hmul2(shi, u2h2(kH2_m64)));
+        }
+        mins[r] = byte_pair_h2(q < 2 ? m0 : m1, msel);
+    }
+    float acc[NT][4], accm[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = accm[n][i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int c = j >> 2;
+        const int sh = 2 * ((q >> 1) + 2 * c);  // bit of the low-nibble codes (chunk q/2 + 2c)
+        const uint32_t x0 = u4w(w[0][c], j & 3), x1 = u4w(w[1][c], j & 3);
+        const uint32_t e0 = u4w(e[0], j & 3), e1 = u4w(e[1], j & 3);
+        const uint32_t bl0 = (e0 >> sh) & 0x01010101u, bl1 = (e1 >> sh) & 0x01010101u;
+        const uint32_t bh0 = (e0 >> (sh + 1)) & 0x01010101u, bh1 = (e1 >> (sh + 1)) & 0x01010101u;
+        // low nibbles: bytes 0, 2 keep bit 4 of their halves; bytes 1, 3 via >> 8
+        const uint32_t l0 = ((bl0 << 4) & 0x00100010u) | 0x64006400u, l1 = ((bl1 << 4) & 0x00100010u) | 0x64006400u;
+        const uint32_t l2 = ((bl0 >> 4) & 0x00100010u) | 0x64006400u, l3 = ((bl1 >> 4) & 0x00100010u) | 0x64006400u;
+        // high nibbles (16n): the 5th bit is worth 256, bit 8 of the half
+        const uint32_t h0 = ((bh0 << 8) & 0x01000100u) | 0x64006400u, h1 = ((bh1 << 8) & 0x01000100u) | 0x64006400u;
+        const uint32_t h2 = (bh0 & 0x01000100u) | 0x64006400u, h3 = (bh1 & 0x01000100u) | 0x64006400u;
+        const uint32_t s_lo = xbl + 8u * NT * 32 * (2 * j), s_hi = s_lo + 8u * NT * 32;  // steps 2j, 2j+1
+        q5k_step<NT, 0x000F000Fu>(acc, x0, x1, x0 >> 8, x1 >> 8, mlo[0][c], alo[0][c], mlo[1][c], alo[1][c], s_lo,
+                                  l0, l1, l2, l3);
+        q5k_step<NT, 0x00F000F0u>(acc, x0, x1, x0 >> 8, x1 >> 8, mhi[0][c], ahi[0][c], mhi[1][c], ahi[1][c], s_hi,
+                                  h0, h1, h2, h3);
     }
     {
         const uint32_t s_m = xbl + 8u * NT * 32 * 16;
@@ -525,7 +653,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
     const int64_t rp_begin = rps * rc / G;
     const int64_t rp_end = rps * (rc + 1) / G;
     const int total = static_cast<int>((rp_end - rp_begin + kMmaRowPairs - 1) / kMmaRowPairs);
-    constexpr int BS = FMT == 1 ? kQ4Bytes : kQ6Bytes;
+    constexpr int BS = block_bytes_of<FMT>();
     const int kb0 = ks * a.nbs;
     const int nbl = a.nb - kb0 < a.nbs ? a.nb - kb0 : a.nbs;
     const uint32_t rem = static_cast<uint32_t>(kb0 * BS) & 15u;  // Q6_K ranges may start off a 16-byte boundary
@@ -602,6 +730,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
                 for (int b = cw; b < nbl; b += kConsumerWarps) {
                     const uint32_t xbl = xlane + 8u * NT * 32 * mma_steps<FMT>() * b, bsc = bsc_s + 8u * NC * b;
                     if constexpr (FMT == 1) q4k_mma_block<NT>(rg, rg8, b, xbl, bsc, sel, msel, q, ys, ym);
+                    else if constexpr (FMT == 3) q5k_mma_block<NT>(rg, rg8, b, xbl, bsc, sel, msel, q, ys, ym);
                     else if (((rem >> 1) + b) & 1) q6k_mma_block<NT, true>(rg, rg8, b, xbl, bsc, q, ys);
                     else q6k_mma_block<NT, false>(rg, rg8, b, xbl, bsc, q, ys);
                 }

@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
         // this step's activations, staged by all consumer threads
         const GemvArgs a = step_view(s);
         float rinv = 1.f;
-        if (s.fmt == 1) {
+        if (s.fmt != 2) {  // Q4_K and Q5_K: integer regions
             if (s.pro) stage_all<1, 1, true, true>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
             else stage_all<1, 1, true, false>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
         } else {
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
         int u_rp, u_b, u_H, group, part;
         bool u_active;
         int kappa = 0;
-        if (s.fmt == 1) {
+        if (s.fmt != 2) {
             const int LR = s.lanes_per_rp;
             u_rp = ct / LR;
             const int u = ct - u_rp * LR;
@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
         }
         const int parts = s.parts;
         const bool direct = parts == 1;
-        const int region = s.fmt == 1 ? 2 * u_b + u_H : ((kappa * (nb >> 3) + (u_b >> 3)) << 1) + u_H;
+        const int region = s.fmt != 2 ? 2 * u_b + u_H : ((kappa * (nb >> 3) + (u_b >> 3)) << 1) + u_H;
         const uint32_t xri = x_region(xs_s, u_b, u_H);
         const uint32_t xr = xs_s + 4 * (region * kRegion);
         const uint32_t wp_s = smem_u32(smem + A.wp_offset) + 4 * g * (2 * s.ps * parts * 2);
@@ -240,6 +240,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
             if (work) {
                 const uint32_t rw = sbuf_s + slot * A.slot_bytes + 2 * u_rp * srow;
                 if (s.fmt == 1) q4k_unit_int(rw, srow, u_b, u_H, xri, out);
+                else if (s.fmt == 3) q5k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else q6k_unit_dispatch<1>(kappa, rw, srow, u_b, u_H, xr, xcs, out);
             }
             // butterfly over the lanes of this row pair (fixed order)

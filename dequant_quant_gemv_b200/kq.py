@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(_PKG, "libkq.so")
 
 Q4_K = 1
 Q6_K = 2
-FORMATS = {"q4_k": Q4_K, "q6_k": Q6_K}
+Q5_K = 3
+FORMATS = {"q4_k": Q4_K, "q6_k": Q6_K, "q5_k": Q5_K}
 BLOCK_BYTES = {Q4_K: 144, Q6_K: 210}
 
 OK = 0

@@ -1,6 +1,6 @@
 /*
  * kq.h — libkq: decode-time matrix-vector products over GGUF K-quant
- * weights (Q4_K, Q6_K) on NVIDIA B200 (sm_100a), with the weights
+ * weights (Q4_K, Q5_K, Q6_K) on NVIDIA B200 (sm_100a), with the weights
  * dequantised only in registers inside the fused kernels.
  *
  * What the method is (by page):
@@ -22,6 +22,13 @@
  *   Q4_K super-block, 144 bytes, 256 weights in 8 sub-blocks of 32:
  *     fp16 d | fp16 dmin | 12 bytes of 6-bit scales sc_j and mins m_j |
  *     128 bytes of 4-bit quants q.   w = d*sc_j*q - dmin*m_j.
+ *   Q5_K super-block, 176 bytes, 256 weights in 8 sub-blocks of 32:
+ *     fp16 d | fp16 dmin | 12 bytes of scales and mins (as Q4_K) |
+ *     32 bytes qh of 5th bits | 128 bytes of low 4 bits.  Weight 64c+l
+ *     (l < 32) takes the low nibble of byte 32c+l and bit 2c of qh[l];
+ *     weight 64c+32+l the high nibble and bit 2c+1.
+ *     w = d*sc_j*q - dmin*m_j, q in 0..31.  (A K-quant of the Q2_K..Q6_K
+ *     family "RunNburn - Run a 295B MoE ..." runs natively.)
  *   Q6_K super-block, 210 bytes, 256 weights in 16 groups of 16:
  *     128 bytes low 4 bits | 64 bytes high 2 bits | 16 int8 scales s_g |
  *     fp16 d.   w = d*s_g*(q - 32), q in 0..63.
@@ -32,13 +39,14 @@
  *  - All pointers named W, x, y, ids, status are DEVICE pointers owned by the
  *    caller; libkq never frees or retains them past the call (the chain object
  *    below is the exception and says so).
- *  - W must be 16-byte aligned, and so must every row: always true for Q4_K;
- *    for Q6_K it requires K % 2048 == 0.  x and y must be 4-byte aligned.
+ *  - W must be 16-byte aligned, and so must every row: always true for Q4_K
+ *    and Q5_K; for Q6_K it requires K % 2048 == 0.  x and y must be 4-byte
+ *    aligned.
  *  - Calls are asynchronous on `stream` (0 = the legacy default stream).  The
  *    return value reports argument validation and launch errors only
  *    (KQ_ERR_CUDA carries cudaGetLastError()); kq_last_error() gives text.
  *  - Arithmetic: quants are unpacked exactly; sums are fp32 (or exact
- *    integers).  Single-column Q4_K rounds each activation to a 14-bit
+ *    integers).  Single-column Q4_K and Q5_K round each activation to a 14-bit
  *    integer on a power-of-two grid per group of 32 (error at most 2^-14 of
  *    the group's largest |x|); single-column Q6_K multiplies in fp32; two or
  *    more columns run on the tensor cores with exact fp16 weight operands and
@@ -73,7 +81,8 @@ typedef struct CUstream_st* kq_stream_t;
 
 typedef enum {
     KQ_FMT_Q4_K = 1,
-    KQ_FMT_Q6_K = 2
+    KQ_FMT_Q6_K = 2,
+    KQ_FMT_Q5_K = 3
 } kq_fmt;
 
 typedef enum {

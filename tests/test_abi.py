@@ -47,7 +47,9 @@ def test_host_only_helpers(libkq):
     assert L.kq_row_bytes(1, 4096) == 16 * 144
     assert L.kq_row_bytes(2, 14336) == 56 * 210
     assert L.kq_row_bytes(1, 300) == 0
-    assert L.kq_block_bytes(3) == 0
+    assert L.kq_block_bytes(3) == 176                 # Q5_K
+    assert L.kq_row_bytes(3, 4096) == 16 * 176
+    assert L.kq_block_bytes(4) == 0                   # no such format
     assert L.kq_status_str(0) == b"ok"
     assert L.kq_version() >= 100
 

@@ -26,7 +26,8 @@ def _cuda():
 
 
 # ------------------------------------------------------------ bit-exact
-@pytest.mark.parametrize("fmt,N,K", [("q4_k", 4096, 4096), ("q6_k", 64, 14336), ("q6_k", 3, 2048)])
+@pytest.mark.parametrize("fmt,N,K", [("q4_k", 4096, 4096), ("q6_k", 64, 14336), ("q6_k", 3, 2048),
+                                     ("q5_k", 2048, 4096), ("q5_k", 3, 256)])
 def test_unpack_bit_exact(fmt, N, K):
     W = matrix(fmt, 1000 + N, N, K)
     nb = N * K // 256
@@ -44,6 +45,8 @@ SHAPES = [
     ("q4_k", 257, 4096), ("q4_k", 301, 8192), ("q4_k", 5, 1280), ("q4_k", 9, 32768), ("q4_k", 2, 5120),
     ("q6_k", 1, 2048), ("q6_k", 5, 2048), ("q6_k", 64, 14336), ("q6_k", 37, 28672), ("q6_k", 300, 4096),
     ("q6_k", 11, 16384),
+    ("q5_k", 1, 256), ("q5_k", 7, 768), ("q5_k", 257, 4096), ("q5_k", 301, 8192), ("q5_k", 9, 32768),
+    ("q5_k", 5, 1280), ("q5_k", 4096, 4096), ("q5_k", 2, 14336),
 ]
 
 
@@ -86,6 +89,34 @@ def test_q4k_zero_quants_and_zero_mins_give_exact_zero():
     assert torch.all(y == 0)
 
 
+def test_q5k_zero_quants_and_zero_mins_give_exact_zero():
+    N, K = 70, 4096
+    nb = N * K // 256
+    lg = kqgen.q5k_draw(121, nb)
+    W = kqgen.q5k_pack(np.zeros_like(lg["q"]), lg["sc"], np.zeros_like(lg["m"]), lg["d"], lg["dmin"])
+    y = kq.gemv(dev(W), "q5_k", N, K, dev(x_vec(122, K)))
+    assert torch.all(y == 0)
+    Y = kq.gemv_multi(dev(W), "q5_k", N, K, dev(np.stack([x_vec(123 + c, K) for c in range(3)])))
+    assert torch.all(Y == 0)
+
+
+def test_q5k_zero_quants_closed_form():
+    """All-zero Q5_K quants: y = -sum_j dmin*m_j*(sum of x over sub-block j),
+    as for Q4_K (the 5th bits all zero too)."""
+    N, K = 70, 4096
+    nb = N * K // 256
+    lg = kqgen.q5k_draw(124, nb)
+    W = kqgen.q5k_pack(np.zeros_like(lg["q"]), lg["sc"], lg["m"], lg["d"], lg["dmin"])
+    x = x_vec(125, K)
+    y = kq.gemv(dev(W), "q5_k", N, K, dev(x))
+    X = x.astype(np.float64).reshape(K // 32, 32).sum(axis=1).reshape(K // 256, 8)
+    dmin = lg["dmin"].view(np.float16).astype(np.float64).reshape(N, K // 256)
+    m = lg["m"].astype(np.float64).reshape(N, K // 256, 8)
+    want = -np.einsum("rb,rbj,bj->r", dmin, m, X)
+    s = np.einsum("rb,rbj,bj->r", dmin, m, np.abs(x.astype(np.float64)).reshape(K // 32, 32).sum(1).reshape(K // 256, 8))
+    assert_close(y, want, s, "q5k zero quants")
+
+
 def test_q4k_zero_quants_closed_form():
     N, K = 70, 4096
     nb = N * K // 256
@@ -122,7 +153,7 @@ def test_unit_scales_integer_matvec():
     assert_close(y, Q @ x.astype(np.float64), np.abs(Q) @ np.abs(x.astype(np.float64)), "unit scales")
 
 
-@pytest.mark.parametrize("fmt,K", [("q4_k", 4096), ("q6_k", 14336)])
+@pytest.mark.parametrize("fmt,K", [("q4_k", 4096), ("q6_k", 14336), ("q5_k", 4096)])
 def test_one_hot_extracts_column(fmt, K):
     N = 16
     W = matrix(fmt, 29, N, K)
@@ -153,7 +184,9 @@ def test_linearity():
 # ---------------------------------------------------------- multi column
 @pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q4_k", 17, 768),
                                      ("q4_k", 4096, 4096), ("q4_k", 33, 14336), ("q6_k", 64, 4096),
-                                     ("q6_k", 41, 2048), ("q6_k", 4096, 2048), ("q6_k", 3, 14336)])
+                                     ("q6_k", 41, 2048), ("q6_k", 4096, 2048), ("q6_k", 3, 14336),
+                                     ("q5_k", 300, 4096), ("q5_k", 33, 14336), ("q5_k", 4096, 4096),
+                                     ("q5_k", 17, 768)])
 @pytest.mark.parametrize("k", [2, 3, 4, 5, 8])
 def test_multi_columns_independent_and_match_oracle(fmt, N, K, k):
     """Each column of a k-column call equals the same column of an 8-column
@@ -171,7 +204,7 @@ def test_multi_columns_independent_and_match_oracle(fmt, N, K, k):
         assert_close(Y[c], y_ref[c], s_ref[c], f"col {c}")
 
 
-@pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336)])
+@pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q5_k", 300, 4096)])
 def test_single_column_of_multi_call_matches_oracle(fmt, N, K):
     """k = 1 through gemv_multi is the single-column kernel, bitwise."""
     W = matrix(fmt, 32, N, K)
@@ -184,7 +217,7 @@ def test_single_column_of_multi_call_matches_oracle(fmt, N, K):
     assert_close(Y[0], y_ref, s_ref)
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k"])
 @pytest.mark.parametrize("scale", [1e-30, 1e-6, 1.0, 3e3, 1e20])
 def test_multi_column_scale_range(fmt, scale):
     """Activations far from 1 in either direction (the kernel rescales each
@@ -252,12 +285,13 @@ def test_invalid_arguments_are_rejected():
 
 
 # ------------------------------------------- single-column integer path
-def test_q4k_single_column_within_activation_rounding_bound():
-    """Single-column Q4_K rounds each activation to a 14-bit integer on a
-    power-of-two grid per group of 32, so |x - x'| <= 2^-14 * (largest |x|
-    of the group).  The error must stay within that bound (plus fp32
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k"])
+def test_single_column_within_activation_rounding_bound(fmt):
+    """Single-column Q4_K and Q5_K round each activation to a 14-bit integer
+    on a power-of-two grid per group of 32, so |x - x'| <= 2^-14 * (largest
+    |x| of the group).  The error must stay within that bound (plus fp32
     rounding slack), computed from the oracle's dequantised weights."""
-    fmt, N, K = "q4_k", 256, 4096
+    N, K = 256, 4096
     W = matrix(fmt, 77, N, K)
     x = x_vec(78, K)
     y = kq.gemv(dev(W), fmt, N, K, dev(x)).cpu().numpy().astype(np.float64)
@@ -270,7 +304,7 @@ def test_q4k_single_column_within_activation_rounding_bound():
     assert np.all(err <= bound + slack), float(np.max(err / (bound + slack)))
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k"])
 @pytest.mark.parametrize("scale", [1e-30, 1e-6, 3e3, 1e20])
 def test_single_column_scale_range(fmt, scale):
     """Single column with activations far from 1: the integer path scales

@@ -26,6 +26,8 @@ def _cuda():
     ("q4_k", 16, 2048, 768, True),    # down shape, one x per routed id
     ("q6_k", 6, 130, 2048, True),
     ("q4_k", 5, 33, 256, True),       # odd rows per expert
+    ("q5_k", 16, 768, 2048, False),
+    ("q5_k", 8, 2048, 768, True),
 ])
 def test_moe_parity(fmt, E, N, K, per_id):
     W = matrix(fmt, 300 + E + N, E * N, K)

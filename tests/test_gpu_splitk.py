@@ -20,7 +20,8 @@ def _cuda():
 
 
 SHAPES = [("q4_k", 1, 4096), ("q4_k", 2, 4096), ("q4_k", 17, 4096), ("q4_k", 64, 32768), ("q4_k", 100, 2048),
-          ("q4_k", 5, 768), ("q6_k", 3, 14336), ("q6_k", 64, 28672), ("q6_k", 9, 2048)]
+          ("q4_k", 5, 768), ("q6_k", 3, 14336), ("q6_k", 64, 28672), ("q6_k", 9, 2048), ("q5_k", 17, 4096),
+          ("q5_k", 3, 14336)]
 
 
 @pytest.mark.parametrize("fmt,N,K", SHAPES)
