@@ -107,6 +107,8 @@ WORKLOADS = {
     "llama70b_resident_steps": "the 70B-shaped resident chain through kq_gemv_steps",
     "llama70b_stream": "Llama-3.3-70B-shaped decode chain, 80 layers, weights in pinned host memory streamed "
                        "through 4 device layer slots",
+    "llama70b_stream_20gb": "the streamed 70B-shaped chain within a 20 GB device budget: the leading layers that "
+                            "fit stay resident beside 4 slots, the rest stream (kq_chain_plan)",
 }
 
 
@@ -388,7 +390,7 @@ class Streamed:
 
     graphable = False
 
-    def __init__(self, torch, kq, kqgen, spec, seed, n_slots=4):
+    def __init__(self, torch, kq, kqgen, spec, seed, n_slots=4, budget=None):
         self.torch, self.kq, self.spec = torch, kq, spec
         self.weight_bytes = sum(N * row_bytes(f, K) for mats in spec for (_, f, N, K, _) in mats)
         # one host buffer for every weight, page-locked in place (the torch
@@ -417,7 +419,15 @@ class Streamed:
                 xo += K
                 yo += N
         self.xs, self.ys = xs, ys
-        self.chain = kq.Chain(mats, n_slots=n_slots)
+        # with a device-memory budget: the leading layers that fit stay
+        # resident (kq_chain_plan), the rest stream
+        self.n_resident = 0
+        if budget is not None:
+            self.n_resident, n_slots = kq.chain_plan([[(None, f, N, K) for (_, f, N, K) in r] for r in mats], budget,
+                                                     max_slots=n_slots)
+        self.streamed_bytes = sum(N * row_bytes(f, K) for li, r in enumerate(mats) for (_, f, N, K) in r
+                                  if li >= self.n_resident)
+        self.chain = kq.Chain(mats, n_slots=n_slots, n_resident=self.n_resident)
         self.launches = [None] * sum(len(r) for r in mats)
 
     def step(self, stream):
@@ -450,6 +460,8 @@ def make_workload(name, torch, kq, kqgen, seed):
         return Resident(torch, kq, kqgen, chain_spec("llama70b"), seed, steps=name.endswith("_steps"))
     if name == "llama70b_stream":
         return Streamed(torch, kq, kqgen, chain_spec("llama70b"), seed)
+    if name == "llama70b_stream_20gb":
+        return Streamed(torch, kq, kqgen, chain_spec("llama70b"), seed, budget=20 * 10**9)
     raise KeyError(name)
 
 
@@ -677,10 +689,12 @@ def bench_kq(args, rank, world):
         result["kernels"] = per_kind
     if isinstance(wl, Streamed):
         pk = h2d_peak_gbs(torch)
+        h2d = job_rate(wl.streamed_bytes, args.steps, world, ms) / 1e9 / world
         result["roofline"] = {"bound": "pcie_h2d", "kernel": "H2D copies of the layer ring",
-                              "achieved": round(gbs / world, 2), "peak": round(pk, 2),
+                              "achieved": round(h2d, 2), "peak": round(pk, 2),
                               "peak_source": "measured here (512 MiB pinned copy)", "unit": "GB/s",
-                              "frac": round(gbs / world / pk, 4), "traffic": None}
+                              "frac": round(h2d / pk, 4), "traffic": None,
+                              "streamed_bytes_per_step": wl.streamed_bytes, "resident_layers": wl.n_resident}
         result["gpu_launches"] = 4 * len(wl.spec) * args.steps
     return result
 
@@ -699,7 +713,7 @@ def cpu_baseline(args, budget_s=15.0):
     else:
         base = {"llama8b_chain": "llama8b", "llama8b_q5k_chain": "llama8b_q5k", "verify8b_q5k_k8": "llama8b_q5k", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
                 "llama8b_layer_fused_steps": "llama8b", "llama70b_resident": "llama70b",
-                "llama70b_resident_steps": "llama70b", "llama70b_stream": "llama70b"}
+                "llama70b_resident_steps": "llama70b", "llama70b_stream": "llama70b", "llama70b_stream_20gb": "llama70b"}
         name = base.get(args.workload, "llama8b" if args.workload.startswith("verify") else args.workload)
         spec = chain_spec(name)
         per_token = sum(N * row_bytes(f, K) for mats in spec for (_, f, N, K, _) in mats)
@@ -744,8 +758,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.steps is None:
-        args.steps = {"llama70b_stream": 3, "llama70b_resident": 50, "llama70b_resident_steps": 50}.get(args.workload,
-                                                                                                       300)
+        args.steps = {"llama70b_stream": 3, "llama70b_stream_20gb": 5, "llama70b_resident": 50,
+                      "llama70b_resident_steps": 50}.get(args.workload, 300)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
 

@@ -16,6 +16,13 @@
 // The copy engine therefore runs up to n_slots layers ahead of the SMs, and
 // the kernels are exactly the resident kq_gemv kernels, so a streamed run
 // gives bitwise the same outputs as a resident run.
+//
+// Residency ("Kortex: Streaming 70B Models on Consumer GPUs", Key components:
+// the layers that fit stay in VRAM, the rest stream): the first n_resident
+// layers are copied once, when the chain is created, into device memory of
+// their own; a run launches their GEMVs straight away and streams only the
+// remaining layers, layer l through slot (l - n_resident) % n_slots.
+// kq_chain_plan picks n_resident and n_slots for a device-memory budget.
 #include <cuda_runtime.h>
 
 #include <chrono>
@@ -32,6 +39,8 @@
 struct kq_chain {
     std::vector<kq_matrix_desc> mats;   // host-pinned weights, n_layers * per_layer
     int n_layers = 0, per_layer = 0, n_slots = 0;
+    int n_resident = 0;                 // leading layers kept in `resident`
+    uint8_t* resident = nullptr;        // n_resident * slot_bytes device bytes
     size_t slot_bytes = 0;
     std::vector<size_t> offsets;        // byte offset of each matrix within its slot
     uint8_t* ring = nullptr;            // n_slots * slot_bytes device bytes
@@ -56,6 +65,20 @@ int chain_fail(int status, const char* msg, cudaError_t err = cudaSuccess) {
 
 size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
 
+// Bytes of one layer as the chain lays it out (each matrix 256-byte
+// aligned), and the matrices' offsets; 0 if a layer's shapes are invalid.
+size_t layer_layout(const kq_matrix_desc* mats, int per_layer, std::vector<size_t>* offsets) {
+    size_t off = 0;
+    for (int m = 0; m < per_layer; ++m) {
+        const kq_matrix_desc& d = mats[m];
+        const size_t rb = kq_row_bytes(d.fmt, d.K);
+        if (rb == 0 || d.N < 1) return 0;
+        if (offsets) (*offsets)[m] = off;
+        off = round_up(off + static_cast<size_t>(d.N) * rb, 256);
+    }
+    return off;
+}
+
 void destroy(kq_chain* c) {
     if (!c) return;
     for (auto e : c->ready) cudaEventDestroy(e);
@@ -63,6 +86,7 @@ void destroy(kq_chain* c) {
     if (c->done) cudaEventDestroy(c->done);
     if (c->copy) cudaStreamDestroy(c->copy);
     if (c->ring) cudaFree(c->ring);
+    if (c->resident) cudaFree(c->resident);
     delete c;
 }
 
@@ -72,29 +96,52 @@ extern "C" {
 
 KQ_API const char* kq_chain_last_error(void) { return g_chain_err; }
 
-KQ_API int kq_chain_create(const kq_matrix_desc* mats, int n_layers, int mats_per_layer, int n_slots,
-                           kq_chain** out) {
+KQ_API int kq_chain_plan(const kq_matrix_desc* mats, int n_layers, int mats_per_layer, size_t budget_bytes,
+                         int max_slots, int* n_resident, int* n_slots) {
+    g_chain_err[0] = 0;
+    if (!mats || !n_resident || !n_slots || n_layers < 1 || mats_per_layer < 1 || max_slots < 1)
+        return chain_fail(KQ_ERR_INVALID_ARG, "bad arguments");
+    const size_t lb = layer_layout(mats, mats_per_layer, nullptr);
+    if (lb == 0) return chain_fail(KQ_ERR_INVALID_ARG, "bad matrix shape or format");
+    if (static_cast<size_t>(n_layers) * lb <= budget_bytes) {  // everything stays resident
+        *n_resident = n_layers;
+        *n_slots = 0;
+        return KQ_OK;
+    }
+    if (budget_bytes < lb) return chain_fail(KQ_ERR_OOM, "the budget does not hold one layer");
+    size_t slots = static_cast<size_t>(max_slots < n_layers ? max_slots : n_layers);
+    while (slots > 1 && slots * lb > budget_bytes) --slots;
+    size_t res = (budget_bytes - slots * lb) / lb;
+    if (res > static_cast<size_t>(n_layers) - slots) res = static_cast<size_t>(n_layers) - slots;
+    *n_resident = static_cast<int>(res);
+    *n_slots = static_cast<int>(slots);
+    return KQ_OK;
+}
+
+KQ_API int kq_chain_create_resident(const kq_matrix_desc* mats, int n_layers, int mats_per_layer, int n_resident,
+                                    int n_slots, kq_chain** out) {
     g_chain_err[0] = 0;
     if (!out) return chain_fail(KQ_ERR_INVALID_ARG, "out is NULL");
     *out = nullptr;
-    if (!mats || n_layers < 1 || mats_per_layer < 1 || n_slots < 1)
-        return chain_fail(KQ_ERR_INVALID_ARG, "bad layer / slot counts");
+    if (!mats || n_layers < 1 || mats_per_layer < 1 || n_resident < 0 || n_resident > n_layers || n_slots < 0 ||
+        (n_resident < n_layers && n_slots < 1))
+        return chain_fail(KQ_ERR_INVALID_ARG, "bad layer / resident / slot counts");
     kq_chain* c = new (std::nothrow) kq_chain();
     if (!c) return chain_fail(KQ_ERR_OOM, "host allocation");
     c->n_layers = n_layers;
     c->per_layer = mats_per_layer;
-    c->n_slots = n_slots < n_layers ? n_slots : n_layers;
+    c->n_resident = n_resident;
+    const int streamed = n_layers - n_resident;
+    c->n_slots = streamed == 0 ? 0 : (n_slots < streamed ? n_slots : streamed);
     c->mats.assign(mats, mats + static_cast<size_t>(n_layers) * mats_per_layer);
     c->offsets.resize(mats_per_layer);
     // slot layout: the matrices of a layer one after another, 256-byte
     // aligned; every layer must have the same matrix shapes
-    size_t off = 0;
-    for (int m = 0; m < mats_per_layer; ++m) {
-        const kq_matrix_desc& d = c->mats[m];
-        c->offsets[m] = off;
-        off = round_up(off + static_cast<size_t>(d.N) * kq_row_bytes(d.fmt, d.K), 256);
+    c->slot_bytes = layer_layout(c->mats.data(), mats_per_layer, &c->offsets);
+    if (c->slot_bytes == 0) {
+        destroy(c);
+        return chain_fail(KQ_ERR_INVALID_ARG, "layers must share matrix formats and shapes");
     }
-    c->slot_bytes = off;
     for (int l = 0; l < n_layers; ++l)
         for (int m = 0; m < mats_per_layer; ++m) {
             const kq_matrix_desc& d = c->mats[static_cast<size_t>(l) * mats_per_layer + m];
@@ -116,11 +163,12 @@ KQ_API int kq_chain_create(const kq_matrix_desc* mats, int n_layers, int mats_pe
             }
         }
     cudaError_t err = cudaGetDevice(&c->device);
-    if (err == cudaSuccess) err = cudaMalloc(&c->ring, c->slot_bytes * c->n_slots);
+    if (err == cudaSuccess && c->n_slots > 0) err = cudaMalloc(&c->ring, c->slot_bytes * c->n_slots);
+    if (err == cudaSuccess && n_resident > 0) err = cudaMalloc(&c->resident, c->slot_bytes * n_resident);
     if (err != cudaSuccess) {
         cudaGetLastError();
         destroy(c);
-        return chain_fail(KQ_ERR_OOM, "device ring allocation", err);
+        return chain_fail(KQ_ERR_OOM, "device slot / resident allocation", err);
     }
     err = cudaStreamCreateWithFlags(&c->copy, cudaStreamNonBlocking);
     c->ready.resize(c->n_slots, nullptr);
@@ -134,11 +182,36 @@ KQ_API int kq_chain_create(const kq_matrix_desc* mats, int n_layers, int mats_pe
         destroy(c);
         return chain_fail(KQ_ERR_CUDA, "stream/event creation", err);
     }
+    // the resident layers, copied once
+    for (int l = 0; l < n_resident && err == cudaSuccess; ++l)
+        for (int m = 0; m < mats_per_layer && err == cudaSuccess; ++m) {
+            const kq_matrix_desc& d = c->mats[static_cast<size_t>(l) * mats_per_layer + m];
+            err = cudaMemcpyAsync(c->resident + static_cast<size_t>(l) * c->slot_bytes + c->offsets[m], d.W,
+                                  static_cast<size_t>(d.N) * kq_row_bytes(d.fmt, d.K), cudaMemcpyHostToDevice,
+                                  c->copy);
+        }
+    if (err == cudaSuccess) err = cudaStreamSynchronize(c->copy);
+    if (err != cudaSuccess) {
+        destroy(c);
+        return chain_fail(KQ_ERR_CUDA, "resident layer copy", err);
+    }
     const char* f = getenv("KQ_FAULT");
     if (f && strncmp(f, "copy@", 5) == 0) c->fault_layer = atoi(f + 5);
     *out = c;
     return KQ_OK;
 }
+
+KQ_API int kq_chain_create(const kq_matrix_desc* mats, int n_layers, int mats_per_layer, int n_slots,
+                           kq_chain** out) {
+    if (n_slots < 1) {
+        g_chain_err[0] = 0;
+        if (out) *out = nullptr;
+        return chain_fail(KQ_ERR_INVALID_ARG, "bad layer / slot counts");
+    }
+    return kq_chain_create_resident(mats, n_layers, mats_per_layer, 0, n_slots, out);
+}
+
+KQ_API int kq_chain_resident_layers(const kq_chain* c) { return c ? c->n_resident : 0; }
 
 KQ_API size_t kq_chain_slot_bytes(const kq_chain* c) { return c ? c->slot_bytes : 0; }
 
@@ -151,7 +224,18 @@ KQ_API int kq_chain_run(kq_chain* c, const float* const* x, float* const* y, kq_
     if (err == cudaSuccess) err = cudaStreamWaitEvent(c->copy, c->done, 0);
     if (err != cudaSuccess) return chain_fail(KQ_ERR_CUDA, "stream ordering", err);
     for (int l = 0; l < c->n_layers; ++l) {
-        const int s = l % c->n_slots;
+        if (l < c->n_resident) {  // a resident layer: its GEMVs only
+            const uint8_t* base = c->resident + static_cast<size_t>(l) * c->slot_bytes;
+            for (int m = 0; m < c->per_layer; ++m) {
+                const size_t i = static_cast<size_t>(l) * c->per_layer + m;
+                const kq_matrix_desc& d = c->mats[i];
+                int st = kq_gemv(base + c->offsets[m], d.fmt, d.N, d.K, x[i], y[i], compute);
+                if (st != KQ_OK) return chain_fail(st, kq_last_error());
+            }
+            continue;
+        }
+        const int j = l - c->n_resident;  // streamed layer number
+        const int s = j % c->n_slots;
         uint8_t* slot = c->ring + static_cast<size_t>(s) * c->slot_bytes;
         if (l == c->fault_layer) {
             // injected failure: stop issuing; what is queued drains normally
@@ -159,7 +243,7 @@ KQ_API int kq_chain_run(kq_chain* c, const float* const* x, float* const* y, kq_
             cudaEventRecord(c->done, cs);
             return chain_fail(KQ_ERR_INJECTED, "KQ_FAULT: copy of the requested layer refused");
         }
-        if (l >= c->n_slots) {
+        if (j >= c->n_slots) {
             err = cudaStreamWaitEvent(c->copy, c->freed[s], 0);
             if (err != cudaSuccess) return chain_fail(KQ_ERR_CUDA, "wait slot free", err);
         }

@@ -264,6 +264,14 @@ def _chain_sigs(L):
     L.kq_chain_create.restype = ctypes.c_int
     L.kq_chain_create.argtypes = [ctypes.POINTER(MatrixDesc), ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.POINTER(vp)]
+    L.kq_chain_create_resident.restype = ctypes.c_int
+    L.kq_chain_create_resident.argtypes = [ctypes.POINTER(MatrixDesc), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int, ctypes.POINTER(vp)]
+    L.kq_chain_plan.restype = ctypes.c_int
+    L.kq_chain_plan.argtypes = [ctypes.POINTER(MatrixDesc), ctypes.c_int, ctypes.c_int, ctypes.c_size_t,
+                                ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    L.kq_chain_resident_layers.restype = ctypes.c_int
+    L.kq_chain_resident_layers.argtypes = [vp]
     L.kq_chain_slot_bytes.restype = ctypes.c_size_t
     L.kq_chain_slot_bytes.argtypes = [vp]
     L.kq_chain_run.restype = ctypes.c_int
@@ -276,14 +284,32 @@ def _chain_sigs(L):
     L._chain_ready = True
 
 
+def chain_plan(layers, budget_bytes: int, max_slots: int = 4):
+    """kq_chain_plan: (n_resident, n_slots) for a device-memory budget.
+    layers: list over layers of lists of (W, fmt, N, K) (W unused here)."""
+    L = lib()
+    _chain_sigs(L)
+    flat = [m for layer in layers for m in layer]
+    arr = (MatrixDesc * len(flat))()
+    for i, (W, fmt, N, K) in enumerate(flat):
+        arr[i] = MatrixDesc(None if W is None else W.data_ptr(), _fmt(fmt), N, K)
+    r, s = ctypes.c_int(), ctypes.c_int()
+    st = L.kq_chain_plan(arr, len(layers), len(layers[0]), budget_bytes, max_slots, ctypes.byref(r), ctypes.byref(s))
+    if st != OK:
+        raise KQError(st, "kq_chain_plan", L.kq_chain_last_error().decode())
+    return int(r.value), int(s.value)
+
+
 class Chain:
     """Layer chain whose weights stay in pinned host memory and stream
     through ``n_slots`` device slots (kq_chain_* in kq.h).
 
     mats: list over layers of lists of (W_host_pinned_uint8_tensor, fmt, N, K).
+    n_resident: leading layers copied once into device memory of their own
+    (kq_chain_create_resident); the rest stream.
     """
 
-    def __init__(self, mats, n_slots: int = 4):
+    def __init__(self, mats, n_slots: int = 4, n_resident: int = 0):
         L = lib()
         _chain_sigs(L)
         self._L = L
@@ -297,14 +323,18 @@ class Chain:
                 raise ValueError("chain weights must be host memory")
             arr[i] = MatrixDesc(W.data_ptr(), _fmt(fmt), N, K)
         h = ctypes.c_void_p()
-        st = L.kq_chain_create(arr, self.n_layers, self.per_layer, n_slots, ctypes.byref(h))
+        st = L.kq_chain_create_resident(arr, self.n_layers, self.per_layer, n_resident, n_slots, ctypes.byref(h))
         if st != OK:
-            raise KQError(st, "kq_chain_create", L.kq_chain_last_error().decode())
+            raise KQError(st, "kq_chain_create_resident", L.kq_chain_last_error().decode())
         self._h = h
 
     @property
     def slot_bytes(self) -> int:
         return int(self._L.kq_chain_slot_bytes(self._h))
+
+    @property
+    def resident_layers(self) -> int:
+        return int(self._L.kq_chain_resident_layers(self._h))
 
     def run(self, xs, ys, stream=None) -> None:
         n = self.n_layers * self.per_layer

@@ -327,6 +327,29 @@ typedef struct kq_chain kq_chain;
 KQ_API int kq_chain_create(const kq_matrix_desc* mats, int n_layers, int mats_per_layer, int n_slots,
                            kq_chain** out);
 
+/* Residency for a device-memory budget ("Kortex: Streaming 70B Models on
+ * Consumer GPUs", Key components: layers that fit stay in VRAM, the rest
+ * stream): *n_resident leading layers stay resident next to a ring of
+ * *n_slots slots (1 <= *n_slots <= max_slots), together within
+ * budget_bytes of device memory (layer bytes as kq_chain_slot_bytes counts
+ * them; activations and outputs are not counted).  Every layer fits:
+ * *n_resident = n_layers, *n_slots = 0.  Host arithmetic only.
+ * Errors: KQ_ERR_INVALID_ARG, KQ_ERR_OOM (the budget does not hold one
+ * layer). */
+KQ_API int kq_chain_plan(const kq_matrix_desc* mats, int n_layers, int mats_per_layer, size_t budget_bytes,
+                         int max_slots, int* n_resident, int* n_slots);
+
+/* kq_chain_create with the first n_resident layers (0..n_layers) copied
+ * once, during this call, into device memory of their own; a run launches
+ * their GEMVs directly and streams only the other layers, through n_slots
+ * slots (>= 1 unless every layer is resident).  Outputs equal a resident
+ * run bitwise.  Errors as kq_chain_create. */
+KQ_API int kq_chain_create_resident(const kq_matrix_desc* mats, int n_layers, int mats_per_layer, int n_resident,
+                                    int n_slots, kq_chain** out);
+
+/* Resident leading layers of a chain. */
+KQ_API int kq_chain_resident_layers(const kq_chain* c);
+
 /* Device bytes of one slot (one layer's matrices, 256-byte aligned each). */
 KQ_API size_t kq_chain_slot_bytes(const kq_chain* c);
 

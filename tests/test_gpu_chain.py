@@ -105,3 +105,30 @@ def test_wait_timeout_is_reported_then_completes():
     ch.wait(60000)
     ch.close()
     assert finished_early in (True, False)
+
+
+@pytest.mark.parametrize("n_resident,n_slots", [(2, 1), (5, 2), (7, 1), (0, 3)])
+def test_resident_prefix_then_stream_equals_resident_bitwise(n_resident, n_slots):
+    """The first n_resident layers stay in device memory, the rest stream
+    ("Kortex: Streaming 70B Models on Consumer GPUs", Key components): the
+    outputs equal resident kq_gemv calls bit for bit, on two runs."""
+    layers, xs = make_layers(7, seed=11)
+    flat = [m for layer in layers for m in layer]
+    ch = kq.Chain(layers, n_slots=n_slots, n_resident=n_resident)
+    assert ch.resident_layers == n_resident
+    for _ in range(2):
+        ys = [torch.full((N,), float("nan"), device="cuda") for (_, _, N, _) in flat]
+        ch.run(xs, ys)
+        ch.wait(60000)
+        for i, (W, fmt, N, K) in enumerate(flat):
+            assert torch.equal(ys[i], kq.gemv(W.cuda(), fmt, N, K, xs[i])), i
+
+
+def test_resident_counts_are_checked():
+    layers, _ = make_layers(3, seed=12)
+    with pytest.raises(kq.KQError):
+        kq.Chain(layers, n_slots=0, n_resident=1)      # streamed layers need a slot
+    with pytest.raises(kq.KQError):
+        kq.Chain(layers, n_slots=1, n_resident=4)      # more than the layers
+    ch = kq.Chain(layers, n_slots=0, n_resident=3)     # everything resident: no ring
+    assert ch.resident_layers == 3
