@@ -4,7 +4,7 @@ arithmetic).
 
 The C source ``kqgen.c`` draws logical values with a counter-based
 SplitMix64 stream and encodes them into the GGUF K-quant super-block layout
-(Q4_K: 144 bytes, Q5_K: 176 bytes, Q6_K: 210 bytes, 256 weights each).  This wrapper builds it
+(Q2_K: 84 bytes, Q3_K: 110, Q4_K: 144, Q5_K: 176, Q6_K: 210; 256 weights each).  This wrapper builds it
 with gcc on first use and returns numpy arrays.
 """
 from __future__ import annotations
@@ -22,6 +22,8 @@ _lib = None
 
 Q4_K_BLOCK_BYTES = 144
 Q5_K_BLOCK_BYTES = 176
+Q2_K_BLOCK_BYTES = 84
+Q3_K_BLOCK_BYTES = 110
 Q6_K_BLOCK_BYTES = 210
 QK = 256  # weights per super-block
 
@@ -53,6 +55,12 @@ def _load():
         lib.kqg_q5k_draw.argtypes = [u64, i64, vp, vp, vp, vp, vp]
         lib.kqg_q5k_pack.argtypes = [i64, vp, vp, vp, vp, vp, vp]
         lib.kqg_q5k_fill.argtypes = [u64, i64, i64, vp, i32]
+        lib.kqg_q2k_draw.argtypes = [u64, i64, vp, vp, vp, vp, vp]
+        lib.kqg_q2k_pack.argtypes = [i64, vp, vp, vp, vp, vp, vp]
+        lib.kqg_q2k_fill.argtypes = [u64, i64, i64, vp, i32]
+        lib.kqg_q3k_draw.argtypes = [u64, i64, vp, vp, vp]
+        lib.kqg_q3k_pack.argtypes = [i64, vp, vp, vp, vp]
+        lib.kqg_q3k_fill.argtypes = [u64, i64, i64, vp, i32]
         lib.kqg_q6k_draw.argtypes = [u64, i64, vp, vp, vp]
         lib.kqg_q6k_pack.argtypes = [i64, vp, vp, vp, vp]
         lib.kqg_q6k_fill.argtypes = [u64, i64, i64, vp, i32]
@@ -88,7 +96,8 @@ def f16_bits(v: float) -> int:
 
 
 def block_bytes(fmt: str) -> int:
-    return {"q4_k": Q4_K_BLOCK_BYTES, "q5_k": Q5_K_BLOCK_BYTES, "q6_k": Q6_K_BLOCK_BYTES}[fmt]
+    return {"q4_k": Q4_K_BLOCK_BYTES, "q5_k": Q5_K_BLOCK_BYTES, "q6_k": Q6_K_BLOCK_BYTES, "q2_k": Q2_K_BLOCK_BYTES,
+            "q3_k": Q3_K_BLOCK_BYTES}[fmt]
 
 
 def row_bytes(fmt: str, K: int) -> int:
@@ -168,6 +177,70 @@ def q5k_fill(key: int, nblocks: int, out: np.ndarray | None = None, b0: int = 0,
     return out
 
 
+# ----------------------------------------------------------------- Q2_K
+def q2k_draw(key: int, nblocks: int) -> dict:
+    """Logical values of Q2_K super-blocks: q (nb,256) u8 in 0..3, sc/m
+    (nb,16) u8 in 0..15, d/dmin (nb,) fp16 bit patterns."""
+    q = np.empty((nblocks, 256), np.uint8)
+    sc = np.empty((nblocks, 16), np.uint8)
+    m = np.empty((nblocks, 16), np.uint8)
+    d = np.empty(nblocks, np.uint16)
+    dmin = np.empty(nblocks, np.uint16)
+    _load().kqg_q2k_draw(key, nblocks, _ptr(q), _ptr(sc), _ptr(m), _ptr(d), _ptr(dmin))
+    return dict(q=q, sc=sc, m=m, d=d, dmin=dmin)
+
+
+def q2k_pack(q, sc, m, d, dmin) -> np.ndarray:
+    q = np.ascontiguousarray(q, np.uint8).reshape(-1, 256)
+    nb = q.shape[0]
+    sc = np.ascontiguousarray(sc, np.uint8).reshape(nb, 16)
+    m = np.ascontiguousarray(m, np.uint8).reshape(nb, 16)
+    d = np.ascontiguousarray(d, np.uint16).reshape(nb)
+    dmin = np.ascontiguousarray(dmin, np.uint16).reshape(nb)
+    out = np.empty(nb * Q2_K_BLOCK_BYTES, np.uint8)
+    _load().kqg_q2k_pack(nb, _ptr(q), _ptr(sc), _ptr(m), _ptr(d), _ptr(dmin), _ptr(out))
+    return out
+
+
+def q2k_fill(key: int, nblocks: int, out: np.ndarray | None = None, b0: int = 0,
+             nthreads: int | None = None) -> np.ndarray:
+    if out is None:
+        out = np.empty(nblocks * Q2_K_BLOCK_BYTES, np.uint8)
+    assert out.nbytes >= nblocks * Q2_K_BLOCK_BYTES and out.dtype == np.uint8
+    _load().kqg_q2k_fill(key, b0, nblocks, _ptr(out), nthreads or default_threads())
+    return out
+
+
+# ----------------------------------------------------------------- Q3_K
+def q3k_draw(key: int, nblocks: int) -> dict:
+    """Logical values of Q3_K super-blocks: q (nb,256) int8 in -4..3, v
+    (nb,16) u8 6-bit scales (used as v - 32), d (nb,) fp16 bit patterns."""
+    q = np.empty((nblocks, 256), np.int8)
+    v = np.empty((nblocks, 16), np.uint8)
+    d = np.empty(nblocks, np.uint16)
+    _load().kqg_q3k_draw(key, nblocks, _ptr(q), _ptr(v), _ptr(d))
+    return dict(q=q, v=v, d=d)
+
+
+def q3k_pack(q, v, d) -> np.ndarray:
+    q = np.ascontiguousarray(q, np.int8).reshape(-1, 256)
+    nb = q.shape[0]
+    v = np.ascontiguousarray(v, np.uint8).reshape(nb, 16)
+    d = np.ascontiguousarray(d, np.uint16).reshape(nb)
+    out = np.empty(nb * Q3_K_BLOCK_BYTES, np.uint8)
+    _load().kqg_q3k_pack(nb, _ptr(q), _ptr(v), _ptr(d), _ptr(out))
+    return out
+
+
+def q3k_fill(key: int, nblocks: int, out: np.ndarray | None = None, b0: int = 0,
+             nthreads: int | None = None) -> np.ndarray:
+    if out is None:
+        out = np.empty(nblocks * Q3_K_BLOCK_BYTES, np.uint8)
+    assert out.nbytes >= nblocks * Q3_K_BLOCK_BYTES and out.dtype == np.uint8
+    _load().kqg_q3k_fill(key, b0, nblocks, _ptr(out), nthreads or default_threads())
+    return out
+
+
 # ----------------------------------------------------------------- Q6_K
 def q6k_draw(key: int, nblocks: int) -> dict:
     """Logical values of Q6_K super-blocks: q (nb,256) u8 in 0..63,
@@ -204,6 +277,10 @@ def fill(fmt: str, key: int, nblocks: int, out: np.ndarray | None = None,
         return q4k_fill(key, nblocks, out, nthreads=nthreads)
     if fmt == "q5_k":
         return q5k_fill(key, nblocks, out, nthreads=nthreads)
+    if fmt == "q2_k":
+        return q2k_fill(key, nblocks, out, nthreads=nthreads)
+    if fmt == "q3_k":
+        return q3k_fill(key, nblocks, out, nthreads=nthreads)
     if fmt == "q6_k":
         return q6k_fill(key, nblocks, out, nthreads=nthreads)
     raise ValueError(fmt)

@@ -36,6 +36,21 @@
  *     low 4 bits in the high nibble of the same byte and its 5th bit in bit
  *     2c+1 of qh[l].  The fill draws quants uniform over 0..31, the rest as
  *     Q4_K.
+ *   Q2_K, 84 B: [0,16) scale bytes | [16,80) 64 quant bytes | [80,82) d fp16 |
+ *                [82,84) dmin fp16.
+ *     Scale byte j (j<16, the 16-weight sub-block j): low nibble scale,
+ *     high nibble min.  Weight 128n+32j+l (n<2, j<4, l<32) is bits 2j..2j+1
+ *     of quant byte 32n+l.  The fill draws quants uniform over 0..3, scales
+ *     and mins over 0..15, d and dmin as Q4_K.
+ *   Q3_K, 110 B: [0,32) hmask | [32,96) 64 quant bytes | [96,108) 12 scale
+ *                bytes | [108,110) d fp16.
+ *     Weight 128n+32j+l has its low 2 bits at bits 2j..2j+1 of quant byte
+ *     32n+l and its third bit at bit 4n+j of hmask[l]; its value is
+ *     (low | third << 2) - 4, in -4..3.  Sub-block j (16 weights) has a
+ *     6-bit scale v_j, used as v_j - 32: its low 4 bits are the low nibble
+ *     of scale byte j (j<8) or the high nibble of byte j-8 (j>=8), its top
+ *     2 bits are bits 2(j/4)..2(j/4)+1 of byte 8 + j%4.  The fill draws the
+ *     values uniform over -4..3, v_j over 0..63, d as Q4_K.
  *   Q6_K, 210 B: [0,128) ql | [128,192) qh | [192,208) int8 scales |
  *                [208,210) d fp16.
  *     Half h (0..1) covers weights 128h..128h+127.  For l<32 and t<4, weight
@@ -233,6 +248,125 @@ void kqg_q5k_fill(uint64_t key, int64_t b0, int64_t nblocks, uint8_t* out, int n
         uint16_t d, dmin;
         kqg_q5k_draw_block(key, (uint64_t)(b0 + b), q, sc, m, &d, &dmin);
         kqg_q5k_pack_block(q, sc, m, d, dmin, out + 176 * b);
+    }
+}
+
+/* ---------------------------------------------------------------- Q2_K */
+
+static void kqg_q2k_draw_block(uint64_t key, uint64_t b, uint8_t q[256], uint8_t sc[16], uint8_t m[16],
+                               uint16_t* d, uint16_t* dmin) {
+    const uint64_t base = b * 32;
+    for (int k = 0; k < 8; ++k) {
+        uint64_t r = kqg_draw(key, base + k);
+        for (int i = 0; i < 32; ++i) q[32 * k + i] = (uint8_t)((r >> (2 * i)) & 3);
+    }
+    uint64_t r = kqg_draw(key, base + 8);
+    for (int j = 0; j < 16; ++j) {
+        sc[j] = (uint8_t)((r >> (4 * j)) & 15);
+    }
+    r = kqg_draw(key, base + 9);
+    for (int j = 0; j < 16; ++j) m[j] = (uint8_t)((r >> (4 * j)) & 15);
+    double z0, z1;
+    kqg_box_muller(key, base + 10, &z0, &z1);
+    *d = kqg_f16_bits(fabs(z0) * 1e-3);
+    *dmin = kqg_f16_bits(fabs(z1) * 1e-3);
+}
+
+static void kqg_q2k_pack_block(const uint8_t q[256], const uint8_t sc[16], const uint8_t m[16], uint16_t d,
+                               uint16_t dmin, uint8_t* out) {
+    for (int j = 0; j < 16; ++j) out[j] = (uint8_t)((sc[j] & 15) | ((m[j] & 15) << 4));
+    uint8_t* qs = out + 16;
+    memset(qs, 0, 64);
+    for (int n = 0; n < 2; ++n)
+        for (int j = 0; j < 4; ++j)
+            for (int l = 0; l < 32; ++l) qs[32 * n + l] |= (uint8_t)((q[128 * n + 32 * j + l] & 3) << (2 * j));
+    out[80] = (uint8_t)(d & 0xFF);
+    out[81] = (uint8_t)(d >> 8);
+    out[82] = (uint8_t)(dmin & 0xFF);
+    out[83] = (uint8_t)(dmin >> 8);
+}
+
+void kqg_q2k_draw(uint64_t key, int64_t nblocks, uint8_t* q, uint8_t* sc, uint8_t* m, uint16_t* d,
+                  uint16_t* dmin) {
+    for (int64_t b = 0; b < nblocks; ++b)
+        kqg_q2k_draw_block(key, (uint64_t)b, q + 256 * b, sc + 16 * b, m + 16 * b, d + b, dmin + b);
+}
+
+void kqg_q2k_pack(int64_t nblocks, const uint8_t* q, const uint8_t* sc, const uint8_t* m, const uint16_t* d,
+                  const uint16_t* dmin, uint8_t* out) {
+    for (int64_t b = 0; b < nblocks; ++b)
+        kqg_q2k_pack_block(q + 256 * b, sc + 16 * b, m + 16 * b, d[b], dmin[b], out + 84 * b);
+}
+
+void kqg_q2k_fill(uint64_t key, int64_t b0, int64_t nblocks, uint8_t* out, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int64_t b = 0; b < nblocks; ++b) {
+        uint8_t q[256], sc[16], m[16];
+        uint16_t d, dmin;
+        kqg_q2k_draw_block(key, (uint64_t)(b0 + b), q, sc, m, &d, &dmin);
+        kqg_q2k_pack_block(q, sc, m, d, dmin, out + 84 * b);
+    }
+}
+
+/* ---------------------------------------------------------------- Q3_K */
+
+/* q: the signed values -4..3; v: the 6-bit scales 0..63 (used as v - 32). */
+static void kqg_q3k_draw_block(uint64_t key, uint64_t b, int8_t q[256], uint8_t v[16], uint16_t* d) {
+    const uint64_t base = b * 32;
+    for (int i = 0; i < 256; ++i) {
+        uint64_t r = kqg_draw(key, base + (uint64_t)(i / 21));
+        q[i] = (int8_t)((int)((r >> (3 * (i % 21))) & 7) - 4);
+    }
+    uint64_t r0 = kqg_draw(key, base + 13), r1 = kqg_draw(key, base + 14);
+    for (int j = 0; j < 16; ++j) {
+        uint64_t r = j < 10 ? r0 : r1;
+        v[j] = (uint8_t)((r >> (6 * (j < 10 ? j : j - 10))) & 63);
+    }
+    double z0, z1;
+    kqg_box_muller(key, base + 15, &z0, &z1);
+    *d = kqg_f16_bits(fabs(z0) * 1e-3);
+}
+
+static void kqg_q3k_pack_block(const int8_t q[256], const uint8_t v[16], uint16_t d, uint8_t* out) {
+    uint8_t* hm = out;
+    uint8_t* qs = out + 32;
+    uint8_t* sb = out + 96;
+    memset(out, 0, 108);
+    for (int n = 0; n < 2; ++n)
+        for (int j = 0; j < 4; ++j)
+            for (int l = 0; l < 32; ++l) {
+                const int u = q[128 * n + 32 * j + l] + 4;  /* 0..7 */
+                qs[32 * n + l] |= (uint8_t)((u & 3) << (2 * j));
+                hm[l] |= (uint8_t)(((u >> 2) & 1) << (4 * n + j));
+            }
+    for (int j = 0; j < 16; ++j) {
+        const int lo = v[j] & 15, hi = (v[j] >> 4) & 3;
+        if (j < 8) sb[j] |= (uint8_t)lo;
+        else sb[j - 8] |= (uint8_t)(lo << 4);
+        sb[8 + (j % 4)] |= (uint8_t)(hi << (2 * (j / 4)));
+    }
+    out[108] = (uint8_t)(d & 0xFF);
+    out[109] = (uint8_t)(d >> 8);
+}
+
+void kqg_q3k_draw(uint64_t key, int64_t nblocks, int8_t* q, uint8_t* v, uint16_t* d) {
+    for (int64_t b = 0; b < nblocks; ++b) kqg_q3k_draw_block(key, (uint64_t)b, q + 256 * b, v + 16 * b, d + b);
+}
+
+void kqg_q3k_pack(int64_t nblocks, const int8_t* q, const uint8_t* v, const uint16_t* d, uint8_t* out) {
+    for (int64_t b = 0; b < nblocks; ++b) kqg_q3k_pack_block(q + 256 * b, v + 16 * b, d[b], out + 110 * b);
+}
+
+void kqg_q3k_fill(uint64_t key, int64_t b0, int64_t nblocks, uint8_t* out, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int64_t b = 0; b < nblocks; ++b) {
+        int8_t q[256];
+        uint8_t v[16];
+        uint16_t d;
+        kqg_q3k_draw_block(key, (uint64_t)(b0 + b), q, v, &d);
+        kqg_q3k_pack_block(q, v, d, out + 110 * b);
     }
 }
 

@@ -24,6 +24,10 @@
  *     w = d*sc_j*q - dmin*m_j as Q4_K, with q a 5-bit quant (0..31).
  *   Q6_K (210 B, 256 weights = 16 groups of 16):
  *     w = d*s_g*(q - 32) for weight in group g, s_g a signed byte.
+ *   Q2_K (84 B, 16 groups of 16): w = d*sc_g*q - dmin*m_g, q in 0..3,
+ *     sc_g and m_g 4-bit.
+ *   Q3_K (110 B, 16 groups of 16): w = d*(v_g - 32)*q, q in -4..3, v_g a
+ *     6-bit scale.
  *
  * Every step is a literal loop; no blocking, fusion or reordering.
  */
@@ -32,7 +36,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { KQO_Q4_K = 1, KQO_Q6_K = 2, KQO_Q5_K = 3 };
+enum { KQO_Q4_K = 1, KQO_Q6_K = 2, KQO_Q5_K = 3, KQO_Q2_K = 4, KQO_Q3_K = 5 };
 
 /* IEEE binary16 -> double (exact), including subnormals, inf and NaN. */
 double kqo_f16(uint16_t h) {
@@ -113,6 +117,48 @@ void kqo_q5k_unpack(const uint8_t* blk, uint8_t q[256], uint8_t sc[8], uint8_t m
     }
 }
 
+/* Q2_K super-block -> logical fields.
+ * Bytes 0..15: one byte per 16-weight group g, scale in the low nibble, min
+ * in the high nibble.  Bytes 16..79: quants; weight 128n + 32j + l (n < 2,
+ * j < 4, l < 32) is bits 2j..2j+1 of byte 16 + 32n + l.  Then d, dmin. */
+void kqo_q2k_unpack(const uint8_t* blk, uint8_t q[256], uint8_t sc[16], uint8_t m[16], double* d, double* dmin) {
+    for (int g = 0; g < 16; ++g) {
+        sc[g] = blk[g] & 15;
+        m[g] = blk[g] >> 4;
+    }
+    for (int i = 0; i < 256; ++i) {
+        int n = i / 128, j = (i % 128) / 32, l = i % 32;
+        q[i] = (uint8_t)((blk[16 + 32 * n + l] >> (2 * j)) & 3);
+    }
+    *d = kqo_f16(rd16(blk + 80));
+    *dmin = kqo_f16(rd16(blk + 82));
+}
+
+/* Q3_K super-block -> logical fields.
+ * Bytes 0..31 hmask, 32..95 quants, 96..107 scales, then d.  Weight
+ * 128n + 32j + l: low 2 bits = bits 2j..2j+1 of byte 32 + 32n + l; third bit
+ * = bit 4n + j of hmask[l]; value = (low | third << 2) - 4.  Group g's 6-bit
+ * scale: low 4 bits from the low nibble of scale byte g (g < 8) or the high
+ * nibble of byte g - 8 (g >= 8); top 2 bits from bits 2(g/4)..2(g/4)+1 of
+ * scale byte 8 + g%4.  The group multiplies by (v - 32). */
+void kqo_q3k_unpack(const uint8_t* blk, int8_t q[256], uint8_t v[16], double* d) {
+    const uint8_t* hm = blk;
+    const uint8_t* qs = blk + 32;
+    const uint8_t* sb = blk + 96;
+    for (int i = 0; i < 256; ++i) {
+        int n = i / 128, j = (i % 128) / 32, l = i % 32;
+        int low = (qs[32 * n + l] >> (2 * j)) & 3;
+        int third = (hm[l] >> (4 * n + j)) & 1;
+        q[i] = (int8_t)((low | (third << 2)) - 4);
+    }
+    for (int g = 0; g < 16; ++g) {
+        int lo = g < 8 ? (sb[g] & 15) : (sb[g - 8] >> 4);
+        int hi = (sb[8 + g % 4] >> (2 * (g / 4))) & 3;
+        v[g] = (uint8_t)(lo | (hi << 4));
+    }
+    *d = kqo_f16(rd16(blk + 108));
+}
+
 /* Q6_K super-block -> logical fields.
  * Layout: ql[128] (low 4 bits), qh[64] (top 2 bits), 16 signed scales, d.
  * Weight i = 128h + 32t + l (h<2, t<4, l<32): low bits from
@@ -133,7 +179,8 @@ void kqo_q6k_unpack(const uint8_t* blk, uint8_t q[256], int8_t s[16], double* d)
 }
 
 static int64_t block_bytes(int fmt) {
-    return fmt == KQO_Q4_K ? 144 : fmt == KQO_Q6_K ? 210 : fmt == KQO_Q5_K ? 176 : -1;
+    return fmt == KQO_Q4_K ? 144 : fmt == KQO_Q6_K ? 210 : fmt == KQO_Q5_K ? 176 : fmt == KQO_Q2_K ? 84
+                                                                         : fmt == KQO_Q3_K ? 110 : -1;
 }
 
 /* Dequantise one row of K weights (K/256 consecutive super-blocks). */
@@ -152,6 +199,23 @@ int kqo_dequant_row(int fmt, const uint8_t* row, int64_t K, double* w) {
             for (int i = 0; i < 256; ++i) {
                 int j = i / 32;
                 wb[i] = d * sc[j] * q[i] - dmin * m[j];
+            }
+        } else if (fmt == KQO_Q2_K) {
+            uint8_t sc[16], m[16];
+            double d, dmin;
+            kqo_q2k_unpack(blk, q, sc, m, &d, &dmin);
+            for (int i = 0; i < 256; ++i) {
+                int g = i / 16;
+                wb[i] = d * sc[g] * q[i] - dmin * m[g];
+            }
+        } else if (fmt == KQO_Q3_K) {
+            int8_t qq[256];
+            uint8_t v[16];
+            double d;
+            kqo_q3k_unpack(blk, qq, v, &d);
+            for (int i = 0; i < 256; ++i) {
+                int g = i / 16;
+                wb[i] = d * ((int)v[g] - 32) * qq[i];
             }
         } else {
             int8_t s[16];
@@ -271,7 +335,12 @@ int kqo_gemv_x64(int fmt, const uint8_t* W, int64_t N, int64_t K, const double* 
  *                     before -32)
  *   sc[16*b + j]      Q4_K, Q5_K: sc_0..7 then m_0..7; Q6_K: the 16 signed
  *                     scales as two's-complement bytes
- *   d[2*b], d[2*b+1]  Q4_K, Q5_K: d, dmin; Q6_K: d, 0 (fp16 widened exactly) */
+ *                     Q2_K: the 16 raw scale bytes (scale | min << 4);
+ *                     Q3_K: the 16 6-bit scales v (before -32)
+ *                     (Q2_K quants 0..3; Q3_K values -4..3 as two's-complement
+ *                     bytes)
+ *   d[2*b], d[2*b+1]  Q4_K, Q5_K, Q2_K: d, dmin; Q6_K, Q3_K: d, 0 (fp16
+ *                     widened exactly) */
 int kqo_unpack(int fmt, const uint8_t* W, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d) {
     int64_t bb = block_bytes(fmt);
     if (bb < 0) return -1;
@@ -283,6 +352,18 @@ int kqo_unpack(int fmt, const uint8_t* W, int64_t nblocks, uint8_t* q, uint8_t* 
             else kqo_q5k_unpack(blk, q + 256 * b, sc + 16 * b, sc + 16 * b + 8, &dd, &dm);
             d[2 * b] = (float)dd;
             d[2 * b + 1] = (float)dm;
+        } else if (fmt == KQO_Q2_K) {
+            uint8_t s2[16], m2[16];
+            double dd, dm;
+            kqo_q2k_unpack(blk, q + 256 * b, s2, m2, &dd, &dm);
+            for (int g = 0; g < 16; ++g) sc[16 * b + g] = (uint8_t)(s2[g] | (m2[g] << 4));
+            d[2 * b] = (float)dd;
+            d[2 * b + 1] = (float)dm;
+        } else if (fmt == KQO_Q3_K) {
+            double dd;
+            kqo_q3k_unpack(blk, (int8_t*)(q + 256 * b), sc + 16 * b, &dd);
+            d[2 * b] = (float)dd;
+            d[2 * b + 1] = 0.0f;
         } else {
             double dd;
             kqo_q6k_unpack(blk, q + 256 * b, (int8_t*)(sc + 16 * b), &dd);

@@ -109,7 +109,67 @@ def test_q5k_hand_worked_block(golden_dir):
     assert y[0] == float(g["y_ones"][0])
 
 
+def test_q2k_hand_worked_block(golden_dir):
+    g = _read_golden(os.path.join(golden_dir, "q2k_block_worked.txt"))
+    scales = np.array([j | ((15 - j) << 4) for j in range(16)], np.uint8)
+    blk = np.concatenate([scales, np.arange(64, dtype=np.uint8), np.array([int(h, 16) for h in g["d"]], np.uint8),
+                          np.array([int(h, 16) for h in g["dmin"]], np.uint8)])
+    assert blk.size == 84
+    q, sc, d = oracle.unpack("q2_k", blk, 1)
+    assert (sc & 15).tolist() == list(range(16)) and (sc >> 4).tolist() == [15 - j for j in range(16)]
+    assert d.tolist() == [1.0, 0.5]
+    w = oracle.dequant("q2_k", blk, 1, 256)[0]
+    for i, qi, wi in g["w"]:
+        assert q[i] == qi, i
+        assert w[i] == wi, i
+    y, _ = oracle.gemv("q2_k", blk, 1, 256, np.ones(256, np.float32))
+    assert y[0] == float(g["y_ones"][0])
+
+
+def test_q3k_hand_worked_block(golden_dir):
+    g = _read_golden(os.path.join(golden_dir, "q3k_block_worked.txt"))
+    blk = np.concatenate([np.arange(32, dtype=np.uint8), np.arange(64, dtype=np.uint8),
+                          np.array([int(h, 16) for h in g["scales"]], np.uint8),
+                          np.array([int(h, 16) for h in g["d"]], np.uint8)])
+    assert blk.size == 110
+    q, sc, d = oracle.unpack("q3_k", blk, 1)
+    assert sc.tolist() == [int(v) for v in g["v"]]
+    assert d.tolist() == [1.0, 0.0]
+    w = oracle.dequant("q3_k", blk, 1, 256)[0]
+    qs = q.view(np.int8)
+    for i, qi, wi in g["w"]:
+        assert qs[i] == qi, i
+        assert w[i] == wi, i
+    y, _ = oracle.gemv("q3_k", blk, 1, 256, np.ones(256, np.float32))
+    assert y[0] == float(g["y_ones"][0])
+
+
 # ----------------------------------------------- exhaustive round trips
+def test_q2k_q3k_roundtrip_all_values_all_positions():
+    """Every quant value in every position and every scale (and Q2_K min)
+    value in every slot survive generator packing and oracle unpacking."""
+    nb = 64
+    b, i = np.meshgrid(np.arange(nb), np.arange(256), indexing="ij")
+    b16, j16 = np.meshgrid(np.arange(nb), np.arange(16), indexing="ij")
+    q2 = ((i * 5 + b) % 4).astype(np.uint8)
+    sc2 = ((b16 + 3 * j16) % 16).astype(np.uint8)
+    m2 = ((15 - b16 + j16) % 16).astype(np.uint8)
+    W2 = kqgen.q2k_pack(q2, sc2, m2, np.full(nb, 0x3C00, np.uint16), np.full(nb, 0x3800, np.uint16))
+    q, sc, d = oracle.unpack("q2_k", W2, nb)
+    assert np.array_equal(q.reshape(nb, 256), q2)
+    assert np.array_equal(sc.reshape(nb, 16) & 15, sc2) and np.array_equal(sc.reshape(nb, 16) >> 4, m2)
+    assert all(len(set(q2[:, k].tolist())) == 4 for k in range(256))
+    assert all(len(set(sc2[:, k].tolist())) == 16 and len(set(m2[:, k].tolist())) == 16 for k in range(16))
+    q3 = ((i * 3 + b) % 8 - 4).astype(np.int8)
+    v3 = ((b16 + 5 * j16) % 64).astype(np.uint8)
+    W3 = kqgen.q3k_pack(q3, v3, np.full(nb, 0x3C00, np.uint16))
+    q, sc, d = oracle.unpack("q3_k", W3, nb)
+    assert np.array_equal(q.view(np.int8).reshape(nb, 256), q3)
+    assert np.array_equal(sc.reshape(nb, 16), v3)
+    assert all(len(set(q3[:, k].tolist())) == 8 for k in range(256))
+    assert all(len(set(v3[:, k].tolist())) == 64 for k in range(16))
+
+
 def test_q5k_quant_and_scale_roundtrip_all_positions():
     """Every 5-bit value in every quant position, and every 6-bit value in
     every scale and min slot, survive generator packing and oracle unpacking."""
@@ -272,7 +332,7 @@ def test_q6k_mid_quants_give_exact_zero_and_zero_quants_closed_form():
 
 
 # -------------------------------------------------------------- invariants
-@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k", "q2_k", "q3_k"])
 def test_linearity_in_x(fmt):
     N, K = 8, 1024
     W = kqgen.matrix(fmt, 11, N, K)
@@ -286,7 +346,7 @@ def test_linearity_in_x(fmt):
     assert np.all(np.abs(yc - (2 * y1 - 3 * y2)) <= 1e-12 * (2 * s1 + 3 * s2))
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k", "q2_k", "q3_k"])
 def test_one_hot_extracts_column_and_ones_give_row_sums(fmt):
     N, K = 4, 512
     W = kqgen.matrix(fmt, 12, N, K)
@@ -301,7 +361,7 @@ def test_one_hot_extracts_column_and_ones_give_row_sums(fmt):
     assert np.allclose(s, np.abs(Wd).sum(axis=1), rtol=1e-13)
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k", "q2_k", "q3_k"])
 def test_brute_force_tiny_from_logical_values(fmt):
     """Dense W built from the generator's logical values (never its bytes)
     matches the oracle's byte path."""
@@ -315,6 +375,20 @@ def test_brute_force_tiny_from_logical_values(fmt):
         sc = np.repeat(lg["sc"].astype(np.float64), 32, axis=1)
         m = np.repeat(lg["m"].astype(np.float64), 32, axis=1)
         dense = (d * sc * lg["q"] - dm * m).reshape(N, K)
+    elif fmt == "q2_k":
+        lg = kqgen.q2k_draw(35, nb)
+        W = kqgen.q2k_pack(**lg)
+        d = lg["d"].view(np.float16).astype(np.float64)[:, None]
+        dm = lg["dmin"].view(np.float16).astype(np.float64)[:, None]
+        sc = np.repeat(lg["sc"].astype(np.float64), 16, axis=1)
+        m = np.repeat(lg["m"].astype(np.float64), 16, axis=1)
+        dense = (d * sc * lg["q"] - dm * m).reshape(N, K)
+    elif fmt == "q3_k":
+        lg = kqgen.q3k_draw(36, nb)
+        W = kqgen.q3k_pack(**lg)
+        d = lg["d"].view(np.float16).astype(np.float64)[:, None]
+        v = np.repeat(lg["v"].astype(np.float64) - 32, 16, axis=1)
+        dense = (d * v * lg["q"].astype(np.float64)).reshape(N, K)
     else:
         lg = kqgen.q6k_draw(32, nb)
         W = kqgen.q6k_pack(**lg)
