@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "K-quant dequant-GEMV weight GB/s (% of B200 HBM peak); layer-chain tok/s"
 QK = 256
-BLOCK = {"q4_k": 144, "q5_k": 176, "q6_k": 210}
+BLOCK = {"q4_k": 144, "q5_k": 176, "q6_k": 210, "q2_k": 84, "q3_k": 110}
 SEED = 0xC0FFEE + 1
 
 
@@ -50,14 +50,14 @@ def row_bytes(fmt, K):
     return K // QK * BLOCK[fmt]
 
 
-def dense_layer(hidden, heads, kv_heads, head_dim, ffn, fmt="q4_k"):
+def dense_layer(hidden, heads, kv_heads, head_dim, ffn, fmt="q4_k", down_fmt="q6_k"):
     """(name, fmt, N, K, x-slot): q|k|v share the attention input, gate|up
     share the FFN input; each is one launch over the stacked rows.  `fmt`
-    is the format of all but down, which stays Q6_K (as in Q4_K_M and Q5_K_M
-    files)."""
+    is the format of all but down, which is `down_fmt` (Q6_K in Q4_K_M and
+    Q5_K_M files)."""
     qkv = (heads + 2 * kv_heads) * head_dim
     return [("qkv", fmt, qkv, hidden, 0), ("o", fmt, hidden, heads * head_dim, 1),
-            ("gate_up", fmt, 2 * ffn, hidden, 2), ("down", "q6_k", hidden, ffn, 3)]
+            ("gate_up", fmt, 2 * ffn, hidden, 2), ("down", down_fmt, hidden, ffn, 3)]
 
 
 L8B = dict(hidden=4096, heads=32, kv_heads=8, head_dim=128, ffn=14336)
@@ -70,6 +70,10 @@ def chain_spec(kind):
         return [dense_layer(**L8B) for _ in range(32)]
     if kind == "llama8b_q5k":
         return [dense_layer(**L8B, fmt="q5_k") for _ in range(32)]
+    if kind == "llama8b_q2k":
+        return [dense_layer(**L8B, fmt="q2_k", down_fmt="q3_k") for _ in range(32)]
+    if kind == "llama8b_q3k":
+        return [dense_layer(**L8B, fmt="q3_k", down_fmt="q4_k") for _ in range(32)]
     if kind == "llama70b":
         return [dense_layer(**L70B) for _ in range(80)]
     if kind == "gemv_q4k_4096":
@@ -78,6 +82,12 @@ def chain_spec(kind):
         return [[("gate_up", "q4_k", 28672, 4096, 0)] for _ in range(8)]
     if kind == "gateup_q5k":
         return [[("gate_up", "q5_k", 28672, 4096, 0)] for _ in range(8)]
+    if kind == "gateup_q2k":
+        return [[("gate_up", "q2_k", 28672, 4096, 0)] for _ in range(8)]
+    if kind == "gateup_q3k":
+        return [[("gate_up", "q3_k", 28672, 4096, 0)] for _ in range(8)]
+    if kind == "down_q3k":
+        return [[("down", "q3_k", 4096, 14336, 0)] for _ in range(8)]
     if kind == "down_q6k":
         return [[("down", "q6_k", 4096, 14336, 0)] for _ in range(8)]
     raise KeyError(kind)
@@ -89,6 +99,13 @@ WORKLOADS = {
                          "(a Q5_K_M file's formats), 32 layers, batch 1",
     "verify8b_q5k_k8": "the Q5_K 8B-shaped chain, speculative-verify GEMV with k=8 activation columns",
     "gateup_q5k": "Q5_K GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
+    "llama8b_q2k_chain": "Llama-3.1-8B-shaped decode chain with Q2_K qkv, o and gate|up and Q3_K down, "
+                         "32 layers, batch 1",
+    "llama8b_q3k_chain": "Llama-3.1-8B-shaped decode chain with Q3_K qkv, o and gate|up and Q4_K down, "
+                         "32 layers, batch 1",
+    "gateup_q2k": "Q2_K GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
+    "gateup_q3k": "Q3_K GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
+    "down_q3k": "Q3_K GEMV 4096 x 14336 (8B down), 8 distinct copies rotated",
     "llama8b_chain_steps": "the same chain through kq_gemv_steps (16 matvecs per persistent launch, each "
                            "waiting for the one before)",
     "llama8b_layer_fused": "the 8B-shaped chain with RMSNorm fused into qkv and gate|up and the SiLU-gated "
@@ -449,7 +466,9 @@ def make_workload(name, torch, kq, kqgen, seed):
         return Resident(torch, kq, kqgen, chain_spec("llama8b_q5k"), seed)
     if name == "verify8b_q5k_k8":
         return Resident(torch, kq, kqgen, chain_spec("llama8b_q5k"), seed, k=8)
-    if name in ("gemv_q4k_4096", "gateup_q4k", "gateup_q5k", "down_q6k"):
+    if name in ("llama8b_q2k_chain", "llama8b_q3k_chain"):
+        return Resident(torch, kq, kqgen, chain_spec(name[:-len("_chain")]), seed)
+    if name in ("gemv_q4k_4096", "gateup_q4k", "gateup_q5k", "down_q6k", "gateup_q2k", "gateup_q3k", "down_q3k"):
         return Resident(torch, kq, kqgen, chain_spec(name), seed)
     if name.startswith("verify8b_k"):
         k = int(name[len("verify8b_k"):])
@@ -711,7 +730,8 @@ def cpu_baseline(args, budget_s=15.0):
         per_token = MOE30B["layers"] * MOE30B["top"] * (2 * MOE30B["ffn"] * row_bytes("q4_k", MOE30B["hidden"])
                                                         + MOE30B["hidden"] * row_bytes("q4_k", MOE30B["ffn"]))
     else:
-        base = {"llama8b_chain": "llama8b", "llama8b_q5k_chain": "llama8b_q5k", "verify8b_q5k_k8": "llama8b_q5k", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
+        base = {"llama8b_chain": "llama8b", "llama8b_q5k_chain": "llama8b_q5k", "verify8b_q5k_k8": "llama8b_q5k",
+                "llama8b_q2k_chain": "llama8b_q2k", "llama8b_q3k_chain": "llama8b_q3k", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
                 "llama8b_layer_fused_steps": "llama8b", "llama70b_resident": "llama70b",
                 "llama70b_resident_steps": "llama70b", "llama70b_stream": "llama70b", "llama70b_stream_20gb": "llama70b"}
         name = base.get(args.workload, "llama8b" if args.workload.startswith("verify") else args.workload)

@@ -106,12 +106,15 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     cudaError_t err = dev_info(di);
     if (err != cudaSuccess) return cuda_fail(err, "device query");
     const int nb = a.nbs;  // blocks per K range (all of K unless split)
-    if (fmt == KQ_FMT_Q5_K && ncol > 1)
-        return fail(KQ_ERR_UNSUPPORTED, "Q5_K with %d columns runs on the tensor-core kernel only", ncol);
-    if (fmt != KQ_FMT_Q6_K) {  // Q4_K, Q5_K
+    if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q6_K && ncol > 1)
+        return fail(KQ_ERR_UNSUPPORTED, "format %d with %d columns: not in this kernel", fmt, ncol);
+    if ((fmt == KQ_FMT_Q2_K && nb % 4 != 0) || (fmt == KQ_FMT_Q3_K && nb % 8 != 0))
+        return fail(KQ_ERR_UNSUPPORTED, "%s rows must be 16-byte aligned (K %% %d == 0), K=%lld",
+                    fmt == KQ_FMT_Q2_K ? "Q2_K" : "Q3_K", fmt == KQ_FMT_Q2_K ? 1024 : 2048, (long long)a.K);
+    if (fmt != KQ_FMT_Q6_K) {  // Q2_K..Q5_K: lanes take (row pair, block, half)
         const int ur = 2 * nb;  // half-block units per row pair
         const int lr = ur <= 32 ? next_pow2(ur) : static_cast<int>(round_up(ur, 32));
-        if (lr > kConsumers) return fail(KQ_ERR_UNSUPPORTED, "Q4_K with K=%lld > 32768", (long long)a.K);
+        if (lr > kConsumers) return fail(KQ_ERR_UNSUPPORTED, "K=%lld > 32768", (long long)a.K);
         a.lanes_per_rp = lr;
         a.ps = kConsumers / lr;
         a.parts = lr > 32 ? lr / 32 : 1;
@@ -135,7 +138,7 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     const int ng = ncol == 1 ? 2 : 1;
     const bool shared_x = a.x_seg_stride == 0;
     const size_t wp_bytes = round_up(sizeof(float) * ng * 2 * a.ps * a.parts * 2 * ncol, 128);
-    // one column of Q4_K: integer activation regions (2 x 336 bytes per
+    // one column (not Q6_K): integer activation regions (2 x 336 bytes per
     // super-block); otherwise fp32 regions
     const size_t xcopy = ncol == 1 && fmt != KQ_FMT_Q6_K ? static_cast<size_t>(672) * nb
                                                           : sizeof(float) * ncol * 2 * nb * kRegion;
@@ -252,6 +255,8 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     DevInfo di;
     cudaError_t err = dev_info(di);
     if (err != cudaSuccess) return cuda_fail(err, "device query");
+    if (fmt == KQ_FMT_Q2_K || fmt == KQ_FMT_Q3_K)
+        return fail(KQ_ERR_UNSUPPORTED, "no tensor-core kernel for format %d", fmt);
     if (fmt == KQ_FMT_Q6_K && a.nb % 8 != 0)
         return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
     // RMSNorm scratch after the ring: 8 columns' sums per super-block, 8 norms
@@ -341,8 +346,10 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
 
 static bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
+static bool known_format(int fmt) { return fmt >= KQ_FMT_Q4_K && fmt <= KQ_FMT_Q3_K; }
+
 static int check_matrix(const void* W, int fmt, int64_t N, int64_t K) {
-    if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q5_K && fmt != KQ_FMT_Q6_K)
+    if (!known_format(fmt))
         return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
     if (N < 0 || K < 0) return fail(KQ_ERR_INVALID_ARG, "negative size N=%lld K=%lld", (long long)N, (long long)K);
     if (K % 256 != 0) return fail(KQ_ERR_INVALID_ARG, "K=%lld is not a multiple of 256", (long long)K);
@@ -360,9 +367,11 @@ static int check_matrix(const void* W, int fmt, int64_t N, int64_t K) {
 static int padded_cols(int k) { return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : 8; }
 
 static cudaError_t dispatch(const GemvArgs& a, const LaunchPlan& p, int fmt, int ncol, cudaStream_t s) {
-    if (fmt == KQ_FMT_Q5_K) {
-        if (ncol == 1) return launch_one<3, 1, 2>(a, p, s);
-        return cudaErrorNotSupported;  // (plan_gemv refuses it first)
+    if (fmt == KQ_FMT_Q5_K || fmt == KQ_FMT_Q2_K || fmt == KQ_FMT_Q3_K) {
+        if (ncol != 1) return cudaErrorNotSupported;  // (plan_gemv refuses it first)
+        if (fmt == KQ_FMT_Q5_K) return launch_one<3, 1, 2>(a, p, s);
+        if (fmt == KQ_FMT_Q2_K) return launch_one<4, 1, 2>(a, p, s);
+        return launch_one<5, 1, 2>(a, p, s);
     }
     if (fmt == KQ_FMT_Q4_K) {
         switch (ncol) {
@@ -400,8 +409,9 @@ static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt,
 
 // Calls with 2 or more columns (speculative verify) run on the tensor-core
 // kernel, every column group of the call included, so a column's arithmetic
-// never depends on how the call was grouped.
-static bool use_mma(int, int k) { return k >= 2; }
+// never depends on how the call was grouped.  Q2_K and Q3_K have no
+// tensor-core kernel: their columns run one single-column launch each.
+static bool use_mma(int fmt, int k) { return k >= 2 && fmt != KQ_FMT_Q2_K && fmt != KQ_FMT_Q3_K; }
 
 static int plan_for(int fmt, int k, bool mma, GemvArgs& a, LaunchPlan& p) {
     if (mma) return plan_mma(fmt, k <= 4 ? 1 : 2, a, p);
@@ -426,15 +436,15 @@ static int run(GemvArgs& a, int fmt, int k, bool mma, cudaStream_t stream) {
 }
 
 // Split over K across CTAs for matrices with fewer row pairs than SMs:
-// S ranges of nbs super-blocks each (a multiple of 8 for Q6_K, keeping every
-// range 16-byte aligned).  A pure function of (fmt, N, K, SM count), so
+// S ranges of nbs super-blocks each (a multiple of 8 for Q3_K and Q6_K, of
+// 4 for Q2_K, keeping every range 16-byte aligned).  A pure function of (fmt, N, K, SM count), so
 // single- and multi-column calls split alike.
 static void choose_split(int fmt, int64_t N, int nb, int sm_count, int* S, int* nbs) {
     *S = 1;
     *nbs = nb;
     const int64_t P = (N + 1) / 2;
     if (P * 2 > sm_count) return;                       // enough row pairs already
-    const int unit = fmt == KQ_FMT_Q6_K ? 8 : 1;
+    const int unit = fmt == KQ_FMT_Q6_K || fmt == KQ_FMT_Q3_K ? 8 : fmt == KQ_FMT_Q2_K ? 4 : 1;
     const int max_s = nb / unit;
     int want = static_cast<int>((sm_count + P - 1) / P);
     if (want > max_s) want = max_s;
@@ -519,7 +529,14 @@ const char* kq_status_str(int status) {
 const char* kq_last_error(void) { return g_last_error; }
 
 size_t kq_block_bytes(int fmt) {
-    return fmt == KQ_FMT_Q4_K ? kQ4Bytes : fmt == KQ_FMT_Q6_K ? kQ6Bytes : fmt == KQ_FMT_Q5_K ? kQ5Bytes : 0;
+    switch (fmt) {
+        case KQ_FMT_Q4_K: return kQ4Bytes;
+        case KQ_FMT_Q6_K: return kQ6Bytes;
+        case KQ_FMT_Q5_K: return kQ5Bytes;
+        case KQ_FMT_Q2_K: return kQ2Bytes;
+        case KQ_FMT_Q3_K: return kQ3Bytes;
+        default: return 0;
+    }
 }
 
 size_t kq_row_bytes(int fmt, int64_t K) {
@@ -807,7 +824,7 @@ static int split_for(int fmt, int64_t N, int64_t K, int* S, int* nbs) {
 }
 
 size_t kq_splitk_workspace_bytes(int fmt, int64_t N, int64_t K, int k) {
-    if ((fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q5_K && fmt != KQ_FMT_Q6_K) || N < 1 || K < 256 || K % 256 != 0 || k < 1 ||
+    if (!known_format(fmt) || N < 1 || K < 256 || K % 256 != 0 || k < 1 ||
         k > 8)
         return 0;
     int S = 1, nbs = 0;
@@ -851,8 +868,7 @@ int kq_gemv_splitk(const void* W, int fmt, int64_t N, int64_t K, const float* x,
 
 int kq_unpack(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d, kq_stream_t stream) {
     g_last_error[0] = 0;
-    if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q5_K && fmt != KQ_FMT_Q6_K)
-        return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
+    if (!known_format(fmt)) return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
     if (n_blocks < 0) return fail(KQ_ERR_INVALID_ARG, "n_blocks < 0");
     if (n_blocks == 0) return KQ_OK;
     if (!W || !q || !sc || !d) return fail(KQ_ERR_INVALID_ARG, "NULL pointer");

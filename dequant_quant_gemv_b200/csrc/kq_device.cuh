@@ -11,10 +11,12 @@ namespace kq {
 constexpr int kQ4Bytes = 144;      // Q4_K super-block
 constexpr int kQ6Bytes = 210;      // Q6_K super-block
 constexpr int kQ5Bytes = 176;      // Q5_K super-block
-// Bytes of a super-block of format FMT (1 Q4_K, 2 Q6_K, 3 Q5_K).
+constexpr int kQ2Bytes = 84;       // Q2_K super-block
+constexpr int kQ3Bytes = 110;      // Q3_K super-block
+// Bytes of a super-block of format FMT (1 Q4_K, 2 Q6_K, 3 Q5_K, 4 Q2_K, 5 Q3_K).
 template <int FMT>
 __host__ __device__ constexpr int block_bytes_of() {
-    return FMT == 1 ? kQ4Bytes : FMT == 2 ? kQ6Bytes : kQ5Bytes;
+    return FMT == 1 ? kQ4Bytes : FMT == 2 ? kQ6Bytes : FMT == 3 ? kQ5Bytes : FMT == 4 ? kQ2Bytes : kQ3Bytes;
 }
 constexpr int kConsumerWarps = 8;  // warps that dequantise and multiply
 constexpr int kConsumers = kConsumerWarps * 32;

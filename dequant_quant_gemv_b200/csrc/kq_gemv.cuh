@@ -653,7 +653,7 @@ __device__ __noinline__ void stage_x_pro(const ProStage p, uint32_t xs, int ct, 
 // 6-bit codes cost more to assemble than the DP4A saves.)
 
 constexpr int kXGroupBytes = 64;  // 32 high bytes, then 32 low bytes
-constexpr int kXInfoBytes = 16;   // Xg, P (and 8 bytes of padding)
+constexpr int kXInfoBytes = 16;   // Xg, P; with S16 also the int sums of xi 0..15 and 16..31
 // A region holds the 4 groups of one half super-block (its bytes, then its
 // 4 info records) plus 16 bytes of padding: 336 bytes = 21 16-byte units,
 // an odd count, so the regions of 8 consecutive lanes (consecutive halves
@@ -669,8 +669,10 @@ __device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H) {
 // position), U groups' loads in flight.  PRO: with the prologue a.pro, its
 // second operand (gamma, or u) loaded beside x; RMSNorm's partial sums of
 // squares (raw x, per lane in group order, then a butterfly) go to
-// part[0][warp] and the inverse norm to pro_inv_addr(part).
-template <bool PRO>
+// part[0][warp] and the inverse norm to pro_inv_addr(part).  S16: the info
+// record also holds the integer sums of the group's first and last 16 xi
+// (for formats whose scales and offsets cover 16 weights).
+template <bool PRO, bool S16 = false>
 __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, int warp, int nwarps, int lane,
                                    int bar, int nthr, int kb0, int nbl, uint32_t part) {
     constexpr int U = 8;  // one round of loads for K = 4096 and 16 warps
@@ -709,12 +711,22 @@ __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, 
                 sh = sh > 100 ? 100 : sh < -100 ? -100 : sh;
             }
             const int xi = __float2int_rn(v[u] * __int_as_float((sh + 127) << 23));
-            const float X = static_cast<float>(__reduce_add_sync(0xffffffffu, xi)) * __int_as_float((127 - sh) << 23);
+            const int tot = __reduce_add_sync(0xffffffffu, xi);
+            const float X = static_cast<float>(tot) * __int_as_float((127 - sh) << 23);
             const uint32_t xr = x_region(xs, G >> 3, (G >> 2) & 1), k = G & 3;
             asm volatile("st.shared.u8 [%0], %1;" ::"r"(xr + kXGroupBytes * k + lane), "r"(xi >> 8) : "memory");
             asm volatile("st.shared.u8 [%0], %1;" ::"r"(xr + kXGroupBytes * k + 32 + lane), "r"(xi & 255)
                          : "memory");
-            if (lane == 0) {
+            if constexpr (S16) {
+                const int first = __reduce_add_sync(0xffffffffu, lane < 16 ? xi : 0);
+                if (lane == 0) {
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                     xr + 4 * kXGroupBytes + kXInfoBytes * k),
+                                 "r"(__float_as_uint(X)), "r"(static_cast<uint32_t>((127 - sh) << 23)), "r"(first),
+                                 "r"(tot - first)
+                                 : "memory");
+                }
+            } else if (lane == 0) {
                 asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(xr + 4 * kXGroupBytes + kXInfoBytes * k),
                              "r"(__float_as_uint(X)), "r"(static_cast<uint32_t>((127 - sh) << 23))
                              : "memory");
@@ -850,6 +862,135 @@ __device__ __forceinline__ void q5k_unit_int(uint32_t row0, int row_bytes, int b
     out[1][0] = y[1];
 }
 
+// Q2_K unit, one column, on DP4A: row pair at row0, super-block b (84
+// bytes: 16 scale|min bytes, 64 quant bytes, d, dmin; 4-byte aligned), half
+// H.  Weight 128H + 32j + l is bits 2j of quant byte 32H + l, in 16-weight
+// group 8H + 2j + l/16.  Per group the exact S = sum q*xi, then
+// y += d*sc*P*S - dmin*m*P*(the group's 16-sum of xi).
+__device__ __forceinline__ void q2k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
+                                             float (&out)[2][1]) {
+    uint32_t Q[2][8], sw[2][2];
+    float dd[2], dm[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint32_t blk = row0 + r * row_bytes + b * kQ2Bytes;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) Q[r][t] = ld_s32(blk + 16 + 32 * H + 4 * t);
+        sw[r][0] = ld_s32(blk + 8 * H);
+        sw[r][1] = ld_s32(blk + 8 * H + 4);
+        const uint32_t dw = ld_s32(blk + 80);
+        dd[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw & 0xFFFFu)));
+        dm[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw >> 16)));
+    }
+    float y[2] = {0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * j);  // X, P, 16-sums
+        const float P = __uint_as_float(info.y);
+#pragma unroll
+        for (int sh = 0; sh < 2; ++sh) {
+            const uint4 xh = ld_s128(xr + kXGroupBytes * j + 16 * sh);
+            const uint4 xl = ld_s128(xr + kXGroupBytes * j + 32 + 16 * sh);
+            int hi[2] = {0, 0};
+            uint32_t lo[2] = {0u, 0u};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const uint32_t q = (Q[r][4 * sh + m] >> (2 * j)) & 0x03030303u;
+                    hi[r] = dp4a_us(q, u4w(xh, m), hi[r]);
+                    lo[r] = dp4a_uu(q, u4w(xl, m), lo[r]);
+                }
+            }
+            const float x16 = static_cast<float>(static_cast<int>(sh ? info.w : info.z)) * P;
+            const int g = 2 * j + sh;  // group within the half
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t sb = (sw[r][g >> 2] >> (8 * (g & 3))) & 0xFFu;
+                const float S = static_cast<float>(hi[r] * 256 + static_cast<int>(lo[r]));
+                y[r] = fmaf(dd[r] * static_cast<float>(sb & 15u) * P, S, y[r]);
+                y[r] = fmaf(-dm[r] * static_cast<float>(sb >> 4), x16, y[r]);
+            }
+        }
+    }
+    out[0][0] = y[0];
+    out[1][0] = y[1];
+}
+
+// Q3_K unit, one column, on DP4A: row pair at row0, super-block b (110
+// bytes: hmask[32], 64 quant bytes, 12 scale bytes, d), half H.  Blocks are
+// 2-byte aligned only and the parity of b varies across the lanes, so each
+// stream of words is loaded from the 4-byte aligned address at or below
+// its start (one word more than it needs) and every word rebuilt by a byte
+// permute whose selector is picked by b's parity.  Weight 128H + 32j + l:
+// q + 4 = (bits 2j of quant byte 32H + l) | (bit 4H + j of hmask[l]) << 2,
+// in 0..7; per 16-weight group the exact S = sum (q+4)*xi - 4*(16-sum of xi)
+// and y += d*(v - 32)*P*S with v the group's 6-bit scale.
+__device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
+                                             float (&out)[2][1]) {
+    const bool odd = b & 1;
+    const uint32_t sel = odd ? 0x5432u : 0x3210u;
+    uint32_t Q[2][8], M[2][8], sc[2][2], hs[2];
+    float dd[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint32_t bw = row0 + r * row_bytes + b * kQ3Bytes - (odd ? 2 : 0);  // 4-byte aligned
+        uint32_t L[9];
+#pragma unroll
+        for (int t = 0; t < 9; ++t) L[t] = ld_s32(bw + 32 + 32 * H + 4 * t);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) Q[r][t] = __byte_perm(L[t], L[t + 1], sel);
+#pragma unroll
+        for (int t = 0; t < 9; ++t) L[t] = ld_s32(bw + 4 * t);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) M[r][t] = __byte_perm(L[t], L[t + 1], sel);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) L[t] = ld_s32(bw + 96 + 4 * t);
+        // the half's 8 groups: low 4 bits from scale bytes 0..7 (nibble H),
+        // high 2 bits from bytes 8..11 (bits 2(g/4)+4H .. of byte 8 + g%4)
+        sc[r][0] = (__byte_perm(L[0], L[1], sel) >> (4 * H)) & 0x0F0F0F0Fu;
+        sc[r][1] = (__byte_perm(L[1], L[2], sel) >> (4 * H)) & 0x0F0F0F0Fu;
+        hs[r] = __byte_perm(L[2], L[3], sel) >> (4 * H);
+        dd[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(L[3] >> (odd ? 16 : 0))));
+    }
+    float y[2] = {0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * j);  // X, P, 16-sums
+        const float P = __uint_as_float(info.y);
+#pragma unroll
+        for (int sh = 0; sh < 2; ++sh) {
+            const uint4 xh = ld_s128(xr + kXGroupBytes * j + 16 * sh);
+            const uint4 xl = ld_s128(xr + kXGroupBytes * j + 32 + 16 * sh);
+            int hi[2] = {0, 0};
+            uint32_t lo[2] = {0u, 0u};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int t = 4 * sh + m;
+                    const uint32_t q = ((Q[r][t] >> (2 * j)) & 0x03030303u) |
+                                       (((M[r][t] >> (4 * H + j)) & 0x01010101u) << 2);
+                    hi[r] = dp4a_us(q, u4w(xh, m), hi[r]);
+                    lo[r] = dp4a_uu(q, u4w(xl, m), lo[r]);
+                }
+            }
+            const int x16 = static_cast<int>(sh ? info.w : info.z);
+            const int g = 2 * j + sh;  // group within the half
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t lo4 = (sc[r][g >> 2] >> (8 * (g & 3))) & 15u;
+                const uint32_t hi2 = (hs[r] >> (8 * (g & 3) + 2 * (g >> 2))) & 3u;
+                const float v = static_cast<float>(static_cast<int>(lo4 | (hi2 << 4)) - 32);
+                const int S = hi[r] * 256 + static_cast<int>(lo[r]) - 4 * x16;
+                y[r] = fmaf(dd[r] * v * P, static_cast<float>(S), y[r]);
+            }
+        }
+    }
+    out[0][0] = y[0];
+    out[1][0] = y[1];
+}
+
 // Dispatch a Q6_K unit to the code path of its alignment class.
 template <int NCOL>
 __device__ __forceinline__ void q6k_unit_dispatch(int kappa, uint32_t row0, int row_bytes, int b, int H,
@@ -864,7 +1005,8 @@ __device__ __forceinline__ void q6k_unit_dispatch(int kappa, uint32_t row0, int 
 template <int FMT, int NCOL, bool INT, bool PRO>
 __device__ __forceinline__ void stage_all(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar,
                                           int kb0, int nbl, uint32_t part) {
-    if constexpr (INT) stage_x_int<PRO>(a, seg, xs, ct >> 5, nthr >> 5, ct & 31, bar, nthr, kb0, nbl, part);
+    if constexpr (INT)
+        stage_x_int<PRO, (FMT == 4 || FMT == 5)>(a, seg, xs, ct >> 5, nthr >> 5, ct & 31, bar, nthr, kb0, nbl, part);
     else if constexpr (PRO)
         stage_x_pro<FMT, NCOL>(ProStage{a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256,
                                         a.pro == 1 ? a.gamma + static_cast<int64_t>(kb0) * 256 : nullptr, a.K, a.ldx,
@@ -913,7 +1055,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     const int64_t rp_begin = P * rc / G;
     const int64_t rp_end = P * (rc + 1) / G;
     constexpr int BS = block_bytes_of<FMT>();
-    static_assert(FMT != 3 || NCOL == 1, "Q5_K with several columns runs on the tensor cores");
+    static_assert(FMT <= 2 || NCOL == 1, "Q5_K, Q2_K and Q3_K: one column per launch in this kernel");
     const int kb0 = ks * a.nbs;
     const int nbl = a.nb - kb0 < a.nbs ? a.nb - kb0 : a.nbs;       // blocks in this range
     const int srow = a.ksplit > 1 ? a.nbs * BS : static_cast<int>(a.row_bytes);  // staged row stride
@@ -1019,8 +1161,12 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             const uint32_t row0 = sbuf_s + slot * a.stage_bytes + 2 * u_rp * srow;
             if constexpr (INT && FMT == 1) {
                 q4k_unit_int(row0, srow, u_b, u_H, xri, out);
-            } else if constexpr (INT) {
+            } else if constexpr (INT && FMT == 3) {
                 q5k_unit_int(row0, srow, u_b, u_H, xri, out);
+            } else if constexpr (INT && FMT == 4) {
+                q2k_unit_int(row0, srow, u_b, u_H, xri, out);
+            } else if constexpr (INT && FMT == 5) {
+                q3k_unit_int(row0, srow, u_b, u_H, xri, out);
             } else if constexpr (FMT == 1) {
                 q4k_unit<NCOL>(row0, srow, u_b, u_H, xr, xcs, out);
             } else {

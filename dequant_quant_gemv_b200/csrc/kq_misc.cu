@@ -48,6 +48,37 @@ __global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_
                     static_cast<uint8_t>(((v >> (8 * k + 4)) & 15u) | (((eb >> (2 * c + 1)) & 1u) << 4));
             }
         }
+    } else if (fmt == 4) {
+        // Q2_K: 4-byte aligned blocks
+        const uint8_t* blk = W + b * kQ2Bytes;
+        for (int g = 0; g < 16; ++g) sc[16 * b + g] = blk[g];
+        for (int i = 0; i < 64; ++i) {
+            const uint32_t v = blk[16 + i];
+            const int n = i >> 5, l = i & 31;
+            for (int j = 0; j < 4; ++j) q[256 * b + 128 * n + 32 * j + l] = static_cast<uint8_t>((v >> (2 * j)) & 3u);
+        }
+        const uint32_t dw = *reinterpret_cast<const uint32_t*>(blk + 80);
+        d[2 * b] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw & 0xFFFFu)));
+        d[2 * b + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw >> 16)));
+    } else if (fmt == 5) {
+        // Q3_K: 2-byte aligned blocks, read by bytes
+        const uint8_t* blk = W + b * kQ3Bytes;
+        for (int i = 0; i < 64; ++i) {
+            const uint32_t v = blk[32 + i];
+            const int n = i >> 5, l = i & 31;
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t third = (blk[l] >> (4 * n + j)) & 1u;
+                q[256 * b + 128 * n + 32 * j + l] = static_cast<uint8_t>(((v >> (2 * j)) & 3u) + 4 * third - 4);
+            }
+        }
+        for (int g = 0; g < 16; ++g) {
+            const uint32_t lo = g < 8 ? (blk[96 + g] & 15u) : (blk[96 + g - 8] >> 4);
+            const uint32_t hi = (blk[104 + (g & 3)] >> (2 * (g >> 2))) & 3u;
+            sc[16 * b + g] = static_cast<uint8_t>(lo | (hi << 4));
+        }
+        const unsigned short dh = static_cast<unsigned short>(blk[108] | (blk[109] << 8));
+        d[2 * b] = __half2float(__ushort_as_half(dh));
+        d[2 * b + 1] = 0.0f;
     } else {
         const uint8_t* blk = W + b * kQ6Bytes;  // 2-byte aligned only
         auto word = [&](int off) -> uint32_t {

@@ -181,7 +181,10 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
         // this step's activations, staged by all consumer threads
         const GemvArgs a = step_view(s);
         float rinv = 1.f;
-        if (s.fmt != 2) {  // Q4_K and Q5_K: integer regions
+        if (s.fmt == 4 || s.fmt == 5) {  // Q2_K and Q3_K: integer regions with 16-sums
+            if (s.pro) stage_all<4, 1, true, true>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
+            else stage_all<4, 1, true, false>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
+        } else if (s.fmt != 2) {  // Q4_K and Q5_K: integer regions
             if (s.pro) stage_all<1, 1, true, true>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
             else stage_all<1, 1, true, false>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
         } else {
@@ -241,6 +244,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
                 const uint32_t rw = sbuf_s + slot * A.slot_bytes + 2 * u_rp * srow;
                 if (s.fmt == 1) q4k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else if (s.fmt == 3) q5k_unit_int(rw, srow, u_b, u_H, xri, out);
+                else if (s.fmt == 4) q2k_unit_int(rw, srow, u_b, u_H, xri, out);
+                else if (s.fmt == 5) q3k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else q6k_unit_dispatch<1>(kappa, rw, srow, u_b, u_H, xr, xcs, out);
             }
             // butterfly over the lanes of this row pair (fixed order)

@@ -18,8 +18,10 @@ LIB_PATH = os.path.join(_PKG, "libkq.so")
 Q4_K = 1
 Q6_K = 2
 Q5_K = 3
-FORMATS = {"q4_k": Q4_K, "q6_k": Q6_K, "q5_k": Q5_K}
-BLOCK_BYTES = {Q4_K: 144, Q6_K: 210}
+Q2_K = 4
+Q3_K = 5
+FORMATS = {"q4_k": Q4_K, "q6_k": Q6_K, "q5_k": Q5_K, "q2_k": Q2_K, "q3_k": Q3_K}
+BLOCK_BYTES = {Q4_K: 144, Q6_K: 210, Q5_K: 176, Q2_K: 84, Q3_K: 110}
 
 OK = 0
 STATUS = {0: "KQ_OK", 1: "KQ_ERR_INVALID_ARG", 2: "KQ_ERR_UNSUPPORTED", 3: "KQ_ERR_NOT_PINNED",

@@ -1,6 +1,6 @@
 /*
  * kq.h — libkq: decode-time matrix-vector products over GGUF K-quant
- * weights (Q4_K, Q5_K, Q6_K) on NVIDIA B200 (sm_100a), with the weights
+ * weights (Q2_K, Q3_K, Q4_K, Q5_K, Q6_K) on NVIDIA B200 (sm_100a), with the weights
  * dequantised only in registers inside the fused kernels.
  *
  * What the method is (by page):
@@ -29,6 +29,16 @@
  *     weight 64c+32+l the high nibble and bit 2c+1.
  *     w = d*sc_j*q - dmin*m_j, q in 0..31.  (A K-quant of the Q2_K..Q6_K
  *     family "RunNburn - Run a 295B MoE ..." runs natively.)
+ *   Q2_K super-block, 84 bytes, 256 weights in 16 groups of 16:
+ *     16 bytes sc_g | m_g << 4 | 64 bytes of 2-bit quants | fp16 d | fp16
+ *     dmin.  Weight 128n+32j+l is bits 2j..2j+1 of quant byte 32n+l; its
+ *     group is g = i/16.   w = d*sc_g*q - dmin*m_g, q in 0..3.
+ *   Q3_K super-block, 110 bytes, 256 weights in 16 groups of 16:
+ *     32 bytes hmask | 64 bytes of low 2 bits | 12 bytes of 6-bit scales
+ *     v_g | fp16 d.  Weight 128n+32j+l: low bits as Q2_K, third bit = bit
+ *     4n+j of hmask[l], q = (low | third << 2) - 4 in -4..3; v_g: low 4 bits
+ *     from scale byte g (g < 8, low nibble) or g-8 (high nibble), top 2
+ *     bits from bits 2(g/4) of byte 8 + g%4.   w = d*(v_g - 32)*q.
  *   Q6_K super-block, 210 bytes, 256 weights in 16 groups of 16:
  *     128 bytes low 4 bits | 64 bytes high 2 bits | 16 int8 scales s_g |
  *     fp16 d.   w = d*s_g*(q - 32), q in 0..63.
@@ -40,18 +50,19 @@
  *    caller; libkq never frees or retains them past the call (the chain object
  *    below is the exception and says so).
  *  - W must be 16-byte aligned, and so must every row: always true for Q4_K
- *    and Q5_K; for Q6_K it requires K % 2048 == 0.  x and y must be 4-byte
- *    aligned.
+ *    and Q5_K; Q2_K requires K % 1024 == 0, Q3_K and Q6_K K % 2048 == 0
+ *    (else KQ_ERR_UNSUPPORTED).  x and y must be 4-byte aligned.
  *  - Calls are asynchronous on `stream` (0 = the legacy default stream).  The
  *    return value reports argument validation and launch errors only
  *    (KQ_ERR_CUDA carries cudaGetLastError()); kq_last_error() gives text.
  *  - Arithmetic: quants are unpacked exactly; sums are fp32 (or exact
- *    integers).  Single-column Q4_K and Q5_K round each activation to a 14-bit
+ *    integers).  Single-column Q2_K..Q5_K round each activation to a 14-bit
  *    integer on a power-of-two grid per group of 32 (error at most 2^-14 of
  *    the group's largest |x|); single-column Q6_K multiplies in fp32; two or
- *    more columns run on the tensor cores with exact fp16 weight operands and
+ *    more columns of Q4_K..Q6_K run on the tensor cores with exact fp16 weight operands and
  *    activations split into two fp16 terms (22 bits) after a power-of-two
- *    scale per super-block.  Every output satisfies
+ *    scale per super-block; several columns of Q2_K and Q3_K run one
+ *    single-column launch per column.  Every output satisfies
  *    |y - y_exact| <= 1e-3 * sum_i |w_i x_i| + 1e-6 for activations of
  *    comparable magnitude within each group of 32.
  *    Results are deterministic: the same inputs give bitwise-equal outputs;
@@ -82,7 +93,9 @@ typedef struct CUstream_st* kq_stream_t;
 typedef enum {
     KQ_FMT_Q4_K = 1,
     KQ_FMT_Q6_K = 2,
-    KQ_FMT_Q5_K = 3
+    KQ_FMT_Q5_K = 3,
+    KQ_FMT_Q2_K = 4,
+    KQ_FMT_Q3_K = 5
 } kq_fmt;
 
 typedef enum {
@@ -111,7 +124,8 @@ KQ_API const char* kq_last_error(void);
  * hanging.  Synchronous.  *out is a HOST int. */
 KQ_API int kq_device_fault(int* out);
 
-/* Bytes per super-block (144 or 210) or 0 for an unknown format. */
+/* Bytes per super-block (Q2_K 84, Q3_K 110, Q4_K 144, Q5_K 176, Q6_K 210)
+ * or 0 for an unknown format. */
 KQ_API size_t kq_block_bytes(int fmt);
 
 /* Bytes per weight row: (K/256) * kq_block_bytes(fmt); 0 if K % 256 != 0. */
@@ -281,10 +295,13 @@ KQ_API int kq_moe_gemv(const void* W_experts, int fmt, int E, int64_t N, int64_t
  * kq_unpack — debug: the integer fields of n_blocks consecutive super-blocks
  * as the GEMV kernels decode them (for bit-exact comparison).
  *   q:  n_blocks*256 bytes, quant of weight i of block b at q[256b+i]
- *       (Q4_K 0..15; Q6_K 0..63, before the -32 offset)
- *   sc: n_blocks*16 bytes; Q4_K: sc_0..7 then m_0..7; Q6_K: the 16 int8
- *       scales as two's-complement bytes
- *   d:  n_blocks*2 floats; Q4_K: d, dmin; Q6_K: d, 0 (fp16 widened exactly)
+ *       (Q2_K 0..3; Q3_K -4..3 as two's-complement bytes; Q4_K 0..15;
+ *       Q5_K 0..31; Q6_K 0..63, before the -32 offset)
+ *   sc: n_blocks*16 bytes; Q4_K, Q5_K: sc_0..7 then m_0..7; Q2_K: the 16
+ *       bytes sc_g | m_g << 4 as stored; Q3_K: the 16 6-bit v_g (before the
+ *       -32 offset); Q6_K: the 16 int8 scales as two's-complement bytes
+ *   d:  n_blocks*2 floats; Q2_K, Q4_K, Q5_K: d, dmin; Q3_K, Q6_K: d, 0
+ *       (fp16 widened exactly)
  * All device pointers; W must be 16-byte aligned.
  */
 KQ_API int kq_unpack(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d,

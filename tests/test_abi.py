@@ -49,7 +49,11 @@ def test_host_only_helpers(libkq):
     assert L.kq_row_bytes(1, 300) == 0
     assert L.kq_block_bytes(3) == 176                 # Q5_K
     assert L.kq_row_bytes(3, 4096) == 16 * 176
-    assert L.kq_block_bytes(4) == 0                   # no such format
+    assert L.kq_block_bytes(4) == 84                  # Q2_K
+    assert L.kq_block_bytes(5) == 110                 # Q3_K
+    assert L.kq_row_bytes(5, 2048) == 8 * 110
+    assert L.kq_block_bytes(6) == 0                   # no such format
+    assert L.kq_block_bytes(0) == 0
     assert L.kq_status_str(0) == b"ok"
     assert L.kq_version() >= 100
 

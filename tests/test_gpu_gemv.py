@@ -27,7 +27,9 @@ def _cuda():
 
 # ------------------------------------------------------------ bit-exact
 @pytest.mark.parametrize("fmt,N,K", [("q4_k", 4096, 4096), ("q6_k", 64, 14336), ("q6_k", 3, 2048),
-                                     ("q5_k", 2048, 4096), ("q5_k", 3, 256)])
+                                     ("q5_k", 2048, 4096), ("q5_k", 3, 256), ("q2_k", 512, 4096),
+                                     ("q2_k", 3, 1024), ("q3_k", 512, 4096), ("q3_k", 3, 2048),
+                                     ("q3_k", 1, 256)])
 def test_unpack_bit_exact(fmt, N, K):
     W = matrix(fmt, 1000 + N, N, K)
     nb = N * K // 256
@@ -47,6 +49,10 @@ SHAPES = [
     ("q6_k", 11, 16384),
     ("q5_k", 1, 256), ("q5_k", 7, 768), ("q5_k", 257, 4096), ("q5_k", 301, 8192), ("q5_k", 9, 32768),
     ("q5_k", 5, 1280), ("q5_k", 4096, 4096), ("q5_k", 2, 14336),
+    ("q2_k", 1, 1024), ("q2_k", 3, 1024), ("q2_k", 257, 4096), ("q2_k", 301, 8192), ("q2_k", 9, 32768),
+    ("q2_k", 5, 3072), ("q2_k", 4096, 4096), ("q2_k", 2, 14336),
+    ("q3_k", 1, 2048), ("q3_k", 5, 2048), ("q3_k", 257, 4096), ("q3_k", 301, 8192), ("q3_k", 9, 32768),
+    ("q3_k", 37, 6144), ("q3_k", 4096, 4096), ("q3_k", 2, 14336),
 ]
 
 
@@ -115,6 +121,38 @@ def test_q5k_zero_quants_closed_form():
     want = -np.einsum("rb,rbj,bj->r", dmin, m, X)
     s = np.einsum("rb,rbj,bj->r", dmin, m, np.abs(x.astype(np.float64)).reshape(K // 32, 32).sum(1).reshape(K // 256, 8))
     assert_close(y, want, s, "q5k zero quants")
+
+
+def test_q2k_zero_quants_closed_form():
+    """All-zero Q2_K quants: y = -sum_g dmin*m_g*(sum of x over 16-weight
+    group g); with zero mins as well, y = 0 exactly."""
+    N, K = 70, 4096
+    nb = N * K // 256
+    lg = kqgen.q2k_draw(126, nb)
+    W = kqgen.q2k_pack(np.zeros_like(lg["q"]), lg["sc"], lg["m"], lg["d"], lg["dmin"])
+    x = x_vec(127, K)
+    y = kq.gemv(dev(W), "q2_k", N, K, dev(x))
+    X = x.astype(np.float64).reshape(K // 256, 16, 16).sum(axis=2)
+    A = np.abs(x.astype(np.float64)).reshape(K // 256, 16, 16).sum(axis=2)
+    dmin = lg["dmin"].view(np.float16).astype(np.float64).reshape(N, K // 256)
+    m = lg["m"].astype(np.float64).reshape(N, K // 256, 16)
+    want = -np.einsum("rb,rbg,bg->r", dmin, m, X)
+    assert_close(y, want, np.einsum("rb,rbg,bg->r", dmin, m, A), "q2k zero quants")
+    W0 = kqgen.q2k_pack(np.zeros_like(lg["q"]), lg["sc"], np.zeros_like(lg["m"]), lg["d"], lg["dmin"])
+    assert torch.all(kq.gemv(dev(W0), "q2_k", N, K, dev(x)) == 0)
+
+
+def test_q3k_zero_values_and_scales_give_exact_zero():
+    """Q3_K quants of value 0 (third bit set, low bits 0), or every scale at
+    its offset v = 32, give y = 0 exactly."""
+    N, K = 70, 4096
+    nb = N * K // 256
+    lg = kqgen.q3k_draw(128, nb)
+    x = dev(x_vec(129, K))
+    W = kqgen.q3k_pack(np.zeros_like(lg["q"]), lg["v"], lg["d"])
+    assert torch.all(kq.gemv(dev(W), "q3_k", N, K, x) == 0)
+    W = kqgen.q3k_pack(lg["q"], np.full_like(lg["v"], 32), lg["d"])
+    assert torch.all(kq.gemv(dev(W), "q3_k", N, K, x) == 0)
 
 
 def test_q4k_zero_quants_closed_form():
@@ -186,7 +224,8 @@ def test_linearity():
                                      ("q4_k", 4096, 4096), ("q4_k", 33, 14336), ("q6_k", 64, 4096),
                                      ("q6_k", 41, 2048), ("q6_k", 4096, 2048), ("q6_k", 3, 14336),
                                      ("q5_k", 300, 4096), ("q5_k", 33, 14336), ("q5_k", 4096, 4096),
-                                     ("q5_k", 17, 768)])
+                                     ("q5_k", 17, 768), ("q2_k", 300, 4096), ("q2_k", 33, 14336),
+                                     ("q3_k", 300, 4096), ("q3_k", 33, 14336)])
 @pytest.mark.parametrize("k", [2, 3, 4, 5, 8])
 def test_multi_columns_independent_and_match_oracle(fmt, N, K, k):
     """Each column of a k-column call equals the same column of an 8-column
@@ -204,7 +243,8 @@ def test_multi_columns_independent_and_match_oracle(fmt, N, K, k):
         assert_close(Y[c], y_ref[c], s_ref[c], f"col {c}")
 
 
-@pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q5_k", 300, 4096)])
+@pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q5_k", 300, 4096),
+                                     ("q2_k", 300, 4096), ("q3_k", 300, 4096)])
 def test_single_column_of_multi_call_matches_oracle(fmt, N, K):
     """k = 1 through gemv_multi is the single-column kernel, bitwise."""
     W = matrix(fmt, 32, N, K)
@@ -217,7 +257,7 @@ def test_single_column_of_multi_call_matches_oracle(fmt, N, K):
     assert_close(Y[0], y_ref, s_ref)
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k", "q2_k", "q3_k"])
 @pytest.mark.parametrize("scale", [1e-30, 1e-6, 1.0, 3e3, 1e20])
 def test_multi_column_scale_range(fmt, scale):
     """Activations far from 1 in either direction (the kernel rescales each
@@ -279,15 +319,22 @@ def test_invalid_arguments_are_rejected():
     with pytest.raises(kq.KQError) as e:
         kq.gemv(Wq6, "q6_k", 1, 2304, x9, y)    # rows not 16-byte aligned
     assert e.value.status == 2
+    for fmt, Kbad in (("q2_k", 2304), ("q3_k", 1024)):
+        with pytest.raises(kq.KQError) as e:
+            kq.gemv(Wq6, fmt, 1, Kbad, x9, y)   # rows not 16-byte aligned
+        assert e.value.status == 2
+        with pytest.raises(kq.KQError) as e:
+            kq.gemv_multi(Wq6, fmt, 1, Kbad, torch.zeros((3, Kbad), device="cuda"))
+        assert e.value.status == 2
     with pytest.raises(kq.KQError):
         kq.gemv_multi(W, "q4_k", 4, 256, torch.zeros((9, 256), device="cuda"))
     assert kq.device_fault() == 0
 
 
 # ------------------------------------------- single-column integer path
-@pytest.mark.parametrize("fmt", ["q4_k", "q5_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q2_k", "q3_k"])
 def test_single_column_within_activation_rounding_bound(fmt):
-    """Single-column Q4_K and Q5_K round each activation to a 14-bit integer
+    """Single-column Q2_K..Q5_K round each activation to a 14-bit integer
     on a power-of-two grid per group of 32, so |x - x'| <= 2^-14 * (largest
     |x| of the group).  The error must stay within that bound (plus fp32
     rounding slack), computed from the oracle's dequantised weights."""
@@ -304,7 +351,7 @@ def test_single_column_within_activation_rounding_bound(fmt):
     assert np.all(err <= bound + slack), float(np.max(err / (bound + slack)))
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k", "q2_k", "q3_k"])
 @pytest.mark.parametrize("scale", [1e-30, 1e-6, 3e3, 1e20])
 def test_single_column_scale_range(fmt, scale):
     """Single column with activations far from 1: the integer path scales

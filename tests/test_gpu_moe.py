@@ -28,6 +28,10 @@ def _cuda():
     ("q4_k", 5, 33, 256, True),       # odd rows per expert
     ("q5_k", 16, 768, 2048, False),
     ("q5_k", 8, 2048, 768, True),
+    ("q2_k", 16, 768, 2048, False),
+    ("q2_k", 8, 2048, 1024, True),
+    ("q3_k", 8, 512, 2048, True),
+    ("q3_k", 6, 130, 4096, False),
 ])
 def test_moe_parity(fmt, E, N, K, per_id):
     W = matrix(fmt, 300 + E + N, E * N, K)

@@ -21,7 +21,7 @@ def _cuda():
 
 SHAPES = [("q4_k", 1, 4096), ("q4_k", 2, 4096), ("q4_k", 17, 4096), ("q4_k", 64, 32768), ("q4_k", 100, 2048),
           ("q4_k", 5, 768), ("q6_k", 3, 14336), ("q6_k", 64, 28672), ("q6_k", 9, 2048), ("q5_k", 17, 4096),
-          ("q5_k", 3, 14336)]
+          ("q5_k", 3, 14336), ("q2_k", 17, 4096), ("q2_k", 3, 14336), ("q3_k", 17, 4096), ("q3_k", 3, 14336)]
 
 
 @pytest.mark.parametrize("fmt,N,K", SHAPES)
@@ -29,7 +29,8 @@ def test_splitk_parity(fmt, N, K):
     W = matrix(fmt, 900 + N, N, K)
     x = x_vec(901 + K, K)
     Wt, xt = dev(W), dev(x)
-    # Q6_K ranges are multiples of 8 blocks, so K = 2048 cannot split
+    # Q6_K ranges are multiples of 8 blocks, so K = 2048 cannot split (as
+    # are Q3_K's; Q2_K's are multiples of 4)
     splits = kq.splitk_workspace_bytes(fmt, N, K, 1) > 0
     assert splits or (fmt == "q6_k" and K // 256 < 16)
     y = kq.gemv_splitk(Wt, fmt, N, K, xt)

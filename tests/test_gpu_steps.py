@@ -44,7 +44,8 @@ def one_by_one(specs):
 LAYER = [("q4_k", 6144, 4096, "rmsnorm"), ("q4_k", 4096, 4096, "none"), ("q4_k", 300, 4096, "none"),
          ("q6_k", 4096, 14336, "swiglu"), ("q4_k", 64, 768, "none"), ("q6_k", 48, 14336, "none"),
          ("q4_k", 1, 256, "rmsnorm"), ("q4_k", 2048, 8192, "none"), ("q5_k", 1024, 4096, "rmsnorm"),
-         ("q5_k", 96, 14336, "swiglu")]
+         ("q5_k", 96, 14336, "swiglu"), ("q2_k", 1024, 4096, "rmsnorm"), ("q3_k", 96, 14336, "swiglu"),
+         ("q2_k", 40, 14336, "none"), ("q3_k", 300, 4096, "none")]
 
 
 def build(seed, shapes):
