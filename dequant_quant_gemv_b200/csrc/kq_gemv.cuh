@@ -647,10 +647,8 @@ __device__ __noinline__ void stage_x_pro(const ProStage p, uint32_t xs, int ct, 
 // P*xi, up to fp32 rounding of the per-sub-block terms.  |x - P*xi| <= P/2
 // <= 2^-14 * (largest |x| of the group), so |y - y_exact| <= 2^-14 * sum
 // over groups of (max_g |x|) * sum_{i in g} |w_i|.  All-zero quants with
-// zero mins give y = 0 exactly.  The group's largest |x| and the sum of
-// its xi are one warp reduction each (redux.sync on the bit patterns of
-// |x|, which order like the values, and on the xi).  (A Q6_K variant measured slower than its fp32 units: its
-// 6-bit codes cost more to assemble than the DP4A saves.)
+// zero mins give y = 0 exactly.  (A Q6_K variant measured slower than its
+// fp32 units: its 6-bit codes cost more to assemble than the DP4A saves.)
 
 constexpr int kXGroupBytes = 64;  // 32 high bytes, then 32 low bytes
 constexpr int kXInfoBytes = 16;   // Xg, P; with S16 also the int sums of xi 0..15 and 16..31
@@ -665,71 +663,91 @@ __device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H) {
 }
 
 // Stage the K range [256*kb0, 256*(kb0+nbl)) of segment `seg` as above,
-// into the regions at `xs`.  One warp per group of 32 activations (lane =
-// position), U groups' loads in flight.  PRO: with the prologue a.pro, its
+// into the regions at `xs`.  A warp takes 4 groups of 32 activations (one
+// region) per pass: lane l holds 4 consecutive values of group l / 8, loaded
+// as one float4; a group's largest |x| and the sum of its xi are butterflies
+// over its 8 lanes, and each lane writes its 4 high and 4 low bytes as one
+// word each.  U passes' loads in flight.  PRO: with the prologue a.pro, its
 // second operand (gamma, or u) loaded beside x; RMSNorm's partial sums of
-// squares (raw x, per lane in group order, then a butterfly) go to
-// part[0][warp] and the inverse norm to pro_inv_addr(part).  S16: the info
-// record also holds the integer sums of the group's first and last 16 xi
-// (for formats whose scales and offsets cover 16 weights).
+// squares (raw x, per lane, then a butterfly) go to part[0][warp] and the
+// inverse norm to pro_inv_addr(part).  S16: the info record also holds the
+// integer sums of the group's first and last 16 xi (for formats whose
+// scales and offsets cover 16 weights).
 template <bool PRO, bool S16 = false>
 __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, int warp, int nwarps, int lane,
                                    int bar, int nthr, int kb0, int nbl, uint32_t part) {
-    constexpr int U = 8;  // one round of loads for K = 4096 and 16 warps
+    constexpr int U = 2;  // one round of loads for K = 4096 and 16 warps
     const float* xg = a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256;
-    const int groups = 8 * nbl;
+    const int quads = 2 * nbl;  // passes of 4 groups (128 activations)
     const bool rms = PRO && a.pro == 1;
     const float* sg = PRO ? (rms ? a.gamma + static_cast<int64_t>(kb0) * 256 : xg + a.K) : nullptr;
+    const int sub = lane >> 3;     // the lane's group within the pass
+    const int e = 4 * (lane & 7);  // its first position in the group
     float sq = 0.f;
-    for (int base = warp; base < groups; base += nwarps * U) {
-        float v[U], w[U];
+    for (int base = warp; base < quads; base += nwarps * U) {
+        float4 v[U], w[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int G = base + nwarps * u;
-            v[u] = G < groups ? ld_x(xg + 32 * G + lane) : 0.f;
-            if constexpr (PRO) w[u] = G < groups ? ld_x(sg + 32 * G + lane) : 0.f;
+            const int Q = base + nwarps * u;
+            const int off = 128 * Q + 32 * sub + e;
+            v[u] = Q < quads ? ld_f4(xg + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+            if constexpr (PRO) w[u] = Q < quads ? ld_f4(sg + off) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         if constexpr (PRO) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if (rms) {
-                    sq = fmaf(v[u], v[u], sq);
-                    v[u] *= w[u];
+                    sq = fmaf(v[u].x, v[u].x, sq);
+                    sq = fmaf(v[u].y, v[u].y, sq);
+                    sq = fmaf(v[u].z, v[u].z, sq);
+                    sq = fmaf(v[u].w, v[u].w, sq);
+                    v[u] = make_float4(v[u].x * w[u].x, v[u].y * w[u].y, v[u].z * w[u].z, v[u].w * w[u].w);
                 } else {
-                    v[u] = silu_gate(v[u], w[u]);
+                    v[u] = make_float4(silu_gate(v[u].x, w[u].x), silu_gate(v[u].y, w[u].y),
+                                       silu_gate(v[u].z, w[u].z), silu_gate(v[u].w, w[u].w));
                 }
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int G = base + nwarps * u;
-            if (G >= groups) break;  // warp-uniform
-            const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(v[u]) & 0x7FFFFFFFu);
+            const int Q = base + nwarps * u;
+            if (Q >= quads) break;  // warp-uniform
+            float m = fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w)));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+            const uint32_t mb = __float_as_uint(m);
             int sh = 0;
             if (mb != 0u) {
                 sh = 13 - (static_cast<int>(mb >> 23) - 127);
                 sh = sh > 100 ? 100 : sh < -100 ? -100 : sh;
             }
-            const int xi = __float2int_rn(v[u] * __int_as_float((sh + 127) << 23));
-            const int tot = __reduce_add_sync(0xffffffffu, xi);
-            const float X = static_cast<float>(tot) * __int_as_float((127 - sh) << 23);
-            const uint32_t xr = x_region(xs, G >> 3, (G >> 2) & 1), k = G & 3;
-            asm volatile("st.shared.u8 [%0], %1;" ::"r"(xr + kXGroupBytes * k + lane), "r"(xi >> 8) : "memory");
-            asm volatile("st.shared.u8 [%0], %1;" ::"r"(xr + kXGroupBytes * k + 32 + lane), "r"(xi & 255)
-                         : "memory");
-            if constexpr (S16) {
-                const int first = __reduce_add_sync(0xffffffffu, lane < 16 ? xi : 0);
-                if (lane == 0) {
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                                     xr + 4 * kXGroupBytes + kXInfoBytes * k),
-                                 "r"(__float_as_uint(X)), "r"(static_cast<uint32_t>((127 - sh) << 23)), "r"(first),
-                                 "r"(tot - first)
+            const float sc = __int_as_float((sh + 127) << 23);
+            const int x0 = __float2int_rn(v[u].x * sc), x1 = __float2int_rn(v[u].y * sc);
+            const int x2 = __float2int_rn(v[u].z * sc), x3 = __float2int_rn(v[u].w * sc);
+            int t = (x0 + x1) + (x2 + x3);
+            t += __shfl_xor_sync(0xffffffffu, t, 1);
+            t += __shfl_xor_sync(0xffffffffu, t, 2);
+            const int first = t;  // on lanes 0..3 of the group: its first 16
+            t += __shfl_xor_sync(0xffffffffu, t, 4);
+            const uint32_t xr = x_region(xs, Q >> 1, Q & 1);
+            // byte 1 of each xi (the signed high byte), then byte 0
+            const uint32_t hb = __byte_perm(__byte_perm(x0, x1, 0x0051u), __byte_perm(x2, x3, 0x0051u), 0x5410u);
+            const uint32_t lb = __byte_perm(__byte_perm(x0, x1, 0x0040u), __byte_perm(x2, x3, 0x0040u), 0x5410u);
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(xr + kXGroupBytes * sub + e), "r"(hb) : "memory");
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(xr + kXGroupBytes * sub + 32 + e), "r"(lb) : "memory");
+            if ((lane & 7) == 0) {
+                const float X = static_cast<float>(t) * __int_as_float((127 - sh) << 23);
+                const uint32_t ir = xr + 4 * kXGroupBytes + kXInfoBytes * sub;
+                if constexpr (S16) {
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ir), "r"(__float_as_uint(X)),
+                                 "r"(static_cast<uint32_t>((127 - sh) << 23)), "r"(first), "r"(t - first)
+                                 : "memory");
+                } else {
+                    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(ir), "r"(__float_as_uint(X)),
+                                 "r"(static_cast<uint32_t>((127 - sh) << 23))
                                  : "memory");
                 }
-            } else if (lane == 0) {
-                asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(xr + 4 * kXGroupBytes + kXInfoBytes * k),
-                             "r"(__float_as_uint(X)), "r"(static_cast<uint32_t>((127 - sh) << 23))
-                             : "memory");
             }
         }
     }
