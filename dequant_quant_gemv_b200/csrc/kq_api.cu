@@ -111,7 +111,9 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     if ((fmt == KQ_FMT_Q2_K && nb % 4 != 0) || (fmt == KQ_FMT_Q3_K && nb % 8 != 0))
         return fail(KQ_ERR_UNSUPPORTED, "%s rows must be 16-byte aligned (K %% %d == 0), K=%lld",
                     fmt == KQ_FMT_Q2_K ? "Q2_K" : "Q3_K", fmt == KQ_FMT_Q2_K ? 1024 : 2048, (long long)a.K);
-    if (fmt != KQ_FMT_Q6_K) {  // Q2_K..Q5_K: lanes take (row pair, block, half)
+    if (fmt == KQ_FMT_Q6_K && nb % 8 != 0)
+        return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
+    if (fmt != KQ_FMT_Q6_K || ncol == 1) {  // lanes take (row pair, block, half)
         const int ur = 2 * nb;  // half-block units per row pair
         const int lr = ur <= 32 ? next_pow2(ur) : static_cast<int>(round_up(ur, 32));
         if (lr > kConsumers) return fail(KQ_ERR_UNSUPPORTED, "K=%lld > 32768", (long long)a.K);
@@ -119,9 +121,6 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
         a.ps = kConsumers / lr;
         a.parts = lr > 32 ? lr / 32 : 1;
     } else {
-        if (nb % 8 != 0)
-            return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld",
-                        (long long)a.K);
         const int urw = 2 * (nb / 8);  // units per row pair in each of the 8 warps
         if (urw > 32) return fail(KQ_ERR_UNSUPPORTED, "Q6_K with K=%lld > 32768", (long long)a.K);
         const int lrw = next_pow2(urw);
@@ -138,9 +137,9 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     const int ng = ncol == 1 ? 2 : 1;
     const bool shared_x = a.x_seg_stride == 0;
     const size_t wp_bytes = round_up(sizeof(float) * ng * 2 * a.ps * a.parts * 2 * ncol, 128);
-    // one column (not Q6_K): integer activation regions (2 x 336 bytes per
+    // one column: integer activation regions (2 x 336 bytes per
     // super-block); otherwise fp32 regions
-    const size_t xcopy = ncol == 1 && fmt != KQ_FMT_Q6_K ? static_cast<size_t>(672) * nb
+    const size_t xcopy = ncol == 1 ? static_cast<size_t>(672) * nb
                                                           : sizeof(float) * ncol * 2 * nb * kRegion;
     const size_t xs_bytes = round_up((shared_x ? 1 : ng) * xcopy, 128);
     const size_t head = kHeadBytes;

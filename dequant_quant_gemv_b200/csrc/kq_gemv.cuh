@@ -1009,6 +1009,89 @@ __device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b
     out[1][0] = y[1];
 }
 
+// Q6_K unit, one column, on DP4A: row pair at row0, super-block b (210
+// bytes: ql[128], qh[64], 16 int8 scales, d), half H.  Blocks are 2-byte
+// aligned only and b's parity varies across the lanes, so each stream is
+// loaded from the 4-byte boundary at or below its start, one word more than
+// it needs, and every word rebuilt by a byte permute with a parity-chosen
+// selector (one code path for all lanes; an even block's extra words are
+// its own or its neighbour's bytes, and a row's last block is odd).  Weight
+// 128H + 32t + l: low 4 bits from ql[64H + 32(t%2) + l] (nibble t/2), top 2
+// bits from bits 2t of qh[32H + l]; 16-weight group 2t + l/16 of the half
+// has scale s = scales[8H + 2t + l/16].  Per group the exact
+// S = sum q*xi - 32*(its 16-sum of xi) = sum (q - 32)*xi, |S| <= 2^23, and
+// y = d * sum over groups of s*P*S.
+__device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
+                                             float (&out)[2][1]) {
+    const bool odd = b & 1;
+    const uint32_t sel = odd ? 0x5432u : 0x3210u;
+    uint32_t bw[2], sc[2][2];
+    float dd[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        bw[r] = row0 + r * row_bytes + b * kQ6Bytes - (odd ? 2 : 0);  // 4-byte aligned
+        const uint32_t s0 = ld_s32(bw[r] + 192 + 8 * H), s1 = ld_s32(bw[r] + 196 + 8 * H),
+                       s2 = ld_s32(bw[r] + 200 + 8 * H);
+        sc[r][0] = __byte_perm(s0, s1, sel);
+        sc[r][1] = __byte_perm(s1, s2, sel);
+        dd[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(ld_s32(bw[r] + 208) >> (odd ? 16 : 0))));
+    }
+    float y[2] = {0.f, 0.f};
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        // positions l = 16s .. 16s+15: words of ql (A: t = 0, 2; B: t = 1, 3) and qh
+        uint32_t A[2][4], B[2][4], Hh[2][4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            uint32_t L[5];
+#pragma unroll
+            for (int k = 0; k < 5; ++k) L[k] = ld_s32(bw[r] + 64 * H + 16 * s + 4 * k);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) A[r][m] = __byte_perm(L[m], L[m + 1], sel);
+#pragma unroll
+            for (int k = 0; k < 5; ++k) L[k] = ld_s32(bw[r] + 64 * H + 32 + 16 * s + 4 * k);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) B[r][m] = __byte_perm(L[m], L[m + 1], sel);
+#pragma unroll
+            for (int k = 0; k < 5; ++k) L[k] = ld_s32(bw[r] + 128 + 32 * H + 16 * s + 4 * k);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) Hh[r][m] = __byte_perm(L[m], L[m + 1], sel);
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const uint4 xh = ld_s128(xr + kXGroupBytes * t + 16 * s);
+            const uint4 xl = ld_s128(xr + kXGroupBytes * t + 32 + 16 * s);
+            int hi[2] = {0, 0};
+            uint32_t lo[2] = {0u, 0u};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const uint32_t src = (t & 1) ? B[r][m] : A[r][m];
+                    const uint32_t low = ((t & 2) ? (src >> 4) : src) & 0x0F0F0F0Fu;
+                    const uint32_t top = t == 0 ? (Hh[r][m] << 4) : t == 1 ? (Hh[r][m] << 2)
+                                                      : t == 2 ? Hh[r][m] : (Hh[r][m] >> 2);
+                    const uint32_t q = low | (top & 0x30303030u);
+                    hi[r] = dp4a_us(q, u4w(xh, m), hi[r]);
+                    lo[r] = dp4a_uu(q, u4w(xl, m), lo[r]);
+                }
+            }
+            const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * t);  // X, P, 16-sums
+            const float P = __uint_as_float(info.y);
+            const int x32 = 32 * static_cast<int>(s ? info.w : info.z);
+            const int g = 2 * t + s;  // group within the half
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int S = hi[r] * 256 + static_cast<int>(lo[r]) - x32;
+                const float sv = static_cast<float>(static_cast<int8_t>((sc[r][g >> 2] >> (8 * (g & 3))) & 0xFFu));
+                y[r] = fmaf(sv * P, static_cast<float>(S), y[r]);
+            }
+        }
+    }
+    out[0][0] = y[0] * dd[0];
+    out[1][0] = y[1] * dd[1];
+}
+
 // Dispatch a Q6_K unit to the code path of its alignment class.
 template <int NCOL>
 __device__ __forceinline__ void q6k_unit_dispatch(int kappa, uint32_t row0, int row_bytes, int b, int H,
@@ -1024,7 +1107,7 @@ template <int FMT, int NCOL, bool INT, bool PRO>
 __device__ __forceinline__ void stage_all(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar,
                                           int kb0, int nbl, uint32_t part) {
     if constexpr (INT)
-        stage_x_int<PRO, (FMT == 4 || FMT == 5)>(a, seg, xs, ct >> 5, nthr >> 5, ct & 31, bar, nthr, kb0, nbl, part);
+        stage_x_int<PRO, (FMT == 2 || FMT == 4 || FMT == 5)>(a, seg, xs, ct >> 5, nthr >> 5, ct & 31, bar, nthr, kb0, nbl, part);
     else if constexpr (PRO)
         stage_x_pro<FMT, NCOL>(ProStage{a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256,
                                         a.pro == 1 ? a.gamma + static_cast<int64_t>(kb0) * 256 : nullptr, a.K, a.ldx,
@@ -1103,7 +1186,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     int u_rp, u_b, u_H, group, part;
     bool u_active;
     int kappa = 0;
-    if (FMT != 2) {  // Q4_K and Q5_K: lanes take (row pair, block, half)
+    if (FMT != 2 || NCOL == 1) {  // lanes take (row pair, block, half)
         const int LR = a.lanes_per_rp;
         u_rp = ct / LR;
         const int u = ct - u_rp * LR;
@@ -1128,15 +1211,13 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     // single column with whole row pairs per warp: no cross-warp reduction
     const bool direct = NCOL == 1 && parts == 1;
     int region;
-    if (FMT != 2) region = 2 * u_b + u_H;
+    if (FMT != 2 || NCOL == 1) region = 2 * u_b + u_H;
     else region = ((kappa * (nb >> 3) + (u_b >> 3)) << 1) + u_H;
     const int wp_group = 2 * a.ps * parts * 2 * NCOL;     // floats of one group's double buffer
     // activation copy: fp32 regions (several columns) or the integer groups
-    // of the single-column path (kXGroupBytes + kXInfoBytes per 32 weights)
-    // the integer path serves single-column Q4_K and Q5_K; Q6_K keeps the
-    // fp32 units (measured faster for it twice: 21.0 vs 26.6 and 20.0 vs
-    // 22.4 us on the 8B down matrix)
-    constexpr bool INT = NCOL == 1 && FMT != 2;
+    // of the single-column path (kXGroupBytes + kXInfoBytes per 32 weights),
+    // which serves every format
+    constexpr bool INT = NCOL == 1;
     const uint32_t xcopy = INT ? kXRegionBytes * 2 * nb : 4 * NCOL * xcs;
     const uint32_t xs_s = smem_u32(xs) + (shared_x ? 0 : g * xcopy);
     const uint32_t xri = x_region(xs_s, u_b, u_H);  // this lane's integer region (Q4_K)
@@ -1185,6 +1266,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
                 q2k_unit_int(row0, srow, u_b, u_H, xri, out);
             } else if constexpr (INT && FMT == 5) {
                 q3k_unit_int(row0, srow, u_b, u_H, xri, out);
+            } else if constexpr (INT) {
+                q6k_unit_int(row0, srow, u_b, u_H, xri, out);
             } else if constexpr (FMT == 1) {
                 q4k_unit<NCOL>(row0, srow, u_b, u_H, xr, xcs, out);
             } else {

@@ -140,7 +140,6 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
     const int ct_all = tid - 32;               // 0 .. NG*256-1
     const int g = NG == 2 ? (ct_all >> 8) : 0;
     const int ct = ct_all & (kConsumers - 1);  // thread within the group
-    const int cw = ct >> 5;                    // warp within the group
     const int gbar = 1 + g;                    // the group's named barrier
     const int nthr = NG * kConsumers;          // all consumer threads (named barrier 3)
     const uint32_t xs_s = smem_u32(smem + A.xs_offset);
@@ -181,49 +180,27 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
         // this step's activations, staged by all consumer threads
         const GemvArgs a = step_view(s);
         float rinv = 1.f;
-        if (s.fmt == 4 || s.fmt == 5) {  // Q2_K and Q3_K: integer regions with 16-sums
-            if (s.pro) stage_all<4, 1, true, true>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
-            else stage_all<4, 1, true, false>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
-        } else if (s.fmt != 2) {  // Q4_K and Q5_K: integer regions
+        if (s.fmt != 1 && s.fmt != 3) {  // Q2_K, Q3_K, Q6_K: integer regions with 16-sums
+            if (s.pro) stage_all<2, 1, true, true>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
+            else stage_all<2, 1, true, false>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
+        } else {  // Q4_K and Q5_K: integer regions
             if (s.pro) stage_all<1, 1, true, true>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
             else stage_all<1, 1, true, false>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
-        } else {
-            if (s.pro) stage_all<2, 1, false, true>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
-            else stage_all<2, 1, false, false>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
         }
         if (s.pro == 1) rinv = ld_s32f(pro_inv_addr(pro_r));
 
         // this lane's unit within a stage (as in the single-column kernel)
         const int nb = s.nb;
-        const int xcs = 2 * nb * kRegion;
-        int u_rp, u_b, u_H, group, part;
-        bool u_active;
-        int kappa = 0;
-        if (s.fmt != 2) {
-            const int LR = s.lanes_per_rp;
-            u_rp = ct / LR;
-            const int u = ct - u_rp * LR;
-            u_active = u < 2 * nb;
-            u_b = u >> 1;
-            u_H = u & 1;
-            group = LR < 32 ? LR : 32;
-            part = LR > 32 ? (u >> 5) : 0;
-        } else {
-            const int LRw = s.lanes_per_rp;
-            kappa = cw;
-            u_rp = lane / LRw;
-            const int u = lane - u_rp * LRw;
-            u_active = u < 2 * (nb >> 3);
-            u_b = 8 * (u >> 1) + kappa;
-            u_H = u & 1;
-            group = LRw;
-            part = kappa;
-        }
+        const int LR = s.lanes_per_rp;
+        const int u_rp = ct / LR;
+        const int u = ct - u_rp * LR;
+        const bool u_active = u < 2 * nb;
+        const int u_b = u >> 1, u_H = u & 1;
+        const int group = LR < 32 ? LR : 32;
+        const int part = LR > 32 ? (u >> 5) : 0;
         const int parts = s.parts;
         const bool direct = parts == 1;
-        const int region = s.fmt != 2 ? 2 * u_b + u_H : ((kappa * (nb >> 3) + (u_b >> 3)) << 1) + u_H;
         const uint32_t xri = x_region(xs_s, u_b, u_H);
-        const uint32_t xr = xs_s + 4 * (region * kRegion);
         const uint32_t wp_s = smem_u32(smem + A.wp_offset) + 4 * g * (2 * s.ps * parts * 2);
         const int srow = static_cast<int>(s.row_bytes);
 
@@ -246,7 +223,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
                 else if (s.fmt == 3) q5k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else if (s.fmt == 4) q2k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else if (s.fmt == 5) q3k_unit_int(rw, srow, u_b, u_H, xri, out);
-                else q6k_unit_dispatch<1>(kappa, rw, srow, u_b, u_H, xr, xcs, out);
+                else q6k_unit_int(rw, srow, u_b, u_H, xri, out);
             }
             // butterfly over the lanes of this row pair (fixed order)
 #pragma unroll

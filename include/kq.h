@@ -56,9 +56,9 @@
  *    return value reports argument validation and launch errors only
  *    (KQ_ERR_CUDA carries cudaGetLastError()); kq_last_error() gives text.
  *  - Arithmetic: quants are unpacked exactly; sums are fp32 (or exact
- *    integers).  Single-column Q2_K..Q5_K round each activation to a 14-bit
+ *    integers).  A single column rounds each activation to a 14-bit
  *    integer on a power-of-two grid per group of 32 (error at most 2^-14 of
- *    the group's largest |x|); single-column Q6_K multiplies in fp32; two or
+ *    the group's largest |x|), every format alike; two or
  *    more columns of Q4_K..Q6_K run on the tensor cores with exact fp16 weight operands and
  *    activations split into two fp16 terms (22 bits) after a power-of-two
  *    scale per super-block; several columns of Q2_K and Q3_K run one

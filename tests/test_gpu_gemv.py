@@ -332,9 +332,9 @@ def test_invalid_arguments_are_rejected():
 
 
 # ------------------------------------------- single-column integer path
-@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q2_k", "q3_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q2_k", "q3_k", "q6_k"])
 def test_single_column_within_activation_rounding_bound(fmt):
-    """Single-column Q2_K..Q5_K round each activation to a 14-bit integer
+    """A single column (every format) rounds each activation to a 14-bit integer
     on a power-of-two grid per group of 32, so |x - x'| <= 2^-14 * (largest
     |x| of the group).  The error must stay within that bound (plus fp32
     rounding slack), computed from the oracle's dequantised weights."""
