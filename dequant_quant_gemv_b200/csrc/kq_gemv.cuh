@@ -676,7 +676,7 @@ __device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H) {
 template <bool PRO, bool S16 = false>
 __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, int warp, int nwarps, int lane,
                                    int bar, int nthr, int kb0, int nbl, uint32_t part) {
-    constexpr int U = 2;  // one round of loads for K = 4096 and 16 warps
+    constexpr int U = PRO ? 4 : 8;  // one round of loads for K up to 16384 (8 with a prologue) and 16 warps
     const float* xg = a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256;
     const int quads = 2 * nbl;  // passes of 4 groups (128 activations)
     const bool rms = PRO && a.pro == 1;
@@ -796,7 +796,8 @@ __device__ __forceinline__ void q4k_unit_int(uint32_t row0, int row_bytes, int b
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
                     const uint32_t w = u4w(r ? q1 : q0, t);
-                    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+                    // high nibbles in place: 16*q, the 1/16 folded into the scale
+                    const uint32_t lo = w & 0x0F0F0F0Fu, hi = w & 0xF0F0F0F0u;
                     hL[r] = dp4a_us(lo, u4w(xhL, t), hL[r]);
                     lL[r] = dp4a_uu(lo, u4w(xlL, t), lL[r]);
                     hH[r] = dp4a_us(hi, u4w(xhH, t), hH[r]);
@@ -812,7 +813,7 @@ __device__ __forceinline__ void q4k_unit_int(uint32_t row0, int row_bytes, int b
             const float sH = static_cast<float>(hH[r] * 256 + static_cast<int>(lH[r]));
             y[r] = fmaf(dd[r] * byte_f(sc4[r], 2 * cc) * iL.y, sL, y[r]);
             y[r] = fmaf(-dm[r] * byte_f(m4[r], 2 * cc), iL.x, y[r]);
-            y[r] = fmaf(dd[r] * byte_f(sc4[r], 2 * cc + 1) * iH.y, sH, y[r]);
+            y[r] = fmaf(dd[r] * byte_f(sc4[r], 2 * cc + 1) * (iH.y * 0.0625f), sH, y[r]);
             y[r] = fmaf(-dm[r] * byte_f(m4[r], 2 * cc + 1), iH.x, y[r]);
         }
     }
@@ -883,8 +884,9 @@ __device__ __forceinline__ void q5k_unit_int(uint32_t row0, int row_bytes, int b
 // Q2_K unit, one column, on DP4A: row pair at row0, super-block b (84
 // bytes: 16 scale|min bytes, 64 quant bytes, d, dmin; 4-byte aligned), half
 // H.  Weight 128H + 32j + l is bits 2j of quant byte 32H + l, in 16-weight
-// group 8H + 2j + l/16.  Per group the exact S = sum q*xi, then
-// y += d*sc*P*S - dmin*m*P*(the group's 16-sum of xi).
+// group 8H + 2j + l/16.  The codes of plane j are used in place (4^j * q,
+// no shift), the 4^-j folded into the group's factor.  Per group the exact
+// S = sum q*xi, then y += d*sc*P*S - dmin*m*P*(the group's 16-sum of xi).
 __device__ __forceinline__ void q2k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
                                              float (&out)[2][1]) {
     uint32_t Q[2][8], sw[2][2];
@@ -905,6 +907,7 @@ __device__ __forceinline__ void q2k_unit_int(uint32_t row0, int row_bytes, int b
     for (int j = 0; j < 4; ++j) {
         const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * j);  // X, P, 16-sums
         const float P = __uint_as_float(info.y);
+        const float Pj = P * (1.0f / static_cast<float>(1 << (2 * j)));  // undoes the 4^j of the in-place codes
 #pragma unroll
         for (int sh = 0; sh < 2; ++sh) {
             const uint4 xh = ld_s128(xr + kXGroupBytes * j + 16 * sh);
@@ -915,7 +918,7 @@ __device__ __forceinline__ void q2k_unit_int(uint32_t row0, int row_bytes, int b
             for (int m = 0; m < 4; ++m) {
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
-                    const uint32_t q = (Q[r][4 * sh + m] >> (2 * j)) & 0x03030303u;
+                    const uint32_t q = Q[r][4 * sh + m] & (0x03030303u << (2 * j));  // 4^j * q
                     hi[r] = dp4a_us(q, u4w(xh, m), hi[r]);
                     lo[r] = dp4a_uu(q, u4w(xl, m), lo[r]);
                 }
@@ -926,7 +929,7 @@ __device__ __forceinline__ void q2k_unit_int(uint32_t row0, int row_bytes, int b
             for (int r = 0; r < 2; ++r) {
                 const uint32_t sb = (sw[r][g >> 2] >> (8 * (g & 3))) & 0xFFu;
                 const float S = static_cast<float>(hi[r] * 256 + static_cast<int>(lo[r]));
-                y[r] = fmaf(dd[r] * static_cast<float>(sb & 15u) * P, S, y[r]);
+                y[r] = fmaf(dd[r] * static_cast<float>(sb & 15u) * Pj, S, y[r]);
                 y[r] = fmaf(-dm[r] * static_cast<float>(sb >> 4), x16, y[r]);
             }
         }
@@ -942,8 +945,9 @@ __device__ __forceinline__ void q2k_unit_int(uint32_t row0, int row_bytes, int b
 // its start (one word more than it needs) and every word rebuilt by a byte
 // permute whose selector is picked by b's parity.  Weight 128H + 32j + l:
 // q + 4 = (bits 2j of quant byte 32H + l) | (bit 4H + j of hmask[l]) << 2,
-// in 0..7; per 16-weight group the exact S = sum (q+4)*xi - 4*(16-sum of xi)
-// and y += d*(v - 32)*P*S with v the group's 6-bit scale.
+// in 0..7, assembled in place as 4^j * (q + 4) (the 4^-j folded into the
+// group's factor); per 16-weight group the exact S = sum (q+4)*xi -
+// 4*(16-sum of xi) and y += d*(v - 32)*P*S with v the group's 6-bit scale.
 __device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
                                              float (&out)[2][1]) {
     const bool odd = b & 1;
@@ -975,7 +979,8 @@ __device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * j);  // X, P, 16-sums
-        const float P = __uint_as_float(info.y);
+        const int jj = j < 3 ? j : 2;  // the plane's codes sit at bits 2jj..2jj+2
+        const float Pj = __uint_as_float(info.y) * (1.0f / static_cast<float>(1 << (2 * jj)));
 #pragma unroll
         for (int sh = 0; sh < 2; ++sh) {
             const uint4 xh = ld_s128(xr + kXGroupBytes * j + 16 * sh);
@@ -987,13 +992,18 @@ __device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
                     const int t = 4 * sh + m;
-                    const uint32_t q = ((Q[r][t] >> (2 * j)) & 0x03030303u) |
-                                       (((M[r][t] >> (4 * H + j)) & 0x01010101u) << 2);
+                    // 4^jj * (q + 4): the low bits in place (plane 3 moved down to
+                    // plane 2's bits, so that the three bits fit a byte), the third
+                    // bit rotated next to them (a rotation keeps each byte's bit
+                    // 4H + j inside its byte)
+                    const uint32_t lowb = j < 3 ? Q[r][t] : Q[r][t] >> 2;
+                    const uint32_t hb = __funnelshift_l(M[r][t], M[r][t], (2 * jj + 2 - 4 * H - j) & 31);
+                    const uint32_t q = (lowb & (0x03030303u << (2 * jj))) | (hb & (0x04040404u << (2 * jj)));
                     hi[r] = dp4a_us(q, u4w(xh, m), hi[r]);
                     lo[r] = dp4a_uu(q, u4w(xl, m), lo[r]);
                 }
             }
-            const int x16 = static_cast<int>(sh ? info.w : info.z);
+            const int x16 = static_cast<int>(sh ? info.w : info.z) << (2 * jj);
             const int g = 2 * j + sh;  // group within the half
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
@@ -1001,7 +1011,7 @@ __device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b
                 const uint32_t hi2 = (hs[r] >> (8 * (g & 3) + 2 * (g >> 2))) & 3u;
                 const float v = static_cast<float>(static_cast<int>(lo4 | (hi2 << 4)) - 32);
                 const int S = hi[r] * 256 + static_cast<int>(lo[r]) - 4 * x16;
-                y[r] = fmaf(dd[r] * v * P, static_cast<float>(S), y[r]);
+                y[r] = fmaf(dd[r] * v * Pj, static_cast<float>(S), y[r]);
             }
         }
     }
