@@ -366,6 +366,7 @@ __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empt
                                uint8_t* sbuf, int64_t rp_begin, int64_t rp_end, int64_t rps, int ns, int kb0,
                                int nbl, int srow, bool contiguous) {
     if (a.ids) pdl_wait();  // routed ids may come from the previous grid
+    const uint64_t pol = l2_evict_first();
     StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
     Stage st;
     bool ok = true;
@@ -385,14 +386,14 @@ __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empt
             if (contiguous) {
                 const uint32_t bytes = static_cast<uint32_t>(st.nrows * a.row_bytes);
                 mbar_arrive_expect_tx(&full[slot], bytes);
-                bulk_g2s(dst, src, bytes, &full[slot]);
+                bulk_g2s(dst, src, bytes, &full[slot], pol);
             } else {
                 const int64_t off = static_cast<int64_t>(kb0) * BS;
                 const int64_t off16 = off & ~int64_t(15);
                 const uint32_t rbytes = static_cast<uint32_t>((off + nbl * BS - off16 + 15) & ~int64_t(15));
                 mbar_arrive_expect_tx(&full[slot], rbytes * st.nrows);
                 for (int i = 0; i < st.nrows; ++i)
-                    bulk_g2s(dst + i * srow, src + i * a.row_bytes + off16, rbytes, &full[slot]);
+                    bulk_g2s(dst + i * srow, src + i * a.row_bytes + off16, rbytes, &full[slot], pol);
             }
         } else {
             mbar_arrive(&full[slot]);
@@ -708,45 +709,73 @@ __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, 
                 }
             }
         }
+        // the passes advance two at a time in lockstep (a pair past the end
+        // is skipped; a pass past the end inside a pair works on zeros and
+        // stores nothing), so that their shuffle and conversion latencies
+        // overlap
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int Q = base + nwarps * u;
-            if (Q >= quads) break;  // warp-uniform
-            float m = fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w)));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-            const uint32_t mb = __float_as_uint(m);
-            int sh = 0;
-            if (mb != 0u) {
-                sh = 13 - (static_cast<int>(mb >> 23) - 127);
-                sh = sh > 100 ? 100 : sh < -100 ? -100 : sh;
+        for (int c = 0; c < U; c += 2) {
+            if (base + nwarps * c >= quads) break;  // warp-uniform
+            float m[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const float4 w4 = v[c + u];
+                m[u] = fmaxf(fmaxf(fabsf(w4.x), fabsf(w4.y)), fmaxf(fabsf(w4.z), fabsf(w4.w)));
             }
-            const float sc = __int_as_float((sh + 127) << 23);
-            const int x0 = __float2int_rn(v[u].x * sc), x1 = __float2int_rn(v[u].y * sc);
-            const int x2 = __float2int_rn(v[u].z * sc), x3 = __float2int_rn(v[u].w * sc);
-            int t = (x0 + x1) + (x2 + x3);
-            t += __shfl_xor_sync(0xffffffffu, t, 1);
-            t += __shfl_xor_sync(0xffffffffu, t, 2);
-            const int first = t;  // on lanes 0..3 of the group: its first 16
-            t += __shfl_xor_sync(0xffffffffu, t, 4);
-            const uint32_t xr = x_region(xs, Q >> 1, Q & 1);
-            // byte 1 of each xi (the signed high byte), then byte 0
-            const uint32_t hb = __byte_perm(__byte_perm(x0, x1, 0x0051u), __byte_perm(x2, x3, 0x0051u), 0x5410u);
-            const uint32_t lb = __byte_perm(__byte_perm(x0, x1, 0x0040u), __byte_perm(x2, x3, 0x0040u), 0x5410u);
-            asm volatile("st.shared.u32 [%0], %1;" ::"r"(xr + kXGroupBytes * sub + e), "r"(hb) : "memory");
-            asm volatile("st.shared.u32 [%0], %1;" ::"r"(xr + kXGroupBytes * sub + 32 + e), "r"(lb) : "memory");
-            if ((lane & 7) == 0) {
-                const float X = static_cast<float>(t) * __int_as_float((127 - sh) << 23);
-                const uint32_t ir = xr + 4 * kXGroupBytes + kXInfoBytes * sub;
-                if constexpr (S16) {
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ir), "r"(__float_as_uint(X)),
-                                 "r"(static_cast<uint32_t>((127 - sh) << 23)), "r"(first), "r"(t - first)
-                                 : "memory");
-                } else {
-                    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(ir), "r"(__float_as_uint(X)),
-                                 "r"(static_cast<uint32_t>((127 - sh) << 23))
-                                 : "memory");
+#pragma unroll
+            for (int off = 1; off <= 4; off <<= 1)
+#pragma unroll
+                for (int u = 0; u < 2; ++u) m[u] = fmaxf(m[u], __shfl_xor_sync(0xffffffffu, m[u], off));
+            int sh[2], t[2], first[2];
+            uint32_t hb[2], lb[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t mb = __float_as_uint(m[u]);
+                int ex = 0;
+                if (mb != 0u) {
+                    ex = 13 - (static_cast<int>(mb >> 23) - 127);
+                    ex = ex > 100 ? 100 : ex < -100 ? -100 : ex;
+                }
+                sh[u] = ex;
+                const float sc = __int_as_float((ex + 127) << 23);
+                const float4 w4 = v[c + u];
+                const int x0 = __float2int_rn(w4.x * sc), x1 = __float2int_rn(w4.y * sc);
+                const int x2 = __float2int_rn(w4.z * sc), x3 = __float2int_rn(w4.w * sc);
+                t[u] = (x0 + x1) + (x2 + x3);
+                // byte 1 of each xi (the signed high byte), then byte 0
+                hb[u] = __byte_perm(__byte_perm(x0, x1, 0x0051u), __byte_perm(x2, x3, 0x0051u), 0x5410u);
+                lb[u] = __byte_perm(__byte_perm(x0, x1, 0x0040u), __byte_perm(x2, x3, 0x0040u), 0x5410u);
+            }
+#pragma unroll
+            for (int off = 1; off <= 4; off <<= 1) {
+#pragma unroll
+                for (int u = 0; u < 2; ++u) t[u] += __shfl_xor_sync(0xffffffffu, t[u], off);
+                if (off == 2) {
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) first[u] = t[u];  // on lanes 0..3 of a group: its first 16
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int Q = base + nwarps * (c + u);
+                if (Q >= quads) break;  // warp-uniform
+                const uint32_t xr = x_region(xs, Q >> 1, Q & 1);
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(xr + kXGroupBytes * sub + e), "r"(hb[u]) : "memory");
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(xr + kXGroupBytes * sub + 32 + e), "r"(lb[u])
+                             : "memory");
+                if ((lane & 7) == 0) {
+                    const float X = static_cast<float>(t[u]) * __int_as_float((127 - sh[u]) << 23);
+                    const uint32_t ir = xr + 4 * kXGroupBytes + kXInfoBytes * sub;
+                    if constexpr (S16) {
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ir), "r"(__float_as_uint(X)),
+                                     "r"(static_cast<uint32_t>((127 - sh[u]) << 23)), "r"(first[u]),
+                                     "r"(t[u] - first[u])
+                                     : "memory");
+                    } else {
+                        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(ir), "r"(__float_as_uint(X)),
+                                     "r"(static_cast<uint32_t>((127 - sh[u]) << 23))
+                                     : "memory");
+                    }
                 }
             }
         }

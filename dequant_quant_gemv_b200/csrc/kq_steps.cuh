@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
     if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
+            const uint64_t pol = l2_evict_first();
             int slot = -1, count = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
                     const uint32_t bytes = static_cast<uint32_t>(rows * s.row_bytes);
                     mbar_arrive_expect_tx(&full[slot], bytes);
                     bulk_g2s(sbuf + static_cast<size_t>(slot) * A.slot_bytes, s.W + row0 * s.row_bytes, bytes,
-                             &full[slot]);
+                             &full[slot], pol);
                 }
             }
             // let every copy issued land before the CTA can exit
