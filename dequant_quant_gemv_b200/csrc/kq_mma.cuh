@@ -161,17 +161,16 @@ __device__ __forceinline__ void b_slot(int w, int& s, int& q) {
 // (column, block) is scaled by its own power of two 2^sh (largest |x| of
 // the block into [2^14, 2^15)) and its sums by 2^(sh-5); `bscale` gets
 // (2^-sh, 2^(5-sh)) per block and column.  Columns >= ncol_real are zero.
-// One warp per (column, block) item, two float4 per lane, several items'
-// loads in flight.  PRO: with the prologue a.pro, its second operand
+// One warp per (column, block) item, two float4 per lane, U items' loads in
+// flight.  PRO: with the prologue a.pro, its second operand
 // (gamma, or u) loaded beside x; for RMSNorm each item's sum of squares of
 // the raw x (block_sq) goes to part[col][kb0 + bl] (a.nb per column), and
 // with `publish` (a cluster) each storing lane also releases it at cluster
 // scope.
-template <int FMT, int NT, bool PRO>
+template <int FMT, int NT, bool PRO, int U>
 __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, int nwarps, int lane, int bar,
                          int kb0, int nbl, uint32_t part, bool publish) {
     constexpr int NC = 4 * NT;
-    constexpr int U = 4;  // items per warp in flight
     const float* xg = a.x + static_cast<int64_t>(kb0) * 256;
     const int kr = a.ncol_real;
     const int items = NC * nbl;
@@ -222,36 +221,68 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                 }
             }
         }
+        // items advance two at a time in lockstep (a pair past the end is
+        // skipped; an item past the end inside a pair stores nothing), so
+        // that their shuffle latencies overlap
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int it = base + nwarps * u;
-            if (it >= items) break;  // warp-uniform
-            const int col = it / nbl, bl = it - col * nbl;
-            float m = 0.f;
+        for (int c = 0; c < U; c += 2) {
+            if (base + nwarps * c >= items) break;  // warp-uniform
+            float m[2];
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-                m = fmaxf(m, fmaxf(fmaxf(fabsf(v[u][h].x), fabsf(v[u][h].y)), fmaxf(fabsf(v[u][h].z), fabsf(v[u][h].w))));
+            for (int u2 = 0; u2 < 2; ++u2) {
+                m[u2] = 0.f;
 #pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            const int sh = col_shift(__float_as_uint(m));
-            const float sc = pow2f(sh), scm = pow2f(sh - 5);
+                for (int h = 0; h < 2; ++h) {
+                    const float4 t = v[c + u2][h];
+                    m[u2] = fmaxf(m[u2], fmaxf(fmaxf(fabsf(t.x), fabsf(t.y)), fmaxf(fabsf(t.z), fabsf(t.w))));
+                }
+            }
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float4 t = make_float4(v[u][h].x * sc, v[u][h].y * sc, v[u][h].z * sc, v[u][h].w * sc);
-                int st, sq;
-                b_slot<FMT>(128 * h + 4 * lane, st, sq);
-                store_b_entry<FMT, NT>(xb, bl, st, sq, col, t);
-                if constexpr (FMT == 2) continue;
-                // sub-block 4h + lane/8: the 8 lanes of this group, fixed order
-                float X = (v[u][h].x + v[u][h].y) + (v[u][h].z + v[u][h].w);
-                X += __shfl_xor_sync(0xffffffffu, X, 1);
-                X += __shfl_xor_sync(0xffffffffu, X, 2);
-                X += __shfl_xor_sync(0xffffffffu, X, 4);
-                if ((lane & 7) == 0) {
+            for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+                for (int u2 = 0; u2 < 2; ++u2) m[u2] = fmaxf(m[u2], __shfl_xor_sync(0xffffffffu, m[u2], off));
+            float X[2][2];
+#pragma unroll
+            for (int u2 = 0; u2 < 2; ++u2) {
+                const int it = base + nwarps * (c + u2);
+                const bool valid = it < items;  // warp-uniform
+                const int col = it / nbl, bl = it - col * nbl;
+                const int sh = col_shift(__float_as_uint(m[u2]));
+                const float sc = pow2f(sh);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float4 t = make_float4(v[c + u2][h].x * sc, v[c + u2][h].y * sc, v[c + u2][h].z * sc,
+                                                 v[c + u2][h].w * sc);
+                    int st, sq;
+                    b_slot<FMT>(128 * h + 4 * lane, st, sq);
+                    if (valid) store_b_entry<FMT, NT>(xb, bl, st, sq, col, t);
+                    X[u2][h] = (v[c + u2][h].x + v[c + u2][h].y) + (v[c + u2][h].z + v[c + u2][h].w);
+                }
+                if (valid && lane == 0) {
+                    bscale[2 * (bl * NC + col)] = pow2f(-sh);
+                    bscale[2 * (bl * NC + col) + 1] = pow2f(5 - sh);
+                }
+            }
+            if constexpr (FMT == 2) continue;
+            // sub-block 4h + lane/8: the 8 lanes of its group, fixed order
+#pragma unroll
+            for (int off = 1; off <= 4; off <<= 1)
+#pragma unroll
+                for (int u2 = 0; u2 < 2; ++u2)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) X[u2][h] += __shfl_xor_sync(0xffffffffu, X[u2][h], off);
+#pragma unroll
+            for (int u2 = 0; u2 < 2; ++u2) {
+                const int it = base + nwarps * (c + u2);
+                if (it >= items || (lane & 7) != 0) continue;
+                const int col = it / nbl, bl = it - col * nbl;
+                const float scm = pow2f(col_shift(__float_as_uint(m[u2])) - 5);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
                     const int j = 4 * h + (lane >> 3);
-                    X *= scm;
-                    const __half xh = __float2half_rn(X);
-                    const __half xl = __float2half_rn(X - __half2float(xh));
+                    const float Xs = X[u2][h] * scm;
+                    const __half xh = __float2half_rn(Xs);
+                    const __half xl = __float2half_rn(Xs - __half2float(xh));
                     const int nt = col >> 2, gh = 2 * (col & 3), q = j >> 1;
                     const uint32_t step =
                         xb + 8u * static_cast<uint32_t>(((bl * mma_steps<FMT>() + 16) * 32) * NT + nt);
@@ -263,10 +294,6 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                         st_s32u(el + 4, 0u);
                     }
                 }
-            }
-            if (lane == 0) {
-                bscale[2 * (bl * NC + col)] = pow2f(-sh);
-                bscale[2 * (bl * NC + col) + 1] = pow2f(5 - sh);
             }
         }
     }
@@ -682,7 +709,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
         // RMSNorm scratch: partial sums of squares [column][super-block], then
         // the columns' 1/rms
         const uint32_t pro_s = smem_u32(smem + a.pro_offset), pro_inv = pro_s + 4u * 8 * a.nb;
-        stage_xb<FMT, NT, PRO>(a, xb_s, bscale, ct_all >> 5, NG * kConsumerWarps, lane, 3, kb0, nbl, pro_s, cl);
+        stage_xb<FMT, NT, PRO, (PRO || NG == 2) ? 4 : 8>(a, xb_s, bscale, ct_all >> 5, NG * kConsumerWarps, lane, 3, kb0, nbl, pro_s, cl);
         if constexpr (PRO) {
             if (a.pro == 1) {
                 // each CTA of a cluster has its own blocks' sums: tell the
