@@ -4,7 +4,8 @@ arithmetic).
 
 The C source ``kqgen.c`` draws logical values with a counter-based
 SplitMix64 stream and encodes them into the GGUF K-quant super-block layout
-(Q2_K: 84 bytes, Q3_K: 110, Q4_K: 144, Q5_K: 176, Q6_K: 210; 256 weights each).  This wrapper builds it
+(Q2_K: 84 bytes, Q3_K: 110, Q4_K: 144, Q5_K: 176, Q6_K: 210; 256 weights each;
+Q8_0 in units of eight 34-byte blocks, 272 bytes per 256 weights).  This wrapper builds it
 with gcc on first use and returns numpy arrays.
 """
 from __future__ import annotations
@@ -25,6 +26,7 @@ Q5_K_BLOCK_BYTES = 176
 Q2_K_BLOCK_BYTES = 84
 Q3_K_BLOCK_BYTES = 110
 Q6_K_BLOCK_BYTES = 210
+Q8_0_UNIT_BYTES = 272  # eight 34-byte Q8_0 blocks: 256 weights
 QK = 256  # weights per super-block
 
 
@@ -64,6 +66,9 @@ def _load():
         lib.kqg_q6k_draw.argtypes = [u64, i64, vp, vp, vp]
         lib.kqg_q6k_pack.argtypes = [i64, vp, vp, vp, vp]
         lib.kqg_q6k_fill.argtypes = [u64, i64, i64, vp, i32]
+        lib.kqg_q80_draw.argtypes = [u64, i64, vp, vp]
+        lib.kqg_q80_pack.argtypes = [i64, vp, vp, vp]
+        lib.kqg_q80_fill.argtypes = [u64, i64, i64, vp, i32]
         lib.kqg_normal_f32.argtypes = [u64, i64, vp, i32]
         lib.kqg_topk_ids.restype = i32
         lib.kqg_topk_ids.argtypes = [u64, i32, i32, vp]
@@ -97,7 +102,7 @@ def f16_bits(v: float) -> int:
 
 def block_bytes(fmt: str) -> int:
     return {"q4_k": Q4_K_BLOCK_BYTES, "q5_k": Q5_K_BLOCK_BYTES, "q6_k": Q6_K_BLOCK_BYTES, "q2_k": Q2_K_BLOCK_BYTES,
-            "q3_k": Q3_K_BLOCK_BYTES}[fmt]
+            "q3_k": Q3_K_BLOCK_BYTES, "q8_0": Q8_0_UNIT_BYTES}[fmt]
 
 
 def row_bytes(fmt: str, K: int) -> int:
@@ -271,6 +276,35 @@ def q6k_fill(key: int, nblocks: int, out: np.ndarray | None = None, b0: int = 0,
     return out
 
 
+# ----------------------------------------------------------------- Q8_0
+def q80_draw(key: int, nunits: int) -> dict:
+    """Logical values of Q8_0 data in units of 8 blocks (256 weights): q
+    (nu,256) int8 over -128..127, d (nu,8) fp16 bit patterns (one per block
+    of 32)."""
+    q = np.empty((nunits, 256), np.int8)
+    d = np.empty((nunits, 8), np.uint16)
+    _load().kqg_q80_draw(key, nunits, _ptr(q), _ptr(d))
+    return dict(q=q, d=d)
+
+
+def q80_pack(q, d) -> np.ndarray:
+    q = np.ascontiguousarray(q, np.int8).reshape(-1, 256)
+    nu = q.shape[0]
+    d = np.ascontiguousarray(d, np.uint16).reshape(nu, 8)
+    out = np.empty(nu * Q8_0_UNIT_BYTES, np.uint8)
+    _load().kqg_q80_pack(nu, _ptr(q), _ptr(d), _ptr(out))
+    return out
+
+
+def q80_fill(key: int, nunits: int, out: np.ndarray | None = None, b0: int = 0,
+             nthreads: int | None = None) -> np.ndarray:
+    if out is None:
+        out = np.empty(nunits * Q8_0_UNIT_BYTES, np.uint8)
+    assert out.nbytes >= nunits * Q8_0_UNIT_BYTES and out.dtype == np.uint8
+    _load().kqg_q80_fill(key, b0, nunits, _ptr(out), nthreads or default_threads())
+    return out
+
+
 def fill(fmt: str, key: int, nblocks: int, out: np.ndarray | None = None,
          nthreads: int | None = None) -> np.ndarray:
     if fmt == "q4_k":
@@ -283,6 +317,8 @@ def fill(fmt: str, key: int, nblocks: int, out: np.ndarray | None = None,
         return q3k_fill(key, nblocks, out, nthreads=nthreads)
     if fmt == "q6_k":
         return q6k_fill(key, nblocks, out, nthreads=nthreads)
+    if fmt == "q8_0":
+        return q80_fill(key, nblocks, out, nthreads=nthreads)
     raise ValueError(fmt)
 
 

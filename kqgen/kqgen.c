@@ -51,6 +51,10 @@
  *     of scale byte j (j<8) or the high nibble of byte j-8 (j>=8), its top
  *     2 bits are bits 2(j/4)..2(j/4)+1 of byte 8 + j%4.  The fill draws the
  *     values uniform over -4..3, v_j over 0..63, d as Q4_K.
+ *   Q8_0, 34 B per 32 weights: [0,2) d fp16 | [2,34) 32 int8 quants;
+ *     w = d*q.  Handled in units of 8 blocks (256 weights, 272 B), like the
+ *     super-blocks of the K-quants.  The fill draws quants uniform over the
+ *     whole int8 range -128..127 and d as Q4_K.
  *   Q6_K, 210 B: [0,128) ql | [128,192) qh | [192,208) int8 scales |
  *                [208,210) d fp16.
  *     Half h (0..1) covers weights 128h..128h+127.  For l<32 and t<4, weight
@@ -425,6 +429,51 @@ void kqg_q6k_fill(uint64_t key, int64_t b0, int64_t nblocks, uint8_t* out, int n
         uint16_t d;
         kqg_q6k_draw_block(key, (uint64_t)(b0 + b), q, s, &d);
         kqg_q6k_pack_block(q, s, d, out + 210 * b);
+    }
+}
+
+/* ---------------------------------------------------------------- Q8_0 */
+
+/* One unit of 8 blocks: q the 256 int8 quants, d the 8 fp16 block scales. */
+static void kqg_q80_draw_unit(uint64_t key, uint64_t u, int8_t q[256], uint16_t d[8]) {
+    const uint64_t base = u * 40;
+    for (int k = 0; k < 32; ++k) {
+        uint64_t r = kqg_draw(key, base + k);
+        for (int i = 0; i < 8; ++i) q[8 * k + i] = (int8_t)(uint8_t)((r >> (8 * i)) & 0xFF);
+    }
+    for (int j = 0; j < 8; j += 2) {
+        double z0, z1;
+        kqg_box_muller(key, base + 32 + j, &z0, &z1);
+        d[j] = kqg_f16_bits(fabs(z0) * 1e-3);
+        d[j + 1] = kqg_f16_bits(fabs(z1) * 1e-3);
+    }
+}
+
+static void kqg_q80_pack_unit(const int8_t q[256], const uint16_t d[8], uint8_t* out) {
+    for (int j = 0; j < 8; ++j) {
+        uint8_t* blk = out + 34 * j;
+        blk[0] = (uint8_t)(d[j] & 0xFF);
+        blk[1] = (uint8_t)(d[j] >> 8);
+        for (int i = 0; i < 32; ++i) blk[2 + i] = (uint8_t)q[32 * j + i];
+    }
+}
+
+void kqg_q80_draw(uint64_t key, int64_t nunits, int8_t* q, uint16_t* d) {
+    for (int64_t u = 0; u < nunits; ++u) kqg_q80_draw_unit(key, (uint64_t)u, q + 256 * u, d + 8 * u);
+}
+
+void kqg_q80_pack(int64_t nunits, const int8_t* q, const uint16_t* d, uint8_t* out) {
+    for (int64_t u = 0; u < nunits; ++u) kqg_q80_pack_unit(q + 256 * u, d + 8 * u, out + 272 * u);
+}
+
+void kqg_q80_fill(uint64_t key, int64_t u0, int64_t nunits, uint8_t* out, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int64_t u = 0; u < nunits; ++u) {
+        int8_t q[256];
+        uint16_t d[8];
+        kqg_q80_draw_unit(key, (uint64_t)(u0 + u), q, d);
+        kqg_q80_pack_unit(q, d, out + 272 * u);
     }
 }
 

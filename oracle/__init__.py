@@ -34,9 +34,10 @@ _SRC = os.path.join(_HERE, "kq_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "libkq_oracle.so")
 _lib = None
 
-Q4_K, Q6_K, Q5_K, Q2_K, Q3_K = 1, 2, 3, 4, 5
-FMT = {"q4_k": Q4_K, "q6_k": Q6_K, "q5_k": Q5_K, "q2_k": Q2_K, "q3_k": Q3_K}
-BLOCK_BYTES = {Q4_K: 144, Q6_K: 210, Q5_K: 176, Q2_K: 84, Q3_K: 110}
+Q4_K, Q6_K, Q5_K, Q2_K, Q3_K, Q8_0 = 1, 2, 3, 4, 5, 6
+FMT = {"q4_k": Q4_K, "q6_k": Q6_K, "q5_k": Q5_K, "q2_k": Q2_K, "q3_k": Q3_K, "q8_0": Q8_0}
+# bytes per 256 weights (Q8_0: eight 34-byte blocks)
+BLOCK_BYTES = {Q4_K: 144, Q6_K: 210, Q5_K: 176, Q2_K: 84, Q3_K: 110, Q8_0: 272}
 
 
 def build(force: bool = False) -> str:

@@ -28,6 +28,9 @@
  *     sc_g and m_g 4-bit.
  *   Q3_K (110 B, 16 groups of 16): w = d*(v_g - 32)*q, q in -4..3, v_g a
  *     6-bit scale.
+ *   Q8_0 (34 B per block of 32: fp16 d, then 32 int8 quants): w = d*q.  A
+ *     row of K weights is K/32 consecutive blocks; here taken 8 blocks (256
+ *     weights, 272 B) at a time, like the K-quant super-blocks.
  *
  * Every step is a literal loop; no blocking, fusion or reordering.
  */
@@ -36,7 +39,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { KQO_Q4_K = 1, KQO_Q6_K = 2, KQO_Q5_K = 3, KQO_Q2_K = 4, KQO_Q3_K = 5 };
+enum { KQO_Q4_K = 1, KQO_Q6_K = 2, KQO_Q5_K = 3, KQO_Q2_K = 4, KQO_Q3_K = 5, KQO_Q8_0 = 6 };
 
 /* IEEE binary16 -> double (exact), including subnormals, inf and NaN. */
 double kqo_f16(uint16_t h) {
@@ -178,9 +181,20 @@ void kqo_q6k_unpack(const uint8_t* blk, uint8_t q[256], int8_t s[16], double* d)
     *d = kqo_f16(rd16(blk + 208));
 }
 
+/* Q8_0, eight blocks (256 weights) -> logical fields: block j at byte 34j
+ * holds d_j (fp16) and then the int8 quants of weights 32j..32j+31. */
+void kqo_q80_unpack(const uint8_t* unit, int8_t q[256], double d[8]) {
+    for (int j = 0; j < 8; ++j) {
+        const uint8_t* blk = unit + 34 * j;
+        d[j] = kqo_f16(rd16(blk));
+        for (int i = 0; i < 32; ++i) q[32 * j + i] = (int8_t)blk[2 + i];
+    }
+}
+
+/* Bytes per 256 weights. */
 static int64_t block_bytes(int fmt) {
     return fmt == KQO_Q4_K ? 144 : fmt == KQO_Q6_K ? 210 : fmt == KQO_Q5_K ? 176 : fmt == KQO_Q2_K ? 84
-                                                                         : fmt == KQO_Q3_K ? 110 : -1;
+         : fmt == KQO_Q3_K ? 110 : fmt == KQO_Q8_0 ? 272 : -1;
 }
 
 /* Dequantise one row of K weights (K/256 consecutive super-blocks). */
@@ -217,6 +231,11 @@ int kqo_dequant_row(int fmt, const uint8_t* row, int64_t K, double* w) {
                 int g = i / 16;
                 wb[i] = d * ((int)v[g] - 32) * qq[i];
             }
+        } else if (fmt == KQO_Q8_0) {
+            int8_t qq[256];
+            double d[8];
+            kqo_q80_unpack(blk, qq, d);
+            for (int i = 0; i < 256; ++i) wb[i] = d[i / 32] * qq[i];
         } else {
             int8_t s[16];
             double d;
@@ -336,11 +355,13 @@ int kqo_gemv_x64(int fmt, const uint8_t* W, int64_t N, int64_t K, const double* 
  *   sc[16*b + j]      Q4_K, Q5_K: sc_0..7 then m_0..7; Q6_K: the 16 signed
  *                     scales as two's-complement bytes
  *                     Q2_K: the 16 raw scale bytes (scale | min << 4);
- *                     Q3_K: the 16 6-bit scales v (before -32)
- *                     (Q2_K quants 0..3; Q3_K values -4..3 as two's-complement
- *                     bytes)
+ *                     Q3_K: the 16 6-bit scales v (before -32);
+ *                     Q8_0: the 8 blocks' fp16 scales, raw (little-endian)
+ *                     (Q2_K quants 0..3; Q3_K values -4..3 and Q8_0 quants
+ *                     as two's-complement bytes)
  *   d[2*b], d[2*b+1]  Q4_K, Q5_K, Q2_K: d, dmin; Q6_K, Q3_K: d, 0 (fp16
- *                     widened exactly) */
+ *                     widened exactly); Q8_0: 0, 0
+ * (For Q8_0, b counts units of eight 34-byte blocks, 256 weights.) */
 int kqo_unpack(int fmt, const uint8_t* W, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d) {
     int64_t bb = block_bytes(fmt);
     if (bb < 0) return -1;
@@ -363,6 +384,15 @@ int kqo_unpack(int fmt, const uint8_t* W, int64_t nblocks, uint8_t* q, uint8_t* 
             double dd;
             kqo_q3k_unpack(blk, (int8_t*)(q + 256 * b), sc + 16 * b, &dd);
             d[2 * b] = (float)dd;
+            d[2 * b + 1] = 0.0f;
+        } else if (fmt == KQO_Q8_0) {
+            double dd[8];
+            kqo_q80_unpack(blk, (int8_t*)(q + 256 * b), dd);
+            for (int j = 0; j < 8; ++j) {  /* the raw fp16 scale bits */
+                sc[16 * b + 2 * j] = blk[34 * j];
+                sc[16 * b + 2 * j + 1] = blk[34 * j + 1];
+            }
+            d[2 * b] = 0.0f;
             d[2 * b + 1] = 0.0f;
         } else {
             double dd;

@@ -3,7 +3,8 @@ than the oracle itself — hand-worked blocks, library routines, closed forms,
 invariants and exhaustive round trips.
 
 Formats: GGUF K-quants Q4_K and Q5_K (w = d*sc_j*q - dmin*m_j per 32-weight
-sub-block, q of 4 or 5 bits) and Q6_K (w = d*s_g*(q-32) per 16-weight group),
+sub-block, q of 4 or 5 bits), Q6_K (w = d*s_g*(q-32) per 16-weight group),
+Q2_K, Q3_K, and the 8-bit Q8_0 (w = d*q per block of 32),
 the formats the pages name ("Out-of-core LLM inference engine written from scratch in Rust",
 Results: Q4_K_M; "RunNburn - Run a 295B MoE ...": K-quants Q2_K..Q6_K).
 """
@@ -144,7 +145,50 @@ def test_q3k_hand_worked_block(golden_dir):
     assert y[0] == float(g["y_ones"][0])
 
 
+def _q80_golden_unit(g):
+    """The worked unit's bytes, from its stated d bytes and quant rules."""
+    dbytes = [int(h, 16) for h in g["d"]]
+    out = []
+    for j in range(8):
+        q = [i - 16 for i in range(32)] if j % 2 == 0 else [8 * i - 128 for i in range(31)] + [127]
+        out += dbytes[2 * j:2 * j + 2] + [v & 0xFF for v in q]
+    return np.array(out, np.uint8)
+
+
+def test_q80_hand_worked_unit(golden_dir):
+    g = _read_golden(os.path.join(golden_dir, "q80_unit_worked.txt"))
+    blk = _q80_golden_unit(g)
+    assert blk.size == 272
+    q, sc, d = oracle.unpack("q8_0", blk, 1)
+    assert sc.tolist() == [int(h, 16) for h in g["d"]]   # the raw fp16 scales
+    assert d.tolist() == [0.0, 0.0]
+    w = oracle.dequant("q8_0", blk, 1, 256)[0]
+    qs = q.view(np.int8)
+    for i, qi, wi in g["w"]:
+        assert qs[i] == qi, i
+        assert w[i] == wi, i
+    y, _ = oracle.gemv("q8_0", blk, 1, 256, np.ones(256, np.float32))
+    assert y[0] == float(g["y_ones"][0])
+
+
 # ----------------------------------------------- exhaustive round trips
+def test_q80_roundtrip_all_values_all_positions():
+    """Every int8 value in every quant position, and each block's scale,
+    survive generator packing and oracle unpacking."""
+    nu = 256
+    u, i = np.meshgrid(np.arange(nu), np.arange(256), indexing="ij")
+    q = ((i * 7 + u) % 256 - 128).astype(np.int8)
+    d = ((np.arange(nu)[:, None] * 8 + np.arange(8)[None, :]) * 37 % 0x7C00).astype(np.uint16)
+    W = kqgen.q80_pack(q, d)
+    qo, sc, _ = oracle.unpack("q8_0", W, nu)
+    assert np.array_equal(qo.view(np.int8).reshape(nu, 256), q)
+    assert np.array_equal(sc.reshape(nu, 16).view(np.uint16).reshape(nu, 8), d)
+    assert all(len(set(q[:, k].tolist())) == 256 for k in range(256))
+    wd = oracle.dequant("q8_0", W, nu, 256)
+    want = d.view(np.float16).astype(np.float64).repeat(32, axis=1) * q.astype(np.float64)
+    assert np.array_equal(wd, want)
+
+
 def test_q2k_q3k_roundtrip_all_values_all_positions():
     """Every quant value in every position and every scale (and Q2_K min)
     value in every slot survive generator packing and oracle unpacking."""
@@ -332,7 +376,7 @@ def test_q6k_mid_quants_give_exact_zero_and_zero_quants_closed_form():
 
 
 # -------------------------------------------------------------- invariants
-@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k", "q2_k", "q3_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k", "q2_k", "q3_k", "q8_0"])
 def test_linearity_in_x(fmt):
     N, K = 8, 1024
     W = kqgen.matrix(fmt, 11, N, K)
@@ -346,7 +390,7 @@ def test_linearity_in_x(fmt):
     assert np.all(np.abs(yc - (2 * y1 - 3 * y2)) <= 1e-12 * (2 * s1 + 3 * s2))
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k", "q2_k", "q3_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k", "q2_k", "q3_k", "q8_0"])
 def test_one_hot_extracts_column_and_ones_give_row_sums(fmt):
     N, K = 4, 512
     W = kqgen.matrix(fmt, 12, N, K)
@@ -361,7 +405,7 @@ def test_one_hot_extracts_column_and_ones_give_row_sums(fmt):
     assert np.allclose(s, np.abs(Wd).sum(axis=1), rtol=1e-13)
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k", "q2_k", "q3_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q6_k", "q2_k", "q3_k", "q8_0"])
 def test_brute_force_tiny_from_logical_values(fmt):
     """Dense W built from the generator's logical values (never its bytes)
     matches the oracle's byte path."""
@@ -389,6 +433,11 @@ def test_brute_force_tiny_from_logical_values(fmt):
         d = lg["d"].view(np.float16).astype(np.float64)[:, None]
         v = np.repeat(lg["v"].astype(np.float64) - 32, 16, axis=1)
         dense = (d * v * lg["q"].astype(np.float64)).reshape(N, K)
+    elif fmt == "q8_0":
+        lg = kqgen.q80_draw(37, nb)
+        W = kqgen.q80_pack(**lg)
+        d = np.repeat(lg["d"].view(np.float16).astype(np.float64), 32, axis=1)
+        dense = (d * lg["q"].astype(np.float64)).reshape(N, K)
     else:
         lg = kqgen.q6k_draw(32, nb)
         W = kqgen.q6k_pack(**lg)
