@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "K-quant dequant-GEMV weight GB/s (% of B200 HBM peak); layer-chain tok/s"
 QK = 256
-BLOCK = {"q4_k": 144, "q5_k": 176, "q6_k": 210, "q2_k": 84, "q3_k": 110}
+BLOCK = {"q4_k": 144, "q5_k": 176, "q6_k": 210, "q2_k": 84, "q3_k": 110, "q8_0": 272}  # bytes per 256 weights
 SEED = 0xC0FFEE + 1
 
 
@@ -74,6 +74,8 @@ def chain_spec(kind):
         return [dense_layer(**L8B, fmt="q2_k", down_fmt="q3_k") for _ in range(32)]
     if kind == "llama8b_q3k":
         return [dense_layer(**L8B, fmt="q3_k", down_fmt="q4_k") for _ in range(32)]
+    if kind == "llama8b_q80":
+        return [dense_layer(**L8B, fmt="q8_0", down_fmt="q8_0") for _ in range(32)]
     if kind == "llama70b":
         return [dense_layer(**L70B) for _ in range(80)]
     if kind == "gemv_q4k_4096":
@@ -86,6 +88,8 @@ def chain_spec(kind):
         return [[("gate_up", "q2_k", 28672, 4096, 0)] for _ in range(8)]
     if kind == "gateup_q3k":
         return [[("gate_up", "q3_k", 28672, 4096, 0)] for _ in range(8)]
+    if kind == "gateup_q80":
+        return [[("gate_up", "q8_0", 28672, 4096, 0)] for _ in range(8)]
     if kind == "down_q3k":
         return [[("down", "q3_k", 4096, 14336, 0)] for _ in range(8)]
     if kind == "down_q6k":
@@ -106,6 +110,8 @@ WORKLOADS = {
     "gateup_q2k": "Q2_K GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
     "gateup_q3k": "Q3_K GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
     "down_q3k": "Q3_K GEMV 4096 x 14336 (8B down), 8 distinct copies rotated",
+    "llama8b_q80_chain": "Llama-3.1-8B-shaped decode chain with every matrix in Q8_0, 32 layers, batch 1",
+    "gateup_q80": "Q8_0 GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
     "llama8b_chain_steps": "the same chain through kq_gemv_steps (16 matvecs per persistent launch, each "
                            "waiting for the one before)",
     "llama8b_layer_fused": "the 8B-shaped chain with RMSNorm fused into qkv and gate|up and the SiLU-gated "
@@ -466,9 +472,10 @@ def make_workload(name, torch, kq, kqgen, seed):
         return Resident(torch, kq, kqgen, chain_spec("llama8b_q5k"), seed)
     if name == "verify8b_q5k_k8":
         return Resident(torch, kq, kqgen, chain_spec("llama8b_q5k"), seed, k=8)
-    if name in ("llama8b_q2k_chain", "llama8b_q3k_chain"):
+    if name in ("llama8b_q2k_chain", "llama8b_q3k_chain", "llama8b_q80_chain"):
         return Resident(torch, kq, kqgen, chain_spec(name[:-len("_chain")]), seed)
-    if name in ("gemv_q4k_4096", "gateup_q4k", "gateup_q5k", "down_q6k", "gateup_q2k", "gateup_q3k", "down_q3k"):
+    if name in ("gemv_q4k_4096", "gateup_q4k", "gateup_q5k", "down_q6k", "gateup_q2k", "gateup_q3k", "down_q3k",
+                "gateup_q80"):
         return Resident(torch, kq, kqgen, chain_spec(name), seed)
     if name.startswith("verify8b_k"):
         k = int(name[len("verify8b_k"):])
@@ -756,7 +763,8 @@ def cpu_baseline(args, budget_s=15.0):
                                                         + MOE30B["hidden"] * row_bytes("q4_k", MOE30B["ffn"]))
     else:
         base = {"llama8b_chain": "llama8b", "llama8b_q5k_chain": "llama8b_q5k", "verify8b_q5k_k8": "llama8b_q5k",
-                "llama8b_q2k_chain": "llama8b_q2k", "llama8b_q3k_chain": "llama8b_q3k", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
+                "llama8b_q2k_chain": "llama8b_q2k", "llama8b_q3k_chain": "llama8b_q3k",
+                "llama8b_q80_chain": "llama8b_q80", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
                 "llama8b_layer_fused_steps": "llama8b", "llama70b_resident": "llama70b",
                 "llama70b_resident_steps": "llama70b", "llama70b_stream": "llama70b", "llama70b_stream_20gb": "llama70b"}
         name = base.get(args.workload, "llama8b" if args.workload.startswith("verify") else args.workload)

@@ -254,7 +254,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     DevInfo di;
     cudaError_t err = dev_info(di);
     if (err != cudaSuccess) return cuda_fail(err, "device query");
-    if (fmt == KQ_FMT_Q2_K || fmt == KQ_FMT_Q3_K)
+    if (fmt == KQ_FMT_Q2_K || fmt == KQ_FMT_Q3_K || fmt == KQ_FMT_Q8_0)
         return fail(KQ_ERR_UNSUPPORTED, "no tensor-core kernel for format %d", fmt);
     if (fmt == KQ_FMT_Q6_K && a.nb % 8 != 0)
         return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
@@ -345,7 +345,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
 
 static bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
-static bool known_format(int fmt) { return fmt >= KQ_FMT_Q4_K && fmt <= KQ_FMT_Q3_K; }
+static bool known_format(int fmt) { return fmt >= KQ_FMT_Q4_K && fmt <= KQ_FMT_Q8_0; }
 
 static int check_matrix(const void* W, int fmt, int64_t N, int64_t K) {
     if (!known_format(fmt))
@@ -366,11 +366,12 @@ static int check_matrix(const void* W, int fmt, int64_t N, int64_t K) {
 static int padded_cols(int k) { return k <= 1 ? 1 : k <= 2 ? 2 : k <= 4 ? 4 : 8; }
 
 static cudaError_t dispatch(const GemvArgs& a, const LaunchPlan& p, int fmt, int ncol, cudaStream_t s) {
-    if (fmt == KQ_FMT_Q5_K || fmt == KQ_FMT_Q2_K || fmt == KQ_FMT_Q3_K) {
+    if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q6_K) {
         if (ncol != 1) return cudaErrorNotSupported;  // (plan_gemv refuses it first)
         if (fmt == KQ_FMT_Q5_K) return launch_one<3, 1, 2>(a, p, s);
         if (fmt == KQ_FMT_Q2_K) return launch_one<4, 1, 2>(a, p, s);
-        return launch_one<5, 1, 2>(a, p, s);
+        if (fmt == KQ_FMT_Q3_K) return launch_one<5, 1, 2>(a, p, s);
+        return launch_one<6, 1, 2>(a, p, s);
     }
     if (fmt == KQ_FMT_Q4_K) {
         switch (ncol) {
@@ -408,9 +409,11 @@ static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt,
 
 // Calls with 2 or more columns (speculative verify) run on the tensor-core
 // kernel, every column group of the call included, so a column's arithmetic
-// never depends on how the call was grouped.  Q2_K and Q3_K have no
+// never depends on how the call was grouped.  Q2_K, Q3_K and Q8_0 have no
 // tensor-core kernel: their columns run one single-column launch each.
-static bool use_mma(int fmt, int k) { return k >= 2 && fmt != KQ_FMT_Q2_K && fmt != KQ_FMT_Q3_K; }
+static bool use_mma(int fmt, int k) {
+    return k >= 2 && fmt != KQ_FMT_Q2_K && fmt != KQ_FMT_Q3_K && fmt != KQ_FMT_Q8_0;
+}
 
 static int plan_for(int fmt, int k, bool mma, GemvArgs& a, LaunchPlan& p) {
     if (mma) return plan_mma(fmt, k <= 4 ? 1 : 2, a, p);
@@ -534,6 +537,7 @@ size_t kq_block_bytes(int fmt) {
         case KQ_FMT_Q5_K: return kQ5Bytes;
         case KQ_FMT_Q2_K: return kQ2Bytes;
         case KQ_FMT_Q3_K: return kQ3Bytes;
+        case KQ_FMT_Q8_0: return kQ80Bytes;
         default: return 0;
     }
 }

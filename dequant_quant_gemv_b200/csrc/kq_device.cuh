@@ -13,10 +13,13 @@ constexpr int kQ6Bytes = 210;      // Q6_K super-block
 constexpr int kQ5Bytes = 176;      // Q5_K super-block
 constexpr int kQ2Bytes = 84;       // Q2_K super-block
 constexpr int kQ3Bytes = 110;      // Q3_K super-block
-// Bytes of a super-block of format FMT (1 Q4_K, 2 Q6_K, 3 Q5_K, 4 Q2_K, 5 Q3_K).
+constexpr int kQ80Bytes = 272;     // Q8_0: eight 34-byte blocks (256 weights)
+// Bytes per 256 weights of format FMT (1 Q4_K, 2 Q6_K, 3 Q5_K, 4 Q2_K, 5
+// Q3_K, 6 Q8_0).
 template <int FMT>
 __host__ __device__ constexpr int block_bytes_of() {
-    return FMT == 1 ? kQ4Bytes : FMT == 2 ? kQ6Bytes : FMT == 3 ? kQ5Bytes : FMT == 4 ? kQ2Bytes : kQ3Bytes;
+    return FMT == 1 ? kQ4Bytes : FMT == 2 ? kQ6Bytes : FMT == 3 ? kQ5Bytes : FMT == 4 ? kQ2Bytes
+         : FMT == 5 ? kQ3Bytes : kQ80Bytes;
 }
 constexpr int kConsumerWarps = 8;  // warps that dequantise and multiply
 constexpr int kConsumers = kConsumerWarps * 32;
@@ -203,6 +206,11 @@ __device__ __forceinline__ float2 ld_s64f(uint32_t a) {
     asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
     return v;
 }
+__device__ __forceinline__ uint2 ld_s2w(uint32_t a) {  // two words, 8-byte aligned
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
 __device__ __forceinline__ uint32_t ld_s32(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
@@ -236,6 +244,17 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
 __device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;
     asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+// Signed quants (Q8_0) with signed (ss) or unsigned (su) activation bytes.
+__device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
 }
 

@@ -1048,6 +1048,68 @@ __device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b
     out[1][0] = y[1];
 }
 
+// Q8_0 unit, one column, on DP4A: row pair at row0, unit b of eight
+// 34-byte blocks (272 bytes, 256 weights), half H = blocks 4H..4H+3 (136
+// bytes from an 8-byte boundary).  Block k of the half (weights 128H + 32k +
+// l, activation group k of the region) starts at byte 34k: fp16 d, then 32
+// int8 quants.  Blocks 0 and 2 start on a 4-byte boundary (their quant
+// words are rebuilt from two loaded words by a byte permute), blocks 1 and
+// 3 two bytes past one (their quant words are aligned).  The half is read as
+// two runs of 18 words (8-byte loads), one per pair of blocks.  Per block
+// the exact int32 S = sum q*xi (|S| <= 2^26) and y += d*P*S.
+__device__ __forceinline__ void q80_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
+                                             float (&out)[2][1]) {
+    float y[2] = {0.f, 0.f};
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {  // blocks 2p and 2p+1: bytes 68p .. 68p+67 of the half
+        uint32_t Wd[2][18];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint32_t base = row0 + r * row_bytes + b * kQ80Bytes + 136 * H + 64 * p;  // 8-byte aligned
+#pragma unroll
+            for (int i = 0; i < 9; ++i) {
+                const uint2 v = ld_s2w(base + 8 * i);
+                Wd[r][2 * i] = v.x;
+                Wd[r][2 * i + 1] = v.y;
+            }
+        }
+        // block 2p starts at word p (byte 4p of the run), block 2p+1 at byte
+        // 34 + 4p: word 8 + p, two bytes in
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            const int k = 2 * p + kk;
+            const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * k);  // X, P
+            const float P = __uint_as_float(info.y);
+            int hi[2] = {0, 0}, lo[2] = {0, 0};
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                const uint4 xh = ld_s128(xr + kXGroupBytes * k + 16 * s);
+                const uint4 xl = ld_s128(xr + kXGroupBytes * k + 32 + 16 * s);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int i = 4 * s + m;  // quant word i of the block
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const uint32_t q = kk == 0 ? __byte_perm(Wd[r][p + i], Wd[r][p + i + 1], 0x5432u)
+                                                   : Wd[r][9 + p + i];
+                        hi[r] = dp4a_ss(q, u4w(xh, m), hi[r]);
+                        lo[r] = dp4a_su(q, u4w(xl, m), lo[r]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t dw = kk == 0 ? (Wd[r][p] & 0xFFFFu) : (Wd[r][8 + p] >> 16);
+                const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(dw)));
+                const int S = hi[r] * 256 + lo[r];
+                y[r] = fmaf(d * P, static_cast<float>(S), y[r]);
+            }
+        }
+    }
+    out[0][0] = y[0];
+    out[1][0] = y[1];
+}
+
 // Q6_K unit, one column, on DP4A: row pair at row0, super-block b (210
 // bytes: ql[128], qh[64], 16 int8 scales, d), half H.  Blocks are 2-byte
 // aligned only and b's parity varies across the lanes, so each stream is
@@ -1195,7 +1257,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     const int64_t rp_begin = P * rc / G;
     const int64_t rp_end = P * (rc + 1) / G;
     constexpr int BS = block_bytes_of<FMT>();
-    static_assert(FMT <= 2 || NCOL == 1, "Q5_K, Q2_K and Q3_K: one column per launch in this kernel");
+    static_assert(FMT <= 2 || NCOL == 1, "Q5_K, Q2_K, Q3_K and Q8_0: one column per launch in this kernel");
     const int kb0 = ks * a.nbs;
     const int nbl = a.nb - kb0 < a.nbs ? a.nb - kb0 : a.nbs;       // blocks in this range
     const int srow = a.ksplit > 1 ? a.nbs * BS : static_cast<int>(a.row_bytes);  // staged row stride
@@ -1305,6 +1367,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
                 q2k_unit_int(row0, srow, u_b, u_H, xri, out);
             } else if constexpr (INT && FMT == 5) {
                 q3k_unit_int(row0, srow, u_b, u_H, xri, out);
+            } else if constexpr (INT && FMT == 6) {
+                q80_unit_int(row0, srow, u_b, u_H, xri, out);
             } else if constexpr (INT) {
                 q6k_unit_int(row0, srow, u_b, u_H, xri, out);
             } else if constexpr (FMT == 1) {

@@ -60,6 +60,16 @@ __global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_
         const uint32_t dw = *reinterpret_cast<const uint32_t*>(blk + 80);
         d[2 * b] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw & 0xFFFFu)));
         d[2 * b + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw >> 16)));
+    } else if (fmt == 6) {
+        // Q8_0: a unit of eight 34-byte blocks, read by bytes
+        const uint8_t* u = W + b * kQ80Bytes;
+        for (int j = 0; j < 8; ++j) {
+            sc[16 * b + 2 * j] = u[34 * j];
+            sc[16 * b + 2 * j + 1] = u[34 * j + 1];
+            for (int i = 0; i < 32; ++i) q[256 * b + 32 * j + i] = u[34 * j + 2 + i];
+        }
+        d[2 * b] = 0.0f;
+        d[2 * b + 1] = 0.0f;
     } else if (fmt == 5) {
         // Q3_K: 2-byte aligned blocks, read by bytes
         const uint8_t* blk = W + b * kQ3Bytes;

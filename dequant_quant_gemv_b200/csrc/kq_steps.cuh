@@ -181,10 +181,10 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
         // this step's activations, staged by all consumer threads
         const GemvArgs a = step_view(s);
         float rinv = 1.f;
-        if (s.fmt != 1 && s.fmt != 3) {  // Q2_K, Q3_K, Q6_K: integer regions with 16-sums
+        if (s.fmt == 2 || s.fmt == 4 || s.fmt == 5) {  // Q2_K, Q3_K, Q6_K: integer regions with 16-sums
             if (s.pro) stage_all<2, 1, true, true>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
             else stage_all<2, 1, true, false>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
-        } else {  // Q4_K and Q5_K: integer regions
+        } else {  // Q4_K, Q5_K, Q8_0: integer regions
             if (s.pro) stage_all<1, 1, true, true>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
             else stage_all<1, 1, true, false>(a, 0, xs_s, ct_all, nthr, 3, 0, s.nb, pro_r);
         }
@@ -224,6 +224,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
                 else if (s.fmt == 3) q5k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else if (s.fmt == 4) q2k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else if (s.fmt == 5) q3k_unit_int(rw, srow, u_b, u_H, xri, out);
+                else if (s.fmt == 6) q80_unit_int(rw, srow, u_b, u_H, xri, out);
                 else q6k_unit_int(rw, srow, u_b, u_H, xri, out);
             }
             // butterfly over the lanes of this row pair (fixed order)

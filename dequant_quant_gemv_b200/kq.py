@@ -20,8 +20,9 @@ Q6_K = 2
 Q5_K = 3
 Q2_K = 4
 Q3_K = 5
-FORMATS = {"q4_k": Q4_K, "q6_k": Q6_K, "q5_k": Q5_K, "q2_k": Q2_K, "q3_k": Q3_K}
-BLOCK_BYTES = {Q4_K: 144, Q6_K: 210, Q5_K: 176, Q2_K: 84, Q3_K: 110}
+Q8_0 = 6
+FORMATS = {"q4_k": Q4_K, "q6_k": Q6_K, "q5_k": Q5_K, "q2_k": Q2_K, "q3_k": Q3_K, "q8_0": Q8_0}
+BLOCK_BYTES = {Q4_K: 144, Q6_K: 210, Q5_K: 176, Q2_K: 84, Q3_K: 110, Q8_0: 272}  # per 256 weights
 
 OK = 0
 STATUS = {0: "KQ_OK", 1: "KQ_ERR_INVALID_ARG", 2: "KQ_ERR_UNSUPPORTED", 3: "KQ_ERR_NOT_PINNED",

@@ -1,6 +1,6 @@
 /*
  * kq.h — libkq: decode-time matrix-vector products over GGUF K-quant
- * weights (Q2_K, Q3_K, Q4_K, Q5_K, Q6_K) on NVIDIA B200 (sm_100a), with the weights
+ * weights (Q2_K, Q3_K, Q4_K, Q5_K, Q6_K, and Q8_0) on NVIDIA B200 (sm_100a), with the weights
  * dequantised only in registers inside the fused kernels.
  *
  * What the method is (by page):
@@ -42,15 +42,19 @@
  *   Q6_K super-block, 210 bytes, 256 weights in 16 groups of 16:
  *     128 bytes low 4 bits | 64 bytes high 2 bits | 16 int8 scales s_g |
  *     fp16 d.   w = d*s_g*(q - 32), q in 0..63.
- *   (The GGUF K-quant bit layout; the pages name the formats but print no
+ *   Q8_0 blocks, 34 bytes per 32 weights: fp16 d | 32 int8 quants q.
+ *     w = d*q.  A row is K/32 consecutive blocks; the library takes them
+ *     in units of 8 blocks (256 weights, 272 bytes), so K % 256 == 0 here
+ *     too.
+ *   (The GGUF bit layout; the pages name the formats but print no
  *   layout.)
  *
  * Conventions for every entry point:
  *  - All pointers named W, x, y, ids, status are DEVICE pointers owned by the
  *    caller; libkq never frees or retains them past the call (the chain object
  *    below is the exception and says so).
- *  - W must be 16-byte aligned, and so must every row: always true for Q4_K
- *    and Q5_K; Q2_K requires K % 1024 == 0, Q3_K and Q6_K K % 2048 == 0
+ *  - W must be 16-byte aligned, and so must every row: always true for Q4_K,
+ *    Q5_K and Q8_0; Q2_K requires K % 1024 == 0, Q3_K and Q6_K K % 2048 == 0
  *    (else KQ_ERR_UNSUPPORTED).  x and y must be 4-byte aligned.
  *  - Calls are asynchronous on `stream` (0 = the legacy default stream).  The
  *    return value reports argument validation and launch errors only
@@ -61,7 +65,7 @@
  *    the group's largest |x|), every format alike; two or
  *    more columns of Q4_K..Q6_K run on the tensor cores with exact fp16 weight operands and
  *    activations split into two fp16 terms (22 bits) after a power-of-two
- *    scale per super-block; several columns of Q2_K and Q3_K run one
+ *    scale per super-block; several columns of Q2_K, Q3_K and Q8_0 run one
  *    single-column launch per column.  Every output satisfies
  *    |y - y_exact| <= 1e-3 * sum_i |w_i x_i| + 1e-6 for activations of
  *    comparable magnitude within each group of 32.
@@ -95,7 +99,8 @@ typedef enum {
     KQ_FMT_Q6_K = 2,
     KQ_FMT_Q5_K = 3,
     KQ_FMT_Q2_K = 4,
-    KQ_FMT_Q3_K = 5
+    KQ_FMT_Q3_K = 5,
+    KQ_FMT_Q8_0 = 6
 } kq_fmt;
 
 typedef enum {
@@ -124,8 +129,8 @@ KQ_API const char* kq_last_error(void);
  * hanging.  Synchronous.  *out is a HOST int. */
 KQ_API int kq_device_fault(int* out);
 
-/* Bytes per super-block (Q2_K 84, Q3_K 110, Q4_K 144, Q5_K 176, Q6_K 210)
- * or 0 for an unknown format. */
+/* Bytes per super-block (Q2_K 84, Q3_K 110, Q4_K 144, Q5_K 176, Q6_K 210;
+ * Q8_0 272, per 8 blocks of 32 weights) or 0 for an unknown format. */
 KQ_API size_t kq_block_bytes(int fmt);
 
 /* Bytes per weight row: (K/256) * kq_block_bytes(fmt); 0 if K % 256 != 0. */
@@ -301,7 +306,10 @@ KQ_API int kq_moe_gemv(const void* W_experts, int fmt, int E, int64_t N, int64_t
  *       bytes sc_g | m_g << 4 as stored; Q3_K: the 16 6-bit v_g (before the
  *       -32 offset); Q6_K: the 16 int8 scales as two's-complement bytes
  *   d:  n_blocks*2 floats; Q2_K, Q4_K, Q5_K: d, dmin; Q3_K, Q6_K: d, 0
- *       (fp16 widened exactly)
+ *       (fp16 widened exactly); Q8_0: 0, 0
+ *   For Q8_0 a "block" here is a unit of 8 blocks (256 weights): q holds its
+ *   int8 quants as two's-complement bytes and sc the 8 fp16 scales d as raw
+ *   little-endian bytes.
  * All device pointers; W must be 16-byte aligned.
  */
 KQ_API int kq_unpack(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d,

@@ -52,7 +52,9 @@ def test_host_only_helpers(libkq):
     assert L.kq_block_bytes(4) == 84                  # Q2_K
     assert L.kq_block_bytes(5) == 110                 # Q3_K
     assert L.kq_row_bytes(5, 2048) == 8 * 110
-    assert L.kq_block_bytes(6) == 0                   # no such format
+    assert L.kq_block_bytes(6) == 272                 # Q8_0, per 8 blocks of 32
+    assert L.kq_row_bytes(6, 4096) == 16 * 272
+    assert L.kq_block_bytes(7) == 0                   # no such format
     assert L.kq_block_bytes(0) == 0
     assert L.kq_status_str(0) == b"ok"
     assert L.kq_version() >= 100

@@ -22,7 +22,8 @@ def _cuda():
 
 
 SHAPES = [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q6_k", 130, 2048), ("q4_k", 40, 768), ("q5_k", 200, 4096),
-          ("q5_k", 24, 14336), ("q2_k", 200, 4096), ("q2_k", 24, 14336), ("q3_k", 200, 4096), ("q3_k", 24, 14336)]
+          ("q5_k", 24, 14336), ("q2_k", 200, 4096), ("q2_k", 24, 14336), ("q3_k", 200, 4096), ("q3_k", 24, 14336),
+          ("q8_0", 200, 4096), ("q8_0", 24, 14336)]
 
 
 @pytest.mark.parametrize("fmt,N,K", SHAPES)

@@ -29,7 +29,7 @@ def _cuda():
 @pytest.mark.parametrize("fmt,N,K", [("q4_k", 4096, 4096), ("q6_k", 64, 14336), ("q6_k", 3, 2048),
                                      ("q5_k", 2048, 4096), ("q5_k", 3, 256), ("q2_k", 512, 4096),
                                      ("q2_k", 3, 1024), ("q3_k", 512, 4096), ("q3_k", 3, 2048),
-                                     ("q3_k", 1, 256)])
+                                     ("q3_k", 1, 256), ("q8_0", 512, 4096), ("q8_0", 3, 256)])
 def test_unpack_bit_exact(fmt, N, K):
     W = matrix(fmt, 1000 + N, N, K)
     nb = N * K // 256
@@ -53,6 +53,8 @@ SHAPES = [
     ("q2_k", 5, 3072), ("q2_k", 4096, 4096), ("q2_k", 2, 14336),
     ("q3_k", 1, 2048), ("q3_k", 5, 2048), ("q3_k", 257, 4096), ("q3_k", 301, 8192), ("q3_k", 9, 32768),
     ("q3_k", 37, 6144), ("q3_k", 4096, 4096), ("q3_k", 2, 14336),
+    ("q8_0", 1, 256), ("q8_0", 7, 768), ("q8_0", 257, 4096), ("q8_0", 301, 8192), ("q8_0", 9, 32768),
+    ("q8_0", 5, 1280), ("q8_0", 4096, 4096), ("q8_0", 2, 14336),
 ]
 
 
@@ -155,6 +157,18 @@ def test_q3k_zero_values_and_scales_give_exact_zero():
     assert torch.all(kq.gemv(dev(W), "q3_k", N, K, x) == 0)
 
 
+def test_q80_zero_quants_or_scales_give_exact_zero():
+    """Q8_0 with every quant 0, or every block scale 0, gives y = 0 exactly."""
+    N, K = 70, 4096
+    nu = N * K // 256
+    lg = kqgen.q80_draw(130, nu)
+    x = dev(x_vec(131, K))
+    W = kqgen.q80_pack(np.zeros_like(lg["q"]), lg["d"])
+    assert torch.all(kq.gemv(dev(W), "q8_0", N, K, x) == 0)
+    W = kqgen.q80_pack(lg["q"], np.zeros_like(lg["d"]))
+    assert torch.all(kq.gemv(dev(W), "q8_0", N, K, x) == 0)
+
+
 def test_q4k_zero_quants_closed_form():
     N, K = 70, 4096
     nb = N * K // 256
@@ -225,7 +239,8 @@ def test_linearity():
                                      ("q6_k", 41, 2048), ("q6_k", 4096, 2048), ("q6_k", 3, 14336),
                                      ("q5_k", 300, 4096), ("q5_k", 33, 14336), ("q5_k", 4096, 4096),
                                      ("q5_k", 17, 768), ("q2_k", 300, 4096), ("q2_k", 33, 14336),
-                                     ("q3_k", 300, 4096), ("q3_k", 33, 14336)])
+                                     ("q3_k", 300, 4096), ("q3_k", 33, 14336), ("q8_0", 300, 4096),
+                                     ("q8_0", 17, 768)])
 @pytest.mark.parametrize("k", [2, 3, 4, 5, 8])
 def test_multi_columns_independent_and_match_oracle(fmt, N, K, k):
     """Each column of a k-column call equals the same column of an 8-column
@@ -244,7 +259,7 @@ def test_multi_columns_independent_and_match_oracle(fmt, N, K, k):
 
 
 @pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q5_k", 300, 4096),
-                                     ("q2_k", 300, 4096), ("q3_k", 300, 4096)])
+                                     ("q2_k", 300, 4096), ("q3_k", 300, 4096), ("q8_0", 300, 4096)])
 def test_single_column_of_multi_call_matches_oracle(fmt, N, K):
     """k = 1 through gemv_multi is the single-column kernel, bitwise."""
     W = matrix(fmt, 32, N, K)
@@ -257,7 +272,7 @@ def test_single_column_of_multi_call_matches_oracle(fmt, N, K):
     assert_close(Y[0], y_ref, s_ref)
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k", "q2_k", "q3_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k", "q2_k", "q3_k", "q8_0"])
 @pytest.mark.parametrize("scale", [1e-30, 1e-6, 1.0, 3e3, 1e20])
 def test_multi_column_scale_range(fmt, scale):
     """Activations far from 1 in either direction (the kernel rescales each
@@ -332,7 +347,7 @@ def test_invalid_arguments_are_rejected():
 
 
 # ------------------------------------------- single-column integer path
-@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q2_k", "q3_k", "q6_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q5_k", "q2_k", "q3_k", "q6_k", "q8_0"])
 def test_single_column_within_activation_rounding_bound(fmt):
     """A single column (every format) rounds each activation to a 14-bit integer
     on a power-of-two grid per group of 32, so |x - x'| <= 2^-14 * (largest
@@ -351,7 +366,7 @@ def test_single_column_within_activation_rounding_bound(fmt):
     assert np.all(err <= bound + slack), float(np.max(err / (bound + slack)))
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k", "q2_k", "q3_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k", "q2_k", "q3_k", "q8_0"])
 @pytest.mark.parametrize("scale", [1e-30, 1e-6, 3e3, 1e20])
 def test_single_column_scale_range(fmt, scale):
     """Single column with activations far from 1: the integer path scales

@@ -32,6 +32,8 @@ def _cuda():
     ("q2_k", 8, 2048, 1024, True),
     ("q3_k", 8, 512, 2048, True),
     ("q3_k", 6, 130, 4096, False),
+    ("q8_0", 16, 768, 2048, False),
+    ("q8_0", 8, 2048, 768, True),
 ])
 def test_moe_parity(fmt, E, N, K, per_id):
     W = matrix(fmt, 300 + E + N, E * N, K)

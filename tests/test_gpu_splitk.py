@@ -21,7 +21,8 @@ def _cuda():
 
 SHAPES = [("q4_k", 1, 4096), ("q4_k", 2, 4096), ("q4_k", 17, 4096), ("q4_k", 64, 32768), ("q4_k", 100, 2048),
           ("q4_k", 5, 768), ("q6_k", 3, 14336), ("q6_k", 64, 28672), ("q6_k", 9, 2048), ("q5_k", 17, 4096),
-          ("q5_k", 3, 14336), ("q2_k", 17, 4096), ("q2_k", 3, 14336), ("q3_k", 17, 4096), ("q3_k", 3, 14336)]
+          ("q5_k", 3, 14336), ("q2_k", 17, 4096), ("q2_k", 3, 14336), ("q3_k", 17, 4096), ("q3_k", 3, 14336),
+          ("q8_0", 17, 4096), ("q8_0", 3, 14336), ("q8_0", 5, 768)]
 
 
 @pytest.mark.parametrize("fmt,N,K", SHAPES)

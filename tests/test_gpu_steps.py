@@ -45,7 +45,8 @@ LAYER = [("q4_k", 6144, 4096, "rmsnorm"), ("q4_k", 4096, 4096, "none"), ("q4_k",
          ("q6_k", 4096, 14336, "swiglu"), ("q4_k", 64, 768, "none"), ("q6_k", 48, 14336, "none"),
          ("q4_k", 1, 256, "rmsnorm"), ("q4_k", 2048, 8192, "none"), ("q5_k", 1024, 4096, "rmsnorm"),
          ("q5_k", 96, 14336, "swiglu"), ("q2_k", 1024, 4096, "rmsnorm"), ("q3_k", 96, 14336, "swiglu"),
-         ("q2_k", 40, 14336, "none"), ("q3_k", 300, 4096, "none")]
+         ("q2_k", 40, 14336, "none"), ("q3_k", 300, 4096, "none"), ("q8_0", 512, 4096, "rmsnorm"),
+         ("q8_0", 64, 14336, "swiglu")]
 
 
 def build(seed, shapes):
