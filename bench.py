@@ -126,6 +126,8 @@ WORKLOADS = {
     "verify8b_k8": "8B-shaped chain, speculative-verify GEMV with k=8 activation columns",
     "moe30b": "Qwen3-30B-A3B-shaped MoE GEMVs: 48 layers x 128 experts (gate|up 1536x2048, down 2048x768, "
               "Q4_K), top-8 routed ids per token, batch 1",
+    "moe30b_stream": "the moe30b GEMVs with all experts in pinned host memory (16.3 GB): per token and layer "
+                     "the 8 routed experts' gate|up and down copied to the device on demand (kq_moe_stream)",
     "llama70b_resident": "Llama-3.3-70B-shaped decode chain, 80 layers, Q4_K + Q6_K down, resident in HBM",
     "llama70b_resident_steps": "the 70B-shaped resident chain through kq_gemv_steps",
     "llama70b_stream": "Llama-3.3-70B-shaped decode chain, 80 layers, weights in pinned host memory streamed "
@@ -463,6 +465,60 @@ class Streamed:
         return [self.X], [self.Y]
 
 
+class MoEStreamed(MoE):
+    """The MoE GEMVs with every expert in pinned host memory: per layer and
+    token the 8 routed experts' gate|up and down matrices are copied to the
+    device on demand (kq_moe_stream) and the routed GEMVs read the copies."""
+
+    graphable = False
+
+    def __init__(self, torch, kq, kqgen, seed, tokens=4):
+        c = MOE30B
+        self.torch, self.kq = torch, kq
+        H, E, top, F, Lyr = c["hidden"], c["experts"], c["top"], c["ffn"], c["layers"]
+        self.E, self.top, self.H, self.F, self.L = E, top, H, F, Lyr
+        self.gu_stride = 2 * F * row_bytes("q4_k", H)
+        self.dn_stride = H * row_bytes("q4_k", F)
+        self.weight_bytes = Lyr * top * (self.gu_stride + self.dn_stride)
+        self.streamed_bytes = self.weight_bytes
+        self.n_resident = 0
+        # every layer's experts in one host stack per matrix kind (expert
+        # l*E + e is expert e of layer l), page-locked in place
+        self.hgu = np.empty(Lyr * E * self.gu_stride, np.uint8)
+        self.hdn = np.empty(Lyr * E * self.dn_stride, np.uint8)
+        for l in range(Lyr):
+            kqgen.matrix("q4_k", kqgen.tensor_seed(seed, l, 0), E * 2 * F, H,
+                         out=self.hgu[l * E * self.gu_stride:(l + 1) * E * self.gu_stride])
+            kqgen.matrix("q4_k", kqgen.tensor_seed(seed, l, 1), E * H, F,
+                         out=self.hdn[l * E * self.dn_stride:(l + 1) * E * self.dn_stride])
+        for h in (self.hgu, self.hdn):
+            rc = torch.cuda.cudart().cudaHostRegister(h.ctypes.data, h.nbytes, 0)
+            if int(rc) != 0:
+                raise RuntimeError(f"cudaHostRegister failed ({rc})")
+        self.msgu = kq.MoEStream(torch.from_numpy(self.hgu), "q4_k", Lyr * E, 2 * F, H, max_ids=top, n_sets=2)
+        self.msdn = kq.MoEStream(torch.from_numpy(self.hdn), "q4_k", Lyr * E, H, F, max_ids=top, n_sets=2)
+        self.ids_all = np.stack([np.stack([kqgen.topk_ids(kqgen.tensor_seed(seed ^ 0x1D5, t, l), E, top) + l * E
+                                           for l in range(Lyr)]) for t in range(tokens)]).astype(np.int32)
+        self.t = 0
+        self.X = torch.from_numpy(kqgen.normal_f32(seed ^ 0x77, Lyr * H + Lyr * top * F)).cuda()
+        self.Y = torch.empty(Lyr * top * 2 * F + Lyr * top * H, dtype=torch.float32, device="cuda")
+        self.launches = [(l, j) for l in range(Lyr) for j in range(2)]
+        torch.cuda.synchronize()
+
+    def launch(self, l, j, stream):
+        ids = self.ids_all[self.t % self.ids_all.shape[0], l]
+        if j == 0:
+            self.msgu.run(ids, self.xg(l), 0, self.yg(l), stream=stream)
+        else:
+            self.msdn.run(ids, self.xd(l), self.F, self.yd(l), stream=stream)
+
+    def advance(self):
+        self.t += 1
+
+    def kinds(self):
+        return {}
+
+
 def make_workload(name, torch, kq, kqgen, seed):
     if name in ("llama8b_chain", "llama8b_chain_steps"):
         return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed, steps=name.endswith("_steps"))
@@ -482,6 +538,8 @@ def make_workload(name, torch, kq, kqgen, seed):
         return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed, k=k)
     if name == "moe30b":
         return MoE(torch, kq, kqgen, seed)
+    if name == "moe30b_stream":
+        return MoEStreamed(torch, kq, kqgen, seed)
     if name in ("llama70b_resident", "llama70b_resident_steps"):
         return Resident(torch, kq, kqgen, chain_spec("llama70b"), seed, steps=name.endswith("_steps"))
     if name == "llama70b_stream":
@@ -738,15 +796,17 @@ def bench_kq(args, rank, world):
                               "traffic": measured_traffic(dk["fmt"], dk["N"], dk["K"], k),
                               "algorithmic_bytes": dk["bytes"]}
         result["kernels"] = per_kind
-    if isinstance(wl, Streamed):
+    if isinstance(wl, (Streamed, MoEStreamed)):
         pk = h2d_peak_gbs(torch)
         h2d = job_rate(wl.streamed_bytes, args.steps, world, ms) / 1e9 / world
-        result["roofline"] = {"bound": "pcie_h2d", "kernel": "H2D copies of the layer ring",
+        result["roofline"] = {"bound": "pcie_h2d",
+                              "kernel": "H2D copies of the routed experts" if isinstance(wl, MoEStreamed)
+                              else "H2D copies of the layer ring",
                               "achieved": round(h2d, 2), "peak": round(pk, 2),
                               "peak_source": "measured here (512 MiB pinned copy)", "unit": "GB/s",
                               "frac": round(h2d / pk, 4), "traffic": None,
                               "streamed_bytes_per_step": wl.streamed_bytes, "resident_layers": wl.n_resident}
-        result["gpu_launches"] = 4 * len(wl.spec) * args.steps
+        result["gpu_launches"] = len(wl.launches) * args.steps
     return result
 
 
@@ -756,7 +816,7 @@ def cpu_baseline(args, budget_s=15.0):
     import kqgen
     import oracle
 
-    if args.workload == "moe30b":
+    if args.workload in ("moe30b", "moe30b_stream"):
         spec = [[("moe_gate_up", "q4_k", 2 * MOE30B["ffn"], MOE30B["hidden"], 0),
                  ("moe_down", "q4_k", MOE30B["hidden"], MOE30B["ffn"], 1)]] * MOE30B["layers"]
         per_token = MOE30B["layers"] * MOE30B["top"] * (2 * MOE30B["ffn"] * row_bytes("q4_k", MOE30B["hidden"])

@@ -10,6 +10,8 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
+
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -301,6 +303,75 @@ def chain_plan(layers, budget_bytes: int, max_slots: int = 4):
     if st != OK:
         raise KQError(st, "kq_chain_plan", L.kq_chain_last_error().decode())
     return int(r.value), int(s.value)
+
+
+def _moe_stream_sigs(L):
+    if getattr(L, "_moe_stream_sigs", False):
+        return
+    i64, i32, vp, sz = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+    L.kq_moe_stream_create.restype = i32
+    L.kq_moe_stream_create.argtypes = [vp, i32, i32, i64, i64, sz, i32, i32, ctypes.POINTER(vp)]
+    L.kq_moe_stream_run.restype = i32
+    L.kq_moe_stream_run.argtypes = [vp, vp, i32, vp, i64, vp, vp]
+    L.kq_moe_stream_wait.restype = i32
+    L.kq_moe_stream_wait.argtypes = [vp, i64]
+    L.kq_moe_stream_destroy.restype = None
+    L.kq_moe_stream_destroy.argtypes = [vp]
+    L.kq_moe_stream_last_error.restype = ctypes.c_char_p
+    L._moe_stream_sigs = True
+
+
+class MoEStream:
+    """Routed experts kept in pinned host memory and copied to the device on
+    demand (kq_moe_stream_* in kq.h).
+
+    W_host: pinned uint8 tensor holding E expert matrices (N x K in fmt),
+    expert e at byte e * stride (default N * row_bytes)."""
+
+    def __init__(self, W_host, fmt, E: int, N: int, K: int, max_ids: int, n_sets: int = 2,
+                 stride: int | None = None):
+        L = lib()
+        _moe_stream_sigs(L)
+        self._L = L
+        if W_host.is_cuda:
+            raise ValueError("streamed experts must be host memory")
+        self._keep = W_host
+        self.N, self.K, self.max_ids = N, K, max_ids
+        stride = stride if stride is not None else N * row_bytes(fmt, K)
+        h = ctypes.c_void_p()
+        st = L.kq_moe_stream_create(W_host.data_ptr(), _fmt(fmt), E, N, K, stride, max_ids, n_sets,
+                                    ctypes.byref(h))
+        if st != OK:
+            raise KQError(st, "kq_moe_stream_create", L.kq_moe_stream_last_error().decode())
+        self._h = h
+
+    def run(self, ids_host, x, x_stride: int = 0, y=None, stream=None):
+        """ids_host: int32 numpy array or CPU tensor; x, y: device tensors."""
+        ids = np.ascontiguousarray(np.asarray(ids_host, dtype=np.int32))
+        n = int(ids.size)
+        if y is None:
+            y = torch.empty((n, self.N), dtype=torch.float32, device=x.device)
+        st = self._L.kq_moe_stream_run(self._h, ids.ctypes.data, n, _dev(x, "x", torch.float32), x_stride,
+                                       _dev(y, "y", torch.float32), _stream(stream))
+        if st != OK:
+            raise KQError(st, "kq_moe_stream_run", self._L.kq_moe_stream_last_error().decode())
+        return y
+
+    def wait(self, timeout_ms: int = -1) -> None:
+        st = self._L.kq_moe_stream_wait(self._h, timeout_ms)
+        if st != OK:
+            raise KQError(st, "kq_moe_stream_wait", self._L.kq_moe_stream_last_error().decode())
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._L.kq_moe_stream_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class Chain:

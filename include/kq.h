@@ -297,6 +297,46 @@ KQ_API int kq_moe_gemv(const void* W_experts, int fmt, int E, int64_t N, int64_t
                 int64_t x_stride, float* y, int32_t* status, kq_stream_t stream);
 
 /*
+ * Streamed MoE — the routed experts' weights stay in PAGE-LOCKED HOST memory
+ * and only the selected experts are copied to the device, per call
+ * ("RunNburn - Run a 295B MoE from a 98GB GGUF on a 64GB RAM Desktop": the
+ * experts a token selects are gathered on demand; "Out-of-core LLM
+ * inference engine ...", Approach: weights stream through VRAM slots while
+ * the GPU computes).
+ *
+ * kq_moe_stream_create: the expert stack W_host (HOST pointer, page-locked,
+ *   owned by the caller and kept alive and unchanged until destroy): E
+ *   matrices of N x K in `fmt`, matrix e at W_host + e*expert_stride_bytes
+ *   (stride >= N*row_bytes).  max_ids: the most ids one run routes; n_sets
+ *   (>= 1): sets of max_ids device slots used in turn, so the copies of the
+ *   next run overlap the GEMV of this one.  Allocates n_sets*max_ids slots of
+ *   N*row_bytes (rounded up to 256) bytes, a copy stream and events.
+ *   KQ_ERR_NOT_PINNED if W_host is not page-locked, KQ_ERR_OOM if the slots
+ *   do not fit.
+ * kq_moe_stream_run: ids_host (HOST int32, n_ids <= max_ids, each in [0, E),
+ *   else KQ_ERR_INVALID_ARG and nothing is enqueued); x, y as kq_moe_gemv
+ *   (DEVICE).  Enqueues, on the object's copy stream, the H2D copies of the
+ *   routed experts into the next slot set (after the GEMV that last read
+ *   that set), then on `compute` the routed GEMV over the set.  Asynchronous.
+ *   y[i] equals, bitwise, kq_moe_gemv with the same experts resident in
+ *   device memory.  The copies wait only for the GEMV that last read their
+ *   set, so they overlap the GEMVs of the other sets.
+ * kq_moe_stream_wait: host-side polling until the last run finished;
+ *   KQ_ERR_TIMEOUT after timeout_ms (negative: no limit).
+ * kq_moe_stream_destroy: waits for the copies, frees slots, stream, events.
+ */
+typedef struct kq_moe_stream kq_moe_stream;
+
+KQ_API int kq_moe_stream_create(const void* W_host, int fmt, int E, int64_t N, int64_t K,
+                                size_t expert_stride_bytes, int max_ids, int n_sets, kq_moe_stream** out);
+KQ_API int kq_moe_stream_run(kq_moe_stream* s, const int32_t* ids_host, int n_ids, const float* x,
+                             int64_t x_stride, float* y, kq_stream_t compute);
+KQ_API int kq_moe_stream_wait(kq_moe_stream* s, int64_t timeout_ms);
+KQ_API void kq_moe_stream_destroy(kq_moe_stream* s);
+/* Text describing the last streamed-MoE failure on the calling thread. */
+KQ_API const char* kq_moe_stream_last_error(void);
+
+/*
  * kq_unpack — debug: the integer fields of n_blocks consecutive super-blocks
  * as the GEMV kernels decode them (for bit-exact comparison).
  *   q:  n_blocks*256 bytes, quant of weight i of block b at q[256b+i]
