@@ -374,6 +374,84 @@ class MoEStream:
             pass
 
 
+def gguf_format(ggml_type: int) -> int:
+    """libkq format id of a ggml type id (0 if none): kq_gguf_kq_format."""
+    L = lib()
+    L.kq_gguf_kq_format.restype = ctypes.c_int
+    L.kq_gguf_kq_format.argtypes = [ctypes.c_int]
+    return int(L.kq_gguf_kq_format(int(ggml_type)))
+
+
+class GGUF:
+    """Tensor table and tensor bytes of a GGUF file (kq_gguf_* in kq.h)."""
+
+    def __init__(self, path: str):
+        L = lib()
+        if not getattr(L, "_gguf_sigs", False):
+            i32, vp, u64 = ctypes.c_int, ctypes.c_void_p, ctypes.c_uint64
+            L.kq_gguf_open.restype = i32
+            L.kq_gguf_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(vp)]
+            L.kq_gguf_tensor_count.restype = i32
+            L.kq_gguf_tensor_count.argtypes = [vp]
+            L.kq_gguf_tensor_info.restype = i32
+            L.kq_gguf_tensor_info.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(i32),
+                                              ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_int64),
+                                              ctypes.POINTER(u64), ctypes.POINTER(u64)]
+            L.kq_gguf_find.restype = i32
+            L.kq_gguf_find.argtypes = [vp, ctypes.c_char_p]
+            L.kq_gguf_kq_format.restype = i32
+            L.kq_gguf_kq_format.argtypes = [i32]
+            L.kq_gguf_read.restype = i32
+            L.kq_gguf_read.argtypes = [vp, i32, vp, u64]
+            L.kq_gguf_close.restype = None
+            L.kq_gguf_close.argtypes = [vp]
+            L.kq_gguf_last_error.restype = ctypes.c_char_p
+            L._gguf_sigs = True
+        self._L = L
+        h = ctypes.c_void_p()
+        st = L.kq_gguf_open(os.fsencode(path), ctypes.byref(h))
+        if st != OK:
+            raise KQError(st, "kq_gguf_open", L.kq_gguf_last_error().decode())
+        self._h = h
+
+    def __len__(self) -> int:
+        return int(self._L.kq_gguf_tensor_count(self._h))
+
+    def info(self, i: int) -> dict:
+        name, t, nd = ctypes.c_char_p(), ctypes.c_int(), ctypes.c_int()
+        dims = (ctypes.c_int64 * 4)()
+        off, nb = ctypes.c_uint64(), ctypes.c_uint64()
+        st = self._L.kq_gguf_tensor_info(self._h, i, ctypes.byref(name), ctypes.byref(t), ctypes.byref(nd), dims,
+                                         ctypes.byref(off), ctypes.byref(nb))
+        if st != OK:
+            raise KQError(st, "kq_gguf_tensor_info", self._L.kq_gguf_last_error().decode())
+        return dict(name=name.value.decode(), type=t.value, dims=list(dims)[:nd.value], offset=off.value,
+                    nbytes=nb.value, fmt=int(self._L.kq_gguf_kq_format(t.value)))
+
+    def find(self, name: str) -> int:
+        return int(self._L.kq_gguf_find(self._h, name.encode()))
+
+    def read(self, name_or_index) -> np.ndarray:
+        i = name_or_index if isinstance(name_or_index, int) else self.find(name_or_index)
+        nb = self.info(i)["nbytes"]
+        out = np.empty(nb, np.uint8)
+        st = self._L.kq_gguf_read(self._h, i, out.ctypes.data, nb)
+        if st != OK:
+            raise KQError(st, "kq_gguf_read", self._L.kq_gguf_last_error().decode())
+        return out
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._L.kq_gguf_close(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
 class Chain:
     """Layer chain whose weights stay in pinned host memory and stream
     through ``n_slots`` device slots (kq_chain_* in kq.h).

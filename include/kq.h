@@ -337,6 +337,44 @@ KQ_API void kq_moe_stream_destroy(kq_moe_stream* s);
 KQ_API const char* kq_moe_stream_last_error(void);
 
 /*
+ * GGUF reader (host only) — the tensor table of a GGUF model file (versions
+ * 2 and 3) and its tensors' bytes on demand, so that a weight stored in the
+ * file can be handed to the GEMV entry points.  A 2-D weight of N rows and
+ * K inputs has dims {K, N} (dims[0] innermost); its rows follow one another
+ * in the file, which is libkq's matrix layout: copy its bytes to the device
+ * (16-byte aligned) and call kq_gemv(W, kq_gguf_kq_format(type), N, K, ...).
+ * The pages load GGUF files ("Out-of-core LLM inference engine ...",
+ * Results: Q4_K_M; "RunNburn - Run a 295B MoE from a 98GB GGUF ...") but
+ * print no format; this follows the public GGUF layout.
+ *
+ * kq_gguf_open: reads the header, skips the metadata (except
+ *   general.alignment) and reads the tensor table.  KQ_ERR_INVALID_ARG for a
+ *   missing file, a bad magic or version, a truncated or malformed table, or
+ *   tensor data past the end of the file.  The object keeps the file open
+ *   until kq_gguf_close; one object must not be read by two threads at once.
+ * kq_gguf_tensor_info: name (valid until close), ggml type id, dims (unused
+ *   ones 1), absolute file offset and byte size (0 for a type this reader
+ *   does not size: F32, F16, BF16, Q8_0 and Q2_K..Q6_K are sized).
+ * kq_gguf_find: index of the named tensor, or -1.
+ * kq_gguf_kq_format: the KQ_FMT_* of a ggml type id (Q4_K 12, Q5_K 13,
+ *   Q6_K 14, Q2_K 10, Q3_K 11, Q8_0 8), 0 for none.
+ * kq_gguf_read: copies tensor i (nbytes must equal its size) into dst
+ *   (HOST memory, page-locked or not).
+ */
+typedef struct kq_gguf kq_gguf;
+
+KQ_API int kq_gguf_open(const char* path, kq_gguf** out);
+KQ_API int kq_gguf_tensor_count(const kq_gguf* g);
+KQ_API int kq_gguf_tensor_info(const kq_gguf* g, int i, const char** name, int* ggml_type, int* n_dims,
+                               int64_t dims[4], uint64_t* file_offset, uint64_t* nbytes);
+KQ_API int kq_gguf_find(const kq_gguf* g, const char* name);
+KQ_API int kq_gguf_kq_format(int ggml_type);
+KQ_API int kq_gguf_read(const kq_gguf* g, int i, void* dst, uint64_t nbytes);
+KQ_API void kq_gguf_close(kq_gguf* g);
+/* Text describing the last GGUF failure on the calling thread. */
+KQ_API const char* kq_gguf_last_error(void);
+
+/*
  * kq_unpack — debug: the integer fields of n_blocks consecutive super-blocks
  * as the GEMV kernels decode them (for bit-exact comparison).
  *   q:  n_blocks*256 bytes, quant of weight i of block b at q[256b+i]
