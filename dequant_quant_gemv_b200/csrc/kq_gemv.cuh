@@ -931,12 +931,15 @@ __device__ __forceinline__ void q2k_unit_int(uint32_t row0, int row_bytes, int b
         dd[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw & 0xFFFFu)));
         dm[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw >> 16)));
     }
-    float y[2] = {0.f, 0.f};
+    // per 32-group j and row: the exact int32 sums sc*S and m*(16-sum) of
+    // its two 16-groups (|.| < 2^31), folded into fp32 once per j
+    float yd[2] = {0.f, 0.f}, ym[2] = {0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * j);  // X, P, 16-sums
         const float P = __uint_as_float(info.y);
         const float Pj = P * (1.0f / static_cast<float>(1 << (2 * j)));  // undoes the 4^j of the in-place codes
+        int isum[2] = {0, 0}, msum[2] = {0, 0};
 #pragma unroll
         for (int sh = 0; sh < 2; ++sh) {
             const uint4 xh = ld_s128(xr + kXGroupBytes * j + 16 * sh);
@@ -952,19 +955,23 @@ __device__ __forceinline__ void q2k_unit_int(uint32_t row0, int row_bytes, int b
                     lo[r] = dp4a_uu(q, u4w(xl, m), lo[r]);
                 }
             }
-            const float x16 = static_cast<float>(static_cast<int>(sh ? info.w : info.z)) * P;
+            const int x16 = static_cast<int>(sh ? info.w : info.z);
             const int g = 2 * j + sh;  // group within the half
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                const uint32_t sb = (sw[r][g >> 2] >> (8 * (g & 3))) & 0xFFu;
-                const float S = static_cast<float>(hi[r] * 256 + static_cast<int>(lo[r]));
-                y[r] = fmaf(dd[r] * static_cast<float>(sb & 15u) * Pj, S, y[r]);
-                y[r] = fmaf(-dm[r] * static_cast<float>(sb >> 4), x16, y[r]);
+                const int sb = static_cast<int>((sw[r][g >> 2] >> (8 * (g & 3))) & 0xFFu);
+                isum[r] += (sb & 15) * (hi[r] * 256 + static_cast<int>(lo[r]));
+                msum[r] += (sb >> 4) * x16;
             }
         }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            yd[r] = fmaf(Pj, static_cast<float>(isum[r]), yd[r]);
+            ym[r] = fmaf(P, static_cast<float>(msum[r]), ym[r]);
+        }
     }
-    out[0][0] = y[0];
-    out[1][0] = y[1];
+    out[0][0] = dd[0] * yd[0] - dm[0] * ym[0];
+    out[1][0] = dd[1] * yd[1] - dm[1] * ym[1];
 }
 
 // Q3_K unit, one column, on DP4A: row pair at row0, super-block b (110
@@ -974,9 +981,11 @@ __device__ __forceinline__ void q2k_unit_int(uint32_t row0, int row_bytes, int b
 // its start (one word more than it needs) and every word rebuilt by a byte
 // permute whose selector is picked by b's parity.  Weight 128H + 32j + l:
 // q + 4 = (bits 2j of quant byte 32H + l) | (bit 4H + j of hmask[l]) << 2,
-// in 0..7, assembled in place as 4^j * (q + 4) (the 4^-j folded into the
-// group's factor); per 16-weight group the exact S = sum (q+4)*xi -
-// 4*(16-sum of xi) and y += d*(v - 32)*P*S with v the group's 6-bit scale.
+// in 0..7, assembled in place as 4^jj * (q + 4) with jj = min(j, 2) (the
+// 4^-jj folded into the group's factor).  Per 16-weight group the exact
+// S = sum (q+4)*xi - 4*(16-sum of xi); per 32-group the int32 sum of
+// (v - 32)*S over its two groups (|.| < 2^31, v the 6-bit scale); y = d *
+// sum over 32-groups of P*(that sum), in fp32.
 __device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
                                              float (&out)[2][1]) {
     const bool odd = b & 1;
@@ -1004,12 +1013,15 @@ __device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b
         hs[r] = __byte_perm(L[2], L[3], sel) >> (4 * H);
         dd[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(L[3] >> (odd ? 16 : 0))));
     }
+    // per 32-group j and row: the exact int32 sum of (v - 32)*S over its two
+    // 16-groups (|.| < 2^31), folded into fp32 once per j
     float y[2] = {0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * j);  // X, P, 16-sums
         const int jj = j < 3 ? j : 2;  // the plane's codes sit at bits 2jj..2jj+2
         const float Pj = __uint_as_float(info.y) * (1.0f / static_cast<float>(1 << (2 * jj)));
+        int isum[2] = {0, 0};
 #pragma unroll
         for (int sh = 0; sh < 2; ++sh) {
             const uint4 xh = ld_s128(xr + kXGroupBytes * j + 16 * sh);
@@ -1038,14 +1050,15 @@ __device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b
             for (int r = 0; r < 2; ++r) {
                 const uint32_t lo4 = (sc[r][g >> 2] >> (8 * (g & 3))) & 15u;
                 const uint32_t hi2 = (hs[r] >> (8 * (g & 3) + 2 * (g >> 2))) & 3u;
-                const float v = static_cast<float>(static_cast<int>(lo4 | (hi2 << 4)) - 32);
-                const int S = hi[r] * 256 + static_cast<int>(lo[r]) - 4 * x16;
-                y[r] = fmaf(dd[r] * v * Pj, static_cast<float>(S), y[r]);
+                const int v = static_cast<int>(lo4 | (hi2 << 4)) - 32;
+                isum[r] += v * (hi[r] * 256 + static_cast<int>(lo[r]) - 4 * x16);
             }
         }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) y[r] = fmaf(Pj, static_cast<float>(isum[r]), y[r]);
     }
-    out[0][0] = y[0];
-    out[1][0] = y[1];
+    out[0][0] = dd[0] * y[0];
+    out[1][0] = dd[1] * y[1];
 }
 
 // Q8_0 unit, one column, on DP4A: row pair at row0, unit b of eight
