@@ -101,13 +101,6 @@ static int next_pow2(int v) {
 
 static size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
 
-// Ring depth for `ng` consumer groups.  Two groups take alternate stages, so
-// with an even depth every slot belongs to one group, which has consumed the
-// slot's previous stage before it waits on the slot again.  With an odd
-// depth a slot alternates between the groups, and a group could wait on it
-// while the other group's stage in it has not landed yet: its parity wait
-// (which cannot tell phase k from phase k + 2) would then return at once.
-static size_t ring_depth(size_t ns, int ng) { return ng == 2 && ns > 2 && ns % 2 == 1 ? ns - 1 : ns; }
 
 int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     DevInfo di;
@@ -167,7 +160,6 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     const int64_t per_cta = (P + grid / a.ksplit - 1) / (grid / a.ksplit);
     const int64_t need = (per_cta + a.ps - 1) / a.ps + (a.n_seg > 1 ? 1 : 0);
     if (static_cast<int64_t>(ns) > need) ns = need < 2 ? 2 : static_cast<size_t>(need);
-    ns = ring_depth(ns, ng);
     a.nstage = static_cast<int>(ns);
     a.stage_bytes = static_cast<int>(stage);
     a.wp_offset = static_cast<int>(head);
@@ -313,7 +305,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     if (L.fixed + 2 * L.stage > limit)
         return fail(KQ_ERR_UNSUPPORTED, "K=%lld with %d columns needs %zu bytes of shared memory (limit %zu)",
                     (long long)a.K, 4 * nt, L.fixed + 2 * L.stage, limit);
-    size_t ns = ring_depth((limit - L.fixed) / L.stage, ng);
+    size_t ns = (limit - L.fixed) / L.stage;
     if (ns > kMaxStages) ns = kMaxStages;
     const int64_t rps = (a.N + 1) / 2;
     const int64_t tiles = (rps + 7) / 8;  // 16-row stages of the matrix
@@ -329,7 +321,6 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     const int64_t per_cta = (rps + grid / S - 1) / (grid / S);
     const int64_t need = (per_cta + 7) / 8 + 1;
     if (static_cast<int64_t>(ns) > need) ns = need < 2 ? 2 : static_cast<size_t>(need);
-    ns = ring_depth(ns, ng);
     a.ksplit = S;
     a.nbs = nbs;
     a.cluster = cl ? 1 : 0;
@@ -731,7 +722,6 @@ int kq_gemv_steps(const kq_step* steps, int n_steps, kq_stream_t stream) {
             return fail(KQ_ERR_UNSUPPORTED, "steps %d..%d need %zu bytes of shared memory together (limit %zu)",
                         run.front(), run.back(), fixed + 2 * slot, limit);
         if (ns > kMaxStages) ns = kMaxStages;
-        ns = ring_depth(ns, 2);  // the steps kernel runs two consumer groups
         op.args.ns = static_cast<int>(ns);
         op.args.slot_bytes = static_cast<int>(slot);
         op.args.wp_offset = kHeadBytes;

@@ -1363,6 +1363,13 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             staged_seg = st.seg;
         }
         const int slot = it.slot;
+        // Two groups take alternate stages.  With an odd ring depth a slot
+        // alternates between them, so a group first waits until the other
+        // group has released the slot's previous stage: only then can the
+        // parity wait on `full` not pass on a phase two ahead (it cannot
+        // tell phase k from phase k + 2).
+        if (NG == 2 && (ns & 1) && it.count > ns && !mbar_wait_bounded(&empty[slot], it.phase ^ 1u, abort_flag))
+            raise_fault(a, abort_flag, 6);
         if (!mbar_wait_bounded(&full[slot], it.phase, abort_flag)) raise_fault(a, abort_flag, 6);
         float out[2][NCOL];
 #pragma unroll

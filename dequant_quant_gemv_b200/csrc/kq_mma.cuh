@@ -744,6 +744,10 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
             const int slot = it.slot;
             const int si = it.count - 1;  // this stage's index in the CTA's sequence
             if (NG == 2 && (si & 1) != g_id) continue;
+            // with an odd ring depth, first the other group's release of the
+            // slot's previous stage (see gemv_kernel)
+            if (NG == 2 && (ns & 1) && si >= ns && !mbar_wait_bounded(&empty[slot], it.phase ^ 1u, abort_flag))
+                raise_fault(a, abort_flag, 6);
             if (!mbar_wait_bounded(&full[slot], it.phase, abort_flag)) raise_fault(a, abort_flag, 6);
             float ys[2][NT], ym[2][NT];
 #pragma unroll

@@ -215,6 +215,10 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
             const int nrp = rp1 - off < s.ps ? rp1 - off : s.ps;
             const int64_t row0 = 2 * static_cast<int64_t>(off);
             const int nrows = static_cast<int>(s.N - row0 < 2 * nrp ? s.N - row0 : 2 * nrp);
+            // with an odd ring depth, first the other group's release of the
+            // slot's previous stage (see gemv_kernel)
+            if (NG == 2 && (ns & 1) && k >= ns && !mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag))
+                raise_fault(fa, abort_flag, 6);
             if (!mbar_wait_bounded(&full[slot], phase, abort_flag)) raise_fault(fa, abort_flag, 6);
             float out[2][1] = {{0.f}, {0.f}};
             const bool work = u_active && u_rp < nrp && !*abort_flag;
