@@ -573,37 +573,18 @@ def h2d_peak_gbs(torch, nbytes=512 << 20, reps=5):
 # the profiles), keyed by (format, N, K, columns).  Valid only for the kernel sources they
 # were taken on: any change to csrc/ changes the hash and the bench reports
 # traffic as null until the counters are taken again.
-TRAFFIC_SOURCES = "a923a337f8a53c4d"
+TRAFFIC_SOURCES = "856d8462f0a836b9"
 TRAFFIC = {
-    # gemv_kernel (single column): the 8B-shaped chains' matrices
-    ("q4_k", 6144, 4096, 1): 14_238_280 + 24,
-    ("q4_k", 4096, 4096, 1): 9_520_896,
-    ("q4_k", 28672, 4096, 1): 66_142_928 + 3_160,
-    ("q6_k", 4096, 14336, 1): 48_293_056 + 64,
-    ("q4_k", 4096, 14336, 1): 33_153_792,
-    ("q5_k", 6144, 4096, 1): 17_389_312,
-    ("q5_k", 4096, 4096, 1): 11_616_768,
-    ("q5_k", 28672, 4096, 1): 80_825_600 + 276_736,
-    ("q2_k", 6144, 4096, 1): 8_340_224,
-    ("q2_k", 4096, 4096, 1): 5_587_968,
-    ("q2_k", 28672, 4096, 1): 38_618_112,
-    ("q3_k", 4096, 14336, 1): 25_360_128,
-    ("q3_k", 6144, 4096, 1): 10_900_736,
-    ("q3_k", 4096, 4096, 1): 7_291_904,
-    ("q3_k", 28672, 4096, 1): 50_545_664,
-    # mma_kernel (tensor cores), 2, 4 and 8 columns
-    ("q4_k", 6144, 4096, 2): 14_240_256,
-    ("q4_k", 4096, 4096, 2): 9_521_920,
-    ("q4_k", 28672, 4096, 2): 66_145_024 + 256,
-    ("q6_k", 4096, 14336, 2): 48_343_808,
-    ("q4_k", 6144, 4096, 4): 14_273_280,
-    ("q4_k", 4096, 4096, 4): 9_554_432,
-    ("q4_k", 28672, 4096, 4): 66_177_792 + 8_448,
-    ("q6_k", 4096, 14336, 4): 48_454_656,
+    # gemv_kernel (single column, DP4A): the 8B-shaped chain's matrices
+    ("q4_k", 6144, 4096, 1): 14_238_352 + 16,
+    ("q4_k", 4096, 4096, 1): 9_519_656,
+    ("q4_k", 28672, 4096, 1): 66_142_952 + 4_448,
+    ("q6_k", 4096, 14336, 1): 48_292_560 + 8,
+    # mma_kernel (tensor cores), 8 columns
     ("q4_k", 6144, 4096, 8): 14_353_920,
     ("q4_k", 4096, 4096, 8): 9_634_816,
     ("q4_k", 28672, 4096, 8): 66_258_176,
-    ("q6_k", 4096, 14336, 8): 48_694_272,
+    ("q6_k", 4096, 14336, 8): 48_694_528,
 }
 
 
