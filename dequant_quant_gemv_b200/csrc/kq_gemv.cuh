@@ -633,23 +633,25 @@ __device__ __noinline__ void stage_x_pro(const ProStage p, uint32_t xs, int ct, 
                    ct >> 5, ct & 31, bar, nthr, 0);
 }
 
-// ------------------------- single column, Q4_K and Q5_K: integer dot path
+// ------------------------------- single column: the integer dot path
 //
-// One Q4_K or Q5_K column runs its inner products on DP4A (four byte products per
-// instruction, exact int32 sums).  The activations of each group of 32
-// consecutive weights are scaled by a power of two 2^sh that puts the
-// group's largest |x| in [2^13, 2^14), rounded to integers xi (|xi| <= 2^14)
-// and stored as a signed high byte xi >> 8 and an unsigned low byte xi & 255
-// (xi = 256*hi + lo).  Per group the staging also keeps P = 2^-sh and
-// Xg = P * sum of the xi (an exact integer sum, |sum| <= 2^19).  A
-// sub-block's sum S of q*xi is then exact (|S| <= 31 * 32 * 2^14 < 2^24 for
-// Q5_K's 5-bit codes, so exact in fp32 too), and y = sum over sub-blocks of d*sc*P*S - dmin*m*Xg in fp32: the
+// One column of any format runs its inner products on DP4A (four byte
+// products per instruction, exact int32 sums).  The activations of each
+// group of 32 consecutive weights are scaled by a power of two 2^sh that
+// puts the group's largest |x| in [2^13, 2^14), rounded to integers xi
+// (|xi| <= 2^14) and stored as a signed high byte xi >> 8 and an unsigned
+// low byte xi & 255 (xi = 256*hi + lo).  Per group the staging also keeps
+// P = 2^-sh and Xg = P * sum of the xi (an exact integer sum, |sum| <=
+// 2^19), and for formats whose scales cover 16 weights the integer sums of
+// the group's two halves.  A sub-block's sum S of q*xi is then exact (for
+// Q5_K's 5-bit codes |S| <= 31 * 32 * 2^14 < 2^24, so exact in fp32 too),
+// and for Q4_K y = sum over sub-blocks of d*sc*P*S - dmin*m*Xg in fp32: the
 // exact dot product of the dequantised weights with the rounded activations
-// P*xi, up to fp32 rounding of the per-sub-block terms.  |x - P*xi| <= P/2
-// <= 2^-14 * (largest |x| of the group), so |y - y_exact| <= 2^-14 * sum
-// over groups of (max_g |x|) * sum_{i in g} |w_i|.  All-zero quants with
-// zero mins give y = 0 exactly.  (A Q6_K variant measured slower than its
-// fp32 units: its 6-bit codes cost more to assemble than the DP4A saves.)
+// P*xi, up to fp32 rounding of the per-sub-block terms (the other formats'
+// units state their own forms).  |x - P*xi| <= P/2 <= 2^-14 * (largest |x|
+// of the group), so |y - y_exact| <= 2^-14 * sum over groups of
+// (max_g |x|) * sum_{i in g} |w_i|.  All-zero quants with zero mins give
+// y = 0 exactly.
 
 constexpr int kXGroupBytes = 64;  // 32 high bytes, then 32 low bytes
 constexpr int kXInfoBytes = 16;   // Xg, P; with S16 also the int sums of xi 0..15 and 16..31
@@ -1334,7 +1336,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     constexpr bool INT = NCOL == 1;
     const uint32_t xcopy = INT ? kXRegionBytes * 2 * nb : 4 * NCOL * xcs;
     const uint32_t xs_s = smem_u32(xs) + (shared_x ? 0 : g * xcopy);
-    const uint32_t xri = x_region(xs_s, u_b, u_H);  // this lane's integer region (Q4_K)
+    const uint32_t xri = x_region(xs_s, u_b, u_H);  // this lane's integer region
     const uint32_t sbuf_s = smem_u32(sbuf), wp_s = smem_u32(wp) + 4 * g * wp_group;
     const uint32_t xr = xs_s + 4 * (region * kRegion);
 

@@ -35,7 +35,7 @@ struct GemvArgs {
     float* partial;          // ksplit x ncol_real x N partial sums (ksplit > 1)
     // schedule (from plan_gemv)
     int ps;                  // row pairs per stage
-    int lanes_per_rp;        // Q4_K: lanes per row pair; Q6_K: per row pair and warp
+    int lanes_per_rp;        // lanes per row pair (several-column Q6_K: per row pair and warp)
     int parts;               // partial sums per row pair
     int nstage;
     int stage_bytes;
