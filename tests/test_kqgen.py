@@ -3,6 +3,7 @@ and the value distributions the workloads specify (Q4_K quants uniform
 0..15, scales/mins uniform 0..63, d/dmin = |N(0,1)|*1e-3 in fp16, x ~ N(0,1)
 fp32; Q6_K quants 0..63, scales -64..63)."""
 import numpy as np
+import pytest
 
 import kqgen
 import oracle
@@ -37,6 +38,38 @@ def test_fill_is_thread_count_independent_and_matches_draw_pack():
     # offset fill = tail of the full fill
     tail = kqgen.q4k_fill(99, 10, b0=nb - 10, nthreads=2)
     assert np.array_equal(tail, a[(nb - 10) * 144:])
+
+
+@pytest.mark.parametrize("fmt", ["q5_k", "q2_k", "q3_k", "q8_0"])
+def test_fill_matches_draw_pack_other_formats(fmt):
+    nb = 29
+    draw = {"q5_k": kqgen.q5k_draw, "q2_k": kqgen.q2k_draw, "q3_k": kqgen.q3k_draw, "q8_0": kqgen.q80_draw}[fmt]
+    pack = {"q5_k": kqgen.q5k_pack, "q2_k": kqgen.q2k_pack, "q3_k": kqgen.q3k_pack, "q8_0": kqgen.q80_pack}[fmt]
+    a = kqgen.fill(fmt, 77, nb, nthreads=1)
+    assert np.array_equal(a, kqgen.fill(fmt, 77, nb, nthreads=5))
+    assert np.array_equal(a, pack(**draw(77, nb)))
+    assert a.size == nb * kqgen.block_bytes(fmt)
+
+
+def test_other_format_distributions():
+    """The fill draws every value of each field's range, uniformly."""
+    lg = kqgen.q5k_draw(9, 2000)
+    c = np.bincount(lg["q"].ravel(), minlength=32)
+    assert c.size == 32 and np.all(np.abs(c / c.mean() - 1) < 0.05)
+    lg = kqgen.q2k_draw(10, 2000)
+    for f, n in (("q", 4), ("sc", 16), ("m", 16)):
+        c = np.bincount(lg[f].ravel(), minlength=n)
+        assert c.size == n and np.all(np.abs(c / c.mean() - 1) < 0.1), f
+    lg = kqgen.q3k_draw(11, 2000)
+    c = np.bincount(lg["q"].astype(int).ravel() + 4, minlength=8)
+    assert c.size == 8 and np.all(np.abs(c / c.mean() - 1) < 0.05)
+    c = np.bincount(lg["v"].ravel(), minlength=64)
+    assert c.size == 64 and np.all(np.abs(c / c.mean() - 1) < 0.2)
+    lg = kqgen.q80_draw(12, 2000)
+    c = np.bincount(lg["q"].astype(int).ravel() + 128, minlength=256)
+    assert c.size == 256 and np.all(np.abs(c / c.mean() - 1) < 0.1)
+    d = lg["d"].view(np.float16).astype(np.float64)
+    assert np.all(d >= 0) and abs(d.mean() / 1e-3 - np.sqrt(2 / np.pi)) < 0.03
 
 
 def test_q4k_distributions():

@@ -513,7 +513,7 @@ def test_swiglu_hand_values_and_identities():
     assert np.allclose(oracle.swiglu(np.concatenate([gate, up])), s * up, rtol=1e-15)
 
 
-@pytest.mark.parametrize("fmt", ["q4_k", "q6_k"])
+@pytest.mark.parametrize("fmt", ["q4_k", "q6_k", "q5_k", "q2_k", "q3_k", "q8_0"])
 def test_gemv_fused_reduces_to_plain_forms(fmt):
     """The fused oracle with no prologue equals the plain GEMV (float inputs
     widen exactly); with a prologue it is the plain product of the
