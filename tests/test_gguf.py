@@ -38,10 +38,11 @@ META = [("general.architecture", gw.STRING, "llama"),
 
 
 @pytest.mark.parametrize("alignment", [32, 64, 256])
-def test_table_sizes_and_bytes(tmp_path, alignment):
+@pytest.mark.parametrize("version", [2, 3])
+def test_table_sizes_and_bytes(tmp_path, alignment, version):
     ts = _tensors()
     p = str(tmp_path / "m.gguf")
-    gw.write(p, ts, META, alignment=alignment)
+    gw.write(p, ts, META, alignment=alignment, version=version)
     g = kq.GGUF(p)
     assert len(g) == len(ts)
     sizes = {12: 144 * 2 * 8, 14: 210 * 8 * 4, 8: 34 * 8 * 3, 0: 4 * 512, 2: 0}
