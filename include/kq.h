@@ -324,6 +324,7 @@ KQ_API int kq_moe_gemv(const void* W_experts, int fmt, int E, int64_t N, int64_t
  * kq_moe_stream_wait: host-side polling until the last run finished;
  *   KQ_ERR_TIMEOUT after timeout_ms (negative: no limit).
  * kq_moe_stream_destroy: waits for the copies, frees slots, stream, events.
+ * One object must not be used by two threads at once.
  */
 typedef struct kq_moe_stream kq_moe_stream;
 
