@@ -140,59 +140,98 @@ WORKLOADS = {
 
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clock / throttle samples while the timed region runs."""
+    """SM clock, power and throttle-reason samples taken while the timed
+    region runs: NVML polled every millisecond from a thread (nvidia-smi at
+    50 ms if NVML is missing).  Only samples between start() and stop() --
+    the timed region -- are kept."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.active = False
+        self.done = False
+        self.mx = None
+        self.nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.mx = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.nvml = None
+
+    def _sample_nvml(self):
+        n = self.nvml
+        try:
+            fn = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or n.nvmlDeviceGetCurrentClocksThrottleReasons
+            return (float(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)),
+                    n.nvmlDeviceGetPowerUsage(self.h) / 1000.0, int(fn(self.h)))
+        except Exception:
+            return None
+
+    def _loop(self):
+        while not self.done:
+            if self.active:
+                smp = self._sample_nvml()
+                if smp is not None:
+                    self.samples.append(smp)
+            time.sleep(0.001)
+
+    def _smi_loop(self):
+        fields = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
+        try:
+            proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={fields}",
+                                     "--format=csv,noheader,nounits", "-lms", "50"],
+                                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            return
+        self.proc = proc
+        for line in proc.stdout:
+            if not self.active:
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            try:
+                bits = sum(v for (nm, v), st in zip(self.REASONS.items(), parts[3:7]) if st.lower() == "active")
+                self.mx = float(parts[1])
+                self.samples.append((float(parts[0]), float(parts[2]), bits))
+            except (ValueError, IndexError):
+                continue
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-            time.sleep(0.2)
-        except (FileNotFoundError, OSError):
-            self.proc = None
+        self.proc = None
+        self.t = threading.Thread(target=self._loop if self.nvml else self._smi_loop, daemon=True)
+        self.t.start()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def start(self):
+        self.active = True
+
+    def stop(self):
+        self.active = False
 
     def __exit__(self, *exc):
+        self.done = True
+        self.active = False
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        self.t.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons, pw = [], None, set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-                pw.append(float(parts[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[3:7]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
-                "power_w_max": max(pw) if pw else None, "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [a for a, _, _ in self.samples]
+        pw = [b for _, b, _ in self.samples]
+        reasons = sorted(nm for nm, bit in self.REASONS.items() if any(r & bit for _, _, r in self.samples))
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": self.mx,
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(sm),
+                "source": "nvml, 1 ms" if self.nvml else "nvidia-smi, 50 ms"}
 
 
 # --------------------------------------------------------------- workloads
@@ -520,6 +559,52 @@ class MoEStreamed(MoE):
         return {}
 
 
+CHAIN_BASE = {"llama8b_chain": "llama8b", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
+              "llama8b_layer_fused_steps": "llama8b", "llama8b_q5k_chain": "llama8b_q5k",
+              "verify8b_q5k_k8": "llama8b_q5k", "llama8b_q2k_chain": "llama8b_q2k",
+              "llama8b_q3k_chain": "llama8b_q3k", "llama8b_q80_chain": "llama8b_q80",
+              "llama70b_resident": "llama70b", "llama70b_resident_steps": "llama70b",
+              "llama70b_stream": "llama70b", "llama70b_stream_20gb": "llama70b"}
+
+
+def workload_spec(name):
+    """(spec, columns) of a chain-shaped workload, or (None, 1) for MoE."""
+    if name in ("moe30b", "moe30b_stream"):
+        return None, 1
+    if name.startswith("verify8b_k"):
+        return chain_spec("llama8b"), int(name[len("verify8b_k"):])
+    k = 8 if name == "verify8b_q5k_k8" else 1
+    return chain_spec(CHAIN_BASE.get(name, name)), k
+
+
+def workload_config(name, world):
+    """The `config` of the JSON line, computed on the host from the shapes
+    alone, so that both arms (the GPU path and the oracle) report the same
+    keys and values."""
+    spec, k = workload_spec(name)
+    if spec is None:
+        c = MOE30B
+        weight_bytes = c["layers"] * c["top"] * (2 * c["ffn"] * row_bytes("q4_k", c["hidden"])
+                                                + c["hidden"] * row_bytes("q4_k", c["ffn"]))
+        launches = 2 * c["layers"]
+    else:
+        weight_bytes = sum(N * row_bytes(f, K) for mats in spec for (_, f, N, K, _) in mats)
+        launches = sum(len(m) for m in spec)
+        if name.endswith("_steps"):
+            launches = -(-launches // 16)
+    return {"workload": name, "desc": WORKLOADS[name], "weight_bytes_per_step": weight_bytes,
+            "launches_per_step": launches, "columns": k, "batch": 1, "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (no flush)" if weight_bytes > 2 * 126e6 else "rotating copies"}
+
+
+def dtype_of(name):
+    """The arithmetic the path computes in (fp32 accumulation throughout)."""
+    spec, k = workload_spec(name)
+    if k == 1:
+        return "f32 acc; activations int14 per group of 32, exact int32 sub-block sums (DP4A)"
+    return "f32 acc; exact fp16 weight operands x two-term fp16 activations (22 bits), tensor cores"
+
+
 def make_workload(name, torch, kq, kqgen, seed):
     if name in ("llama8b_chain", "llama8b_chain_steps"):
         return Resident(torch, kq, kqgen, chain_spec("llama8b"), seed, steps=name.endswith("_steps"))
@@ -566,6 +651,30 @@ def h2d_peak_gbs(torch, nbytes=512 << 20, reps=5):
         best = max(best, nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9)
     del h, d
     return best
+
+
+def read_roofline(torch, kq, nbytes=2 << 30, reps=5):
+    """Read-only HBM bandwidth (GB/s) of a 2 GiB buffer read once, best of
+    `reps`, by the two probes of kq_read_probe: 16-byte loads from a full
+    grid, and the GEMV kernels' own bulk-copy ring with no work per stage."""
+    buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    buf.random_(0, 255)
+    out = torch.zeros(1, dtype=torch.int32, device="cuda")
+    res = {}
+    for mode, name in ((0, "loads"), (1, "bulk_ring")):
+        kq.read_probe(buf, mode, out)
+        torch.cuda.synchronize()
+        best = 0.0
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            kq.read_probe(buf, mode, out)
+            e1.record()
+            torch.cuda.synchronize()
+            best = max(best, nbytes / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+        res[name] = round(best, 1)
+    del buf
+    return res
 
 
 # -------------------------------------------------- measured DRAM traffic
@@ -687,11 +796,13 @@ def bench_kq(args, rank, world):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
         torch.cuda.synchronize()
+        clk.start()
         e0.record(stream)
         for _ in range(args.steps):
             run_step()
         e1.record(stream)
         torch.cuda.synchronize()
+        clk.stop()
     ms = max_over_ranks(e0.elapsed_time(e1), "cuda")
     ms_step = ms / args.steps
     k = getattr(wl, "k", 1)
@@ -765,13 +876,10 @@ def bench_kq(args, rank, world):
     result = {
         "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, kqgen)",
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype_of(args.workload),
+        "data": "synthetic (seeded, kqgen)",
         "tok_per_s": round(tok_s, 3), "frac_of_hbm_peak": round(gbs / world / hbm, 4),
-        "config": {"workload": args.workload, "desc": WORKLOADS[args.workload],
-                   "weight_bytes_per_step": wl.weight_bytes,
-                   "launches_per_step": wl.launches_per_step if getattr(wl, "use_steps", False) else len(wl.launches),
-                   "columns": k, "batch": 1, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (no flush)" if wl.weight_bytes > 2 * 126e6 else "rotating copies"},
+        "config": workload_config(args.workload, world),
         "e2e": {"value": round(job_rate(wl.weight_bytes, args.steps, world, ems) / 1e9, 2), "unit": "GB/s",
                 "tok_per_s": round(job_rate(k, args.steps, world, ems), 3),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -783,11 +891,16 @@ def bench_kq(args, rank, world):
         dk = per_kind[dom]
         kname = ("mma_kernel (tensor cores)" if k >= 2 else
                  "steps_kernel (multi-step launch)" if getattr(wl, "use_steps", False) else "gemv_kernel")
+        rd = read_roofline(torch, kq)
+        rpk = max(rd.values())
         result["roofline"] = {"bound": "hbm", "kernel": f"{kname} {dk['fmt']} {dom} {dk['N']}x{dk['K']}",
-                              "achieved": dk["gbs"], "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
-                              "frac": round(dk["gbs"] / hbm, 4),
+                              "achieved": dk["gbs"], "peak": hbm, "peak_source": f"{peak_src} copy (read+write)",
+                              "unit": "GB/s", "frac": round(dk["gbs"] / hbm, 4),
+                              "read_peak": rd, "frac_of_read_peak": round(dk["gbs"] / rpk, 4),
+                              "frac_of_nominal_8tbs": round(dk["gbs"] / 8000.0, 4),
                               "traffic": measured_traffic(dk["fmt"], dk["N"], dk["K"], k),
                               "algorithmic_bytes": dk["bytes"]}
+        result["frac_of_read_peak"] = round(gbs / world / rpk, 4)
         result["kernels"] = per_kind
     if isinstance(wl, (Streamed, MoEStreamed)):
         pk = h2d_peak_gbs(torch)
@@ -803,55 +916,63 @@ def bench_kq(args, rank, world):
     return result
 
 
-def cpu_baseline(args, budget_s=15.0):
+def cpu_baseline(args, budget_s=15.0, single_s=5.0):
     """The oracle as it stands, on a bounded sample of the workload: the
-    first rows of each matrix kind, timed on all host cores."""
+    first rows of each matrix of the leading layers, timed on all host cores
+    (OpenMP over rows) and, on a smaller share of the same sample, on one
+    core.  For the 70B-shaped chains the sample is at most the first 4
+    layers and tok/s is extrapolated from the sample's byte rate to the
+    whole chain's bytes per token."""
     import kqgen
     import oracle
 
-    if args.workload in ("moe30b", "moe30b_stream"):
+    spec, _ = workload_spec(args.workload)
+    if spec is None:
         spec = [[("moe_gate_up", "q4_k", 2 * MOE30B["ffn"], MOE30B["hidden"], 0),
                  ("moe_down", "q4_k", MOE30B["hidden"], MOE30B["ffn"], 1)]] * MOE30B["layers"]
-        per_token = MOE30B["layers"] * MOE30B["top"] * (2 * MOE30B["ffn"] * row_bytes("q4_k", MOE30B["hidden"])
-                                                        + MOE30B["hidden"] * row_bytes("q4_k", MOE30B["ffn"]))
-    else:
-        base = {"llama8b_chain": "llama8b", "llama8b_q5k_chain": "llama8b_q5k", "verify8b_q5k_k8": "llama8b_q5k",
-                "llama8b_q2k_chain": "llama8b_q2k", "llama8b_q3k_chain": "llama8b_q3k",
-                "llama8b_q80_chain": "llama8b_q80", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
-                "llama8b_layer_fused_steps": "llama8b", "llama70b_resident": "llama70b",
-                "llama70b_resident_steps": "llama70b", "llama70b_stream": "llama70b", "llama70b_stream_20gb": "llama70b"}
-        name = base.get(args.workload, "llama8b" if args.workload.startswith("verify") else args.workload)
-        spec = chain_spec(name)
-        per_token = sum(N * row_bytes(f, K) for mats in spec for (_, f, N, K, _) in mats)
+    per_token = workload_config(args.workload, 1)["weight_bytes_per_step"]
+    max_layers = 4 if CHAIN_BASE.get(args.workload) == "llama70b" else len(spec)
     cores = len(os.sched_getaffinity(0))
-    done_bytes, t_total, rows_done, li = 0, 0.0, 0, 0
-    t_start = time.time()
-    while time.time() - t_start < budget_s and li < len(spec):
-        for mi, (name, fmt, N, K, slot) in enumerate(spec[li]):
-            nrows = min(N, 512)
-            W = kqgen.matrix(fmt, kqgen.tensor_seed(SEED, li, mi), nrows, K)
-            x = kqgen.normal_f32(kqgen.tensor_seed(SEED ^ 0x5A5A, li, slot), K)
-            t0 = time.perf_counter()
-            if args.workload.startswith("llama8b_layer_fused") and name != "o":
-                # the fused forms: RMSNorm (unit weights) before qkv and
-                # gate|up, the SiLU-gated product of a [g; u] input before down
-                if name == "down":
-                    gu = kqgen.normal_f32(kqgen.tensor_seed(SEED ^ 0x5A5A, li, slot), 2 * K)
-                    oracle.gemv_fused(fmt, W, nrows, K, gu, "swiglu", nthreads=cores)
+    fused = args.workload.startswith("llama8b_layer_fused")
+
+    def run(nthreads, budget):
+        done_bytes, t_total, rows_done, li = 0, 0.0, 0, 0
+        t_start = time.time()
+        while time.time() - t_start < budget and li < min(len(spec), max_layers):
+            for mi, (name, fmt, N, K, slot) in enumerate(spec[li]):
+                nrows = min(N, 512)
+                W = kqgen.matrix(fmt, kqgen.tensor_seed(SEED, li, mi), nrows, K)
+                x = kqgen.normal_f32(kqgen.tensor_seed(SEED ^ 0x5A5A, li, 0 if slot is None else slot), K)
+                t0 = time.perf_counter()
+                if fused and name != "o":
+                    # the fused forms: RMSNorm (unit weights) before qkv and
+                    # gate|up, the SiLU-gated product of a [g; u] input before down
+                    if name == "down":
+                        gu = kqgen.normal_f32(kqgen.tensor_seed(SEED ^ 0x5A5A, li, 3), 2 * K)
+                        oracle.gemv_fused(fmt, W, nrows, K, gu, "swiglu", nthreads=nthreads)
+                    else:
+                        oracle.gemv_fused(fmt, W, nrows, K, x, "rmsnorm", np.ones(K, np.float32), 1e-5,
+                                          nthreads=nthreads)
                 else:
-                    oracle.gemv_fused(fmt, W, nrows, K, x, "rmsnorm", np.ones(K, np.float32), 1e-5,
-                                      nthreads=cores)
-            else:
-                oracle.gemv(fmt, W, nrows, K, x, nthreads=cores)
-            t_total += time.perf_counter() - t0
-            done_bytes += nrows * row_bytes(fmt, K)
-            rows_done += nrows
-        li += 1
-    gbs = done_bytes / t_total / 1e9
+                    oracle.gemv(fmt, W, nrows, K, x, nthreads=nthreads)
+                t_total += time.perf_counter() - t0
+                done_bytes += nrows * row_bytes(fmt, K)
+                rows_done += nrows
+            li += 1
+        return done_bytes / t_total / 1e9, li, rows_done, done_bytes
+
+    gbs, li, rows_done, done_bytes = run(cores, budget_s)
+    gbs1, li1, rows1, bytes1 = run(1, single_s)
+    extrap = (f"; tok/s extrapolated from the sample's rate to the whole chain's {per_token / 1e9:.2f} GB per token"
+              if max_layers < len(spec) else "")
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "tok_per_s": round(gbs * 1e9 / per_token, 6),
             "sample": f"first <=512 rows of each matrix of {li} layer(s) ({rows_done} rows, "
-                      f"{done_bytes / 1e6:.1f} MB of weights), fp64 oracle, OpenMP over rows"}
+                      f"{done_bytes / 1e6:.1f} MB of weights), fp64 oracle, OpenMP over rows{extrap}",
+            "single_thread": {"value": round(gbs1, 4), "unit": "GB/s", "cores": 1,
+                              "tok_per_s": round(gbs1 * 1e9 / per_token, 6),
+                              "sample": f"first <=512 rows of each matrix of {li1} layer(s) ({rows1} rows, "
+                                        f"{bytes1 / 1e6:.1f} MB), one thread"}}
 
 
 def main():
@@ -876,7 +997,7 @@ def main():
         line = {"metric": METRIC, "value": cb["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64", "data": "synthetic (seeded, kqgen)", "impl": "reference",
-                "config": {"workload": args.workload, "desc": WORKLOADS[args.workload]},
+                "config": workload_config(args.workload, world),
                 "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)

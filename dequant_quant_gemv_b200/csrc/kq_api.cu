@@ -2,7 +2,9 @@
 // launch of the fused K-quant GEMV kernels (see include/kq.h).
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -421,8 +423,20 @@ static int plan_for(int fmt, int k, bool mma, GemvArgs& a, LaunchPlan& p) {
     return plan_gemv(fmt, padded_cols(k), a, p);
 }
 
+// kq_inject("hold@S"): the next single-column launch withholds stage S of
+// CTA 0 and gives its bounded waits 1 ms (one-shot; 0 = none).
+static std::atomic<int> g_inject_hold{0};
+constexpr unsigned long long kInjectWaitNs = 1000000ull;
+
 static int run(GemvArgs& a, int fmt, int k, bool mma, cudaStream_t stream) {
     a.ncol_real = k;
+    if (!mma && g_inject_hold.load(std::memory_order_relaxed) != 0) {
+        const int hold = g_inject_hold.exchange(0);
+        if (hold) {
+            a.test_hold = hold;
+            a.wait_ns = kInjectWaitNs;
+        }
+    }
     cudaError_t err = fault_word(&a.fault);
     if (err != cudaSuccess) return cuda_fail(err, "fault word");
     LaunchPlan p;
@@ -530,6 +544,37 @@ const char* kq_status_str(int status) {
 }
 
 const char* kq_last_error(void) { return g_last_error; }
+
+int kq_read_probe(const void* src, size_t bytes, int mode, uint32_t* out, kq_stream_t stream) {
+    g_last_error[0] = 0;
+    if (mode != 0 && mode != 1) return fail(KQ_ERR_INVALID_ARG, "unknown probe mode %d", mode);
+    if (!src || !out || !aligned(src, 16) || !aligned(out, 4) || bytes % 16 != 0)
+        return fail(KQ_ERR_INVALID_ARG, "src must be 16-byte aligned, bytes a multiple of 16, out non-NULL");
+    if (bytes == 0) return KQ_OK;
+    DevInfo di;
+    cudaError_t err = dev_info(di);
+    if (err != cudaSuccess) return cuda_fail(err, "device query");
+    err = launch_probe(src, bytes, mode, out, di.sm_count, reinterpret_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return cuda_fail(err, "probe launch");
+    return KQ_OK;
+}
+
+int kq_inject(const char* spec) {
+    g_last_error[0] = 0;
+    if (!spec || !spec[0]) {
+        g_inject_hold.store(0);
+        return KQ_OK;
+    }
+    if (strncmp(spec, "hold@", 5) == 0) {
+        char* end = nullptr;
+        const long v = strtol(spec + 5, &end, 10);
+        if (end && *end == 0 && v >= 1 && v <= 1000000) {
+            g_inject_hold.store(static_cast<int>(v));
+            return KQ_OK;
+        }
+    }
+    return fail(KQ_ERR_INVALID_ARG, "unknown injection '%s'", spec);
+}
 
 size_t kq_block_bytes(int fmt) {
     switch (fmt) {
@@ -870,14 +915,29 @@ int kq_gemv_splitk(const void* W, int fmt, int64_t N, int64_t K, const float* x,
     return run_grouped(a, fmt, k, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int kq_unpack(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d, kq_stream_t stream) {
+int kq_unpack(const void* W, int fmt, int64_t n_blocks, int8_t* q, uint8_t* sc_or_s, uint8_t* m, float* d,
+              float* dmin, kq_stream_t stream) {
+    g_last_error[0] = 0;
+    if (!known_format(fmt)) return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
+    if (n_blocks < 0) return fail(KQ_ERR_INVALID_ARG, "n_blocks < 0");
+    if (n_blocks == 0) return KQ_OK;
+    if (!W || !q || !sc_or_s || !d) return fail(KQ_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(W, 16) || !aligned(d, 4) || !aligned(dmin, 4)) return fail(KQ_ERR_INVALID_ARG, "misaligned pointer");
+    cudaError_t err = launch_unpack(static_cast<const uint8_t*>(W), fmt, n_blocks, reinterpret_cast<uint8_t*>(q),
+                                    sc_or_s, m, d, dmin, true, reinterpret_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return cuda_fail(err, "unpack launch");
+    return KQ_OK;
+}
+
+int kq_unpack_fields(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d,
+                     kq_stream_t stream) {
     g_last_error[0] = 0;
     if (!known_format(fmt)) return fail(KQ_ERR_INVALID_ARG, "unknown format %d", fmt);
     if (n_blocks < 0) return fail(KQ_ERR_INVALID_ARG, "n_blocks < 0");
     if (n_blocks == 0) return KQ_OK;
     if (!W || !q || !sc || !d) return fail(KQ_ERR_INVALID_ARG, "NULL pointer");
     if (!aligned(W, 16) || !aligned(d, 4)) return fail(KQ_ERR_INVALID_ARG, "misaligned pointer");
-    cudaError_t err = launch_unpack(static_cast<const uint8_t*>(W), fmt, n_blocks, q, sc, d,
+    cudaError_t err = launch_unpack(static_cast<const uint8_t*>(W), fmt, n_blocks, q, sc, nullptr, d, nullptr, false,
                                     reinterpret_cast<cudaStream_t>(stream));
     if (err != cudaSuccess) return cuda_fail(err, "unpack launch");
     return KQ_OK;

@@ -2,8 +2,8 @@
 // ring of device slots, overlapped with the fused GEMV kernels.
 //
 // "Out-of-core LLM inference engine written from scratch in Rust", Approach:
-// layer weights move through a ring of VRAM slots while the GPU computes
-// nearby layers; "Kortex: Streaming 70B Models on Consumer GPUs", Key
+// layers are copied into a fixed set of device slots and run while other
+// layers compute; "Kortex: Streaming 70B Models on Consumer GPUs", Key
 // components 2 (the streaming pipeline overlaps transfers with compute).
 //
 // Schedule for layer l in slot s = l % n_slots (everything is enqueued up
@@ -223,6 +223,12 @@ KQ_API int kq_chain_run(kq_chain* c, const float* const* x, float* const* y, kq_
     cudaError_t err = cudaEventRecord(c->done, cs);
     if (err == cudaSuccess) err = cudaStreamWaitEvent(c->copy, c->done, 0);
     if (err != cudaSuccess) return chain_fail(KQ_ERR_CUDA, "stream ordering", err);
+    // A run that stops part-way re-records `done` on the compute stream
+    // first, so that kq_chain_wait covers every GEMV already queued.
+    auto stop = [&](int status, const char* what, cudaError_t e) {
+        cudaEventRecord(c->done, cs);
+        return chain_fail(status, what, e);
+    };
     for (int l = 0; l < c->n_layers; ++l) {
         if (l < c->n_resident) {  // a resident layer: its GEMVs only
             const uint8_t* base = c->resident + static_cast<size_t>(l) * c->slot_bytes;
@@ -230,7 +236,7 @@ KQ_API int kq_chain_run(kq_chain* c, const float* const* x, float* const* y, kq_
                 const size_t i = static_cast<size_t>(l) * c->per_layer + m;
                 const kq_matrix_desc& d = c->mats[i];
                 int st = kq_gemv(base + c->offsets[m], d.fmt, d.N, d.K, x[i], y[i], compute);
-                if (st != KQ_OK) return chain_fail(st, kq_last_error());
+                if (st != KQ_OK) return stop(st, kq_last_error(), cudaSuccess);
             }
             continue;
         }
@@ -240,30 +246,29 @@ KQ_API int kq_chain_run(kq_chain* c, const float* const* x, float* const* y, kq_
         if (l == c->fault_layer) {
             // injected failure: stop issuing; what is queued drains normally
             // and kq_chain_wait still covers it
-            cudaEventRecord(c->done, cs);
-            return chain_fail(KQ_ERR_INJECTED, "KQ_FAULT: copy of the requested layer refused");
+            return stop(KQ_ERR_INJECTED, "KQ_FAULT: copy of the requested layer refused", cudaSuccess);
         }
         if (j >= c->n_slots) {
             err = cudaStreamWaitEvent(c->copy, c->freed[s], 0);
-            if (err != cudaSuccess) return chain_fail(KQ_ERR_CUDA, "wait slot free", err);
+            if (err != cudaSuccess) return stop(KQ_ERR_CUDA, "wait slot free", err);
         }
         for (int m = 0; m < c->per_layer; ++m) {
             const kq_matrix_desc& d = c->mats[static_cast<size_t>(l) * c->per_layer + m];
             err = cudaMemcpyAsync(slot + c->offsets[m], d.W, static_cast<size_t>(d.N) * kq_row_bytes(d.fmt, d.K),
                                   cudaMemcpyHostToDevice, c->copy);
-            if (err != cudaSuccess) return chain_fail(KQ_ERR_CUDA, "H2D copy", err);
+            if (err != cudaSuccess) return stop(KQ_ERR_CUDA, "H2D copy", err);
         }
         err = cudaEventRecord(c->ready[s], c->copy);
         if (err == cudaSuccess) err = cudaStreamWaitEvent(cs, c->ready[s], 0);
-        if (err != cudaSuccess) return chain_fail(KQ_ERR_CUDA, "slot ready", err);
+        if (err != cudaSuccess) return stop(KQ_ERR_CUDA, "slot ready", err);
         for (int m = 0; m < c->per_layer; ++m) {
             const size_t i = static_cast<size_t>(l) * c->per_layer + m;
             const kq_matrix_desc& d = c->mats[i];
             int st = kq_gemv(slot + c->offsets[m], d.fmt, d.N, d.K, x[i], y[i], compute);
-            if (st != KQ_OK) return chain_fail(st, kq_last_error());
+            if (st != KQ_OK) return stop(st, kq_last_error(), cudaSuccess);
         }
         err = cudaEventRecord(c->freed[s], cs);
-        if (err != cudaSuccess) return chain_fail(KQ_ERR_CUDA, "slot free", err);
+        if (err != cudaSuccess) return stop(KQ_ERR_CUDA, "slot free", err);
     }
     err = cudaEventRecord(c->done, cs);
     if (err != cudaSuccess) return chain_fail(KQ_ERR_CUDA, "done event", err);
@@ -295,5 +300,35 @@ KQ_API void kq_chain_destroy(kq_chain* c) {
     cudaStreamSynchronize(c->copy);
     destroy(c);
 }
+
+KQ_API int kq_stream_chain_create(const kq_layer_desc* layers, int n_layers, int n_slots, kq_chain** out) {
+    g_chain_err[0] = 0;
+    if (out) *out = nullptr;
+    if (!layers || !out || n_layers < 1 || n_slots < 1) return chain_fail(KQ_ERR_INVALID_ARG, "bad arguments");
+    const int per = layers[0].n_mats;
+    if (per < 1) return chain_fail(KQ_ERR_INVALID_ARG, "a layer without matrices");
+    std::vector<kq_matrix_desc> flat;
+    flat.reserve(static_cast<size_t>(n_layers) * per);
+    for (int l = 0; l < n_layers; ++l) {
+        if (layers[l].n_mats != per || !layers[l].mats)
+            return chain_fail(KQ_ERR_INVALID_ARG, "layers must share matrix formats and shapes");
+        for (int m = 0; m < per; ++m) flat.push_back(layers[l].mats[m]);
+    }
+    return kq_chain_create(flat.data(), n_layers, per, n_slots, out);
+}
+
+KQ_API int kq_stream_chain(kq_chain* c, const float* const* x_in, float* const* y_out, kq_stream_t compute,
+                           int64_t timeout_ms) {
+    const int st = kq_chain_run(c, x_in, y_out, compute);
+    if (st != KQ_OK) {
+        // what was queued still completes; wait for it (bounded) so that the
+        // caller gets the run's own error, not a busy chain
+        if (c) kq_chain_wait(c, timeout_ms);
+        return st;
+    }
+    return kq_chain_wait(c, timeout_ms);
+}
+
+KQ_API void kq_stream_chain_destroy(kq_chain* c) { kq_chain_destroy(c); }
 
 }  // extern "C"

@@ -73,17 +73,49 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for phase `parity` of `bar` to complete, giving up after kWaitNs or
+// Wait for phase `parity` of `bar` to complete, giving up after limit_ns or
 // when another thread of the CTA has raised `abort_flag`.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  unsigned long long limit_ns = kWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// The producer's last wait before its CTA may exit: phase `parity` of a
+// ring slot's `full` barrier, which completes when a bulk copy it issued
+// into this CTA's shared memory has landed.  Unlike mbar_wait_bounded it
+// does not give up when the CTA has aborted (a copy in flight must land
+// before the shared memory can be released), only after kWaitNs.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
         if (globaltimer_ns() - t0 > kWaitNs) return false;
     }
 }
+
+// The producer's record of its ring: which slots last received a bulk copy
+// (and at which phase).  A slot is reused only after the consumers released
+// it, and the producer issues nothing once the CTA has aborted, so each slot
+// holds at most one copy that may still be in flight; drain() waits for
+// each before the CTA exits, abort or not.
+struct RingTrack {
+    uint32_t issued = 0, phase = 0;
+    __device__ __forceinline__ void issue(int slot, uint32_t ph) {
+        issued |= 1u << slot;
+        phase = (phase & ~(1u << slot)) | ((ph & 1u) << slot);
+    }
+    __device__ __forceinline__ void skip(int slot) { issued &= ~(1u << slot); }
+    __device__ void drain(uint64_t* full, int ns) const {
+        for (int s = 0; s < ns; ++s)
+            if ((issued >> s) & 1u) mbar_wait_drain(&full[s], (phase >> s) & 1u);
+    }
+};
 
 // ------------------------------------------------------------- clusters
 

@@ -367,16 +367,23 @@ __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empt
                                int nbl, int srow, bool contiguous) {
     if (a.ids) pdl_wait();  // routed ids may come from the previous grid
     const uint64_t pol = l2_evict_first();
+    const unsigned long long lim = a.wait_ns && blockIdx.x == 0 ? a.wait_ns : kWaitNs;
     StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
     Stage st;
-    bool ok = true;
+    RingTrack ring;
     while (it.next(st)) {
         const int slot = it.slot;
         // a reused slot: wait until the consumers released its last stage
-        if (it.count > ns && !mbar_wait_bounded(&empty[slot], it.phase ^ 1u, abort_flag)) {
+        if (it.count > ns && !mbar_wait_bounded(&empty[slot], it.phase ^ 1u, abort_flag, lim)) {
             raise_fault(a, abort_flag, 6);
-            ok = false;
             break;
+        }
+        if (*abort_flag) break;  // nothing more is issued once the CTA has aborted
+        if (a.test_hold && blockIdx.x == 0 && it.count == a.test_hold) {
+            // test hook (kq_inject "hold@S"): this stage is never copied, so
+            // the consumers' bounded wait for it runs out
+            ring.skip(slot);
+            continue;
         }
         int64_t e = st.seg;
         if (a.ids) e = a.ids[st.seg];
@@ -395,21 +402,15 @@ __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empt
                 for (int i = 0; i < st.nrows; ++i)
                     bulk_g2s(dst + i * srow, src + i * a.row_bytes + off16, rbytes, &full[slot], pol);
             }
+            ring.issue(slot, it.phase);
         } else {
             mbar_arrive(&full[slot]);
+            ring.skip(slot);
         }
     }
-    // Let every copy this CTA issued land before the CTA can exit.
-    int issued = ok ? it.count : it.count - 1;
-    int sl = ok ? it.slot : (it.slot == 0 ? ns - 1 : it.slot - 1);
-    uint32_t ph = ok ? it.phase : (it.slot == 0 ? it.phase ^ 1u : it.phase);
-    for (int i = 0; i < issued && i < ns; ++i) {
-        if (!mbar_wait_bounded(&full[sl], ph, abort_flag)) break;
-        if (--sl < 0) {
-            sl = ns - 1;
-            ph ^= 1u;
-        }
-    }
+    // Let every copy this CTA issued land before the CTA can exit, abort or
+    // not (bounded).
+    ring.drain(full, ns);
 }
 
 // ------------------------------------------------------------- prologue
@@ -1342,6 +1343,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
 
     StageIter it(rp_begin, rp_end, rps, a.N, a.ps, ns);
     Stage st;
+    const unsigned long long wait_lim = a.wait_ns && blockIdx.x == 0 ? a.wait_ns : kWaitNs;
     int64_t staged_seg = -1;
     // prologue scratch: one region for a shared copy, else the group's own
     const uint32_t pro_r = smem_u32(smem + a.pro_offset) + (shared_x ? 0 : g * kProRegion);
@@ -1370,9 +1372,10 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
         // group has released the slot's previous stage: only then can the
         // parity wait on `full` not pass on a phase two ahead (it cannot
         // tell phase k from phase k + 2).
-        if (NG == 2 && (ns & 1) && it.count > ns && !mbar_wait_bounded(&empty[slot], it.phase ^ 1u, abort_flag))
+        if (NG == 2 && (ns & 1) && it.count > ns &&
+            !mbar_wait_bounded(&empty[slot], it.phase ^ 1u, abort_flag, wait_lim))
             raise_fault(a, abort_flag, 6);
-        if (!mbar_wait_bounded(&full[slot], it.phase, abort_flag)) raise_fault(a, abort_flag, 6);
+        if (!mbar_wait_bounded(&full[slot], it.phase, abort_flag, wait_lim)) raise_fault(a, abort_flag, 6);
         float out[2][NCOL];
 #pragma unroll
         for (int r = 0; r < 2; ++r)

@@ -50,6 +50,11 @@ struct GemvArgs {
     const float* gamma;      // RMSNorm weights (K)
     float eps;
     int pro_offset;          // RMSNorm scratch (kProBytes) after the stage ring
+    // test hooks (kq_inject): CTA 0's producer never copies its stage number
+    // test_hold (1-based; 0 = none), and CTA 0's bounded waits give up after
+    // wait_ns (0 = the default limit)
+    int test_hold;
+    unsigned long long wait_ns;
 };
 
 // ---------------------------------------------------- multi-step launch
@@ -118,9 +123,11 @@ cudaError_t mma_active_clusters(int cluster, size_t smem_bytes, bool pro, int* o
 cudaError_t fault_word(int** out);
 cudaError_t launch_splitk_combine(const float* partial, int S, int ncol, int64_t N, float* y, int64_t ldy,
                                   cudaStream_t stream);
-cudaError_t launch_unpack(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d,
-                          cudaStream_t stream);
+cudaError_t launch_unpack(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, uint8_t* m, float* d,
+                          float* dmin, bool split, cudaStream_t stream);
 cudaError_t ensure_smem_attr(const void* func, size_t bytes);
+// Read-only bandwidth probes (kq_read_probe): mode 0 loads, mode 1 bulk-copy ring.
+cudaError_t launch_probe(const void* src, size_t bytes, int mode, uint32_t* out, int sm_count, cudaStream_t s);
 cudaError_t read_and_clear_fault(int* out);
 // Records `msg` as the calling thread's kq_last_error() text; returns status.
 int set_last_error(int status, const char* msg);

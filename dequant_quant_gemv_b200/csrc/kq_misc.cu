@@ -16,10 +16,18 @@ __device__ int g_kq_fault = 0;
 // ------------------------------------------------------- debug unpack
 
 // One thread per super-block: the integer fields, decoded with the same
-// helpers the GEMV kernels use.
-__global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d) {
+// helpers the GEMV kernels use.  Each format branch fills the block's quants
+// (written at once) and its 16 scale and 16 min bytes, d and dmin; `split`
+// selects the output form: the separate arrays of kq_unpack (sc_or_s, m,
+// d, dmin, one entry or 16 bytes per block) or the packed form of
+// kq_unpack_fields (sc: 16 bytes per block, d: d and dmin per block).
+__global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, uint8_t* m,
+                              float* d, float* dmin, bool split) {
     const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (b >= nblocks) return;
+    uint8_t S[16], M[16];
+    for (int g = 0; g < 16; ++g) S[g] = M[g] = 0;
+    float dv = 0.0f, dmv = 0.0f;
     if (fmt == 1 || fmt == 3) {
         // Q4_K, Q5_K: the same header; Q5_K quants sit after its 32 qh bytes
         const uint8_t* blk = W + b * (fmt == 1 ? kQ4Bytes : kQ5Bytes);
@@ -29,12 +37,12 @@ __global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_
             uint32_t sc4, m4;
             q4k_half_scales(hd.y, hd.z, hd.w, H, sc4, m4);
             for (int k = 0; k < 4; ++k) {
-                sc[16 * b + 4 * H + k] = static_cast<uint8_t>(sc4 >> (8 * k));
-                sc[16 * b + 8 + 4 * H + k] = static_cast<uint8_t>(m4 >> (8 * k));
+                S[4 * H + k] = static_cast<uint8_t>(sc4 >> (8 * k));
+                M[4 * H + k] = static_cast<uint8_t>(m4 >> (8 * k));
             }
         }
-        d[2 * b] = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x & 0xFFFFu)));
-        d[2 * b + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x >> 16)));
+        dv = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x & 0xFFFFu)));
+        dmv = __half2float(__ushort_as_half(static_cast<unsigned short>(hd.x >> 16)));
         for (int w = 0; w < 32; ++w) {
             const uint32_t v = *reinterpret_cast<const uint32_t*>(qs + 4 * w);
             const int c = w >> 3, l0 = (w & 7) * 4;
@@ -51,25 +59,27 @@ __global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_
     } else if (fmt == 4) {
         // Q2_K: 4-byte aligned blocks
         const uint8_t* blk = W + b * kQ2Bytes;
-        for (int g = 0; g < 16; ++g) sc[16 * b + g] = blk[g];
+        for (int g = 0; g < 16; ++g) {
+            S[g] = blk[g] & 15u;
+            M[g] = blk[g] >> 4;
+        }
         for (int i = 0; i < 64; ++i) {
             const uint32_t v = blk[16 + i];
             const int n = i >> 5, l = i & 31;
             for (int j = 0; j < 4; ++j) q[256 * b + 128 * n + 32 * j + l] = static_cast<uint8_t>((v >> (2 * j)) & 3u);
         }
         const uint32_t dw = *reinterpret_cast<const uint32_t*>(blk + 80);
-        d[2 * b] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw & 0xFFFFu)));
-        d[2 * b + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw >> 16)));
+        dv = __half2float(__ushort_as_half(static_cast<unsigned short>(dw & 0xFFFFu)));
+        dmv = __half2float(__ushort_as_half(static_cast<unsigned short>(dw >> 16)));
     } else if (fmt == 6) {
-        // Q8_0: a unit of eight 34-byte blocks, read by bytes
+        // Q8_0: a unit of eight 34-byte blocks, read by bytes; S holds the
+        // eight fp16 scales as raw little-endian bytes
         const uint8_t* u = W + b * kQ80Bytes;
         for (int j = 0; j < 8; ++j) {
-            sc[16 * b + 2 * j] = u[34 * j];
-            sc[16 * b + 2 * j + 1] = u[34 * j + 1];
+            S[2 * j] = u[34 * j];
+            S[2 * j + 1] = u[34 * j + 1];
             for (int i = 0; i < 32; ++i) q[256 * b + 32 * j + i] = u[34 * j + 2 + i];
         }
-        d[2 * b] = 0.0f;
-        d[2 * b + 1] = 0.0f;
     } else if (fmt == 5) {
         // Q3_K: 2-byte aligned blocks, read by bytes
         const uint8_t* blk = W + b * kQ3Bytes;
@@ -84,11 +94,10 @@ __global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_
         for (int g = 0; g < 16; ++g) {
             const uint32_t lo = g < 8 ? (blk[96 + g] & 15u) : (blk[96 + g - 8] >> 4);
             const uint32_t hi = (blk[104 + (g & 3)] >> (2 * (g >> 2))) & 3u;
-            sc[16 * b + g] = static_cast<uint8_t>(lo | (hi << 4));
+            S[g] = static_cast<uint8_t>(lo | (hi << 4));
         }
         const unsigned short dh = static_cast<unsigned short>(blk[108] | (blk[109] << 8));
-        d[2 * b] = __half2float(__ushort_as_half(dh));
-        d[2 * b + 1] = 0.0f;
+        dv = __half2float(__ushort_as_half(dh));
     } else {
         const uint8_t* blk = W + b * kQ6Bytes;  // 2-byte aligned only
         auto word = [&](int off) -> uint32_t {
@@ -104,19 +113,32 @@ __global__ void unpack_kernel(const uint8_t* W, int fmt, int64_t nblocks, uint8_
                     for (int k = 0; k < 4; ++k)
                         q[256 * b + 128 * H + 32 * t + 4 * s + k] = static_cast<uint8_t>(qv[t] >> (8 * k));
             }
-        for (int g = 0; g < 16; ++g) sc[16 * b + g] = blk[192 + g];
+        for (int g = 0; g < 16; ++g) S[g] = blk[192 + g];
         const unsigned short dh = static_cast<unsigned short>(blk[208] | (blk[209] << 8));
-        d[2 * b] = __half2float(__ushort_as_half(dh));
-        d[2 * b + 1] = 0.0f;
+        dv = __half2float(__ushort_as_half(dh));
+    }
+    if (split) {
+        for (int g = 0; g < 16; ++g) sc[16 * b + g] = S[g];
+        if (m)
+            for (int g = 0; g < 16; ++g) m[16 * b + g] = M[g];
+        d[b] = dv;
+        if (dmin) dmin[b] = dmv;
+    } else {
+        // Q4_K, Q5_K: sc_0..7 then m_0..7; Q2_K: the stored bytes sc | m << 4
+        const bool eight = fmt == 1 || fmt == 3;
+        for (int g = 0; g < 16; ++g)
+            sc[16 * b + g] = eight ? (g < 8 ? S[g] : M[g - 8]) : (fmt == 4 ? static_cast<uint8_t>(S[g] | (M[g] << 4)) : S[g]);
+        d[2 * b] = dv;
+        d[2 * b + 1] = dmv;
     }
 }
 
-cudaError_t launch_unpack(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, float* d,
-                          cudaStream_t stream) {
+cudaError_t launch_unpack(const uint8_t* W, int fmt, int64_t nblocks, uint8_t* q, uint8_t* sc, uint8_t* m, float* d,
+                          float* dmin, bool split, cudaStream_t stream) {
     const int threads = 128;
     const int64_t grid = (nblocks + threads - 1) / threads;
     if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-    unpack_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(W, fmt, nblocks, q, sc, d);
+    unpack_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(W, fmt, nblocks, q, sc, m, d, dmin, split);
     return cudaGetLastError();
 }
 

@@ -2,8 +2,8 @@
 //
 // "RunNburn - Run a 295B MoE from a 98GB GGUF on a 64GB RAM Desktop": only
 // the experts a token selects are fetched, on demand; "Out-of-core LLM
-// inference engine written from scratch in Rust", Approach: weights move
-// through VRAM slots while the GPU computes.
+// inference engine written from scratch in Rust", Approach: weight copies
+// into device slots overlap the computation.
 //
 // Schedule of run r in slot set t = r % n_sets (everything enqueued up
 // front; the host never blocks):

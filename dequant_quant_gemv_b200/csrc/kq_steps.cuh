@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
             int slot = -1, count = 0;
             uint32_t phase = 0;
             bool ok = true;
+            RingTrack ring;
             for (int si = 0; si < A.n && ok; ++si) {
                 const StepArgs& s = A.st[si];
                 int rp0, rp1;
@@ -116,23 +117,20 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
                         ok = false;
                         break;
                     }
+                    if (*abort_flag) {  // nothing more is issued once the CTA has aborted
+                        ok = false;
+                        break;
+                    }
                     const uint32_t bytes = static_cast<uint32_t>(rows * s.row_bytes);
                     mbar_arrive_expect_tx(&full[slot], bytes);
                     bulk_g2s(sbuf + static_cast<size_t>(slot) * A.slot_bytes, s.W + row0 * s.row_bytes, bytes,
                              &full[slot], pol);
+                    ring.issue(slot, phase);
                 }
             }
-            // let every copy issued land before the CTA can exit
-            const int issued = ok ? count : count - 1;
-            int sl = ok ? slot : (slot == 0 ? ns - 1 : slot - 1);
-            uint32_t ph = ok ? phase : (slot == 0 ? phase ^ 1u : phase);
-            for (int i = 0; i < issued && i < ns; ++i) {
-                if (!mbar_wait_bounded(&full[sl], ph, abort_flag)) break;
-                if (--sl < 0) {
-                    sl = ns - 1;
-                    ph ^= 1u;
-                }
-            }
+            // let every copy issued land before the CTA can exit, abort or
+            // not (bounded)
+            ring.drain(full, ns);
         }
         return;
     }

@@ -79,7 +79,9 @@ def lib() -> ctypes.CDLL:
         L.kq_moe_gemv.restype = i32
         L.kq_moe_gemv.argtypes = [vp, i32, i32, i64, i64, sz, vp, i32, vp, i64, vp, vp, vp]
         L.kq_unpack.restype = i32
-        L.kq_unpack.argtypes = [vp, i32, i64, vp, vp, vp, vp]
+        L.kq_unpack.argtypes = [vp, i32, i64, vp, vp, vp, vp, vp, vp]
+        L.kq_unpack_fields.restype = i32
+        L.kq_unpack_fields.argtypes = [vp, i32, i64, vp, vp, vp, vp]
         L.kq_gemv_fused.restype = i32
         L.kq_gemv_fused.argtypes = [vp, i32, i64, i64, vp, i64, i32, ctypes.POINTER(Prologue), vp, i64, vp]
         L.kq_gemv_steps.restype = i32
@@ -242,13 +244,47 @@ def moe_gemv(W_experts: torch.Tensor, fmt, E: int, N: int, K: int, ids: torch.Te
 
 
 def unpack(W: torch.Tensor, fmt, n_blocks: int, stream=None):
-    """(q, sc, d) integer fields as decoded on the GPU (see kq.h)."""
+    """(q, sc, d) integer fields as decoded on the GPU, packed form
+    (kq_unpack_fields in kq.h)."""
     q = torch.empty(n_blocks * 256, dtype=torch.uint8, device=W.device)
     sc = torch.empty(n_blocks * 16, dtype=torch.uint8, device=W.device)
     d = torch.empty(n_blocks * 2, dtype=torch.float32, device=W.device)
-    _check(lib().kq_unpack(_dev(W, "W"), _fmt(fmt), n_blocks, q.data_ptr(), sc.data_ptr(), d.data_ptr(),
-                           _stream(stream)), "kq_unpack")
+    _check(lib().kq_unpack_fields(_dev(W, "W"), _fmt(fmt), n_blocks, q.data_ptr(), sc.data_ptr(), d.data_ptr(),
+                                  _stream(stream)), "kq_unpack_fields")
     return q, sc, d
+
+
+def unpack_split(W: torch.Tensor, fmt, n_blocks: int, stream=None):
+    """(q, sc_or_s, m, d, dmin) as decoded on the GPU (kq_unpack in kq.h):
+    q int8 (n_blocks*256), sc_or_s and m uint8 (n_blocks*16 each), d and
+    dmin float32 (n_blocks each)."""
+    q = torch.empty(n_blocks * 256, dtype=torch.int8, device=W.device)
+    sc = torch.empty(n_blocks * 16, dtype=torch.uint8, device=W.device)
+    m = torch.empty(n_blocks * 16, dtype=torch.uint8, device=W.device)
+    d = torch.empty(n_blocks, dtype=torch.float32, device=W.device)
+    dmin = torch.empty(n_blocks, dtype=torch.float32, device=W.device)
+    _check(lib().kq_unpack(_dev(W, "W"), _fmt(fmt), n_blocks, q.data_ptr(), sc.data_ptr(), m.data_ptr(),
+                           d.data_ptr(), dmin.data_ptr(), _stream(stream)), "kq_unpack")
+    return q, sc, m, d, dmin
+
+
+def read_probe(buf: torch.Tensor, mode: int, out: torch.Tensor, stream=None) -> None:
+    """kq_read_probe: read `buf` once (mode 0 loads, mode 1 the bulk-copy
+    ring of the GEMV kernels); XOR of the data into out (int32, 1 element)."""
+    L = lib()
+    L.kq_read_probe.restype = ctypes.c_int
+    L.kq_read_probe.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    _check(L.kq_read_probe(_dev(buf, "buf"), buf.numel() * buf.element_size(), mode, _dev(out, "out"),
+                           _stream(stream)), "kq_read_probe")
+
+
+def inject(spec: str | None) -> None:
+    """kq_inject: test hook ("hold@S" withholds one weight stage of the next
+    single-column launch so that its bounded wait runs out)."""
+    L = lib()
+    L.kq_inject.restype = ctypes.c_int
+    L.kq_inject.argtypes = [ctypes.c_char_p]
+    _check(L.kq_inject(spec.encode() if spec else None), "kq_inject")
 
 
 def device_fault() -> int:
@@ -512,3 +548,61 @@ class Chain:
             self.close()
         except Exception:
             pass
+
+
+class LayerDesc(ctypes.Structure):
+    """kq_layer_desc: one layer's matrices for kq_stream_chain_create."""
+    _fields_ = [("mats", ctypes.POINTER(MatrixDesc)), ("n_mats", ctypes.c_int)]
+
+
+class StreamChain(Chain):
+    """The streamed chain through the per-layer entry points
+    kq_stream_chain_create / kq_stream_chain / kq_stream_chain_destroy."""
+
+    def __init__(self, mats, n_slots: int = 4):
+        L = lib()
+        _chain_sigs(L)
+        if not getattr(L, "_stream_chain_ready", False):
+            vp = ctypes.c_void_p
+            L.kq_stream_chain_create.restype = ctypes.c_int
+            L.kq_stream_chain_create.argtypes = [ctypes.POINTER(LayerDesc), ctypes.c_int, ctypes.c_int,
+                                                 ctypes.POINTER(vp)]
+            L.kq_stream_chain.restype = ctypes.c_int
+            L.kq_stream_chain.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), vp, ctypes.c_int64]
+            L.kq_stream_chain_destroy.restype = None
+            L.kq_stream_chain_destroy.argtypes = [vp]
+            L._stream_chain_ready = True
+        self._L = L
+        self.n_layers = len(mats)
+        self.per_layer = len(mats[0])
+        self._keep = [m[0] for layer in mats for m in layer]
+        self._arrays = []
+        layers = (LayerDesc * self.n_layers)()
+        for l, layer in enumerate(mats):
+            arr = (MatrixDesc * len(layer))()
+            for i, (W, fmt, N, K) in enumerate(layer):
+                if W.is_cuda:
+                    raise ValueError("chain weights must be host memory")
+                arr[i] = MatrixDesc(W.data_ptr(), _fmt(fmt), N, K)
+            self._arrays.append(arr)
+            layers[l] = LayerDesc(arr, len(layer))
+        h = ctypes.c_void_p()
+        st = L.kq_stream_chain_create(layers, self.n_layers, n_slots, ctypes.byref(h))
+        if st != OK:
+            raise KQError(st, "kq_stream_chain_create", L.kq_chain_last_error().decode())
+        self._h = h
+
+    def run_wait(self, xs, ys, timeout_ms: int = -1, stream=None) -> None:
+        """kq_stream_chain: one pass, waited for on the host (bounded)."""
+        n = self.n_layers * self.per_layer
+        assert len(xs) == n and len(ys) == n
+        xa = (ctypes.c_void_p * n)(*[_dev(x, "x", torch.float32) for x in xs])
+        ya = (ctypes.c_void_p * n)(*[_dev(y, "y", torch.float32) for y in ys])
+        st = self._L.kq_stream_chain(self._h, xa, ya, _stream(stream), timeout_ms)
+        if st != OK:
+            raise KQError(st, "kq_stream_chain", self._L.kq_chain_last_error().decode())
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._L.kq_stream_chain_destroy(self._h)
+            self._h = None

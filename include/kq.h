@@ -6,9 +6,10 @@
  * What the method is (by page):
  *  - "Out-of-core LLM inference engine written from scratch in Rust",
  *    Approach: quantised weights are dequantised inside fused matmul kernels;
- *    speculative decoding verifies several positions with one pass; layer
- *    weights move through a ring of VRAM slots while the GPU computes nearby
- *    layers.  Results: Llama-3.3-70B Q4_K_M; a fully resident 30B MoE.
+ *    speculative decoding verifies several positions with one pass; each
+ *    layer is copied into one of a fixed set of device slots and runs there
+ *    while copies of other layers proceed.  Results: Llama-3.3-70B Q4_K_M;
+ *    a fully resident 30B MoE.
  *  - "Kortex: Streaming 70B Models on Consumer GPUs", Key components 2-3:
  *    the streaming pipeline overlaps transfers with compute; weights are
  *    dequantised only in GPU registers.  Token generation is memory-bandwidth
@@ -128,6 +129,31 @@ KQ_API const char* kq_last_error(void);
  * kernel whose bounded wait ran out sets it to KQ_ERR_TIMEOUT instead of
  * hanging.  Synchronous.  *out is a HOST int. */
 KQ_API int kq_device_fault(int* out);
+
+/* Test hook for the failure-detection tests: a device-side wait that runs
+ * out.  spec "hold@S" (S >= 1): the next single-column GEMV launch (kq_gemv,
+ * or a one-column group of kq_gemv_multi) does not copy the S-th weight stage
+ * of its first CTA, and that CTA's bounded waits give up after 1 ms instead
+ * of 2 s;
+ * the consumers waiting for that stage then time out, the CTA stops, lets
+ * the copies it issued land, and the launch ends with the fault word set to
+ * KQ_ERR_TIMEOUT (read it with kq_device_fault); that CTA's outputs are
+ * undefined.  One-shot; NULL or "" cancels.  No trap, no hang: the context
+ * stays usable.  Process-wide; KQ_ERR_INVALID_ARG for another spec. */
+KQ_API int kq_inject(const char* spec);
+
+/* Measurement helper: reads `bytes` (a multiple of 16) at src (DEVICE,
+ * 16-byte aligned) once and XORs what it read into *out (DEVICE uint32), so
+ * that the time of the call is the device's read-only bandwidth -- the
+ * ceiling of a GEMV, which only reads its weights (decode is bound by the
+ * weight bytes: "Kortex: Streaming 70B Models on Consumer GPUs", the
+ * paragraph before the first table).  mode 0: 16-byte loads from every
+ * thread of a full grid; mode 1: the GEMV kernels' weight path, one CTA per
+ * SM bulk-copying (TMA, no multicast) 48 KiB stages of a contiguous range
+ * into a 4-slot shared-memory ring, one warp reading each stage from shared
+ * memory and releasing it (no other work).  Asynchronous on `stream`.  Errors: KQ_ERR_INVALID_ARG,
+ * KQ_ERR_CUDA; a bounded wait that runs out sets the fault word. */
+KQ_API int kq_read_probe(const void* src, size_t bytes, int mode, uint32_t* out, kq_stream_t stream);
 
 /* Bytes per super-block (Q2_K 84, Q3_K 110, Q4_K 144, Q5_K 176, Q6_K 210;
  * Q8_0 272, per 8 blocks of 32 weights) or 0 for an unknown format. */
@@ -259,15 +285,21 @@ KQ_API int kq_gemv_splitk(const void* W, int fmt, int64_t N, int64_t K, const fl
  * outputs.  Such callers cannot supply the split-K workspace, so this call
  * keeps the partial sums in a 64 KiB array built into the library (every GPU
  * that loads libkq holds it until the process exits).  It calls no cudaMalloc,
- * cudaFree or allocating routine.
+ * cudaFree or allocating routine (the first call per device aside: see
+ * below).
  *   Arguments, layout and results are those of kq_gemv_splitk (the same
  *   kernels and summation order, so the outputs are identical).
  *   Errors: KQ_ERR_UNSUPPORTED when the split would need more partial sums
  *   than the 64 KiB hold (16384 floats = ranges * k * N); the text is in
  *   kq_last_error().  Other errors as kq_gemv_splitk.
  *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   (cudaGetSymbolAddress) with that device current.  With CUDA's lazy
+ *   module loading (the default) that lookup may load the library's device
+ *   module, which allocates device memory and takes driver locks, so make
+ *   the first call per device outside real-time and capture code (a
+ *   warm-up call at start-up); every later call allocates nothing.  The
+ *   looked-up address is cached per device: after cudaDeviceReset the
+ *   library must be unloaded and loaded again.
  *   All calls share the one array: calls that overlap on the GPU (other
  *   streams, other threads) race on it and must be ordered by the caller.
  *   Nothing in it needs clearing between calls: each call writes every
@@ -301,8 +333,8 @@ KQ_API int kq_moe_gemv(const void* W_experts, int fmt, int E, int64_t N, int64_t
  * and only the selected experts are copied to the device, per call
  * ("RunNburn - Run a 295B MoE from a 98GB GGUF on a 64GB RAM Desktop": the
  * experts a token selects are gathered on demand; "Out-of-core LLM
- * inference engine ...", Approach: weights stream through VRAM slots while
- * the GPU computes).
+ * inference engine ...", Approach: weight copies into device slots proceed
+ * alongside the computation).
  *
  * kq_moe_stream_create: the expert stack W_host (HOST pointer, page-locked,
  *   owned by the caller and kept alive and unchanged until destroy): E
@@ -377,27 +409,45 @@ KQ_API const char* kq_gguf_last_error(void);
 
 /*
  * kq_unpack — debug: the integer fields of n_blocks consecutive super-blocks
- * as the GEMV kernels decode them (for bit-exact comparison).
- *   q:  n_blocks*256 bytes, quant of weight i of block b at q[256b+i]
- *       (Q2_K 0..3; Q3_K -4..3 as two's-complement bytes; Q4_K 0..15;
- *       Q5_K 0..31; Q6_K 0..63, before the -32 offset)
- *   sc: n_blocks*16 bytes; Q4_K, Q5_K: sc_0..7 then m_0..7; Q2_K: the 16
- *       bytes sc_g | m_g << 4 as stored; Q3_K: the 16 6-bit v_g (before the
- *       -32 offset); Q6_K: the 16 int8 scales as two's-complement bytes
- *   d:  n_blocks*2 floats; Q2_K, Q4_K, Q5_K: d, dmin; Q3_K, Q6_K: d, 0
- *       (fp16 widened exactly); Q8_0: 0, 0
- *   For Q8_0 a "block" here is a unit of 8 blocks (256 weights): q holds its
- *   int8 quants as two's-complement bytes and sc the 8 fp16 scales d as raw
- *   little-endian bytes.
- * All device pointers; W must be 16-byte aligned.
+ * as the GEMV kernels decode them, for bit-exact comparison with a plain
+ * decoder (the pages ask that quants be unpacked exactly: "Kortex: Streaming
+ * 70B Models on Consumer GPUs", Key components 3, dequantisation in
+ * registers; the block layouts are those above).
+ *   q:       n_blocks*256 int8, quant of weight i of block b at q[256b+i]
+ *            (Q2_K 0..3; Q3_K -4..3; Q4_K 0..15; Q5_K 0..31; Q6_K 0..63,
+ *            before the -32 offset; Q8_0 the int8 quants)
+ *   sc_or_s: n_blocks*16 bytes, the block's group scales at 16b+g: Q4_K and
+ *            Q5_K sc_0..7 (bytes 8..15 zero); Q2_K the 16 4-bit sc_g; Q3_K
+ *            the 16 6-bit v_g (before the -32 offset); Q6_K the 16 int8 s_g
+ *            as two's-complement bytes; Q8_0 its eight fp16 d as raw
+ *            little-endian bytes
+ *   m:       n_blocks*16 bytes or NULL: Q4_K and Q5_K m_0..7 (bytes 8..15
+ *            zero); Q2_K the 16 4-bit m_g; other formats zeros
+ *   d:       n_blocks floats: d widened exactly from fp16 (Q8_0: 0)
+ *   dmin:    n_blocks floats or NULL: dmin of Q2_K, Q4_K and Q5_K (else 0)
+ *   For Q8_0 a "block" here is a unit of 8 blocks (256 weights).
+ * All device pointers; W must be 16-byte aligned, d and dmin 4-byte aligned.
+ * Errors: KQ_ERR_INVALID_ARG (unknown format, n_blocks < 0, a NULL q,
+ * sc_or_s or d, misalignment), KQ_ERR_CUDA.
  */
-KQ_API int kq_unpack(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d,
-              kq_stream_t stream);
+KQ_API int kq_unpack(const void* W, int fmt, int64_t n_blocks, int8_t* q, uint8_t* sc_or_s, uint8_t* m, float* d,
+                     float* dmin, kq_stream_t stream);
+
+/*
+ * kq_unpack_fields — the same decode in a packed form (three arrays):
+ *   q:  n_blocks*256 bytes, as kq_unpack
+ *   sc: n_blocks*16 bytes; Q4_K, Q5_K: sc_0..7 then m_0..7; Q2_K: the 16
+ *       bytes sc_g | m_g << 4 as stored; Q3_K, Q6_K, Q8_0: as kq_unpack
+ *   d:  n_blocks*2 floats: d, dmin (0 where the format has none)
+ * Errors as kq_unpack.
+ */
+KQ_API int kq_unpack_fields(const void* W, int fmt, int64_t n_blocks, uint8_t* q, uint8_t* sc, float* d,
+                            kq_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Streamed layer chain ("Out-of-core LLM inference engine written from
- * scratch in Rust", Approach: layer weights move through a ring of VRAM
- * slots while the GPU computes nearby layers; "Kortex: Streaming 70B Models
+ * scratch in Rust", Approach: layers are copied into a fixed set of device
+ * slots and run while other layers compute; "Kortex: Streaming 70B Models
  * on Consumer GPUs", Key components 2: the pipeline overlaps transfers with
  * compute).
  *
@@ -474,6 +524,31 @@ KQ_API const char* kq_chain_last_error(void);
 
 /* Waits for the chain's copies, then frees its slots, stream and events. */
 KQ_API void kq_chain_destroy(kq_chain* c);
+
+/* The streamed chain by layer (the same object and schedule as kq_chain_*,
+ * for callers that hold their weights per layer). */
+typedef struct kq_layer_desc {
+    const kq_matrix_desc* mats;  /* HOST array of n_mats matrices (weights page-locked) */
+    int n_mats;
+} kq_layer_desc;
+
+/* kq_chain_create over n_layers layer descriptors (every layer with the same
+ * n_mats, formats and shapes; the descriptor arrays are read during the call
+ * only).  Errors as kq_chain_create; on error *out is NULL. */
+KQ_API int kq_stream_chain_create(const kq_layer_desc* layers, int n_layers, int n_slots, kq_chain** out);
+
+/* One streamed pass, waited for: kq_chain_run(c, x_in, y_out, compute), then
+ * kq_chain_wait(c, timeout_ms).  x_in / y_out: HOST arrays of n_layers *
+ * n_mats DEVICE pointers, layer major.  KQ_OK once the pass has finished;
+ * KQ_ERR_TIMEOUT if it has not within timeout_ms (negative: no limit) -- the
+ * pass then goes on on the device and kq_chain_wait can wait for it again.
+ * A run that fails part-way returns its own error after what it queued has
+ * drained (bounded by timeout_ms). */
+KQ_API int kq_stream_chain(kq_chain* c, const float* const* x_in, float* const* y_out, kq_stream_t compute,
+                           int64_t timeout_ms);
+
+/* kq_chain_destroy. */
+KQ_API void kq_stream_chain_destroy(kq_chain* c);
 
 #ifdef __cplusplus
 }

@@ -11,7 +11,7 @@ in natural index order.  Sources, by page:
    Approach (weights dequantised inside fused matmul kernels; speculative
    decoding verifies several positions in one pass) and Results (Q4_K_M).
  - "Kortex: Streaming 70B Models on Consumer GPUs", Key components 2-3
-   (streaming pipeline through VRAM slots; dequantise only in registers).
+   (layers copied into device slots while others compute; dequantise only in registers).
  - "RunNburn - Run a 295B MoE ...": selected experts per token, native
    K-quant kernels.
 

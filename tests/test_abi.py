@@ -28,7 +28,8 @@ def libkq():
 
 def test_header_declares_entry_points():
     names = declared_symbols()
-    for n in ("kq_gemv", "kq_gemv_multi", "kq_moe_gemv", "kq_unpack", "kq_row_bytes", "kq_status_str"):
+    for n in ("kq_gemv", "kq_gemv_multi", "kq_moe_gemv", "kq_unpack", "kq_row_bytes", "kq_status_str",
+              "kq_stream_chain_create", "kq_stream_chain", "kq_stream_chain_destroy"):
         assert n in names
 
 

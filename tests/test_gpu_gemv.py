@@ -41,6 +41,31 @@ def test_unpack_bit_exact(fmt, N, K):
     assert np.array_equal(d.cpu().numpy().view(np.uint32), d0.view(np.uint32))
 
 
+@pytest.mark.parametrize("fmt,N,K", [("q4_k", 512, 4096), ("q6_k", 64, 14336), ("q5_k", 256, 4096),
+                                     ("q2_k", 128, 4096), ("q3_k", 128, 4096), ("q8_0", 128, 4096)])
+def test_unpack_separate_arrays_bit_exact(fmt, N, K):
+    """kq_unpack (q, sc_or_s, m, d, dmin as separate arrays) against the
+    oracle's unpacker, field by field."""
+    W = matrix(fmt, 2000 + N, N, K)
+    nb = N * K // 256
+    q, sc, m, d, dmin = (t.cpu().numpy() for t in kq.unpack_split(dev(W), fmt, nb))
+    q0, sc0, d0 = oracle.unpack(fmt, W, nb)
+    sc0 = sc0.reshape(nb, 16)
+    assert np.array_equal(q.view(np.uint8), q0)
+    z8 = np.zeros((nb, 8), np.uint8)
+    if fmt in ("q4_k", "q5_k"):
+        want_sc, want_m = np.hstack([sc0[:, :8], z8]), np.hstack([sc0[:, 8:], z8])
+    elif fmt == "q2_k":
+        want_sc, want_m = sc0 & 15, sc0 >> 4
+    else:
+        want_sc, want_m = sc0, np.zeros_like(sc0)
+    assert np.array_equal(sc.reshape(nb, 16), want_sc)
+    assert np.array_equal(m.reshape(nb, 16), want_m)
+    d0 = d0.reshape(nb, 2)
+    assert np.array_equal(d.view(np.uint32), np.ascontiguousarray(d0[:, 0]).view(np.uint32))
+    assert np.array_equal(dmin.view(np.uint32), np.ascontiguousarray(d0[:, 1]).view(np.uint32))
+
+
 # -------------------------------------------------- parity, many shapes
 SHAPES = [
     ("q4_k", 1, 256), ("q4_k", 3, 256), ("q4_k", 7, 768), ("q4_k", 33, 2048), ("q4_k", 64, 4096),

@@ -77,8 +77,18 @@ def test_unpack_and_workspace_sizes():
     L = kq.lib()
     L.kq_splitk_workspace_bytes.restype = ctypes.c_size_t
     L.kq_splitk_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
-    assert L.kq_unpack(P, 9, 4, P, P, P, None) == INVALID
-    assert L.kq_unpack(P, 1, -1, P, P, P, None) == INVALID
-    assert L.kq_unpack(P, 1, 0, P, P, P, None) == 0
+    assert L.kq_unpack_fields(P, 9, 4, P, P, P, None) == INVALID
+    assert L.kq_unpack_fields(P, 1, -1, P, P, P, None) == INVALID
+    assert L.kq_unpack_fields(P, 1, 0, P, P, P, None) == 0
+    # the separate-array form: unknown format, negative count, NULL q / sc / d,
+    # misaligned d or dmin; m and dmin may be NULL
+    assert L.kq_unpack(P, 9, 4, P, P, P, P, P, None) == INVALID
+    assert L.kq_unpack(P, 1, -1, P, P, P, P, P, None) == INVALID
+    assert L.kq_unpack(P, 1, 4, 0, P, P, P, P, None) == INVALID
+    assert L.kq_unpack(P, 1, 4, P, 0, P, P, P, None) == INVALID
+    assert L.kq_unpack(P, 1, 4, P, P, P, 0, P, None) == INVALID
+    assert L.kq_unpack(P, 1, 4, P, P, P, P + 2, P, None) == INVALID
+    assert L.kq_unpack(P, 1, 4, P, P, P, P, P + 2, None) == INVALID
+    assert L.kq_unpack(P, 1, 0, P, P, None, P, None, None) == 0
     for bad in ((9, 64, 4096, 1), (1, 0, 4096, 1), (1, 64, 100, 1), (1, 64, 4096, 0), (1, 64, 4096, 9)):
         assert L.kq_splitk_workspace_bytes(*bad) == 0

@@ -5,11 +5,13 @@ arena, a plugin handed only its inputs and outputs.  Instead of a
 caller-provided workspace it keeps its partial sums in a small array built
 into the library.
 
-The test drives it through the C ABI and compares it with kq_gemv_splitk fed
-a workspace allocated here, within the parity tolerance, on two calls in a
-row with different inputs (the built-in array keeps the previous call's
-contents).  It lives in its own file, collected last, and sets up everything
-it needs, so it passes alone in a fresh process or after the other tests.
+The test drives it through the C ABI on two calls in a row with different
+inputs (the built-in array keeps the previous call's contents).  It runs the
+same kernels in the same summation order as kq_gemv_splitk fed a workspace
+allocated here, so the two outputs must be equal bit for bit; each output is
+also checked against the oracle within the parity tolerance.  It lives in
+its own file, collected last, and sets up everything it needs, so it passes
+alone in a fresh process or after the other tests.
 """
 import numpy as np
 import pytest
@@ -44,6 +46,7 @@ def test_noalloc_matches_workspace_entry_point_twice(fmt, N, K, k):
         ws = torch.empty(kq.splitk_workspace_bytes(fmt, N, K, k) // 4, dtype=torch.float32, device="cuda")
         Y_ws = kq.gemv_splitk(Wt, fmt, N, K, Xt, workspace=ws)
         torch.cuda.synchronize()
-        _, s = oracle.gemv_multi(fmt, W, N, K, X, nthreads=0)
-        diff = (Y_na.double() - Y_ws.double()).abs().cpu().numpy()
-        assert np.all(diff <= REL * s + ABS), (call, float(diff.max()))
+        assert torch.equal(Y_na, Y_ws), (call, float((Y_na - Y_ws).abs().max()))
+        y_ref, s = oracle.gemv_multi(fmt, W, N, K, X, nthreads=0)
+        err = np.abs(Y_na.double().cpu().numpy() - y_ref)
+        assert np.all(err <= REL * s + ABS), (call, float((err / (REL * s + ABS)).max()))
