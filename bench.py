@@ -801,6 +801,10 @@ def bench_kq(args, rank, world):
         for _ in range(args.steps):
             run_step()
         e1.record(stream)
+        # poll (releasing the interpreter lock) so that the clock thread
+        # keeps sampling until the timed work has finished
+        while not e1.query():
+            time.sleep(0.0002)
         torch.cuda.synchronize()
         clk.stop()
     ms = max_over_ranks(e0.elapsed_time(e1), "cuda")

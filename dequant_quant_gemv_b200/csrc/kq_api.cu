@@ -116,7 +116,17 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
                     fmt == KQ_FMT_Q2_K ? "Q2_K" : "Q3_K", fmt == KQ_FMT_Q2_K ? 1024 : 2048, (long long)a.K);
     if (fmt == KQ_FMT_Q6_K && nb % 8 != 0)
         return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
-    if (fmt != KQ_FMT_Q6_K || ncol == 1) {  // lanes take (row pair, block, half)
+    a.par = 0;
+    if (fmt == KQ_FMT_Q6_K && ncol == 1 && nb >= 24 && nb % 2 == 0) {
+        // block-parity lane order: each parity's nb half-block units on whole
+        // warps of their own, so that a warp's blocks share their alignment
+        const int lr = 2 * static_cast<int>(round_up(nb, 32));
+        if (lr > kConsumers) return fail(KQ_ERR_UNSUPPORTED, "K=%lld > 32768", (long long)a.K);
+        a.par = nb;
+        a.lanes_per_rp = lr;
+        a.ps = kConsumers / lr;
+        a.parts = lr / 32;
+    } else if (fmt != KQ_FMT_Q6_K || ncol == 1) {  // lanes take (row pair, block, half)
         const int ur = 2 * nb;  // half-block units per row pair
         const int lr = ur <= 32 ? next_pow2(ur) : static_cast<int>(round_up(ur, 32));
         if (lr > kConsumers) return fail(KQ_ERR_UNSUPPORTED, "K=%lld > 32768", (long long)a.K);
@@ -719,6 +729,7 @@ int kq_gemv_steps(const kq_step* steps, int n_steps, kq_stream_t stream) {
                 sa.after = q.after != 0;
                 sa.ps = a.ps;
                 sa.lanes_per_rp = a.lanes_per_rp;
+                sa.par = a.par;
                 sa.parts = a.parts;
                 P.stage = static_cast<size_t>(a.stage_bytes);
                 P.wp = static_cast<size_t>(a.xs_offset - a.wp_offset);

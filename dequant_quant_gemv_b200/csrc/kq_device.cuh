@@ -278,6 +278,14 @@ __device__ __forceinline__ uint32_t dp4a_uu(uint32_t a, uint32_t b, uint32_t c) 
     asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
 }
+// Byte k of w as a sign-extended int (one byte permute whose selector
+// replicates the byte's sign bit into the upper bytes).
+__device__ __forceinline__ int sext_byte(uint32_t w, int k) {
+    uint32_t r;
+    const uint32_t sel = static_cast<uint32_t>(k) | ((8u + static_cast<uint32_t>(k)) * 0x1110u);
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(w), "r"(sel));
+    return static_cast<int>(r);
+}
 // Signed quants (Q8_0) with signed (ss) or unsigned (su) activation bytes.
 __device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
     int d;

@@ -666,8 +666,47 @@ __device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H) {
     return xs + kXRegionBytes * (2 * b + H);
 }
 
+// Position of the region of block b, half H: 2b + H, or with the
+// block-parity lane order over `par` blocks (single-column Q6_K) the even
+// blocks' regions first and then the odd blocks', so that consecutive lanes
+// of a warp (which take consecutive blocks of one parity) still read
+// consecutive regions.
+__device__ __forceinline__ int x_pos(int b, int H, int par) {
+    return par ? (b & 1) * par + 2 * (b >> 1) + H : 2 * b + H;
+}
+
+// The unit of consumer thread ct in the single-column lane layout: LR lanes
+// per row pair; lane u of a row pair takes block u/2, half u%2, or with the
+// block-parity order (par > 0) the first half of the row pair's lanes take
+// its even blocks and the second half the odd ones (a warp never mixes the
+// two alignment classes).  pos: the unit's activation region (x_pos).
+struct LaneUnit {
+    int rp, b, H, pos;
+    bool active;
+};
+__device__ __forceinline__ LaneUnit lane_unit(int ct, int LR, int nbl, int par) {
+    LaneUnit L;
+    L.rp = ct / LR;
+    const int u = ct - L.rp * LR;
+    if (par) {
+        const int LRp = LR >> 1;
+        const int p = u >= LRp ? 1 : 0;
+        const int up = u - p * LRp;
+        L.b = 2 * (up >> 1) + p;
+        L.H = up & 1;
+        L.active = L.b < nbl;
+        L.pos = p * par + up;
+    } else {
+        L.b = u >> 1;
+        L.H = u & 1;
+        L.active = u < 2 * nbl;
+        L.pos = u;
+    }
+    return L;
+}
+
 // Stage the K range [256*kb0, 256*(kb0+nbl)) of segment `seg` as above,
-// into the regions at `xs`.  A warp takes 4 groups of 32 activations (one
+// into the regions at `xs` (positions by x_pos).  A warp takes 4 groups of 32 activations (one
 // region) per pass: lane l holds 4 consecutive values of group l / 8, loaded
 // as one float4; a group's largest |x| and the sum of its xi are butterflies
 // over its 8 lanes, and each lane writes its 4 high and 4 low bytes as one
@@ -679,7 +718,7 @@ __device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H) {
 // scales and offsets cover 16 weights).
 template <bool PRO, bool S16 = false>
 __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, int warp, int nwarps, int lane,
-                                   int bar, int nthr, int kb0, int nbl, uint32_t part) {
+                                   int bar, int nthr, int kb0, int nbl, uint32_t part, int par = 0) {
     constexpr int U = PRO ? 4 : 8;  // one round of loads for K up to 16384 (8 with a prologue) and 16 warps
     const float* xg = a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256;
     const int quads = 2 * nbl;  // passes of 4 groups (128 activations)
@@ -762,7 +801,7 @@ __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, 
             for (int u = 0; u < 2; ++u) {
                 const int Q = base + nwarps * (c + u);
                 if (Q >= quads) break;  // warp-uniform
-                const uint32_t xr = x_region(xs, Q >> 1, Q & 1);
+                const uint32_t xr = xs + kXRegionBytes * x_pos(Q >> 1, Q & 1, par);
                 asm volatile("st.shared.u32 [%0], %1;" ::"r"(xr + kXGroupBytes * sub + e), "r"(hb[u]) : "memory");
                 asm volatile("st.shared.u32 [%0], %1;" ::"r"(xr + kXGroupBytes * sub + 32 + e), "r"(lb[u])
                              : "memory");
@@ -1128,29 +1167,51 @@ __device__ __forceinline__ void q80_unit_int(uint32_t row0, int row_bytes, int b
 
 // Q6_K unit, one column, on DP4A: row pair at row0, super-block b (210
 // bytes: ql[128], qh[64], 16 int8 scales, d), half H.  Blocks are 2-byte
-// aligned only and b's parity varies across the lanes, so each stream is
-// loaded from the 4-byte boundary at or below its start, one word more than
-// it needs, and every word rebuilt by a byte permute with a parity-chosen
-// selector (one code path for all lanes; an even block's extra words are
-// its own or its neighbour's bytes, and a row's last block is odd).  Weight
-// 128H + 32t + l: low 4 bits from ql[64H + 32(t%2) + l] (nibble t/2), top 2
-// bits from bits 2t of qh[32H + l]; 16-weight group 2t + l/16 of the half
-// has scale s = scales[8H + 2t + l/16].  Per group the exact
-// S = sum q*xi - 32*(its 16-sum of xi) = sum (q - 32)*xi, |S| <= 2^23, and
-// y = d * sum over groups of s*P*S.
+// aligned only: a block at an even index of a 16-byte aligned row starts on
+// a 4-byte boundary, one at an odd index 2 bytes past one.  ODD = 0: an
+// aligned block, its words loaded as they are; ODD = 1: each stream is
+// loaded from the 4-byte boundary below its start, one word more than it
+// needs, and every word rebuilt by a byte permute; ODD = 2: the class is
+// taken from b per lane (the lanes of a warp mix both; an even block's
+// extra words are its own or its neighbour's bytes, and a row's last block
+// is odd).  Weight 128H + 32t + l: low 4 bits from ql[64H + 32(t%2) + l]
+// (nibble t/2), top 2 bits from bits 2t of qh[32H + l]; 16-weight group
+// 2t + l/16 of the half has scale s = scales[8H + 2t + l/16].  Per group the
+// exact S = sum q*xi - 32*(its 16-sum of xi) = sum (q - 32)*xi, |S| <= 2^23,
+// and T = s*S (|T| <= 2^30, an exact int32); y = d * sum over groups of
+// P*T in fp32.
+template <int ODD>
 __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
                                              float (&out)[2][1]) {
-    const bool odd = b & 1;
+    const bool odd = ODD == 2 ? (b & 1) != 0 : ODD == 1;
     const uint32_t sel = odd ? 0x5432u : 0x3210u;
+    // the 4 words at base (4-byte aligned) of a stream starting at base + 2*odd
+    auto words = [&](uint32_t base, uint32_t (&w)[4]) {
+        if constexpr (ODD == 0) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) w[m] = ld_s32(base + 4 * m);
+        } else {
+            uint32_t L[5];
+#pragma unroll
+            for (int k = 0; k < 5; ++k) L[k] = ld_s32(base + 4 * k);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) w[m] = __byte_perm(L[m], L[m + 1], sel);
+        }
+    };
     uint32_t bw[2], sc[2][2];
     float dd[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         bw[r] = row0 + r * row_bytes + b * kQ6Bytes - (odd ? 2 : 0);  // 4-byte aligned
-        const uint32_t s0 = ld_s32(bw[r] + 192 + 8 * H), s1 = ld_s32(bw[r] + 196 + 8 * H),
-                       s2 = ld_s32(bw[r] + 200 + 8 * H);
-        sc[r][0] = __byte_perm(s0, s1, sel);
-        sc[r][1] = __byte_perm(s1, s2, sel);
+        if (ODD == 0) {
+            sc[r][0] = ld_s32(bw[r] + 192 + 8 * H);
+            sc[r][1] = ld_s32(bw[r] + 196 + 8 * H);
+        } else {
+            const uint32_t s0 = ld_s32(bw[r] + 192 + 8 * H), s1 = ld_s32(bw[r] + 196 + 8 * H),
+                           s2 = ld_s32(bw[r] + 200 + 8 * H);
+            sc[r][0] = __byte_perm(s0, s1, sel);
+            sc[r][1] = __byte_perm(s1, s2, sel);
+        }
         dd[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(ld_s32(bw[r] + 208) >> (odd ? 16 : 0))));
     }
     float y[2] = {0.f, 0.f};
@@ -1160,26 +1221,17 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
         uint32_t A[2][4], B[2][4], Hh[2][4];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-            uint32_t L[5];
-#pragma unroll
-            for (int k = 0; k < 5; ++k) L[k] = ld_s32(bw[r] + 64 * H + 16 * s + 4 * k);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) A[r][m] = __byte_perm(L[m], L[m + 1], sel);
-#pragma unroll
-            for (int k = 0; k < 5; ++k) L[k] = ld_s32(bw[r] + 64 * H + 32 + 16 * s + 4 * k);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) B[r][m] = __byte_perm(L[m], L[m + 1], sel);
-#pragma unroll
-            for (int k = 0; k < 5; ++k) L[k] = ld_s32(bw[r] + 128 + 32 * H + 16 * s + 4 * k);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) Hh[r][m] = __byte_perm(L[m], L[m + 1], sel);
+            words(bw[r] + 64 * H + 16 * s, A[r]);
+            words(bw[r] + 64 * H + 32 + 16 * s, B[r]);
+            words(bw[r] + 128 + 32 * H + 16 * s, Hh[r]);
         }
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const uint4 xh = ld_s128(xr + kXGroupBytes * t + 16 * s);
             const uint4 xl = ld_s128(xr + kXGroupBytes * t + 32 + 16 * s);
-            int hi[2] = {0, 0};
-            uint32_t lo[2] = {0u, 0u};
+            // two accumulator chains per row and plane (m even / odd)
+            int hi[2][2] = {{0, 0}, {0, 0}};
+            uint32_t lo[2][2] = {{0u, 0u}, {0u, 0u}};
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
 #pragma unroll
@@ -1189,8 +1241,8 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
                     const uint32_t top = t == 0 ? (Hh[r][m] << 4) : t == 1 ? (Hh[r][m] << 2)
                                                       : t == 2 ? Hh[r][m] : (Hh[r][m] >> 2);
                     const uint32_t q = low | (top & 0x30303030u);
-                    hi[r] = dp4a_us(q, u4w(xh, m), hi[r]);
-                    lo[r] = dp4a_uu(q, u4w(xl, m), lo[r]);
+                    hi[r][m & 1] = dp4a_us(q, u4w(xh, m), hi[r][m & 1]);
+                    lo[r][m & 1] = dp4a_uu(q, u4w(xl, m), lo[r][m & 1]);
                 }
             }
             const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * t);  // X, P, 16-sums
@@ -1199,9 +1251,9 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
             const int g = 2 * t + s;  // group within the half
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                const int S = hi[r] * 256 + static_cast<int>(lo[r]) - x32;
-                const float sv = static_cast<float>(static_cast<int8_t>((sc[r][g >> 2] >> (8 * (g & 3))) & 0xFFu));
-                y[r] = fmaf(sv * P, static_cast<float>(S), y[r]);
+                const int S = (hi[r][0] + hi[r][1]) * 256 + static_cast<int>(lo[r][0] + lo[r][1]) - x32;
+                const int sv = sext_byte(sc[r][g >> 2], g & 3);  // the group's int8 scale
+                y[r] = fmaf(P, static_cast<float>(sv * S), y[r]);
             }
         }
     }
@@ -1224,7 +1276,8 @@ template <int FMT, int NCOL, bool INT, bool PRO>
 __device__ __forceinline__ void stage_all(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar,
                                           int kb0, int nbl, uint32_t part) {
     if constexpr (INT)
-        stage_x_int<PRO, (FMT == 2 || FMT == 4 || FMT == 5)>(a, seg, xs, ct >> 5, nthr >> 5, ct & 31, bar, nthr, kb0, nbl, part);
+        stage_x_int<PRO, (FMT == 2 || FMT == 4 || FMT == 5)>(a, seg, xs, ct >> 5, nthr >> 5, ct & 31, bar, nthr, kb0,
+                                                             nbl, part, a.par);
     else if constexpr (PRO)
         stage_x_pro<FMT, NCOL>(ProStage{a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256,
                                         a.pro == 1 ? a.gamma + static_cast<int64_t>(kb0) * 256 : nullptr, a.K, a.ldx,
@@ -1303,15 +1356,17 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     int u_rp, u_b, u_H, group, part;
     bool u_active;
     int kappa = 0;
+    int u_pos = 0;  // the lane's integer activation region (single column)
     if (FMT != 2 || NCOL == 1) {  // lanes take (row pair, block, half)
         const int LR = a.lanes_per_rp;
-        u_rp = ct / LR;
-        const int u = ct - u_rp * LR;
-        u_active = u < 2 * nbl;
-        u_b = u >> 1;
-        u_H = u & 1;
+        const LaneUnit L = lane_unit(ct, LR, nbl, a.par);
+        u_rp = L.rp;
+        u_b = L.b;
+        u_H = L.H;
+        u_active = L.active;
+        u_pos = L.pos;
         group = LR < 32 ? LR : 32;
-        part = LR > 32 ? (u >> 5) : 0;
+        part = LR > 32 ? ((ct - u_rp * LR) >> 5) : 0;
     } else {
         const int LRw = a.lanes_per_rp;  // lanes per row pair inside one warp
         kappa = cw;
@@ -1337,7 +1392,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
     constexpr bool INT = NCOL == 1;
     const uint32_t xcopy = INT ? kXRegionBytes * 2 * nb : 4 * NCOL * xcs;
     const uint32_t xs_s = smem_u32(xs) + (shared_x ? 0 : g * xcopy);
-    const uint32_t xri = x_region(xs_s, u_b, u_H);  // this lane's integer region
+    const uint32_t xri = xs_s + kXRegionBytes * u_pos;  // this lane's integer region
     const uint32_t sbuf_s = smem_u32(sbuf), wp_s = smem_u32(wp) + 4 * g * wp_group;
     const uint32_t xr = xs_s + 4 * (region * kRegion);
 
@@ -1395,7 +1450,9 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             } else if constexpr (INT && FMT == 6) {
                 q80_unit_int(row0, srow, u_b, u_H, xri, out);
             } else if constexpr (INT) {
-                q6k_unit_int(row0, srow, u_b, u_H, xri, out);
+                if (a.par == 0) q6k_unit_int<2>(row0, srow, u_b, u_H, xri, out);
+                else if (u_b & 1) q6k_unit_int<1>(row0, srow, u_b, u_H, xri, out);
+                else q6k_unit_int<0>(row0, srow, u_b, u_H, xri, out);
             } else if constexpr (FMT == 1) {
                 q4k_unit<NCOL>(row0, srow, u_b, u_H, xr, xcs, out);
             } else {

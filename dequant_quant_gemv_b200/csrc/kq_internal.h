@@ -36,6 +36,7 @@ struct GemvArgs {
     // schedule (from plan_gemv)
     int ps;                  // row pairs per stage
     int lanes_per_rp;        // lanes per row pair (several-column Q6_K: per row pair and warp)
+    int par;                 // single-column Q6_K: block-parity lane order over par blocks (0: off)
     int parts;               // partial sums per row pair
     int nstage;
     int stage_bytes;
@@ -74,6 +75,7 @@ struct StepArgs {
     int after;           // wait for every CTA to finish the steps before this one
     int ps;              // row pairs per stage
     int lanes_per_rp;    // as in GemvArgs
+    int par;             // as in GemvArgs
     int parts;
 };
 

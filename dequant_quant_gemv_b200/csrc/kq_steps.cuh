@@ -58,6 +58,7 @@ __device__ __forceinline__ GemvArgs step_view(const StepArgs& s) {
     a.ksplit = 1;
     a.ps = s.ps;
     a.lanes_per_rp = s.lanes_per_rp;
+    a.par = s.par;
     a.parts = s.parts;
     a.pro = s.pro;
     a.gamma = s.gamma;
@@ -191,15 +192,14 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
         // this lane's unit within a stage (as in the single-column kernel)
         const int nb = s.nb;
         const int LR = s.lanes_per_rp;
-        const int u_rp = ct / LR;
-        const int u = ct - u_rp * LR;
-        const bool u_active = u < 2 * nb;
-        const int u_b = u >> 1, u_H = u & 1;
+        const LaneUnit L = lane_unit(ct, LR, nb, s.par);
+        const int u_rp = L.rp, u_b = L.b, u_H = L.H;
+        const bool u_active = L.active;
         const int group = LR < 32 ? LR : 32;
-        const int part = LR > 32 ? (u >> 5) : 0;
+        const int part = LR > 32 ? ((ct - u_rp * LR) >> 5) : 0;
         const int parts = s.parts;
         const bool direct = parts == 1;
-        const uint32_t xri = x_region(xs_s, u_b, u_H);
+        const uint32_t xri = xs_s + kXRegionBytes * L.pos;
         const uint32_t wp_s = smem_u32(smem + A.wp_offset) + 4 * g * (2 * s.ps * parts * 2);
         const int srow = static_cast<int>(s.row_bytes);
 
@@ -227,7 +227,9 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
                 else if (s.fmt == 4) q2k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else if (s.fmt == 5) q3k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else if (s.fmt == 6) q80_unit_int(rw, srow, u_b, u_H, xri, out);
-                else q6k_unit_int(rw, srow, u_b, u_H, xri, out);
+                else if (s.par == 0) q6k_unit_int<2>(rw, srow, u_b, u_H, xri, out);
+                else if (u_b & 1) q6k_unit_int<1>(rw, srow, u_b, u_H, xri, out);
+                else q6k_unit_int<0>(rw, srow, u_b, u_H, xri, out);
             }
             // butterfly over the lanes of this row pair (fixed order)
 #pragma unroll
