@@ -149,7 +149,13 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     // multi-column kernels need more registers per thread and keep one.
     const int ng = ncol == 1 ? 2 : 1;
     const bool shared_x = a.x_seg_stride == 0;
-    const size_t wp_bytes = round_up(sizeof(float) * ng * 2 * a.ps * a.parts * 2 * ncol, 128);
+    // partial sums: the general kernel's group buffers, or (one column) the
+    // larger of those and the single-matrix kernel's per-slot buffers
+    size_t wp_bytes = round_up(sizeof(float) * ng * 2 * a.ps * a.parts * 2 * ncol, 128);
+    if (ncol == 1) {
+        const size_t lean = round_up(static_cast<size_t>(kMaxStages) * a.ps * (8 * a.parts + 8), 128);
+        if (lean > wp_bytes) wp_bytes = lean;
+    }
     // one column: integer activation regions (2 x 336 bytes per
     // super-block); otherwise fp32 regions
     const size_t xcopy = ncol == 1 ? static_cast<size_t>(672) * nb
@@ -402,6 +408,19 @@ static cudaError_t dispatch(const GemvArgs& a, const LaunchPlan& p, int fmt, int
     }
 }
 
+// One column of one whole matrix: the lean single-matrix kernel.
+static cudaError_t dispatch_gemv1(const GemvArgs& a, const LaunchPlan& p, int fmt, cudaStream_t s) {
+    const bool pro = a.pro != 0;
+    switch (fmt) {
+        case KQ_FMT_Q4_K: return pro ? launch_gemv1<1, true>(a, p, s) : launch_gemv1<1, false>(a, p, s);
+        case KQ_FMT_Q6_K: return pro ? launch_gemv1<2, true>(a, p, s) : launch_gemv1<2, false>(a, p, s);
+        case KQ_FMT_Q5_K: return pro ? launch_gemv1<3, true>(a, p, s) : launch_gemv1<3, false>(a, p, s);
+        case KQ_FMT_Q2_K: return pro ? launch_gemv1<4, true>(a, p, s) : launch_gemv1<4, false>(a, p, s);
+        case KQ_FMT_Q3_K: return pro ? launch_gemv1<5, true>(a, p, s) : launch_gemv1<5, false>(a, p, s);
+        default: return pro ? launch_gemv1<6, true>(a, p, s) : launch_gemv1<6, false>(a, p, s);
+    }
+}
+
 static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt, int nt, cudaStream_t s) {
     const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 4 : 8) + (nt - 1) * 2 + (p.ng - 1);
     switch (key) {
@@ -453,6 +472,8 @@ static int run(GemvArgs& a, int fmt, int k, bool mma, cudaStream_t stream) {
     int st = plan_for(fmt, k, mma, a, p);
     if (st != KQ_OK) return st;
     if (mma) err = dispatch_mma(a, p, fmt, k <= 4 ? 1 : 2, stream);
+    else if (k == 1 && a.n_seg == 1 && !a.ids && a.ksplit == 1 && a.x_seg_stride == 0)
+        err = dispatch_gemv1(a, p, fmt, stream);
     else err = dispatch(a, p, fmt, padded_cols(k), stream);
     if (err != cudaSuccess) return cuda_fail(err, "kernel launch");
     if (a.ksplit > 1 && !a.cluster) {  // cluster splits add their partial sums in the kernel

@@ -116,6 +116,9 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p);
 
 template <int FMT, int NCOL, int NG>
 cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
+// The single-column GEMV of one whole matrix (one segment, K unsplit).
+template <int FMT, bool PRO>
+cudaError_t launch_gemv1(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
 // Tensor-core kernel for 2..8 columns: NT n-tiles of 8 (4 columns each).
 int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p);
 template <int FMT, int NT, int NG>

@@ -71,9 +71,6 @@ __device__ __forceinline__ uint32_t h22u(__half2 v) { return *reinterpret_cast<c
 __device__ __forceinline__ uint32_t pack_h2(__half lo, __half hi) {
     return static_cast<uint32_t>(__half_as_ushort(lo)) | (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
 }
-__device__ __forceinline__ void st_s64u(uint32_t a, uint32_t x, uint32_t y) {
-    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
-}
 __device__ __forceinline__ void st_s32u(uint32_t a, uint32_t v) {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
