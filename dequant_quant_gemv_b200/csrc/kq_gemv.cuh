@@ -361,10 +361,16 @@ __device__ inline void prefetch_activations(const GemvArgs& a, int kb0, int nbl)
 // from the 16-byte boundary at or below the range start (bulk copies move
 // whole 16-byte units), so the range begins (kb0 * BS) % 16 bytes into the
 // smem row.  Rows are multiples of 16 bytes, so no copy leaves its row.
+// `staged` (single-matrix kernel): after its first `lead` stages the
+// producer waits until the consumers have staged the activations (they set
+// *staged), so that the activation loads do not queue behind a full ring of
+// weight copies; the wait is a hint and gives up after kStagedWaitNs.
+constexpr unsigned long long kStagedWaitNs = 100000ull;
+
 template <int BS>
 __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empty, volatile int* abort_flag,
                                uint8_t* sbuf, int64_t rp_begin, int64_t rp_end, int64_t rps, int ns, int kb0,
-                               int nbl, int srow, bool contiguous) {
+                               int nbl, int srow, bool contiguous, volatile int* staged = nullptr, int lead = 0) {
     if (a.ids) pdl_wait();  // routed ids may come from the previous grid
     const uint64_t pol = l2_evict_first();
     const unsigned long long lim = a.wait_ns && blockIdx.x == 0 ? a.wait_ns : kWaitNs;
@@ -406,6 +412,11 @@ __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empt
         } else {
             mbar_arrive(&full[slot]);
             ring.skip(slot);
+        }
+        if (staged && it.count == lead) {
+            const unsigned long long t0 = globaltimer_ns();
+            while (!*staged && !*abort_flag && globaltimer_ns() - t0 < kStagedWaitNs) {
+            }
         }
     }
     // Let every copy this CTA issued land before the CTA can exit, abort or
@@ -1229,9 +1240,8 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
         for (int t = 0; t < 4; ++t) {
             const uint4 xh = ld_s128(xr + kXGroupBytes * t + 16 * s);
             const uint4 xl = ld_s128(xr + kXGroupBytes * t + 32 + 16 * s);
-            // two accumulator chains per row and plane (m even / odd)
-            int hi[2][2] = {{0, 0}, {0, 0}};
-            uint32_t lo[2][2] = {{0u, 0u}, {0u, 0u}};
+            int hi[2] = {0, 0};
+            uint32_t lo[2] = {0u, 0u};
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
 #pragma unroll
@@ -1241,8 +1251,8 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
                     const uint32_t top = t == 0 ? (Hh[r][m] << 4) : t == 1 ? (Hh[r][m] << 2)
                                                       : t == 2 ? Hh[r][m] : (Hh[r][m] >> 2);
                     const uint32_t q = low | (top & 0x30303030u);
-                    hi[r][m & 1] = dp4a_us(q, u4w(xh, m), hi[r][m & 1]);
-                    lo[r][m & 1] = dp4a_uu(q, u4w(xl, m), lo[r][m & 1]);
+                    hi[r] = dp4a_us(q, u4w(xh, m), hi[r]);
+                    lo[r] = dp4a_uu(q, u4w(xl, m), lo[r]);
                 }
             }
             const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * t);  // X, P, 16-sums
@@ -1251,7 +1261,7 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
             const int g = 2 * t + s;  // group within the half
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                const int S = (hi[r][0] + hi[r][1]) * 256 + static_cast<int>(lo[r][0] + lo[r][1]) - x32;
+                const int S = hi[r] * 256 + static_cast<int>(lo[r]) - x32;
                 const int sv = sext_byte(sc[r][g >> 2], g & 3);  // the group's int8 scale
                 y[r] = fmaf(P, static_cast<float>(sv * S), y[r]);
             }

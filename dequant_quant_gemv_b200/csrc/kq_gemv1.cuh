@@ -33,12 +33,20 @@ __host__ __device__ constexpr int lean_red_bytes(int ps, int parts) {
     return kMaxStages * ps * (8 * parts + 8);
 }
 
-template <int FMT, bool PRO, bool DIRECT>
+// Weight stages copied before the producer waits for the activation
+// staging (measured on the 8B-shaped chain: 2 beat 1 and a full ring).
+constexpr int kLeadStages = 2;
+
+// FULL: a row pair spans at least a whole warp (lanes_per_rp >= 32), so the
+// butterfly runs all five levels unconditionally.  PAR: the block-parity
+// lane order (single-column Q6_K).
+template <int FMT, bool PRO, bool DIRECT, bool FULL, bool PAR>
 __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __grid_constant__ GemvArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 2 * kMaxStages * 8);
+    volatile int* staged = abort_flag + 1;  // set once the activations are staged
     uint8_t* sbuf = smem + a.sbuf_offset;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -55,6 +63,7 @@ __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __g
         if (!DIRECT)
             for (int i = 0; i < ns * ps; ++i) mbar_init(&red[i], parts);
         *abort_flag = 0;
+        *staged = 0;
         fence_barrier_init();
     }
     __syncthreads();
@@ -69,7 +78,7 @@ __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __g
         if (lane == 0) {
             prefetch_activations(a, 0, nb);
             produce_stages<BS>(a, full, empty, abort_flag, sbuf, rp_begin, rp_end, rps, ns, 0, nb,
-                               static_cast<int>(a.row_bytes), true);
+                               static_cast<int>(a.row_bytes), true, staged, kLeadStages);
         }
         return;
     }
@@ -79,7 +88,7 @@ __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __g
     const int g = ct_all >> 8;                 // consumer group: stages s = g, g + 2, ...
     const int ct = ct_all & (kConsumers - 1);
     const int LR = a.lanes_per_rp;
-    const LaneUnit L = lane_unit(ct, LR, nb, a.par);
+    const LaneUnit L = lane_unit(ct, LR, nb, PAR ? a.par : 0);
     const int part = DIRECT ? 0 : ((ct - L.rp * LR) >> 5);
     const uint32_t xs_s = smem_u32(smem + a.xs_offset);
     const uint32_t xri = xs_s + kXRegionBytes * L.pos;
@@ -95,6 +104,7 @@ __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __g
     stage_all<FMT, 1, true, PRO>(a, 0, xs_s, ct_all, 2 * kConsumers, 3, 0, nb, pro_r);
     float rinv = 1.f;
     if (PRO && a.pro == 1) rinv = ld_s32f(pro_inv_addr(pro_r));
+    if (ct_all == 0) *staged = 1;
 
     const int64_t nrp_all = rp_end - rp_begin;
     const int nst = static_cast<int>((nrp_all + ps - 1) / ps);
@@ -123,16 +133,14 @@ __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __g
             else if constexpr (FMT == 4) q2k_unit_int(row0, srow, L.b, L.H, xri, out);
             else if constexpr (FMT == 5) q3k_unit_int(row0, srow, L.b, L.H, xri, out);
             else if constexpr (FMT == 6) q80_unit_int(row0, srow, L.b, L.H, xri, out);
-            else {
-                if (a.par == 0) q6k_unit_int<2>(row0, srow, L.b, L.H, xri, out);
-                else if (L.b & 1) q6k_unit_int<1>(row0, srow, L.b, L.H, xri, out);
-                else q6k_unit_int<0>(row0, srow, L.b, L.H, xri, out);
-            }
+            else if constexpr (!PAR) q6k_unit_int<2>(row0, srow, L.b, L.H, xri, out);
+            else if (L.b & 1) q6k_unit_int<1>(row0, srow, L.b, L.H, xri, out);
+            else q6k_unit_int<0>(row0, srow, L.b, L.H, xri, out);
         }
         // butterfly over the lanes of this row pair (fixed order)
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) {
-            if (off < LR) {
+            if (FULL || off < LR) {
                 out[0][0] += __shfl_xor_sync(0xffffffffu, out[0][0], off);
                 out[1][0] += __shfl_xor_sync(0xffffffffu, out[1][0], off);
             }
@@ -184,7 +192,12 @@ __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __g
 
 template <int FMT, bool PRO>
 cudaError_t launch_gemv1(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream) {
-    auto kern = a.parts == 1 ? gemv1_kernel<FMT, PRO, true> : gemv1_kernel<FMT, PRO, false>;
+    // the layouts that occur: a row pair on part of a warp, on one whole
+    // warp, or on several (with the parity order only for Q6_K)
+    auto kern = a.lanes_per_rp < 32 ? gemv1_kernel<FMT, PRO, true, false, false>
+              : a.parts == 1        ? gemv1_kernel<FMT, PRO, true, true, false>
+              : (FMT == 2 && a.par) ? gemv1_kernel<FMT, PRO, false, true, FMT == 2>
+                                    : gemv1_kernel<FMT, PRO, false, true, false>;
     cudaError_t err = ensure_smem_attr(reinterpret_cast<const void*>(kern), p.smem_bytes);
     if (err != cudaSuccess) return err;
     cudaLaunchConfig_t cfg = {};
