@@ -111,13 +111,16 @@ int plan_gemv(int fmt, int ncol, GemvArgs& a, LaunchPlan& p) {
     const int nb = a.nbs;  // blocks per K range (all of K unless split)
     if (fmt != KQ_FMT_Q4_K && fmt != KQ_FMT_Q6_K && ncol > 1)
         return fail(KQ_ERR_UNSUPPORTED, "format %d with %d columns: not in this kernel", fmt, ncol);
-    if ((fmt == KQ_FMT_Q2_K && nb % 4 != 0) || (fmt == KQ_FMT_Q3_K && nb % 8 != 0))
-        return fail(KQ_ERR_UNSUPPORTED, "%s rows must be 16-byte aligned (K %% %d == 0), K=%lld",
-                    fmt == KQ_FMT_Q2_K ? "Q2_K" : "Q3_K", fmt == KQ_FMT_Q2_K ? 1024 : 2048, (long long)a.K);
-    if (fmt == KQ_FMT_Q6_K && nb % 8 != 0)
-        return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
+    // Rows (and split-K ranges) off the 16-byte grid: whole stages are copied
+    // from the boundary below their start, but per-row copies (split K) need
+    // 16-byte rows, and the several-column Q6_K layout 16-byte blocks groups.
+    const bool rows16 = a.row_bytes % 16 == 0;
+    if (a.ksplit > 1 && (!rows16 || (static_cast<int64_t>(nb) * kq_block_bytes(fmt)) % 16 != 0))
+        return fail(KQ_ERR_UNSUPPORTED, "split K needs 16-byte aligned rows and ranges, K=%lld", (long long)a.K);
+    if (fmt == KQ_FMT_Q6_K && ncol > 1 && nb % 8 != 0)
+        return fail(KQ_ERR_UNSUPPORTED, "Q6_K with %d columns needs K %% 2048 == 0, K=%lld", ncol, (long long)a.K);
     a.par = 0;
-    if (fmt == KQ_FMT_Q6_K && ncol == 1 && nb >= 24 && nb % 2 == 0) {
+    if (fmt == KQ_FMT_Q6_K && ncol == 1 && nb >= 24 && nb % 2 == 0 && a.row_bytes % 4 == 0) {
         // block-parity lane order: each parity's nb half-block units on whole
         // warps of their own, so that a warp's blocks share their alignment
         const int lr = 2 * static_cast<int>(round_up(nb, 32));
@@ -443,8 +446,9 @@ static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt,
 // kernel, every column group of the call included, so a column's arithmetic
 // never depends on how the call was grouped.  Q2_K, Q3_K and Q8_0 have no
 // tensor-core kernel: their columns run one single-column launch each.
-static bool use_mma(int fmt, int k) {
-    return k >= 2 && fmt != KQ_FMT_Q2_K && fmt != KQ_FMT_Q3_K && fmt != KQ_FMT_Q8_0;
+static bool use_mma(int fmt, int k, int64_t row_bytes) {
+    // (its per-row copies need 16-byte rows)
+    return k >= 2 && fmt != KQ_FMT_Q2_K && fmt != KQ_FMT_Q3_K && fmt != KQ_FMT_Q8_0 && row_bytes % 16 == 0;
 }
 
 static int plan_for(int fmt, int k, bool mma, GemvArgs& a, LaunchPlan& p) {
@@ -492,6 +496,7 @@ static void choose_split(int fmt, int64_t N, int nb, int sm_count, int* S, int* 
     *nbs = nb;
     const int64_t P = (N + 1) / 2;
     if (P * 2 > sm_count) return;                       // enough row pairs already
+    if (static_cast<int64_t>(nb) * kq_block_bytes(fmt) % 16 != 0) return;  // rows off the 16-byte grid
     const int unit = fmt == KQ_FMT_Q6_K || fmt == KQ_FMT_Q3_K ? 8 : fmt == KQ_FMT_Q2_K ? 4 : 1;
     const int max_s = nb / unit;
     int want = static_cast<int>((sm_count + P - 1) / P);
@@ -520,7 +525,7 @@ static int max_fitting_cols(const GemvArgs& proto, int fmt, bool mma) {
 static int run_grouped(GemvArgs& a, int fmt, int k, cudaStream_t stream) {
     // the tensor-core kernel when its activation fragments fit (for the
     // whole call), else the CUDA-core kernel
-    bool mma = use_mma(fmt, k);
+    bool mma = use_mma(fmt, k, a.row_bytes);
     int g = mma ? max_fitting_cols(a, fmt, true) : 0;
     if (g == 0) {
         mma = false;

@@ -397,9 +397,16 @@ __device__ void produce_stages(const GemvArgs& a, uint64_t* full, uint64_t* empt
             const uint8_t* src = a.W + e * a.seg_stride + st.row0 * a.row_bytes;
             uint8_t* dst = sbuf + static_cast<size_t>(slot) * a.stage_bytes;
             if (contiguous) {
-                const uint32_t bytes = static_cast<uint32_t>(st.nrows * a.row_bytes);
+                // rows need not be 16-byte aligned: copy whole 16-byte units
+                // from the boundary at or below the stage's first byte (the
+                // consumers index from src % 16); the last unit never reaches
+                // past the 16-byte granule of the stage's last byte
+                const uintptr_t s0 = reinterpret_cast<uintptr_t>(src);
+                const uintptr_t b0 = s0 & ~uintptr_t(15);
+                const uintptr_t e0 = (s0 + static_cast<uintptr_t>(st.nrows * a.row_bytes) + 15) & ~uintptr_t(15);
+                const uint32_t bytes = static_cast<uint32_t>(e0 - b0);
                 mbar_arrive_expect_tx(&full[slot], bytes);
-                bulk_g2s(dst, src, bytes, &full[slot], pol);
+                bulk_g2s(dst, reinterpret_cast<const void*>(b0), bytes, &full[slot], pol);
             } else {
                 const int64_t off = static_cast<int64_t>(kb0) * BS;
                 const int64_t off16 = off & ~int64_t(15);
@@ -1041,13 +1048,15 @@ __device__ __forceinline__ void q2k_unit_int(uint32_t row0, int row_bytes, int b
 // sum over 32-groups of P*(that sum), in fp32.
 __device__ __forceinline__ void q3k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
                                              float (&out)[2][1]) {
-    const bool odd = b & 1;
-    const uint32_t sel = odd ? 0x5432u : 0x3210u;
     uint32_t Q[2][8], M[2][8], sc[2][2], hs[2];
     float dd[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-        const uint32_t bw = row0 + r * row_bytes + b * kQ3Bytes - (odd ? 2 : 0);  // 4-byte aligned
+        // the block's alignment class, read off its address (per row)
+        const uint32_t addr = row0 + r * row_bytes + b * kQ3Bytes;
+        const bool odd = (addr & 2u) != 0;
+        const uint32_t sel = odd ? 0x5432u : 0x3210u;
+        const uint32_t bw = addr - (odd ? 2u : 0u);  // 4-byte aligned
         uint32_t L[9];
 #pragma unroll
         for (int t = 0; t < 9; ++t) L[t] = ld_s32(bw + 32 + 32 * H + 4 * t);
@@ -1179,13 +1188,14 @@ __device__ __forceinline__ void q80_unit_int(uint32_t row0, int row_bytes, int b
 // Q6_K unit, one column, on DP4A: row pair at row0, super-block b (210
 // bytes: ql[128], qh[64], 16 int8 scales, d), half H.  Blocks are 2-byte
 // aligned only: a block at an even index of a 16-byte aligned row starts on
-// a 4-byte boundary, one at an odd index 2 bytes past one.  ODD = 0: an
+// a 4-byte boundary, one at an odd index 2 bytes past one (rows whose
+// length is not a multiple of 16 bytes shift this per row).  ODD = 0: an
 // aligned block, its words loaded as they are; ODD = 1: each stream is
 // loaded from the 4-byte boundary below its start, one word more than it
 // needs, and every word rebuilt by a byte permute; ODD = 2: the class is
-// taken from b per lane (the lanes of a warp mix both; an even block's
-// extra words are its own or its neighbour's bytes, and a row's last block
-// is odd).  Weight 128H + 32t + l: low 4 bits from ql[64H + 32(t%2) + l]
+// read off each row's block address (the lanes of a warp mix both; the
+// extra word is the block's own or its neighbour's bytes, or at the end of
+// a stage the slot's slack).  Weight 128H + 32t + l: low 4 bits from ql[64H + 32(t%2) + l]
 // (nibble t/2), top 2 bits from bits 2t of qh[32H + l]; 16-weight group
 // 2t + l/16 of the half has scale s = scales[8H + 2t + l/16].  Per group the
 // exact S = sum q*xi - 32*(its 16-sum of xi) = sum (q - 32)*xi, |S| <= 2^23,
@@ -1194,10 +1204,21 @@ __device__ __forceinline__ void q80_unit_int(uint32_t row0, int row_bytes, int b
 template <int ODD>
 __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b, int H, uint32_t xr,
                                              float (&out)[2][1]) {
-    const bool odd = ODD == 2 ? (b & 1) != 0 : ODD == 1;
-    const uint32_t sel = odd ? 0x5432u : 0x3210u;
-    // the 4 words at base (4-byte aligned) of a stream starting at base + 2*odd
-    auto words = [&](uint32_t base, uint32_t (&w)[4]) {
+    // each row's alignment class: fixed by ODD, or (ODD == 2) read off the
+    // block's shared-memory address, which also covers rows whose length is
+    // not a multiple of 4 bytes (the two rows of a pair then differ)
+    bool odd[2];
+    uint32_t sel[2], bw[2], sc[2][2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const uint32_t addr = row0 + r * row_bytes + b * kQ6Bytes;
+        odd[r] = ODD == 2 ? (addr & 2u) != 0 : ODD == 1;
+        sel[r] = odd[r] ? 0x5432u : 0x3210u;
+        bw[r] = addr - (odd[r] ? 2u : 0u);  // 4-byte aligned
+    }
+    // the 4 words at base (4-byte aligned) of a stream of row r starting at
+    // base + 2*odd[r]
+    auto words = [&](int r, uint32_t base, uint32_t (&w)[4]) {
         if constexpr (ODD == 0) {
 #pragma unroll
             for (int m = 0; m < 4; ++m) w[m] = ld_s32(base + 4 * m);
@@ -1206,24 +1227,23 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
 #pragma unroll
             for (int k = 0; k < 5; ++k) L[k] = ld_s32(base + 4 * k);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) w[m] = __byte_perm(L[m], L[m + 1], sel);
+            for (int m = 0; m < 4; ++m) w[m] = __byte_perm(L[m], L[m + 1], sel[r]);
         }
     };
-    uint32_t bw[2], sc[2][2];
     float dd[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-        bw[r] = row0 + r * row_bytes + b * kQ6Bytes - (odd ? 2 : 0);  // 4-byte aligned
         if (ODD == 0) {
             sc[r][0] = ld_s32(bw[r] + 192 + 8 * H);
             sc[r][1] = ld_s32(bw[r] + 196 + 8 * H);
         } else {
             const uint32_t s0 = ld_s32(bw[r] + 192 + 8 * H), s1 = ld_s32(bw[r] + 196 + 8 * H),
                            s2 = ld_s32(bw[r] + 200 + 8 * H);
-            sc[r][0] = __byte_perm(s0, s1, sel);
-            sc[r][1] = __byte_perm(s1, s2, sel);
+            sc[r][0] = __byte_perm(s0, s1, sel[r]);
+            sc[r][1] = __byte_perm(s1, s2, sel[r]);
         }
-        dd[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(ld_s32(bw[r] + 208) >> (odd ? 16 : 0))));
+        dd[r] = __half2float(
+            __ushort_as_half(static_cast<unsigned short>(ld_s32(bw[r] + 208) >> (odd[r] ? 16 : 0))));
     }
     float y[2] = {0.f, 0.f};
 #pragma unroll
@@ -1232,9 +1252,9 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
         uint32_t A[2][4], B[2][4], Hh[2][4];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-            words(bw[r] + 64 * H + 16 * s, A[r]);
-            words(bw[r] + 64 * H + 32 + 16 * s, B[r]);
-            words(bw[r] + 128 + 32 * H + 16 * s, Hh[r]);
+            words(r, bw[r] + 64 * H + 16 * s, A[r]);
+            words(r, bw[r] + 64 * H + 32 + 16 * s, B[r]);
+            words(r, bw[r] + 128 + 32 * H + 16 * s, Hh[r]);
         }
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -1448,7 +1468,13 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) gemv_kernel(const __g
             for (int j = 0; j < NCOL; ++j) out[r][j] = 0.f;
         const bool work = u_active && u_rp < st.nrp && !*abort_flag;
         if (work) {
-            const uint32_t row0 = sbuf_s + slot * a.stage_bytes + 2 * u_rp * srow;
+            uint32_t row0 = sbuf_s + slot * a.stage_bytes + 2 * u_rp * srow;
+            if (a.ksplit == 1) {  // a contiguous stage starts src % 16 bytes into its slot
+                int64_t e = st.seg;
+                if (a.ids) e = a.ids[st.seg];
+                row0 += static_cast<uint32_t>(
+                    reinterpret_cast<uintptr_t>(a.W + e * a.seg_stride + st.row0 * a.row_bytes) & 15u);
+            }
             if constexpr (INT && FMT == 1) {
                 q4k_unit_int(row0, srow, u_b, u_H, xri, out);
             } else if constexpr (INT && FMT == 3) {

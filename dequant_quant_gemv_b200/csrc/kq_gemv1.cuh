@@ -127,7 +127,9 @@ __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __g
         }
         float out[2][1] = {{0.f}, {0.f}};
         if (mine && !dead) {
-            const uint32_t row0 = sbuf_s + static_cast<uint32_t>(slot) * stage_bytes;
+            // the stage starts (its first byte's address % 16) into its slot
+            const uint32_t row0 = sbuf_s + static_cast<uint32_t>(slot) * stage_bytes +
+                                  static_cast<uint32_t>(reinterpret_cast<uintptr_t>(a.W + 2 * rp0 * a.row_bytes) & 15u);
             if constexpr (FMT == 1) q4k_unit_int(row0, srow, L.b, L.H, xri, out);
             else if constexpr (FMT == 3) q5k_unit_int(row0, srow, L.b, L.H, xri, out);
             else if constexpr (FMT == 4) q2k_unit_int(row0, srow, L.b, L.H, xri, out);

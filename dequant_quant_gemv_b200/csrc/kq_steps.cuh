@@ -122,9 +122,14 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
                         ok = false;
                         break;
                     }
-                    const uint32_t bytes = static_cast<uint32_t>(rows * s.row_bytes);
+                    // from the 16-byte boundary at or below the stage's
+                    // first byte (rows need not be 16-byte aligned)
+                    const uintptr_t s0 = reinterpret_cast<uintptr_t>(s.W + row0 * s.row_bytes);
+                    const uintptr_t b0 = s0 & ~uintptr_t(15);
+                    const uintptr_t e0 = (s0 + static_cast<uintptr_t>(rows * s.row_bytes) + 15) & ~uintptr_t(15);
+                    const uint32_t bytes = static_cast<uint32_t>(e0 - b0);
                     mbar_arrive_expect_tx(&full[slot], bytes);
-                    bulk_g2s(sbuf + static_cast<size_t>(slot) * A.slot_bytes, s.W + row0 * s.row_bytes, bytes,
+                    bulk_g2s(sbuf + static_cast<size_t>(slot) * A.slot_bytes, reinterpret_cast<const void*>(b0), bytes,
                              &full[slot], pol);
                     ring.issue(slot, phase);
                 }
@@ -221,7 +226,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) steps_kernel(const __
             float out[2][1] = {{0.f}, {0.f}};
             const bool work = u_active && u_rp < nrp && !*abort_flag;
             if (work) {
-                const uint32_t rw = sbuf_s + slot * A.slot_bytes + 2 * u_rp * srow;
+                const uint32_t rw = sbuf_s + slot * A.slot_bytes + 2 * u_rp * srow +
+                                    static_cast<uint32_t>(reinterpret_cast<uintptr_t>(s.W + row0 * s.row_bytes) & 15u);
                 if (s.fmt == 1) q4k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else if (s.fmt == 3) q5k_unit_int(rw, srow, u_b, u_H, xri, out);
                 else if (s.fmt == 4) q2k_unit_int(rw, srow, u_b, u_H, xri, out);

@@ -54,9 +54,13 @@
  *  - All pointers named W, x, y, ids, status are DEVICE pointers owned by the
  *    caller; libkq never frees or retains them past the call (the chain object
  *    below is the exception and says so).
- *  - W must be 16-byte aligned, and so must every row: always true for Q4_K,
- *    Q5_K and Q8_0; Q2_K requires K % 1024 == 0, Q3_K and Q6_K K % 2048 == 0
- *    (else KQ_ERR_UNSUPPORTED).  x and y must be 4-byte aligned.
+ *  - W must be 16-byte aligned; its rows need not be (a Q6_K row of K = 2560
+ *    is 2100 bytes, of K = 2304 1890): weights are copied in whole 16-byte
+ *    units from the boundary at or below a stage's first byte, so a call
+ *    may read up to 15 bytes past the last row, never past the 16-byte
+ *    granule that holds the matrix's last byte.  Two or more columns of
+ *    Q6_K with K % 2048 != 0 run one single-column launch per column.  x and
+ *    y must be 4-byte aligned.
  *  - Calls are asynchronous on `stream` (0 = the legacy default stream).  The
  *    return value reports argument validation and launch errors only
  *    (KQ_ERR_CUDA carries cudaGetLastError()); kq_last_error() gives text.
@@ -107,7 +111,7 @@ typedef enum {
 typedef enum {
     KQ_OK = 0,
     KQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad format, misalignment */
-    KQ_ERR_UNSUPPORTED = 2,   /* valid but not handled (e.g. Q6_K with K % 2048 != 0) */
+    KQ_ERR_UNSUPPORTED = 2,   /* valid but not handled (e.g. K > 32768, or beyond shared memory) */
     KQ_ERR_NOT_PINNED = 3,    /* host memory that must be page-locked is not */
     KQ_ERR_OOM = 4,           /* a device or pinned allocation failed */
     KQ_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */

@@ -136,7 +136,7 @@ def test_invalid_step_launches_nothing():
     bad_k = kq.make_step(*specs[1][:5], ys[1])
     bad_k.K = 3000                                   # not a multiple of 256
     bad_q6 = kq.make_step(*specs[1][:5], ys[1])
-    bad_q6.K = 1024                                  # Q6_K rows must be 16-byte aligned
+    bad_q6.x = None                                  # NULL activations
     bad_pro = kq.make_step(*specs[0][:5], ys[0], "rmsnorm", specs[0][4], 0.0)  # eps = 0
     for bad in (bad_fmt, bad_k, bad_q6, bad_pro):
         arr = (kq.Step * 3)(good[0], bad, good[1])

@@ -37,11 +37,13 @@ def test_gemv_multi_rejects(args, status):
     assert kq.lib().kq_last_error() != b""
 
 
-def test_unaligned_rows_are_unsupported():
-    # Q6_K and Q3_K need K % 2048, Q2_K K % 1024 for 16-byte aligned rows
-    for fmt, K in ((2, 2304), (5, 1024), (4, 2304)):
-        st = multi(fmt=fmt, K=K, ldx=K)
-        assert st in (UNSUPPORTED, 5), (fmt, K)   # (5: a device query failed first on a host without CUDA)
+def test_rows_off_the_16_byte_grid_pass_validation():
+    # Q6_K, Q3_K and Q2_K rows need not be 16-byte aligned: such shapes are
+    # not rejected as invalid (on a host without CUDA the device query fails)
+    for fmt, K in ((2, 2304), (5, 1024), (4, 2304), (2, 5120)):
+        for k in (1, 8):
+            st = multi(fmt=fmt, K=K, ldx=K, k=k)
+            assert st not in (INVALID, UNSUPPORTED), (fmt, K, k, st)
 
 
 def test_n_zero_is_a_no_op():
