@@ -210,11 +210,11 @@ static MmaLayout mma_layout(int fmt, int nt, int nbs, int S, int ng) {
     const size_t res = fmt == KQ_FMT_Q6_K ? 16 : 64;
     L.sp = srow <= res ? res : round_up(srow - res, 128) + res;
     L.stage = round_up(16 * L.sp, 128);
-    const size_t nc = 4 * static_cast<size_t>(nt);
+    const size_t nc = 8 * static_cast<size_t>(nt);  // columns of nt n-tiles
     L.wp = sizeof(float) * ng * 2 * kConsumerWarps * 16 * nc;
     L.bs = round_up(sizeof(float) * 2 * nc * nbs, 128);
     L.red = S > 1 ? sizeof(float) * 2 * (S - 1) * 16 * nc : 0;
-    L.xb = static_cast<size_t>(nbs) * (fmt == KQ_FMT_Q6_K ? 16 : 17) * 32 * nt * 8;
+    L.xb = static_cast<size_t>(nbs) * (fmt == KQ_FMT_Q6_K ? 16 : 18) * 32 * nt * 8;
     L.fixed = kHeadBytes + L.wp + L.bs + L.red + L.xb;
     return L;
 }
@@ -241,20 +241,15 @@ static cudaError_t active_clusters(int fmt, int nt, int ng, int S, size_t smem, 
                 return cudaSuccess;
             }
     }
-    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 4 : 8) + (nt - 1) * 2 + (ng - 1);
+    // (one n-tile of 8 columns serves every column count)
+    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 2 : 4) + (ng - 1);
     switch (key) {
-        case 8: err = mma_active_clusters<3, 1, 1>(S, smem, pro, out); break;
-        case 9: err = mma_active_clusters<3, 1, 2>(S, smem, pro, out); break;
-        case 10: err = mma_active_clusters<3, 2, 1>(S, smem, pro, out); break;
-        case 11: err = mma_active_clusters<3, 2, 2>(S, smem, pro, out); break;
         case 0: err = mma_active_clusters<1, 1, 1>(S, smem, pro, out); break;
         case 1: err = mma_active_clusters<1, 1, 2>(S, smem, pro, out); break;
-        case 2: err = mma_active_clusters<1, 2, 1>(S, smem, pro, out); break;
-        case 3: err = mma_active_clusters<1, 2, 2>(S, smem, pro, out); break;
-        case 4: err = mma_active_clusters<2, 1, 1>(S, smem, pro, out); break;
-        case 5: err = mma_active_clusters<2, 1, 2>(S, smem, pro, out); break;
-        case 6: err = mma_active_clusters<2, 2, 1>(S, smem, pro, out); break;
-        default: err = mma_active_clusters<2, 2, 2>(S, smem, pro, out); break;
+        case 2: err = mma_active_clusters<2, 1, 1>(S, smem, pro, out); break;
+        case 3: err = mma_active_clusters<2, 1, 2>(S, smem, pro, out); break;
+        case 4: err = mma_active_clusters<3, 1, 1>(S, smem, pro, out); break;
+        default: err = mma_active_clusters<3, 1, 2>(S, smem, pro, out); break;
     }
     if (err != cudaSuccess) return err;
     std::lock_guard<std::mutex> lk(mu);
@@ -289,7 +284,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
         int best = 0, best_use = 0;
         for (int s = 1; s <= 8 && s <= a.nb; ++s) {
             if (a.nb % s != 0) continue;
-            const MmaLayout L8 = mma_layout(fmt, 2, a.nb / s, s, 1);
+            const MmaLayout L8 = mma_layout(fmt, 1, a.nb / s, s, 1);
             if (L8.fixed + 2 * L8.stage > limit) continue;
             int use = di.sm_count;
             if (s > 1) {
@@ -325,7 +320,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     }
     if (L.fixed + 2 * L.stage > limit)
         return fail(KQ_ERR_UNSUPPORTED, "K=%lld with %d columns needs %zu bytes of shared memory (limit %zu)",
-                    (long long)a.K, 4 * nt, L.fixed + 2 * L.stage, limit);
+                    (long long)a.K, 8 * nt, L.fixed + 2 * L.stage, limit);
     size_t ns = (limit - L.fixed) / L.stage;
     if (ns > kMaxStages) ns = kMaxStages;
     const int64_t rps = (a.N + 1) / 2;
@@ -424,21 +419,16 @@ static cudaError_t dispatch_gemv1(const GemvArgs& a, const LaunchPlan& p, int fm
     }
 }
 
-static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt, int nt, cudaStream_t s) {
-    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 4 : 8) + (nt - 1) * 2 + (p.ng - 1);
+static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt, cudaStream_t s) {
+    // one n-tile of 8 columns serves every column count
+    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 2 : 4) + (p.ng - 1);
     switch (key) {
-        case 8: return launch_mma<3, 1, 1>(a, p, s);
-        case 9: return launch_mma<3, 1, 2>(a, p, s);
-        case 10: return launch_mma<3, 2, 1>(a, p, s);
-        case 11: return launch_mma<3, 2, 2>(a, p, s);
         case 0: return launch_mma<1, 1, 1>(a, p, s);
         case 1: return launch_mma<1, 1, 2>(a, p, s);
-        case 2: return launch_mma<1, 2, 1>(a, p, s);
-        case 3: return launch_mma<1, 2, 2>(a, p, s);
-        case 4: return launch_mma<2, 1, 1>(a, p, s);
-        case 5: return launch_mma<2, 1, 2>(a, p, s);
-        case 6: return launch_mma<2, 2, 1>(a, p, s);
-        default: return launch_mma<2, 2, 2>(a, p, s);
+        case 2: return launch_mma<2, 1, 1>(a, p, s);
+        case 3: return launch_mma<2, 1, 2>(a, p, s);
+        case 4: return launch_mma<3, 1, 1>(a, p, s);
+        default: return launch_mma<3, 1, 2>(a, p, s);
     }
 }
 
@@ -452,7 +442,7 @@ static bool use_mma(int fmt, int k, int64_t row_bytes) {
 }
 
 static int plan_for(int fmt, int k, bool mma, GemvArgs& a, LaunchPlan& p) {
-    if (mma) return plan_mma(fmt, k <= 4 ? 1 : 2, a, p);
+    if (mma) return plan_mma(fmt, 1, a, p);
     return plan_gemv(fmt, padded_cols(k), a, p);
 }
 
@@ -475,7 +465,7 @@ static int run(GemvArgs& a, int fmt, int k, bool mma, cudaStream_t stream) {
     LaunchPlan p;
     int st = plan_for(fmt, k, mma, a, p);
     if (st != KQ_OK) return st;
-    if (mma) err = dispatch_mma(a, p, fmt, k <= 4 ? 1 : 2, stream);
+    if (mma) err = dispatch_mma(a, p, fmt, stream);
     else if (k == 1 && a.n_seg == 1 && !a.ids && a.ksplit == 1 && a.x_seg_stride == 0)
         err = dispatch_gemv1(a, p, fmt, stream);
     else err = dispatch(a, p, fmt, padded_cols(k), stream);

@@ -8,7 +8,5 @@ namespace kq {
     template cudaError_t mma_active_clusters<F, T, G>(int, size_t, bool, int*);
 KQ_MMA_INST(3, 1, 1)
 KQ_MMA_INST(3, 1, 2)
-KQ_MMA_INST(3, 2, 1)
-KQ_MMA_INST(3, 2, 2)
 #undef KQ_MMA_INST
 }  // namespace kq

@@ -119,7 +119,7 @@ cudaError_t launch_one(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stre
 // The single-column GEMV of one whole matrix (one segment, K unsplit).
 template <int FMT, bool PRO>
 cudaError_t launch_gemv1(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);
-// Tensor-core kernel for 2..8 columns: NT n-tiles of 8 (4 columns each).
+// Tensor-core kernel for 2..8 columns: NT n-tiles of 8 columns (NT = 1).
 int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p);
 template <int FMT, int NT, int NG>
 cudaError_t launch_mma(const GemvArgs& a, const LaunchPlan& p, cudaStream_t stream);

@@ -12,14 +12,17 @@
 // sub-block scale and a quant, which fp16 represents exactly for Q4_K
 // (|sc*q| <= 63*15 < 2048): one fp16 FMA per two weights turns a nibble
 // placed in the mantissa of 1024 (0x6400 | n) into sc*n with no rounding.
-// The B operand (activations) is each fp32 value split into two fp16 terms
-// hi + lo (22 bits), after a power-of-two scale per column and super-block
-// that keeps the largest |x| of the block in [2^14, 2^15), so neither term
-// overflows and small values keep their absolute precision.  d and the min
-// term are applied per super-block in fp32: y = sum_b 2^-e_b d_b S_b - sum_b
-// 2^(5-e_b) dmin_b M_b, where S_b = sum sc*q*x (16 K-steps) and M_b =
-// sum_j m_j X_j (one more K-step whose A holds the 8 mins and B the
-// sub-block sums of x, scaled by 2^(e_b-5) to stay in fp16 range).
+// The B operand (activations) is each fp32 value rounded to fp16 after a
+// power-of-two scale per column and super-block that keeps the largest |x|
+// of the block in [2^14, 2^15): a relative error of at most 2^-11 per
+// activation, so with exact weights |y - y_exact| <= 2^-11 sum_i |w_i x_i|
+// (half the stated bound), and one n-tile of 8 B columns carries 8
+// activation columns.  d and the min term are applied per super-block in
+// fp32: y = sum_b 2^-e_b d_b S_b - sum_b 2^(5-e_b) dmin_b M_b, where S_b =
+// sum sc*q*x (16 K-steps) and M_b = sum_j m_j X_j (two more K-steps whose A
+// holds the 8 mins and B the sub-block sums of x, scaled by 2^(e_b-5) and
+// split into a high and a low fp16 term, so that the min term, which may
+// nearly cancel the other, keeps 22 bits).
 //
 // Schedule.  The persistent CTA and its TMA ring are those of gemv_kernel;
 // a stage is 16 rows (one m16 tile), copied row by row into smem rows
@@ -38,9 +41,10 @@
 namespace kq {
 
 constexpr int kMmaRowPairs = 8;  // 16 rows per stage
-// K-steps per super-block: 16 of quants, plus one of mins for Q4_K
+// K-steps per super-block: 16 of quants, plus (Q4_K, Q5_K) two of mins
+// whose activation sums are split into a high and a low fp16 term
 template <int FMT>
-__host__ __device__ constexpr int mma_steps() { return FMT == 2 ? 16 : 17; }
+__host__ __device__ constexpr int mma_steps() { return FMT == 2 ? 16 : 18; }
 
 // D += A * B for one m16n8k16 tile (row-major A, column-major B).
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -106,21 +110,19 @@ __device__ __forceinline__ int col_shift(uint32_t amax_bits) {
 }
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((e + 127) << 23); }
 
-// B-fragment entry of K-step s for this column's hi and lo terms: the
-// column occupies B columns 2c' (hi) and 2c'+1 (lo) of n-tile col/4,
-// c' = col%4, i.e. lanes g = 2c' and 2c'+1 (lane = 4g + q).  reg0 holds
-// the K positions 2q, 2q+1 and reg1 2q+8, 2q+9: activations 0, 2 and 1, 3
-// of the group of four that feeds the quant word at those positions.
+// B-fragment entry of K-step s for one column: the column is B column
+// col%8 of n-tile col/8, i.e. lane 4*(col%8) + q.  reg0 holds the K
+// positions 2q, 2q+1 and reg1 2q+8, 2q+9: activations 0, 2 and 1, 3 of the
+// group of four that feeds the quant word at those positions, each rounded
+// to fp16 (relative error at most 2^-11; the block's power-of-two scale
+// keeps them normal fp16 numbers unless far below the block's largest).
 template <int FMT, int NT>
 __device__ __forceinline__ void store_b_entry(uint32_t xb, int bl, int s, int q, int col, float4 v) {
-    const int nt = col >> 2, gh = 2 * (col & 3);
+    const int nt = col >> 3, gc = col & 7;
     const __half h0 = __float2half_rn(v.x), h1 = __float2half_rn(v.y), h2 = __float2half_rn(v.z),
                  h3 = __float2half_rn(v.w);
-    const __half l0 = __float2half_rn(v.x - __half2float(h0)), l1 = __float2half_rn(v.y - __half2float(h1)),
-                 l2 = __float2half_rn(v.z - __half2float(h2)), l3 = __float2half_rn(v.w - __half2float(h3));
     const uint32_t step = xb + 8u * static_cast<uint32_t>(((bl * mma_steps<FMT>() + s) * 32) * NT + nt);
-    st_s64u(step + 8u * NT * (4 * gh + q), pack_h2(h0, h2), pack_h2(h1, h3));
-    st_s64u(step + 8u * NT * (4 * (gh + 1) + q), pack_h2(l0, l2), pack_h2(l1, l3));
+    st_s64u(step + 8u * NT * (4 * gc + q), pack_h2(h0, h2), pack_h2(h1, h3));
 }
 
 // Where 4 consecutive activations w..w+3 (w a multiple of 4) of a block go:
@@ -152,12 +154,17 @@ __device__ __forceinline__ void b_slot(int w, int& s, int& q) {
 }
 
 // Stage the activations of the K range [256*kb0, 256*(kb0+nbl)) as
-// B fragments (see b_slot) plus, for Q4_K, per block the min step: lane (g, q)
-// holds (X_2q, X_2q+1) of its column's hi or lo term and zeros for K
-// positions 8..15, X_j being the sub-block sum of 32 activations.  Each
+// B fragments (see b_slot) plus, for Q4_K and Q5_K, per block the two min
+// steps (16: high terms, 17: low terms): lane (g, q) holds (X_2q, X_2q+1)
+// of column g's term and zeros for K positions 8..15, X_j being the
+// sub-block sum of 32 activations, split hi + lo so that the min term keeps
+// 22 bits (dmin*m*X may nearly cancel d*sc*q*x).  Each
 // (column, block) is scaled by its own power of two 2^sh (largest |x| of
 // the block into [2^14, 2^15)) and its sums by 2^(sh-5); `bscale` gets
-// (2^-sh, 2^(5-sh)) per block and column.  Columns >= ncol_real are zero.
+// (2^-sh, 2^(5-sh)) per block and column.  Only the ncol_real columns are
+// staged: a column's products never mix with another column's, so the
+// entries of the padding columns (whose outputs are not stored) are left as
+// they are.
 // One warp per (column, block) item, two float4 per lane, U items' loads in
 // flight.  PRO: with the prologue a.pro, its second operand
 // (gamma, or u) loaded beside x; for RMSNorm each item's sum of squares of
@@ -167,10 +174,10 @@ __device__ __forceinline__ void b_slot(int w, int& s, int& q) {
 template <int FMT, int NT, bool PRO, int U>
 __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, int nwarps, int lane, int bar,
                          int kb0, int nbl, uint32_t part, bool publish) {
-    constexpr int NC = 4 * NT;
+    constexpr int NC = 8 * NT;
     const float* xg = a.x + static_cast<int64_t>(kb0) * 256;
     const int kr = a.ncol_real;
-    const int items = NC * nbl;
+    const int items = kr * nbl;
     const bool rms = PRO && a.pro == 1;
     for (int base = cw; base < items; base += nwarps * U) {
         float4 v[U][2], w[U][2];
@@ -280,10 +287,10 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                     const float Xs = X[u2][h] * scm;
                     const __half xh = __float2half_rn(Xs);
                     const __half xl = __float2half_rn(Xs - __half2float(xh));
-                    const int nt = col >> 2, gh = 2 * (col & 3), q = j >> 1;
+                    const int nt = col >> 3, gc = col & 7, q = j >> 1;
                     const uint32_t step =
                         xb + 8u * static_cast<uint32_t>(((bl * mma_steps<FMT>() + 16) * 32) * NT + nt);
-                    const uint32_t eh = step + 8u * NT * (4 * gh + q), el = step + 8u * NT * (4 * (gh + 1) + q);
+                    const uint32_t eh = step + 8u * NT * (4 * gc + q), el = eh + 8u * NT * 32;  // steps 16, 17
                     st_s16u(eh + 2 * (j & 1), __half_as_ushort(xh));
                     st_s16u(el + 2 * (j & 1), __half_as_ushort(xl));
                     if ((j & 1) == 0) {
@@ -350,11 +357,11 @@ __device__ __forceinline__ void q4k_step(float (&d)[NT][4], uint32_t xg, uint32_
 // Rows g and g+8 of the stage (smem rows rg, rg8), super-block b, this
 // lane's K positions (q = lane%4); B fragments of the block at `xbl` (this
 // lane's entry of step 0).  Adds d*S and dmin*M into ys / ym for the lane's
-// columns 4*nt + q.
+// columns 8n + 2q and 8n + 2q + 1 (at [2n] and [2n + 1]).
 template <int NT>
 __device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t bsc,
-                                              uint32_t sel, uint32_t msel, int q, float (&ys)[2][NT],
-                                              float (&ym)[2][NT]) {
+                                              uint32_t sel, uint32_t msel, int q, float (&ys)[2][2 * NT],
+                                              float (&ym)[2][2 * NT]) {
     const uint32_t o = static_cast<uint32_t>(b) * kQ4Bytes;
     const uint4 hg = ld_s128(rg + o), hg8 = ld_s128(rg8 + o);
     uint4 w[2][2];  // [row][chunk q / q+4]
@@ -395,11 +402,12 @@ __device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, 
         q4k_step<NT, 0x00F000F0u>(acc, x0, x1, x0 >> 8, x1 >> 8, mhi[0][c], ahi[0][c], mhi[1][c], ahi[1][c], s_hi);
     }
     {
-        const uint32_t s_m = xbl + 8u * NT * 32 * 16;
+        const uint32_t s_m = xbl + 8u * NT * 32 * 16;  // steps 16 (high terms) and 17 (low terms)
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-            const uint2 bm = ld_s64u(s_m + 8 * n);
-            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bm.x, bm.y);
+            const uint2 bh = ld_s64u(s_m + 8 * n), bl = ld_s64u(s_m + 8u * NT * 32 + 8 * n);
+            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bh.x, bh.y);
+            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bl.x, bl.y);
         }
     }
     const float d0 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg.x & 0xFFFFu)));
@@ -408,11 +416,16 @@ __device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, 
     const float m1 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg8.x >> 16)));
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-        const float2 f = ld_s64f(bsc + 8u * (4 * n + q));  // (2^-sh, 2^(5-sh)) of column 4n+q
-        ys[0][n] = fmaf(d0 * f.x, acc[n][0] + acc[n][1], ys[0][n]);
-        ys[1][n] = fmaf(d1 * f.x, acc[n][2] + acc[n][3], ys[1][n]);
-        ym[0][n] = fmaf(m0 * f.y, accm[n][0] + accm[n][1], ym[0][n]);
-        ym[1][n] = fmaf(m1 * f.y, accm[n][2] + accm[n][3], ym[1][n]);
+        // this lane's columns 8n + 2q and 8n + 2q + 1: (2^-sh, 2^(5-sh)) each
+        const float4 f = ld_s128f(bsc + 8u * (8 * n + 2 * q));
+        ys[0][2 * n] = fmaf(d0 * f.x, acc[n][0], ys[0][2 * n]);
+        ys[0][2 * n + 1] = fmaf(d0 * f.z, acc[n][1], ys[0][2 * n + 1]);
+        ys[1][2 * n] = fmaf(d1 * f.x, acc[n][2], ys[1][2 * n]);
+        ys[1][2 * n + 1] = fmaf(d1 * f.z, acc[n][3], ys[1][2 * n + 1]);
+        ym[0][2 * n] = fmaf(m0 * f.y, accm[n][0], ym[0][2 * n]);
+        ym[0][2 * n + 1] = fmaf(m0 * f.w, accm[n][1], ym[0][2 * n + 1]);
+        ym[1][2 * n] = fmaf(m1 * f.y, accm[n][2], ym[1][2 * n]);
+        ym[1][2 * n + 1] = fmaf(m1 * f.w, accm[n][3], ym[1][2 * n + 1]);
     }
 }
 
@@ -469,8 +482,8 @@ __device__ __forceinline__ void q5k_step(float (&d)[NT][4], uint32_t xg, uint32_
 // l = 16(q%2) .. 16(q%2)+15, which serve both of its chunks q/2 and q/2 + 2.
 template <int NT>
 __device__ __forceinline__ void q5k_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t bsc,
-                                              uint32_t sel, uint32_t msel, int q, float (&ys)[2][NT],
-                                              float (&ym)[2][NT]) {
+                                              uint32_t sel, uint32_t msel, int q, float (&ys)[2][2 * NT],
+                                              float (&ym)[2][2 * NT]) {
     const uint32_t o = static_cast<uint32_t>(b) * kQ5Bytes;
     const uint4 hg = ld_s128(rg + o), hg8 = ld_s128(rg8 + o);
     uint4 w[2][2];  // [row][chunk q / q+4 (16-byte segments)]
@@ -523,11 +536,12 @@ __device__ __forceinline__ void q5k_mma_block(uint32_t rg, uint32_t rg8, int b, 
                                   h0, h1, h2, h3);
     }
     {
-        const uint32_t s_m = xbl + 8u * NT * 32 * 16;
+        const uint32_t s_m = xbl + 8u * NT * 32 * 16;  // steps 16 (high terms) and 17 (low terms)
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-            const uint2 bm = ld_s64u(s_m + 8 * n);
-            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bm.x, bm.y);
+            const uint2 bh = ld_s64u(s_m + 8 * n), bl = ld_s64u(s_m + 8u * NT * 32 + 8 * n);
+            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bh.x, bh.y);
+            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bl.x, bl.y);
         }
     }
     const float d0 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg.x & 0xFFFFu)));
@@ -536,11 +550,16 @@ __device__ __forceinline__ void q5k_mma_block(uint32_t rg, uint32_t rg8, int b, 
     const float m1 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg8.x >> 16)));
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-        const float2 f = ld_s64f(bsc + 8u * (4 * n + q));  // (2^-sh, 2^(5-sh)) of column 4n+q
-        ys[0][n] = fmaf(d0 * f.x, acc[n][0] + acc[n][1], ys[0][n]);
-        ys[1][n] = fmaf(d1 * f.x, acc[n][2] + acc[n][3], ys[1][n]);
-        ym[0][n] = fmaf(m0 * f.y, accm[n][0] + accm[n][1], ym[0][n]);
-        ym[1][n] = fmaf(m1 * f.y, accm[n][2] + accm[n][3], ym[1][n]);
+        // this lane's columns 8n + 2q and 8n + 2q + 1: (2^-sh, 2^(5-sh)) each
+        const float4 f = ld_s128f(bsc + 8u * (8 * n + 2 * q));
+        ys[0][2 * n] = fmaf(d0 * f.x, acc[n][0], ys[0][2 * n]);
+        ys[0][2 * n + 1] = fmaf(d0 * f.z, acc[n][1], ys[0][2 * n + 1]);
+        ys[1][2 * n] = fmaf(d1 * f.x, acc[n][2], ys[1][2 * n]);
+        ys[1][2 * n + 1] = fmaf(d1 * f.z, acc[n][3], ys[1][2 * n + 1]);
+        ym[0][2 * n] = fmaf(m0 * f.y, accm[n][0], ym[0][2 * n]);
+        ym[0][2 * n + 1] = fmaf(m0 * f.w, accm[n][1], ym[0][2 * n + 1]);
+        ym[1][2 * n] = fmaf(m1 * f.y, accm[n][2], ym[1][2 * n]);
+        ym[1][2 * n + 1] = fmaf(m1 * f.w, accm[n][3], ym[1][2 * n + 1]);
     }
 }
 
@@ -551,7 +570,7 @@ __device__ __forceinline__ void q5k_mma_block(uint32_t rg, uint32_t rg8, int b, 
 // to fp16, within 2^-11 of that weight).  Adds 2^-sh * d * S into ys.
 template <int NT, bool ODD>
 __device__ __forceinline__ void q6k_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t bsc, int q,
-                                              float (&ys)[2][NT]) {
+                                              float (&ys)[2][2 * NT]) {
     uint32_t A[2][4], B[2][4], H[2][4];
     __half2 S[2][4][2];  // [row][combination][t/2]: scales of quarters (t even, t odd)
     float dsc[2];
@@ -618,9 +637,11 @@ __device__ __forceinline__ void q6k_mma_block(uint32_t rg, uint32_t rg8, int b, 
     }
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-        const float f = ld_s32f(bsc + 8u * (4 * n + q));  // 2^-sh of column 4n+q
-        ys[0][n] = fmaf(dsc[0] * f, acc[n][0] + acc[n][1], ys[0][n]);
-        ys[1][n] = fmaf(dsc[1] * f, acc[n][2] + acc[n][3], ys[1][n]);
+        const float4 f = ld_s128f(bsc + 8u * (8 * n + 2 * q));  // 2^-sh of columns 8n + 2q, 8n + 2q + 1
+        ys[0][2 * n] = fmaf(dsc[0] * f.x, acc[n][0], ys[0][2 * n]);
+        ys[0][2 * n + 1] = fmaf(dsc[0] * f.z, acc[n][1], ys[0][2 * n + 1]);
+        ys[1][2 * n] = fmaf(dsc[1] * f.x, acc[n][2], ys[1][2 * n]);
+        ys[1][2 * n + 1] = fmaf(dsc[1] * f.z, acc[n][3], ys[1][2 * n + 1]);
     }
 }
 
@@ -637,7 +658,7 @@ __device__ __forceinline__ void q6k_mma_block(uint32_t rg, uint32_t rg8, int b, 
 // while another may still address its shared memory) brackets it all.
 template <int FMT, int NT, int NG, bool PRO>
 __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __grid_constant__ GemvArgs a) {
-    constexpr int NC = 4 * NT;
+    constexpr int NC = 8 * NT;
     constexpr int NRED = 16 * NC;  // values of one stage's partial sums
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -746,11 +767,11 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
             if (NG == 2 && (ns & 1) && si >= ns && !mbar_wait_bounded(&empty[slot], it.phase ^ 1u, abort_flag))
                 raise_fault(a, abort_flag, 6);
             if (!mbar_wait_bounded(&full[slot], it.phase, abort_flag)) raise_fault(a, abort_flag, 6);
-            float ys[2][NT], ym[2][NT];
+            float ys[2][2 * NT], ym[2][2 * NT];  // rows g, g+8; columns 8n + 2q + c at [2n + c]
 #pragma unroll
             for (int r = 0; r < 2; ++r)
 #pragma unroll
-                for (int n = 0; n < NT; ++n) ys[r][n] = ym[r][n] = 0.f;
+                for (int n = 0; n < 2 * NT; ++n) ys[r][n] = ym[r][n] = 0.f;
             if (!*abort_flag) {
                 // the K range starts `rem` bytes into each smem row (see produce_stages)
                 const uint32_t rg = sbuf_s + slot * a.stage_bytes + g * a.sp + rem;
@@ -770,7 +791,10 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
             for (int r = 0; r < 2; ++r)
 #pragma unroll
                 for (int n = 0; n < NT; ++n)
-                    st_s32f(wb + 4u * ((cw * 16 + g + 8 * r) * NC + 4 * n + q), ys[r][n] - ym[r][n]);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        st_s32f(wb + 4u * ((cw * 16 + g + 8 * r) * NC + 8 * n + 2 * q + c),
+                                ys[r][2 * n + c] - ym[r][2 * n + c]);
             const bool stop = named_bar_or(1 + g_id, kConsumers, *abort_flag != 0);
             if (lane == 0) mbar_arrive(&empty[slot]);
             if (stop) break;
