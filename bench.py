@@ -602,7 +602,7 @@ def dtype_of(name):
     spec, k = workload_spec(name)
     if k == 1:
         return "f32 acc; activations int14 per group of 32, exact int32 sub-block sums (DP4A)"
-    return "f32 acc; exact fp16 weight operands x two-term fp16 activations (22 bits), tensor cores"
+    return "f32 acc; exact fp16 weight operands x fp16 activations (one term per column and super-block scale), tensor cores"
 
 
 def make_workload(name, torch, kq, kqgen, seed):
