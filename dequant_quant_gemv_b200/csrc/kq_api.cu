@@ -214,7 +214,7 @@ static MmaLayout mma_layout(int fmt, int nt, int nbs, int S, int ng) {
     L.wp = sizeof(float) * ng * 2 * kConsumerWarps * 16 * nc;
     L.bs = round_up(sizeof(float) * 2 * nc * nbs, 128);
     L.red = S > 1 ? sizeof(float) * 2 * (S - 1) * 16 * nc : 0;
-    L.xb = static_cast<size_t>(nbs) * (fmt == KQ_FMT_Q6_K ? 16 : 18) * 32 * nt * 8;
+    L.xb = static_cast<size_t>(nbs) * nt * (16 * 256 + (fmt == KQ_FMT_Q6_K ? 0 : 2 * 128));
     L.fixed = kHeadBytes + L.wp + L.bs + L.red + L.xb;
     return L;
 }

@@ -19,8 +19,8 @@
 // (half the stated bound), and one n-tile of 8 B columns carries 8
 // activation columns.  d and the min term are applied per super-block in
 // fp32: y = sum_b 2^-e_b d_b S_b - sum_b 2^(5-e_b) dmin_b M_b, where S_b =
-// sum sc*q*x (16 K-steps) and M_b = sum_j m_j X_j (two more K-steps whose A
-// holds the 8 mins and B the sub-block sums of x, scaled by 2^(e_b-5) and
+// sum sc*q*x (16 K-steps) and M_b = sum_j m_j X_j (two m16n8k8 steps whose
+// A holds the 8 mins and B the sub-block sums of x, scaled by 2^(e_b-5) and
 // split into a high and a low fp16 term, so that the min term, which may
 // nearly cancel the other, keeps 22 bits).
 //
@@ -41,10 +41,22 @@
 namespace kq {
 
 constexpr int kMmaRowPairs = 8;  // 16 rows per stage
-// K-steps per super-block: 16 of quants, plus (Q4_K, Q5_K) two of mins
-// whose activation sums are split into a high and a low fp16 term
+// B fragments of one super-block: 16 K-steps of quants (m16n8k16: 8 bytes
+// per lane and n-tile), plus for Q4_K and Q5_K two of mins (m16n8k8, the
+// activation sums split into a high and a low fp16 term: 4 bytes per lane
+// and n-tile)
 template <int FMT>
-__host__ __device__ constexpr int mma_steps() { return FMT == 2 ? 16 : 18; }
+__host__ __device__ constexpr int xb_block_bytes(int nt) {
+    return nt * (16 * 256 + (FMT == 2 ? 0 : 2 * 128));
+}
+
+// D += A * B for one m16n8k8 tile (the min steps: A = the 8 mins of rows
+// g and g+8, B = the sub-block sums of x).
+__device__ __forceinline__ void mma1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+    asm("mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(b0));
+}
 
 // D += A * B for one m16n8k16 tile (row-major A, column-major B).
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -121,7 +133,7 @@ __device__ __forceinline__ void store_b_entry(uint32_t xb, int bl, int s, int q,
     const int nt = col >> 3, gc = col & 7;
     const __half h0 = __float2half_rn(v.x), h1 = __float2half_rn(v.y), h2 = __float2half_rn(v.z),
                  h3 = __float2half_rn(v.w);
-    const uint32_t step = xb + 8u * static_cast<uint32_t>(((bl * mma_steps<FMT>() + s) * 32) * NT + nt);
+    const uint32_t step = xb + static_cast<uint32_t>(bl * xb_block_bytes<FMT>(NT)) + 8u * (s * 32 * NT + nt);
     st_s64u(step + 8u * NT * (4 * gc + q), pack_h2(h0, h2), pack_h2(h1, h3));
 }
 
@@ -288,15 +300,12 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                     const __half xh = __float2half_rn(Xs);
                     const __half xl = __float2half_rn(Xs - __half2float(xh));
                     const int nt = col >> 3, gc = col & 7, q = j >> 1;
+                    // the min steps after the block's 16 quant steps: high terms, then low
                     const uint32_t step =
-                        xb + 8u * static_cast<uint32_t>(((bl * mma_steps<FMT>() + 16) * 32) * NT + nt);
-                    const uint32_t eh = step + 8u * NT * (4 * gc + q), el = eh + 8u * NT * 32;  // steps 16, 17
+                        xb + static_cast<uint32_t>(bl * xb_block_bytes<FMT>(NT)) + 16u * 256u * NT + 4u * nt;
+                    const uint32_t eh = step + 4u * NT * (4 * gc + q), el = eh + 128u * NT;
                     st_s16u(eh + 2 * (j & 1), __half_as_ushort(xh));
                     st_s16u(el + 2 * (j & 1), __half_as_ushort(xl));
-                    if ((j & 1) == 0) {
-                        st_s32u(eh + 4, 0u);
-                        st_s32u(el + 4, 0u);
-                    }
                 }
             }
         }
@@ -359,9 +368,9 @@ __device__ __forceinline__ void q4k_step(float (&d)[NT][4], uint32_t xg, uint32_
 // lane's entry of step 0).  Adds d*S and dmin*M into ys / ym for the lane's
 // columns 8n + 2q and 8n + 2q + 1 (at [2n] and [2n + 1]).
 template <int NT>
-__device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t bsc,
-                                              uint32_t sel, uint32_t msel, int q, float (&ys)[2][2 * NT],
-                                              float (&ym)[2][2 * NT]) {
+__device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t xml,
+                                              uint32_t bsc, uint32_t sel, uint32_t msel, int q,
+                                              float (&ys)[2][2 * NT], float (&ym)[2][2 * NT]) {
     const uint32_t o = static_cast<uint32_t>(b) * kQ4Bytes;
     const uint4 hg = ld_s128(rg + o), hg8 = ld_s128(rg8 + o);
     uint4 w[2][2];  // [row][chunk q / q+4]
@@ -402,12 +411,11 @@ __device__ __forceinline__ void q4k_mma_block(uint32_t rg, uint32_t rg8, int b, 
         q4k_step<NT, 0x00F000F0u>(acc, x0, x1, x0 >> 8, x1 >> 8, mhi[0][c], ahi[0][c], mhi[1][c], ahi[1][c], s_hi);
     }
     {
-        const uint32_t s_m = xbl + 8u * NT * 32 * 16;  // steps 16 (high terms) and 17 (low terms)
+        // the min steps (high terms, then low): this lane's entries at xml
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-            const uint2 bh = ld_s64u(s_m + 8 * n), bl = ld_s64u(s_m + 8u * NT * 32 + 8 * n);
-            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bh.x, bh.y);
-            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bl.x, bl.y);
+            mma1688(accm[n], mins[0], mins[1], ld_s32(xml + 4 * n));
+            mma1688(accm[n], mins[0], mins[1], ld_s32(xml + 128u * NT + 4 * n));
         }
     }
     const float d0 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg.x & 0xFFFFu)));
@@ -481,9 +489,9 @@ __device__ __forceinline__ void q5k_step(float (&d)[NT][4], uint32_t xg, uint32_
 // offsets (quants at 48, qh at 16), the lane's 5th bits from qh bytes
 // l = 16(q%2) .. 16(q%2)+15, which serve both of its chunks q/2 and q/2 + 2.
 template <int NT>
-__device__ __forceinline__ void q5k_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t bsc,
-                                              uint32_t sel, uint32_t msel, int q, float (&ys)[2][2 * NT],
-                                              float (&ym)[2][2 * NT]) {
+__device__ __forceinline__ void q5k_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t xml,
+                                              uint32_t bsc, uint32_t sel, uint32_t msel, int q,
+                                              float (&ys)[2][2 * NT], float (&ym)[2][2 * NT]) {
     const uint32_t o = static_cast<uint32_t>(b) * kQ5Bytes;
     const uint4 hg = ld_s128(rg + o), hg8 = ld_s128(rg8 + o);
     uint4 w[2][2];  // [row][chunk q / q+4 (16-byte segments)]
@@ -536,12 +544,11 @@ __device__ __forceinline__ void q5k_mma_block(uint32_t rg, uint32_t rg8, int b, 
                                   h0, h1, h2, h3);
     }
     {
-        const uint32_t s_m = xbl + 8u * NT * 32 * 16;  // steps 16 (high terms) and 17 (low terms)
+        // the min steps (high terms, then low): this lane's entries at xml
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-            const uint2 bh = ld_s64u(s_m + 8 * n), bl = ld_s64u(s_m + 8u * NT * 32 + 8 * n);
-            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bh.x, bh.y);
-            mma16816(accm[n], mins[0], mins[1], 0u, 0u, bl.x, bl.y);
+            mma1688(accm[n], mins[0], mins[1], ld_s32(xml + 4 * n));
+            mma1688(accm[n], mins[0], mins[1], ld_s32(xml + 128u * NT + 4 * n));
         }
     }
     const float d0 = __half2float(__ushort_as_half(static_cast<unsigned short>(hg.x & 0xFFFFu)));
@@ -753,7 +760,8 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
         const uint32_t p0 = 2u * static_cast<uint32_t>(q >> 1), pm = 2u * static_cast<uint32_t>(q & 1);
         const uint32_t sel = 0x4040u | p0 | ((p0 + 1) << 8);
         const uint32_t msel = 0x4040u | pm | ((pm + 1) << 8);
-        const uint32_t xlane = xb_s + 8u * NT * lane;
+        const uint32_t xlane = xb_s + 8u * NT * lane;            // this lane's quant-step entries
+        const uint32_t xmlane = xb_s + 16u * 256u * NT + 4u * NT * lane;  // and min-step entries
         const uint32_t bsc_s = smem_u32(bscale);
 
         StageIter it(rp_begin, rp_end, rps, a.N, kMmaRowPairs, ns);
@@ -777,9 +785,10 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
                 const uint32_t rg = sbuf_s + slot * a.stage_bytes + g * a.sp + rem;
                 const uint32_t rg8 = rg + 8 * a.sp;
                 for (int b = cw; b < nbl; b += kConsumerWarps) {
-                    const uint32_t xbl = xlane + 8u * NT * 32 * mma_steps<FMT>() * b, bsc = bsc_s + 8u * NC * b;
-                    if constexpr (FMT == 1) q4k_mma_block<NT>(rg, rg8, b, xbl, bsc, sel, msel, q, ys, ym);
-                    else if constexpr (FMT == 3) q5k_mma_block<NT>(rg, rg8, b, xbl, bsc, sel, msel, q, ys, ym);
+                    const uint32_t xbo = static_cast<uint32_t>(xb_block_bytes<FMT>(NT) * b);
+                    const uint32_t xbl = xlane + xbo, xml = xmlane + xbo, bsc = bsc_s + 8u * NC * b;
+                    if constexpr (FMT == 1) q4k_mma_block<NT>(rg, rg8, b, xbl, xml, bsc, sel, msel, q, ys, ym);
+                    else if constexpr (FMT == 3) q5k_mma_block<NT>(rg, rg8, b, xbl, xml, bsc, sel, msel, q, ys, ym);
                     else if (((rem >> 1) + b) & 1) q6k_mma_block<NT, true>(rg, rg8, b, xbl, bsc, q, ys);
                     else q6k_mma_block<NT, false>(rg, rg8, b, xbl, bsc, q, ys);
                 }
