@@ -684,18 +684,18 @@ def read_roofline(torch, kq, nbytes=2 << 30, reps=5):
 # were taken on: any change to the code in csrc/ (comments aside) changes the
 # hash and the bench reports traffic as null until the counters are taken
 # again.
-TRAFFIC_SOURCES = "61358c298239c3d9"
+TRAFFIC_SOURCES = "3c44f95227685c6b"
 TRAFFIC = {
-    # gemv_kernel (single column, DP4A): the 8B-shaped chain's matrices
-    ("q4_k", 6144, 4096, 1): 14_238_352 + 16,
-    ("q4_k", 4096, 4096, 1): 9_519_656,
-    ("q4_k", 28672, 4096, 1): 66_142_952 + 4_448,
-    ("q6_k", 4096, 14336, 1): 48_292_560 + 8,
+    # gemv1_kernel (single column, DP4A): the 8B-shaped chain's matrices
+    ("q4_k", 6144, 4096, 1): 14_217_128,
+    ("q4_k", 4096, 4096, 1): 9_498_400,
+    ("q4_k", 28672, 4096, 1): 66_121_720 + 2_168,
+    ("q6_k", 4096, 14336, 1): 48_287_584 + 192,
     # mma_kernel (tensor cores), 8 columns
-    ("q4_k", 6144, 4096, 8): 14_353_920,
-    ("q4_k", 4096, 4096, 8): 9_634_816,
-    ("q4_k", 28672, 4096, 8): 66_258_176,
-    ("q6_k", 4096, 14336, 8): 48_694_528,
+    ("q4_k", 6144, 4096, 8): 14_338_304,
+    ("q4_k", 4096, 4096, 8): 9_618_944,
+    ("q4_k", 28672, 4096, 8): 66_242_304,
+    ("q6_k", 4096, 14336, 8): 48_706_560,
 }
 
 
@@ -894,7 +894,8 @@ def bench_kq(args, rank, world):
         dom = max(per_kind, key=lambda n: per_kind[n]["share"])
         dk = per_kind[dom]
         kname = ("mma_kernel (tensor cores)" if k >= 2 else
-                 "steps_kernel (multi-step launch)" if getattr(wl, "use_steps", False) else "gemv_kernel")
+                 "steps_kernel (multi-step launch)" if getattr(wl, "use_steps", False) else
+                 "gemv_kernel (routed segments)" if isinstance(wl, MoE) else "gemv1_kernel")
         rd = read_roofline(torch, kq)
         rpk = max(rd.values())
         result["roofline"] = {"bound": "hbm", "kernel": f"{kname} {dk['fmt']} {dom} {dk['N']}x{dk['K']}",
