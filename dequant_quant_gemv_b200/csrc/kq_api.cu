@@ -207,7 +207,7 @@ static MmaLayout mma_layout(int fmt, int nt, int nbs, int S, int ng) {
     // the residue mod 128 that spreads the 8 rows of a warp over distinct
     // banks
     const size_t srow = static_cast<size_t>(nbs) * kq_block_bytes(fmt) + 16 + 4;
-    const size_t res = fmt == KQ_FMT_Q6_K ? 16 : 64;
+    const size_t res = fmt == KQ_FMT_Q6_K || fmt == KQ_FMT_Q8_0 ? 16 : 64;
     L.sp = srow <= res ? res : round_up(srow - res, 128) + res;
     L.stage = round_up(16 * L.sp, 128);
     const size_t nc = 8 * static_cast<size_t>(nt);  // columns of nt n-tiles
@@ -242,14 +242,16 @@ static cudaError_t active_clusters(int fmt, int nt, int ng, int S, size_t smem, 
             }
     }
     // (one n-tile of 8 columns serves every column count)
-    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 2 : 4) + (ng - 1);
+    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 2 : fmt == KQ_FMT_Q5_K ? 4 : 6) + (ng - 1);
     switch (key) {
         case 0: err = mma_active_clusters<1, 1, 1>(S, smem, pro, out); break;
         case 1: err = mma_active_clusters<1, 1, 2>(S, smem, pro, out); break;
         case 2: err = mma_active_clusters<2, 1, 1>(S, smem, pro, out); break;
         case 3: err = mma_active_clusters<2, 1, 2>(S, smem, pro, out); break;
         case 4: err = mma_active_clusters<3, 1, 1>(S, smem, pro, out); break;
-        default: err = mma_active_clusters<3, 1, 2>(S, smem, pro, out); break;
+        case 5: err = mma_active_clusters<3, 1, 2>(S, smem, pro, out); break;
+        case 6: err = mma_active_clusters<6, 1, 1>(S, smem, pro, out); break;
+        default: err = mma_active_clusters<6, 1, 2>(S, smem, pro, out); break;
     }
     if (err != cudaSuccess) return err;
     std::lock_guard<std::mutex> lk(mu);
@@ -271,7 +273,7 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     DevInfo di;
     cudaError_t err = dev_info(di);
     if (err != cudaSuccess) return cuda_fail(err, "device query");
-    if (fmt == KQ_FMT_Q2_K || fmt == KQ_FMT_Q3_K || fmt == KQ_FMT_Q8_0)
+    if (fmt == KQ_FMT_Q2_K || fmt == KQ_FMT_Q3_K)
         return fail(KQ_ERR_UNSUPPORTED, "no tensor-core kernel for format %d", fmt);
     if (fmt == KQ_FMT_Q6_K && a.nb % 8 != 0)
         return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
@@ -421,24 +423,26 @@ static cudaError_t dispatch_gemv1(const GemvArgs& a, const LaunchPlan& p, int fm
 
 static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt, cudaStream_t s) {
     // one n-tile of 8 columns serves every column count
-    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 2 : 4) + (p.ng - 1);
+    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 2 : fmt == KQ_FMT_Q5_K ? 4 : 6) + (p.ng - 1);
     switch (key) {
         case 0: return launch_mma<1, 1, 1>(a, p, s);
         case 1: return launch_mma<1, 1, 2>(a, p, s);
         case 2: return launch_mma<2, 1, 1>(a, p, s);
         case 3: return launch_mma<2, 1, 2>(a, p, s);
         case 4: return launch_mma<3, 1, 1>(a, p, s);
-        default: return launch_mma<3, 1, 2>(a, p, s);
+        case 5: return launch_mma<3, 1, 2>(a, p, s);
+        case 6: return launch_mma<6, 1, 1>(a, p, s);
+        default: return launch_mma<6, 1, 2>(a, p, s);
     }
 }
 
 // Calls with 2 or more columns (speculative verify) run on the tensor-core
 // kernel, every column group of the call included, so a column's arithmetic
-// never depends on how the call was grouped.  Q2_K, Q3_K and Q8_0 have no
+// never depends on how the call was grouped.  Q2_K and Q3_K have no
 // tensor-core kernel: their columns run one single-column launch each.
 static bool use_mma(int fmt, int k, int64_t row_bytes) {
     // (its per-row copies need 16-byte rows)
-    return k >= 2 && fmt != KQ_FMT_Q2_K && fmt != KQ_FMT_Q3_K && fmt != KQ_FMT_Q8_0 && row_bytes % 16 == 0;
+    return k >= 2 && fmt != KQ_FMT_Q2_K && fmt != KQ_FMT_Q3_K && row_bytes % 16 == 0;
 }
 
 static int plan_for(int fmt, int k, bool mma, GemvArgs& a, LaunchPlan& p) {

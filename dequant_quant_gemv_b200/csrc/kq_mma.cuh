@@ -41,13 +41,13 @@
 namespace kq {
 
 constexpr int kMmaRowPairs = 8;  // 16 rows per stage
-// B fragments of one super-block: 16 K-steps of quants (m16n8k16: 8 bytes
-// per lane and n-tile), plus for Q4_K and Q5_K two of mins (m16n8k8, the
+// B fragments of one super-block (256 weights): 16 K-steps of quants
+// (m16n8k16: 8 bytes per lane and n-tile), plus for Q4_K and Q5_K two of mins (m16n8k8, the
 // activation sums split into a high and a low fp16 term: 4 bytes per lane
 // and n-tile)
 template <int FMT>
 __host__ __device__ constexpr int xb_block_bytes(int nt) {
-    return nt * (16 * 256 + (FMT == 2 ? 0 : 2 * 128));
+    return nt * (16 * 256 + (FMT == 2 || FMT == 6 ? 0 : 2 * 128));
 }
 
 // D += A * B for one m16n8k8 tile (the min steps: A = the 8 mins of rows
@@ -145,6 +145,10 @@ __device__ __forceinline__ void store_b_entry(uint32_t xb, int bl, int s, int q,
 // chunk beta/16.  Lane q reads chunks q and q+4; word u of chunk q+4c feeds
 // K-step pair j = 4c + u: step 2j (low nibbles) or 2j+1 (high).
 //
+// Q8_0: the unit of 256 weights is 8 blocks of 32 (fp16 d, then 32 int8
+// quants); block j's quant word u (weights 32j + 4u .. +3) feeds K-step
+// 2j + u/4, lane u%4, so that a K-step holds 16 weights of one block.
+//
 // Q6_K: weight w = 128n + 32t + l takes its low bits from ql[64n + l +
 // 32(t%2)] (nibble t/2) and its top bits from bits 2t of qh[32n + l].  Lane
 // q reads the 4-byte groups lg = q and q+4 of each half n, l = 4lg..4lg+3;
@@ -152,7 +156,11 @@ __device__ __forceinline__ void store_b_entry(uint32_t xb, int bl, int s, int q,
 // feed K-step s = 4c + t.
 template <int FMT>
 __device__ __forceinline__ void b_slot(int w, int& s, int& q) {
-    if constexpr (FMT != 2) {  // Q4_K and Q5_K share the quant order
+    if constexpr (FMT == 6) {  // Q8_0: word u = (w%32)/4 of block w/32 feeds step 2*(w/32) + u/4, lane u%4
+        const int u = (w & 31) >> 2;
+        q = u & 3;
+        s = 2 * (w >> 5) + (u >> 2);
+    } else if constexpr (FMT != 2) {  // Q4_K and Q5_K share the quant order
         const int hi = (w >> 5) & 1;
         const int beta = 32 * (w >> 6) + (w & 31);
         const int ch = beta >> 4, u = (beta >> 2) & 3;
@@ -279,7 +287,7 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                     bscale[2 * (bl * NC + col) + 1] = pow2f(5 - sh);
                 }
             }
-            if constexpr (FMT == 2) continue;
+            if constexpr (FMT == 2 || FMT == 6) continue;
             // sub-block 4h + lane/8: the 8 lanes of its group, fixed order
 #pragma unroll
             for (int off = 1; off <= 4; off <<= 1)
@@ -652,6 +660,79 @@ __device__ __forceinline__ void q6k_mma_block(uint32_t rg, uint32_t rg8, int b, 
     }
 }
 
+// Q8_0: rows g and g+8, unit b (8 blocks of 34 bytes), this lane's quant
+// words q and 4 + q of each block.  A = q exactly (byte ^ 0x80 = q + 128
+// in the mantissa of 1024 by byte permute, minus 1152); a block's two
+// K-steps sum into their own accumulator, which is scaled by the block's d
+// in fp32.  Blocks at even j have their quants 2 bytes past a 4-byte
+// boundary (words rebuilt from two loaded words), odd j aligned ones.  Adds
+// 2^-sh * sum_j d_j S_j into ys.
+template <int NT>
+__device__ __forceinline__ void q80_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t bsc, int q,
+                                              float (&ys)[2][2 * NT]) {
+    const uint32_t o = static_cast<uint32_t>(b) * kQ80Bytes;
+    const __half2 m1152 = u2h2(0xE480E480u);  // (-1152, -1152)
+    float yb[2][2 * NT];  // sum over the unit's blocks of d * S, rows g and g+8
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int n = 0; n < 2 * NT; ++n) yb[r][n] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        uint32_t w[2][2];
+        float d[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint32_t base = (r ? rg8 : rg) + o + 34u * j;  // block j: d, then the quants
+            if (j & 1) {  // quants on a 4-byte boundary, d in the upper half of the word below
+                w[r][0] = ld_s32(base + 2 + 4 * q);
+                w[r][1] = ld_s32(base + 18 + 4 * q);
+                d[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(ld_s32(base - 2) >> 16)));
+            } else {
+                w[r][0] = __byte_perm(ld_s32(base + 4 * q), ld_s32(base + 4 + 4 * q), 0x5432u);
+                w[r][1] = __byte_perm(ld_s32(base + 16 + 4 * q), ld_s32(base + 20 + 4 * q), 0x5432u);
+                d[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(ld_s32(base) & 0xFFFFu)));
+            }
+        }
+        float acc[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t lo[2], hi[2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint32_t t = w[r][h] ^ 0x80808080u;
+                lo[r] = h22u(__hadd2(u2h2(__byte_perm(t, 0x64646464u, 0x4240u)), m1152));
+                hi[r] = h22u(__hadd2(u2h2(__byte_perm(t, 0x64646464u, 0x4341u)), m1152));
+            }
+            const uint32_t sp = xbl + 8u * NT * 32 * (2 * j + h);
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const uint2 bv = ld_s64u(sp + 8 * n);
+                mma16816(acc[n], lo[0], lo[1], hi[0], hi[1], bv.x, bv.y);
+            }
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            yb[0][2 * n] = fmaf(d[0], acc[n][0], yb[0][2 * n]);
+            yb[0][2 * n + 1] = fmaf(d[0], acc[n][1], yb[0][2 * n + 1]);
+            yb[1][2 * n] = fmaf(d[1], acc[n][2], yb[1][2 * n]);
+            yb[1][2 * n + 1] = fmaf(d[1], acc[n][3], yb[1][2 * n + 1]);
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const float4 f = ld_s128f(bsc + 8u * (8 * n + 2 * q));  // 2^-sh of columns 8n + 2q, 8n + 2q + 1
+        ys[0][2 * n] = fmaf(f.x, yb[0][2 * n], ys[0][2 * n]);
+        ys[0][2 * n + 1] = fmaf(f.z, yb[0][2 * n + 1], ys[0][2 * n + 1]);
+        ys[1][2 * n] = fmaf(f.x, yb[1][2 * n], ys[1][2 * n]);
+        ys[1][2 * n + 1] = fmaf(f.z, yb[1][2 * n + 1], ys[1][2 * n + 1]);
+    }
+}
+
 // ------------------------------------------------------------ the kernel
 
 // Split K inside a cluster (a.cluster): the ksplit CTAs of a cluster share
@@ -789,6 +870,7 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
                     const uint32_t xbl = xlane + xbo, xml = xmlane + xbo, bsc = bsc_s + 8u * NC * b;
                     if constexpr (FMT == 1) q4k_mma_block<NT>(rg, rg8, b, xbl, xml, bsc, sel, msel, q, ys, ym);
                     else if constexpr (FMT == 3) q5k_mma_block<NT>(rg, rg8, b, xbl, xml, bsc, sel, msel, q, ys, ym);
+                    else if constexpr (FMT == 6) q80_mma_block<NT>(rg, rg8, b, xbl, bsc, q, ys);
                     else if (((rem >> 1) + b) & 1) q6k_mma_block<NT, true>(rg, rg8, b, xbl, bsc, q, ys);
                     else q6k_mma_block<NT, false>(rg, rg8, b, xbl, bsc, q, ys);
                 }

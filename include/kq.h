@@ -68,12 +68,13 @@
  *    integers).  A single column rounds each activation to a 14-bit
  *    integer on a power-of-two grid per group of 32 (error at most 2^-14 of
  *    the group's largest |x|), every format alike; two or
- *    more columns of Q4_K..Q6_K run on the tensor cores with exact fp16
- *    weight operands (Q6_K scales beyond +-64 rounded to fp16) and each
- *    activation rounded to fp16 after a power-of-two scale per column and
- *    super-block (relative error at most 2^-11, so |y - y_exact| <= 2^-11 *
- *    sum_i |w_i x_i| from the activations); several columns of Q2_K, Q3_K
- *    and Q8_0 run one single-column launch per column.  Every output satisfies
+ *    more columns of Q4_K..Q6_K and Q8_0 run on the tensor cores with exact
+ *    fp16 weight operands (sc*q; Q8_0 the int8 q, its d applied per block in
+ *    fp32; Q6_K scales beyond +-64 rounded to fp16) and each activation
+ *    rounded to fp16 after a power-of-two scale per column and super-block
+ *    (relative error at most 2^-11, so |y - y_exact| <= 2^-11 * sum_i |w_i
+ *    x_i| from the activations); several columns of Q2_K and Q3_K run one
+ *    single-column launch per column.  Every output satisfies
  *    |y - y_exact| <= 1e-3 * sum_i |w_i x_i| + 1e-6 for activations of
  *    comparable magnitude within each group of 32.
  *    Results are deterministic: the same inputs give bitwise-equal outputs;
