@@ -114,6 +114,8 @@ WORKLOADS = {
     "llama8b_q80_chain": "Llama-3.1-8B-shaped decode chain with every matrix in Q8_0, 32 layers, batch 1",
     "gateup_q80": "Q8_0 GEMV 28672 x 4096 (8B gate|up), 8 distinct copies rotated",
     "verify8b_q80_k8": "the Q8_0 8B-shaped chain, speculative-verify GEMV with k=8 activation columns",
+    "verify8b_q2k_k8": "the Q2_K 8B-shaped chain (Q3_K down), speculative-verify GEMV with k=8 activation columns",
+    "verify8b_q3k_k8": "the Q3_K 8B-shaped chain (Q4_K down), speculative-verify GEMV with k=8 activation columns",
     "llama8b_chain_steps": "the same chain through kq_gemv_steps (16 matvecs per persistent launch, each "
                            "waiting for the one before)",
     "llama8b_layer_fused": "the 8B-shaped chain with RMSNorm fused into qkv and gate|up and the SiLU-gated "
@@ -562,7 +564,8 @@ class MoEStreamed(MoE):
 
 CHAIN_BASE = {"llama8b_chain": "llama8b", "llama8b_chain_steps": "llama8b", "llama8b_layer_fused": "llama8b",
               "llama8b_layer_fused_steps": "llama8b", "llama8b_q5k_chain": "llama8b_q5k",
-              "verify8b_q5k_k8": "llama8b_q5k", "verify8b_q80_k8": "llama8b_q80", "llama8b_q2k_chain": "llama8b_q2k",
+              "verify8b_q5k_k8": "llama8b_q5k", "verify8b_q80_k8": "llama8b_q80", "verify8b_q2k_k8": "llama8b_q2k", "verify8b_q3k_k8": "llama8b_q3k",
+              "llama8b_q2k_chain": "llama8b_q2k",
               "llama8b_q3k_chain": "llama8b_q3k", "llama8b_q80_chain": "llama8b_q80",
               "llama70b_resident": "llama70b", "llama70b_resident_steps": "llama70b",
               "llama70b_stream": "llama70b", "llama70b_stream_20gb": "llama70b"}
@@ -574,7 +577,7 @@ def workload_spec(name):
         return None, 1
     if name.startswith("verify8b_k"):
         return chain_spec("llama8b"), int(name[len("verify8b_k"):])
-    k = 8 if name in ("verify8b_q5k_k8", "verify8b_q80_k8") else 1
+    k = 8 if name in ("verify8b_q5k_k8", "verify8b_q80_k8", "verify8b_q2k_k8", "verify8b_q3k_k8") else 1
     return chain_spec(CHAIN_BASE.get(name, name)), k
 
 
@@ -615,8 +618,8 @@ def make_workload(name, torch, kq, kqgen, seed):
         return Resident(torch, kq, kqgen, chain_spec("llama8b_q5k"), seed)
     if name == "verify8b_q5k_k8":
         return Resident(torch, kq, kqgen, chain_spec("llama8b_q5k"), seed, k=8)
-    if name == "verify8b_q80_k8":
-        return Resident(torch, kq, kqgen, chain_spec("llama8b_q80"), seed, k=8)
+    if name in ("verify8b_q80_k8", "verify8b_q2k_k8", "verify8b_q3k_k8"):
+        return Resident(torch, kq, kqgen, chain_spec(CHAIN_BASE[name]), seed, k=8)
     if name in ("llama8b_q2k_chain", "llama8b_q3k_chain", "llama8b_q80_chain"):
         return Resident(torch, kq, kqgen, chain_spec(name[:-len("_chain")]), seed)
     if name in ("gemv_q4k_4096", "gateup_q4k", "gateup_q5k", "down_q6k", "gateup_q2k", "gateup_q3k", "down_q3k",

@@ -207,16 +207,30 @@ static MmaLayout mma_layout(int fmt, int nt, int nbs, int S, int ng) {
     // the residue mod 128 that spreads the 8 rows of a warp over distinct
     // banks
     const size_t srow = static_cast<size_t>(nbs) * kq_block_bytes(fmt) + 16 + 4;
-    const size_t res = fmt == KQ_FMT_Q6_K || fmt == KQ_FMT_Q8_0 ? 16 : 64;
+    const size_t res = fmt == KQ_FMT_Q4_K || fmt == KQ_FMT_Q5_K ? 64 : 16;
     L.sp = srow <= res ? res : round_up(srow - res, 128) + res;
     L.stage = round_up(16 * L.sp, 128);
     const size_t nc = 8 * static_cast<size_t>(nt);  // columns of nt n-tiles
     L.wp = sizeof(float) * ng * 2 * kConsumerWarps * 16 * nc;
     L.bs = round_up(sizeof(float) * 2 * nc * nbs, 128);
     L.red = S > 1 ? sizeof(float) * 2 * (S - 1) * 16 * nc : 0;
-    L.xb = static_cast<size_t>(nbs) * nt * (16 * 256 + (fmt == KQ_FMT_Q6_K ? 0 : 2 * 128));
+    const size_t min_steps = fmt == KQ_FMT_Q6_K || fmt == KQ_FMT_Q8_0 ? 0
+                           : fmt == KQ_FMT_Q2_K || fmt == KQ_FMT_Q3_K ? 2 * 256 : 2 * 128;
+    L.xb = static_cast<size_t>(nbs) * nt * (16 * 256 + min_steps);
     L.fixed = kHeadBytes + L.wp + L.bs + L.red + L.xb;
     return L;
+}
+
+// Instantiation key of the tensor-core kernel per format (+ groups - 1).
+static int mma_key(int fmt) {
+    switch (fmt) {
+        case KQ_FMT_Q4_K: return 0;
+        case KQ_FMT_Q6_K: return 2;
+        case KQ_FMT_Q5_K: return 4;
+        case KQ_FMT_Q8_0: return 6;
+        case KQ_FMT_Q2_K: return 8;
+        default: return 10;  // Q3_K
+    }
 }
 
 static cudaError_t active_clusters(int fmt, int nt, int ng, int S, size_t smem, bool pro, int* out) {
@@ -242,7 +256,7 @@ static cudaError_t active_clusters(int fmt, int nt, int ng, int S, size_t smem, 
             }
     }
     // (one n-tile of 8 columns serves every column count)
-    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 2 : fmt == KQ_FMT_Q5_K ? 4 : 6) + (ng - 1);
+    const int key = mma_key(fmt) + (ng - 1);
     switch (key) {
         case 0: err = mma_active_clusters<1, 1, 1>(S, smem, pro, out); break;
         case 1: err = mma_active_clusters<1, 1, 2>(S, smem, pro, out); break;
@@ -251,7 +265,11 @@ static cudaError_t active_clusters(int fmt, int nt, int ng, int S, size_t smem, 
         case 4: err = mma_active_clusters<3, 1, 1>(S, smem, pro, out); break;
         case 5: err = mma_active_clusters<3, 1, 2>(S, smem, pro, out); break;
         case 6: err = mma_active_clusters<6, 1, 1>(S, smem, pro, out); break;
-        default: err = mma_active_clusters<6, 1, 2>(S, smem, pro, out); break;
+        case 7: err = mma_active_clusters<6, 1, 2>(S, smem, pro, out); break;
+        case 8: err = mma_active_clusters<4, 1, 1>(S, smem, pro, out); break;
+        case 9: err = mma_active_clusters<4, 1, 2>(S, smem, pro, out); break;
+        case 10: err = mma_active_clusters<5, 1, 1>(S, smem, pro, out); break;
+        default: err = mma_active_clusters<5, 1, 2>(S, smem, pro, out); break;
     }
     if (err != cudaSuccess) return err;
     std::lock_guard<std::mutex> lk(mu);
@@ -273,8 +291,6 @@ int plan_mma(int fmt, int nt, GemvArgs& a, LaunchPlan& p) {
     DevInfo di;
     cudaError_t err = dev_info(di);
     if (err != cudaSuccess) return cuda_fail(err, "device query");
-    if (fmt == KQ_FMT_Q2_K || fmt == KQ_FMT_Q3_K)
-        return fail(KQ_ERR_UNSUPPORTED, "no tensor-core kernel for format %d", fmt);
     if (fmt == KQ_FMT_Q6_K && a.nb % 8 != 0)
         return fail(KQ_ERR_UNSUPPORTED, "Q6_K rows must be 16-byte aligned (K %% 2048 == 0), K=%lld", (long long)a.K);
     // RMSNorm scratch after the ring: 8 columns' sums per super-block, 8 norms
@@ -423,7 +439,7 @@ static cudaError_t dispatch_gemv1(const GemvArgs& a, const LaunchPlan& p, int fm
 
 static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt, cudaStream_t s) {
     // one n-tile of 8 columns serves every column count
-    const int key = (fmt == KQ_FMT_Q4_K ? 0 : fmt == KQ_FMT_Q6_K ? 2 : fmt == KQ_FMT_Q5_K ? 4 : 6) + (p.ng - 1);
+    const int key = mma_key(fmt) + (p.ng - 1);
     switch (key) {
         case 0: return launch_mma<1, 1, 1>(a, p, s);
         case 1: return launch_mma<1, 1, 2>(a, p, s);
@@ -432,17 +448,21 @@ static cudaError_t dispatch_mma(const GemvArgs& a, const LaunchPlan& p, int fmt,
         case 4: return launch_mma<3, 1, 1>(a, p, s);
         case 5: return launch_mma<3, 1, 2>(a, p, s);
         case 6: return launch_mma<6, 1, 1>(a, p, s);
-        default: return launch_mma<6, 1, 2>(a, p, s);
+        case 7: return launch_mma<6, 1, 2>(a, p, s);
+        case 8: return launch_mma<4, 1, 1>(a, p, s);
+        case 9: return launch_mma<4, 1, 2>(a, p, s);
+        case 10: return launch_mma<5, 1, 1>(a, p, s);
+        default: return launch_mma<5, 1, 2>(a, p, s);
     }
 }
 
 // Calls with 2 or more columns (speculative verify) run on the tensor-core
 // kernel, every column group of the call included, so a column's arithmetic
-// never depends on how the call was grouped.  Q2_K and Q3_K have no
-// tensor-core kernel: their columns run one single-column launch each.
+// never depends on how the call was grouped.  Its per-row copies need
+// 16-byte rows; other shapes run one single-column launch per column.
 static bool use_mma(int fmt, int k, int64_t row_bytes) {
-    // (its per-row copies need 16-byte rows)
-    return k >= 2 && fmt != KQ_FMT_Q2_K && fmt != KQ_FMT_Q3_K && row_bytes % 16 == 0;
+    (void)fmt;
+    return k >= 2 && row_bytes % 16 == 0;
 }
 
 static int plan_for(int fmt, int k, bool mma, GemvArgs& a, LaunchPlan& p) {

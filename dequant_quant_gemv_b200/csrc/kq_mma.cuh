@@ -47,7 +47,7 @@ constexpr int kMmaRowPairs = 8;  // 16 rows per stage
 // and n-tile)
 template <int FMT>
 __host__ __device__ constexpr int xb_block_bytes(int nt) {
-    return nt * (16 * 256 + (FMT == 2 || FMT == 6 ? 0 : 2 * 128));
+    return nt * (16 * 256 + (FMT == 2 || FMT == 6 ? 0 : FMT == 4 || FMT == 5 ? 2 * 256 : 2 * 128));
 }
 
 // D += A * B for one m16n8k8 tile (the min steps: A = the 8 mins of rows
@@ -145,6 +145,12 @@ __device__ __forceinline__ void store_b_entry(uint32_t xb, int bl, int s, int q,
 // chunk beta/16.  Lane q reads chunks q and q+4; word u of chunk q+4c feeds
 // K-step pair j = 4c + u: step 2j (low nibbles) or 2j+1 (high).
 //
+// Q2_K, Q3_K: weight w = 128n + 32j + l has its 2 low bits at bits 2j of
+// quant byte 32n + l, so quant word u (bytes 4u..4u+3) holds weights
+// 128n + 32j + 4(u%8) .. +3 of n = u/8 for every j.  K-step s reads word s;
+// lane q takes the bits of j = q, so that each lane's weights of a step sit
+// in one 16-weight group (8n + 2q + (u%8)/4) and one shift.
+//
 // Q8_0: the unit of 256 weights is 8 blocks of 32 (fp16 d, then 32 int8
 // quants); block j's quant word u (weights 32j + 4u .. +3) feeds K-step
 // 2j + u/4, lane u%4, so that a K-step holds 16 weights of one block.
@@ -156,7 +162,10 @@ __device__ __forceinline__ void store_b_entry(uint32_t xb, int bl, int s, int q,
 // feed K-step s = 4c + t.
 template <int FMT>
 __device__ __forceinline__ void b_slot(int w, int& s, int& q) {
-    if constexpr (FMT == 6) {  // Q8_0: word u = (w%32)/4 of block w/32 feeds step 2*(w/32) + u/4, lane u%4
+    if constexpr (FMT == 4 || FMT == 5) {  // Q2_K, Q3_K: weight 128n + 32j + l: step 8n + l/4, lane j
+        q = (w >> 5) & 3;
+        s = 8 * (w >> 7) + ((w & 31) >> 2);
+    } else if constexpr (FMT == 6) {  // Q8_0: word u = (w%32)/4 of block w/32 feeds step 2*(w/32) + u/4, lane u%4
         const int u = (w & 31) >> 2;
         q = u & 3;
         s = 2 * (w >> 5) + (u >> 2);
@@ -280,7 +289,16 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                     int st, sq;
                     b_slot<FMT>(128 * h + 4 * lane, st, sq);
                     if (valid) store_b_entry<FMT, NT>(xb, bl, st, sq, col, t);
-                    X[u2][h] = (v[c + u2][h].x + v[c + u2][h].y) + (v[c + u2][h].z + v[c + u2][h].w);
+                    if constexpr (FMT == 5) {
+                        // Q3_K's code offset (-4 per weight) is a min step: its
+                        // sums take the same fp16 activations as the quant steps
+                        // (scaled by 2^sh), so that for a code of 4 (weight 0)
+                        // the two terms cancel exactly
+                        auto hr = [](float f) { return __half2float(__float2half_rn(f)); };
+                        X[u2][h] = (hr(t.x) + hr(t.y)) + (hr(t.z) + hr(t.w));
+                    } else {
+                        X[u2][h] = (v[c + u2][h].x + v[c + u2][h].y) + (v[c + u2][h].z + v[c + u2][h].w);
+                    }
                 }
                 if (valid && lane == 0) {
                     bscale[2 * (bl * NC + col)] = pow2f(-sh);
@@ -288,6 +306,39 @@ __device__ void stage_xb(const GemvArgs& a, uint32_t xb, float* bscale, int cw, 
                 }
             }
             if constexpr (FMT == 2 || FMT == 6) continue;
+            if constexpr (FMT == 4 || FMT == 5) {
+                // 16-weight group 8h + lane/4: the 4 lanes of its group, fixed
+                // order; K position g of the two min steps (m16n8k16: lane
+                // (column, (g%8)/2), register g/8, half g%2)
+#pragma unroll
+                for (int off = 1; off <= 2; off <<= 1)
+#pragma unroll
+                    for (int u2 = 0; u2 < 2; ++u2)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) X[u2][h] += __shfl_xor_sync(0xffffffffu, X[u2][h], off);
+#pragma unroll
+                for (int u2 = 0; u2 < 2; ++u2) {
+                    const int it = base + nwarps * (c + u2);
+                    if (it >= items || (lane & 3) != 0) continue;
+                    const int col = it / nbl, bl = it - col * nbl;
+                    // (Q3_K's sums are of the scaled activations already)
+                    const float scm = FMT == 5 ? 0.03125f : pow2f(col_shift(__float_as_uint(m[u2])) - 5);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int g16 = 8 * h + (lane >> 2);
+                        const float Xs = X[u2][h] * scm;
+                        const __half xh = __float2half_rn(Xs);
+                        const __half xl = __float2half_rn(Xs - __half2float(xh));
+                        const int nt = col >> 3, gc = col & 7, q = (g16 & 7) >> 1;
+                        const uint32_t step =
+                            xb + static_cast<uint32_t>(bl * xb_block_bytes<FMT>(NT)) + 16u * 256u * NT + 8u * nt;
+                        const uint32_t eh = step + 8u * NT * (4 * gc + q) + 4u * (g16 >> 3) + 2u * (g16 & 1);
+                        st_s16u(eh, __half_as_ushort(xh));
+                        st_s16u(eh + 256u * NT, __half_as_ushort(xl));
+                    }
+                }
+                continue;
+            }
             // sub-block 4h + lane/8: the 8 lanes of its group, fixed order
 #pragma unroll
             for (int off = 1; off <= 4; off <<= 1)
@@ -660,6 +711,144 @@ __device__ __forceinline__ void q6k_mma_block(uint32_t rg, uint32_t rg8, int b, 
     }
 }
 
+// Q2_K / Q3_K K-step (see b_slot): the 2-bit (Q3_K: with its third bit)
+// code fields of bytes 0, 2 (t, t8) and 1, 3 (ts, ts8: the words shifted
+// right by 8) of rows g and g+8, already masked into the mantissa of 1024
+// (1024 + v*4^q), times (sc/4^q) minus 1024*sc/4^q: sc*v exactly, one fp16
+// FMA per two weights.
+template <int NT>
+__device__ __forceinline__ void q23_step(float (&d)[NT][4], uint32_t t, uint32_t t8, uint32_t ts, uint32_t ts8,
+                                         uint32_t m, uint32_t a, uint32_t m8, uint32_t a8, uint32_t baddr) {
+    const uint32_t a0 = hfma2u(t, m, a), a1 = hfma2u(t8, m8, a8);
+    const uint32_t a2 = hfma2u(ts, m, a), a3 = hfma2u(ts8, m8, a8);
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const uint2 bv = ld_s64u(baddr + 8 * n);
+        mma16816(d[n], a0, a1, a2, a3, bv.x, bv.y);
+    }
+}
+
+// (v0, v1) - off, exactly: bytes p0, p0 + 1 of `w` (each < 64 + off) as the
+// fp16 pair 1024 + v by byte permute, minus 1024 + off.
+__device__ __forceinline__ __half2 byte_pair_minus(uint32_t w, uint32_t sel, uint32_t off_h2) {
+    return __hsub2(u2h2(__byte_perm(w, 0x64646464u, sel)), u2h2(off_h2));
+}
+
+// Q2_K (Q3 = false; 84-byte blocks: 16 scale bytes sc | m << 4, 64 quant
+// bytes, d, dmin) and Q3_K (Q3 = true; 110-byte blocks: 32 high-bit bytes,
+// 64 quant bytes, 12 bytes of 6-bit scales v, d; a Q3_K block at an odd
+// index is 2 bytes off the 4-byte grid (ODD), its words rebuilt by a byte
+// permute): rows g and g+8, super-block b, this lane's shift j = q (see
+// b_slot).  A = sc*v exactly (Q2_K: sc 0..15, v 0..3; Q3_K: sc = v_g - 32,
+// v = the 3-bit code 0..7); the code's offset (Q3_K: -4) and the mins
+// (Q2_K) form the min steps: A = the 16 groups' m (Q2_K) or 4*(v_g - 32)
+// (Q3_K), B = the groups' activation sums.  Adds d*S and dmin*M (Q3_K: d*M)
+// into ys / ym as the Q4_K block does.
+template <int NT, bool Q3, bool ODD>
+__device__ __forceinline__ void q23_mma_block(uint32_t rg, uint32_t rg8, int b, uint32_t xbl, uint32_t bsc, int q,
+                                              float (&ys)[2][2 * NT], float (&ym)[2][2 * NT]) {
+    constexpr uint32_t BS = Q3 ? kQ3Bytes : kQ2Bytes;
+    constexpr int QW = Q3 ? 8 : 4;  // first quant word of the block
+    const uint32_t mq = 0x00030003u << (2 * q);  // bits 2q, 2q+1 of bytes 0 and 2
+    const uint32_t hq = 0x00040004u << (2 * q);  // bit 2q + 2 of either half (Q3_K's third bit)
+    const uint32_t sel = 0x4040u | (2u * (q & 1)) | ((2u * (q & 1) + 1u) << 8);  // bytes 2(q%2), +1
+    const __half2 pw = u2h2(q == 0 ? 0x3C003C00u : q == 1 ? 0x34003400u : q == 2 ? 0x2C002C00u : 0x24002400u);
+    uint32_t bw[2];
+    uint32_t mh[2][2][2], ah[2][2][2], mins[2][2];  // [row][n][h]; mins [row][n]: K positions 2q(+1) (+8)
+    float dd[2], dm[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        bw[r] = (r ? rg8 : rg) + static_cast<uint32_t>(b) * BS - (ODD ? 2u : 0u);
+        auto ldw = [&](int i) -> uint32_t {
+            if constexpr (ODD) return __byte_perm(ld_s32(bw[r] + 4 * i), ld_s32(bw[r] + 4 * i + 4), 0x5432u);
+            else return ld_s32(bw[r] + 4 * i);
+        };
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+            __half2 sv;  // (sc of group 8n + 2q, of 8n + 2q + 1)
+            if constexpr (!Q3) {
+                const uint32_t w = ldw(2 * n + (q >> 1));  // scale bytes 8n + 4(q/2) .. +3
+                sv = byte_pair_minus(w & 0x0F0F0F0Fu, sel, 0x64006400u);
+                mins[r][n] = h22u(byte_pair_minus((w >> 4) & 0x0F0F0F0Fu, sel, 0x64006400u));
+            } else {
+                // v_g: low 4 bits from byte g (g < 8) or the high nibble of
+                // byte g - 8, top 2 bits from bits 2(g/4) of byte 8 + g%4
+                const uint32_t lo = ldw(24 + (q >> 1)), hi = ldw(26);
+                const uint32_t lo4 = (n ? lo >> 4 : lo) & 0x0F0F0F0Fu;
+                const uint32_t hi2 = (hi >> (2 * (2 * n + (q >> 1)))) & 0x03030303u;
+                sv = byte_pair_minus(lo4 | (hi2 << 4), sel, 0x64206420u);  // v - 32
+                mins[r][n] = h22u(__hmul2(sv, u2h2(0x44004400u)));          // 4*(v - 32)
+            }
+            const __half2 svq = __hmul2(sv, pw);  // sc / 4^q
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const __half2 m = h ? __high2half2(svq) : __low2half2(svq);
+                mh[r][n][h] = h22u(m);
+                ah[r][n][h] = h22u(__hmul2(m, u2h2(kH2_m1024)));
+            }
+        }
+        const uint32_t dw = Q3 ? ldw(27) : ldw(20);
+        dd[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(dw & 0xFFFFu)));
+        dm[r] = Q3 ? dd[r] : __half2float(__ushort_as_half(static_cast<unsigned short>(dw >> 16)));
+    }
+    float acc[NT][4], accm[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = accm[n][i] = 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const int n = u >> 3, h = (u >> 2) & 1;
+        uint32_t t[2], ts[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint32_t bwr = bw[r];
+            auto ldw = [&](int i) -> uint32_t {
+                if constexpr (ODD) return __byte_perm(ld_s32(bwr + 4 * i), ld_s32(bwr + 4 * i + 4), 0x5432u);
+                else return ld_s32(bwr + 4 * i);
+            };
+            const uint32_t x = ldw(QW + u);
+            t[r] = (x & mq) | 0x64006400u;
+            ts[r] = ((x >> 8) & mq) | 0x64006400u;
+            if constexpr (Q3) {
+                // bit 4n + q of each high-bit byte (weights l..l+3) to bit
+                // 2q + 2 of its half (bytes 1 and 3 first moved down by 8, so
+                // that no bit leaves the word)
+                const uint32_t hw = ldw(u & 7);
+                auto place = [&](uint32_t v) -> uint32_t {
+                    return n == 0 ? v << (q + 2) : q >= 2 ? v << (q - 2) : v >> (2 - q);
+                };
+                t[r] |= place(hw) & hq;
+                ts[r] |= place(hw >> 8) & hq;
+            }
+        }
+        q23_step<NT>(acc, t[0], t[1], ts[0], ts[1], mh[0][n][h], ah[0][n][h], mh[1][n][h], ah[1][n][h],
+                     xbl + 8u * NT * 32 * u);
+    }
+    {
+        // the min steps (high terms, then low): K = the 16 groups
+        const uint32_t s_m = xbl + 8u * NT * 32 * 16;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const uint2 bh = ld_s64u(s_m + 8 * n), bl = ld_s64u(s_m + 8u * NT * 32 + 8 * n);
+            mma16816(accm[n], mins[0][0], mins[1][0], mins[0][1], mins[1][1], bh.x, bh.y);
+            mma16816(accm[n], mins[0][0], mins[1][0], mins[0][1], mins[1][1], bl.x, bl.y);
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const float4 f = ld_s128f(bsc + 8u * (8 * n + 2 * q));  // (2^-sh, 2^(5-sh)) of columns 8n + 2q, +1
+        ys[0][2 * n] = fmaf(dd[0] * f.x, acc[n][0], ys[0][2 * n]);
+        ys[0][2 * n + 1] = fmaf(dd[0] * f.z, acc[n][1], ys[0][2 * n + 1]);
+        ys[1][2 * n] = fmaf(dd[1] * f.x, acc[n][2], ys[1][2 * n]);
+        ys[1][2 * n + 1] = fmaf(dd[1] * f.z, acc[n][3], ys[1][2 * n + 1]);
+        ym[0][2 * n] = fmaf(dm[0] * f.y, accm[n][0], ym[0][2 * n]);
+        ym[0][2 * n + 1] = fmaf(dm[0] * f.w, accm[n][1], ym[0][2 * n + 1]);
+        ym[1][2 * n] = fmaf(dm[1] * f.y, accm[n][2], ym[1][2 * n]);
+        ym[1][2 * n + 1] = fmaf(dm[1] * f.w, accm[n][3], ym[1][2 * n + 1]);
+    }
+}
+
 // Q8_0: rows g and g+8, unit b (8 blocks of 34 bytes), this lane's quant
 // words q and 4 + q of each block.  A = q exactly (byte ^ 0x80 = q + 128
 // in the mantissa of 1024 by byte permute, minus 1152); a block's two
@@ -871,6 +1060,11 @@ __global__ void __launch_bounds__(32 + NG * kConsumers, 1) mma_kernel(const __gr
                     if constexpr (FMT == 1) q4k_mma_block<NT>(rg, rg8, b, xbl, xml, bsc, sel, msel, q, ys, ym);
                     else if constexpr (FMT == 3) q5k_mma_block<NT>(rg, rg8, b, xbl, xml, bsc, sel, msel, q, ys, ym);
                     else if constexpr (FMT == 6) q80_mma_block<NT>(rg, rg8, b, xbl, bsc, q, ys);
+                    else if constexpr (FMT == 4) q23_mma_block<NT, false, false>(rg, rg8, b, xbl, bsc, q, ys, ym);
+                    else if constexpr (FMT == 5) {
+                        if (((rem >> 1) + b) & 1) q23_mma_block<NT, true, true>(rg, rg8, b, xbl, bsc, q, ys, ym);
+                        else q23_mma_block<NT, true, false>(rg, rg8, b, xbl, bsc, q, ys, ym);
+                    }
                     else if (((rem >> 1) + b) & 1) q6k_mma_block<NT, true>(rg, rg8, b, xbl, bsc, q, ys);
                     else q6k_mma_block<NT, false>(rg, rg8, b, xbl, bsc, q, ys);
                 }

@@ -59,7 +59,8 @@
  *    units from the boundary at or below a stage's first byte, so a call
  *    may read up to 15 bytes past the last row, never past the 16-byte
  *    granule that holds the matrix's last byte.  Two or more columns of
- *    Q6_K with K % 2048 != 0 run one single-column launch per column.  x and
+ *    Q6_K with K % 2048 != 0 (any format whose rows are not a multiple of 16
+ *    bytes) run one single-column launch per column.  x and
  *    y must be 4-byte aligned.
  *  - Calls are asynchronous on `stream` (0 = the legacy default stream).  The
  *    return value reports argument validation and launch errors only
@@ -68,13 +69,14 @@
  *    integers).  A single column rounds each activation to a 14-bit
  *    integer on a power-of-two grid per group of 32 (error at most 2^-14 of
  *    the group's largest |x|), every format alike; two or
- *    more columns of Q4_K..Q6_K and Q8_0 run on the tensor cores with exact
- *    fp16 weight operands (sc*q; Q8_0 the int8 q, its d applied per block in
- *    fp32; Q6_K scales beyond +-64 rounded to fp16) and each activation
- *    rounded to fp16 after a power-of-two scale per column and super-block
- *    (relative error at most 2^-11, so |y - y_exact| <= 2^-11 * sum_i |w_i
- *    x_i| from the activations); several columns of Q2_K and Q3_K run one
- *    single-column launch per column.  Every output satisfies
+ *    more columns run on the tensor cores with exact fp16 weight operands
+ *    (sc*q; Q8_0 the int8 q, its d applied per block in fp32; Q3_K the code
+ *    0..7, its -4 offset a separate term over the same rounded activations;
+ *    Q6_K scales beyond +-64 rounded to fp16) and each activation rounded to
+ *    fp16 after a power-of-two scale per column and super-block (relative
+ *    error at most 2^-11, so |y - y_exact| <= 2^-11 * sum_i |w_i x_i| from
+ *    the activations); shapes whose rows are not a multiple of 16 bytes run
+ *    one single-column launch per column.  Every output satisfies
  *    |y - y_exact| <= 1e-3 * sum_i |w_i x_i| + 1e-6 for activations of
  *    comparable magnitude within each group of 32.
  *    Results are deterministic: the same inputs give bitwise-equal outputs;
