@@ -332,6 +332,20 @@ class Resident:
     def io(self):
         return [self.X], [self.Y]
 
+    def layer_io(self):
+        """Per layer: (x offset, x length, y offset, y length) in elements
+        of X and Y (each layer's slots are contiguous, in layer order)."""
+        out = []
+        for li, mats in enumerate(self.spec):
+            xs = [self.xslot[(li, slot)] for (_, _, _, _, slot) in mats if slot is not None]
+            ys = [self.yslot[(li, mi)] for mi in range(len(mats))]
+            x0 = min(o for o, _ in xs)
+            x1 = max(o + self.k * K for o, K in xs)
+            y0 = min(o for o, _ in ys)
+            y1 = max(o + self.k * N for o, N in ys)
+            out.append((x0, x1 - x0, y0, y1 - y0))
+        return out
+
 
 class FusedLayer(Resident):
     """The 8B chain with the decode layer's glue inside the GEMVs: qkv and
@@ -861,6 +875,42 @@ def bench_kq(args, rank, world):
         run_step()
         for h, d in zip(yh, yout):
             h.copy_(d, non_blocking=True)
+
+    if type(wl) is Resident and not wl.use_steps:
+        # the decode chain: layer l's activations come in on a copy stream
+        # while earlier layers compute, and its outputs go back on another
+        # as soon as its launches are done (one graph per step)
+        cs_in, cs_out = torch.cuda.Stream(), torch.cuda.Stream()
+        X, Y, XH, YH = xin[0], yout[0], xh[0], yh[0]
+        lio = wl.layer_io()
+        g_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_e2e, stream=stream):
+            fork = torch.cuda.Event()
+            fork.record(stream)
+            cs_in.wait_event(fork)
+            cs_out.wait_event(fork)
+            ev_in = []
+            for (x0, xn, _, _) in lio:
+                with torch.cuda.stream(cs_in):
+                    X[x0:x0 + xn].copy_(XH[x0:x0 + xn], non_blocking=True)
+                    e = torch.cuda.Event()
+                    e.record(cs_in)
+                ev_in.append(e)
+            for li, (_, _, y0, yn) in enumerate(lio):
+                stream.wait_event(ev_in[li])
+                for mi in range(len(wl.spec[li])):
+                    wl.launch(li, mi, stream)
+                done = torch.cuda.Event()
+                done.record(stream)
+                cs_out.wait_event(done)
+                with torch.cuda.stream(cs_out):
+                    YH[y0:y0 + yn].copy_(Y[y0:y0 + yn], non_blocking=True)
+            join = torch.cuda.Event()
+            join.record(cs_out)
+            stream.wait_event(join)
+
+        def e2e_step():  # noqa: F811 (the pipelined form for the chain)
+            g_e2e.replay()
 
     for _ in range(max(1, args.warmup)):
         e2e_step()
