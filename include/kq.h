@@ -189,9 +189,12 @@ KQ_API int kq_gemv(const void* W, int fmt, int64_t N, int64_t K, const float* x,
  *   y + c*ldy (N floats each, ldy >= N); 1 <= k <= 8.
  * The verify pass of speculative decoding ("Out-of-core LLM inference engine
  * ...", Approach: several positions verified with one pass of the large
- * model).  With k >= 2 the products run on the tensor cores; column c then
- * equals column c of any other k >= 2 call on the same activations bitwise,
- * and kq_gemv within the tolerance.  k = 1 equals kq_gemv bitwise.
+ * model).  With k >= 2 the products run on the tensor cores (every format,
+ * rows a multiple of 16 bytes); column c then equals column c of any other
+ * k >= 2 call on the same activations bitwise, and kq_gemv within the
+ * tolerance.  Rows off the 16-byte grid run one single-column launch per
+ * column (each column equal to kq_gemv bitwise).  k = 1 equals kq_gemv
+ * bitwise.
  */
 KQ_API int kq_gemv_multi(const void* W, int fmt, int64_t N, int64_t K, const float* x, int64_t ldx,
                   int k, float* y, int64_t ldy, kq_stream_t stream);
