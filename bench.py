@@ -704,18 +704,18 @@ def read_roofline(torch, kq, nbytes=2 << 30, reps=5):
 # were taken on: any change to the code in csrc/ (comments aside) changes the
 # hash and the bench reports traffic as null until the counters are taken
 # again.
-TRAFFIC_SOURCES = "3f96087547b6bca5"
+TRAFFIC_SOURCES = "6ad46e0790ec7bdf"
 TRAFFIC = {
     # gemv1_kernel (single column, DP4A): the 8B-shaped chain's matrices
-    ("q4_k", 6144, 4096, 1): 14_216_952,
-    ("q4_k", 4096, 4096, 1): 9_498_248,
-    ("q4_k", 28672, 4096, 1): 66_121_704 + 3_104,
-    ("q6_k", 4096, 14336, 1): 48_287_040 + 320,
+    ("q4_k", 6144, 4096, 1): 14_215_256,
+    ("q4_k", 4096, 4096, 1): 9_496_864,
+    ("q4_k", 28672, 4096, 1): 66_120_832 + 2_576,
+    ("q6_k", 4096, 14336, 1): 48_287_912 + 264,
     # mma_kernel (tensor cores), 8 columns
-    ("q4_k", 6144, 4096, 8): 14_338_304,
-    ("q4_k", 4096, 4096, 8): 9_618_688,
-    ("q4_k", 28672, 4096, 8): 66_242_304,
-    ("q6_k", 4096, 14336, 8): 48_682_752,
+    ("q4_k", 6144, 4096, 8): 14_338_048,
+    ("q4_k", 4096, 4096, 8): 9_619_200,
+    ("q4_k", 28672, 4096, 8): 66_242_048,
+    ("q6_k", 4096, 14336, 8): 48_682_496,
 }
 
 
@@ -877,34 +877,64 @@ def bench_kq(args, rank, world):
             h.copy_(d, non_blocking=True)
 
     if type(wl) is Resident and not wl.use_steps:
-        # the decode chain: layer l's activations come in on a copy stream
-        # while earlier layers compute, and its outputs go back on another
-        # as soon as its launches are done (one graph per step)
+        # the decode chain: the activations come in on a copy stream while
+        # earlier layers compute, and the outputs go back on another once
+        # their launches are done (one graph per step).  A launch that waits
+        # for a copy loses its programmatic overlap with the launch before
+        # it (1.5-4 us measured per wait), so the copies go in a few
+        # chunks that grow fourfold: inputs of layer 0, of the next 3, the
+        # next 12, then the rest (each chunk copied while the layers before
+        # it compute, a layer's compute taking ~15x its copy); outputs in
+        # the mirrored chunks, the last layer's alone (the one copy left
+        # exposed after the last launch).
         cs_in, cs_out = torch.cuda.Stream(), torch.cuda.Stream()
         X, Y, XH, YH = xin[0], yout[0], xh[0], yh[0]
         lio = wl.layer_io()
+        nl = len(lio)
+
+        sizes, left = [], nl
+        for n in (1, 3, 12):
+            if left > n:
+                sizes.append(n)
+                left -= n
+        sizes.append(left)
+
+        def spans(sz):
+            out, i = [], 0
+            for n in sz:
+                out.append((i, i + n - 1))
+                i += n
+            return out
+
+        in_chunks = spans(sizes)
+        out_chunks = spans(sizes[::-1])
         g_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_e2e, stream=stream):
             fork = torch.cuda.Event()
             fork.record(stream)
             cs_in.wait_event(fork)
             cs_out.wait_event(fork)
-            ev_in = []
-            for (x0, xn, _, _) in lio:
+            ev_in = {}
+            for (a, b) in in_chunks:
+                x0, x1 = lio[a][0], lio[b][0] + lio[b][1]
                 with torch.cuda.stream(cs_in):
-                    X[x0:x0 + xn].copy_(XH[x0:x0 + xn], non_blocking=True)
+                    X[x0:x1].copy_(XH[x0:x1], non_blocking=True)
                     e = torch.cuda.Event()
                     e.record(cs_in)
-                ev_in.append(e)
-            for li, (_, _, y0, yn) in enumerate(lio):
-                stream.wait_event(ev_in[li])
+                ev_in[a] = e
+            out_last = {b: a for (a, b) in out_chunks}
+            for li in range(nl):
+                if li in ev_in:
+                    stream.wait_event(ev_in[li])
                 for mi in range(len(wl.spec[li])):
                     wl.launch(li, mi, stream)
-                done = torch.cuda.Event()
-                done.record(stream)
-                cs_out.wait_event(done)
-                with torch.cuda.stream(cs_out):
-                    YH[y0:y0 + yn].copy_(Y[y0:y0 + yn], non_blocking=True)
+                if li in out_last:
+                    y0, y1 = lio[out_last[li]][2], lio[li][2] + lio[li][3]
+                    done = torch.cuda.Event()
+                    done.record(stream)
+                    cs_out.wait_event(done)
+                    with torch.cuda.stream(cs_out):
+                        YH[y0:y1].copy_(Y[y0:y1], non_blocking=True)
             join = torch.cuda.Event()
             join.record(cs_out)
             stream.wait_event(join)

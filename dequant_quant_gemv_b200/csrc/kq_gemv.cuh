@@ -684,20 +684,49 @@ __device__ __forceinline__ uint32_t x_region(uint32_t xs, int b, int H) {
     return xs + kXRegionBytes * (2 * b + H);
 }
 
-// Position of the region of block b, half H: 2b + H, or with the
-// block-parity lane order over `par` blocks (single-column Q6_K) the even
-// blocks' regions first and then the odd blocks', so that consecutive lanes
-// of a warp (which take consecutive blocks of one parity) still read
-// consecutive regions.
+// Block-parity lane order over `par` blocks (single-column Q6_K, par even):
+// each parity's par/2 blocks (block pair index i, block 2i + p) take
+// round_up(par, 32) lanes of their own, so that a warp never mixes the two
+// alignment classes.  Within a parity the lanes come in pairs of warps over
+// 32 consecutive i: lane l of the first warp takes block i = 32c + l, half
+// l % 2, and lane l of the second the other half of the same block.  A
+// lane's words of one kind lie at bank 9i + 8H + const (qh; ql 16H, scales
+// 2H): blocks of one parity are 420 bytes = 105 words apart.  Two lanes of
+// one warp with the same half are an even number 0 < |i - j| < 32 of block
+// pairs apart, with different halves an odd number, so their banks differ
+// by 9(i - j) or by an odd number plus an even offset: never 0 mod 32, and
+// every ql, qh and scale load of a warp hits 32 distinct banks (the old
+// order, two lanes per block, put lanes i and i + 8 of different halves on
+// one qh bank).  A last warp without a partner
+// (round_up(par, 32) / 32 odd) keeps two lanes per block, (i, half) = (l/2,
+// l%2), as a lone warp of 16 blocks cannot avoid the 8-word overlap.
+//
+// Position of the region of block b, half H: 2b + H, or in the
+// block-parity order the lane's index among the parity's active lanes after
+// the previous parity's par regions (consecutive lanes read consecutive
+// regions, the first warp of a pair its nc blocks' regions and then the
+// second warp its nc).
 __device__ __forceinline__ int x_pos(int b, int H, int par) {
-    return par ? (b & 1) * par + 2 * (b >> 1) + H : 2 * b + H;
+    if (!par) return 2 * b + H;
+    const int p = b & 1, i = b >> 1, c = i >> 5, l = i & 31;
+    const int m = (par + 31) >> 5;  // warps per parity
+    int d;
+    if (2 * c + 1 < m) {
+        const int rest = (par >> 1) - 32 * c;  // blocks of this parity from 32c
+        const int nc = rest < 32 ? rest : 32;
+        d = 64 * c + (((H ^ l) & 1) ? nc : 0) + l;
+    } else {
+        d = 64 * c + 2 * l + H;
+    }
+    return p * par + d;
 }
 
 // The unit of consumer thread ct in the single-column lane layout: LR lanes
 // per row pair; lane u of a row pair takes block u/2, half u%2, or with the
-// block-parity order (par > 0) the first half of the row pair's lanes take
-// its even blocks and the second half the odd ones (a warp never mixes the
-// two alignment classes).  pos: the unit's activation region (x_pos).
+// block-parity order (par > 0; LR = 2 round_up(par, 32)) one half of the
+// row pair's lanes take its even blocks and the other half the odd ones
+// (which half, alternating per 128 lanes of the group), in the warp-pair
+// order above.  pos: the unit's activation region (x_pos).
 struct LaneUnit {
     int rp, b, H, pos;
     bool active;
@@ -708,12 +737,25 @@ __device__ __forceinline__ LaneUnit lane_unit(int ct, int LR, int nbl, int par) 
     const int u = ct - L.rp * LR;
     if (par) {
         const int LRp = LR >> 1;
-        const int p = u >= LRp ? 1 : 0;
-        const int up = u - p * LRp;
-        L.b = 2 * (up >> 1) + p;
-        L.H = up & 1;
+        const int hi = u >= LRp ? 1 : 0;
+        const int up = u - hi * LRp;
+        // the parity of the lanes' blocks, swapped for every other 128
+        // lanes of the group: the warps of a row pair alternate between the
+        // 4 schedulers (warp w on w % 4), and odd blocks cost more (their
+        // words are realigned), so each scheduler gets both kinds
+        const int p = hi ^ (((L.rp * LR) >> 7) & 1);
+        const int w = up >> 5, l = up & 31, c = w >> 1;
+        int i;
+        if ((w | 1) < (LRp >> 5)) {  // a warp of a pair
+            i = 32 * c + l;
+            L.H = (l ^ w) & 1;
+        } else {
+            i = 32 * c + (l >> 1);
+            L.H = l & 1;
+        }
+        L.b = 2 * i + p;
         L.active = L.b < nbl;
-        L.pos = p * par + up;
+        L.pos = x_pos(L.b, L.H, par);
     } else {
         L.b = u >> 1;
         L.H = u & 1;
@@ -747,6 +789,13 @@ __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, 
     float sq = 0.f;
     for (int base = warp; base < quads; base += nwarps * U) {
         float4 v[U], w[U];
+        // the region positions of this round's U passes in the block-parity
+        // order, one pass per lane (lane u: pass u), then broadcast per pass
+        int pos_l = 0;
+        if (par) {
+            const int Ql = base + nwarps * (lane & (U - 1));
+            pos_l = x_pos(Ql >> 1, Ql & 1, par);
+        }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int Q = base + nwarps * u;
@@ -819,7 +868,8 @@ __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, 
             for (int u = 0; u < 2; ++u) {
                 const int Q = base + nwarps * (c + u);
                 if (Q >= quads) break;  // warp-uniform
-                const uint32_t xr = xs + kXRegionBytes * x_pos(Q >> 1, Q & 1, par);
+                const int pos = par ? __shfl_sync(0xffffffffu, pos_l, c + u) : Q;
+                const uint32_t xr = xs + kXRegionBytes * pos;
                 asm volatile("st.shared.u32 [%0], %1;" ::"r"(xr + kXGroupBytes * sub + e), "r"(hb[u]) : "memory");
                 asm volatile("st.shared.u32 [%0], %1;" ::"r"(xr + kXGroupBytes * sub + 32 + e), "r"(lb[u])
                              : "memory");
@@ -1245,6 +1295,17 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
         dd[r] = __half2float(
             __ushort_as_half(static_cast<unsigned short>(ld_s32(bw[r] + 208) >> (odd[r] ? 16 : 0))));
     }
+    // the half's 4 groups: P and 32 times the integer sums of their two
+    // 16-weight halves (loaded once for both s)
+    float Pg[4];
+    uint32_t x32[4][2];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * t);  // X, P, 16-sums
+        Pg[t] = __uint_as_float(info.y);
+        x32[t][0] = 32u * info.z;
+        x32[t][1] = 32u * info.w;
+    }
     float y[2] = {0.f, 0.f};
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
@@ -1260,8 +1321,10 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
         for (int t = 0; t < 4; ++t) {
             const uint4 xh = ld_s128(xr + kXGroupBytes * t + 16 * s);
             const uint4 xl = ld_s128(xr + kXGroupBytes * t + 32 + 16 * s);
+            // the low-byte sums start at -32 * (16-sum of xi), mod 2^32: the
+            // exact int32 S = 256*hi + lo - 32*sum below (|each| < 2^31)
             int hi[2] = {0, 0};
-            uint32_t lo[2] = {0u, 0u};
+            uint32_t lo[2] = {0u - x32[t][s], 0u - x32[t][s]};
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
 #pragma unroll
@@ -1275,15 +1338,12 @@ __device__ __forceinline__ void q6k_unit_int(uint32_t row0, int row_bytes, int b
                     lo[r] = dp4a_uu(q, u4w(xl, m), lo[r]);
                 }
             }
-            const uint4 info = ld_s128(xr + 4 * kXGroupBytes + kXInfoBytes * t);  // X, P, 16-sums
-            const float P = __uint_as_float(info.y);
-            const int x32 = 32 * static_cast<int>(s ? info.w : info.z);
             const int g = 2 * t + s;  // group within the half
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                const int S = hi[r] * 256 + static_cast<int>(lo[r]) - x32;
+                const int S = hi[r] * 256 + static_cast<int>(lo[r]);
                 const int sv = sext_byte(sc[r][g >> 2], g & 3);  // the group's int8 scale
-                y[r] = fmaf(P, static_cast<float>(sv * S), y[r]);
+                y[r] = fmaf(Pg[t], static_cast<float>(sv * S), y[r]);
             }
         }
     }
@@ -1302,12 +1362,14 @@ __device__ __forceinline__ void q6k_unit_dispatch(int kappa, uint32_t row0, int 
 // Stage a segment's activations for the kernel below: threads ct of nthr
 // (whole warps), integer regions (INT) or fp32 regions, with or without the
 // prologue (PRO).
-template <int FMT, int NCOL, bool INT, bool PRO>
+// PAR: the launch may use the block-parity region order (a.par; only
+// single-column Q6_K), otherwise the regions are in plain order at compile time.
+template <int FMT, int NCOL, bool INT, bool PRO, bool PAR = (FMT == 2)>
 __device__ __forceinline__ void stage_all(const GemvArgs& a, int64_t seg, uint32_t xs, int ct, int nthr, int bar,
                                           int kb0, int nbl, uint32_t part) {
     if constexpr (INT)
         stage_x_int<PRO, (FMT == 2 || FMT == 4 || FMT == 5)>(a, seg, xs, ct >> 5, nthr >> 5, ct & 31, bar, nthr, kb0,
-                                                             nbl, part, a.par);
+                                                             nbl, part, PAR ? a.par : 0);
     else if constexpr (PRO)
         stage_x_pro<FMT, NCOL>(ProStage{a.x + seg * a.x_seg_stride + static_cast<int64_t>(kb0) * 256,
                                         a.pro == 1 ? a.gamma + static_cast<int64_t>(kb0) * 256 : nullptr, a.K, a.ldx,

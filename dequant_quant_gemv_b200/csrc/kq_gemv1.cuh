@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __g
     float* const y = a.y;
     pdl_wait();                      // activations may come from the previous grid
     pdl_launch_dependents();
-    stage_all<FMT, 1, true, PRO>(a, 0, xs_s, ct_all, 2 * kConsumers, 3, 0, nb, pro_r);
+    stage_all<FMT, 1, true, PRO, PAR>(a, 0, xs_s, ct_all, 2 * kConsumers, 3, 0, nb, pro_r);
     float rinv = 1.f;
     if (PRO && a.pro == 1) rinv = ld_s32f(pro_inv_addr(pro_r));
     if (ct_all == 0) *staged = 1;
