@@ -112,9 +112,14 @@ __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __g
     uint32_t phase = 0;
     bool dead = false;  // a wait of this lane ran out
     const bool lead = DIRECT ? (lane & ((LR < 32 ? LR : 32) - 1)) == 0 : lane == 0;
+    // When LR does not divide the group's 256 lanes (LR = 96, 160, 192 or
+    // 224), the warps past its ps row pairs hold no unit: they only keep the
+    // ring's protocol (wait for each stage, release it) and never touch the
+    // stage's bytes or a row pair's partial buffer.
+    const bool in_stage = L.rp < ps;
     for (int s = g; s < nst; s += 2) {
         const int64_t rp0 = rp_begin + static_cast<int64_t>(s) * ps;
-        const bool mine = L.active && rp0 + L.rp < rp_end;
+        const bool mine = in_stage && L.active && rp0 + L.rp < rp_end;
         // with an odd ring depth a slot alternates between the groups: first
         // the other group's release of the slot's previous stage
         if ((ns & 1) && s >= ns && !mbar_wait_bounded(&empty[slot], phase ^ 1u, abort_flag, wait_lim)) {
@@ -149,11 +154,13 @@ __global__ void __launch_bounds__(32 + 2 * kConsumers, 1) gemv1_kernel(const __g
         }
         if constexpr (DIRECT) {
             if (lane == 0) mbar_arrive(&empty[slot]);
-            if (lead && rp0 + L.rp < rp_end) {
+            if (lead && in_stage && rp0 + L.rp < rp_end) {
                 const int64_t row = 2 * (rp0 + L.rp);
                 y[row] = out[0][0] * rinv;
                 if (row + 1 < N) y[row + 1] = out[1][0] * rinv;
             }
+        } else if (!in_stage) {
+            if (lane == 0) mbar_arrive(&empty[slot]);
         } else {
             const int k = slot * ps + L.rp;  // this row pair's partial buffer and barrier
             if (lane == 0) {

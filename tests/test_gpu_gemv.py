@@ -72,6 +72,10 @@ SHAPES = [
     ("q4_k", 257, 4096), ("q4_k", 301, 8192), ("q4_k", 5, 1280), ("q4_k", 9, 32768), ("q4_k", 2, 5120),
     ("q6_k", 1, 2048), ("q6_k", 5, 2048), ("q6_k", 64, 14336), ("q6_k", 37, 28672), ("q6_k", 300, 4096),
     ("q6_k", 11, 16384),
+    # the block-parity lane order's layouts: one lone warp per parity (24
+    # blocks), warp pairs over part-filled chunks (36), a pair and a lone
+    # warp (80), a full lone warp (96), two pairs (128, the largest K)
+    ("q6_k", 9, 6144), ("q6_k", 13, 9216), ("q6_k", 7, 20480), ("q6_k", 5, 24576), ("q6_k", 3, 32768),
     ("q5_k", 1, 256), ("q5_k", 7, 768), ("q5_k", 257, 4096), ("q5_k", 301, 8192), ("q5_k", 9, 32768),
     ("q5_k", 5, 1280), ("q5_k", 4096, 4096), ("q5_k", 2, 14336),
     ("q2_k", 1, 1024), ("q2_k", 3, 1024), ("q2_k", 257, 4096), ("q2_k", 301, 8192), ("q2_k", 9, 32768),
@@ -90,6 +94,26 @@ def test_gemv_parity(fmt, N, K):
     y = kq.gemv(dev(W), fmt, N, K, dev(x))
     y_ref, s_ref = oracle_gemv(fmt, W, N, K, x)
     assert_close(y, y_ref, s_ref, f"{fmt} {N}x{K}")
+
+
+# Lane layouts whose row pairs do not fill a consumer group's 256 lanes (96,
+# 160, 192 or 224 lanes per row pair): the warps past a stage's row pairs
+# must stay out of the units and the partial-sum reductions.  Enough rows
+# that every CTA takes several stages; no bounded wait may run out.
+IDLE_WARP_SHAPES = [("q4_k", 1000, 10240), ("q4_k", 600, 20480), ("q4_k", 500, 24576), ("q4_k", 400, 28672),
+                    ("q6_k", 700, 20480), ("q6_k", 500, 24576), ("q5_k", 400, 28672), ("q8_0", 600, 20480),
+                    ("q2_k", 500, 20480), ("q3_k", 500, 24576)]
+
+
+@pytest.mark.parametrize("fmt,N,K", IDLE_WARP_SHAPES)
+def test_gemv_idle_warp_layouts(fmt, N, K):
+    kq.device_fault()  # read and clear
+    W = matrix(fmt, 11 * N + K, N, K)
+    x = x_vec(N + 5 * K, K)
+    y = kq.gemv(dev(W), fmt, N, K, dev(x))
+    y_ref, s_ref = oracle_gemv(fmt, W, N, K, x)
+    assert_close(y, y_ref, s_ref, f"{fmt} {N}x{K}")
+    assert kq.device_fault() == 0
 
 
 def test_gemv_single_q4k_4096_full():

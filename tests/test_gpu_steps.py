@@ -70,6 +70,19 @@ def test_independent_steps_equal_single_calls_bitwise(after):
         assert torch.equal(y, r), i
 
 
+# Q6_K in the block-parity lane order, each of its layouts (24, 36, 80, 96
+# and 128 blocks: lone warps, part-filled warp pairs, both, two pairs)
+@pytest.mark.parametrize("K", [6144, 9216, 20480, 24576, 32768])
+def test_q6k_parity_layouts_steps_equal_single_calls(K):
+    specs = build(1300 + K // 256, [("q6_k", 37, K, "none"), ("q6_k", 6, K, "rmsnorm"), ("q6_k", 21, K, "swiglu")])
+    ys = [nan(N) for (_, _, N, _, _, _, _) in specs]
+    kq.gemv_steps([kq.make_step(W, f, N, K_, x, y, kind, g, 1e-5, True)
+                   for (W, f, N, K_, x, kind, g), y in zip(specs, ys)])
+    ref = one_by_one(specs)
+    for i, (y, r) in enumerate(zip(ys, ref)):
+        assert torch.equal(y, r), i
+
+
 def test_chained_ffn_steps_equal_single_calls_and_oracle():
     """gate|up (RMSNorm) -> down (SiLU-gated [g; u] read from gate|up's
     output), three layers deep, in one call: each down step waits for its
