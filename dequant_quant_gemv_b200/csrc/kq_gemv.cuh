@@ -789,8 +789,9 @@ __device__ inline void stage_x_int(const GemvArgs& a, int64_t seg, uint32_t xs, 
     float sq = 0.f;
     for (int base = warp; base < quads; base += nwarps * U) {
         float4 v[U], w[U];
-        // the region positions of this round's U passes in the block-parity
-        // order, one pass per lane (lane u: pass u), then broadcast per pass
+        // the region positions of the U passes loaded together here, in the
+        // block-parity order: one pass per lane (lane u: pass u), then
+        // broadcast per pass
         int pos_l = 0;
         if (par) {
             const int Ql = base + nwarps * (lane & (U - 1));
