@@ -307,6 +307,23 @@ def test_multi_columns_independent_and_match_oracle(fmt, N, K, k):
         assert_close(Y[c], y_ref[c], s_ref[c], f"col {c}")
 
 
+# Several columns at the K of the single-column idle-warp layouts (and of
+# the larger K-range splits of the tensor-core kernel): every format, 8
+# columns, against the oracle; no bounded wait may run out.
+@pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 10240), ("q4_k", 200, 20480), ("q6_k", 300, 20480),
+                                     ("q6_k", 200, 24576), ("q5_k", 200, 28672), ("q8_0", 300, 20480),
+                                     ("q2_k", 300, 20480), ("q3_k", 200, 24576)])
+def test_multi_columns_large_k_match_oracle(fmt, N, K):
+    kq.device_fault()  # read and clear
+    W = matrix(fmt, 37 + K // 256, N, K)
+    X = np.stack([x_vec(200 + c + K, K) for c in range(8)])
+    Y = kq.gemv_multi(dev(W), fmt, N, K, dev(X))
+    y_ref, s_ref = oracle.gemv_multi(fmt, W, N, K, X, nthreads=0)
+    for c in range(8):
+        assert_close(Y[c], y_ref[c], s_ref[c], f"{fmt} {N}x{K} col {c}")
+    assert kq.device_fault() == 0
+
+
 @pytest.mark.parametrize("fmt,N,K", [("q4_k", 300, 4096), ("q6_k", 66, 14336), ("q5_k", 300, 4096),
                                      ("q2_k", 300, 4096), ("q3_k", 300, 4096), ("q8_0", 300, 4096)])
 def test_single_column_of_multi_call_matches_oracle(fmt, N, K):
